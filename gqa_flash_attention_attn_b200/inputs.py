@@ -1,0 +1,119 @@
+"""Seeded synthetic inputs and the named workloads.
+
+This module holds no attention arithmetic.  It draws Q, K, V for both the CUDA
+path and the float64 oracle, so the two sides always see identical bf16 values.
+
+Recipe: a ``torch.Generator`` seeded with ``seed`` draws q, k, v in that order
+as iid N(0, 1) float32 and casts each to bf16 (round to nearest even).  The
+shapes follow the workloads that the pages measure (head dims 64 to 512,
+grouped-query heads, 8-row speculative-verify steps, prefill at depth): see
+``WORKLOADS``.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    """One attention problem: shapes, mask, scale and (for decode) splits."""
+    name: str
+    kind: str            # "prefill" or "decode"
+    B: int
+    Hq: int
+    Hkv: int
+    Sq: int
+    Skv: int
+    D: int
+    q_offset: int
+    causal: bool
+    out_dtype: str       # "bf16" or "f32"
+    num_splits: int = 1
+    note: str = ""
+
+    @property
+    def scale(self) -> float:
+        # the float32 value both sides receive
+        return float(torch.tensor(1.0 / math.sqrt(self.D), dtype=torch.float32))
+
+    def visible_pairs_per_head(self) -> int:
+        """Number of visible (query row, key) pairs for one (batch, head)."""
+        if not self.causal:
+            return self.Sq * self.Skv
+        total = 0
+        for s in range(self.Sq):
+            total += min(self.Skv, self.q_offset + s + 1)
+        return total
+
+    def flops(self) -> int:
+        """Algorithmic FLOPs: 4*D per visible (query, key) pair."""
+        return 4 * self.D * self.visible_pairs_per_head() * self.B * self.Hq
+
+    def io_bytes(self) -> int:
+        """Algorithmic bytes: Q, K, V read once (bf16); O and LSE written once."""
+        ob = 2 if self.out_dtype == "bf16" else 4
+        q = self.B * self.Sq * self.Hq * self.D * 2
+        kv = 2 * self.B * self.Skv * self.Hkv * self.D * 2
+        o = self.B * self.Sq * self.Hq * self.D * ob
+        lse = self.B * self.Hq * self.Sq * 4
+        return q + kv + o + lse
+
+
+WORKLOADS = {
+    "tiny_causal_gqa_prefill": Workload(
+        "tiny_causal_gqa_prefill", "prefill", B=1, Hq=4, Hkv=1, Sq=128, Skv=128, D=64,
+        q_offset=0, causal=True, out_dtype="f32",
+        note="B1 Hq4 Hkv1 S128 D64, fp32 out"),
+    "gqa_causal_prefill_4k_d128": Workload(
+        "gqa_causal_prefill_4k_d128", "prefill", B=1, Hq=32, Hkv=8, Sq=4096, Skv=4096, D=128,
+        q_offset=0, causal=True, out_dtype="bf16",
+        note="B1 Hq32 Hkv8 S4096 D128, bf16 out"),
+    "prefill_at_depth_d256": Workload(
+        "prefill_at_depth_d256", "prefill", B=1, Hq=16, Hkv=8, Sq=2048, Skv=10240, D=256,
+        q_offset=8192, causal=True, out_dtype="bf16",
+        note="2048 new queries at depth 8192 over 10240 keys, D256"),
+    "split_kv_decode_d512": Workload(
+        "split_kv_decode_d512", "decode", B=16, Hq=16, Hkv=1, Sq=1, Skv=16384, D=512,
+        q_offset=16383, causal=True, out_dtype="bf16", num_splits=32,
+        note="B16 Hq16 Hkv1 Skv16384 D512, 32 splits merged by LSE"),
+    "spec_verify_decode_d128": Workload(
+        "spec_verify_decode_d128", "decode", B=4, Hq=32, Hkv=8, Sq=8, Skv=32768, D=128,
+        q_offset=32760, causal=True, out_dtype="bf16", num_splits=16,
+        note="8 draft rows per sequence, causal among themselves, Skv 32768"),
+}
+
+
+def make_qkv(B, Hq, Hkv, Sq, Skv, D, *, seed=0, device="cpu"):
+    """Seeded q [B,Sq,Hq,D], k and v [B,Skv,Hkv,D], all bf16, drawn q, k, v in order."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    q = torch.randn((B, Sq, Hq, D), generator=gen, dtype=torch.float32, device=device)
+    q = q.to(torch.bfloat16)
+    k = torch.randn((B, Skv, Hkv, D), generator=gen, dtype=torch.float32, device=device)
+    k = k.to(torch.bfloat16)
+    v = torch.randn((B, Skv, Hkv, D), generator=gen, dtype=torch.float32, device=device)
+    v = v.to(torch.bfloat16)
+    return q, k, v
+
+
+def make_workload_inputs(w: Workload, *, seed=0, device="cpu"):
+    return make_qkv(w.B, w.Hq, w.Hkv, w.Sq, w.Skv, w.D, seed=seed, device=device)
+
+
+def sample_rows(w: Workload, n: int, *, seed=1234, include_edges=True):
+    """(b, h, s) triples spread over the problem, including its corners."""
+    gen = torch.Generator().manual_seed(seed)
+    b = torch.randint(0, w.B, (n,), generator=gen)
+    h = torch.randint(0, w.Hq, (n,), generator=gen)
+    s = torch.randint(0, w.Sq, (n,), generator=gen)
+    rows = torch.stack([b, h, s], dim=1).tolist()
+    if include_edges:
+        for bb in {0, w.B - 1}:
+            for hh in {0, w.Hq - 1}:
+                for ss in {0, 1, w.Sq // 2, w.Sq - 1}:
+                    if 0 <= ss < w.Sq:
+                        rows.append([bb, hh, ss])
+    return rows

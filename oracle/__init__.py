@@ -1,0 +1,171 @@
+"""Float64 CPU oracle for grouped-query attention.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg may import this package.  The CUDA library never
+imports, links or calls it, and it imports nothing from the CUDA library.
+
+The arithmetic lives in ``oracle.c`` (plain C, fp64, OpenMP over rows); this
+module compiles it with gcc on first use and marshals numpy arrays.  Every
+function takes arrays that are widened EXACTLY from the values the GPU sees
+(bf16 -> float64 is exact), and the scale as the same float32 value the GPU
+receives, widened.
+
+Functions and the passage each follows (all pinned by tests/test_oracle_pins.py):
+  attention       the definition of softmax attention with grouped-query heads
+                  ("ggml-org/llama.cpp PR #28507", Setup: GQA 8; FLASH_ATTN_EXT
+                  case list: nr23, mask=1)
+  attention_rows  the same definition on selected (b, h, s) rows
+  probs           the normalised attention weights of one row
+  split           per-split partials with their LSE metadata
+                  ("Anbeeld/beellama.cpp PR #149", Overview: every block
+                  publishes its (max, rowsum))
+  merge           the LSE combine of split partials (same page, review of the
+                  combine kernel for parallel_blocks > 1)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+_i64 = ctypes.c_int64
+_dp = ctypes.POINTER(ctypes.c_double)
+_lp = ctypes.POINTER(ctypes.c_int64)
+
+
+def build(src: str = _SRC, out: str = _LIB_PATH, extra_flags=()) -> str:
+    """Compile oracle.c into a shared library (gcc -O2, OpenMP, no fast-math)."""
+    cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c99", *extra_flags,
+           "-o", out, src, "-lm"]
+    subprocess.run(cmd, check=True)
+    return out
+
+
+def _needs_build(src: str, out: str) -> bool:
+    return (not os.path.exists(out)) or os.path.getmtime(out) < os.path.getmtime(src)
+
+
+def load(path: str | None = None):
+    """Load (building if stale) the oracle library; returns a ctypes handle."""
+    global _lib
+    if path is not None:
+        return _bind(ctypes.CDLL(path))
+    with _lock:
+        if _lib is None:
+            if _needs_build(_SRC, _LIB_PATH):
+                build()
+            _lib = _bind(ctypes.CDLL(_LIB_PATH))
+    return _lib
+
+
+def _bind(lib):
+    lib.oracle_attention.argtypes = [_dp, _dp, _dp, _dp, _dp] + [_i64] * 7 + [ctypes.c_int, ctypes.c_double]
+    lib.oracle_attention.restype = None
+    lib.oracle_attention_rows.argtypes = [_dp, _dp, _dp, _lp, _i64, _dp, _dp] + [_i64] * 7 + [ctypes.c_int, ctypes.c_double]
+    lib.oracle_attention_rows.restype = None
+    lib.oracle_probs.argtypes = [_dp, _dp, _i64, _i64, _i64, _dp] + [_i64] * 6 + [ctypes.c_int, ctypes.c_double]
+    lib.oracle_probs.restype = None
+    lib.oracle_split.argtypes = [_dp, _dp, _dp, _dp, _dp] + [_i64] * 7 + [ctypes.c_int, ctypes.c_double, _i64]
+    lib.oracle_split.restype = None
+    lib.oracle_merge.argtypes = [_dp, _dp, _dp, _dp] + [_i64] * 5
+    lib.oracle_merge.restype = None
+    lib.oracle_num_threads.argtypes = []
+    lib.oracle_num_threads.restype = ctypes.c_int
+    return lib
+
+
+def _f64(x) -> np.ndarray:
+    """Widen to a contiguous float64 numpy array (exact for bf16/fp32 inputs)."""
+    if hasattr(x, "detach"):  # torch tensor
+        x = x.detach().to("cpu")
+        x = x.double().numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(_dp)
+
+
+def _dims(q, k):
+    B, Sq, Hq, D = q.shape
+    Bk, Skv, Hkv, Dk = k.shape
+    if Bk != B or Dk != D:
+        raise ValueError("q and k disagree on batch or head dim")
+    if Hq % Hkv != 0:
+        raise ValueError("Hq must be a multiple of Hkv")
+    return B, Hq, Hkv, Sq, Skv, D
+
+
+def num_threads(lib=None) -> int:
+    return (lib or load()).oracle_num_threads()
+
+
+def attention(q, k, v, *, scale, causal=True, q_offset=0, lib=None):
+    """O [B,Sq,Hq,D] and LSE [B,Hq,Sq] in float64 for the whole problem."""
+    lib = lib or load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, Hkv, Sq, Skv, D = _dims(q, k)
+    out = np.zeros((B, Sq, Hq, D), dtype=np.float64)
+    lse = np.zeros((B, Hq, Sq), dtype=np.float64)
+    lib.oracle_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                         B, Hq, Hkv, Sq, Skv, D, int(q_offset), int(bool(causal)), float(scale))
+    return out, lse
+
+
+def attention_rows(q, k, v, rows, *, scale, causal=True, q_offset=0, lib=None):
+    """O rows [n,D] and LSE [n] for the (b, h, s) triples in ``rows``."""
+    lib = lib or load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, Hkv, Sq, Skv, D = _dims(q, k)
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
+    n = rows.shape[0]
+    out = np.zeros((n, D), dtype=np.float64)
+    lse = np.zeros((n,), dtype=np.float64)
+    lib.oracle_attention_rows(_ptr(q), _ptr(k), _ptr(v), rows.ctypes.data_as(_lp), n,
+                              _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Skv, D,
+                              int(q_offset), int(bool(causal)), float(scale))
+    return out, lse
+
+
+def probs(q, k, b, h, s, *, scale, causal=True, q_offset=0, lib=None):
+    """Normalised attention weights of row (b, h, s) over all Skv keys."""
+    lib = lib or load()
+    q, k = _f64(q), _f64(k)
+    B, Hq, Hkv, Sq, Skv, D = _dims(q, k)
+    p = np.zeros((Skv,), dtype=np.float64)
+    lib.oracle_probs(_ptr(q), _ptr(k), int(b), int(h), int(s), _ptr(p),
+                     Hq, Hkv, Sq, Skv, D, int(q_offset), int(bool(causal)), float(scale))
+    return p
+
+
+def split(q, k, v, num_splits, *, scale, causal=True, q_offset=0, lib=None):
+    """Per-split partial O [S,B,Sq,Hq,D] and LSE [S,B,Hq,Sq]."""
+    lib = lib or load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, Hkv, Sq, Skv, D = _dims(q, k)
+    pout = np.zeros((num_splits, B, Sq, Hq, D), dtype=np.float64)
+    plse = np.zeros((num_splits, B, Hq, Sq), dtype=np.float64)
+    lib.oracle_split(_ptr(q), _ptr(k), _ptr(v), _ptr(pout), _ptr(plse),
+                     B, Hq, Hkv, Sq, Skv, D, int(q_offset), int(bool(causal)), float(scale),
+                     int(num_splits))
+    return pout, plse
+
+
+def merge(pout, plse, lib=None):
+    """Combine split partials: returns O [B,Sq,Hq,D] and LSE [B,Hq,Sq]."""
+    lib = lib or load()
+    pout, plse = _f64(pout), _f64(plse)
+    S, B, Sq, Hq, D = pout.shape
+    out = np.zeros((B, Sq, Hq, D), dtype=np.float64)
+    lse = np.zeros((B, Hq, Sq), dtype=np.float64)
+    lib.oracle_merge(_ptr(pout), _ptr(plse), _ptr(out), _ptr(lse), B, Hq, Sq, D, S)
+    return out, lse

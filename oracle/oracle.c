@@ -1,0 +1,243 @@
+/*
+ * Float64 CPU oracle for grouped-query scaled-dot-product attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path links, loads or calls
+ * this file: only the tests, the smoke check and the benchmark's CPU-baseline
+ * leg do.  It shares no code, header, table or helper with the CUDA library.
+ *
+ * What it computes (the plain definition, written out, no blocking, no online
+ * softmax).  For batch b, query head h, query row s, with group size
+ * g = Hq / Hkv and K/V head kvh = h / g:
+ *
+ *     pos   = q_offset + s
+ *     T     = { t in [0, Skv) : !causal  or  t <= pos }
+ *     z_t   = scale * sum_d Q[b,s,h,d] * K[b,t,kvh,d]
+ *     m     = max_{t in T} z_t
+ *     l     = sum_{t in T} exp(z_t - m)
+ *     O[b,s,h,:] = sum_{t in T} exp(z_t - m) / l * V[b,t,kvh,:]
+ *     LSE[b,h,s] = m + ln(l)                      (natural log, scaled logits)
+ *
+ * Sources on the pages:
+ *   - grouped-query heads sharing one K/V head: "ggml-org/llama.cpp PR #28507",
+ *     Setup ("GQA 8") and the FLASH_ATTN_EXT test case list (nr23 broadcast
+ *     ratio, mask=1), read as the contiguous-group broadcast kvh = h / g;
+ *   - the scale applied to Q.K: "AstrAI commit log, gqa_prefill_attn_mma.cuh",
+ *     the pre-scaled Q item (here the scale multiplies the exact fp64 dot
+ *     product, which is the same quantity without a rounding step);
+ *   - per-row (max, rowsum) metadata and the merge of split tiles:
+ *     "Anbeeld/beellama.cpp PR #149", Overview (ub>64 fix: every block
+ *     publishes its (max, rowsum)) and the review's note on the combine
+ *     kernel for parallel_blocks > 1.
+ *
+ * Readings where the pages are silent:
+ *   - layout: Q, O are [B, Sq, Hq, D]; K, V are [B, Skv, Hkv, D];
+ *     LSE is [B, Hq, Sq]; all contiguous, row-major;
+ *   - causal alignment: key t is visible to row s iff t <= q_offset + s;
+ *   - split sigma of num_splits covers keys [sigma*c, min((sigma+1)*c, Skv)),
+ *     c = ceil(Skv / num_splits); a split with no visible key for a row
+ *     publishes lse = -inf and O = 0 for that row, and the merge gives it
+ *     weight zero.
+ *
+ * Every input is a double array; callers widen bf16 values exactly.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+static int64_t q_index(int64_t b, int64_t s, int64_t h, int64_t Sq, int64_t Hq, int64_t D) {
+    return ((b * Sq + s) * Hq + h) * D;
+}
+
+static int64_t kv_index(int64_t b, int64_t t, int64_t kvh, int64_t Skv, int64_t Hkv, int64_t D) {
+    return ((b * Skv + t) * Hkv + kvh) * D;
+}
+
+/* One output row restricted to keys [t_lo, t_hi).  z is scratch of length
+ * >= t_hi - t_lo.  Returns the LSE (or -inf when no key is visible, in which
+ * case o_row is all zeros). */
+static double attend_row(const double* q, const double* k, const double* v,
+                         int64_t b, int64_t h, int64_t s,
+                         int64_t Hq, int64_t Hkv, int64_t Sq, int64_t Skv, int64_t D,
+                         int64_t q_offset, int causal, double scale,
+                         int64_t t_lo, int64_t t_hi, double* z, double* o_row) {
+    const int64_t g = Hq / Hkv;
+    const int64_t kvh = h / g;
+    const int64_t pos = q_offset + s;
+    const double* qr = q + q_index(b, s, h, Sq, Hq, D);
+
+    int64_t last = t_hi;                       /* exclusive upper bound of T */
+    if (causal && pos + 1 < last) last = pos + 1;
+    for (int64_t d = 0; d < D; ++d) o_row[d] = 0.0;
+    if (last <= t_lo) return -INFINITY;
+
+    /* pass 1: logits and their maximum */
+    double m = -INFINITY;
+    for (int64_t t = t_lo; t < last; ++t) {
+        const double* kr = k + kv_index(b, t, kvh, Skv, Hkv, D);
+        double acc = 0.0;
+        for (int64_t d = 0; d < D; ++d) acc += qr[d] * kr[d];
+        const double zt = scale * acc;
+        z[t - t_lo] = zt;
+        if (zt > m) m = zt;
+    }
+    /* pass 2: exponentials, their sum, and the weighted sum of V rows */
+    double l = 0.0;
+    for (int64_t t = t_lo; t < last; ++t) {
+        const double p = exp(z[t - t_lo] - m);
+        z[t - t_lo] = p;
+        l += p;
+    }
+    for (int64_t t = t_lo; t < last; ++t) {
+        const double w = z[t - t_lo] / l;
+        const double* vr = v + kv_index(b, t, kvh, Skv, Hkv, D);
+        for (int64_t d = 0; d < D; ++d) o_row[d] += w * vr[d];
+    }
+    return m + log(l);
+}
+
+/* Full attention: out [B,Sq,Hq,D], lse [B,Hq,Sq]. */
+void oracle_attention(const double* q, const double* k, const double* v,
+                      double* out, double* lse,
+                      int64_t B, int64_t Hq, int64_t Hkv, int64_t Sq, int64_t Skv, int64_t D,
+                      int64_t q_offset, int causal, double scale) {
+    const int64_t rows = B * Hq * Sq;
+#pragma omp parallel
+    {
+        double* z = (double*)malloc(sizeof(double) * (size_t)(Skv > 0 ? Skv : 1));
+#pragma omp for schedule(dynamic, 16)
+        for (int64_t r = 0; r < rows; ++r) {
+            const int64_t b = r / (Hq * Sq);
+            const int64_t h = (r / Sq) % Hq;
+            const int64_t s = r % Sq;
+            double* o_row = out + q_index(b, s, h, Sq, Hq, D);
+            lse[(b * Hq + h) * Sq + s] =
+                attend_row(q, k, v, b, h, s, Hq, Hkv, Sq, Skv, D, q_offset, causal, scale,
+                           0, Skv, z, o_row);
+        }
+        free(z);
+    }
+}
+
+/* Selected rows only: rows is n triples (b, h, s); out_rows [n, D]; lse_rows [n]. */
+void oracle_attention_rows(const double* q, const double* k, const double* v,
+                           const int64_t* rows, int64_t n, double* out_rows, double* lse_rows,
+                           int64_t B, int64_t Hq, int64_t Hkv, int64_t Sq, int64_t Skv, int64_t D,
+                           int64_t q_offset, int causal, double scale) {
+    (void)B;
+#pragma omp parallel
+    {
+        double* z = (double*)malloc(sizeof(double) * (size_t)(Skv > 0 ? Skv : 1));
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t i = 0; i < n; ++i) {
+            const int64_t b = rows[3 * i], h = rows[3 * i + 1], s = rows[3 * i + 2];
+            lse_rows[i] = attend_row(q, k, v, b, h, s, Hq, Hkv, Sq, Skv, D, q_offset, causal,
+                                     scale, 0, Skv, z, out_rows + i * D);
+        }
+        free(z);
+    }
+}
+
+/* The normalised attention weights of one row, written to p[0..Skv); masked keys get 0. */
+void oracle_probs(const double* q, const double* k,
+                  int64_t b, int64_t h, int64_t s, double* p,
+                  int64_t Hq, int64_t Hkv, int64_t Sq, int64_t Skv, int64_t D,
+                  int64_t q_offset, int causal, double scale) {
+    const int64_t g = Hq / Hkv;
+    const int64_t kvh = h / g;
+    const int64_t pos = q_offset + s;
+    const double* qr = q + q_index(b, s, h, Sq, Hq, D);
+    double m = -INFINITY;
+    for (int64_t t = 0; t < Skv; ++t) {
+        if (causal && t > pos) { p[t] = -INFINITY; continue; }
+        const double* kr = k + kv_index(b, t, kvh, Skv, Hkv, D);
+        double acc = 0.0;
+        for (int64_t d = 0; d < D; ++d) acc += qr[d] * kr[d];
+        p[t] = scale * acc;
+        if (p[t] > m) m = p[t];
+    }
+    double l = 0.0;
+    for (int64_t t = 0; t < Skv; ++t) {
+        p[t] = (p[t] == -INFINITY) ? 0.0 : exp(p[t] - m);
+        l += p[t];
+    }
+    for (int64_t t = 0; t < Skv; ++t) p[t] /= l;
+}
+
+/* Split-KV partials: pout [S,B,Sq,Hq,D] (each split normalised on its own keys),
+ * plse [S,B,Hq,Sq]. */
+void oracle_split(const double* q, const double* k, const double* v,
+                  double* pout, double* plse,
+                  int64_t B, int64_t Hq, int64_t Hkv, int64_t Sq, int64_t Skv, int64_t D,
+                  int64_t q_offset, int causal, double scale, int64_t num_splits) {
+    const int64_t chunk = (Skv + num_splits - 1) / num_splits;
+    const int64_t rows = B * Hq * Sq;
+    const int64_t total = num_splits * rows;
+#pragma omp parallel
+    {
+        double* z = (double*)malloc(sizeof(double) * (size_t)(chunk > 0 ? chunk : 1));
+#pragma omp for schedule(dynamic, 16)
+        for (int64_t i = 0; i < total; ++i) {
+            const int64_t sigma = i / rows;
+            const int64_t r = i % rows;
+            const int64_t b = r / (Hq * Sq);
+            const int64_t h = (r / Sq) % Hq;
+            const int64_t s = r % Sq;
+            int64_t lo = sigma * chunk, hi = lo + chunk;
+            if (lo > Skv) lo = Skv;
+            if (hi > Skv) hi = Skv;
+            double* o_row = pout + sigma * (B * Sq * Hq * D) + q_index(b, s, h, Sq, Hq, D);
+            plse[sigma * rows + (b * Hq + h) * Sq + s] =
+                attend_row(q, k, v, b, h, s, Hq, Hkv, Sq, Skv, D, q_offset, causal, scale,
+                           lo, hi, z, o_row);
+        }
+        free(z);
+    }
+}
+
+/* Merge of split partials by their log-sum-exp:
+ *   M = max_sigma lse_sigma,  w_sigma = exp(lse_sigma - M),
+ *   O = sum w_sigma O_sigma / sum w_sigma,  lse = M + ln(sum w_sigma).
+ * A split with lse = -inf has weight 0; if every split is -inf the row is
+ * O = 0, lse = -inf. */
+void oracle_merge(const double* pout, const double* plse, double* out, double* lse,
+                  int64_t B, int64_t Hq, int64_t Sq, int64_t D, int64_t num_splits) {
+    const int64_t rows = B * Hq * Sq;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        const int64_t b = r / (Hq * Sq);
+        const int64_t h = (r / Sq) % Hq;
+        const int64_t s = r % Sq;
+        double* o_row = out + q_index(b, s, h, Sq, Hq, D);
+        double M = -INFINITY;
+        for (int64_t sg = 0; sg < num_splits; ++sg) {
+            const double x = plse[sg * rows + r];
+            if (x > M) M = x;
+        }
+        for (int64_t d = 0; d < D; ++d) o_row[d] = 0.0;
+        if (M == -INFINITY) { lse[r] = -INFINITY; continue; }
+        double wsum = 0.0;
+        for (int64_t sg = 0; sg < num_splits; ++sg) {
+            const double x = plse[sg * rows + r];
+            if (x == -INFINITY) continue;
+            const double w = exp(x - M);
+            wsum += w;
+            const double* pr = pout + sg * (B * Sq * Hq * D) + q_index(b, s, h, Sq, Hq, D);
+            for (int64_t d = 0; d < D; ++d) o_row[d] += w * pr[d];
+        }
+        for (int64_t d = 0; d < D; ++d) o_row[d] /= wsum;
+        lse[r] = M + log(wsum);
+    }
+}
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

@@ -1,0 +1,52 @@
+"""Fail-demo acceptance for the oracle's pins.
+
+Each case plants one plausible mistake in a copy of oracle.c (CPU only), builds
+it, and requires that at least one pin rejects it.  A pin set that let any of
+these through would not be pinning the oracle.
+"""
+import os
+
+import pytest
+
+import oracle
+from oracle_pins import ALL_PINS
+
+SRC = os.path.join(os.path.dirname(os.path.abspath(oracle.__file__)), "oracle.c")
+
+# (name, text in oracle.c, replacement); every occurrence is replaced
+MUTANTS = [
+    ("causal_off_by_one", "if (causal && pos + 1 < last) last = pos + 1;",
+     "if (causal && pos < last) last = pos;"),
+    ("causal_sees_one_more", "if (causal && pos + 1 < last) last = pos + 1;",
+     "if (causal && pos + 2 < last) last = pos + 2;"),
+    ("no_max_subtraction", "const double p = exp(z[t - t_lo] - m);", "const double p = exp(z[t - t_lo]);"),
+    ("lse_drops_max", "return m + log(l);", "return log(l);"),
+    ("lse_base_two", "return m + log(l);", "return m + log2(l);"),
+    ("scale_dropped", "const double zt = scale * acc;", "const double zt = acc;"),
+    ("scale_squared", "const double zt = scale * acc;", "const double zt = scale * scale * acc;"),
+    ("gqa_modulo_mapping", "const int64_t kvh = h / g;", "const int64_t kvh = h % Hkv;"),
+    ("value_row_from_key_zero", "const double* vr = v + kv_index(b, t, kvh, Skv, Hkv, D);",
+     "const double* vr = v + kv_index(b, t_lo, kvh, Skv, Hkv, D);"),
+    ("unnormalised_output", "const double w = z[t - t_lo] / l;", "const double w = z[t - t_lo];"),
+    ("merge_weight_sign", "const double w = exp(x - M);", "const double w = exp(M - x);"),
+    ("merge_lse_no_max", "lse[r] = M + log(wsum);", "lse[r] = log(wsum);"),
+    ("split_chunk_floor", "const int64_t chunk = (Skv + num_splits - 1) / num_splits;",
+     "const int64_t chunk = Skv / num_splits;"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_mutant_is_caught(tmp_path, name, old, new):
+    src = open(SRC).read()
+    assert src.count(old) >= 1, f"mutation site for {name} not found"
+    mutant = tmp_path / "oracle_mutant.c"
+    mutant.write_text(src.replace(old, new))
+    so = oracle.build(str(mutant), str(tmp_path / "liboracle_mutant.so"))
+    lib = oracle.load(so)
+    caught = []
+    for pin in ALL_PINS:
+        try:
+            pin(lib)
+        except (AssertionError, ValueError, FloatingPointError):
+            caught.append(pin.__name__)
+    assert caught, f"no pin rejects the planted mistake {name}"
