@@ -1,0 +1,217 @@
+"""Grouped-query flash attention for NVIDIA B200 (sm_100a).
+
+Thin Python binding over the C ABI in ``include/attn.h`` (libgqa_attn.so):
+argument marshalling and output allocation with torch, nothing else.  Every
+step of the computation runs in the library's CUDA kernels; there is no CPU or
+library fallback, and every call raises if the library is missing or reports
+an error.
+
+Layouts: q/out [B, Sq, Hq, D], k/v [B, Skv, Hkv, D] (bf16, contiguous),
+lse [B, Hq, Sq] fp32, partials [S, B, Sq, Hq, D] and [S, B, Hq, Sq] fp32.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+import threading
+
+import torch
+
+__all__ = [
+    "AttnError", "library", "library_path", "declared_functions", "prefill", "decode_split",
+    "merge", "decode", "decode_workspace_bytes", "last_status", "status_string",
+    "watchdog_selftest", "version", "ATTN_OK", "ATTN_ERR_INVALID_ARG", "ATTN_ERR_UNSUPPORTED",
+    "ATTN_ERR_ALIGNMENT", "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT",
+]
+
+ATTN_OK = 0
+ATTN_ERR_INVALID_ARG = -1
+ATTN_ERR_UNSUPPORTED = -2
+ATTN_ERR_ALIGNMENT = -3
+ATTN_ERR_CUDA = -4
+ATTN_ERR_TIMEOUT = -5
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_HEADER = os.path.join(os.path.dirname(_PKG), "include", "attn.h")
+_lock = threading.Lock()
+_lib = None
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_f = ctypes.c_float
+
+_SIGNATURES = {
+    "attn_prefill": (_i, [_vp, _vp, _vp, _vp, _vp] + [_i] * 8 + [_f, _i, _vp]),
+    "attn_decode_split": (_i, [_vp, _vp, _vp, _vp, _vp] + [_i] * 8 + [_f, _i, _vp]),
+    "attn_merge": (_i, [_vp, _vp, _vp, _vp] + [_i] * 6 + [_vp]),
+    "attn_decode_workspace_bytes": (ctypes.c_size_t, [_i] * 5),
+    "attn_last_status": (_i, [_vp]),
+    "attn_status_string": (ctypes.c_char_p, [_i]),
+    "attn_watchdog_selftest": (_i, [ctypes.c_ulonglong, _vp]),
+    "attn_version": (_i, []),
+}
+
+
+class AttnError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {status_string(status)} ({status})")
+
+
+def library_path() -> str:
+    return os.path.join(_PKG, "libgqa_attn.so")
+
+
+def library():
+    """The loaded C library; raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            path = library_path()
+            if not os.path.exists(path):
+                raise RuntimeError(
+                    f"{path} is missing: build it with `python -m gqa_flash_attention_attn_b200.build`")
+            lib = ctypes.CDLL(path)
+            for name, (res, args) in _SIGNATURES.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = lib
+    return _lib
+
+
+def declared_functions() -> list[str]:
+    """Names of the functions include/attn.h declares."""
+    text = open(_HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_[a-z0-9_]+)\s*\(", text)))
+
+
+def status_string(status: int) -> str:
+    return library().attn_status_string(int(status)).decode()
+
+
+def version() -> int:
+    return library().attn_version()
+
+
+def _stream_ptr(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check(fn: str, status: int):
+    if status != ATTN_OK:
+        raise AttnError(fn, status)
+
+
+def _need(t, name, dtype, ndim):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+_OUT_CODES = {torch.bfloat16: 0, torch.float32: 1}
+
+
+def prefill(q, k, v, *, causal=True, q_offset=0, scale=None, out_dtype=torch.bfloat16,
+            out=None, lse=None, return_lse=True, stream=None):
+    """O = softmax(scale * Q K^T + causal mask) V and its LSE, in one launch."""
+    _need(q, "q", torch.bfloat16, 4)
+    _need(k, "k", torch.bfloat16, 4)
+    _need(v, "v", torch.bfloat16, 4)
+    B, Sq, Hq, D = q.shape
+    _, Skv, Hkv, _ = k.shape
+    if v.shape != k.shape or k.shape[0] != B or k.shape[3] != D:
+        raise ValueError("k/v shapes do not match q")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty((B, Sq, Hq, D), dtype=out_dtype, device=q.device)
+    else:
+        _need(out, "out", out.dtype, 4)
+    if out.dtype not in _OUT_CODES:
+        raise ValueError("out must be bf16 or fp32")
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    st = library().attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Skv, D,
+                                int(q_offset), int(bool(causal)), float(scale), _OUT_CODES[out.dtype],
+                                _stream_ptr(stream))
+    _check("attn_prefill", st)
+    return out, lse
+
+
+def decode_workspace_bytes(B, Hq, Sq, D, num_splits) -> int:
+    return library().attn_decode_workspace_bytes(B, Hq, Sq, D, num_splits)
+
+
+def decode_split(q, k, v, num_splits, *, causal=True, q_offset=0, scale=None,
+                 partial_out=None, partial_lse=None, stream=None):
+    """Per-split normalised partial outputs [S,B,Sq,Hq,D] and LSEs [S,B,Hq,Sq]."""
+    _need(q, "q", torch.bfloat16, 4)
+    _need(k, "k", torch.bfloat16, 4)
+    _need(v, "v", torch.bfloat16, 4)
+    B, Sq, Hq, D = q.shape
+    _, Skv, Hkv, _ = k.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if partial_out is None:
+        partial_out = torch.empty((num_splits, B, Sq, Hq, D), dtype=torch.float32, device=q.device)
+    if partial_lse is None:
+        partial_lse = torch.empty((num_splits, B, Hq, Sq), dtype=torch.float32, device=q.device)
+    st = library().attn_decode_split(_ptr(q), _ptr(k), _ptr(v), _ptr(partial_out), _ptr(partial_lse), B, Hq,
+                                     Hkv, Sq, Skv, D, int(q_offset), int(bool(causal)), float(scale),
+                                     int(num_splits), _stream_ptr(stream))
+    _check("attn_decode_split", st)
+    return partial_out, partial_lse
+
+
+def merge(partial_out, partial_lse, *, out_dtype=torch.bfloat16, out=None, lse=None, return_lse=True,
+          stream=None):
+    """Combine split partials by their LSE into out [B,Sq,Hq,D] and lse [B,Hq,Sq]."""
+    _need(partial_out, "partial_out", torch.float32, 5)
+    _need(partial_lse, "partial_lse", torch.float32, 4)
+    S, B, Sq, Hq, D = partial_out.shape
+    if out is None:
+        out = torch.empty((B, Sq, Hq, D), dtype=out_dtype, device=partial_out.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=partial_out.device)
+    st = library().attn_merge(_ptr(partial_out), _ptr(partial_lse), _ptr(out), _ptr(lse), B, Hq, Sq, D, S,
+                              _OUT_CODES[out.dtype], _stream_ptr(stream))
+    _check("attn_merge", st)
+    return out, lse
+
+
+def decode(q, k, v, num_splits, *, causal=True, q_offset=0, scale=None, out_dtype=torch.bfloat16,
+           workspace=None, out=None, lse=None, stream=None):
+    """Split-KV decode followed by the LSE merge (two launches on one stream)."""
+    B, Sq, Hq, D = q.shape
+    po = pl = None
+    if workspace is not None:
+        po, pl = workspace
+    po, pl = decode_split(q, k, v, num_splits, causal=causal, q_offset=q_offset, scale=scale,
+                          partial_out=po, partial_lse=pl, stream=stream)
+    return merge(po, pl, out_dtype=out_dtype, out=out, lse=lse, stream=stream)
+
+
+def last_status(stream=None) -> int:
+    """Synchronise, then read and clear the device status word."""
+    return library().attn_last_status(_stream_ptr(stream))
+
+
+def watchdog_selftest(limit_ns: int, stream=None):
+    _check("attn_watchdog_selftest", library().attn_watchdog_selftest(int(limit_ns), _stream_ptr(stream)))

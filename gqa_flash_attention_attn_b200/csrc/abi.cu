@@ -1,0 +1,230 @@
+// C ABI of the library: argument checks, TMA descriptors, launches, status.
+// Every check that can fail runs on the host before any CUDA call, so bad
+// arguments never reach a kernel.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/attn.h"
+#include "kernels.h"
+
+namespace gqa {
+int prefill_slots(int D);
+int decode_max_nbuf();
+}  // namespace gqa
+
+namespace {
+
+__device__ int g_attn_status = 0;
+
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per pipeline wait
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr size_t kTwoCtaSmemLimit = 115712;  // two CTAs per SM
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+std::mutex g_mu;
+EncodeTiledFn g_encode = nullptr;
+int* g_status_ptr[64] = {nullptr};
+
+int cuda_fail() { return ATTN_ERR_CUDA; }
+
+EncodeTiledFn encoder() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_encode == nullptr) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  }
+  return g_encode;
+}
+
+int* status_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_status_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_attn_status) != cudaSuccess) return nullptr;
+    g_status_ptr[dev] = static_cast<int*>(p);
+  }
+  return g_status_ptr[dev];
+}
+
+// bf16 tensor [d3][d2][d1][d0] (d0 innermost), tiled with 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t d3, uint32_t b0,
+              uint32_t b1, uint32_t b2, uint32_t b3) {
+  EncodeTiledFn enc = encoder();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[4] = {d0, d1, d2, d3};
+  const cuuint64_t strides[3] = {d0 * 2, d0 * d1 * 2, d0 * d1 * d2 * 2};
+  const cuuint32_t box[4] = {b0, b1, b2, b3};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  std::memset(m, 0, sizeof(*m));
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// Shape checks shared by prefill and decode.
+int check_common(const void* q, const void* k, const void* v, int B, int Hq, int Hkv, int Sq, int Skv, int D,
+                 int q_offset, int causal, float scale) {
+  if (q == nullptr || k == nullptr || v == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Sq < 1 || Skv < 1 || D < 1) return ATTN_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (q_offset < 0 || (long long)q_offset + Sq > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  // TMA strides must stay below 2^40 bytes
+  if ((long double)B * Sq * Hq * D * 4 >= 1099511627776.0L) return ATTN_ERR_INVALID_ARG;
+  if ((long double)B * Skv * Hkv * D * 2 >= 1099511627776.0L) return ATTN_ERR_INVALID_ARG;
+  return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_version(void) { return 0x000100; }
+
+const char* attn_status_string(int status) {
+  switch (status) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_INVALID_ARG: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported shape";
+    case ATTN_ERR_ALIGNMENT: return "misaligned pointer";
+    case ATTN_ERR_CUDA: return "CUDA error";
+    case ATTN_ERR_TIMEOUT: return "pipeline wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int attn_prefill(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv,
+                 int Sq, int Skv, int D, int q_offset, int causal, float scale, int out_dtype, void* stream) {
+  int st = check_common(q, k, v, B, Hq, Hkv, Sq, Skv, D, q_offset, causal, scale);
+  if (st != ATTN_OK) return st;
+  if (out == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (out_dtype != ATTN_BF16 && out_dtype != ATTN_F32) return ATTN_ERR_INVALID_ARG;
+  if (D != 64 && D != 128 && D != 256) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16)) return ATTN_ERR_ALIGNMENT;
+  if (lse != nullptr && !aligned(lse, 4)) return ATTN_ERR_ALIGNMENT;
+
+  const int nslot = gqa::prefill_slots(D);
+  const int g = Hq / Hkv;
+  gqa::PrefillParams p{};
+  p.out = out;
+  p.lse = lse;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Sq = Sq; p.Skv = Skv;
+  p.q_offset = q_offset; p.causal = causal; p.out_f32 = (out_dtype == ATTN_F32);
+  p.g = g;
+  p.units_per_kvh = (g + nslot - 1) / nslot;
+  p.n_qt = (Sq + 127) / 128;
+  p.c2 = scale * kLog2e;
+  p.timeout_ns = kWaitLimitNs;
+  if ((long long)p.n_qt * B * Hkv * p.units_per_kvh > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+
+  p.status = status_ptr();
+  if (p.status == nullptr) return cuda_fail();
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q, D, Hq, Sq, B, 64, 1, 128, 1)) return cuda_fail();
+  if (!make_map(&tk, k, D, Hkv, Skv, B, 64, 1, 128, 1)) return cuda_fail();
+  if (!make_map(&tv, v, D, Hkv, Skv, B, 64, 1, 128, 1)) return cuda_fail();
+  return gqa::launch_prefill(D, tq, tk, tv, p, static_cast<cudaStream_t>(stream)) == 0 ? ATTN_OK
+                                                                                          : ATTN_ERR_CUDA;
+}
+
+size_t attn_decode_workspace_bytes(int B, int Hq, int Sq, int D, int num_splits) {
+  if (B < 1 || Hq < 1 || Sq < 1 || D < 1 || num_splits < 1) return 0;
+  const size_t n_out = (size_t)num_splits * B * Sq * Hq * D;
+  const size_t n_lse = (size_t)num_splits * B * Hq * Sq;
+  return (n_out + n_lse) * sizeof(float);
+}
+
+int attn_decode_split(const void* q, const void* k, const void* v, float* partial_out, float* partial_lse,
+                      int B, int Hq, int Hkv, int Sq, int Skv, int D, int q_offset, int causal, float scale,
+                      int num_splits, void* stream) {
+  int st = check_common(q, k, v, B, Hq, Hkv, Sq, Skv, D, q_offset, causal, scale);
+  if (st != ATTN_OK) return st;
+  if (partial_out == nullptr || partial_lse == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (num_splits < 1 || num_splits > Skv || num_splits > 65535) return ATTN_ERR_INVALID_ARG;
+  if (D != 128 && D != 256 && D != 512) return ATTN_ERR_UNSUPPORTED;
+  const int g = Hq / Hkv;
+  const long long R = (long long)g * Sq;
+  const long long RP = (R + 15) / 16 * 16;
+  if (RP * (1 + D / 128) > 256) return ATTN_ERR_UNSUPPORTED;
+  if (g > 256 || Sq > 256) return ATTN_ERR_UNSUPPORTED;  // TMA box extents
+  if ((long long)B * Hkv > 65535) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(partial_out, 16))
+    return ATTN_ERR_ALIGNMENT;
+  if (!aligned(partial_lse, 4)) return ATTN_ERR_ALIGNMENT;
+
+  gqa::DecodeParams p{};
+  p.part_out = partial_out;
+  p.part_lse = partial_lse;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Sq = Sq; p.Skv = Skv;
+  p.q_offset = q_offset; p.causal = causal;
+  p.g = g; p.R = (int)R; p.RP = (int)RP;
+  p.num_splits = num_splits;
+  p.chunk = (Skv + num_splits - 1) / num_splits;
+  int nbuf = 2;
+  while (nbuf < gqa::decode_max_nbuf() && gqa::decode_smem_bytes(D, p.RP, nbuf + 1) <= kTwoCtaSmemLimit) ++nbuf;
+  p.nbuf = nbuf;
+  p.c2 = scale * kLog2e;
+  p.timeout_ns = kWaitLimitNs;
+
+  p.status = status_ptr();
+  if (p.status == nullptr) return cuda_fail();
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q, D, Hq, Sq, B, 64, (uint32_t)g, (uint32_t)Sq, 1)) return cuda_fail();
+  if (!make_map(&tk, k, D, Hkv, Skv, B, 64, 1, 128, 1)) return cuda_fail();
+  if (!make_map(&tv, v, D, Hkv, Skv, B, 64, 1, 128, 1)) return cuda_fail();
+  return gqa::launch_decode_split(D, tq, tk, tv, p, static_cast<cudaStream_t>(stream)) == 0 ? ATTN_OK
+                                                                                               : ATTN_ERR_CUDA;
+}
+
+int attn_merge(const float* partial_out, const float* partial_lse, void* out, float* lse, int B, int Hq, int Sq,
+               int D, int num_splits, int out_dtype, void* stream) {
+  if (partial_out == nullptr || partial_lse == nullptr || out == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Sq < 1 || num_splits < 1) return ATTN_ERR_INVALID_ARG;
+  if (out_dtype != ATTN_BF16 && out_dtype != ATTN_F32) return ATTN_ERR_INVALID_ARG;
+  if (D < 4 || D > 1024 || D % 4 != 0) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned(partial_out, 16) || !aligned(out, out_dtype == ATTN_F32 ? 16 : 8)) return ATTN_ERR_ALIGNMENT;
+  if (!aligned(partial_lse, 4) || (lse != nullptr && !aligned(lse, 4))) return ATTN_ERR_ALIGNMENT;
+  gqa::MergeParams p{};
+  p.part_out = partial_out;
+  p.part_lse = partial_lse;
+  p.out = out;
+  p.lse = lse;
+  p.B = B; p.Hq = Hq; p.Sq = Sq; p.D = D; p.num_splits = num_splits;
+  p.out_f32 = (out_dtype == ATTN_F32);
+  return gqa::launch_merge(p, static_cast<cudaStream_t>(stream)) == 0 ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+int attn_last_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_CUDA;
+  int* sp = status_ptr();
+  if (sp == nullptr) return ATTN_ERR_CUDA;
+  int st = 0;
+  if (cudaMemcpy(&st, sp, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return ATTN_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpy(sp, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return ATTN_ERR_CUDA;
+  return st;
+}
+
+int attn_watchdog_selftest(unsigned long long limit_ns, void* stream) {
+  if (limit_ns < 1000ull) limit_ns = 1000ull;
+  if (limit_ns > 5000000000ull) limit_ns = 5000000000ull;
+  int* sp = status_ptr();
+  if (sp == nullptr) return ATTN_ERR_CUDA;
+  return gqa::launch_watchdog_selftest(sp, limit_ns, static_cast<cudaStream_t>(stream)) == 0 ? ATTN_OK
+                                                                                              : ATTN_ERR_CUDA;
+}
+
+}  // extern "C"

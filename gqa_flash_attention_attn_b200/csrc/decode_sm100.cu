@@ -1,0 +1,407 @@
+// Split-KV decode ("flash decoding") for sm_100a, swapped-operand form.
+//
+// A CTA owns one (split, batch, K/V head).  Its R = g*Sq query rows (all the
+// query heads of the group times the Sq draft rows) are the N side of the
+// MMAs, so the 128 keys of a tile fill the M = 128 side:
+//
+//   S^T [128 keys x RP rows]  = K_tile [128 x D] . Q^T        (tcgen05, TMEM)
+//   O^T [128 d    x RP rows] += V_tile^T [128 d x 128 keys] . P^T  per 128-d chunk
+//
+// The softmax warpgroup holds one key per thread (TMEM lane) and reduces each
+// row across the 128 keys with warp shuffles plus a cross-warp step in shared
+// memory ("Anbeeld/beellama.cpp PR #149", Overview: warp-shuffle reduction,
+// fp32 rescale, QB = 8 query rows per block for verify steps).  P is rounded
+// to bf16 into a 128-byte-swizzled shared buffer that the next MMA reads.
+//
+// Every split publishes its normalised partial O and its log-sum-exp, also
+// when it has no visible key (lse = -inf, O = 0) ("Anbeeld/beellama.cpp PR
+// #149", Overview, ub>64 fix: every block publishes its (max, rowsum)); the
+// merge is attn_merge.  The K/V stream is a ring of 32 KB slots (128 keys x
+// 128 columns, two TMA boxes) fed by one producer thread; the kernel is
+// HBM-bound, so the ring depth and two CTAs per SM set the bytes in flight.
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace gqa {
+namespace {
+
+constexpr int BN = 128;                        // keys per tile
+constexpr uint32_t BOX_BYTES = 128u * 128u;    // 128 rows x 64 bf16
+constexpr uint32_t SLOT_BYTES = 2u * BOX_BYTES;
+constexpr float LN2 = 0.6931471805599453f;
+constexpr int THREADS = 192;                   // warps 0-3 softmax, 4 producer, 5 MMA
+constexpr int WARP_PRODUCER = 4;
+constexpr int WARP_MMA = 5;
+constexpr int MAX_NBUF = 6;
+
+struct Layout {
+  uint32_t off_q, off_p, off_ring, off_red, off_row, off_bar, off_misc, total;
+  __host__ __device__ Layout(int D, int RP, int nbuf) {
+    off_q = 0;
+    const uint32_t qbytes = (uint32_t)(D / 64) * RP * 128u;
+    off_p = (off_q + qbytes + 1023u) & ~1023u;
+    off_ring = (off_p + 2u * RP * 128u + 1023u) & ~1023u;
+    off_red = off_ring + (uint32_t)nbuf * SLOT_BYTES;
+    off_row = off_red + 2u * 4u * RP * 4u;     // red_max[4][RP], red_sum[4][RP]
+    off_bar = off_row + 5u * RP * 4u;          // m, l, alpha, msub, inv
+    off_bar = (off_bar + 7u) & ~7u;
+    off_misc = off_bar + (uint32_t)(1 + 2 * nbuf + 4) * 8u;
+    total = off_misc + 16u + 1024u;
+  }
+};
+
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > limit_ns) break;
+  }
+}
+
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+template <int D>
+__global__ void __launch_bounds__(THREADS, 1)
+    decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
+  constexpr int KC = D / 128;  // 128-column slots per K (or V) tile
+  const int RP = p.RP, R = p.R, g = p.g, nbuf = p.nbuf;
+  const Layout L(D, RP, nbuf);
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  float* red_max = reinterpret_cast<float*>(gbase + L.off_red);
+  float* red_sum = red_max + 4 * RP;
+  float* m_sm = reinterpret_cast<float*>(gbase + L.off_row);
+  float* l_sm = m_sm + RP;
+  float* alpha_sm = l_sm + RP;
+  float* msub_sm = alpha_sm + RP;
+  float* inv_sm = msub_sm + RP;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L.off_misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L.off_misc + 4);
+  volatile int* resc_flag = reinterpret_cast<volatile int*>(gbase + L.off_misc + 8);
+  auto bar = [&](int i) -> uint32_t { return base + L.off_bar + 8u * (uint32_t)i; };
+  const int BAR_Q = 0;
+  auto bar_full = [&](int s) { return 1 + s; };
+  auto bar_empty = [&](int s) { return 1 + nbuf + s; };
+  const int BAR_S = 1 + 2 * nbuf, BAR_P = BAR_S + 1, BAR_PV = BAR_S + 2, BAR_DRAIN = BAR_S + 3;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int split = blockIdx.x;
+  const int b = blockIdx.y / p.Hkv, kvh = blockIdx.y % p.Hkv;
+  const long long lo_ll = (long long)split * p.chunk;
+  const int lo = (int)min(lo_ll, (long long)p.Skv);
+  const int hi = (int)min(lo_ll + p.chunk, (long long)p.Skv);
+  const int eff_hi = p.causal ? min(hi, p.q_offset + p.Sq) : hi;
+  const int n_tiles = eff_hi > lo ? (eff_hi - lo + BN - 1) / BN : 0;
+  const size_t split_out = (size_t)split * p.B * p.Sq * p.Hq * D;
+  const size_t split_lse = (size_t)split * p.B * p.Hq * p.Sq;
+
+  if (n_tiles == 0) {
+    // No visible key in this split: publish (-inf, 0) for every row.
+    for (int i = threadIdx.x; i < R * D; i += THREADS) {
+      const int r = i / D, d = i - r * D;
+      const int s = r / g, h = kvh * g + (r - s * g);
+      p.part_out[split_out + (((size_t)b * p.Sq + s) * p.Hq + h) * D + d] = 0.f;
+    }
+    for (int r = threadIdx.x; r < R; r += THREADS) {
+      const int s = r / g, h = kvh * g + (r - s * g);
+      p.part_lse[split_lse + ((size_t)b * p.Hq + h) * p.Sq + s] = -INFINITY;
+    }
+    return;
+  }
+
+  // Zero the padding rows of Q (rows R..RP-1 of every 64-column box).
+  for (int i = threadIdx.x; i < (D / 64) * (RP - R) * 32; i += THREADS) {
+    const int box = i / ((RP - R) * 32);
+    const int w = i - box * (RP - R) * 32;
+    reinterpret_cast<uint32_t*>(gbase + L.off_q + (uint32_t)box * RP * 128u + (uint32_t)R * 128u)[w] = 0u;
+  }
+  if (threadIdx.x < RP) {
+    m_sm[threadIdx.x] = -INFINITY;
+    l_sm[threadIdx.x] = 0.f;
+  }
+  if (threadIdx.x == 0) {
+    mbar_init(bar(BAR_Q), 1);
+    for (int s = 0; s < nbuf; ++s) {
+      mbar_init(bar(bar_full(s)), 1);
+      mbar_init(bar(bar_empty(s)), 1);
+    }
+    mbar_init(bar(BAR_S), 1);
+    mbar_init(bar(BAR_P), 128);
+    mbar_init(bar(BAR_PV), 1);
+    mbar_init(bar(BAR_DRAIN), 1);
+    *abort_flag = 0;
+    *resc_flag = 0;
+    fence_mbar_init();
+  }
+  uint32_t tmem_cols = 32;
+  while (tmem_cols < (uint32_t)(RP * (1 + KC))) tmem_cols <<= 1;
+  if (warp == WARP_MMA) {
+    tmem_alloc(smem_u32(tmem_slot), tmem_cols);
+    tmem_relinquish();
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t TS = 0;                           // S^T: RP columns
+  auto TO = [&](int c) { return (uint32_t)(RP * (1 + c)); };  // O^T chunk c
+  const Watchdog wd{abort_flag, p.status, p.timeout_ns};
+  int issued = 0;
+
+  if (warp == WARP_PRODUCER) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_arrive_expect_tx(bar(BAR_Q), (uint32_t)(D / 64) * R * 128u);
+      for (int kb = 0; kb < D / 64; ++kb)
+        tma_load_4d(base + L.off_q + (uint32_t)kb * RP * 128u, &tm_q, bar(BAR_Q), kb * 64, kvh * g, 0, b);
+      const int total = n_tiles * 2 * KC;
+      for (int n = 0; n < total; ++n) {
+        const int slot = n % nbuf, use = n / nbuf;
+        if (use > 0 && !mbar_wait(bar(bar_empty(slot)), (uint32_t)(use - 1) & 1u, wd)) break;
+        const int j = n / (2 * KC), within = n - j * 2 * KC;
+        const bool is_v = within >= KC;
+        const int c = is_v ? within - KC : within;
+        const CUtensorMap* tm = is_v ? &tm_v : &tm_k;
+        const int key0 = lo + j * BN;
+        mbar_arrive_expect_tx(bar(bar_full(slot)), SLOT_BYTES);
+        const uint32_t dst = base + L.off_ring + (uint32_t)slot * SLOT_BYTES;
+        tma_load_4d(dst, tm, bar(bar_full(slot)), (2 * c) * 64, kvh, key0, b);
+        tma_load_4d(dst + BOX_BYTES, tm, bar(bar_full(slot)), (2 * c + 1) * 64, kvh, key0, b);
+        issued = n + 1;
+      }
+    }
+  } else if (warp == WARP_MMA) {
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_bf16_f32(128, RP, false, false);
+      const uint32_t idesc_o = idesc_bf16_f32(128, RP, true, false);
+      bool ok = mbar_wait(bar(BAR_Q), 0, wd);
+      tc_fence_after();
+      int n = 0;
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        // S^T = K Q^T over D, one 128-column slot at a time
+        for (int c = 0; ok && c < KC; ++c, ++n) {
+          const int slot = n % nbuf;
+          if (!mbar_wait(bar(bar_full(slot)), (uint32_t)(n / nbuf) & 1u, wd)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t kb = base + L.off_ring + (uint32_t)slot * SLOT_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t in_box = (uint32_t)(kk & 3) * 32u;
+            const uint32_t a = kb + (uint32_t)(kk >> 2) * BOX_BYTES + in_box;
+            const uint32_t qb = base + L.off_q + (uint32_t)(2 * c + (kk >> 2)) * RP * 128u + in_box;
+            mma_ss(tmem + TS, sdesc_sw128(a, 16, 1024), sdesc_sw128(qb, 16, 1024), idesc_s,
+                   (c > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(bar(bar_empty(slot)));
+        }
+        if (!ok) break;
+        mma_commit(bar(BAR_S));
+        if (!mbar_wait(bar(BAR_P), (uint32_t)j & 1u, wd)) { ok = false; break; }
+        tc_fence_after();
+        // O^T(c) += V^T(c) P^T
+        for (int c = 0; ok && c < KC; ++c, ++n) {
+          const int slot = n % nbuf;
+          if (!mbar_wait(bar(bar_full(slot)), (uint32_t)(n / nbuf) & 1u, wd)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t vb = base + L.off_ring + (uint32_t)slot * SLOT_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t a = vb + (uint32_t)kk * 2048u;
+            const uint32_t pb = base + L.off_p + (uint32_t)(kk >> 2) * RP * 128u + (uint32_t)(kk & 3) * 32u;
+            mma_ss(tmem + TO(c), sdesc_sw128(a, BOX_BYTES, 1024), sdesc_sw128(pb, 16, 1024), idesc_o,
+                   (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(bar(bar_empty(slot)));
+        }
+        if (!ok) break;
+        mma_commit(bar(BAR_PV));
+      }
+    }
+  } else {
+    // ---- softmax: thread t <-> key t of the tile (TMEM lane t) ----
+    const int t = threadIdx.x;          // 0..127
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const float c2 = p.c2;
+    uint8_t* pbuf = gbase + L.off_p;
+    bool ok = true;
+    for (int j = 0; j < n_tiles; ++j) {
+      // every give-up is decided jointly (barrier + OR) so no thread is left
+      // waiting at a named barrier or inside a warp-collective TMEM access
+      const bool got_s = mbar_wait(bar(BAR_S), (uint32_t)j & 1u, wd);
+      if (named_bar_or(1, 128, !got_s)) { ok = false; break; }
+      tc_fence_after();
+      const int key = lo + j * BN + t;
+      const bool key_ok = key < hi;
+      // pass 1: per-row max over the tile's visible keys
+      for (int q = 0; q < RP / 16; ++q) {
+        float v[16];
+        tmem_ld16(tmem + lane_off + TS + 16 * q, v);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int r = 16 * q + e;
+          const bool vis = key_ok && r < R && (!p.causal || key <= p.q_offset + r / g);
+          const float x = warp_max(vis ? v[e] : -INFINITY);
+          if (lane == 0) red_max[warp * RP + r] = x;
+        }
+      }
+      named_bar_sync(1, 128);
+      if (t < RP) {
+        const float mt = fmaxf(fmaxf(red_max[t], red_max[RP + t]), fmaxf(red_max[2 * RP + t], red_max[3 * RP + t]));
+        const float m_tile = mt * c2;
+        const float m_old = m_sm[t];
+        float m_new = m_old, alpha = 1.f;
+        if (m_tile > m_old + 8.f) {
+          m_new = m_tile;
+          alpha = ex2_approx(m_old - m_new);
+          *resc_flag = 1;
+        }
+        m_sm[t] = m_new;
+        alpha_sm[t] = alpha;
+        msub_sm[t] = (m_new == -INFINITY) ? 0.f : m_new;
+      }
+      // P (and O) of the previous tile must be consumed before they change
+      const bool got_pv = (j == 0) || mbar_wait(bar(BAR_PV), (uint32_t)(j - 1) & 1u, wd);
+      if (named_bar_or(1, 128, !got_pv)) { ok = false; break; }
+      tc_fence_after();
+      const bool rescale = (j > 0) && (*resc_flag != 0);
+      // pass 2: exponentials, P (bf16) into the swizzled B-operand buffer
+      {
+        const int half = t >> 6, tt = t & 63;
+        uint8_t* pcol = pbuf + (size_t)half * RP * 128 + (size_t)(tt & 7) * 2;
+        const int chunk16 = tt >> 3;
+        for (int q = 0; q < RP / 16; ++q) {
+          float v[16];
+          tmem_ld16(tmem + lane_off + TS + 16 * q, v);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int r = 16 * q + e;
+            const bool vis = key_ok && r < R && (!p.causal || key <= p.q_offset + r / g);
+            const float pv = vis ? ex2_approx(fmaf(v[e], c2, -msub_sm[r])) : 0.f;
+            *reinterpret_cast<__nv_bfloat16*>(pcol + (size_t)r * 128 + ((chunk16 ^ (r & 7)) << 4)) =
+                __float2bfloat16_rn(pv);
+            const float s = warp_sum(pv);
+            if (lane == 0) red_sum[warp * RP + r] = s;
+          }
+        }
+      }
+      if (rescale) {
+        for (int c = 0; c < KC; ++c) {
+          for (int q = 0; q < RP / 16; ++q) {
+            float v[16];
+            const uint32_t addr = tmem + lane_off + TO(c) + 16 * q;
+            tmem_ld16(addr, v);
+            uint32_t u[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) u[e] = __float_as_uint(v[e] * alpha_sm[16 * q + e]);
+            tmem_st16(addr, u);
+          }
+        }
+      }
+      named_bar_sync(1, 128);
+      if (t < RP) {
+        l_sm[t] = alpha_sm[t] * l_sm[t] + (red_sum[t] + red_sum[RP + t]) + (red_sum[2 * RP + t] + red_sum[3 * RP + t]);
+      }
+      if (t == 0) *resc_flag = 0;
+      fence_proxy_async_smem();
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(BAR_P));
+    }
+    // ---- epilogue: normalised partial O and the split's LSE ----
+    const bool got_o = ok && mbar_wait(bar(BAR_PV), (uint32_t)(n_tiles - 1) & 1u, wd);
+    if (ok && !named_bar_or(1, 128, !got_o)) {
+      tc_fence_after();
+      if (t < RP) {
+        const float l = l_sm[t];
+        inv_sm[t] = l > 0.f ? 1.f / l : 0.f;
+        if (t < R) {
+          const int s = t / g, h = kvh * g + (t - s * g);
+          p.part_lse[split_lse + ((size_t)b * p.Hq + h) * p.Sq + s] =
+              l > 0.f ? (m_sm[t] + log2f(l)) * LN2 : -INFINITY;
+        }
+      }
+      named_bar_sync(1, 128);
+      for (int c = 0; c < KC; ++c) {
+        for (int q = 0; q < RP / 16; ++q) {
+          float v[16];
+          tmem_ld16(tmem + lane_off + TO(c) + 16 * q, v);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int r = 16 * q + e;
+            if (r < R) {
+              const int s = r / g, h = kvh * g + (r - s * g);
+              p.part_out[split_out + (((size_t)b * p.Sq + s) * p.Hq + h) * D + c * 128 + t] = v[e] * inv_sm[r];
+            }
+          }
+        }
+      }
+    }
+    tc_fence_before();
+  }
+
+  __syncwarp();
+  __syncthreads();
+  if (*abort_flag) {
+    if (warp == WARP_PRODUCER && lane == 0) {
+      drain_wait(bar(BAR_Q), 0, p.timeout_ns);
+      for (int n = max(0, issued - nbuf); n < issued; ++n)
+        drain_wait(bar(bar_full(n % nbuf)), (uint32_t)(n / nbuf) & 1u, p.timeout_ns);
+    }
+    if (warp == WARP_MMA && lane == 0) {
+      mma_commit(bar(BAR_DRAIN));
+      drain_wait(bar(BAR_DRAIN), 0, p.timeout_ns);
+    }
+    __syncwarp();
+    __syncthreads();
+  }
+  if (warp == WARP_MMA) {
+    tc_fence_after();
+    tmem_dealloc(tmem, tmem_cols);
+  }
+}
+
+template <int D>
+int launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+             const DecodeParams& p, cudaStream_t stream) {
+  const Layout L(D, p.RP, p.nbuf);
+  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)L.total);
+  if (e != cudaSuccess) return (int)e;
+  dim3 grid((unsigned)p.num_splits, (unsigned)(p.B * p.Hkv));
+  decode_split_kernel<D><<<grid, THREADS, L.total, stream>>>(tq, tk, tv, p);
+  return (int)cudaGetLastError();
+}
+
+}  // namespace
+
+size_t decode_smem_bytes(int D, int RP, int nbuf) { return Layout(D, RP, nbuf).total; }
+
+int decode_max_nbuf() { return MAX_NBUF; }
+
+int launch_decode_split(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                        const DecodeParams& p, cudaStream_t stream) {
+  switch (D) {
+    case 128: return launch_t<128>(tq, tk, tv, p, stream);
+    case 256: return launch_t<256>(tq, tk, tv, p, stream);
+    case 512: return launch_t<512>(tq, tk, tv, p, stream);
+    default: return (int)cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace gqa

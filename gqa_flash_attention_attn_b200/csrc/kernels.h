@@ -1,0 +1,51 @@
+// Internal interface between the C-ABI layer (abi.cu) and the kernels.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace gqa {
+
+struct PrefillParams {
+  void* out;          // [B, Sq, Hq, D] bf16 or f32
+  float* lse;         // [B, Hq, Sq] or nullptr
+  int* status;        // device status word
+  int B, Hq, Hkv, Sq, Skv, q_offset, causal, out_f32;
+  int g;              // Hq / Hkv
+  int units_per_kvh;  // head slots per K/V head: ceil(g / NSLOT)
+  int n_qt;           // ceil(Sq / 128)
+  float c2;           // scale * log2(e)
+  unsigned long long timeout_ns;
+};
+
+struct DecodeParams {
+  float* part_out;    // [S, B, Sq, Hq, D]
+  float* part_lse;    // [S, B, Hq, Sq]
+  int* status;
+  int B, Hq, Hkv, Sq, Skv, q_offset, causal;
+  int g, R, RP;       // rows per K/V head = g*Sq, padded to a multiple of 16
+  int num_splits, chunk;  // keys per split
+  int nbuf;           // K/V ring slots (32 KB each)
+  float c2;
+  unsigned long long timeout_ns;
+};
+
+struct MergeParams {
+  const float* part_out;
+  const float* part_lse;
+  void* out;
+  float* lse;
+  int B, Hq, Sq, D, num_splits, out_f32;
+};
+
+// Each returns a cudaError_t value (as int) from the launch.
+int launch_prefill(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                   const PrefillParams& p, cudaStream_t stream);
+size_t prefill_smem_bytes(int D);
+int launch_decode_split(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                        const DecodeParams& p, cudaStream_t stream);
+size_t decode_smem_bytes(int D, int RP, int nbuf);
+int launch_merge(const MergeParams& p, cudaStream_t stream);
+int launch_watchdog_selftest(int* status, unsigned long long limit_ns, cudaStream_t stream);
+
+}  // namespace gqa

@@ -1,0 +1,97 @@
+// Merge of split-KV partials by their log-sum-exp, plus the watchdog self-test.
+//
+// For each output row: M = max_s lse_s, w_s = exp(lse_s - M),
+// out = sum_s w_s O_s / sum_s w_s, lse = M + log(sum_s w_s); splits that
+// published lse = -inf carry weight 0 ("Anbeeld/beellama.cpp PR #149", review
+// of the combine kernel that merges per-block partials for parallel_blocks > 1).
+//
+// HBM-bound: each thread owns 4 consecutive columns of one row (a float4 of
+// every split's partial), so consecutive threads read consecutive 16-byte
+// words of each partial row.
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace gqa {
+namespace {
+
+__global__ void __launch_bounds__(128) merge_kernel(const MergeParams p) {
+  const int f4_per_row = p.D / 4;
+  const long long rows = (long long)p.B * p.Sq * p.Hq;
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= rows * f4_per_row) return;
+  const long long row = idx / f4_per_row;          // (b, s, h) in O order
+  const int f = (int)(idx - row * f4_per_row);
+  const int h = (int)(row % p.Hq);
+  const int s = (int)((row / p.Hq) % p.Sq);
+  const int b = (int)(row / ((long long)p.Hq * p.Sq));
+  const size_t lse_row = ((size_t)b * p.Hq + h) * p.Sq + s;
+  const size_t lse_stride = (size_t)p.B * p.Hq * p.Sq;
+  const size_t out_stride = (size_t)rows * p.D;
+
+  float M = -INFINITY;
+  for (int sg = 0; sg < p.num_splits; ++sg) M = fmaxf(M, __ldg(p.part_lse + sg * lse_stride + lse_row));
+
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float wsum = 0.f;
+  if (M != -INFINITY) {
+    const float4* src = reinterpret_cast<const float4*>(p.part_out + (size_t)row * p.D) + f;
+    for (int sg = 0; sg < p.num_splits; ++sg) {
+      const float x = __ldg(p.part_lse + sg * lse_stride + lse_row);
+      if (x == -INFINITY) continue;
+      const float w = expf(x - M);
+      const float4 o = __ldg(src + sg * (out_stride / 4));
+      wsum += w;
+      acc.x = fmaf(w, o.x, acc.x);
+      acc.y = fmaf(w, o.y, acc.y);
+      acc.z = fmaf(w, o.z, acc.z);
+      acc.w = fmaf(w, o.w, acc.w);
+    }
+    const float inv = 1.f / wsum;
+    acc.x *= inv;
+    acc.y *= inv;
+    acc.z *= inv;
+    acc.w *= inv;
+  }
+  const size_t o_off = (size_t)row * p.D + 4 * (size_t)f;
+  if (p.out_f32) {
+    *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + o_off) = acc;
+  } else {
+    *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.out) + o_off) =
+        make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+  }
+  if (f == 0 && p.lse != nullptr) p.lse[lse_row] = (M == -INFINITY) ? -INFINITY : M + logf(wsum);
+}
+
+// One thread waits on an mbarrier that nothing completes; the bounded wait
+// gives up after limit_ns and records the timeout status.
+__global__ void watchdog_selftest_kernel(int* status, unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t mbar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&mbar), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const Watchdog wd{&abort_flag, status, limit_ns};
+    (void)mbar_wait(smem_u32(&mbar), 0, wd);
+  }
+}
+
+}  // namespace
+
+int launch_merge(const MergeParams& p, cudaStream_t stream) {
+  const long long total = (long long)p.B * p.Sq * p.Hq * (p.D / 4);
+  const long long blocks = (total + 127) / 128;
+  if (blocks <= 0 || blocks > 0x7fffffffLL) return (int)cudaErrorInvalidValue;
+  merge_kernel<<<(unsigned)blocks, 128, 0, stream>>>(p);
+  return (int)cudaGetLastError();
+}
+
+int launch_watchdog_selftest(int* status, unsigned long long limit_ns, cudaStream_t stream) {
+  watchdog_selftest_kernel<<<1, 32, 0, stream>>>(status, limit_ns);
+  return (int)cudaGetLastError();
+}
+
+}  // namespace gqa

@@ -1,0 +1,385 @@
+// Flash-attention prefill forward for sm_100a.
+//
+// One CTA owns a "unit": one 128-row query tile for NSLOT query heads of the
+// same K/V group (NSLOT = 2 for D <= 128, 1 for D = 256), so every K/V tile it
+// stages in shared memory serves NSLOT heads ("ggml-org/llama.cpp PR #28507",
+// Setup: GQA 8; K/V shared-memory staging reused across the query rows of a
+// block).  Roles, one warp each unless noted:
+//
+//   producer   TMA 4-D tiled loads (128-byte swizzle, 64-column boxes): Q once,
+//              then K_0, V_0, K_1, V_1, ... through an NBUF-slot mbarrier ring.
+//   MMA        one thread issues tcgen05.mma: S_i = Q_i K_j^T (both operands in
+//              shared memory, fp32 accumulator in TMEM), then O_i += P_i V_j
+//              with P_i read from TMEM (A operand) and V_j from shared memory.
+//   softmax    one warpgroup per slot, one thread per query row (TMEM lane):
+//              online softmax in fp32 with the running (max, rowsum) per row
+//              ("Anbeeld/beellama.cpp PR #149", Overview: fp32 rescale and
+//              (max, rowsum) metadata), scale*log2(e) folded into the single
+//              FFMA in front of exp2 ("AstrAI commit log,
+//              gqa_prefill_attn_mma.cuh": pre-scaled Q, here without rounding
+//              Q*scale to bf16), P rounded to bf16 into TMEM, O rescaled in
+//              TMEM only when the running max grew by more than 2^8.
+//
+// Causal masking: key t is visible to row s iff t <= q_offset + s; tiles past
+// the last row's diagonal are never loaded.  Every pipeline wait is bounded:
+// on expiry the CTA records a timeout status, drains its own copies and MMAs,
+// frees TMEM and exits.
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace gqa {
+namespace {
+
+constexpr int BM = 128;   // query rows per slot (TMEM lanes)
+constexpr int BN = 128;   // keys per tile
+constexpr uint32_t BOX_BYTES = 128u * 128u;  // 128 rows x 64 bf16 columns
+constexpr float LN2 = 0.6931471805599453f;
+
+template <int D>
+struct PrefillCfg {
+  static constexpr int NSLOT = (D <= 128) ? 2 : 1;
+  static constexpr int KB = D / 64;
+  static constexpr uint32_t TILE = KB * BOX_BYTES;
+  static constexpr int NBUF = (D == 64) ? 8 : (D == 128 ? 4 : 2);
+  static constexpr int THREADS = 128 * NSLOT + 64;
+  static constexpr int WARP_PRODUCER = 4 * NSLOT;
+  static constexpr int WARP_MMA = 4 * NSLOT + 1;
+  static constexpr uint32_t OFF_Q = 0;
+  static constexpr uint32_t OFF_KV = NSLOT * TILE;
+  static constexpr uint32_t OFF_BAR = OFF_KV + NBUF * TILE;
+  // q_full, kv_full[NBUF], kv_empty[NBUF], s_full[2], p_full[2], pv_done[2], drain
+  static constexpr int NBARS = 1 + 2 * NBUF + 6 + 1;
+  static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
+  static constexpr uint32_t SMEM = OFF_MISC + 16 + 1024;  // + alignment slack
+  static constexpr uint32_t TMEM_S = 0;                   // S_i (and P_i) at i*128
+  static constexpr uint32_t TMEM_O = NSLOT * 128;         // O_i at TMEM_O + i*D
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr int BAR_Q = 0;
+  __host__ __device__ static constexpr int bar_full(int b) { return 1 + b; }
+  __host__ __device__ static constexpr int bar_empty(int b) { return 1 + NBUF + b; }
+  __host__ __device__ static constexpr int bar_s(int i) { return 1 + 2 * NBUF + i; }
+  __host__ __device__ static constexpr int bar_p(int i) { return 3 + 2 * NBUF + i; }
+  __host__ __device__ static constexpr int bar_pv(int i) { return 5 + 2 * NBUF + i; }
+  static constexpr int BAR_DRAIN = 7 + 2 * NBUF;
+  static_assert(NSLOT * 128 + NSLOT * D <= 512, "TMEM budget");
+  static_assert(SMEM <= 232448, "shared memory budget");
+  static_assert(D % 64 == 0, "head dim must be a multiple of 64");
+};
+
+// Wait that ignores the abort flag: used only to drain in-flight work.
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > limit_ns) break;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
+  using C = PrefillCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + C::OFF_MISC + 4);
+  auto bar = [&](int i) -> uint32_t { return base + C::OFF_BAR + 8u * (uint32_t)i; };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- which unit: (q-tile, batch, K/V head, slot group), longest first ----
+  const int upk = p.units_per_kvh;
+  const int units_per_qt = p.B * p.Hkv * upk;
+  const int u = blockIdx.x;
+  const int qt_rev = u / units_per_qt;
+  int rem = u - qt_rev * units_per_qt;
+  const int b = rem / (p.Hkv * upk);
+  rem -= b * (p.Hkv * upk);
+  const int kvh = rem / upk;
+  const int grp = rem - kvh * upk;
+  const int qt = p.causal ? (p.n_qt - 1 - qt_rev) : qt_rev;
+  const int s0 = qt * BM;
+  const int hl0 = grp * C::NSLOT;  // local head of slot 0 inside the group
+  const int kv_end = p.causal ? min(p.Skv, p.q_offset + min(s0 + BM, p.Sq)) : p.Skv;
+  const int n_tiles = (kv_end + BN - 1) / BN;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(C::BAR_Q), 1);
+    for (int i = 0; i < C::NBUF; ++i) {
+      mbar_init(bar(C::bar_full(i)), 1);
+      mbar_init(bar(C::bar_empty(i)), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(C::bar_s(i)), 1);
+      mbar_init(bar(C::bar_p(i)), 128);
+      mbar_init(bar(C::bar_pv(i)), 1);
+    }
+    mbar_init(bar(C::BAR_DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == C::WARP_MMA) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Watchdog wd{abort_flag, p.status, p.timeout_ns};
+
+  int issued = 0;  // producer: K/V blocks issued
+
+  if (warp == C::WARP_PRODUCER) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      int nact = 0;
+      for (int i = 0; i < C::NSLOT; ++i) nact += (hl0 + i < p.g) ? 1 : 0;
+      mbar_arrive_expect_tx(bar(C::BAR_Q), (uint32_t)nact * C::TILE);
+      for (int i = 0; i < C::NSLOT; ++i) {
+        if (hl0 + i >= p.g) continue;
+        const int h = kvh * p.g + hl0 + i;
+        for (int kb = 0; kb < C::KB; ++kb)
+          tma_load_4d(base + C::OFF_Q + i * C::TILE + kb * BOX_BYTES, &tm_q, bar(C::BAR_Q), kb * 64, h,
+                      s0, b);
+      }
+      for (int n = 0; n < 2 * n_tiles; ++n) {
+        const int buf = n % C::NBUF;
+        const int use = n / C::NBUF;
+        if (use > 0 && !mbar_wait(bar(C::bar_empty(buf)), (uint32_t)(use - 1) & 1u, wd)) break;
+        const CUtensorMap* tm = (n & 1) ? &tm_v : &tm_k;
+        const int key0 = (n >> 1) * BN;
+        mbar_arrive_expect_tx(bar(C::bar_full(buf)), C::TILE);
+        for (int kb = 0; kb < C::KB; ++kb)
+          tma_load_4d(base + C::OFF_KV + buf * C::TILE + kb * BOX_BYTES, tm, bar(C::bar_full(buf)),
+                      kb * 64, kvh, key0, b);
+        issued = n + 1;
+      }
+    }
+  } else if (warp == C::WARP_MMA) {
+    if (lane == 0) {
+      constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, false, false);
+      constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, false, true);
+      bool ok = mbar_wait(bar(C::BAR_Q), 0, wd);
+      tc_fence_after();
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        // ---- S_i = Q_i K_j^T ----
+        const int nk = 2 * j, bk = nk % C::NBUF;
+        if (!mbar_wait(bar(C::bar_full(bk)), (uint32_t)(nk / C::NBUF) & 1u, wd)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t kbase = base + C::OFF_KV + bk * C::TILE;
+        for (int i = 0; ok && i < C::NSLOT; ++i) {
+          if (hl0 + i >= p.g) continue;
+          if (j > 0) {  // S_i aliases P_i, which the previous P.V reads
+            if (!mbar_wait(bar(C::bar_pv(i)), (uint32_t)(j - 1) & 1u, wd)) { ok = false; break; }
+            tc_fence_after();
+          }
+          const uint32_t qbase = base + C::OFF_Q + i * C::TILE;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (uint32_t)(kk >> 2) * BOX_BYTES + (uint32_t)(kk & 3) * 32u;
+            mma_ss(tmem + C::TMEM_S + i * 128, sdesc_sw128(qbase + off, 16, 1024),
+                   sdesc_sw128(kbase + off, 16, 1024), IDESC_QK, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar(C::bar_s(i)));
+        }
+        if (!ok) break;
+        mma_commit(bar(C::bar_empty(bk)));
+        // ---- O_i += P_i V_j ----
+        const int nv = nk + 1, bv = nv % C::NBUF;
+        if (!mbar_wait(bar(C::bar_full(bv)), (uint32_t)(nv / C::NBUF) & 1u, wd)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t vbase = base + C::OFF_KV + bv * C::TILE;
+        for (int i = 0; ok && i < C::NSLOT; ++i) {
+          if (hl0 + i >= p.g) continue;
+          if (!mbar_wait(bar(C::bar_p(i)), (uint32_t)j & 1u, wd)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            mma_ts(tmem + C::TMEM_O + i * D, tmem + C::TMEM_S + i * 128 + kk * 8,
+                   sdesc_sw128(vbase + kk * 2048u, BOX_BYTES, 1024), IDESC_PV,
+                   (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(bar(C::bar_pv(i)));
+        }
+        if (!ok) break;
+        mma_commit(bar(C::bar_empty(bv)));
+      }
+    }
+  } else {
+    // ---- softmax warpgroups: warp w serves slot w/4, TMEM lanes 32*(w%4).. ----
+    const int slot = warp >> 2;
+    const int wq = warp & 3;
+    const int hl = hl0 + slot;
+    if (hl < p.g) {
+      const int h = kvh * p.g + hl;
+      const int r = wq * 32 + lane;
+      const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+      const uint32_t tS = tmem + lane_off + C::TMEM_S + slot * 128;
+      const uint32_t tO = tmem + lane_off + C::TMEM_O + slot * D;
+      const int s_row = s0 + r;
+      const int vis_end = p.causal ? min(p.Skv, p.q_offset + s_row + 1) : p.Skv;
+      const float c2 = p.c2;
+      float m_use = -INFINITY, l = 0.f;
+      bool ok = true;
+      for (int j = 0; j < n_tiles; ++j) {
+        // a give-up must be warp-uniform: TMEM loads/stores are warp-collective
+        const bool got = mbar_wait(bar(C::bar_s(slot)), (uint32_t)j & 1u, wd);
+        if (__any_sync(0xffffffffu, !got)) { ok = false; break; }
+        tc_fence_after();
+        const int cl = vis_end - j * BN;  // visible columns of this tile for this row
+        const bool masked = cl < BN;
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) {
+          float v[32];
+          tmem_ld32(tS + 32 * c, v);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float x = (masked && (32 * c + e) >= cl) ? -INFINITY : v[e];
+            mx = fmaxf(mx, x);
+          }
+        }
+        const float m_tile = mx * c2;
+        float m_new = m_use, alpha = 1.f;
+        if (m_tile > m_use + 8.f) {
+          m_new = m_tile;
+          alpha = ex2_approx(m_use - m_new);
+        }
+        const float m_sub = (m_new == -INFINITY) ? 0.f : m_new;
+        float sum = 0.f;
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) {
+          float v[32];
+          tmem_ld32(tS + 32 * c, v);
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            float p0 = ex2_approx(fmaf(v[2 * e], c2, -m_sub));
+            float p1 = ex2_approx(fmaf(v[2 * e + 1], c2, -m_sub));
+            if (masked) {
+              if (32 * c + 2 * e >= cl) p0 = 0.f;
+              if (32 * c + 2 * e + 1 >= cl) p1 = 0.f;
+            }
+            sum += p0 + p1;
+            pk[e] = pack_bf16x2(p0, p1);
+          }
+          // P chunk c lands on TMEM columns [16c, 16c+16), already read as S.
+          tmem_st16(tS + 16 * c, pk);
+        }
+        l = l * alpha + sum;
+        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+          // s_full(j) completing implies the previous P.V into O_i completed.
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            float v[32];
+            tmem_ld32(tO + 32 * c, v);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] *= alpha;
+            tmem_st32(tO + 32 * c, v);
+          }
+        }
+        m_use = m_new;
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(C::bar_p(slot)));
+      }
+      const bool got_o = ok && mbar_wait(bar(C::bar_pv(slot)), (uint32_t)(n_tiles - 1) & 1u, wd);
+      if (!__any_sync(0xffffffffu, !got_o)) {
+        tc_fence_after();
+        const float inv_l = 1.f / l;
+        const bool row_ok = s_row < p.Sq;
+        const size_t row_off = (((size_t)b * p.Sq + s_row) * p.Hq + h) * (size_t)D;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          float v[32];
+          tmem_ld32(tO + 32 * c, v);
+          if (row_ok) {
+            if (p.out_f32) {
+              float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + row_off + 32 * c);
+#pragma unroll
+              for (int q4 = 0; q4 < 8; ++q4)
+                dst[q4] = make_float4(v[4 * q4] * inv_l, v[4 * q4 + 1] * inv_l, v[4 * q4 + 2] * inv_l,
+                                      v[4 * q4 + 3] * inv_l);
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + row_off + 32 * c);
+#pragma unroll
+              for (int q8 = 0; q8 < 4; ++q8)
+                dst[q8] = make_uint4(pack_bf16x2(v[8 * q8] * inv_l, v[8 * q8 + 1] * inv_l),
+                                     pack_bf16x2(v[8 * q8 + 2] * inv_l, v[8 * q8 + 3] * inv_l),
+                                     pack_bf16x2(v[8 * q8 + 4] * inv_l, v[8 * q8 + 5] * inv_l),
+                                     pack_bf16x2(v[8 * q8 + 6] * inv_l, v[8 * q8 + 7] * inv_l));
+            }
+          }
+        }
+        if (row_ok && p.lse != nullptr)
+          p.lse[((size_t)b * p.Hq + h) * p.Sq + s_row] = (m_use + log2f(l)) * LN2;
+      }
+      tc_fence_before();
+    }
+  }
+
+  __syncwarp();
+  __syncthreads();
+  if (*abort_flag) {
+    // Nothing may still write this CTA's shared memory or TMEM when it exits.
+    if (warp == C::WARP_PRODUCER && lane == 0) {
+      drain_wait(bar(C::BAR_Q), 0, p.timeout_ns);
+      for (int n = max(0, issued - C::NBUF); n < issued; ++n)
+        drain_wait(bar(C::bar_full(n % C::NBUF)), (uint32_t)(n / C::NBUF) & 1u, p.timeout_ns);
+    }
+    if (warp == C::WARP_MMA && lane == 0) {
+      mma_commit(bar(C::BAR_DRAIN));
+      drain_wait(bar(C::BAR_DRAIN), 0, p.timeout_ns);
+    }
+    __syncwarp();
+    __syncthreads();
+  }
+  if (warp == C::WARP_MMA) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int D>
+int launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+             const PrefillParams& p, cudaStream_t stream) {
+  using C = PrefillCfg<D>;
+  cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)C::SMEM);
+  if (e != cudaSuccess) return (int)e;
+  const long long units = (long long)p.n_qt * p.B * p.Hkv * p.units_per_kvh;
+  if (units <= 0 || units > 0x7fffffffLL) return (int)cudaErrorInvalidValue;
+  prefill_kernel<D><<<(unsigned)units, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, p);
+  return (int)cudaGetLastError();
+}
+
+}  // namespace
+
+size_t prefill_smem_bytes(int D) {
+  switch (D) {
+    case 64: return PrefillCfg<64>::SMEM;
+    case 128: return PrefillCfg<128>::SMEM;
+    case 256: return PrefillCfg<256>::SMEM;
+    default: return 0;
+  }
+}
+
+int prefill_slots(int D) { return D <= 128 ? 2 : 1; }
+
+int launch_prefill(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                   const PrefillParams& p, cudaStream_t stream) {
+  switch (D) {
+    case 64: return launch_t<64>(tq, tk, tv, p, stream);
+    case 128: return launch_t<128>(tq, tk, tv, p, stream);
+    case 256: return launch_t<256>(tq, tk, tv, p, stream);
+    default: return (int)cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace gqa

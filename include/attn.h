@@ -1,0 +1,140 @@
+/*
+ * gqa_attn: forward scaled-dot-product attention with grouped-query heads on
+ * NVIDIA B200 (sm_100a).  C ABI: plain pointers and sizes, no framework types.
+ *
+ *     O   = softmax(scale * Q K^T + causal mask) V
+ *     LSE = log(sum_t exp(scale * q . k_t))      (natural log, visible keys only)
+ *
+ * Query head h reads K/V head h / (Hq / Hkv): contiguous groups of Hq/Hkv query
+ * heads share one K/V head ("ggml-org/llama.cpp PR #28507", Setup: GQA 8, and
+ * the FLASH_ATTN_EXT case list: nr23 broadcast ratio).
+ *
+ * Causal mask: key t is visible to query row s iff t <= q_offset + s, i.e. the
+ * Sq new queries sit at positions q_offset .. q_offset+Sq-1 of the key
+ * sequence (prefill at depth, speculative-verify rows).  q_offset >= 0, so
+ * every row sees at least key 0.
+ *
+ * Layouts (contiguous, row-major, element counts):
+ *     q, out        [B, Sq,  Hq,  D]
+ *     k, v          [B, Skv, Hkv, D]       bf16
+ *     lse           [B, Hq,  Sq]           fp32
+ *     partial_out   [S, B, Sq, Hq, D]      fp32 (S = num_splits)
+ *     partial_lse   [S, B, Hq, Sq]         fp32
+ * q, k, v are bf16.  out is bf16 or fp32 (out_dtype).
+ *
+ * Ownership: every buffer is allocated and owned by the caller and is DEVICE
+ * memory of the current CUDA device; the library allocates nothing per call.
+ * It keeps only one device status word per device (for attn_last_status).
+ *
+ * Asynchrony: every compute call is enqueued on `stream` (a cudaStream_t
+ * passed as void*; NULL means the legacy default stream) and returns at once.
+ * The return value covers argument checks and the launch itself.  A kernel
+ * that gives up on a stalled pipeline (a bounded wait that ran out) records
+ * ATTN_ERR_TIMEOUT in the device status word; attn_last_status() reads it.
+ *
+ * Errors: argument errors are detected on the host before any CUDA call and
+ * leave every output untouched.
+ */
+#ifndef GQA_ATTN_H
+#define GQA_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = -1,  /* null pointer, non-positive size, Hq % Hkv != 0, bad split count */
+  ATTN_ERR_UNSUPPORTED = -2,  /* a head dim or row count this build has no kernel for */
+  ATTN_ERR_ALIGNMENT = -3,    /* q/k/v/out/partials not 16-byte aligned, lse not 4-byte aligned */
+  ATTN_ERR_CUDA = -4,         /* a CUDA runtime/driver call failed (no device, launch error) */
+  ATTN_ERR_TIMEOUT = -5       /* a kernel's bounded pipeline wait ran out (device status) */
+} attn_status;
+
+typedef enum { ATTN_BF16 = 0, ATTN_F32 = 1 } attn_dtype;
+
+/*
+ * Prefill: all Sq query rows against all Skv keys in one pass.  The flash
+ * formulation with an online softmax keeps a running per-row (max, rowsum) and
+ * rescales the output accumulator ("Anbeeld/beellama.cpp PR #149", Overview:
+ * warp-shuffle reduction and fp32 rescale; every tile publishes its (max,
+ * rowsum)); K/V tiles are staged in shared memory and reused by all query rows
+ * of a tile ("ggml-org/llama.cpp PR #28507", the staging change;
+ * "AstrAI commit log, gqa_prefill_attn_mma.cuh", cp.async K/V loads and the
+ * pre-scaled Q, whose scale this library applies in fp32 instead of rounding
+ * Q*scale to bf16).
+ *
+ *   D          64, 128 or 256 (else ATTN_ERR_UNSUPPORTED)
+ *   scale      > 0 and finite (else ATTN_ERR_INVALID_ARG)
+ *   causal     0 or 1; q_offset >= 0
+ *   out_dtype  ATTN_BF16 or ATTN_F32 (round to nearest even for bf16)
+ *   lse        may be NULL (then no LSE is written)
+ */
+int attn_prefill(const void* q, const void* k, const void* v, void* out, float* lse,
+                 int B, int Hq, int Hkv, int Sq, int Skv, int D, int q_offset, int causal,
+                 float scale, int out_dtype, void* stream);
+
+/*
+ * Split-KV decode ("flash decoding"): the keys are cut into num_splits
+ * contiguous chunks of c = ceil(Skv / num_splits) keys; split s covers keys
+ * [s*c, min((s+1)*c, Skv)).  Each split writes its own normalised partial
+ * output and its log-sum-exp.  EVERY split publishes, including a split that
+ * holds no key or whose keys are all masked for a row: that row gets
+ * partial_lse = -inf and partial_out = 0 ("Anbeeld/beellama.cpp PR #149",
+ * Overview, the ub>64 fix: whole-tile blocks must publish their (max, rowsum)
+ * or the merge silently drops their rows).
+ *
+ *   D            128, 256 or 512 (else ATTN_ERR_UNSUPPORTED)
+ *   rows         R = (Hq/Hkv) * Sq query rows share one K/V head; R rounded up
+ *                to a multiple of 16 must satisfy (1 + D/128) * R16 <= 256
+ *                (else ATTN_ERR_UNSUPPORTED)
+ *   num_splits   1 <= num_splits <= Skv (else ATTN_ERR_INVALID_ARG)
+ *   partial_out  num_splits*B*Sq*Hq*D floats; partial_lse num_splits*B*Hq*Sq
+ */
+int attn_decode_split(const void* q, const void* k, const void* v, float* partial_out,
+                      float* partial_lse, int B, int Hq, int Hkv, int Sq, int Skv, int D,
+                      int q_offset, int causal, float scale, int num_splits, void* stream);
+
+/*
+ * Merge of split partials by their log-sum-exp ("Anbeeld/beellama.cpp PR
+ * #149", review note on the combine kernel for parallel_blocks > 1):
+ *     M = max_s lse_s;  w_s = exp(lse_s - M);
+ *     out = sum_s w_s * O_s / sum_s w_s;   lse = M + log(sum_s w_s).
+ * Splits with lse = -inf get weight 0.  lse may be NULL.
+ *   D            any multiple of 4 in [4, 1024] (else ATTN_ERR_UNSUPPORTED)
+ */
+int attn_merge(const float* partial_out, const float* partial_lse, void* out, float* lse,
+               int B, int Hq, int Sq, int D, int num_splits, int out_dtype, void* stream);
+
+/* Bytes of partial_out plus partial_lse that attn_decode_split needs; 0 on
+ * invalid sizes.  Both pieces start 16-byte aligned if the caller places
+ * partial_lse at partial_out + num_splits*B*Sq*Hq*D floats. */
+size_t attn_decode_workspace_bytes(int B, int Hq, int Sq, int D, int num_splits);
+
+/* Synchronises `stream`, then returns and clears the device status word of
+ * the current device: ATTN_OK, or ATTN_ERR_TIMEOUT if a kernel gave up on a
+ * stalled pipeline since the last call.  ATTN_ERR_CUDA if the sync fails. */
+int attn_last_status(void* stream);
+
+/* Human-readable name of a status code (static storage). */
+const char* attn_status_string(int status);
+
+/*
+ * Self-test of the bounded wait: launches one CTA that waits on an mbarrier
+ * nothing will ever complete, with the given limit in nanoseconds (clamped to
+ * [1e3, 5e9]).  The wait gives up, the kernel records ATTN_ERR_TIMEOUT and
+ * exits normally; read it back with attn_last_status().  No hang, no fault.
+ */
+int attn_watchdog_selftest(unsigned long long limit_ns, void* stream);
+
+/* Library version, e.g. 0x000100 for 0.1.0. */
+int attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GQA_ATTN_H */

@@ -1,0 +1,115 @@
+"""The C-ABI library on the host: it loads, exports every declared entry point,
+and rejects bad arguments before any CUDA call (so these run without a GPU)."""
+import ctypes
+
+import pytest
+
+import gqa_flash_attention_attn_b200 as ga
+from gqa_flash_attention_attn_b200 import build as gbuild
+
+
+@pytest.fixture(scope="module")
+def lib():
+    gbuild.build()
+    return ga.library()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = ga.declared_functions()
+    assert {"attn_prefill", "attn_decode_split", "attn_merge", "attn_last_status"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/attn.h but not exported"
+
+
+def test_version_and_status_strings(lib):
+    assert ga.version() == 0x000100
+    assert ga.status_string(ga.ATTN_OK) == "ok"
+    assert ga.status_string(ga.ATTN_ERR_TIMEOUT) == "pipeline wait timed out"
+    assert ga.status_string(12345) == "unknown status"
+
+
+def test_workspace_bytes(lib):
+    S, B, Hq, Sq, D = 32, 16, 16, 1, 512
+    assert ga.decode_workspace_bytes(B, Hq, Sq, D, S) == 4 * (S * B * Sq * Hq * D + S * B * Hq * Sq)
+    assert ga.decode_workspace_bytes(0, Hq, Sq, D, S) == 0
+    assert ga.decode_workspace_bytes(B, Hq, Sq, D, 0) == 0
+
+
+# Fake but 256-byte aligned addresses: the checks must reject before any use.
+P = ctypes.c_void_p(0x10000)
+P2 = ctypes.c_void_p(0x20000)
+MIS = ctypes.c_void_p(0x10008)
+
+
+def _prefill(lib, **kw):
+    a = dict(q=P, k=P, v=P, out=P2, lse=P2, B=1, Hq=8, Hkv=2, Sq=128, Skv=128, D=128, q_offset=0, causal=1,
+             scale=0.125, out_dtype=0)
+    a.update(kw)
+    return lib.attn_prefill(a["q"], a["k"], a["v"], a["out"], a["lse"], a["B"], a["Hq"], a["Hkv"], a["Sq"],
+                            a["Skv"], a["D"], a["q_offset"], a["causal"], a["scale"], a["out_dtype"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), ga.ATTN_ERR_INVALID_ARG),
+    (dict(out=None), ga.ATTN_ERR_INVALID_ARG),
+    (dict(B=0), ga.ATTN_ERR_INVALID_ARG),
+    (dict(Sq=0), ga.ATTN_ERR_INVALID_ARG),
+    (dict(Skv=-1), ga.ATTN_ERR_INVALID_ARG),
+    (dict(Hq=6, Hkv=4), ga.ATTN_ERR_INVALID_ARG),
+    (dict(q_offset=-1), ga.ATTN_ERR_INVALID_ARG),
+    (dict(causal=2), ga.ATTN_ERR_INVALID_ARG),
+    (dict(scale=0.0), ga.ATTN_ERR_INVALID_ARG),
+    (dict(scale=-0.1), ga.ATTN_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), ga.ATTN_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), ga.ATTN_ERR_INVALID_ARG),
+    (dict(out_dtype=7), ga.ATTN_ERR_INVALID_ARG),
+    (dict(D=72), ga.ATTN_ERR_UNSUPPORTED),     # the head size that crashed a staging path
+    (dict(D=32), ga.ATTN_ERR_UNSUPPORTED),
+    (dict(D=512), ga.ATTN_ERR_UNSUPPORTED),
+    (dict(q=MIS), ga.ATTN_ERR_ALIGNMENT),
+    (dict(v=MIS), ga.ATTN_ERR_ALIGNMENT),
+    (dict(out=MIS), ga.ATTN_ERR_ALIGNMENT),
+    (dict(lse=ctypes.c_void_p(0x20002)), ga.ATTN_ERR_ALIGNMENT),
+    (dict(q_offset=2**31 - 100), ga.ATTN_ERR_INVALID_ARG),
+])
+def test_prefill_rejects(lib, kw, status):
+    assert _prefill(lib, **kw) == status
+
+
+def _decode(lib, **kw):
+    a = dict(q=P, k=P, v=P, po=P2, pl=P2, B=16, Hq=16, Hkv=1, Sq=1, Skv=16384, D=512, q_offset=16383, causal=1,
+             scale=0.0441941738, S=32)
+    a.update(kw)
+    return lib.attn_decode_split(a["q"], a["k"], a["v"], a["po"], a["pl"], a["B"], a["Hq"], a["Hkv"], a["Sq"],
+                                 a["Skv"], a["D"], a["q_offset"], a["causal"], a["scale"], a["S"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(S=0), ga.ATTN_ERR_INVALID_ARG),
+    (dict(S=16385), ga.ATTN_ERR_INVALID_ARG),        # more splits than keys
+    (dict(po=None), ga.ATTN_ERR_INVALID_ARG),
+    (dict(pl=None), ga.ATTN_ERR_INVALID_ARG),
+    (dict(Hq=12, Hkv=8), ga.ATTN_ERR_INVALID_ARG),
+    (dict(D=64), ga.ATTN_ERR_UNSUPPORTED),
+    (dict(D=96), ga.ATTN_ERR_UNSUPPORTED),
+    (dict(Hq=64, Sq=1), ga.ATTN_ERR_UNSUPPORTED),   # 64 rows x (1 + 512/128) > 256 TMEM columns
+    (dict(D=128, Hq=32, Hkv=1, Sq=8), ga.ATTN_ERR_UNSUPPORTED),  # 256 rows
+    (dict(po=MIS), ga.ATTN_ERR_ALIGNMENT),
+    (dict(k=MIS), ga.ATTN_ERR_ALIGNMENT),
+    (dict(pl=ctypes.c_void_p(0x20001)), ga.ATTN_ERR_ALIGNMENT),
+])
+def test_decode_rejects(lib, kw, status):
+    assert _decode(lib, **kw) == status
+
+
+@pytest.mark.parametrize("args,status", [
+    ((None, P, P2, P2, 1, 2, 3, 128, 4, 0), ga.ATTN_ERR_INVALID_ARG),
+    ((P, P, P2, P2, 1, 2, 3, 130, 4, 0), ga.ATTN_ERR_UNSUPPORTED),
+    ((P, P, P2, P2, 1, 2, 3, 2048, 4, 0), ga.ATTN_ERR_UNSUPPORTED),
+    ((P, P, P2, P2, 1, 2, 3, 128, 0, 0), ga.ATTN_ERR_INVALID_ARG),
+    ((P, P, P2, P2, 1, 2, 3, 128, 4, 3), ga.ATTN_ERR_INVALID_ARG),
+    ((MIS, P, P2, P2, 1, 2, 3, 128, 4, 0), ga.ATTN_ERR_ALIGNMENT),
+    ((P, P, ctypes.c_void_p(0x20004), P2, 1, 2, 3, 128, 4, 0), ga.ATTN_ERR_ALIGNMENT),
+])
+def test_merge_rejects(lib, args, status):
+    assert lib.attn_merge(*args, None) == status

@@ -1,0 +1,99 @@
+"""Split-KV decode and LSE merge vs the float64 oracle, through the C ABI (B200)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import gqa_flash_attention_attn_b200 as ga
+from gqa_flash_attention_attn_b200.inputs import WORKLOADS, make_qkv, make_workload_inputs, sample_rows
+import oracle
+from parity import (assert_lse_close, assert_o_close, gather_rows, oracle_rows_by_batch, to_f64)
+
+pytestmark = pytest.mark.gpu
+
+# (B, Hq, Hkv, Sq, Skv, D, q_offset, causal, num_splits)
+CASES = [
+    (2, 16, 1, 1, 1000, 512, 999, True, 4),     # single-query decode, D = 512
+    (1, 32, 8, 8, 700, 128, 692, True, 3),      # 8 draft rows per sequence
+    (2, 8, 2, 3, 500, 256, 497, True, 5),
+    (1, 4, 4, 1, 1, 128, 0, True, 1),           # one key
+    (1, 8, 1, 1, 100, 128, 99, True, 30),       # splits 25..29 hold no key
+    (1, 4, 1, 8, 1000, 128, 0, True, 9),        # causal at q_offset 0: most splits fully masked
+    (1, 16, 4, 2, 300, 512, 298, True, 2),      # 8 rows padded to 16
+    (1, 8, 1, 1, 777, 128, 0, False, 6),        # non-causal
+    (1, 16, 2, 8, 515, 128, 507, True, 1),      # 64 rows, one split, ragged tail
+]
+
+
+def _scale(D):
+    return float(torch.tensor(1.0 / math.sqrt(D), dtype=torch.float32))
+
+
+@pytest.mark.parametrize("case", CASES, ids=[f"B{c[0]}H{c[1]}/{c[2]}S{c[3]}x{c[4]}D{c[5]}o{c[6]}S{c[8]}" for c in CASES])
+def test_decode_split_and_merge_match_oracle(case):
+    B, Hq, Hkv, Sq, Skv, D, q_offset, causal, S = case
+    q, k, v = make_qkv(B, Hq, Hkv, Sq, Skv, D, seed=1)
+    scale = _scale(D)
+    po, pl = ga.decode_split(q.cuda(), k.cuda(), v.cuda(), S, causal=causal, q_offset=q_offset, scale=scale)
+    out, lse = ga.merge(po, pl, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert ga.last_status() == ga.ATTN_OK
+    want_po, want_pl = oracle.split(q, k, v, S, scale=scale, causal=causal, q_offset=q_offset)
+    # every split publishes: the -inf pattern of the partial LSE is exact
+    assert_lse_close(pl, want_pl, f"partial lse {case}")
+    assert_o_close(po, want_po, f"partial out {case}")
+    want_o, want_lse = oracle.attention(q, k, v, scale=scale, causal=causal, q_offset=q_offset)
+    assert_o_close(out, want_o, f"merged {case}")
+    assert_lse_close(lse, want_lse, f"merged {case}")
+
+
+def test_merge_of_oracle_partials():
+    # the merge kernel alone, on partials (including -inf splits) from the oracle
+    B, Hq, Hkv, Sq, Skv, D, S = 2, 8, 2, 4, 90, 128, 16
+    q, k, v = make_qkv(B, Hq, Hkv, Sq, Skv, D, seed=2)
+    scale = _scale(D)
+    po, pl = oracle.split(q, k, v, S, scale=scale, causal=True, q_offset=20)
+    assert np.isneginf(pl).any()
+    out, lse = ga.merge(torch.from_numpy(po).float().cuda(), torch.from_numpy(pl).float().cuda(),
+                        out_dtype=torch.float32)
+    want_o, want_lse = oracle.merge(po, pl)
+    assert_o_close(out, want_o, "merge")
+    assert_lse_close(lse, want_lse, "merge")
+
+
+def test_merge_all_splits_empty_gives_zero_and_neg_inf():
+    po = torch.zeros((3, 1, 2, 4, 128), device="cuda")
+    pl = torch.full((3, 1, 4, 2), float("-inf"), device="cuda")
+    out, lse = ga.merge(po, pl, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.all(out == 0)
+    assert torch.all(torch.isneginf(lse))
+
+
+def test_split_count_does_not_change_result():
+    B, Hq, Hkv, Sq, Skv, D = 1, 16, 2, 4, 2000, 128
+    q, k, v = make_qkv(B, Hq, Hkv, Sq, Skv, D, seed=4)
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    ref_o, ref_l = ga.prefill(qc, kc, vc, causal=True, q_offset=Skv - Sq, out_dtype=torch.float32)
+    for S in (1, 2, 7, 16, 63):
+        o, l = ga.decode(qc, kc, vc, S, causal=True, q_offset=Skv - Sq, out_dtype=torch.float32)
+        torch.cuda.synchronize()
+        assert (o - ref_o).abs().max().item() < 2e-2
+        assert (l - ref_l).abs().max().item() < 1e-3
+
+
+@pytest.mark.parametrize("name", ["split_kv_decode_d512", "spec_verify_decode_d128"])
+def test_full_size_workload_sampled_rows(name):
+    w = WORKLOADS[name]
+    q, k, v = make_workload_inputs(w)
+    out, lse = ga.decode(q.cuda(), k.cuda(), v.cuda(), w.num_splits, causal=w.causal, q_offset=w.q_offset,
+                         scale=w.scale, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    assert ga.last_status() == ga.ATTN_OK
+    rows = sample_rows(w, 48)
+    want_o, want_lse = oracle_rows_by_batch(q, k, v, rows, scale=w.scale, causal=w.causal, q_offset=w.q_offset)
+    got_o, got_lse = gather_rows(out, lse, rows)
+    assert_o_close(got_o, want_o, name)
+    assert_lse_close(got_lse, want_lse, name)
+    assert torch.isfinite(out).all() and torch.isfinite(lse).all()
