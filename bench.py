@@ -1,0 +1,424 @@
+"""Benchmark: prefill TFLOP/s and decode KV GB/s on B200, as a fraction of roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one launch sequence of the attention path over one batch of
+synthetic, seeded bf16 inputs already resident in HBM.  The headline workload
+is the GQA causal prefill (B1 Hq32 Hkv8 Sq=Skv=4096 D128); the other four
+workloads (tiny prefill, prefill at depth with D256, D512 split-KV decode with
+its LSE merge, 8-row speculative-verify decode) are timed the same way and
+reported under "workloads".  L2 is flushed (a 256 MiB write) between timed
+steps; the flush is outside the timed events.
+
+Under torchrun (N > 1) every rank runs the same problems independently (the
+path does not shard: replicas only); times are the max over ranks and the
+value is the work of all ranks divided by that time.
+
+--impl reference times the float64 CPU oracle (the parity reference) on a
+bounded row sample of the headline workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+HEADLINE = "gqa_causal_prefill_4k_d128"
+METRIC = "prefill TFLOP/s and decode KV GB/s on 1 B200, as % of roofline"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+FLUSH_BYTES = 256 << 20
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=None, help="time only this workload (profiling)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle budget for cpu_baseline")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ helpers --
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", 0.0)), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def kernel_source_sha(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "gqa_flash_attention_attn_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+KERNEL_SOURCES = {
+    "prefill": ["prefill_sm100.cu", "ptx.cuh"],
+    "decode": ["decode_sm100.cu", "ptx.cuh"],
+    "merge": ["merge.cu", "ptx.cuh"],
+}
+
+
+def profiled_traffic(kind, workload):
+    """DRAM bytes per launch from a committed ncu summary, or None when the
+    summary is missing or the kernel source changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", f"{kind}_{workload}.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m = re.search(r"traffic-bytes-per-launch:\s*([0-9]+)", text)
+    s = re.search(r"kernel-source-sha256:\s*([0-9a-f]+)", text)
+    if not m or not s or s.group(1) != kernel_source_sha(KERNEL_SOURCES[kind]):
+        return None
+    return int(m.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling in the background."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------- the GPU arm --
+def make_runner(ga, w, device):
+    """Device-resident inputs/outputs and a closure that launches one step.
+    Returns (step_fn, n_kernels_per_step, events_split) where the closure
+    records optional inner events between the split and the merge."""
+    from gqa_flash_attention_attn_b200.inputs import make_qkv
+    q, k, v = make_qkv(w.B, w.Hq, w.Hkv, w.Sq, w.Skv, w.D, seed=0, device=device)
+    odt = torch.float32 if w.out_dtype == "f32" else torch.bfloat16
+    out = torch.empty((w.B, w.Sq, w.Hq, w.D), dtype=odt, device=device)
+    lse = torch.empty((w.B, w.Hq, w.Sq), dtype=torch.float32, device=device)
+    if w.kind == "prefill":
+        def step(mid=None):
+            ga.prefill(q, k, v, causal=w.causal, q_offset=w.q_offset, scale=w.scale, out=out, lse=lse)
+        return step, 1, (q, k, v, out, lse)
+    po = torch.empty((w.num_splits, w.B, w.Sq, w.Hq, w.D), dtype=torch.float32, device=device)
+    pl = torch.empty((w.num_splits, w.B, w.Hq, w.Sq), dtype=torch.float32, device=device)
+
+    def step(mid=None):
+        ga.decode_split(q, k, v, w.num_splits, causal=w.causal, q_offset=w.q_offset, scale=w.scale,
+                        partial_out=po, partial_lse=pl)
+        if mid is not None:
+            mid.record()
+        ga.merge(po, pl, out=out, lse=lse)
+    return step, 2, (q, k, v, out, lse)
+
+
+def barrier(dist_on):
+    if dist_on:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, dist_on, device):
+    if not dist_on:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def time_steps(step, steps, warmup, flush, dist_on, device, inner=False):
+    for _ in range(warmup):
+        step()
+        flush.zero_()
+    torch.cuda.synchronize()
+    barrier(dist_on)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for s, m, e in ev:
+        s.record()
+        step(m if inner else None)
+        e.record()
+        flush.zero_()
+    torch.cuda.synchronize()
+    barrier(dist_on)
+    torch.cuda.synchronize()
+    total = sum(s.elapsed_time(e) for s, _, e in ev)
+    first = sum(s.elapsed_time(m) for s, m, _ in ev) if inner else total
+    return total / steps, first / steps
+
+
+def time_e2e(ga, w, steps, warmup, dist_on, device):
+    """Same workload through the public call with pinned host buffers: H2D of
+    q, k, v, the kernels, and D2H of out and lse inside every timed step."""
+    from gqa_flash_attention_attn_b200.inputs import make_qkv
+    q, k, v = make_qkv(w.B, w.Hq, w.Hkv, w.Sq, w.Skv, w.D, seed=0)
+    hq, hk, hv = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    odt = torch.float32 if w.out_dtype == "f32" else torch.bfloat16
+    ho = torch.empty((w.B, w.Sq, w.Hq, w.D), dtype=odt).pin_memory()
+    hl = torch.empty((w.B, w.Hq, w.Sq), dtype=torch.float32).pin_memory()
+    dq, dk, dv = (torch.empty_like(t, device=device) for t in (q, k, v))
+
+    def step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        if w.kind == "prefill":
+            o, l = ga.prefill(dq, dk, dv, causal=w.causal, q_offset=w.q_offset, scale=w.scale, out_dtype=odt)
+        else:
+            o, l = ga.decode(dq, dk, dv, w.num_splits, causal=w.causal, q_offset=w.q_offset, scale=w.scale,
+                             out_dtype=odt)
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(l, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(dist_on)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        step()
+    e.record()
+    torch.cuda.synchronize()
+    barrier(dist_on)
+    ms = max_over_ranks(s.elapsed_time(e) / steps, dist_on, device)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+    d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+    return ms, h2d, d2h
+
+
+def workload_metric(w):
+    """(unit, work per step) for a workload: TFLOP/s for prefill, KV GB/s for decode."""
+    if w.kind == "prefill":
+        return "TFLOP/s", w.flops() / 1e12
+    return "GB/s", w.io_bytes() / 1e9
+
+
+def cpu_baseline(w, seconds):
+    """The float64 oracle, as it stands, on a bounded row sample of workload w."""
+    import numpy as np
+    import oracle
+    from gqa_flash_attention_attn_b200.inputs import make_workload_inputs, sample_rows
+    q, k, v = make_workload_inputs(w)
+    qd, kd, vd = (t.double().numpy() for t in (q, k, v))
+
+    def visible(s):
+        return min(w.Skv, w.q_offset + s + 1) if w.causal else w.Skv
+
+    def run(n, seed):
+        rows = sample_rows(w, n, seed=seed, include_edges=False)
+        t0 = time.perf_counter()
+        oracle.attention_rows(qd, kd, vd, rows, scale=w.scale, causal=w.causal, q_offset=w.q_offset)
+        dt = time.perf_counter() - t0
+        flops = sum(4 * w.D * visible(s) for _, _, s in rows)
+        kv_bytes = sum(2 * 2 * w.D * visible(s) for _, _, s in rows)  # K and V rows each row reads
+        return dt, flops, kv_bytes, len(rows)
+
+    dt, _, _, _ = run(256, 11)
+    n2 = max(256, int(256 * seconds / max(dt, 1e-3)))
+    dt, fl, kvb, n = run(n2, 12)
+    unit, _ = workload_metric(w)
+    value = fl / dt / 1e12 if unit == "TFLOP/s" else kvb / dt / 1e9
+    return {"value": value, "unit": unit, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{n} random (b,h,s) rows of {w.name}, {fl / 1e9:.1f} GFLOP fp64 in {dt:.1f} s"}
+
+
+def run_ours(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist_on = world > 1
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if dist_on:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    import gqa_flash_attention_attn_b200 as ga
+    from gqa_flash_attention_attn_b200.inputs import WORKLOADS
+    ga.library()  # fails loudly when the CUDA library is missing
+
+    hbm, tf_burst, tf_sust, peak_src = peaks()
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    names = [args.workload] if args.workload else [HEADLINE] + [n for n in WORKLOADS if n != HEADLINE]
+    sampler = ClockSampler(local)
+    results = {}
+    sampler.start()
+    for name in names:
+        w = WORKLOADS[name]
+        step, nk, _ = make_runner(ga, w, device)
+        ms, ms_first = time_steps(step, args.steps, args.warmup, flush, dist_on, device, inner=(nk == 2))
+        ms = max_over_ranks(ms, dist_on, device)
+        ms_first = max_over_ranks(ms_first, dist_on, device)
+        status = ga.last_status()
+        if status != ga.ATTN_OK:
+            raise RuntimeError(f"{name}: device status {ga.status_string(status)}")
+        unit, work = workload_metric(w)
+        value = world * work / (ms / 1e3)
+        if w.kind == "prefill":
+            kind, achieved = "prefill", w.flops() / (ms_first / 1e3) / 1e12
+            roof = {"bound": "tensor", "achieved": achieved, "peak": tf_burst, "unit": "TFLOP/s",
+                    "frac": achieved / tf_burst, "peak_source": f"{peak_src} bf16 burst"}
+        else:
+            kind, achieved = "decode", w.io_bytes() / (ms_first / 1e3) / 1e9
+            roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                    "peak_source": f"{peak_src} copy bandwidth"}
+        roof["kernel"] = kind
+        roof["traffic"] = profiled_traffic(kind, name)
+        results[name] = {"value": value, "unit": unit, "ms_per_step": ms, "kernel_ms": ms_first,
+                         "kernels_per_step": nk, "roofline": roof}
+        del step
+        torch.cuda.empty_cache()
+    clocks = sampler.stop()
+
+    head = results[names[0]]
+    w = WORKLOADS[names[0]]
+    e2e_ms, h2d, d2h = time_e2e(ga, w, max(3, args.steps // 5), max(1, args.warmup), dist_on, device)
+    unit, work = workload_metric(w)
+    line = {
+        "metric": METRIC,
+        "value": head["value"],
+        "unit": head["unit"],
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded iid N(0,1) cast to bf16)",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Sq": w.Sq, "Skv": w.Skv, "D": w.D,
+                   "q_offset": w.q_offset, "causal": w.causal, "out": w.out_dtype,
+                   "num_splits": w.num_splits if w.kind == "decode" else None,
+                   "l2": "flushed between timed steps (256 MiB write)", "parallelism": f"replicas x{world}"},
+        "roofline": head["roofline"],
+        "e2e": {"value": world * work / (e2e_ms / 1e3), "unit": unit, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": head["kernels_per_step"] * args.steps,
+        "clocks": clocks,
+        "workloads": {n: {k2: r[k2] for k2 in ("value", "unit", "ms_per_step", "kernel_ms")} |
+                      {"roofline_frac": r["roofline"]["frac"], "bound": r["roofline"]["bound"],
+                       "traffic": r["roofline"]["traffic"]}
+                      for n, r in results.items()},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist_on:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+def run_reference(args):
+    """The float64 CPU oracle timed on a bounded sample per step (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    import numpy as np
+    import oracle
+    from gqa_flash_attention_attn_b200.inputs import WORKLOADS, make_workload_inputs, sample_rows
+    w = WORKLOADS[HEADLINE]
+    q, k, v = make_workload_inputs(w)
+    qd, kd, vd = (t.double().numpy() for t in (q, k, v))
+
+    def one(n, seed):
+        rows = sample_rows(w, n, seed=seed, include_edges=False)
+        fl = sum(4 * w.D * min(w.Skv, w.q_offset + s + 1) for _, _, s in rows)
+        t0 = time.perf_counter()
+        oracle.attention_rows(qd, kd, vd, rows, scale=w.scale, causal=w.causal, q_offset=w.q_offset)
+        return time.perf_counter() - t0, fl
+
+    dt, _ = one(128, 1)
+    n = max(64, int(128 * 1.0 / max(dt, 1e-3)))   # about one second of oracle work per step
+    for i in range(args.warmup):
+        one(n, 100 + i)
+    tot_t, tot_f = 0.0, 0
+    for i in range(args.steps):
+        dt, fl = one(n, 1000 + i)
+        tot_t += dt
+        tot_f += fl
+    value = tot_f / tot_t / 1e12
+    cores = oracle.num_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded iid N(0,1) cast to bf16)",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Sq": w.Sq, "Skv": w.Skv, "D": w.D,
+                   "q_offset": w.q_offset, "causal": w.causal},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{n} random (b,h,s) rows of {w.name} per step"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()
