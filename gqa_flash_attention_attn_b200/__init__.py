@@ -23,7 +23,7 @@ __all__ = [
     "AttnError", "library", "library_path", "declared_functions", "prefill", "decode_split",
     "merge", "decode", "decode_workspace_bytes", "last_status", "status_string",
     "watchdog_selftest", "version", "ATTN_OK", "ATTN_ERR_INVALID_ARG", "ATTN_ERR_UNSUPPORTED",
-    "ATTN_ERR_ALIGNMENT", "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT",
+    "ATTN_ERR_ALIGNMENT", "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT", "ATTN_ERR_TOO_LARGE", "decode_noalloc",
 ]
 
 ATTN_OK = 0
@@ -32,6 +32,7 @@ ATTN_ERR_UNSUPPORTED = -2
 ATTN_ERR_ALIGNMENT = -3
 ATTN_ERR_CUDA = -4
 ATTN_ERR_TIMEOUT = -5
+ATTN_ERR_TOO_LARGE = -6
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _HEADER = os.path.join(os.path.dirname(_PKG), "include", "attn.h")
@@ -51,6 +52,7 @@ _SIGNATURES = {
     "attn_status_string": (ctypes.c_char_p, [_i]),
     "attn_watchdog_selftest": (_i, [ctypes.c_ulonglong, _vp]),
     "attn_version": (_i, []),
+    "attn_decode_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp] + [_i] * 8 + [_f, _i, _i, _vp]),
 }
 
 
@@ -215,3 +217,26 @@ def last_status(stream=None) -> int:
 
 def watchdog_selftest(limit_ns: int, stream=None):
     _check("attn_watchdog_selftest", library().attn_watchdog_selftest(int(limit_ns), _stream_ptr(stream)))
+
+
+def decode_noalloc(q, k, v, num_splits, *, causal=True, q_offset=0, scale=None, out_dtype=torch.bfloat16,
+                   out=None, lse=None, return_lse=True, stream=None):
+    """Split-KV decode + merge with the partials in the library's fixed device
+    array instead of a caller workspace, for callers that cannot allocate
+    device memory.  Same result as decode(); calls must not overlap on the GPU."""
+    _need(q, "q", torch.bfloat16, 4)
+    _need(k, "k", torch.bfloat16, 4)
+    _need(v, "v", torch.bfloat16, 4)
+    B, Sq, Hq, D = q.shape
+    _, Skv, Hkv, _ = k.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty((B, Sq, Hq, D), dtype=out_dtype, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    st = library().attn_decode_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Skv, D,
+                                       int(q_offset), int(bool(causal)), float(scale), int(num_splits),
+                                       _OUT_CODES[out.dtype], _stream_ptr(stream))
+    _check("attn_decode_noalloc", st)
+    return out, lse

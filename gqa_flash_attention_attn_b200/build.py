@@ -13,7 +13,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libgqa_attn.so")
-SOURCES = ["abi.cu", "prefill_sm100.cu", "decode_sm100.cu", "merge.cu"]
+SOURCES = ["abi.cu", "prefill_sm100.cu", "decode_sm100.cu", "merge.cu", "decode_noalloc.cu"]
 HEADERS = ["ptx.cuh", "kernels.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -102,6 +102,7 @@ const char* attn_status_string(int status) {
     case ATTN_ERR_ALIGNMENT: return "misaligned pointer";
     case ATTN_ERR_CUDA: return "CUDA error";
     case ATTN_ERR_TIMEOUT: return "pipeline wait timed out";
+    case ATTN_ERR_TOO_LARGE: return "problem exceeds the fixed no-alloc scratch";
     default: return "unknown status";
   }
 }

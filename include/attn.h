@@ -51,7 +51,8 @@ typedef enum {
   ATTN_ERR_UNSUPPORTED = -2,  /* a head dim or row count this build has no kernel for */
   ATTN_ERR_ALIGNMENT = -3,    /* q/k/v/out/partials not 16-byte aligned, lse not 4-byte aligned */
   ATTN_ERR_CUDA = -4,         /* a CUDA runtime/driver call failed (no device, launch error) */
-  ATTN_ERR_TIMEOUT = -5       /* a kernel's bounded pipeline wait ran out (device status) */
+  ATTN_ERR_TIMEOUT = -5,      /* a kernel's bounded pipeline wait ran out (device status) */
+  ATTN_ERR_TOO_LARGE = -6     /* attn_decode_noalloc: partials exceed the fixed scratch array */
 } attn_status;
 
 typedef enum { ATTN_BF16 = 0, ATTN_F32 = 1 } attn_dtype;
@@ -129,6 +130,35 @@ const char* attn_status_string(int status);
  * exits normally; read it back with attn_last_status().  No hang, no fault.
  */
 int attn_watchdog_selftest(unsigned long long limit_ns, void* stream);
+
+/*
+ * Allocation-free split-KV decode + merge.  The pages have no counterpart:
+ * this serves callers that cannot allocate a device workspace (a plugin host
+ * that owns the whole device memory pool and hands an operator only its
+ * inputs and outputs; a latency-critical decode loop that must not call
+ * cudaMalloc, which can synchronise the device).
+ *
+ * Same arguments and results as attn_decode_split followed by attn_merge into
+ * out [B,Sq,Hq,D] (out_dtype) and lse [B,Hq,Sq] (may be NULL), but the split
+ * partials live in one fixed device array inside the library, of
+ * ATTN_NOALLOC_SCRATCH_BYTES bytes, held by every device that loads the
+ * library until the process exits.  The library calls no cudaMalloc, cudaFree
+ * or other allocating routine.
+ *   - Capacity: num_splits*B*Sq*Hq*D*4 bytes (rounded up to 256) plus
+ *     num_splits*B*Hq*Sq*4 bytes must fit, else ATTN_ERR_TOO_LARGE (checked on
+ *     the host before anything is launched).
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   - All calls share the array and it keeps the last call's contents; nothing
+ *     in it needs clearing, since each call's split kernel writes every
+ *     partial that its merge reads.  Calls whose kernels overlap on the GPU
+ *     (different streams or host threads) race on it: serialise them.
+ */
+#define ATTN_NOALLOC_SCRATCH_BYTES (24u * 1024u * 1024u)
+int attn_decode_noalloc(const void* q, const void* k, const void* v, void* out, float* lse,
+                        int B, int Hq, int Hkv, int Sq, int Skv, int D, int q_offset, int causal,
+                        float scale, int num_splits, int out_dtype, void* stream);
 
 /* Library version, e.g. 0x000100 for 0.1.0. */
 int attn_version(void);
