@@ -159,7 +159,7 @@ int attn_decode_split(const void* q, const void* k, const void* v, float* partia
   const int g = Hq / Hkv;
   const long long R = (long long)g * Sq;
   const long long RP = (R + 15) / 16 * 16;
-  if (RP * (1 + D / 128) > 256) return ATTN_ERR_UNSUPPORTED;
+  if (RP * (2 + D / 128) > 256) return ATTN_ERR_UNSUPPORTED;  // TMEM: two S^T buffers + O^T
   if (g > 256 || Sq > 256) return ATTN_ERR_UNSUPPORTED;  // TMA box extents
   if ((long long)B * Hkv > 65535) return ATTN_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(partial_out, 16))

@@ -16,9 +16,13 @@
 // Every split publishes its normalised partial O and its log-sum-exp, also
 // when it has no visible key (lse = -inf, O = 0) ("Anbeeld/beellama.cpp PR
 // #149", Overview, ub>64 fix: every block publishes its (max, rowsum)); the
-// merge is attn_merge.  The K/V stream is a ring of 32 KB slots (128 keys x
-// 128 columns, two TMA boxes) fed by one producer thread; the kernel is
-// HBM-bound, so the ring depth and two CTAs per SM set the bytes in flight.
+// merge is attn_merge.
+//
+// The kernel is HBM-bound, so the pipeline keeps loads flowing while the
+// softmax works: S^T and P are double-buffered, the MMA thread computes
+// S_{j+1} before it waits for P_j, and the producer streams the ring in the
+// same order (K_0, K_1, V_0, K_2, V_1, ...).  Ring slots are 32 KB (128 keys
+// x 128 columns, two TMA boxes); two CTAs run per SM.
 #include "kernels.h"
 #include "ptx.cuh"
 
@@ -40,12 +44,12 @@ struct Layout {
     off_q = 0;
     const uint32_t qbytes = (uint32_t)(D / 64) * RP * 128u;
     off_p = (off_q + qbytes + 1023u) & ~1023u;
-    off_ring = (off_p + 2u * RP * 128u + 1023u) & ~1023u;
+    off_ring = (off_p + 2u * 2u * RP * 128u + 1023u) & ~1023u;  // two P buffers
     off_red = off_ring + (uint32_t)nbuf * SLOT_BYTES;
     off_row = off_red + 2u * 4u * RP * 4u;     // red_max[4][RP], red_sum[4][RP]
-    off_bar = off_row + 5u * RP * 4u;          // m, l, alpha, msub, inv
+    off_bar = off_row + 6u * RP * 4u;          // m, l, alpha, msub, inv, lim
     off_bar = (off_bar + 7u) & ~7u;
-    off_misc = off_bar + (uint32_t)(1 + 2 * nbuf + 4) * 8u;
+    off_misc = off_bar + (uint32_t)(1 + 2 * nbuf + 7) * 8u;
     total = off_misc + 16u + 1024u;
   }
 };
@@ -57,16 +61,24 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
   }
 }
 
-__device__ __forceinline__ float warp_max(float x) {
+// Reduce 16 per-lane values (one per row) across the 32 lanes of a warp.
+// On return, lanes l and l^16 hold the reduction of row (l & 15) in v[0].
+// 16 shuffles instead of 16 x 5.
+template <bool kMax>
+__device__ __forceinline__ float warp_reduce16(float (&v)[16], int lane) {
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
-  return x;
-}
-
-__device__ __forceinline__ float warp_sum(float x) {
+  for (int step = 8; step >= 1; step >>= 1) {
+    const bool upper = (lane & step) != 0;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-  return x;
+    for (int i = 0; i < step; ++i) {
+      const float send = upper ? v[i] : v[i + step];
+      const float keep = upper ? v[i + step] : v[i];
+      const float recv = __shfl_xor_sync(0xffffffffu, send, step);
+      v[i] = kMax ? fmaxf(keep, recv) : keep + recv;
+    }
+  }
+  const float other = __shfl_xor_sync(0xffffffffu, v[0], 16);
+  return kMax ? fmaxf(v[0], other) : v[0] + other;
 }
 
 template <int D>
@@ -88,6 +100,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   float* alpha_sm = l_sm + RP;
   float* msub_sm = alpha_sm + RP;
   float* inv_sm = msub_sm + RP;
+  int* lim_sm = reinterpret_cast<int*>(inv_sm + RP);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L.off_misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L.off_misc + 4);
   volatile int* resc_flag = reinterpret_cast<volatile int*>(gbase + L.off_misc + 8);
@@ -95,7 +108,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int BAR_Q = 0;
   auto bar_full = [&](int s) { return 1 + s; };
   auto bar_empty = [&](int s) { return 1 + nbuf + s; };
-  const int BAR_S = 1 + 2 * nbuf, BAR_P = BAR_S + 1, BAR_PV = BAR_S + 2, BAR_DRAIN = BAR_S + 3;
+  const int BAR_S0 = 1 + 2 * nbuf;       // s_full[2]
+  const int BAR_P0 = BAR_S0 + 2;         // p_full[2]
+  const int BAR_PV0 = BAR_S0 + 4;        // pv_done per P buffer [2]
+  const int BAR_DRAIN = BAR_S0 + 6;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = blockIdx.x;
@@ -129,8 +145,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     reinterpret_cast<uint32_t*>(gbase + L.off_q + (uint32_t)box * RP * 128u + (uint32_t)R * 128u)[w] = 0u;
   }
   if (threadIdx.x < RP) {
-    m_sm[threadIdx.x] = -INFINITY;
-    l_sm[threadIdx.x] = 0.f;
+    const int r = threadIdx.x;
+    m_sm[r] = -INFINITY;
+    l_sm[r] = 0.f;
+    // last visible key of row r (padding rows see none)
+    lim_sm[r] = r < R ? (p.causal ? p.q_offset + r / g : 0x7fffffff) : -1;
   }
   if (threadIdx.x == 0) {
     mbar_init(bar(BAR_Q), 1);
@@ -138,16 +157,18 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(bar(bar_full(s)), 1);
       mbar_init(bar(bar_empty(s)), 1);
     }
-    mbar_init(bar(BAR_S), 1);
-    mbar_init(bar(BAR_P), 128);
-    mbar_init(bar(BAR_PV), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(BAR_S0 + i), 1);
+      mbar_init(bar(BAR_P0 + i), 128);
+      mbar_init(bar(BAR_PV0 + i), 1);
+    }
     mbar_init(bar(BAR_DRAIN), 1);
     *abort_flag = 0;
     *resc_flag = 0;
     fence_mbar_init();
   }
   uint32_t tmem_cols = 32;
-  while (tmem_cols < (uint32_t)(RP * (1 + KC))) tmem_cols <<= 1;
+  while (tmem_cols < (uint32_t)(RP * (2 + KC))) tmem_cols <<= 1;
   if (warp == WARP_MMA) {
     tmem_alloc(smem_u32(tmem_slot), tmem_cols);
     tmem_relinquish();
@@ -157,8 +178,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t TS = 0;                           // S^T: RP columns
-  auto TO = [&](int c) { return (uint32_t)(RP * (1 + c)); };  // O^T chunk c
+  auto TS = [&](int buf) { return (uint32_t)(RP * buf); };            // S^T buffers
+  auto TO = [&](int c) { return (uint32_t)(RP * (2 + c)); };          // O^T chunk c
+  auto PB = [&](int buf) { return L.off_p + (uint32_t)buf * 2u * RP * 128u; };  // P buffers
   const Watchdog wd{abort_flag, p.status, p.timeout_ns};
   int issued = 0;
 
@@ -170,20 +192,28 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_arrive_expect_tx(bar(BAR_Q), (uint32_t)(D / 64) * R * 128u);
       for (int kb = 0; kb < D / 64; ++kb)
         tma_load_4d(base + L.off_q + (uint32_t)kb * RP * 128u, &tm_q, bar(BAR_Q), kb * 64, kvh * g, 0, b);
-      const int total = n_tiles * 2 * KC;
-      for (int n = 0; n < total; ++n) {
-        const int slot = n % nbuf, use = n / nbuf;
-        if (use > 0 && !mbar_wait(bar(bar_empty(slot)), (uint32_t)(use - 1) & 1u, wd)) break;
-        const int j = n / (2 * KC), within = n - j * 2 * KC;
-        const bool is_v = within >= KC;
-        const int c = is_v ? within - KC : within;
-        const CUtensorMap* tm = is_v ? &tm_v : &tm_k;
-        const int key0 = lo + j * BN;
-        mbar_arrive_expect_tx(bar(bar_full(slot)), SLOT_BYTES);
-        const uint32_t dst = base + L.off_ring + (uint32_t)slot * SLOT_BYTES;
-        tma_load_4d(dst, tm, bar(bar_full(slot)), (2 * c) * 64, kvh, key0, b);
-        tma_load_4d(dst + BOX_BYTES, tm, bar(bar_full(slot)), (2 * c + 1) * 64, kvh, key0, b);
-        issued = n + 1;
+      // ring order: K_0, then (K_{j+1}, V_j) for j = 0..n-1; KC slots each
+      bool ok = true;
+      int n = 0;
+      auto issue = [&](const CUtensorMap* tm, int j) {
+        for (int c = 0; c < KC; ++c, ++n) {
+          const int slot = n % nbuf, use = n / nbuf;
+          if (use > 0 && !mbar_wait(bar(bar_empty(slot)), (uint32_t)(use - 1) & 1u, wd)) {
+            ok = false;
+            return;
+          }
+          mbar_arrive_expect_tx(bar(bar_full(slot)), SLOT_BYTES);
+          const uint32_t dst = base + L.off_ring + (uint32_t)slot * SLOT_BYTES;
+          const int key0 = lo + j * BN;
+          tma_load_4d(dst, tm, bar(bar_full(slot)), (2 * c) * 64, kvh, key0, b);
+          tma_load_4d(dst + BOX_BYTES, tm, bar(bar_full(slot)), (2 * c + 1) * 64, kvh, key0, b);
+          issued = n + 1;
+        }
+      };
+      issue(&tm_k, 0);
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        if (j + 1 < n_tiles) issue(&tm_k, j + 1);
+        if (ok) issue(&tm_v, j);
       }
     }
   } else if (warp == WARP_MMA) {
@@ -193,11 +223,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       bool ok = mbar_wait(bar(BAR_Q), 0, wd);
       tc_fence_after();
       int n = 0;
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        // S^T = K Q^T over D, one 128-column slot at a time
-        for (int c = 0; ok && c < KC; ++c, ++n) {
+      // S^T_j = K_j Q^T into S buffer j%2, one 128-column slot at a time
+      auto mma_s = [&](int j) {
+        for (int c = 0; c < KC; ++c, ++n) {
           const int slot = n % nbuf;
-          if (!mbar_wait(bar(bar_full(slot)), (uint32_t)(n / nbuf) & 1u, wd)) { ok = false; break; }
+          if (!mbar_wait(bar(bar_full(slot)), (uint32_t)(n / nbuf) & 1u, wd)) { ok = false; return; }
           tc_fence_after();
           const uint32_t kb = base + L.off_ring + (uint32_t)slot * SLOT_BYTES;
 #pragma unroll
@@ -205,16 +235,24 @@ __global__ void __launch_bounds__(THREADS, 1)
             const uint32_t in_box = (uint32_t)(kk & 3) * 32u;
             const uint32_t a = kb + (uint32_t)(kk >> 2) * BOX_BYTES + in_box;
             const uint32_t qb = base + L.off_q + (uint32_t)(2 * c + (kk >> 2)) * RP * 128u + in_box;
-            mma_ss(tmem + TS, sdesc_sw128(a, 16, 1024), sdesc_sw128(qb, 16, 1024), idesc_s,
+            mma_ss(tmem + TS(j & 1), sdesc_sw128(a, 16, 1024), sdesc_sw128(qb, 16, 1024), idesc_s,
                    (c > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(bar(bar_empty(slot)));
         }
-        if (!ok) break;
-        mma_commit(bar(BAR_S));
-        if (!mbar_wait(bar(BAR_P), (uint32_t)j & 1u, wd)) { ok = false; break; }
+        mma_commit(bar(BAR_S0 + (j & 1)));
+      };
+      if (ok) mma_s(0);
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        // S buffer (j+1)%2 was last read by softmax j-1, whose P the PV of
+        // tile j-1 (issued before this point) already waited for.
+        if (j + 1 < n_tiles) {
+          mma_s(j + 1);
+          if (!ok) break;
+        }
+        if (!mbar_wait(bar(BAR_P0 + (j & 1)), (uint32_t)(j >> 1) & 1u, wd)) { ok = false; break; }
         tc_fence_after();
-        // O^T(c) += V^T(c) P^T
+        // O^T(c) += V_j^T(c) P_j^T
         for (int c = 0; ok && c < KC; ++c, ++n) {
           const int slot = n % nbuf;
           if (!mbar_wait(bar(bar_full(slot)), (uint32_t)(n / nbuf) & 1u, wd)) { ok = false; break; }
@@ -223,14 +261,14 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t a = vb + (uint32_t)kk * 2048u;
-            const uint32_t pb = base + L.off_p + (uint32_t)(kk >> 2) * RP * 128u + (uint32_t)(kk & 3) * 32u;
+            const uint32_t pb = base + PB(j & 1) + (uint32_t)(kk >> 2) * RP * 128u + (uint32_t)(kk & 3) * 32u;
             mma_ss(tmem + TO(c), sdesc_sw128(a, BOX_BYTES, 1024), sdesc_sw128(pb, 16, 1024), idesc_o,
                    (j > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(bar(bar_empty(slot)));
         }
         if (!ok) break;
-        mma_commit(bar(BAR_PV));
+        mma_commit(bar(BAR_PV0 + (j & 1)));
       }
     }
   } else {
@@ -238,27 +276,29 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int t = threadIdx.x;          // 0..127
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const float c2 = p.c2;
-    uint8_t* pbuf = gbase + L.off_p;
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
+      const int sb = j & 1;
       // every give-up is decided jointly (barrier + OR) so no thread is left
       // waiting at a named barrier or inside a warp-collective TMEM access
-      const bool got_s = mbar_wait(bar(BAR_S), (uint32_t)j & 1u, wd);
+      const bool got_s = mbar_wait(bar(BAR_S0 + sb), (uint32_t)(j >> 1) & 1u, wd);
       if (named_bar_or(1, 128, !got_s)) { ok = false; break; }
       tc_fence_after();
-      const int key = lo + j * BN + t;
-      const bool key_ok = key < hi;
+      const int tile0 = lo + j * BN;
+      const int key = tile0 + t;
+      // whole tile visible to every real row: no per-element mask
+      const bool full = (tile0 + BN - 1 < hi) && (!p.causal || tile0 + BN - 1 <= p.q_offset);
       // pass 1: per-row max over the tile's visible keys
       for (int q = 0; q < RP / 16; ++q) {
         float v[16];
-        tmem_ld16(tmem + lane_off + TS + 16 * q, v);
+        tmem_ld16(tmem + lane_off + TS(sb) + 16 * q, v);
+        if (!full) {
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int r = 16 * q + e;
-          const bool vis = key_ok && r < R && (!p.causal || key <= p.q_offset + r / g);
-          const float x = warp_max(vis ? v[e] : -INFINITY);
-          if (lane == 0) red_max[warp * RP + r] = x;
+          for (int e = 0; e < 16; ++e)
+            if (!(key < hi && key <= lim_sm[16 * q + e])) v[e] = -INFINITY;
         }
+        const float x = warp_reduce16<true>(v, lane);
+        if (lane < 16) red_max[warp * RP + 16 * q + lane] = x;
       }
       named_bar_sync(1, 128);
       if (t < RP) {
@@ -275,32 +315,37 @@ __global__ void __launch_bounds__(THREADS, 1)
         alpha_sm[t] = alpha;
         msub_sm[t] = (m_new == -INFINITY) ? 0.f : m_new;
       }
-      // P (and O) of the previous tile must be consumed before they change
-      const bool got_pv = (j == 0) || mbar_wait(bar(BAR_PV), (uint32_t)(j - 1) & 1u, wd);
-      if (named_bar_or(1, 128, !got_pv)) { ok = false; break; }
+      // P buffer sb was read by the P.V of tile j-2: wait for it before rewriting
+      const bool got_pb = (j < 2) || mbar_wait(bar(BAR_PV0 + sb), (uint32_t)((j - 2) >> 1) & 1u, wd);
+      if (named_bar_or(1, 128, !got_pb)) { ok = false; break; }
       tc_fence_after();
       const bool rescale = (j > 0) && (*resc_flag != 0);
       // pass 2: exponentials, P (bf16) into the swizzled B-operand buffer
       {
         const int half = t >> 6, tt = t & 63;
-        uint8_t* pcol = pbuf + (size_t)half * RP * 128 + (size_t)(tt & 7) * 2;
+        uint8_t* pcol = gbase + PB(sb) + (size_t)half * RP * 128 + (size_t)(tt & 7) * 2;
         const int chunk16 = tt >> 3;
         for (int q = 0; q < RP / 16; ++q) {
           float v[16];
-          tmem_ld16(tmem + lane_off + TS + 16 * q, v);
+          tmem_ld16(tmem + lane_off + TS(sb) + 16 * q, v);
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int r = 16 * q + e;
-            const bool vis = key_ok && r < R && (!p.causal || key <= p.q_offset + r / g);
-            const float pv = vis ? ex2_approx(fmaf(v[e], c2, -msub_sm[r])) : 0.f;
+            float pv = ex2_approx(fmaf(v[e], c2, -msub_sm[r]));
+            if (!full && !(key < hi && key <= lim_sm[r])) pv = 0.f;
             *reinterpret_cast<__nv_bfloat16*>(pcol + (size_t)r * 128 + ((chunk16 ^ (r & 7)) << 4)) =
                 __float2bfloat16_rn(pv);
-            const float s = warp_sum(pv);
-            if (lane == 0) red_sum[warp * RP + r] = s;
+            v[e] = pv;
           }
+          const float s = warp_reduce16<false>(v, lane);
+          if (lane < 16) red_sum[warp * RP + 16 * q + lane] = s;
         }
       }
       if (rescale) {
+        // O^T is accumulated by the P.V of tile j-1: it must have completed
+        const bool got_o = mbar_wait(bar(BAR_PV0 + (sb ^ 1)), (uint32_t)((j - 1) >> 1) & 1u, wd);
+        if (named_bar_or(1, 128, !got_o)) { ok = false; break; }
+        tc_fence_after();
         for (int c = 0; c < KC; ++c) {
           for (int q = 0; q < RP / 16; ++q) {
             float v[16];
@@ -321,10 +366,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       fence_proxy_async_smem();
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(BAR_P));
+      mbar_arrive(bar(BAR_P0 + sb));
     }
     // ---- epilogue: normalised partial O and the split's LSE ----
-    const bool got_o = ok && mbar_wait(bar(BAR_PV), (uint32_t)(n_tiles - 1) & 1u, wd);
+    const int last = n_tiles - 1;
+    const bool got_o = ok && mbar_wait(bar(BAR_PV0 + (last & 1)), (uint32_t)(last >> 1) & 1u, wd);
     if (ok && !named_bar_or(1, 128, !got_o)) {
       tc_fence_after();
       if (t < RP) {

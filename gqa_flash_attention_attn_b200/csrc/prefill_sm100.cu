@@ -233,18 +233,22 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
         if (__any_sync(0xffffffffu, !got)) { ok = false; break; }
         tc_fence_after();
         const int cl = vis_end - j * BN;  // visible columns of this tile for this row
-        const bool masked = cl < BN;
-        float mx = -INFINITY;
+        // one TMEM read of the whole 128-column S row
+        float sv[BN];
+        tmem_ld128(tS, sv);
+        if (__any_sync(0xffffffffu, cl < BN)) {  // diagonal or ragged tile: mask in place
 #pragma unroll
-        for (int c = 0; c < BN / 32; ++c) {
-          float v[32];
-          tmem_ld32(tS + 32 * c, v);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float x = (masked && (32 * c + e) >= cl) ? -INFINITY : v[e];
-            mx = fmaxf(mx, x);
-          }
+          for (int e = 0; e < BN; ++e) sv[e] = (e < cl) ? sv[e] : -INFINITY;
         }
+        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < BN; e += 8) {
+          mx0 = fmax3(mx0, sv[e], sv[e + 1]);
+          mx1 = fmax3(mx1, sv[e + 2], sv[e + 3]);
+          mx2 = fmax3(mx2, sv[e + 4], sv[e + 5]);
+          mx3 = fmax3(mx3, sv[e + 6], sv[e + 7]);
+        }
+        const float mx = fmax3(mx0, mx1, fmaxf(mx2, mx3));
         const float m_tile = mx * c2;
         float m_new = m_use, alpha = 1.f;
         if (m_tile > m_use + 8.f) {
@@ -252,26 +256,22 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
           alpha = ex2_approx(m_use - m_new);
         }
         const float m_sub = (m_new == -INFINITY) ? 0.f : m_new;
-        float sum = 0.f;
+        // p = 2^(s*c2 - m): one packed FFMA per pair, ex2 per element, packed
+        // partial sums, bf16 pairs for the P.V operand (masked s = -inf -> p = 0)
+        const float2 c2v = make_float2(c2, c2);
+        const float2 nmv = make_float2(-m_sub, -m_sub);
+        float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+        uint32_t pk[BN / 2];
 #pragma unroll
-        for (int c = 0; c < BN / 32; ++c) {
-          float v[32];
-          tmem_ld32(tS + 32 * c, v);
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            float p0 = ex2_approx(fmaf(v[2 * e], c2, -m_sub));
-            float p1 = ex2_approx(fmaf(v[2 * e + 1], c2, -m_sub));
-            if (masked) {
-              if (32 * c + 2 * e >= cl) p0 = 0.f;
-              if (32 * c + 2 * e + 1 >= cl) p1 = 0.f;
-            }
-            sum += p0 + p1;
-            pk[e] = pack_bf16x2(p0, p1);
-          }
-          // P chunk c lands on TMEM columns [16c, 16c+16), already read as S.
-          tmem_st16(tS + 16 * c, pk);
+        for (int e = 0; e < BN / 2; ++e) {
+          const float2 x = ffma2(make_float2(sv[2 * e], sv[2 * e + 1]), c2v, nmv);
+          const float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          if (e & 1) acc1 = fadd2(acc1, pr); else acc0 = fadd2(acc0, pr);
+          pk[e] = pack_bf16x2(pr.x, pr.y);
         }
+        const float sum = (acc0.x + acc0.y) + (acc1.x + acc1.y);
+        // P lands on TMEM columns [0, 64) of this slot's S region (already read)
+        tmem_st64(tS, pk);
         l = l * alpha + sum;
         if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
           // s_full(j) completing implies the previous P.V into O_i completed.

@@ -90,8 +90,9 @@ int attn_prefill(const void* q, const void* k, const void* v, void* out, float* 
  *
  *   D            128, 256 or 512 (else ATTN_ERR_UNSUPPORTED)
  *   rows         R = (Hq/Hkv) * Sq query rows share one K/V head; R rounded up
- *                to a multiple of 16 must satisfy (1 + D/128) * R16 <= 256
- *                (else ATTN_ERR_UNSUPPORTED)
+ *                to a multiple of 16 must satisfy (2 + D/128) * R16 <= 256
+ *                (else ATTN_ERR_UNSUPPORTED): at most 128 rows for D = 128,
+ *                64 for D = 256, 32 for D = 512
  *   num_splits   1 <= num_splits <= Skv (else ATTN_ERR_INVALID_ARG)
  *   partial_out  num_splits*B*Sq*Hq*D floats; partial_lse num_splits*B*Hq*Sq
  */

@@ -92,8 +92,10 @@ def _decode(lib, **kw):
     (dict(Hq=12, Hkv=8), ga.ATTN_ERR_INVALID_ARG),
     (dict(D=64), ga.ATTN_ERR_UNSUPPORTED),
     (dict(D=96), ga.ATTN_ERR_UNSUPPORTED),
-    (dict(Hq=64, Sq=1), ga.ATTN_ERR_UNSUPPORTED),   # 64 rows x (1 + 512/128) > 256 TMEM columns
+    (dict(Hq=64, Sq=1), ga.ATTN_ERR_UNSUPPORTED),   # 64 rows x (2 + 512/128) > 256 TMEM columns
     (dict(D=128, Hq=32, Hkv=1, Sq=8), ga.ATTN_ERR_UNSUPPORTED),  # 256 rows
+    (dict(D=512, Hq=48, Hkv=1, Sq=1), ga.ATTN_ERR_UNSUPPORTED),  # 48 x (2 + 4) > 256
+    (dict(D=256, Hq=80, Hkv=1, Sq=1), ga.ATTN_ERR_UNSUPPORTED),  # 80 x (2 + 2) > 256
     (dict(po=MIS), ga.ATTN_ERR_ALIGNMENT),
     (dict(k=MIS), ga.ATTN_ERR_ALIGNMENT),
     (dict(pl=ctypes.c_void_p(0x20001)), ga.ATTN_ERR_ALIGNMENT),
