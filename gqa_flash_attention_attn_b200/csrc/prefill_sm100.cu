@@ -11,6 +11,13 @@
 //   MMA        one thread issues tcgen05.mma: S_i = Q_i K_j^T (both operands in
 //              shared memory, fp32 accumulator in TMEM), then O_i += P_i V_j
 //              with P_i read from TMEM (A operand) and V_j from shared memory.
+//              With two slots the issue order is S0_j, O1 += P1_{j-1} V_{j-1},
+//              S1_j, O0 += P0_j V_j, so while one softmax warpgroup works the
+//              tensor core runs the other slot's two GEMMs.  P_i lives inside
+//              S_i's TMEM columns; the next S_i into that region is issued
+//              right behind the P.V that reads it (tcgen05 MMAs of one CTA
+//              execute in issue order).  With one slot (D = 256) S is double
+//              buffered instead and the ring streams K_0, K_1, V_0, K_2, V_1, ...
 //   softmax    one warpgroup per slot, one thread per query row (TMEM lane):
 //              online softmax in fp32 with the running (max, rowsum) per row
 //              ("Anbeeld/beellama.cpp PR #149", Overview: fp32 rescale and
@@ -51,8 +58,10 @@ struct PrefillCfg {
   static constexpr int NBARS = 1 + 2 * NBUF + 6 + 1;
   static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
   static constexpr uint32_t SMEM = OFF_MISC + 16 + 1024;  // + alignment slack
-  static constexpr uint32_t TMEM_S = 0;                   // S_i (and P_i) at i*128
-  static constexpr uint32_t TMEM_O = NSLOT * 128;         // O_i at TMEM_O + i*D
+  // Two S buffers (one per slot, or a double buffer for one slot), P aliased
+  // at the start of its S buffer, then O per slot.
+  static constexpr uint32_t TMEM_S = 0;                   // S buffer b at b*128
+  static constexpr uint32_t TMEM_O = 256;                 // O_i at TMEM_O + i*D
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int BAR_Q = 0;
   __host__ __device__ static constexpr int bar_full(int b) { return 1 + b; }
@@ -61,7 +70,7 @@ struct PrefillCfg {
   __host__ __device__ static constexpr int bar_p(int i) { return 3 + 2 * NBUF + i; }
   __host__ __device__ static constexpr int bar_pv(int i) { return 5 + 2 * NBUF + i; }
   static constexpr int BAR_DRAIN = 7 + 2 * NBUF;
-  static_assert(NSLOT * 128 + NSLOT * D <= 512, "TMEM budget");
+  static_assert(256 + NSLOT * D <= 512, "TMEM budget");
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(D % 64 == 0, "head dim must be a multiple of 64");
 };
@@ -72,6 +81,23 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
   while (!mbar_try_wait(bar, parity)) {
     if (globaltimer_ns() - t0 > limit_ns) break;
   }
+}
+
+// Item n of the K/V ring: returns true for a V tile, false for a K tile, and
+// the tile index.  Two slots: K_0, V_0, K_1, V_1, ...  One slot (double-
+// buffered S): K_0, K_1, V_0, K_2, V_1, ..., K_{n-1}, V_{n-2}, V_{n-1}.
+template <int NSLOT>
+__device__ __forceinline__ bool ring_item(int n, int n_tiles, int& tile) {
+  if (NSLOT == 2) {
+    tile = n >> 1;
+    return (n & 1) != 0;
+  }
+  if (n == 0) { tile = 0; return false; }
+  if (n == 2 * n_tiles - 1) { tile = n_tiles - 1; return true; }
+  const int m = n - 1;
+  if ((m & 1) == 0) { tile = (m >> 1) + 1; return false; }
+  tile = m >> 1;
+  return true;
 }
 
 template <int D>
@@ -152,8 +178,10 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
         const int buf = n % C::NBUF;
         const int use = n / C::NBUF;
         if (use > 0 && !mbar_wait(bar(C::bar_empty(buf)), (uint32_t)(use - 1) & 1u, wd)) break;
-        const CUtensorMap* tm = (n & 1) ? &tm_v : &tm_k;
-        const int key0 = (n >> 1) * BN;
+        int tile;
+        const bool is_v = ring_item<C::NSLOT>(n, n_tiles, tile);
+        const CUtensorMap* tm = is_v ? &tm_v : &tm_k;
+        const int key0 = tile * BN;
         mbar_arrive_expect_tx(bar(C::bar_full(buf)), C::TILE);
         for (int kb = 0; kb < C::KB; ++kb)
           tma_load_4d(base + C::OFF_KV + buf * C::TILE + kb * BOX_BYTES, tm, bar(C::bar_full(buf)),
@@ -165,50 +193,105 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
     if (lane == 0) {
       constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, false, false);
       constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, false, true);
+      const bool act1 = (C::NSLOT == 2) && (hl0 + 1 < p.g);
+      auto slot_addr = [&](int n) -> uint32_t { return base + C::OFF_KV + (uint32_t)(n % C::NBUF) * C::TILE; };
+      auto wait_full = [&](int n) -> bool {
+        if (!mbar_wait(bar(C::bar_full(n % C::NBUF)), (uint32_t)(n / C::NBUF) & 1u, wd)) return false;
+        tc_fence_after();
+        return true;
+      };
+      auto wait_p = [&](int b, uint32_t phase) -> bool {
+        if (!mbar_wait(bar(C::bar_p(b)), phase & 1u, wd)) return false;
+        tc_fence_after();
+        return true;
+      };
+      // S buffer sb = Q(qslot) K^T
+      auto gemm_s = [&](int sb, int qslot, uint32_t kbase) {
+        const uint32_t qbase = base + C::OFF_Q + (uint32_t)qslot * C::TILE;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (uint32_t)(kk >> 2) * BOX_BYTES + (uint32_t)(kk & 3) * 32u;
+          mma_ss(tmem + C::TMEM_S + sb * 128, sdesc_sw128(qbase + off, 16, 1024),
+                 sdesc_sw128(kbase + off, 16, 1024), IDESC_QK, kk > 0 ? 1u : 0u);
+        }
+      };
+      // O(oslot) (+)= P(from S buffer pb) V
+      auto gemm_pv = [&](int oslot, int pb, uint32_t vbase, bool first) {
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_ts(tmem + C::TMEM_O + oslot * D, tmem + C::TMEM_S + pb * 128 + kk * 8,
+                 sdesc_sw128(vbase + kk * 2048u, BOX_BYTES, 1024), IDESC_PV, (!first || kk > 0) ? 1u : 0u);
+      };
       bool ok = mbar_wait(bar(C::BAR_Q), 0, wd);
       tc_fence_after();
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        // ---- S_i = Q_i K_j^T ----
-        const int nk = 2 * j, bk = nk % C::NBUF;
-        if (!mbar_wait(bar(C::bar_full(bk)), (uint32_t)(nk / C::NBUF) & 1u, wd)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t kbase = base + C::OFF_KV + bk * C::TILE;
-        for (int i = 0; ok && i < C::NSLOT; ++i) {
-          if (hl0 + i >= p.g) continue;
-          if (j > 0) {  // S_i aliases P_i, which the previous P.V reads
-            if (!mbar_wait(bar(C::bar_pv(i)), (uint32_t)(j - 1) & 1u, wd)) { ok = false; break; }
-            tc_fence_after();
+      if (C::NSLOT == 2) {
+        // tile 0
+        if (ok) ok = wait_full(0);
+        if (ok) {
+          gemm_s(0, 0, slot_addr(0));
+          mma_commit(bar(C::bar_s(0)));
+          if (act1) {
+            gemm_s(1, 1, slot_addr(0));
+            mma_commit(bar(C::bar_s(1)));
           }
-          const uint32_t qbase = base + C::OFF_Q + i * C::TILE;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (uint32_t)(kk >> 2) * BOX_BYTES + (uint32_t)(kk & 3) * 32u;
-            mma_ss(tmem + C::TMEM_S + i * 128, sdesc_sw128(qbase + off, 16, 1024),
-                   sdesc_sw128(kbase + off, 16, 1024), IDESC_QK, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(bar(C::bar_s(i)));
+          mma_commit(bar(C::bar_empty(0 % C::NBUF)));
+          ok = wait_full(1) && wait_p(0, 0);
         }
-        if (!ok) break;
-        mma_commit(bar(C::bar_empty(bk)));
-        // ---- O_i += P_i V_j ----
-        const int nv = nk + 1, bv = nv % C::NBUF;
-        if (!mbar_wait(bar(C::bar_full(bv)), (uint32_t)(nv / C::NBUF) & 1u, wd)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t vbase = base + C::OFF_KV + bv * C::TILE;
-        for (int i = 0; ok && i < C::NSLOT; ++i) {
-          if (hl0 + i >= p.g) continue;
-          if (!mbar_wait(bar(C::bar_p(i)), (uint32_t)j & 1u, wd)) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk) {
-            mma_ts(tmem + C::TMEM_O + i * D, tmem + C::TMEM_S + i * 128 + kk * 8,
-                   sdesc_sw128(vbase + kk * 2048u, BOX_BYTES, 1024), IDESC_PV,
-                   (j > 0 || kk > 0) ? 1u : 0u);
-          }
-          mma_commit(bar(C::bar_pv(i)));
+        if (ok) {
+          gemm_pv(0, 0, slot_addr(1), true);
+          mma_commit(bar(C::bar_pv(0)));
         }
-        if (!ok) break;
-        mma_commit(bar(C::bar_empty(bv)));
+        for (int i = 1; ok && i < n_tiles; ++i) {
+          const int nk = 2 * i;
+          if (!(ok = wait_full(nk))) break;
+          gemm_s(0, 0, slot_addr(nk));                       // S0_i (behind O0 += P0_{i-1} V_{i-1})
+          mma_commit(bar(C::bar_s(0)));
+          if (act1) {
+            if (!(ok = wait_p(1, (uint32_t)(i - 1)))) break;
+            gemm_pv(1, 1, slot_addr(nk - 1), i == 1);        // O1 += P1_{i-1} V_{i-1}
+            mma_commit(bar(C::bar_pv(1)));
+          }
+          mma_commit(bar(C::bar_empty((nk - 1) % C::NBUF)));  // V_{i-1} done
+          if (act1) {
+            gemm_s(1, 1, slot_addr(nk));                     // S1_i (behind the P1 read)
+            mma_commit(bar(C::bar_s(1)));
+          }
+          mma_commit(bar(C::bar_empty(nk % C::NBUF)));        // K_i done
+          if (!(ok = wait_full(nk + 1) && wait_p(0, (uint32_t)i))) break;
+          gemm_pv(0, 0, slot_addr(nk + 1), false);           // O0 += P0_i V_i
+          mma_commit(bar(C::bar_pv(0)));
+        }
+        if (ok) {
+          const int nv = 2 * n_tiles - 1;
+          if (act1 && (ok = wait_p(1, (uint32_t)(n_tiles - 1)))) {
+            gemm_pv(1, 1, slot_addr(nv), n_tiles == 1);
+            mma_commit(bar(C::bar_pv(1)));
+          }
+          if (ok) mma_commit(bar(C::bar_empty(nv % C::NBUF)));
+        }
+      } else {
+        // one slot, S double buffered: S_0, then per tile S_{j+1} and O += P_j V_j
+        int n = 0;
+        if (ok && (ok = wait_full(n))) {
+          gemm_s(0, 0, slot_addr(n));
+          mma_commit(bar(C::bar_s(0)));
+          mma_commit(bar(C::bar_empty(n % C::NBUF)));
+          ++n;
+        }
+        for (int j = 0; ok && j < n_tiles; ++j) {
+          if (j + 1 < n_tiles) {
+            if (!(ok = wait_full(n))) break;
+            gemm_s((j + 1) & 1, 0, slot_addr(n));            // behind the P.V that read this buffer
+            mma_commit(bar(C::bar_s((j + 1) & 1)));
+            mma_commit(bar(C::bar_empty(n % C::NBUF)));
+            ++n;
+          }
+          if (!(ok = wait_full(n) && wait_p(j & 1, (uint32_t)(j >> 1)))) break;
+          gemm_pv(0, j & 1, slot_addr(n), j == 0);
+          mma_commit(bar(C::bar_pv(0)));
+          mma_commit(bar(C::bar_empty(n % C::NBUF)));
+          ++n;
+        }
       }
     }
   } else {
@@ -220,7 +303,6 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
       const int h = kvh * p.g + hl;
       const int r = wq * 32 + lane;
       const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-      const uint32_t tS = tmem + lane_off + C::TMEM_S + slot * 128;
       const uint32_t tO = tmem + lane_off + C::TMEM_O + slot * D;
       const int s_row = s0 + r;
       const int vis_end = p.causal ? min(p.Skv, p.q_offset + s_row + 1) : p.Skv;
@@ -228,8 +310,12 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
       float m_use = -INFINITY, l = 0.f;
       bool ok = true;
       for (int j = 0; j < n_tiles; ++j) {
+        // S buffer and its phase: per slot, or alternating for one slot
+        const int sb = (C::NSLOT == 2) ? slot : (j & 1);
+        const uint32_t ph = (C::NSLOT == 2) ? ((uint32_t)j & 1u) : ((uint32_t)(j >> 1) & 1u);
+        const uint32_t tS = tmem + lane_off + C::TMEM_S + sb * 128;
         // a give-up must be warp-uniform: TMEM loads/stores are warp-collective
-        const bool got = mbar_wait(bar(C::bar_s(slot)), (uint32_t)j & 1u, wd);
+        const bool got = mbar_wait(bar(C::bar_s(sb)), ph, wd);
         if (__any_sync(0xffffffffu, !got)) { ok = false; break; }
         tc_fence_after();
         const int cl = vis_end - j * BN;  // visible columns of this tile for this row
@@ -274,7 +360,14 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
         tmem_st64(tS, pk);
         l = l * alpha + sum;
         if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-          // s_full(j) completing implies the previous P.V into O_i completed.
+          // Two slots: S_i(j) was issued behind O_i += P_i(j-1) V, so its
+          // completion implies that P.V completed.  One slot: S(j) was issued
+          // before that P.V, so wait for it here.
+          if (C::NSLOT == 1) {
+            const bool got_pv = mbar_wait(bar(C::bar_pv(0)), (uint32_t)(j - 1) & 1u, wd);
+            if (__any_sync(0xffffffffu, !got_pv)) { ok = false; break; }
+            tc_fence_after();
+          }
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
             float v[32];
@@ -287,9 +380,16 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
         m_use = m_new;
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(C::bar_p(slot)));
+        mbar_arrive(bar(C::bar_p(sb)));
       }
-      const bool got_o = ok && mbar_wait(bar(C::bar_pv(slot)), (uint32_t)(n_tiles - 1) & 1u, wd);
+      // Wait for the last P.V.  A parity wait for completion k is only
+      // unambiguous once completion k-1 has happened: with two slots the
+      // last S_i was issued behind P.V(n-2), with one slot it was not, so
+      // there completion n-2 is awaited first.
+      bool got_o = ok;
+      if (got_o && C::NSLOT == 1 && n_tiles >= 2)
+        got_o = mbar_wait(bar(C::bar_pv(0)), (uint32_t)(n_tiles - 2) & 1u, wd);
+      got_o = got_o && mbar_wait(bar(C::bar_pv(C::NSLOT == 2 ? slot : 0)), (uint32_t)(n_tiles - 1) & 1u, wd);
       if (!__any_sync(0xffffffffu, !got_o)) {
         tc_fence_after();
         const float inv_l = 1.f / l;
