@@ -23,7 +23,7 @@
 #include <cstdint>
 #include <mutex>
 
-#include "../../include/attn.h"
+#include "attn.h"
 #include "kernels.h"
 
 namespace {

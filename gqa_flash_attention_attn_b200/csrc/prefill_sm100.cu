@@ -54,8 +54,8 @@ struct PrefillCfg {
   static constexpr uint32_t OFF_Q = 0;
   static constexpr uint32_t OFF_KV = NSLOT * TILE;
   static constexpr uint32_t OFF_BAR = OFF_KV + NBUF * TILE;
-  // q_full, kv_full[NBUF], kv_empty[NBUF], s_full[2], p_full[2], pv_done[2], drain
-  static constexpr int NBARS = 1 + 2 * NBUF + 6 + 1;
+  // q_full, kv_full[NBUF], kv_empty[NBUF], s_full[2], p_lo[2], p_hi[2], pv_done[2], drain
+  static constexpr int NBARS = 1 + 2 * NBUF + 8 + 1;
   static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
   static constexpr uint32_t SMEM = OFF_MISC + 16 + 1024;  // + alignment slack
   // Two S buffers (one per slot, or a double buffer for one slot), P aliased
@@ -67,9 +67,10 @@ struct PrefillCfg {
   __host__ __device__ static constexpr int bar_full(int b) { return 1 + b; }
   __host__ __device__ static constexpr int bar_empty(int b) { return 1 + NBUF + b; }
   __host__ __device__ static constexpr int bar_s(int i) { return 1 + 2 * NBUF + i; }
-  __host__ __device__ static constexpr int bar_p(int i) { return 3 + 2 * NBUF + i; }
-  __host__ __device__ static constexpr int bar_pv(int i) { return 5 + 2 * NBUF + i; }
-  static constexpr int BAR_DRAIN = 7 + 2 * NBUF;
+  __host__ __device__ static constexpr int bar_plo(int i) { return 3 + 2 * NBUF + i; }
+  __host__ __device__ static constexpr int bar_phi(int i) { return 5 + 2 * NBUF + i; }
+  __host__ __device__ static constexpr int bar_pv(int i) { return 7 + 2 * NBUF + i; }
+  static constexpr int BAR_DRAIN = 9 + 2 * NBUF;
   static_assert(256 + NSLOT * D <= 512, "TMEM budget");
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(D % 64 == 0, "head dim must be a multiple of 64");
@@ -140,7 +141,8 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(C::bar_s(i)), 1);
-      mbar_init(bar(C::bar_p(i)), 128);
+      mbar_init(bar(C::bar_plo(i)), 128);
+      mbar_init(bar(C::bar_phi(i)), 128);
       mbar_init(bar(C::bar_pv(i)), 1);
     }
     mbar_init(bar(C::BAR_DRAIN), 1);
@@ -200,11 +202,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
         tc_fence_after();
         return true;
       };
-      auto wait_p = [&](int b, uint32_t phase) -> bool {
-        if (!mbar_wait(bar(C::bar_p(b)), phase & 1u, wd)) return false;
-        tc_fence_after();
-        return true;
-      };
+
       // S buffer sb = Q(qslot) K^T
       auto gemm_s = [&](int sb, int qslot, uint32_t kbase) {
         const uint32_t qbase = base + C::OFF_Q + (uint32_t)qslot * C::TILE;
@@ -215,12 +213,19 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
                  sdesc_sw128(kbase + off, 16, 1024), IDESC_QK, kk > 0 ? 1u : 0u);
         }
       };
-      // O(oslot) (+)= P(from S buffer pb) V
-      auto gemm_pv = [&](int oslot, int pb, uint32_t vbase, bool first) {
+      // O(oslot) (+)= P(from S buffer pb) V, each half of P as soon as it is
+      // in TMEM (phase: completion index of that buffer's P barriers)
+      auto gemm_pv = [&](int oslot, int pb, uint32_t vbase, bool first, uint32_t phase) -> bool {
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          mma_ts(tmem + C::TMEM_O + oslot * D, tmem + C::TMEM_S + pb * 128 + kk * 8,
-                 sdesc_sw128(vbase + kk * 2048u, BOX_BYTES, 1024), IDESC_PV, (!first || kk > 0) ? 1u : 0u);
+        for (int half = 0; half < 2; ++half) {
+          if (!mbar_wait(bar(half == 0 ? C::bar_plo(pb) : C::bar_phi(pb)), phase & 1u, wd)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = half * (BN / 32); kk < (half + 1) * (BN / 32); ++kk)
+            mma_ts(tmem + C::TMEM_O + oslot * D, tmem + C::TMEM_S + pb * 128 + kk * 8,
+                   sdesc_sw128(vbase + kk * 2048u, BOX_BYTES, 1024), IDESC_PV, (!first || kk > 0) ? 1u : 0u);
+        }
+        return true;
       };
       bool ok = mbar_wait(bar(C::BAR_Q), 0, wd);
       tc_fence_after();
@@ -235,11 +240,8 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
             mma_commit(bar(C::bar_s(1)));
           }
           mma_commit(bar(C::bar_empty(0 % C::NBUF)));
-          ok = wait_full(1) && wait_p(0, 0);
-        }
-        if (ok) {
-          gemm_pv(0, 0, slot_addr(1), true);
-          mma_commit(bar(C::bar_pv(0)));
+          ok = wait_full(1) && gemm_pv(0, 0, slot_addr(1), true, 0);
+          if (ok) mma_commit(bar(C::bar_pv(0)));
         }
         for (int i = 1; ok && i < n_tiles; ++i) {
           const int nk = 2 * i;
@@ -247,8 +249,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
           gemm_s(0, 0, slot_addr(nk));                       // S0_i (behind O0 += P0_{i-1} V_{i-1})
           mma_commit(bar(C::bar_s(0)));
           if (act1) {
-            if (!(ok = wait_p(1, (uint32_t)(i - 1)))) break;
-            gemm_pv(1, 1, slot_addr(nk - 1), i == 1);        // O1 += P1_{i-1} V_{i-1}
+            if (!(ok = gemm_pv(1, 1, slot_addr(nk - 1), i == 1, (uint32_t)(i - 1)))) break;  // O1 += P1_{i-1} V_{i-1}
             mma_commit(bar(C::bar_pv(1)));
           }
           mma_commit(bar(C::bar_empty((nk - 1) % C::NBUF)));  // V_{i-1} done
@@ -257,16 +258,13 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
             mma_commit(bar(C::bar_s(1)));
           }
           mma_commit(bar(C::bar_empty(nk % C::NBUF)));        // K_i done
-          if (!(ok = wait_full(nk + 1) && wait_p(0, (uint32_t)i))) break;
-          gemm_pv(0, 0, slot_addr(nk + 1), false);           // O0 += P0_i V_i
+          if (!(ok = wait_full(nk + 1) && gemm_pv(0, 0, slot_addr(nk + 1), false, (uint32_t)i))) break;  // O0 += P0_i V_i
           mma_commit(bar(C::bar_pv(0)));
         }
         if (ok) {
           const int nv = 2 * n_tiles - 1;
-          if (act1 && (ok = wait_p(1, (uint32_t)(n_tiles - 1)))) {
-            gemm_pv(1, 1, slot_addr(nv), n_tiles == 1);
+          if (act1 && (ok = gemm_pv(1, 1, slot_addr(nv), n_tiles == 1, (uint32_t)(n_tiles - 1))))
             mma_commit(bar(C::bar_pv(1)));
-          }
           if (ok) mma_commit(bar(C::bar_empty(nv % C::NBUF)));
         }
       } else {
@@ -286,8 +284,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
             mma_commit(bar(C::bar_empty(n % C::NBUF)));
             ++n;
           }
-          if (!(ok = wait_full(n) && wait_p(j & 1, (uint32_t)(j >> 1)))) break;
-          gemm_pv(0, j & 1, slot_addr(n), j == 0);
+          if (!(ok = wait_full(n) && gemm_pv(0, j & 1, slot_addr(n), j == 0, (uint32_t)(j >> 1)))) break;
           mma_commit(bar(C::bar_pv(0)));
           mma_commit(bar(C::bar_empty(n % C::NBUF)));
           ++n;
@@ -322,7 +319,8 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
         // one TMEM read of the whole 128-column S row
         float sv[BN];
         tmem_ld128(tS, sv);
-        if (__any_sync(0xffffffffu, cl < BN)) {  // diagonal or ragged tile: mask in place
+        const bool tile_masked = __any_sync(0xffffffffu, cl < BN);
+        if (tile_masked) {  // diagonal or ragged tile: mask in place
 #pragma unroll
           for (int e = 0; e < BN; ++e) sv[e] = (e < cl) ? sv[e] : -INFINITY;
         }
@@ -342,24 +340,8 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
           alpha = ex2_approx(m_use - m_new);
         }
         const float m_sub = (m_new == -INFINITY) ? 0.f : m_new;
-        // p = 2^(s*c2 - m): one packed FFMA per pair, ex2 per element, packed
-        // partial sums, bf16 pairs for the P.V operand (masked s = -inf -> p = 0)
-        const float2 c2v = make_float2(c2, c2);
-        const float2 nmv = make_float2(-m_sub, -m_sub);
-        float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-        uint32_t pk[BN / 2];
-#pragma unroll
-        for (int e = 0; e < BN / 2; ++e) {
-          const float2 x = ffma2(make_float2(sv[2 * e], sv[2 * e + 1]), c2v, nmv);
-          const float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-          if (e & 1) acc1 = fadd2(acc1, pr); else acc0 = fadd2(acc0, pr);
-          pk[e] = pack_bf16x2(pr.x, pr.y);
-        }
-        const float sum = (acc0.x + acc0.y) + (acc1.x + acc1.y);
-        // P lands on TMEM columns [0, 64) of this slot's S region (already read)
-        tmem_st64(tS, pk);
-        l = l * alpha + sum;
         if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+          // O must be rescaled before the first half of P is handed over.
           // Two slots: S_i(j) was issued behind O_i += P_i(j-1) V, so its
           // completion implies that P.V completed.  One slot: S(j) was issued
           // before that P.V, so wait for it here.
@@ -377,10 +359,53 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
             tmem_st32(tO + 32 * c, v);
           }
         }
+        // p = 2^(s*c2 - m): one packed FFMA per pair, ex2 per element, packed
+        // partial sums, bf16 pairs for the P.V operand (masked s = -inf -> p = 0).
+        // P is handed over in two halves (keys 0-63, then 64-127) so the P.V
+        // MMAs on the first half overlap the exponentials of the second.
+        const float2 c2v = make_float2(c2, c2);
+        const float2 nmv = make_float2(-m_sub, -m_sub);
+        float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+        // half 0: keys 0-63 from the registers; P lands on TMEM columns 0-31,
+        // whose S values were read above
+        {
+          uint32_t pk[BN / 4];
+#pragma unroll
+          for (int e = 0; e < BN / 4; ++e) {
+            const float2 x = ffma2(make_float2(sv[2 * e], sv[2 * e + 1]), c2v, nmv);
+            const float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            if (e & 1) acc1 = fadd2(acc1, pr); else acc0 = fadd2(acc0, pr);
+            pk[e] = pack_bf16x2(pr.x, pr.y);
+          }
+          tmem_st32u(tS, pk);
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(bar(C::bar_plo(sb)));
+        }
+        // half 1: keys 64-127, re-read from TMEM columns 64-127 (P only ever
+        // covers columns 0-63), so their registers need not stay live above
+        {
+          float sh[BN / 2];
+          tmem_ld64(tS + BN / 2, sh);
+          if (tile_masked) {
+#pragma unroll
+            for (int e = 0; e < BN / 2; ++e) sh[e] = (e + BN / 2 < cl) ? sh[e] : -INFINITY;
+          }
+          uint32_t pk[BN / 4];
+#pragma unroll
+          for (int e = 0; e < BN / 4; ++e) {
+            const float2 x = ffma2(make_float2(sh[2 * e], sh[2 * e + 1]), c2v, nmv);
+            const float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            if (e & 1) acc1 = fadd2(acc1, pr); else acc0 = fadd2(acc0, pr);
+            pk[e] = pack_bf16x2(pr.x, pr.y);
+          }
+          tmem_st32u(tS + BN / 4, pk);
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(bar(C::bar_phi(sb)));
+        }
+        l = l * alpha + ((acc0.x + acc0.y) + (acc1.x + acc1.y));
         m_use = m_new;
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(bar(C::bar_p(sb)));
       }
       // Wait for the last P.V.  A parity wait for completion k is only
       // unambiguous once completion k-1 has happened: with two slots the
