@@ -5,35 +5,38 @@
 // published lse = -inf carry weight 0 ("Anbeeld/beellama.cpp PR #149", review
 // of the combine kernel that merges per-block partials for parallel_blocks > 1).
 //
-// HBM-bound: a warp owns 128 consecutive columns of one row and each lane a
-// float4 of them, so a warp reads 512 contiguous bytes of every split's
-// partial row, eight splits in flight at a time.
+// Memory-bound: a block owns 128 consecutive columns of one row, each lane a
+// float4 of them, so a warp reads 512 contiguous bytes of a split's partial
+// row; the block's four warps take every fourth split.
 #include "kernels.h"
 #include "ptx.cuh"
 
 namespace gqa {
 namespace {
 
-__global__ void __launch_bounds__(128) merge_kernel(const MergeParams p) {
-  // one warp per (row, 128-column chunk); lane owns one float4 of the chunk
+__global__ void __launch_bounds__(128, 8) merge_kernel(const MergeParams p) {
+  // One block per (row, 128-column chunk).  Warp w accumulates splits
+  // w, w+4, w+8, ... (lane = one float4 of the chunk), so all of a row-chunk's
+  // partial loads are in flight at once; the four warps' sums are combined in
+  // shared memory.
+  __shared__ float4 part_acc[3][32];
+  __shared__ float part_w[3];
   const int f4_per_row = p.D / 4;
   const int chunks = (f4_per_row + 31) / 32;
-  const long long rows = (long long)p.B * p.Sq * p.Hq;
-  const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (gw >= rows * chunks) return;                  // whole warp leaves together
-  const long long row = gw / chunks;                // (b, s, h) in O order
-  const int f = (int)(gw - row * chunks) * 32 + lane;
+  const long long blk = blockIdx.x;
+  const long long row = blk / chunks;                // (b, s, h) in O order
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int f = (int)(blk - row * chunks) * 32 + lane;
   const bool active = f < f4_per_row;
   const int h = (int)(row % p.Hq);
   const int s = (int)((row / p.Hq) % p.Sq);
   const int b = (int)(row / ((long long)p.Hq * p.Sq));
   const size_t lse_row = ((size_t)b * p.Hq + h) * p.Sq + s;
   const size_t lse_stride = (size_t)p.B * p.Hq * p.Sq;
-  const size_t out_stride4 = (size_t)rows * p.D / 4;
+  const size_t out_stride4 = (size_t)p.B * p.Sq * p.Hq * p.D / 4;
   const float4* src = reinterpret_cast<const float4*>(p.part_out + (size_t)row * p.D) + (active ? f : 0);
 
-  // lane i holds lse of splits i, i+32, ...: max over all splits
+  // max of the split LSEs (every warp computes it; the loads are tiny)
   float M = -INFINITY;
   for (int sg = lane; sg < p.num_splits; sg += 32) M = fmaxf(M, __ldg(p.part_lse + sg * lse_stride + lse_row));
 #pragma unroll
@@ -41,38 +44,49 @@ __global__ void __launch_bounds__(128) merge_kernel(const MergeParams p) {
 
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float wsum = 0.f;
-  if (M != -INFINITY) {
-    for (int s0 = 0; s0 < p.num_splits; s0 += 32) {
-      const int sg_l = s0 + lane;
-      const float x = sg_l < p.num_splits ? __ldg(p.part_lse + sg_l * lse_stride + lse_row) : -INFINITY;
-      const float w_l = (x == -INFINITY) ? 0.f : expf(x - M);   // weight of split s0 + lane
-      const int n = min(32, p.num_splits - s0);
-      int i = 0;
-      // eight independent 16-byte loads in flight per lane
-      for (; i + 8 <= n; i += 8) {
-        float4 o[8];
+  // this warp's splits, eight loads in flight per batch; the loads do not
+  // wait for the maximum above (every published partial is finite)
+  for (int s0 = warp; s0 < p.num_splits; s0 += 32) {
+    float4 o[8];
+    float x[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) o[u] = __ldg(src + (size_t)(s0 + i + u) * out_stride4);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float w = __shfl_sync(0xffffffffu, w_l, i + u);
-          wsum += w;
-          acc.x = fmaf(w, o[u].x, acc.x);
-          acc.y = fmaf(w, o[u].y, acc.y);
-          acc.z = fmaf(w, o[u].z, acc.z);
-          acc.w = fmaf(w, o[u].w, acc.w);
-        }
-      }
-      for (; i < n; ++i) {
-        const float4 o = __ldg(src + (size_t)(s0 + i) * out_stride4);
-        const float w = __shfl_sync(0xffffffffu, w_l, i);
-        wsum += w;
-        acc.x = fmaf(w, o.x, acc.x);
-        acc.y = fmaf(w, o.y, acc.y);
-        acc.z = fmaf(w, o.z, acc.z);
-        acc.w = fmaf(w, o.w, acc.w);
+    for (int u = 0; u < 8; ++u) {
+      const int sg = s0 + 4 * u;
+      if (sg < p.num_splits) {
+        o[u] = __ldg(src + (size_t)sg * out_stride4);
+        x[u] = __ldg(p.part_lse + sg * lse_stride + lse_row);
+      } else {
+        x[u] = -INFINITY;
       }
     }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (x[u] != -INFINITY) {
+        const float w = ex2_approx((x[u] - M) * 1.4426950408889634f);
+        wsum += w;
+        acc.x = fmaf(w, o[u].x, acc.x);
+        acc.y = fmaf(w, o[u].y, acc.y);
+        acc.z = fmaf(w, o[u].z, acc.z);
+        acc.w = fmaf(w, o[u].w, acc.w);
+      }
+    }
+  }
+  if (warp > 0) {
+    part_acc[warp - 1][lane] = acc;
+    if (lane == 0) part_w[warp - 1] = wsum;
+  }
+  __syncthreads();
+  if (warp != 0) return;
+#pragma unroll
+  for (int i = 0; i < 3; ++i) {
+    const float4 a = part_acc[i][lane];
+    acc.x += a.x;
+    acc.y += a.y;
+    acc.z += a.z;
+    acc.w += a.w;
+    wsum += part_w[i];
+  }
+  if (M != -INFINITY) {
     const float inv = 1.f / wsum;
     acc.x *= inv;
     acc.y *= inv;
@@ -112,8 +126,7 @@ __global__ void watchdog_selftest_kernel(int* status, unsigned long long limit_n
 
 int launch_merge(const MergeParams& p, cudaStream_t stream) {
   const long long chunks = (p.D / 4 + 31) / 32;
-  const long long warps = (long long)p.B * p.Sq * p.Hq * chunks;
-  const long long blocks = (warps + 3) / 4;
+  const long long blocks = (long long)p.B * p.Sq * p.Hq * chunks;
   if (blocks <= 0 || blocks > 0x7fffffffLL) return (int)cudaErrorInvalidValue;
   merge_kernel<<<(unsigned)blocks, 128, 0, stream>>>(p);
   return (int)cudaGetLastError();

@@ -196,26 +196,32 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
       constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, false, false);
       constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, false, true);
       const bool act1 = (C::NSLOT == 2) && (hl0 + 1 < p.g);
-      auto slot_addr = [&](int n) -> uint32_t { return base + C::OFF_KV + (uint32_t)(n % C::NBUF) * C::TILE; };
       auto wait_full = [&](int n) -> bool {
         if (!mbar_wait(bar(C::bar_full(n % C::NBUF)), (uint32_t)(n / C::NBUF) & 1u, wd)) return false;
         tc_fence_after();
         return true;
       };
 
+      // Descriptors are built once; a K-step only advances the start-address
+      // field (bits 0-13, in 16-byte units), which never carries for these
+      // offsets since every tile lies below 256 KB of shared memory.
+      const uint64_t qdesc0 = sdesc_sw128(base + C::OFF_Q, 16, 1024);
+      const uint64_t kdesc0 = sdesc_sw128(base + C::OFF_KV, 16, 1024);
+      const uint64_t vdesc0 = sdesc_sw128(base + C::OFF_KV, BOX_BYTES, 1024);
       // S buffer sb = Q(qslot) K^T
-      auto gemm_s = [&](int sb, int qslot, uint32_t kbase) {
-        const uint32_t qbase = base + C::OFF_Q + (uint32_t)qslot * C::TILE;
+      auto gemm_s = [&](int sb, int qslot, int ring_n) {
+        const uint64_t qd = qdesc0 + (uint64_t)(((uint32_t)qslot * C::TILE) >> 4);
+        const uint64_t kd = kdesc0 + (uint64_t)(((uint32_t)(ring_n % C::NBUF) * C::TILE) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (uint32_t)(kk >> 2) * BOX_BYTES + (uint32_t)(kk & 3) * 32u;
-          mma_ss(tmem + C::TMEM_S + sb * 128, sdesc_sw128(qbase + off, 16, 1024),
-                 sdesc_sw128(kbase + off, 16, 1024), IDESC_QK, kk > 0 ? 1u : 0u);
+          const uint64_t off = (uint64_t)((((uint32_t)(kk >> 2) * BOX_BYTES) + (uint32_t)(kk & 3) * 32u) >> 4);
+          mma_ss(tmem + C::TMEM_S + sb * 128, qd + off, kd + off, IDESC_QK, kk > 0 ? 1u : 0u);
         }
       };
       // O(oslot) (+)= P(from S buffer pb) V, each half of P as soon as it is
       // in TMEM (phase: completion index of that buffer's P barriers)
-      auto gemm_pv = [&](int oslot, int pb, uint32_t vbase, bool first, uint32_t phase) -> bool {
+      auto gemm_pv = [&](int oslot, int pb, int ring_n, bool first, uint32_t phase) -> bool {
+        const uint64_t vd = vdesc0 + (uint64_t)(((uint32_t)(ring_n % C::NBUF) * C::TILE) >> 4);
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           if (!mbar_wait(bar(half == 0 ? C::bar_plo(pb) : C::bar_phi(pb)), phase & 1u, wd)) return false;
@@ -223,7 +229,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
 #pragma unroll
           for (int kk = half * (BN / 32); kk < (half + 1) * (BN / 32); ++kk)
             mma_ts(tmem + C::TMEM_O + oslot * D, tmem + C::TMEM_S + pb * 128 + kk * 8,
-                   sdesc_sw128(vbase + kk * 2048u, BOX_BYTES, 1024), IDESC_PV, (!first || kk > 0) ? 1u : 0u);
+                   vd + (uint64_t)((kk * 2048u) >> 4), IDESC_PV, (!first || kk > 0) ? 1u : 0u);
         }
         return true;
       };
@@ -233,37 +239,37 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
         // tile 0
         if (ok) ok = wait_full(0);
         if (ok) {
-          gemm_s(0, 0, slot_addr(0));
+          gemm_s(0, 0, 0);
           mma_commit(bar(C::bar_s(0)));
           if (act1) {
-            gemm_s(1, 1, slot_addr(0));
+            gemm_s(1, 1, 0);
             mma_commit(bar(C::bar_s(1)));
           }
           mma_commit(bar(C::bar_empty(0 % C::NBUF)));
-          ok = wait_full(1) && gemm_pv(0, 0, slot_addr(1), true, 0);
+          ok = wait_full(1) && gemm_pv(0, 0, 1, true, 0);
           if (ok) mma_commit(bar(C::bar_pv(0)));
         }
         for (int i = 1; ok && i < n_tiles; ++i) {
           const int nk = 2 * i;
           if (!(ok = wait_full(nk))) break;
-          gemm_s(0, 0, slot_addr(nk));                       // S0_i (behind O0 += P0_{i-1} V_{i-1})
+          gemm_s(0, 0, nk);                       // S0_i (behind O0 += P0_{i-1} V_{i-1})
           mma_commit(bar(C::bar_s(0)));
           if (act1) {
-            if (!(ok = gemm_pv(1, 1, slot_addr(nk - 1), i == 1, (uint32_t)(i - 1)))) break;  // O1 += P1_{i-1} V_{i-1}
+            if (!(ok = gemm_pv(1, 1, nk - 1, i == 1, (uint32_t)(i - 1)))) break;  // O1 += P1_{i-1} V_{i-1}
             mma_commit(bar(C::bar_pv(1)));
           }
           mma_commit(bar(C::bar_empty((nk - 1) % C::NBUF)));  // V_{i-1} done
           if (act1) {
-            gemm_s(1, 1, slot_addr(nk));                     // S1_i (behind the P1 read)
+            gemm_s(1, 1, nk);                     // S1_i (behind the P1 read)
             mma_commit(bar(C::bar_s(1)));
           }
           mma_commit(bar(C::bar_empty(nk % C::NBUF)));        // K_i done
-          if (!(ok = wait_full(nk + 1) && gemm_pv(0, 0, slot_addr(nk + 1), false, (uint32_t)i))) break;  // O0 += P0_i V_i
+          if (!(ok = wait_full(nk + 1) && gemm_pv(0, 0, nk + 1, false, (uint32_t)i))) break;  // O0 += P0_i V_i
           mma_commit(bar(C::bar_pv(0)));
         }
         if (ok) {
           const int nv = 2 * n_tiles - 1;
-          if (act1 && (ok = gemm_pv(1, 1, slot_addr(nv), n_tiles == 1, (uint32_t)(n_tiles - 1))))
+          if (act1 && (ok = gemm_pv(1, 1, nv, n_tiles == 1, (uint32_t)(n_tiles - 1))))
             mma_commit(bar(C::bar_pv(1)));
           if (ok) mma_commit(bar(C::bar_empty(nv % C::NBUF)));
         }
@@ -271,7 +277,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
         // one slot, S double buffered: S_0, then per tile S_{j+1} and O += P_j V_j
         int n = 0;
         if (ok && (ok = wait_full(n))) {
-          gemm_s(0, 0, slot_addr(n));
+          gemm_s(0, 0, n);
           mma_commit(bar(C::bar_s(0)));
           mma_commit(bar(C::bar_empty(n % C::NBUF)));
           ++n;
@@ -279,12 +285,12 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
         for (int j = 0; ok && j < n_tiles; ++j) {
           if (j + 1 < n_tiles) {
             if (!(ok = wait_full(n))) break;
-            gemm_s((j + 1) & 1, 0, slot_addr(n));            // behind the P.V that read this buffer
+            gemm_s((j + 1) & 1, 0, n);            // behind the P.V that read this buffer
             mma_commit(bar(C::bar_s((j + 1) & 1)));
             mma_commit(bar(C::bar_empty(n % C::NBUF)));
             ++n;
           }
-          if (!(ok = wait_full(n) && gemm_pv(0, j & 1, slot_addr(n), j == 0, (uint32_t)(j >> 1)))) break;
+          if (!(ok = wait_full(n) && gemm_pv(0, j & 1, n, j == 0, (uint32_t)(j >> 1)))) break;
           mma_commit(bar(C::bar_pv(0)));
           mma_commit(bar(C::bar_empty(n % C::NBUF)));
           ++n;
@@ -324,15 +330,16 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
 #pragma unroll
           for (int e = 0; e < BN; ++e) sv[e] = (e < cl) ? sv[e] : -INFINITY;
         }
-        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+        // row max: eight independent 3-input max chains, then a small tree
+        float mxc[8];
 #pragma unroll
-        for (int e = 0; e < BN; e += 8) {
-          mx0 = fmax3(mx0, sv[e], sv[e + 1]);
-          mx1 = fmax3(mx1, sv[e + 2], sv[e + 3]);
-          mx2 = fmax3(mx2, sv[e + 4], sv[e + 5]);
-          mx3 = fmax3(mx3, sv[e + 6], sv[e + 7]);
+        for (int c = 0; c < 8; ++c) mxc[c] = fmaxf(sv[2 * c], sv[2 * c + 1]);
+#pragma unroll
+        for (int e = 16; e < BN; e += 16) {
+#pragma unroll
+          for (int c = 0; c < 8; ++c) mxc[c] = fmax3(mxc[c], sv[e + 2 * c], sv[e + 2 * c + 1]);
         }
-        const float mx = fmax3(mx0, mx1, fmaxf(mx2, mx3));
+        const float mx = fmax3(fmax3(mxc[0], mxc[1], mxc[2]), fmax3(mxc[3], mxc[4], mxc[5]), fmaxf(mxc[6], mxc[7]));
         const float m_tile = mx * c2;
         float m_new = m_use, alpha = 1.f;
         if (m_tile > m_use + 8.f) {
