@@ -44,6 +44,18 @@ EncodeTiledFn encoder() {
   return g_encode;
 }
 
+int sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  static int cached[64] = {0};
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
 int* status_ptr() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
@@ -133,6 +145,8 @@ int attn_prefill(const void* q, const void* k, const void* v, void* out, float* 
 
   p.status = status_ptr();
   if (p.status == nullptr) return cuda_fail();
+  p.num_ctas = sm_count();
+  if (p.num_ctas <= 0) return cuda_fail();
   CUtensorMap tq, tk, tv;
   if (!make_map(&tq, q, D, Hq, Sq, B, 64, 1, 128, 1)) return cuda_fail();
   if (!make_map(&tk, k, D, Hkv, Skv, B, 64, 1, 128, 1)) return cuda_fail();

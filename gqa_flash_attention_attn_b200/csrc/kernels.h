@@ -14,6 +14,7 @@ struct PrefillParams {
   int g;              // Hq / Hkv
   int units_per_kvh;  // head slots per K/V head: ceil(g / NSLOT)
   int n_qt;           // ceil(Sq / 128)
+  int num_ctas;       // persistent grid size (SM count)
   float c2;           // scale * log2(e)
   unsigned long long timeout_ns;
 };

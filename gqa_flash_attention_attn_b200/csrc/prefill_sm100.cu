@@ -54,8 +54,9 @@ struct PrefillCfg {
   static constexpr uint32_t OFF_Q = 0;
   static constexpr uint32_t OFF_KV = NSLOT * TILE;
   static constexpr uint32_t OFF_BAR = OFF_KV + NBUF * TILE;
-  // q_full, kv_full[NBUF], kv_empty[NBUF], s_full[2], p_lo[2], p_hi[2], pv_done[2], drain
-  static constexpr int NBARS = 1 + 2 * NBUF + 8 + 1;
+  // q_full, q_empty, kv_full[NBUF], kv_empty[NBUF], s_full[2], p_lo[2], p_hi[2],
+  // pv_done[2], o_free[2], drain
+  static constexpr int NBARS = 2 + 2 * NBUF + 10 + 1;
   static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
   static constexpr uint32_t SMEM = OFF_MISC + 16 + 1024;  // + alignment slack
   // Two S buffers (one per slot, or a double buffer for one slot), P aliased
@@ -64,13 +65,15 @@ struct PrefillCfg {
   static constexpr uint32_t TMEM_O = 256;                 // O_i at TMEM_O + i*D
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int BAR_Q = 0;
-  __host__ __device__ static constexpr int bar_full(int b) { return 1 + b; }
-  __host__ __device__ static constexpr int bar_empty(int b) { return 1 + NBUF + b; }
-  __host__ __device__ static constexpr int bar_s(int i) { return 1 + 2 * NBUF + i; }
-  __host__ __device__ static constexpr int bar_plo(int i) { return 3 + 2 * NBUF + i; }
-  __host__ __device__ static constexpr int bar_phi(int i) { return 5 + 2 * NBUF + i; }
-  __host__ __device__ static constexpr int bar_pv(int i) { return 7 + 2 * NBUF + i; }
-  static constexpr int BAR_DRAIN = 9 + 2 * NBUF;
+  static constexpr int BAR_QE = 1;
+  __host__ __device__ static constexpr int bar_full(int b) { return 2 + b; }
+  __host__ __device__ static constexpr int bar_empty(int b) { return 2 + NBUF + b; }
+  __host__ __device__ static constexpr int bar_s(int i) { return 2 + 2 * NBUF + i; }
+  __host__ __device__ static constexpr int bar_plo(int i) { return 4 + 2 * NBUF + i; }
+  __host__ __device__ static constexpr int bar_phi(int i) { return 6 + 2 * NBUF + i; }
+  __host__ __device__ static constexpr int bar_pv(int i) { return 8 + 2 * NBUF + i; }
+  __host__ __device__ static constexpr int bar_ofree(int i) { return 10 + 2 * NBUF + i; }
+  static constexpr int BAR_DRAIN = 12 + 2 * NBUF;
   static_assert(256 + NSLOT * D <= 512, "TMEM budget");
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(D % 64 == 0, "head dim must be a multiple of 64");
@@ -101,6 +104,42 @@ __device__ __forceinline__ bool ring_item(int n, int n_tiles, int& tile) {
   return true;
 }
 
+// One unit of work: a 128-row query tile for up to NSLOT heads of one K/V group.
+struct Unit {
+  int b, kvh, hl0, s0, n_tiles;
+};
+
+// Unit u in longest-first order: q-tiles with the most visible keys first,
+// then batch, K/V head and head slot group (heads of a group adjacent, so
+// their K/V tiles are shared in L2).
+template <int NSLOT>
+__device__ __forceinline__ Unit unit_at(int u, const PrefillParams& p) {
+  const int upk = p.units_per_kvh;
+  const int units_per_qt = p.B * p.Hkv * upk;
+  const int qt_rev = u / units_per_qt;
+  int rem = u - qt_rev * units_per_qt;
+  Unit x;
+  x.b = rem / (p.Hkv * upk);
+  rem -= x.b * (p.Hkv * upk);
+  x.kvh = rem / upk;
+  x.hl0 = (rem - x.kvh * upk) * NSLOT;
+  const int qt = p.causal ? (p.n_qt - 1 - qt_rev) : qt_rev;
+  x.s0 = qt * BM;
+  const int kv_end = p.causal ? min(p.Skv, p.q_offset + min(x.s0 + BM, p.Sq)) : p.Skv;
+  x.n_tiles = (kv_end + BN - 1) / BN;
+  return x;
+}
+
+// The k-th unit of this CTA, or -1 when it has none left.  Units are dealt to
+// the persistent CTAs row by row in alternating direction (boustrophedon),
+// which with longest-first units balances the load like greedy LPT without a
+// shared counter.
+__device__ __forceinline__ int unit_index(int k, int total) {
+  const long long G = gridDim.x, c = blockIdx.x;
+  const long long u = (long long)k * G + ((k & 1) ? (G - 1 - c) : c);
+  return u < total ? (int)u : -1;
+}
+
 template <int D>
 __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -116,25 +155,11 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-
-  // ---- which unit: (q-tile, batch, K/V head, slot group), longest first ----
-  const int upk = p.units_per_kvh;
-  const int units_per_qt = p.B * p.Hkv * upk;
-  const int u = blockIdx.x;
-  const int qt_rev = u / units_per_qt;
-  int rem = u - qt_rev * units_per_qt;
-  const int b = rem / (p.Hkv * upk);
-  rem -= b * (p.Hkv * upk);
-  const int kvh = rem / upk;
-  const int grp = rem - kvh * upk;
-  const int qt = p.causal ? (p.n_qt - 1 - qt_rev) : qt_rev;
-  const int s0 = qt * BM;
-  const int hl0 = grp * C::NSLOT;  // local head of slot 0 inside the group
-  const int kv_end = p.causal ? min(p.Skv, p.q_offset + min(s0 + BM, p.Sq)) : p.Skv;
-  const int n_tiles = (kv_end + BN - 1) / BN;
+  const int total_units = p.n_qt * p.B * p.Hkv * p.units_per_kvh;
 
   if (threadIdx.x == 0) {
     mbar_init(bar(C::BAR_Q), 1);
+    mbar_init(bar(C::BAR_QE), 1);
     for (int i = 0; i < C::NBUF; ++i) {
       mbar_init(bar(C::bar_full(i)), 1);
       mbar_init(bar(C::bar_empty(i)), 1);
@@ -144,6 +169,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
       mbar_init(bar(C::bar_plo(i)), 128);
       mbar_init(bar(C::bar_phi(i)), 128);
       mbar_init(bar(C::bar_pv(i)), 1);
+      mbar_init(bar(C::bar_ofree(i)), 128);
     }
     mbar_init(bar(C::BAR_DRAIN), 1);
     *abort_flag = 0;
@@ -159,43 +185,52 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
   const uint32_t tmem = *tmem_slot;
   const Watchdog wd{abort_flag, p.status, p.timeout_ns};
 
-  int issued = 0;  // producer: K/V blocks issued
+  int issued = 0;    // producer: K/V ring items issued
+  int q_issued = 0;  // producer: Q tiles issued (one per unit)
 
   if (warp == C::WARP_PRODUCER) {
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      int nact = 0;
-      for (int i = 0; i < C::NSLOT; ++i) nact += (hl0 + i < p.g) ? 1 : 0;
-      mbar_arrive_expect_tx(bar(C::BAR_Q), (uint32_t)nact * C::TILE);
-      for (int i = 0; i < C::NSLOT; ++i) {
-        if (hl0 + i >= p.g) continue;
-        const int h = kvh * p.g + hl0 + i;
-        for (int kb = 0; kb < C::KB; ++kb)
-          tma_load_4d(base + C::OFF_Q + i * C::TILE + kb * BOX_BYTES, &tm_q, bar(C::BAR_Q), kb * 64, h,
-                      s0, b);
-      }
-      for (int n = 0; n < 2 * n_tiles; ++n) {
-        const int buf = n % C::NBUF;
-        const int use = n / C::NBUF;
-        if (use > 0 && !mbar_wait(bar(C::bar_empty(buf)), (uint32_t)(use - 1) & 1u, wd)) break;
-        int tile;
-        const bool is_v = ring_item<C::NSLOT>(n, n_tiles, tile);
-        const CUtensorMap* tm = is_v ? &tm_v : &tm_k;
-        const int key0 = tile * BN;
-        mbar_arrive_expect_tx(bar(C::bar_full(buf)), C::TILE);
-        for (int kb = 0; kb < C::KB; ++kb)
-          tma_load_4d(base + C::OFF_KV + buf * C::TILE + kb * BOX_BYTES, tm, bar(C::bar_full(buf)),
-                      kb * 64, kvh, key0, b);
-        issued = n + 1;
+      int n = 0;
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int u = unit_index(k, total_units);
+        if (u < 0) break;
+        const Unit x = unit_at<C::NSLOT>(u, p);
+        // the previous unit's last S MMA must be done reading Q
+        if (k > 0 && !mbar_wait(bar(C::BAR_QE), (uint32_t)(k - 1) & 1u, wd)) break;
+        int nact = 0;
+        for (int i = 0; i < C::NSLOT; ++i) nact += (x.hl0 + i < p.g) ? 1 : 0;
+        mbar_arrive_expect_tx(bar(C::BAR_Q), (uint32_t)nact * C::TILE);
+        for (int i = 0; i < C::NSLOT; ++i) {
+          if (x.hl0 + i >= p.g) continue;
+          const int h = x.kvh * p.g + x.hl0 + i;
+          for (int kb = 0; kb < C::KB; ++kb)
+            tma_load_4d(base + C::OFF_Q + i * C::TILE + kb * BOX_BYTES, &tm_q, bar(C::BAR_Q), kb * 64, h,
+                        x.s0, x.b);
+        }
+        q_issued = k + 1;
+        for (int m = 0; m < 2 * x.n_tiles; ++m, ++n) {
+          const int buf = n % C::NBUF;
+          const int use = n / C::NBUF;
+          if (use > 0 && !mbar_wait(bar(C::bar_empty(buf)), (uint32_t)(use - 1) & 1u, wd)) { ok = false; break; }
+          int tile;
+          const bool is_v = ring_item<C::NSLOT>(m, x.n_tiles, tile);
+          const CUtensorMap* tm = is_v ? &tm_v : &tm_k;
+          mbar_arrive_expect_tx(bar(C::bar_full(buf)), C::TILE);
+          for (int kb = 0; kb < C::KB; ++kb)
+            tma_load_4d(base + C::OFF_KV + buf * C::TILE + kb * BOX_BYTES, tm, bar(C::bar_full(buf)),
+                        kb * 64, x.kvh, tile * BN, x.b);
+          issued = n + 1;
+        }
       }
     }
   } else if (warp == C::WARP_MMA) {
     if (lane == 0) {
       constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, false, false);
       constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, false, true);
-      const bool act1 = (C::NSLOT == 2) && (hl0 + 1 < p.g);
       auto wait_full = [&](int n) -> bool {
         if (!mbar_wait(bar(C::bar_full(n % C::NBUF)), (uint32_t)(n / C::NBUF) & 1u, wd)) return false;
         tc_fence_after();
@@ -233,89 +268,135 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
         }
         return true;
       };
-      bool ok = mbar_wait(bar(C::BAR_Q), 0, wd);
-      tc_fence_after();
-      if (C::NSLOT == 2) {
-        // tile 0
-        if (ok) ok = wait_full(0);
-        if (ok) {
-          gemm_s(0, 0, 0);
-          mma_commit(bar(C::bar_s(0)));
-          if (act1) {
-            gemm_s(1, 1, 0);
-            mma_commit(bar(C::bar_s(1)));
-          }
-          mma_commit(bar(C::bar_empty(0 % C::NBUF)));
-          ok = wait_full(1) && gemm_pv(0, 0, 1, true, 0);
-          if (ok) mma_commit(bar(C::bar_pv(0)));
-        }
-        for (int i = 1; ok && i < n_tiles; ++i) {
-          const int nk = 2 * i;
-          if (!(ok = wait_full(nk))) break;
-          gemm_s(0, 0, nk);                       // S0_i (behind O0 += P0_{i-1} V_{i-1})
-          mma_commit(bar(C::bar_s(0)));
-          if (act1) {
-            if (!(ok = gemm_pv(1, 1, nk - 1, i == 1, (uint32_t)(i - 1)))) break;  // O1 += P1_{i-1} V_{i-1}
-            mma_commit(bar(C::bar_pv(1)));
-          }
-          mma_commit(bar(C::bar_empty((nk - 1) % C::NBUF)));  // V_{i-1} done
-          if (act1) {
-            gemm_s(1, 1, nk);                     // S1_i (behind the P1 read)
-            mma_commit(bar(C::bar_s(1)));
-          }
-          mma_commit(bar(C::bar_empty(nk % C::NBUF)));        // K_i done
-          if (!(ok = wait_full(nk + 1) && gemm_pv(0, 0, nk + 1, false, (uint32_t)i))) break;  // O0 += P0_i V_i
-          mma_commit(bar(C::bar_pv(0)));
-        }
-        if (ok) {
-          const int nv = 2 * n_tiles - 1;
-          if (act1 && (ok = gemm_pv(1, 1, nv, n_tiles == 1, (uint32_t)(n_tiles - 1))))
-            mma_commit(bar(C::bar_pv(1)));
-          if (ok) mma_commit(bar(C::bar_empty(nv % C::NBUF)));
-        }
-      } else {
-        // one slot, S double buffered: S_0, then per tile S_{j+1} and O += P_j V_j
-        int n = 0;
-        if (ok && (ok = wait_full(n))) {
+      auto wait_ofree = [&](int slot, int units_done) -> bool {
+        // the previous unit's epilogue on this slot must be done reading O
+        if (units_done == 0) return true;
+        if (!mbar_wait(bar(C::bar_ofree(slot)), (uint32_t)(units_done - 1) & 1u, wd)) return false;
+        tc_fence_after();
+        return true;
+      };
+      bool ok = true;
+      int n = 0;                       // ring items consumed
+      int T0 = 0, T1 = 0;              // tiles completed per slot (barrier phases)
+      int U0 = 0, U1 = 0;              // units completed per slot
+      for (int k = 0; ok; ++k) {
+        const int u = unit_index(k, total_units);
+        if (u < 0) break;
+        const Unit x = unit_at<C::NSLOT>(u, p);
+        const int nt = x.n_tiles;
+        const bool act1 = (C::NSLOT == 2) && (x.hl0 + 1 < p.g);
+        if (!(ok = mbar_wait(bar(C::BAR_Q), (uint32_t)k & 1u, wd))) break;
+        tc_fence_after();
+        if (C::NSLOT == 2) {
+          // tile 0
+          if (!(ok = wait_full(n))) break;
           gemm_s(0, 0, n);
           mma_commit(bar(C::bar_s(0)));
+          if (act1) {
+            gemm_s(1, 1, n);
+            mma_commit(bar(C::bar_s(1)));
+          }
+          if (nt == 1) mma_commit(bar(C::BAR_QE));            // last S of the unit
+          mma_commit(bar(C::bar_empty(n % C::NBUF)));
+          if (!(ok = wait_full(n + 1) && wait_ofree(0, U0) &&
+                     gemm_pv(0, 0, n + 1, true, (uint32_t)T0)))
+            break;
+          mma_commit(bar(C::bar_pv(0)));
+          for (int i = 1; i < nt; ++i) {
+            const int nk = n + 2 * i;
+            if (!(ok = wait_full(nk))) break;
+            gemm_s(0, 0, nk);                                 // S0_i (behind O0 += P0_{i-1} V_{i-1})
+            mma_commit(bar(C::bar_s(0)));
+            if (act1) {
+              if (!(ok = (i > 1 || wait_ofree(1, U1)) &&
+                         gemm_pv(1, 1, nk - 1, i == 1, (uint32_t)(T1 + i - 1))))
+                break;                                        // O1 += P1_{i-1} V_{i-1}
+              mma_commit(bar(C::bar_pv(1)));
+            }
+            mma_commit(bar(C::bar_empty((nk - 1) % C::NBUF)));  // V_{i-1} done
+            if (act1) {
+              gemm_s(1, 1, nk);                               // S1_i (behind the P1 read)
+              mma_commit(bar(C::bar_s(1)));
+            }
+            if (i == nt - 1) mma_commit(bar(C::BAR_QE));      // last S of the unit
+            mma_commit(bar(C::bar_empty(nk % C::NBUF)));      // K_i done
+            if (!(ok = wait_full(nk + 1) && gemm_pv(0, 0, nk + 1, false, (uint32_t)(T0 + i)))) break;
+            mma_commit(bar(C::bar_pv(0)));                    // O0 += P0_i V_i
+          }
+          if (!ok) break;
+          const int nv = n + 2 * nt - 1;
+          if (act1) {
+            if (!(ok = (nt > 1 || wait_ofree(1, U1)) &&
+                       gemm_pv(1, 1, nv, nt == 1, (uint32_t)(T1 + nt - 1))))
+              break;
+            mma_commit(bar(C::bar_pv(1)));
+          }
+          mma_commit(bar(C::bar_empty(nv % C::NBUF)));
+          T0 += nt;
+          ++U0;
+          if (act1) {
+            T1 += nt;
+            ++U1;
+          }
+        } else {
+          // one slot, S double buffered across tiles and units: buffer (T0 + j) % 2
+          if (!(ok = wait_full(n))) break;
+          gemm_s(T0 & 1, 0, n);
+          mma_commit(bar(C::bar_s(T0 & 1)));
+          if (nt == 1) mma_commit(bar(C::BAR_QE));
           mma_commit(bar(C::bar_empty(n % C::NBUF)));
           ++n;
-        }
-        for (int j = 0; ok && j < n_tiles; ++j) {
-          if (j + 1 < n_tiles) {
-            if (!(ok = wait_full(n))) break;
-            gemm_s((j + 1) & 1, 0, n);            // behind the P.V that read this buffer
-            mma_commit(bar(C::bar_s((j + 1) & 1)));
+          for (int j = 0; j < nt; ++j) {
+            const int G = T0 + j;
+            if (j + 1 < nt) {
+              if (!(ok = wait_full(n))) break;
+              gemm_s((G + 1) & 1, 0, n);                      // behind the P.V that read this buffer
+              mma_commit(bar(C::bar_s((G + 1) & 1)));
+              if (j + 2 == nt) mma_commit(bar(C::BAR_QE));    // last S of the unit
+              mma_commit(bar(C::bar_empty(n % C::NBUF)));
+              ++n;
+            }
+            if (!(ok = wait_full(n) && (j > 0 || wait_ofree(0, U0)) &&
+                       gemm_pv(0, G & 1, n, j == 0, (uint32_t)(G >> 1))))
+              break;
+            mma_commit(bar(C::bar_pv(0)));
             mma_commit(bar(C::bar_empty(n % C::NBUF)));
             ++n;
           }
-          if (!(ok = wait_full(n) && gemm_pv(0, j & 1, n, j == 0, (uint32_t)(j >> 1)))) break;
-          mma_commit(bar(C::bar_pv(0)));
-          mma_commit(bar(C::bar_empty(n % C::NBUF)));
-          ++n;
+          if (!ok) break;
+          T0 += nt;
+          ++U0;
+          continue;
         }
+        n += 2 * nt;
       }
     }
   } else {
     // ---- softmax warpgroups: warp w serves slot w/4, TMEM lanes 32*(w%4).. ----
     const int slot = warp >> 2;
     const int wq = warp & 3;
-    const int hl = hl0 + slot;
-    if (hl < p.g) {
-      const int h = kvh * p.g + hl;
-      const int r = wq * 32 + lane;
-      const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-      const uint32_t tO = tmem + lane_off + C::TMEM_O + slot * D;
-      const int s_row = s0 + r;
+    const int r = wq * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t tO = tmem + lane_off + C::TMEM_O + slot * D;
+    const float c2 = p.c2;
+    int T = 0;  // tiles this slot completed in earlier units (barrier phases)
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int u = unit_index(k, total_units);
+      if (u < 0) break;
+      const Unit x = unit_at<C::NSLOT>(u, p);
+      const int hl = x.hl0 + slot;
+      if (hl >= p.g) continue;  // slot unused in this unit (odd group size)
+      const int n_tiles = x.n_tiles;
+      const int h = x.kvh * p.g + hl;
+      const int s_row = x.s0 + r;
       const int vis_end = p.causal ? min(p.Skv, p.q_offset + s_row + 1) : p.Skv;
-      const float c2 = p.c2;
       float m_use = -INFINITY, l = 0.f;
-      bool ok = true;
       for (int j = 0; j < n_tiles; ++j) {
+        const int G = T + j;
         // S buffer and its phase: per slot, or alternating for one slot
-        const int sb = (C::NSLOT == 2) ? slot : (j & 1);
-        const uint32_t ph = (C::NSLOT == 2) ? ((uint32_t)j & 1u) : ((uint32_t)(j >> 1) & 1u);
+        const int sb = (C::NSLOT == 2) ? slot : (G & 1);
+        const uint32_t ph = (C::NSLOT == 2) ? ((uint32_t)G & 1u) : ((uint32_t)(G >> 1) & 1u);
         const uint32_t tS = tmem + lane_off + C::TMEM_S + sb * 128;
         // a give-up must be warp-uniform: TMEM loads/stores are warp-collective
         const bool got = mbar_wait(bar(C::bar_s(sb)), ph, wd);
@@ -353,7 +434,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
           // completion implies that P.V completed.  One slot: S(j) was issued
           // before that P.V, so wait for it here.
           if (C::NSLOT == 1) {
-            const bool got_pv = mbar_wait(bar(C::bar_pv(0)), (uint32_t)(j - 1) & 1u, wd);
+            const bool got_pv = mbar_wait(bar(C::bar_pv(0)), (uint32_t)(G - 1) & 1u, wd);
             if (__any_sync(0xffffffffu, !got_pv)) { ok = false; break; }
             tc_fence_after();
           }
@@ -420,13 +501,15 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
       // there completion n-2 is awaited first.
       bool got_o = ok;
       if (got_o && C::NSLOT == 1 && n_tiles >= 2)
-        got_o = mbar_wait(bar(C::bar_pv(0)), (uint32_t)(n_tiles - 2) & 1u, wd);
-      got_o = got_o && mbar_wait(bar(C::bar_pv(C::NSLOT == 2 ? slot : 0)), (uint32_t)(n_tiles - 1) & 1u, wd);
-      if (!__any_sync(0xffffffffu, !got_o)) {
+        got_o = mbar_wait(bar(C::bar_pv(0)), (uint32_t)(T + n_tiles - 2) & 1u, wd);
+      got_o = got_o && mbar_wait(bar(C::bar_pv(C::NSLOT == 2 ? slot : 0)), (uint32_t)(T + n_tiles - 1) & 1u, wd);
+      if (__any_sync(0xffffffffu, !got_o)) {
+        ok = false;
+      } else {
         tc_fence_after();
         const float inv_l = 1.f / l;
         const bool row_ok = s_row < p.Sq;
-        const size_t row_off = (((size_t)b * p.Sq + s_row) * p.Hq + h) * (size_t)D;
+        const size_t row_off = (((size_t)x.b * p.Sq + s_row) * p.Hq + h) * (size_t)D;
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           float v[32];
@@ -450,10 +533,14 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
           }
         }
         if (row_ok && p.lse != nullptr)
-          p.lse[((size_t)b * p.Hq + h) * p.Sq + s_row] = (m_use + log2f(l)) * LN2;
+          p.lse[((size_t)x.b * p.Hq + h) * p.Sq + s_row] = (m_use + log2f(l)) * LN2;
       }
+      // O of this slot may now be overwritten by the next unit's first P.V
       tc_fence_before();
+      mbar_arrive(bar(C::bar_ofree(slot)));
+      T += n_tiles;
     }
+    tc_fence_before();
   }
 
   __syncwarp();
@@ -461,7 +548,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
   if (*abort_flag) {
     // Nothing may still write this CTA's shared memory or TMEM when it exits.
     if (warp == C::WARP_PRODUCER && lane == 0) {
-      drain_wait(bar(C::BAR_Q), 0, p.timeout_ns);
+      if (q_issued > 0) drain_wait(bar(C::BAR_Q), (uint32_t)(q_issued - 1) & 1u, p.timeout_ns);
       for (int n = max(0, issued - C::NBUF); n < issued; ++n)
         drain_wait(bar(C::bar_full(n % C::NBUF)), (uint32_t)(n / C::NBUF) & 1u, p.timeout_ns);
     }
@@ -486,8 +573,9 @@ int launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv
                                        (int)C::SMEM);
   if (e != cudaSuccess) return (int)e;
   const long long units = (long long)p.n_qt * p.B * p.Hkv * p.units_per_kvh;
-  if (units <= 0 || units > 0x7fffffffLL) return (int)cudaErrorInvalidValue;
-  prefill_kernel<D><<<(unsigned)units, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, p);
+  if (units <= 0 || units > 0x7fffffffLL || p.num_ctas <= 0) return (int)cudaErrorInvalidValue;
+  const long long grid = units < p.num_ctas ? units : p.num_ctas;  // persistent: one CTA per SM
+  prefill_kernel<D><<<(unsigned)grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, p);
   return (int)cudaGetLastError();
 }
 
