@@ -190,11 +190,20 @@ def barrier(dist_on):
 
 
 def max_over_ranks(x, dist_on, device):
+    """The largest of every rank's x (a per-step time), same on all ranks."""
     if not dist_on:
         return x
     t = torch.tensor([x], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_throughput(work_per_rank, ms_local, dist_on, device):
+    """Whole-job rate for independent replicas: the work of all ranks divided
+    by the slowest rank's time.  Returns (rate per second, max ms)."""
+    world = torch.distributed.get_world_size() if dist_on else 1
+    ms = max_over_ranks(ms_local, dist_on, device)
+    return world * work_per_rank / (ms / 1e3), ms
 
 
 def time_steps(step, steps, warmup, flush, dist_on, device, inner=False):
@@ -320,13 +329,12 @@ def run_ours(args):
         w = WORKLOADS[name]
         step, nk, _ = make_runner(ga, w, device)
         ms, ms_first = time_steps(step, args.steps, args.warmup, flush, dist_on, device, inner=(nk == 2))
-        ms = max_over_ranks(ms, dist_on, device)
-        ms_first = max_over_ranks(ms_first, dist_on, device)
         status = ga.last_status()
         if status != ga.ATTN_OK:
             raise RuntimeError(f"{name}: device status {ga.status_string(status)}")
         unit, work = workload_metric(w)
-        value = world * work / (ms / 1e3)
+        value, ms = replica_throughput(work, ms, dist_on, device)
+        ms_first = max_over_ranks(ms_first, dist_on, device)
         if w.kind == "prefill":
             kind, achieved = "prefill", w.flops() / (ms_first / 1e3) / 1e12
             roof = {"bound": "tensor", "achieved": achieved, "peak": tf_burst, "unit": "TFLOP/s",
