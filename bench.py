@@ -61,7 +61,7 @@ class L2Flush:
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=None, help="time only this workload (profiling)")
@@ -125,7 +125,8 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "20"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.5)  # let the first samples arrive before the timed work starts
         except OSError:
             self.proc = None
 
@@ -229,42 +230,76 @@ def time_steps(step, steps, warmup, flush, dist_on, device, inner=False):
 
 
 def time_e2e(ga, w, steps, warmup, dist_on, device):
-    """Same workload through the public call with pinned host buffers: H2D of
-    q, k, v, the kernels, and D2H of out and lse inside every timed step."""
+    """Same workload through the public call with pinned host buffers: every
+    step copies its q, k, v host->device, runs the kernels and copies out and
+    lse device->host; all of it is inside the timed region.  Steps are
+    pipelined the way a streaming caller would run them: inputs double
+    buffered on the device, uploads on one stream, kernels on another,
+    downloads on a third, so step i's download overlaps step i+1's upload
+    (PCIe is full duplex) and the kernels overlap both."""
     from gqa_flash_attention_attn_b200.inputs import make_qkv
     q, k, v = make_qkv(w.B, w.Hq, w.Hkv, w.Sq, w.Skv, w.D, seed=0)
     hq, hk, hv = q.pin_memory(), k.pin_memory(), v.pin_memory()
     odt = torch.float32 if w.out_dtype == "f32" else torch.bfloat16
-    ho = torch.empty((w.B, w.Sq, w.Hq, w.D), dtype=odt).pin_memory()
-    hl = torch.empty((w.B, w.Hq, w.Sq), dtype=torch.float32).pin_memory()
-    dq, dk, dv = (torch.empty_like(t, device=device) for t in (q, k, v))
+    ho = [torch.empty((w.B, w.Sq, w.Hq, w.D), dtype=odt).pin_memory() for _ in range(2)]
+    hl = [torch.empty((w.B, w.Hq, w.Sq), dtype=torch.float32).pin_memory() for _ in range(2)]
+    dev_in = [[torch.empty_like(t, device=device) for t in (q, k, v)] for _ in range(2)]
+    dev_out = [torch.empty((w.B, w.Sq, w.Hq, w.D), dtype=odt, device=device) for _ in range(2)]
+    dev_lse = [torch.empty((w.B, w.Hq, w.Sq), dtype=torch.float32, device=device) for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    s_comp = torch.cuda.current_stream(device)
+    ev = lambda: torch.cuda.Event()
+    state = {"in_free": [None, None], "out_free": [None, None]}
 
-    def step():
-        dq.copy_(hq, non_blocking=True)
-        dk.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
+    def step(i):
+        b = i & 1
+        # upload into buffer b once the kernels of step i-2 stopped reading it
+        with torch.cuda.stream(s_in):
+            if state["in_free"][b] is not None:
+                s_in.wait_event(state["in_free"][b])
+            for dst, src in zip(dev_in[b], (hq, hk, hv)):
+                dst.copy_(src, non_blocking=True)
+            uploaded = ev()
+            uploaded.record(s_in)
+        s_comp.wait_event(uploaded)
+        if state["out_free"][b] is not None:
+            s_comp.wait_event(state["out_free"][b])      # step i-2's download of out[b] is done
+        dq, dk, dv = dev_in[b]
         if w.kind == "prefill":
-            o, l = ga.prefill(dq, dk, dv, causal=w.causal, q_offset=w.q_offset, scale=w.scale, out_dtype=odt)
+            ga.prefill(dq, dk, dv, causal=w.causal, q_offset=w.q_offset, scale=w.scale, out=dev_out[b],
+                       lse=dev_lse[b])
         else:
-            o, l = ga.decode(dq, dk, dv, w.num_splits, causal=w.causal, q_offset=w.q_offset, scale=w.scale,
-                             out_dtype=odt)
-        ho.copy_(o, non_blocking=True)
-        hl.copy_(l, non_blocking=True)
+            ga.decode(dq, dk, dv, w.num_splits, causal=w.causal, q_offset=w.q_offset, scale=w.scale,
+                      out=dev_out[b], lse=dev_lse[b])
+        computed = ev()
+        computed.record(s_comp)
+        state["in_free"][b] = computed
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(computed)
+            ho[b].copy_(dev_out[b], non_blocking=True)
+            hl[b].copy_(dev_lse[b], non_blocking=True)
+            downloaded = ev()
+            downloaded.record(s_out)
+        state["out_free"][b] = downloaded
 
-    for _ in range(warmup):
-        step()
+    for i in range(warmup):
+        step(i)
     torch.cuda.synchronize()
     barrier(dist_on)
-    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record()
-    for _ in range(steps):
-        step()
-    e.record()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(s_in)
+    s_comp.wait_event(start)
+    s_out.wait_event(start)
+    for i in range(steps):
+        step(warmup + i)
+    s_in.wait_stream(s_out)
+    s_in.wait_stream(s_comp)
+    end.record(s_in)
     torch.cuda.synchronize()
     barrier(dist_on)
-    ms = max_over_ranks(s.elapsed_time(e) / steps, dist_on, device)
+    ms = max_over_ranks(start.elapsed_time(end) / steps, dist_on, device)
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
-    d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+    d2h = ho[0].numel() * ho[0].element_size() + hl[0].numel() * hl[0].element_size()
     return ms, h2d, d2h
 
 
