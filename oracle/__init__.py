@@ -21,6 +21,9 @@ Functions and the passage each follows (all pinned by tests/test_oracle_pins.py)
                   publishes its (max, rowsum))
   merge           the LSE combine of split partials (same page, review of the
                   combine kernel for parallel_blocks > 1)
+  *_ex            the same with the optional logit terms of the FLASH_ATTN_EXT
+                  operator ("ggml-org/llama.cpp PR #28507", Crash 1: sinks,
+                  max_bias, logit_softcap) and a sliding window (see oracle.c)
 """
 from __future__ import annotations
 
@@ -80,6 +83,19 @@ def _bind(lib):
     lib.oracle_merge.restype = None
     lib.oracle_num_threads.argtypes = []
     lib.oracle_num_threads.restype = ctypes.c_int
+    ext = [ctypes.c_double, ctypes.c_double, _dp, _i64]
+    lib.oracle_attention_ex.argtypes = [_dp, _dp, _dp, _dp, _dp] + [_i64] * 7 + [ctypes.c_int, ctypes.c_double] + ext
+    lib.oracle_attention_ex.restype = None
+    lib.oracle_attention_rows_ex.argtypes = ([_dp, _dp, _dp, _lp, _i64, _dp, _dp] + [_i64] * 7 +
+                                             [ctypes.c_int, ctypes.c_double] + ext)
+    lib.oracle_attention_rows_ex.restype = None
+    lib.oracle_split_ex.argtypes = ([_dp, _dp, _dp, _dp, _dp] + [_i64] * 7 + [ctypes.c_int, ctypes.c_double, _i64] +
+                                    [ctypes.c_double, ctypes.c_double, _i64])
+    lib.oracle_split_ex.restype = None
+    lib.oracle_merge_ex.argtypes = [_dp, _dp, _dp, _dp] + [_i64] * 5 + [_dp]
+    lib.oracle_merge_ex.restype = None
+    lib.oracle_alibi_slope.argtypes = [_i64, _i64, ctypes.c_double]
+    lib.oracle_alibi_slope.restype = ctypes.c_double
     return lib
 
 
@@ -168,4 +184,72 @@ def merge(pout, plse, lib=None):
     out = np.zeros((B, Sq, Hq, D), dtype=np.float64)
     lse = np.zeros((B, Hq, Sq), dtype=np.float64)
     lib.oracle_merge(_ptr(pout), _ptr(plse), _ptr(out), _ptr(lse), B, Hq, Sq, D, S)
+    return out, lse
+
+
+def _sinks_arg(sinks):
+    if sinks is None:
+        return None, None
+    arr = _f64(sinks).reshape(-1)
+    return arr, _ptr(arr)
+
+
+def alibi_slope(h, Hq, max_bias, lib=None):
+    return (lib or load()).oracle_alibi_slope(int(h), int(Hq), float(max_bias))
+
+
+def attention_ex(q, k, v, *, scale, causal=True, q_offset=0, softcap=0.0, alibi_max_bias=0.0, sinks=None,
+                 window=0, lib=None):
+    """attention() with softcap, ALiBi, sink logits [Hq] and a sliding window."""
+    lib = lib or load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, Hkv, Sq, Skv, D = _dims(q, k)
+    sk, skp = _sinks_arg(sinks)
+    out = np.zeros((B, Sq, Hq, D), dtype=np.float64)
+    lse = np.zeros((B, Hq, Sq), dtype=np.float64)
+    lib.oracle_attention_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Skv, D,
+                            int(q_offset), int(bool(causal)), float(scale), float(softcap),
+                            float(alibi_max_bias), skp, int(window))
+    return out, lse
+
+
+def attention_rows_ex(q, k, v, rows, *, scale, causal=True, q_offset=0, softcap=0.0, alibi_max_bias=0.0,
+                      sinks=None, window=0, lib=None):
+    lib = lib or load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, Hkv, Sq, Skv, D = _dims(q, k)
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
+    n = rows.shape[0]
+    sk, skp = _sinks_arg(sinks)
+    out = np.zeros((n, D), dtype=np.float64)
+    lse = np.zeros((n,), dtype=np.float64)
+    lib.oracle_attention_rows_ex(_ptr(q), _ptr(k), _ptr(v), rows.ctypes.data_as(_lp), n, _ptr(out), _ptr(lse),
+                                 B, Hq, Hkv, Sq, Skv, D, int(q_offset), int(bool(causal)), float(scale),
+                                 float(softcap), float(alibi_max_bias), skp, int(window))
+    return out, lse
+
+
+def split_ex(q, k, v, num_splits, *, scale, causal=True, q_offset=0, softcap=0.0, alibi_max_bias=0.0,
+             window=0, lib=None):
+    """split() with softcap, ALiBi and a window (sinks belong to the merge)."""
+    lib = lib or load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, Hkv, Sq, Skv, D = _dims(q, k)
+    pout = np.zeros((num_splits, B, Sq, Hq, D), dtype=np.float64)
+    plse = np.zeros((num_splits, B, Hq, Sq), dtype=np.float64)
+    lib.oracle_split_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(pout), _ptr(plse), B, Hq, Hkv, Sq, Skv, D,
+                        int(q_offset), int(bool(causal)), float(scale), int(num_splits), float(softcap),
+                        float(alibi_max_bias), int(window))
+    return pout, plse
+
+
+def merge_ex(pout, plse, sinks=None, lib=None):
+    """merge() with optional sink logits [Hq] in the denominator."""
+    lib = lib or load()
+    pout, plse = _f64(pout), _f64(plse)
+    S, B, Sq, Hq, D = pout.shape
+    sk, skp = _sinks_arg(sinks)
+    out = np.zeros((B, Sq, Hq, D), dtype=np.float64)
+    lse = np.zeros((B, Hq, Sq), dtype=np.float64)
+    lib.oracle_merge_ex(_ptr(pout), _ptr(plse), _ptr(out), _ptr(lse), B, Hq, Sq, D, S, skp)
     return out, lse

@@ -39,6 +39,19 @@
  *     weight zero.
  *
  * Every input is a double array; callers widen bf16 values exactly.
+ *
+ * Optional terms of the logit (the *_ex functions; all off by default), from
+ * the parameters of the FLASH_ATTN_EXT operator ("ggml-org/llama.cpp PR
+ * #28507", Crash 1: sinks, max_bias, logit_softcap), read as follows:
+ *   softcap c > 0:      z_t = c * tanh(z_t / c)            (on the scaled logit)
+ *   ALiBi max_bias > 0: z_t += slope_h * (t - pos), slopes geometric per head:
+ *                       n2 = largest power of two <= Hq, m0 = 2^(-max_bias/n2),
+ *                       m1 = 2^(-max_bias/(2 n2)); slope_h = m0^(h+1) for
+ *                       h < n2, else m1^(2(h-n2)+1)
+ *   sink logit s_h:     one more term exp(s_h) in the softmax denominator
+ *                       (and in the LSE), with no value row
+ *   window w > 0:       key t is visible only if pos - w < t (with causal,
+ *                       each row sees its w most recent keys)
  */
 #include <math.h>
 #include <stdint.h>
@@ -57,42 +70,65 @@ static int64_t kv_index(int64_t b, int64_t t, int64_t kvh, int64_t Skv, int64_t 
     return ((b * Skv + t) * Hkv + kvh) * D;
 }
 
+typedef struct {
+    double softcap;         /* 0: off */
+    double alibi_max_bias;  /* 0: off */
+    const double* sinks;    /* NULL: off; else [Hq] sink logits */
+    int64_t window;         /* 0: off */
+} oracle_opts;
+
+/* ALiBi slope of head h out of Hq (see the header comment). */
+double oracle_alibi_slope(int64_t h, int64_t Hq, double max_bias) {
+    int64_t n2 = 1;
+    while (n2 * 2 <= Hq) n2 *= 2;
+    const double m0 = pow(2.0, -max_bias / (double)n2);
+    const double m1 = pow(2.0, -max_bias / 2.0 / (double)n2);
+    return h < n2 ? pow(m0, (double)(h + 1)) : pow(m1, (double)(2 * (h - n2) + 1));
+}
+
 /* One output row restricted to keys [t_lo, t_hi).  z is scratch of length
- * >= t_hi - t_lo.  Returns the LSE (or -inf when no key is visible, in which
- * case o_row is all zeros). */
+ * >= t_hi - t_lo.  Returns the LSE (or -inf when no key is visible and there
+ * is no sink, in which case o_row is all zeros).  opt may be NULL. */
 static double attend_row(const double* q, const double* k, const double* v,
                          int64_t b, int64_t h, int64_t s,
                          int64_t Hq, int64_t Hkv, int64_t Sq, int64_t Skv, int64_t D,
                          int64_t q_offset, int causal, double scale,
-                         int64_t t_lo, int64_t t_hi, double* z, double* o_row) {
+                         int64_t t_lo, int64_t t_hi, double* z, double* o_row,
+                         const oracle_opts* opt) {
     const int64_t g = Hq / Hkv;
     const int64_t kvh = h / g;
     const int64_t pos = q_offset + s;
     const double* qr = q + q_index(b, s, h, Sq, Hq, D);
+    const double softcap = opt ? opt->softcap : 0.0;
+    const double slope = (opt && opt->alibi_max_bias > 0.0) ? oracle_alibi_slope(h, Hq, opt->alibi_max_bias) : 0.0;
+    const int has_sink = opt && opt->sinks;
 
+    int64_t first = t_lo;                      /* inclusive lower bound of T */
+    if (opt && opt->window > 0 && pos - opt->window + 1 > first) first = pos - opt->window + 1;
     int64_t last = t_hi;                       /* exclusive upper bound of T */
     if (causal && pos + 1 < last) last = pos + 1;
     for (int64_t d = 0; d < D; ++d) o_row[d] = 0.0;
-    if (last <= t_lo) return -INFINITY;
+    if (last <= first && !has_sink) return -INFINITY;
 
-    /* pass 1: logits and their maximum */
-    double m = -INFINITY;
-    for (int64_t t = t_lo; t < last; ++t) {
+    /* pass 1: logits and their maximum (the sink logit takes part) */
+    double m = has_sink ? opt->sinks[h] : -INFINITY;
+    for (int64_t t = first; t < last; ++t) {
         const double* kr = k + kv_index(b, t, kvh, Skv, Hkv, D);
         double acc = 0.0;
         for (int64_t d = 0; d < D; ++d) acc += qr[d] * kr[d];
         const double zt = scale * acc;
-        z[t - t_lo] = zt;
-        if (zt > m) m = zt;
+        const double zc = softcap > 0.0 ? softcap * tanh(zt / softcap) : zt;
+        z[t - t_lo] = zc + slope * (double)(t - pos);
+        if (z[t - t_lo] > m) m = z[t - t_lo];
     }
     /* pass 2: exponentials, their sum, and the weighted sum of V rows */
-    double l = 0.0;
-    for (int64_t t = t_lo; t < last; ++t) {
+    double l = has_sink ? exp(opt->sinks[h] - m) : 0.0;
+    for (int64_t t = first; t < last; ++t) {
         const double p = exp(z[t - t_lo] - m);
         z[t - t_lo] = p;
         l += p;
     }
-    for (int64_t t = t_lo; t < last; ++t) {
+    for (int64_t t = first; t < last; ++t) {
         const double w = z[t - t_lo] / l;
         const double* vr = v + kv_index(b, t, kvh, Skv, Hkv, D);
         for (int64_t d = 0; d < D; ++d) o_row[d] += w * vr[d];
@@ -100,11 +136,11 @@ static double attend_row(const double* q, const double* k, const double* v,
     return m + log(l);
 }
 
-/* Full attention: out [B,Sq,Hq,D], lse [B,Hq,Sq]. */
-void oracle_attention(const double* q, const double* k, const double* v,
-                      double* out, double* lse,
-                      int64_t B, int64_t Hq, int64_t Hkv, int64_t Sq, int64_t Skv, int64_t D,
-                      int64_t q_offset, int causal, double scale) {
+/* Full attention: out [B,Sq,Hq,D], lse [B,Hq,Sq]; opt may be NULL. */
+static void attention_impl(const double* q, const double* k, const double* v,
+                           double* out, double* lse,
+                           int64_t B, int64_t Hq, int64_t Hkv, int64_t Sq, int64_t Skv, int64_t D,
+                           int64_t q_offset, int causal, double scale, const oracle_opts* opt) {
     const int64_t rows = B * Hq * Sq;
 #pragma omp parallel
     {
@@ -117,17 +153,17 @@ void oracle_attention(const double* q, const double* k, const double* v,
             double* o_row = out + q_index(b, s, h, Sq, Hq, D);
             lse[(b * Hq + h) * Sq + s] =
                 attend_row(q, k, v, b, h, s, Hq, Hkv, Sq, Skv, D, q_offset, causal, scale,
-                           0, Skv, z, o_row);
+                           0, Skv, z, o_row, opt);
         }
         free(z);
     }
 }
 
 /* Selected rows only: rows is n triples (b, h, s); out_rows [n, D]; lse_rows [n]. */
-void oracle_attention_rows(const double* q, const double* k, const double* v,
-                           const int64_t* rows, int64_t n, double* out_rows, double* lse_rows,
-                           int64_t B, int64_t Hq, int64_t Hkv, int64_t Sq, int64_t Skv, int64_t D,
-                           int64_t q_offset, int causal, double scale) {
+static void attention_rows_impl(const double* q, const double* k, const double* v,
+                                const int64_t* rows, int64_t n, double* out_rows, double* lse_rows,
+                                int64_t B, int64_t Hq, int64_t Hkv, int64_t Sq, int64_t Skv, int64_t D,
+                                int64_t q_offset, int causal, double scale, const oracle_opts* opt) {
     (void)B;
 #pragma omp parallel
     {
@@ -136,7 +172,7 @@ void oracle_attention_rows(const double* q, const double* k, const double* v,
         for (int64_t i = 0; i < n; ++i) {
             const int64_t b = rows[3 * i], h = rows[3 * i + 1], s = rows[3 * i + 2];
             lse_rows[i] = attend_row(q, k, v, b, h, s, Hq, Hkv, Sq, Skv, D, q_offset, causal,
-                                     scale, 0, Skv, z, out_rows + i * D);
+                                     scale, 0, Skv, z, out_rows + i * D, opt);
         }
         free(z);
     }
@@ -169,11 +205,12 @@ void oracle_probs(const double* q, const double* k,
 }
 
 /* Split-KV partials: pout [S,B,Sq,Hq,D] (each split normalised on its own keys),
- * plse [S,B,Hq,Sq]. */
-void oracle_split(const double* q, const double* k, const double* v,
-                  double* pout, double* plse,
-                  int64_t B, int64_t Hq, int64_t Hkv, int64_t Sq, int64_t Skv, int64_t D,
-                  int64_t q_offset, int causal, double scale, int64_t num_splits) {
+ * plse [S,B,Hq,Sq].  Sinks never enter a partial (the merge adds them once). */
+static void split_impl(const double* q, const double* k, const double* v,
+                       double* pout, double* plse,
+                       int64_t B, int64_t Hq, int64_t Hkv, int64_t Sq, int64_t Skv, int64_t D,
+                       int64_t q_offset, int causal, double scale, int64_t num_splits,
+                       const oracle_opts* opt) {
     const int64_t chunk = (Skv + num_splits - 1) / num_splits;
     const int64_t rows = B * Hq * Sq;
     const int64_t total = num_splits * rows;
@@ -193,7 +230,7 @@ void oracle_split(const double* q, const double* k, const double* v,
             double* o_row = pout + sigma * (B * Sq * Hq * D) + q_index(b, s, h, Sq, Hq, D);
             plse[sigma * rows + (b * Hq + h) * Sq + s] =
                 attend_row(q, k, v, b, h, s, Hq, Hkv, Sq, Skv, D, q_offset, causal, scale,
-                           lo, hi, z, o_row);
+                           lo, hi, z, o_row, opt);
         }
         free(z);
     }
@@ -203,9 +240,11 @@ void oracle_split(const double* q, const double* k, const double* v,
  *   M = max_sigma lse_sigma,  w_sigma = exp(lse_sigma - M),
  *   O = sum w_sigma O_sigma / sum w_sigma,  lse = M + ln(sum w_sigma).
  * A split with lse = -inf has weight 0; if every split is -inf the row is
- * O = 0, lse = -inf. */
-void oracle_merge(const double* pout, const double* plse, double* out, double* lse,
-                  int64_t B, int64_t Hq, int64_t Sq, int64_t D, int64_t num_splits) {
+ * O = 0, lse = -inf.  A sink logit s_h (sinks != NULL) joins M and adds
+ * exp(s_h - M) to the denominator only. */
+static void merge_impl(const double* pout, const double* plse, double* out, double* lse,
+                       int64_t B, int64_t Hq, int64_t Sq, int64_t D, int64_t num_splits,
+                       const double* sinks) {
     const int64_t rows = B * Hq * Sq;
 #pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < rows; ++r) {
@@ -213,14 +252,14 @@ void oracle_merge(const double* pout, const double* plse, double* out, double* l
         const int64_t h = (r / Sq) % Hq;
         const int64_t s = r % Sq;
         double* o_row = out + q_index(b, s, h, Sq, Hq, D);
-        double M = -INFINITY;
+        double M = sinks ? sinks[h] : -INFINITY;
         for (int64_t sg = 0; sg < num_splits; ++sg) {
             const double x = plse[sg * rows + r];
             if (x > M) M = x;
         }
         for (int64_t d = 0; d < D; ++d) o_row[d] = 0.0;
         if (M == -INFINITY) { lse[r] = -INFINITY; continue; }
-        double wsum = 0.0;
+        double wsum = sinks ? exp(sinks[h] - M) : 0.0;
         for (int64_t sg = 0; sg < num_splits; ++sg) {
             const double x = plse[sg * rows + r];
             if (x == -INFINITY) continue;
@@ -232,6 +271,73 @@ void oracle_merge(const double* pout, const double* plse, double* out, double* l
         for (int64_t d = 0; d < D; ++d) o_row[d] /= wsum;
         lse[r] = M + log(wsum);
     }
+}
+
+/* ---- public entry points: the plain definition, and the *_ex variants with
+ * the optional logit terms (softcap, ALiBi, sinks, window) ---- */
+void oracle_attention(const double* q, const double* k, const double* v, double* out, double* lse,
+                      int64_t B, int64_t Hq, int64_t Hkv, int64_t Sq, int64_t Skv, int64_t D,
+                      int64_t q_offset, int causal, double scale) {
+    attention_impl(q, k, v, out, lse, B, Hq, Hkv, Sq, Skv, D, q_offset, causal, scale, NULL);
+}
+
+void oracle_attention_rows(const double* q, const double* k, const double* v,
+                           const int64_t* rows, int64_t n, double* out_rows, double* lse_rows,
+                           int64_t B, int64_t Hq, int64_t Hkv, int64_t Sq, int64_t Skv, int64_t D,
+                           int64_t q_offset, int causal, double scale) {
+    attention_rows_impl(q, k, v, rows, n, out_rows, lse_rows, B, Hq, Hkv, Sq, Skv, D, q_offset, causal,
+                        scale, NULL);
+}
+
+void oracle_split(const double* q, const double* k, const double* v, double* pout, double* plse,
+                  int64_t B, int64_t Hq, int64_t Hkv, int64_t Sq, int64_t Skv, int64_t D,
+                  int64_t q_offset, int causal, double scale, int64_t num_splits) {
+    split_impl(q, k, v, pout, plse, B, Hq, Hkv, Sq, Skv, D, q_offset, causal, scale, num_splits, NULL);
+}
+
+void oracle_merge(const double* pout, const double* plse, double* out, double* lse,
+                  int64_t B, int64_t Hq, int64_t Sq, int64_t D, int64_t num_splits) {
+    merge_impl(pout, plse, out, lse, B, Hq, Sq, D, num_splits, NULL);
+}
+
+static oracle_opts make_opts(double softcap, double alibi_max_bias, const double* sinks, int64_t window) {
+    oracle_opts o;
+    o.softcap = softcap;
+    o.alibi_max_bias = alibi_max_bias;
+    o.sinks = sinks;
+    o.window = window;
+    return o;
+}
+
+void oracle_attention_ex(const double* q, const double* k, const double* v, double* out, double* lse,
+                         int64_t B, int64_t Hq, int64_t Hkv, int64_t Sq, int64_t Skv, int64_t D,
+                         int64_t q_offset, int causal, double scale,
+                         double softcap, double alibi_max_bias, const double* sinks, int64_t window) {
+    const oracle_opts o = make_opts(softcap, alibi_max_bias, sinks, window);
+    attention_impl(q, k, v, out, lse, B, Hq, Hkv, Sq, Skv, D, q_offset, causal, scale, &o);
+}
+
+void oracle_attention_rows_ex(const double* q, const double* k, const double* v,
+                              const int64_t* rows, int64_t n, double* out_rows, double* lse_rows,
+                              int64_t B, int64_t Hq, int64_t Hkv, int64_t Sq, int64_t Skv, int64_t D,
+                              int64_t q_offset, int causal, double scale,
+                              double softcap, double alibi_max_bias, const double* sinks, int64_t window) {
+    const oracle_opts o = make_opts(softcap, alibi_max_bias, sinks, window);
+    attention_rows_impl(q, k, v, rows, n, out_rows, lse_rows, B, Hq, Hkv, Sq, Skv, D, q_offset, causal,
+                        scale, &o);
+}
+
+void oracle_split_ex(const double* q, const double* k, const double* v, double* pout, double* plse,
+                     int64_t B, int64_t Hq, int64_t Hkv, int64_t Sq, int64_t Skv, int64_t D,
+                     int64_t q_offset, int causal, double scale, int64_t num_splits,
+                     double softcap, double alibi_max_bias, int64_t window) {
+    const oracle_opts o = make_opts(softcap, alibi_max_bias, NULL, window);
+    split_impl(q, k, v, pout, plse, B, Hq, Hkv, Sq, Skv, D, q_offset, causal, scale, num_splits, &o);
+}
+
+void oracle_merge_ex(const double* pout, const double* plse, double* out, double* lse,
+                     int64_t B, int64_t Hq, int64_t Sq, int64_t D, int64_t num_splits, const double* sinks) {
+    merge_impl(pout, plse, out, lse, B, Hq, Sq, D, num_splits, sinks);
 }
 
 int oracle_num_threads(void) {

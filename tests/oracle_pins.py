@@ -22,6 +22,10 @@ What pins what:
   shift             adding u to every key leaves O and shifts LSE by scale*q.u
   large logits      huge logits give the arg-max V row and LSE = max logit
   scale             (q, scale) and (2q, scale/2) give identical results
+  options           softcap, ALiBi, sinks and window: 40-digit decimal brute
+                    force, the standard ALiBi slope values, geometric-series and
+                    single-key closed forms, limits (huge cap, window 1 / Skv,
+                    sink -inf), split/merge identity, torch SDPA with a bias
 """
 from __future__ import annotations
 
@@ -296,6 +300,176 @@ def pin_scale_power_of_two(lib):
     assert not np.allclose(out, out3)
 
 
+# ---------------------------------------------------------------- options ----
+# Pins for the optional logit terms (softcap, ALiBi, sinks, sliding window).
+
+def _alibi_pow2(h, n, max_bias):
+    """ALiBi slope for a power-of-two head count n: 2^(-max_bias (h+1) / n)."""
+    return 2.0 ** (-max_bias * (h + 1) / n)
+
+
+def pin_ext_bruteforce_decimal(lib):
+    """Textbook softmax in 40-digit decimals with softcap, ALiBi, a sink and a window."""
+    decimal.getcontext().prec = 40
+    Dd = decimal.Decimal
+    rng = _rng(21)
+
+    def tanh(x):
+        e2 = (2 * x).exp()
+        return (e2 - 1) / (e2 + 1)
+
+    for (B, Hq, Hkv, Sq, Skv, D, q_offset, causal, cap, mb, window, use_sink) in [
+        (1, 4, 2, 3, 6, 2, 3, True, 1.5, 8.0, 0, True),
+        (1, 2, 1, 4, 5, 3, 1, True, 0.0, 4.0, 2, False),
+        (2, 2, 2, 2, 4, 2, 0, False, 0.75, 0.0, 0, True),
+        (1, 4, 1, 3, 7, 2, 4, True, 0.0, 0.0, 3, True),
+    ]:
+        q = rng.integers(-2, 3, size=(B, Sq, Hq, D)).astype(np.float64)
+        k = rng.integers(-2, 3, size=(B, Skv, Hkv, D)).astype(np.float64)
+        v = rng.integers(-3, 4, size=(B, Skv, Hkv, D)).astype(np.float64)
+        sinks = rng.integers(-2, 3, size=(Hq,)).astype(np.float64) if use_sink else None
+        scale = 0.5
+        out, lse = oracle.attention_ex(q, k, v, scale=scale, causal=causal, q_offset=q_offset, softcap=cap,
+                                       alibi_max_bias=mb, sinks=sinks, window=window, lib=lib)
+        g = Hq // Hkv
+        for b in range(B):
+            for h in range(Hq):
+                slope = Dd(_alibi_pow2(h, Hq, mb)) if mb > 0 else Dd(0)
+                for s in range(Sq):
+                    pos = q_offset + s
+                    ts = [t for t in range(Skv) if ((not causal) or t <= pos) and (window == 0 or t > pos - window)]
+                    ex = []
+                    for t in ts:
+                        z = Dd(scale) * sum(Dd(int(q[b, s, h, d])) * Dd(int(k[b, t, h // g, d])) for d in range(D))
+                        if cap > 0:
+                            z = Dd(cap) * tanh(z / Dd(cap))
+                        z = z + slope * (t - pos)
+                        ex.append(z.exp())
+                    den = sum(ex) + (Dd(int(sinks[h])).exp() if use_sink else Dd(0))
+                    for d in range(D):
+                        num = sum(e * Dd(int(v[b, t, h // g, d])) for e, t in zip(ex, ts))
+                        assert abs(float(num / den) - out[b, s, h, d]) < 1e-13, (b, h, s, d)
+                    assert abs(float(den.ln()) - lse[b, h, s]) < 1e-13, (b, h, s)
+
+
+def pin_alibi_slopes(lib):
+    """Geometric ALiBi slopes: 2^-1..2^-8 for 8 heads at max_bias 8; for 12 heads
+    the first 8 as for 8 heads, then the odd powers of 2^-1/2."""
+    for h in range(8):
+        assert oracle.alibi_slope(h, 8, 8.0, lib=lib) == 2.0 ** -(h + 1)
+    want12 = [2.0 ** -(h + 1) for h in range(8)] + [2.0 ** -(0.5 + j) for j in range(4)]
+    for h in range(12):
+        assert abs(oracle.alibi_slope(h, 12, 8.0, lib=lib) - want12[h]) < 1e-15
+
+
+def pin_alibi_geometric_closed_form(lib):
+    """Q = 0: the logits are slope*(t - pos), a geometric series in closed form."""
+    rng = _rng(22)
+    B, Hq, Hkv, Sq, Skv, D = 1, 4, 1, 5, 9, 4
+    q = np.zeros((B, Sq, Hq, D))
+    k, v = _normal(rng, (B, Skv, Hkv, D)), _normal(rng, (B, Skv, Hkv, D))
+    q_offset = 3
+    out, lse = oracle.attention_ex(q, k, v, scale=0.3, causal=True, q_offset=q_offset, alibi_max_bias=8.0, lib=lib)
+    for h in range(Hq):
+        r = math.exp(-_alibi_pow2(h, Hq, 8.0))
+        for s in range(Sq):
+            pos = q_offset + s
+            n = min(Skv, pos + 1)
+            w = np.array([r ** (pos - t) for t in range(n)])
+            np.testing.assert_allclose(out[0, s, h], (w[:, None] * v[0, :n, 0]).sum(0) / w.sum(), rtol=0, atol=1e-13)
+            assert abs(lse[0, h, s] - math.log((1 - r ** n) / (1 - r))) < 1e-13
+
+
+def pin_sink_closed_form(lib):
+    """A row that sees one key z with a sink s: O = V e^z/(e^z + e^s), LSE = log(e^z + e^s);
+    a sink of -inf changes nothing."""
+    rng = _rng(23)
+    B, Hq, Hkv, Sq, Skv, D = 1, 4, 2, 3, 6, 8
+    q, k, v = _normal(rng, (B, Sq, Hq, D)), _normal(rng, (B, Skv, Hkv, D)), _normal(rng, (B, Skv, Hkv, D))
+    sinks = np.array([0.5, -1.0, 2.0, 0.0])
+    out, lse = oracle.attention_ex(q, k, v, scale=0.25, causal=True, sinks=sinks, lib=lib)
+    for h in range(Hq):
+        kvh = h // 2
+        z = 0.25 * float(np.dot(q[0, 0, h], k[0, 0, kvh]))
+        w = math.exp(z) / (math.exp(z) + math.exp(sinks[h]))
+        np.testing.assert_allclose(out[0, 0, h], w * v[0, 0, kvh], rtol=0, atol=1e-14)
+        assert abs(lse[0, h, 0] - math.log(math.exp(z) + math.exp(sinks[h]))) < 1e-13
+    o0, l0 = oracle.attention(q, k, v, scale=0.25, causal=True, lib=lib)
+    o1, l1 = oracle.attention_ex(q, k, v, scale=0.25, causal=True, sinks=np.full(Hq, -np.inf), lib=lib)
+    assert np.array_equal(o0, o1) and np.array_equal(l0, l1)
+
+
+def pin_softcap_limits(lib):
+    """A huge cap changes nothing; a small cap bounds every logit by +-cap."""
+    rng = _rng(24)
+    B, Hq, Hkv, Sq, Skv, D = 1, 2, 1, 4, 10, 8
+    q, k, v = _normal(rng, (B, Sq, Hq, D)), _normal(rng, (B, Skv, Hkv, D)), _normal(rng, (B, Skv, Hkv, D))
+    o0, l0 = oracle.attention(q, k, v, scale=0.5, causal=False, lib=lib)
+    o1, l1 = oracle.attention_ex(q, k, v, scale=0.5, causal=False, softcap=1e9, lib=lib)
+    np.testing.assert_allclose(o1, o0, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(l1, l0, rtol=0, atol=1e-12)
+    cap = 0.25
+    o2, l2 = oracle.attention_ex(100.0 * q, k, v, scale=0.5, causal=False, softcap=cap, lib=lib)
+    assert np.all(l2 <= cap + math.log(Skv) + 1e-12) and np.all(l2 >= -cap + math.log(Skv) - 1e-12)
+
+
+def pin_window_limits(lib):
+    """Window 1: each row sees only its own position; a window of Skv is plain causal."""
+    rng = _rng(25)
+    B, Hq, Hkv, Sq, Skv, D = 1, 4, 2, 6, 9, 8
+    q, k, v = _normal(rng, (B, Sq, Hq, D)), _normal(rng, (B, Skv, Hkv, D)), _normal(rng, (B, Skv, Hkv, D))
+    q_offset = 3
+    out, lse = oracle.attention_ex(q, k, v, scale=0.3, causal=True, q_offset=q_offset, window=1, lib=lib)
+    for s in range(Sq):
+        pos = q_offset + s
+        for h in range(Hq):
+            kvh = h // 2
+            assert np.array_equal(out[0, s, h], v[0, pos, kvh])
+            assert abs(lse[0, h, s] - 0.3 * float(np.dot(q[0, s, h], k[0, pos, kvh]))) < 1e-12
+    o0, l0 = oracle.attention(q, k, v, scale=0.3, causal=True, q_offset=q_offset, lib=lib)
+    o1, l1 = oracle.attention_ex(q, k, v, scale=0.3, causal=True, q_offset=q_offset, window=Skv, lib=lib)
+    assert np.array_equal(o0, o1) and np.array_equal(l0, l1)
+
+
+def pin_split_merge_ex(lib):
+    """Merging split partials (sinks added once, by the merge) reproduces the unsplit result."""
+    rng = _rng(26)
+    B, Hq, Hkv, Sq, Skv, D = 1, 4, 2, 3, 29, 8
+    q, k, v = _normal(rng, (B, Sq, Hq, D)), _normal(rng, (B, Skv, Hkv, D)), _normal(rng, (B, Skv, Hkv, D))
+    sinks = np.array([0.3, -0.7, 1.1, 0.0])
+    kw = dict(scale=0.3, causal=True, q_offset=Skv - Sq, softcap=2.0, alibi_max_bias=4.0, window=11)
+    out, lse = oracle.attention_ex(q, k, v, sinks=sinks, lib=lib, **kw)
+    for S in (1, 3, 7):
+        po, pl = oracle.split_ex(q, k, v, S, lib=lib, **kw)
+        mo, ml = oracle.merge_ex(po, pl, sinks=sinks, lib=lib)
+        np.testing.assert_allclose(mo, out, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(ml, lse, rtol=0, atol=1e-12)
+
+
+def pin_torch_sdpa_bias(lib):
+    """torch's float64 SDPA with an additive ALiBi + window bias (masked keys at -inf)."""
+    rng = _rng(27)
+    B, Hq, Hkv, Sq, Skv, D = 1, 8, 2, 5, 13, 16
+    q, k, v = _normal(rng, (B, Sq, Hq, D)), _normal(rng, (B, Skv, Hkv, D)), _normal(rng, (B, Skv, Hkv, D))
+    q_offset, window, mb = 8, 6, 8.0
+    out, lse = oracle.attention_ex(q, k, v, scale=0.2, causal=True, q_offset=q_offset, alibi_max_bias=mb,
+                                   window=window, lib=lib)
+    g = Hq // Hkv
+    tq = torch.from_numpy(q).permute(0, 2, 1, 3)
+    tk = torch.from_numpy(k).permute(0, 2, 1, 3).repeat_interleave(g, dim=1)
+    tv = torch.from_numpy(v).permute(0, 2, 1, 3).repeat_interleave(g, dim=1)
+    pos = torch.arange(Sq, dtype=torch.float64).view(-1, 1) + q_offset
+    t = torch.arange(Skv, dtype=torch.float64).view(1, -1)
+    slopes = torch.tensor([_alibi_pow2(h, Hq, mb) for h in range(Hq)], dtype=torch.float64).view(1, -1, 1, 1)
+    bias = slopes * (t - pos)
+    visible = (t <= pos) & (t > pos - window)
+    bias = bias.masked_fill(~visible, float("-inf"))
+    ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=bias, scale=0.2)
+    np.testing.assert_allclose(out, ref.permute(0, 2, 1, 3).numpy(), rtol=0, atol=1e-12)
+    logits = (tq @ tk.transpose(-1, -2)) * 0.2 + bias
+    np.testing.assert_allclose(lse, torch.logsumexp(logits, dim=-1).numpy(), rtol=0, atol=1e-12)
+
+
 ALL_PINS = [
     pin_bruteforce_decimal,
     pin_golden_three_keys,
@@ -310,4 +484,12 @@ ALL_PINS = [
     pin_shift_invariance,
     pin_large_logits,
     pin_scale_power_of_two,
+    pin_ext_bruteforce_decimal,
+    pin_alibi_slopes,
+    pin_alibi_geometric_closed_form,
+    pin_sink_closed_form,
+    pin_softcap_limits,
+    pin_window_limits,
+    pin_split_merge_ex,
+    pin_torch_sdpa_bias,
 ]

@@ -32,6 +32,13 @@ MUTANTS = [
     ("merge_lse_no_max", "lse[r] = M + log(wsum);", "lse[r] = log(wsum);"),
     ("split_chunk_floor", "const int64_t chunk = (Skv + num_splits - 1) / num_splits;",
      "const int64_t chunk = Skv / num_splits;"),
+    ("alibi_sign", "z[t - t_lo] = zc + slope * (double)(t - pos);", "z[t - t_lo] = zc - slope * (double)(t - pos);"),
+    ("alibi_slope_exponent", "pow(m0, (double)(h + 1))", "pow(m0, (double)h)"),
+    ("softcap_ignored", "softcap * tanh(zt / softcap) : zt;", "zt : zt;"),
+    ("sink_not_in_denominator", "double l = has_sink ? exp(opt->sinks[h] - m) : 0.0;", "double l = 0.0;"),
+    ("window_off_by_one", "if (opt && opt->window > 0 && pos - opt->window + 1 > first) first = pos - opt->window + 1;",
+     "if (opt && opt->window > 0 && pos - opt->window > first) first = pos - opt->window;"),
+    ("merge_sink_dropped", "double wsum = sinks ? exp(sinks[h] - M) : 0.0;", "double wsum = 0.0;"),
 ]
 
 
