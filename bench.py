@@ -164,24 +164,27 @@ def make_runner(ga, w, device):
     """Device-resident inputs/outputs and a closure that launches one step.
     Returns (step_fn, n_kernels_per_step, events_split) where the closure
     records optional inner events between the split and the merge."""
-    from gqa_flash_attention_attn_b200.inputs import make_qkv
+    from gqa_flash_attention_attn_b200.inputs import make_qkv, make_sinks
     q, k, v = make_qkv(w.B, w.Hq, w.Hkv, w.Sq, w.Skv, w.D, seed=0, device=device)
     odt = torch.float32 if w.out_dtype == "f32" else torch.bfloat16
     out = torch.empty((w.B, w.Sq, w.Hq, w.D), dtype=odt, device=device)
     lse = torch.empty((w.B, w.Hq, w.Sq), dtype=torch.float32, device=device)
+    sinks = make_sinks(w.Hq, seed=0).to(device) if w.sinks else None
+    terms = dict(softcap=w.softcap, alibi_max_bias=w.alibi_max_bias, window=w.window)
     if w.kind == "prefill":
         def step(mid=None):
-            ga.prefill(q, k, v, causal=w.causal, q_offset=w.q_offset, scale=w.scale, out=out, lse=lse)
+            ga.prefill(q, k, v, causal=w.causal, q_offset=w.q_offset, scale=w.scale, out=out, lse=lse,
+                       sinks=sinks, **terms)
         return step, 1, (q, k, v, out, lse)
     po = torch.empty((w.num_splits, w.B, w.Sq, w.Hq, w.D), dtype=torch.float32, device=device)
     pl = torch.empty((w.num_splits, w.B, w.Hq, w.Sq), dtype=torch.float32, device=device)
 
     def step(mid=None):
         ga.decode_split(q, k, v, w.num_splits, causal=w.causal, q_offset=w.q_offset, scale=w.scale,
-                        partial_out=po, partial_lse=pl)
+                        partial_out=po, partial_lse=pl, **terms)
         if mid is not None:
             mid.record()
-        ga.merge(po, pl, out=out, lse=lse)
+        ga.merge(po, pl, out=out, lse=lse, sinks=sinks)
     return step, 2, (q, k, v, out, lse)
 
 

@@ -24,6 +24,7 @@ __all__ = [
     "merge", "decode", "decode_workspace_bytes", "last_status", "status_string",
     "watchdog_selftest", "version", "ATTN_OK", "ATTN_ERR_INVALID_ARG", "ATTN_ERR_UNSUPPORTED",
     "ATTN_ERR_ALIGNMENT", "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT", "ATTN_ERR_TOO_LARGE", "decode_noalloc",
+    "AttnOptions",
 ]
 
 ATTN_OK = 0
@@ -53,6 +54,9 @@ _SIGNATURES = {
     "attn_watchdog_selftest": (_i, [ctypes.c_ulonglong, _vp]),
     "attn_version": (_i, []),
     "attn_decode_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp] + [_i] * 8 + [_f, _i, _i, _vp]),
+    "attn_prefill_ex": (_i, [_vp, _vp, _vp, _vp, _vp] + [_i] * 8 + [_f, _i, _vp, _vp]),
+    "attn_decode_split_ex": (_i, [_vp, _vp, _vp, _vp, _vp] + [_i] * 8 + [_f, _i, _vp, _vp]),
+    "attn_merge_ex": (_i, [_vp, _vp, _vp, _vp] + [_i] * 6 + [_vp, _vp]),
 }
 
 
@@ -130,9 +134,33 @@ def _need(t, name, dtype, ndim):
 _OUT_CODES = {torch.bfloat16: 0, torch.float32: 1}
 
 
+class AttnOptions(ctypes.Structure):
+    """The C ``attn_options`` struct: optional logit terms (zero / NULL = off)."""
+    _fields_ = [("softcap", ctypes.c_float), ("alibi_max_bias", ctypes.c_float),
+                ("sinks", ctypes.c_void_p), ("window", ctypes.c_int)]
+
+
+def _options(softcap, alibi_max_bias, sinks, window, Hq):
+    """An AttnOptions for the given terms, or None when every term is off."""
+    if not softcap and not alibi_max_bias and sinks is None and not window:
+        return None
+    if sinks is not None:
+        _need(sinks, "sinks", torch.float32, 1)
+        if sinks.shape[0] != Hq:
+            raise ValueError(f"sinks must have Hq = {Hq} entries")
+    return AttnOptions(float(softcap), float(alibi_max_bias),
+                       None if sinks is None else sinks.data_ptr(), int(window))
+
+
 def prefill(q, k, v, *, causal=True, q_offset=0, scale=None, out_dtype=torch.bfloat16,
-            out=None, lse=None, return_lse=True, stream=None):
-    """O = softmax(scale * Q K^T + causal mask) V and its LSE, in one launch."""
+            out=None, lse=None, return_lse=True, stream=None, softcap=0.0, alibi_max_bias=0.0,
+            sinks=None, window=0):
+    """O = softmax(scale * Q K^T + causal mask) V and its LSE, in one launch.
+
+    Optional logit terms (off by default): softcap (z = c tanh(z / c)),
+    alibi_max_bias (per-head geometric slope times (t - pos)), sinks (fp32 [Hq]
+    logits that join only the softmax denominator) and window (key t visible
+    only when pos - window < t; needs causal and q_offset + Sq <= Skv)."""
     _need(q, "q", torch.bfloat16, 4)
     _need(k, "k", torch.bfloat16, 4)
     _need(v, "v", torch.bfloat16, 4)
@@ -150,10 +178,13 @@ def prefill(q, k, v, *, causal=True, q_offset=0, scale=None, out_dtype=torch.bfl
         raise ValueError("out must be bf16 or fp32")
     if lse is None and return_lse:
         lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
-    st = library().attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Skv, D,
-                                int(q_offset), int(bool(causal)), float(scale), _OUT_CODES[out.dtype],
-                                _stream_ptr(stream))
-    _check("attn_prefill", st)
+    opt = _options(softcap, alibi_max_bias, sinks, window, Hq)
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Skv, D, int(q_offset),
+            int(bool(causal)), float(scale), _OUT_CODES[out.dtype])
+    if opt is None:
+        _check("attn_prefill", library().attn_prefill(*args, _stream_ptr(stream)))
+    else:
+        _check("attn_prefill_ex", library().attn_prefill_ex(*args, ctypes.byref(opt), _stream_ptr(stream)))
     return out, lse
 
 
@@ -162,8 +193,11 @@ def decode_workspace_bytes(B, Hq, Sq, D, num_splits) -> int:
 
 
 def decode_split(q, k, v, num_splits, *, causal=True, q_offset=0, scale=None,
-                 partial_out=None, partial_lse=None, stream=None):
-    """Per-split normalised partial outputs [S,B,Sq,Hq,D] and LSEs [S,B,Hq,Sq]."""
+                 partial_out=None, partial_lse=None, stream=None, softcap=0.0, alibi_max_bias=0.0,
+                 window=0):
+    """Per-split normalised partial outputs [S,B,Sq,Hq,D] and LSEs [S,B,Hq,Sq].
+
+    softcap, alibi_max_bias and window as in prefill(); sinks belong to merge()."""
     _need(q, "q", torch.bfloat16, 4)
     _need(k, "k", torch.bfloat16, 4)
     _need(v, "v", torch.bfloat16, 4)
@@ -175,16 +209,22 @@ def decode_split(q, k, v, num_splits, *, causal=True, q_offset=0, scale=None,
         partial_out = torch.empty((num_splits, B, Sq, Hq, D), dtype=torch.float32, device=q.device)
     if partial_lse is None:
         partial_lse = torch.empty((num_splits, B, Hq, Sq), dtype=torch.float32, device=q.device)
-    st = library().attn_decode_split(_ptr(q), _ptr(k), _ptr(v), _ptr(partial_out), _ptr(partial_lse), B, Hq,
-                                     Hkv, Sq, Skv, D, int(q_offset), int(bool(causal)), float(scale),
-                                     int(num_splits), _stream_ptr(stream))
-    _check("attn_decode_split", st)
+    opt = _options(softcap, alibi_max_bias, None, window, Hq)
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(partial_out), _ptr(partial_lse), B, Hq, Hkv, Sq, Skv, D,
+            int(q_offset), int(bool(causal)), float(scale), int(num_splits))
+    if opt is None:
+        _check("attn_decode_split", library().attn_decode_split(*args, _stream_ptr(stream)))
+    else:
+        _check("attn_decode_split_ex",
+               library().attn_decode_split_ex(*args, ctypes.byref(opt), _stream_ptr(stream)))
     return partial_out, partial_lse
 
 
 def merge(partial_out, partial_lse, *, out_dtype=torch.bfloat16, out=None, lse=None, return_lse=True,
-          stream=None):
-    """Combine split partials by their LSE into out [B,Sq,Hq,D] and lse [B,Hq,Sq]."""
+          stream=None, sinks=None):
+    """Combine split partials by their LSE into out [B,Sq,Hq,D] and lse [B,Hq,Sq].
+
+    sinks: optional fp32 [Hq] logits that join the denominator and the LSE."""
     _need(partial_out, "partial_out", torch.float32, 5)
     _need(partial_lse, "partial_lse", torch.float32, 4)
     S, B, Sq, Hq, D = partial_out.shape
@@ -192,22 +232,29 @@ def merge(partial_out, partial_lse, *, out_dtype=torch.bfloat16, out=None, lse=N
         out = torch.empty((B, Sq, Hq, D), dtype=out_dtype, device=partial_out.device)
     if lse is None and return_lse:
         lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=partial_out.device)
-    st = library().attn_merge(_ptr(partial_out), _ptr(partial_lse), _ptr(out), _ptr(lse), B, Hq, Sq, D, S,
-                              _OUT_CODES[out.dtype], _stream_ptr(stream))
-    _check("attn_merge", st)
+    args = (_ptr(partial_out), _ptr(partial_lse), _ptr(out), _ptr(lse), B, Hq, Sq, D, S, _OUT_CODES[out.dtype])
+    if sinks is None:
+        _check("attn_merge", library().attn_merge(*args, _stream_ptr(stream)))
+    else:
+        _need(sinks, "sinks", torch.float32, 1)
+        if sinks.shape[0] != Hq:
+            raise ValueError(f"sinks must have Hq = {Hq} entries")
+        _check("attn_merge_ex", library().attn_merge_ex(*args, _ptr(sinks), _stream_ptr(stream)))
     return out, lse
 
 
 def decode(q, k, v, num_splits, *, causal=True, q_offset=0, scale=None, out_dtype=torch.bfloat16,
-           workspace=None, out=None, lse=None, stream=None):
+           workspace=None, out=None, lse=None, stream=None, softcap=0.0, alibi_max_bias=0.0, sinks=None,
+           window=0):
     """Split-KV decode followed by the LSE merge (two launches on one stream)."""
     B, Sq, Hq, D = q.shape
     po = pl = None
     if workspace is not None:
         po, pl = workspace
     po, pl = decode_split(q, k, v, num_splits, causal=causal, q_offset=q_offset, scale=scale,
-                          partial_out=po, partial_lse=pl, stream=stream)
-    return merge(po, pl, out_dtype=out_dtype, out=out, lse=lse, stream=stream)
+                          partial_out=po, partial_lse=pl, stream=stream, softcap=softcap,
+                          alibi_max_bias=alibi_max_bias, window=window)
+    return merge(po, pl, out_dtype=out_dtype, out=out, lse=lse, stream=stream, sinks=sinks)
 
 
 def last_status(stream=None) -> int:

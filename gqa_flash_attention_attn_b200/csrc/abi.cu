@@ -100,6 +100,38 @@ int check_common(const void* q, const void* k, const void* v, int B, int Hq, int
   return ATTN_OK;
 }
 
+// Validates *opt and fills the kernels' form of it.  *on is false when every
+// term is off, so the plain kernels run.
+int make_ext(const attn_options* opt, int Hq, int Sq, int Skv, int q_offset, int causal, float scale,
+             bool allow_sinks, gqa::LogitExt* ext, bool* on) {
+  *ext = gqa::LogitExt{};
+  *on = false;
+  if (opt == nullptr) return ATTN_OK;
+  if (!std::isfinite(opt->softcap) || opt->softcap < 0.f) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(opt->alibi_max_bias) || opt->alibi_max_bias < 0.f) return ATTN_ERR_INVALID_ARG;
+  if (opt->window < 0) return ATTN_ERR_INVALID_ARG;
+  if (opt->sinks != nullptr && !allow_sinks) return ATTN_ERR_INVALID_ARG;
+  if (opt->sinks != nullptr && !aligned(opt->sinks, 4)) return ATTN_ERR_ALIGNMENT;
+  if (opt->window > 0 && (causal != 1 || (long long)q_offset + Sq > Skv)) return ATTN_ERR_UNSUPPORTED;
+  if (opt->softcap > 0.f) {
+    ext->cap_a = scale / opt->softcap;
+    ext->cap_b = opt->softcap * kLog2e;
+    if (!(ext->cap_a > 0.f) || !std::isfinite(ext->cap_a)) return ATTN_ERR_INVALID_ARG;
+  }
+  if (opt->alibi_max_bias > 0.f) {
+    int n2 = 1;
+    while (2 * n2 <= Hq) n2 *= 2;
+    ext->alibi = 1;
+    ext->n2 = n2;
+    ext->l2m0 = -opt->alibi_max_bias / (float)n2;
+    ext->l2m1 = -opt->alibi_max_bias / (float)(2 * n2);
+  }
+  ext->sinks = opt->sinks;
+  ext->window = opt->window;
+  *on = ext->cap_a > 0.f || ext->alibi != 0 || ext->sinks != nullptr || ext->window > 0;
+  return ATTN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -121,7 +153,18 @@ const char* attn_status_string(int status) {
 
 int attn_prefill(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv,
                  int Sq, int Skv, int D, int q_offset, int causal, float scale, int out_dtype, void* stream) {
+  return attn_prefill_ex(q, k, v, out, lse, B, Hq, Hkv, Sq, Skv, D, q_offset, causal, scale, out_dtype, nullptr,
+                         stream);
+}
+
+int attn_prefill_ex(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv,
+                    int Sq, int Skv, int D, int q_offset, int causal, float scale, int out_dtype,
+                    const attn_options* opt, void* stream) {
   int st = check_common(q, k, v, B, Hq, Hkv, Sq, Skv, D, q_offset, causal, scale);
+  if (st != ATTN_OK) return st;
+  gqa::LogitExt ext;
+  bool ext_on;
+  st = make_ext(opt, Hq, Sq, Skv, q_offset, causal, scale, true, &ext, &ext_on);
   if (st != ATTN_OK) return st;
   if (out == nullptr) return ATTN_ERR_INVALID_ARG;
   if (out_dtype != ATTN_BF16 && out_dtype != ATTN_F32) return ATTN_ERR_INVALID_ARG;
@@ -141,6 +184,7 @@ int attn_prefill(const void* q, const void* k, const void* v, void* out, float* 
   p.n_qt = (Sq + 127) / 128;
   p.c2 = scale * kLog2e;
   p.timeout_ns = kWaitLimitNs;
+  p.ext = ext;
   if ((long long)p.n_qt * B * Hkv * p.units_per_kvh > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
 
   p.status = status_ptr();
@@ -151,7 +195,7 @@ int attn_prefill(const void* q, const void* k, const void* v, void* out, float* 
   if (!make_map(&tq, q, D, Hq, Sq, B, 64, 1, 128, 1)) return cuda_fail();
   if (!make_map(&tk, k, D, Hkv, Skv, B, 64, 1, 128, 1)) return cuda_fail();
   if (!make_map(&tv, v, D, Hkv, Skv, B, 64, 1, 128, 1)) return cuda_fail();
-  return gqa::launch_prefill(D, tq, tk, tv, p, static_cast<cudaStream_t>(stream)) == 0 ? ATTN_OK
+  return gqa::launch_prefill(D, ext_on, tq, tk, tv, p, static_cast<cudaStream_t>(stream)) == 0 ? ATTN_OK
                                                                                           : ATTN_ERR_CUDA;
 }
 
@@ -165,7 +209,18 @@ size_t attn_decode_workspace_bytes(int B, int Hq, int Sq, int D, int num_splits)
 int attn_decode_split(const void* q, const void* k, const void* v, float* partial_out, float* partial_lse,
                       int B, int Hq, int Hkv, int Sq, int Skv, int D, int q_offset, int causal, float scale,
                       int num_splits, void* stream) {
+  return attn_decode_split_ex(q, k, v, partial_out, partial_lse, B, Hq, Hkv, Sq, Skv, D, q_offset, causal, scale,
+                              num_splits, nullptr, stream);
+}
+
+int attn_decode_split_ex(const void* q, const void* k, const void* v, float* partial_out, float* partial_lse,
+                         int B, int Hq, int Hkv, int Sq, int Skv, int D, int q_offset, int causal, float scale,
+                         int num_splits, const attn_options* opt, void* stream) {
   int st = check_common(q, k, v, B, Hq, Hkv, Sq, Skv, D, q_offset, causal, scale);
+  if (st != ATTN_OK) return st;
+  gqa::LogitExt ext;
+  bool ext_on;
+  st = make_ext(opt, Hq, Sq, Skv, q_offset, causal, scale, false, &ext, &ext_on);
   if (st != ATTN_OK) return st;
   if (partial_out == nullptr || partial_lse == nullptr) return ATTN_ERR_INVALID_ARG;
   if (num_splits < 1 || num_splits > Skv || num_splits > 65535) return ATTN_ERR_INVALID_ARG;
@@ -193,6 +248,7 @@ int attn_decode_split(const void* q, const void* k, const void* v, float* partia
   p.nbuf = nbuf;
   p.c2 = scale * kLog2e;
   p.timeout_ns = kWaitLimitNs;
+  p.ext = ext;
 
   p.status = status_ptr();
   if (p.status == nullptr) return cuda_fail();
@@ -200,19 +256,26 @@ int attn_decode_split(const void* q, const void* k, const void* v, float* partia
   if (!make_map(&tq, q, D, Hq, Sq, B, 64, (uint32_t)g, (uint32_t)Sq, 1)) return cuda_fail();
   if (!make_map(&tk, k, D, Hkv, Skv, B, 64, 1, 128, 1)) return cuda_fail();
   if (!make_map(&tv, v, D, Hkv, Skv, B, 64, 1, 128, 1)) return cuda_fail();
-  return gqa::launch_decode_split(D, tq, tk, tv, p, static_cast<cudaStream_t>(stream)) == 0 ? ATTN_OK
+  return gqa::launch_decode_split(D, ext_on, tq, tk, tv, p, static_cast<cudaStream_t>(stream)) == 0 ? ATTN_OK
                                                                                                : ATTN_ERR_CUDA;
 }
 
 int attn_merge(const float* partial_out, const float* partial_lse, void* out, float* lse, int B, int Hq, int Sq,
                int D, int num_splits, int out_dtype, void* stream) {
+  return attn_merge_ex(partial_out, partial_lse, out, lse, B, Hq, Sq, D, num_splits, out_dtype, nullptr, stream);
+}
+
+int attn_merge_ex(const float* partial_out, const float* partial_lse, void* out, float* lse, int B, int Hq,
+                  int Sq, int D, int num_splits, int out_dtype, const float* sinks, void* stream) {
   if (partial_out == nullptr || partial_lse == nullptr || out == nullptr) return ATTN_ERR_INVALID_ARG;
   if (B < 1 || Hq < 1 || Sq < 1 || num_splits < 1) return ATTN_ERR_INVALID_ARG;
   if (out_dtype != ATTN_BF16 && out_dtype != ATTN_F32) return ATTN_ERR_INVALID_ARG;
   if (D < 4 || D > 1024 || D % 4 != 0) return ATTN_ERR_UNSUPPORTED;
   if (!aligned(partial_out, 16) || !aligned(out, out_dtype == ATTN_F32 ? 16 : 8)) return ATTN_ERR_ALIGNMENT;
   if (!aligned(partial_lse, 4) || (lse != nullptr && !aligned(lse, 4))) return ATTN_ERR_ALIGNMENT;
+  if (sinks != nullptr && !aligned(sinks, 4)) return ATTN_ERR_ALIGNMENT;
   gqa::MergeParams p{};
+  p.sinks = sinks;
   p.part_out = partial_out;
   p.part_lse = partial_lse;
   p.out = out;

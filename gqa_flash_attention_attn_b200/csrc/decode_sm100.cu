@@ -47,7 +47,7 @@ struct Layout {
     off_ring = (off_p + 2u * 2u * RP * 128u + 1023u) & ~1023u;  // two P buffers
     off_red = off_ring + (uint32_t)nbuf * SLOT_BYTES;
     off_row = off_red + 2u * 4u * RP * 4u;     // red_max[4][RP], red_sum[4][RP]
-    off_bar = off_row + 6u * RP * 4u;          // m, l, alpha, msub, inv, lim
+    off_bar = off_row + 9u * RP * 4u;          // m, l, alpha, msub, inv, lim, limlo, pos, slope
     off_bar = (off_bar + 7u) & ~7u;
     off_misc = off_bar + (uint32_t)(1 + 2 * nbuf + 7) * 8u;
     total = off_misc + 16u + 1024u;
@@ -81,7 +81,7 @@ __device__ __forceinline__ float warp_reduce16(float (&v)[16], int lane) {
   return kMax ? fmaxf(v[0], other) : v[0] + other;
 }
 
-template <int D>
+template <int D, bool EXT>
 __global__ void __launch_bounds__(THREADS, 1)
     decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
@@ -100,7 +100,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   float* alpha_sm = l_sm + RP;
   float* msub_sm = alpha_sm + RP;
   float* inv_sm = msub_sm + RP;
-  int* lim_sm = reinterpret_cast<int*>(inv_sm + RP);
+  int* lim_sm = reinterpret_cast<int*>(inv_sm + RP);     // last visible key of row r
+  int* limlo_sm = lim_sm + RP;                             // keys <= this are outside the window
+  int* pos_sm = limlo_sm + RP;                             // query position of row r
+  float* slope_sm = reinterpret_cast<float*>(pos_sm + RP); // ALiBi slope * log2(e) of row r
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L.off_misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L.off_misc + 4);
   volatile int* resc_flag = reinterpret_cast<volatile int*>(gbase + L.off_misc + 8);
@@ -120,7 +123,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int lo = (int)min(lo_ll, (long long)p.Skv);
   const int hi = (int)min(lo_ll + p.chunk, (long long)p.Skv);
   const int eff_hi = p.causal ? min(hi, p.q_offset + p.Sq) : hi;
-  const int n_tiles = eff_hi > lo ? (eff_hi - lo + BN - 1) / BN : 0;
+  // a sliding window hides every key at or before q_offset - window from all rows
+  const int eff_lo = (EXT && p.ext.window > 0) ? max(lo, p.q_offset - p.ext.window + 1) : lo;
+  const int kbase = lo + ((eff_lo - lo) / BN) * BN;   // first tile, on the split's tile grid
+  const int n_tiles = eff_hi > eff_lo ? (eff_hi - kbase + BN - 1) / BN : 0;
   const size_t split_out = (size_t)split * p.B * p.Sq * p.Hq * D;
   const size_t split_lse = (size_t)split * p.B * p.Hq * p.Sq;
 
@@ -150,6 +156,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     l_sm[r] = 0.f;
     // last visible key of row r (padding rows see none)
     lim_sm[r] = r < R ? (p.causal ? p.q_offset + r / g : 0x7fffffff) : -1;
+    pos_sm[r] = p.q_offset + (r < R ? r / g : 0);
+    limlo_sm[r] = (EXT && p.ext.window > 0) ? pos_sm[r] - p.ext.window : -1;
+    slope_sm[r] = (EXT && p.ext.alibi && r < R)
+                      ? alibi_slope_log2e(kvh * g + (r - (r / g) * g), p.ext.l2m0, p.ext.l2m1, p.ext.n2)
+                      : 0.f;
   }
   if (threadIdx.x == 0) {
     mbar_init(bar(BAR_Q), 1);
@@ -204,7 +215,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
           mbar_arrive_expect_tx(bar(bar_full(slot)), SLOT_BYTES);
           const uint32_t dst = base + L.off_ring + (uint32_t)slot * SLOT_BYTES;
-          const int key0 = lo + j * BN;
+          const int key0 = kbase + j * BN;
           tma_load_4d(dst, tm, bar(bar_full(slot)), (2 * c) * 64, kvh, key0, b);
           tma_load_4d(dst + BOX_BYTES, tm, bar(bar_full(slot)), (2 * c + 1) * 64, kvh, key0, b);
           issued = n + 1;
@@ -284,18 +295,31 @@ __global__ void __launch_bounds__(THREADS, 1)
       const bool got_s = mbar_wait(bar(BAR_S0 + sb), (uint32_t)(j >> 1) & 1u, wd);
       if (named_bar_or(1, 128, !got_s)) { ok = false; break; }
       tc_fence_after();
-      const int tile0 = lo + j * BN;
+      const int tile0 = kbase + j * BN;
       const int key = tile0 + t;
       // whole tile visible to every real row: no per-element mask
-      const bool full = (tile0 + BN - 1 < hi) && (!p.causal || tile0 + BN - 1 <= p.q_offset);
+      const bool full = (tile0 + BN - 1 < hi) && (!p.causal || tile0 + BN - 1 <= p.q_offset) &&
+                        (!EXT || p.ext.window == 0 || tile0 >= p.q_offset + p.Sq - p.ext.window);
+      // optional terms: logit in log2 units, softcap and ALiBi applied
+      auto logit2 = [&](float sdot, int r) -> float {
+        const float z = p.ext.cap_a > 0.f ? p.ext.cap_b * tanh_via_exp2(sdot * p.ext.cap_a) : sdot * c2;
+        return fmaf(slope_sm[r], (float)(key - pos_sm[r]), z);
+      };
+      auto visible = [&](int r) -> bool {
+        return key < hi && key <= lim_sm[r] && (!EXT || key > limlo_sm[r]);
+      };
       // pass 1: per-row max over the tile's visible keys
       for (int q = 0; q < RP / 16; ++q) {
         float v[16];
         tmem_ld16(tmem + lane_off + TS(sb) + 16 * q, v);
+        if (EXT) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) v[e] = logit2(v[e], 16 * q + e);
+        }
         if (!full) {
 #pragma unroll
           for (int e = 0; e < 16; ++e)
-            if (!(key < hi && key <= lim_sm[16 * q + e])) v[e] = -INFINITY;
+            if (!visible(16 * q + e)) v[e] = -INFINITY;
         }
         const float x = warp_reduce16<true>(v, lane);
         if (lane < 16) red_max[warp * RP + 16 * q + lane] = x;
@@ -303,7 +327,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       named_bar_sync(1, 128);
       if (t < RP) {
         const float mt = fmaxf(fmaxf(red_max[t], red_max[RP + t]), fmaxf(red_max[2 * RP + t], red_max[3 * RP + t]));
-        const float m_tile = mt * c2;
+        const float m_tile = EXT ? mt : mt * c2;
         const float m_old = m_sm[t];
         float m_new = m_old, alpha = 1.f;
         if (m_tile > m_old + 8.f) {
@@ -331,8 +355,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int r = 16 * q + e;
-            float pv = ex2_approx(fmaf(v[e], c2, -msub_sm[r]));
-            if (!full && !(key < hi && key <= lim_sm[r])) pv = 0.f;
+            float pv = EXT ? ex2_approx(logit2(v[e], r) - msub_sm[r]) : ex2_approx(fmaf(v[e], c2, -msub_sm[r]));
+            if (!full && !visible(r)) pv = 0.f;
             *reinterpret_cast<__nv_bfloat16*>(pcol + (size_t)r * 128 + ((chunk16 ^ (r & 7)) << 4)) =
                 __float2bfloat16_rn(pv);
             v[e] = pv;
@@ -422,15 +446,15 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-template <int D>
+template <int D, bool EXT>
 int launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
              const DecodeParams& p, cudaStream_t stream) {
   const Layout L(D, p.RP, p.nbuf);
-  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, EXT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)L.total);
   if (e != cudaSuccess) return (int)e;
   dim3 grid((unsigned)p.num_splits, (unsigned)(p.B * p.Hkv));
-  decode_split_kernel<D><<<grid, THREADS, L.total, stream>>>(tq, tk, tv, p);
+  decode_split_kernel<D, EXT><<<grid, THREADS, L.total, stream>>>(tq, tk, tv, p);
   return (int)cudaGetLastError();
 }
 
@@ -440,12 +464,12 @@ size_t decode_smem_bytes(int D, int RP, int nbuf) { return Layout(D, RP, nbuf).t
 
 int decode_max_nbuf() { return MAX_NBUF; }
 
-int launch_decode_split(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+int launch_decode_split(int D, bool ext, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                         const DecodeParams& p, cudaStream_t stream) {
   switch (D) {
-    case 128: return launch_t<128>(tq, tk, tv, p, stream);
-    case 256: return launch_t<256>(tq, tk, tv, p, stream);
-    case 512: return launch_t<512>(tq, tk, tv, p, stream);
+    case 128: return ext ? launch_t<128, true>(tq, tk, tv, p, stream) : launch_t<128, false>(tq, tk, tv, p, stream);
+    case 256: return ext ? launch_t<256, true>(tq, tk, tv, p, stream) : launch_t<256, false>(tq, tk, tv, p, stream);
+    case 512: return ext ? launch_t<512, true>(tq, tk, tv, p, stream) : launch_t<512, false>(tq, tk, tv, p, stream);
     default: return (int)cudaErrorInvalidValue;
   }
 }

@@ -6,6 +6,20 @@
 
 namespace gqa {
 
+// Optional logit terms, prepared on the host.  The logit in log2 units is
+//   L = (cap_a > 0 ? cap_b * tanh(s * cap_a) : s * c2) + slope_h * log2(e) * (t - pos)
+// with s the raw Q.K dot product; slope_h = 2^(l2m0 * (h + 1)) for h < n2,
+// else 2^(l2m1 * (2 (h - n2) + 1)), and 0 when alibi is off.
+struct LogitExt {
+  float cap_a;        // scale / softcap, or 0 when off
+  float cap_b;        // softcap * log2(e)
+  int alibi;          // 0: off
+  float l2m0, l2m1;   // log2 of the two ALiBi slope bases
+  int n2;             // largest power of two <= Hq
+  const float* sinks; // [Hq] natural-log sink logits, or nullptr
+  int window;         // 0: off
+};
+
 struct PrefillParams {
   void* out;          // [B, Sq, Hq, D] bf16 or f32
   float* lse;         // [B, Hq, Sq] or nullptr
@@ -17,6 +31,7 @@ struct PrefillParams {
   int num_ctas;       // persistent grid size (SM count)
   float c2;           // scale * log2(e)
   unsigned long long timeout_ns;
+  LogitExt ext;
 };
 
 struct DecodeParams {
@@ -29,6 +44,7 @@ struct DecodeParams {
   int nbuf;           // K/V ring slots (32 KB each)
   float c2;
   unsigned long long timeout_ns;
+  LogitExt ext;       // sinks unused: the merge adds them
 };
 
 struct MergeParams {
@@ -36,14 +52,15 @@ struct MergeParams {
   const float* part_lse;
   void* out;
   float* lse;
+  const float* sinks;  // [Hq] or nullptr
   int B, Hq, Sq, D, num_splits, out_f32;
 };
 
 // Each returns a cudaError_t value (as int) from the launch.
-int launch_prefill(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+int launch_prefill(int D, bool ext, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                    const PrefillParams& p, cudaStream_t stream);
 size_t prefill_smem_bytes(int D);
-int launch_decode_split(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+int launch_decode_split(int D, bool ext, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                         const DecodeParams& p, cudaStream_t stream);
 size_t decode_smem_bytes(int D, int RP, int nbuf);
 int launch_merge(const MergeParams& p, cudaStream_t stream);

@@ -2,7 +2,8 @@
 //
 // For each output row: M = max_s lse_s, w_s = exp(lse_s - M),
 // out = sum_s w_s O_s / sum_s w_s, lse = M + log(sum_s w_s); splits that
-// published lse = -inf carry weight 0 ("Anbeeld/beellama.cpp PR #149", review
+// published lse = -inf carry weight 0; an optional sink logit joins M and the
+// denominator only ("Anbeeld/beellama.cpp PR #149", review
 // of the combine kernel that merges per-block partials for parallel_blocks > 1).
 //
 // Memory-bound: a block owns 128 consecutive columns of one row, each lane a
@@ -36,8 +37,10 @@ __global__ void __launch_bounds__(128, 8) merge_kernel(const MergeParams p) {
   const size_t out_stride4 = (size_t)p.B * p.Sq * p.Hq * p.D / 4;
   const float4* src = reinterpret_cast<const float4*>(p.part_out + (size_t)row * p.D) + (active ? f : 0);
 
-  // max of the split LSEs (every warp computes it; the loads are tiny)
-  float M = -INFINITY;
+  // max of the split LSEs and the sink logit (every warp computes it; the
+  // loads are tiny); the sink joins only the denominator
+  const float sink = p.sinks != nullptr ? __ldg(p.sinks + h) : -INFINITY;
+  float M = sink;
   for (int sg = lane; sg < p.num_splits; sg += 32) M = fmaxf(M, __ldg(p.part_lse + sg * lse_stride + lse_row));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
@@ -71,6 +74,7 @@ __global__ void __launch_bounds__(128, 8) merge_kernel(const MergeParams p) {
       }
     }
   }
+  if (warp == 0 && sink != -INFINITY) wsum += ex2_approx((sink - M) * 1.4426950408889634f);
   if (warp > 0) {
     part_acc[warp - 1][lane] = acc;
     if (lane == 0) part_w[warp - 1] = wsum;

@@ -106,7 +106,9 @@ __device__ __forceinline__ bool ring_item(int n, int n_tiles, int& tile) {
 
 // One unit of work: a 128-row query tile for up to NSLOT heads of one K/V group.
 struct Unit {
-  int b, kvh, hl0, s0, n_tiles;
+  int b, kvh, hl0, s0;
+  int t0;       // first K/V tile the unit visits (a sliding window skips the rest)
+  int n_tiles;  // tiles t0 .. t0 + n_tiles - 1
 };
 
 // Unit u in longest-first order: q-tiles with the most visible keys first,
@@ -126,7 +128,9 @@ __device__ __forceinline__ Unit unit_at(int u, const PrefillParams& p) {
   const int qt = p.causal ? (p.n_qt - 1 - qt_rev) : qt_rev;
   x.s0 = qt * BM;
   const int kv_end = p.causal ? min(p.Skv, p.q_offset + min(x.s0 + BM, p.Sq)) : p.Skv;
-  x.n_tiles = (kv_end + BN - 1) / BN;
+  const int kv_begin = p.ext.window > 0 ? max(0, p.q_offset + x.s0 - p.ext.window + 1) : 0;
+  x.t0 = kv_begin / BN;
+  x.n_tiles = (kv_end + BN - 1) / BN - x.t0;
   return x;
 }
 
@@ -140,7 +144,41 @@ __device__ __forceinline__ int unit_index(int k, int total) {
   return u < total ? (int)u : -1;
 }
 
-template <int D>
+// Logits of N consecutive keys in log2 units with the optional terms:
+// softcap (cap_b tanh(s cap_a)) or plain scaling (s c2), then the ALiBi bias
+// slope2 * (key - pos), dist0 being the first key's distance.
+template <int N>
+__device__ __forceinline__ void ext_logits(float (&v)[N], const LogitExt& x, float c2, float slope2, float dist0) {
+#pragma unroll
+  for (int e = 0; e < N; ++e) {
+    const float z = x.cap_a > 0.f ? x.cap_b * tanh_via_exp2(v[e] * x.cap_a) : v[e] * c2;
+    v[e] = fmaf(slope2, dist0 + (float)e, z);
+  }
+}
+
+// Columns outside [cb, cl) become -inf.
+template <int N>
+__device__ __forceinline__ void mask_cols(float (&v)[N], int cb, int cl) {
+#pragma unroll
+  for (int e = 0; e < N; ++e) v[e] = (e < cl && e >= cb) ? v[e] : -INFINITY;
+}
+
+// Row maximum: eight independent 3-input max chains, then a small tree.
+template <int N>
+__device__ __forceinline__ float row_max(const float (&v)[N]) {
+  static_assert(N % 16 == 0, "row_max takes multiples of 16 columns");
+  float mxc[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) mxc[c] = fmaxf(v[2 * c], v[2 * c + 1]);
+#pragma unroll
+  for (int e = 16; e < N; e += 16) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) mxc[c] = fmax3(mxc[c], v[e + 2 * c], v[e + 2 * c + 1]);
+  }
+  return fmax3(fmax3(mxc[0], mxc[1], mxc[2]), fmax3(mxc[3], mxc[4], mxc[5]), fmaxf(mxc[6], mxc[7]));
+}
+
+template <int D, bool EXT>
 __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
@@ -222,7 +260,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
           mbar_arrive_expect_tx(bar(C::bar_full(buf)), C::TILE);
           for (int kb = 0; kb < C::KB; ++kb)
             tma_load_4d(base + C::OFF_KV + buf * C::TILE + kb * BOX_BYTES, tm, bar(C::bar_full(buf)),
-                        kb * 64, x.kvh, tile * BN, x.b);
+                        kb * 64, x.kvh, (x.t0 + tile) * BN, x.b);
           issued = n + 1;
         }
       }
@@ -390,7 +428,10 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
       const int n_tiles = x.n_tiles;
       const int h = x.kvh * p.g + hl;
       const int s_row = x.s0 + r;
-      const int vis_end = p.causal ? min(p.Skv, p.q_offset + s_row + 1) : p.Skv;
+      const int pos = p.q_offset + s_row;
+      const int vis_end = p.causal ? min(p.Skv, pos + 1) : p.Skv;
+      const int vis_begin = (EXT && p.ext.window > 0) ? pos - p.ext.window + 1 : 0;
+      const float slope2 = (EXT && p.ext.alibi) ? alibi_slope_log2e(h, p.ext.l2m0, p.ext.l2m1, p.ext.n2) : 0.f;
       float m_use = -INFINITY, l = 0.f;
       for (int j = 0; j < n_tiles; ++j) {
         const int G = T + j;
@@ -402,26 +443,33 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
         const bool got = mbar_wait(bar(C::bar_s(sb)), ph, wd);
         if (__any_sync(0xffffffffu, !got)) { ok = false; break; }
         tc_fence_after();
-        const int cl = vis_end - j * BN;  // visible columns of this tile for this row
-        // one TMEM read of the whole 128-column S row
+        const int key0 = (x.t0 + j) * BN;
+        const int cl = vis_end - key0;    // visible columns of this tile: [cb, cl)
+        const int cb = vis_begin - key0;
+        const bool tile_masked = __any_sync(0xffffffffu, cl < BN || cb > 0);
         float sv[BN];
-        tmem_ld128(tS, sv);
-        const bool tile_masked = __any_sync(0xffffffffu, cl < BN);
-        if (tile_masked) {  // diagonal or ragged tile: mask in place
-#pragma unroll
-          for (int e = 0; e < BN; ++e) sv[e] = (e < cl) ? sv[e] : -INFINITY;
+        float mx;
+        if constexpr (EXT) {
+          // logits in log2 units with the optional softcap and ALiBi terms;
+          // keys 64-127 first, for their maximum only, so that one half of
+          // the row is live at a time
+          float sh[BN / 2];
+          tmem_ld64(tS + BN / 2, sh);
+          ext_logits(sh, p.ext, c2, slope2, (float)(key0 + BN / 2 - pos));
+          if (tile_masked) mask_cols(sh, cb - BN / 2, cl - BN / 2);
+          const float mx_hi = row_max(sh);
+          float (&slo)[BN / 2] = *reinterpret_cast<float(*)[BN / 2]>(sv);
+          tmem_ld64(tS, slo);
+          ext_logits(slo, p.ext, c2, slope2, (float)(key0 - pos));
+          if (tile_masked) mask_cols(slo, cb, cl);
+          mx = fmaxf(mx_hi, row_max(slo));
+        } else {
+          // one TMEM read of the whole 128-column S row
+          tmem_ld128(tS, sv);
+          if (tile_masked) mask_cols(sv, cb, cl);
+          mx = row_max(sv);
         }
-        // row max: eight independent 3-input max chains, then a small tree
-        float mxc[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) mxc[c] = fmaxf(sv[2 * c], sv[2 * c + 1]);
-#pragma unroll
-        for (int e = 16; e < BN; e += 16) {
-#pragma unroll
-          for (int c = 0; c < 8; ++c) mxc[c] = fmax3(mxc[c], sv[e + 2 * c], sv[e + 2 * c + 1]);
-        }
-        const float mx = fmax3(fmax3(mxc[0], mxc[1], mxc[2]), fmax3(mxc[3], mxc[4], mxc[5]), fmaxf(mxc[6], mxc[7]));
-        const float m_tile = mx * c2;
+        const float m_tile = EXT ? mx : mx * c2;
         float m_new = m_use, alpha = 1.f;
         if (m_tile > m_use + 8.f) {
           m_new = m_tile;
@@ -451,7 +499,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
         // partial sums, bf16 pairs for the P.V operand (masked s = -inf -> p = 0).
         // P is handed over in two halves (keys 0-63, then 64-127) so the P.V
         // MMAs on the first half overlap the exponentials of the second.
-        const float2 c2v = make_float2(c2, c2);
+        const float2 c2v = EXT ? make_float2(1.f, 1.f) : make_float2(c2, c2);
         const float2 nmv = make_float2(-m_sub, -m_sub);
         float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
         // half 0: keys 0-63 from the registers; P lands on TMEM columns 0-31,
@@ -475,10 +523,8 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
         {
           float sh[BN / 2];
           tmem_ld64(tS + BN / 2, sh);
-          if (tile_masked) {
-#pragma unroll
-            for (int e = 0; e < BN / 2; ++e) sh[e] = (e + BN / 2 < cl) ? sh[e] : -INFINITY;
-          }
+          if constexpr (EXT) ext_logits(sh, p.ext, c2, slope2, (float)(key0 + BN / 2 - pos));
+          if (tile_masked) mask_cols(sh, cb - BN / 2, cl - BN / 2);
           uint32_t pk[BN / 4];
 #pragma unroll
           for (int e = 0; e < BN / 4; ++e) {
@@ -507,7 +553,19 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
         ok = false;
       } else {
         tc_fence_after();
-        const float inv_l = 1.f / l;
+        // The sink joins the denominator against a common maximum M, so a
+        // large sink logit cannot overflow: O = O_acc 2^(m - M) / l',
+        // l' = l 2^(m - M) + 2^(sink - M), LSE = M + log2 l'.
+        float m_fin = m_use, inv_l;
+        if (EXT && p.ext.sinks != nullptr) {
+          const float s2 = __ldg(p.ext.sinks + h) * 1.4426950408889634f;
+          m_fin = fmaxf(m_use, s2);
+          const float a = ex2_approx(m_use - m_fin);
+          l = l * a + ex2_approx(s2 - m_fin);
+          inv_l = a / l;
+        } else {
+          inv_l = l > 0.f ? 1.f / l : 0.f;
+        }
         const bool row_ok = s_row < p.Sq;
         const size_t row_off = (((size_t)x.b * p.Sq + s_row) * p.Hq + h) * (size_t)D;
 #pragma unroll 1
@@ -533,7 +591,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
           }
         }
         if (row_ok && p.lse != nullptr)
-          p.lse[((size_t)x.b * p.Hq + h) * p.Sq + s_row] = (m_use + log2f(l)) * LN2;
+          p.lse[((size_t)x.b * p.Hq + h) * p.Sq + s_row] = l > 0.f ? (m_fin + log2f(l)) * LN2 : -INFINITY;
       }
       // O of this slot may now be overwritten by the next unit's first P.V
       tc_fence_before();
@@ -565,17 +623,17 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
   }
 }
 
-template <int D>
+template <int D, bool EXT>
 int launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
              const PrefillParams& p, cudaStream_t stream) {
   using C = PrefillCfg<D>;
-  cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D, EXT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)C::SMEM);
   if (e != cudaSuccess) return (int)e;
   const long long units = (long long)p.n_qt * p.B * p.Hkv * p.units_per_kvh;
   if (units <= 0 || units > 0x7fffffffLL || p.num_ctas <= 0) return (int)cudaErrorInvalidValue;
   const long long grid = units < p.num_ctas ? units : p.num_ctas;  // persistent: one CTA per SM
-  prefill_kernel<D><<<(unsigned)grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, p);
+  prefill_kernel<D, EXT><<<(unsigned)grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, p);
   return (int)cudaGetLastError();
 }
 
@@ -592,12 +650,12 @@ size_t prefill_smem_bytes(int D) {
 
 int prefill_slots(int D) { return D <= 128 ? 2 : 1; }
 
-int launch_prefill(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+int launch_prefill(int D, bool ext, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                    const PrefillParams& p, cudaStream_t stream) {
   switch (D) {
-    case 64: return launch_t<64>(tq, tk, tv, p, stream);
-    case 128: return launch_t<128>(tq, tk, tv, p, stream);
-    case 256: return launch_t<256>(tq, tk, tv, p, stream);
+    case 64: return ext ? launch_t<64, true>(tq, tk, tv, p, stream) : launch_t<64, false>(tq, tk, tv, p, stream);
+    case 128: return ext ? launch_t<128, true>(tq, tk, tv, p, stream) : launch_t<128, false>(tq, tk, tv, p, stream);
+    case 256: return ext ? launch_t<256, true>(tq, tk, tv, p, stream) : launch_t<256, false>(tq, tk, tv, p, stream);
     default: return (int)cudaErrorInvalidValue;
   }
 }

@@ -306,6 +306,22 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
   return d;
 }
 
+// ---------------------------------------------------- optional logit terms --
+// tanh through the identity tanh(x) = 1 - 2 / (e^(2x) + 1), with e^(2x) from
+// ex2.approx (relative error ~2^-22): accurate to ~1e-7 absolute, unlike the
+// ~5e-4 relative error of the hardware tanh approximation.
+__device__ __forceinline__ float tanh_via_exp2(float x) {
+  float e;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(x * 2.8853900817779268f));  // 2 / ln 2
+  return 1.f - __fdividef(2.f, e + 1.f);
+}
+
+// ALiBi slope of head h (geometric per head; see LogitExt), times log2(e).
+__device__ __forceinline__ float alibi_slope_log2e(int h, float l2m0, float l2m1, int n2) {
+  const float ex = h < n2 ? l2m0 * (float)(h + 1) : l2m1 * (float)(2 * (h - n2) + 1);
+  return exp2f(ex) * 1.4426950408889634f;
+}
+
 // ------------------------------------------------------------ arithmetic ----
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;

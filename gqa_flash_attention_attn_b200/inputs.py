@@ -33,11 +33,27 @@ class Workload:
     out_dtype: str       # "bf16" or "f32"
     num_splits: int = 1
     note: str = ""
+    # optional logit terms (0 / False = off); sinks are drawn by make_sinks(Hq, seed=0)
+    softcap: float = 0.0
+    alibi_max_bias: float = 0.0
+    sinks: bool = False
+    window: int = 0
+
+    @property
+    def has_options(self) -> bool:
+        return bool(self.softcap or self.alibi_max_bias or self.sinks or self.window)
 
     @property
     def scale(self) -> float:
         # the float32 value both sides receive
         return float(torch.tensor(1.0 / math.sqrt(self.D), dtype=torch.float32))
+
+    def visible_range(self, s: int) -> tuple[int, int]:
+        """Keys [lo, hi) that query row s sees (causal mask and window)."""
+        pos = self.q_offset + s
+        hi = min(self.Skv, pos + 1) if self.causal else self.Skv
+        lo = max(0, pos - self.window + 1) if self.window > 0 else 0
+        return lo, max(lo, hi)
 
     def visible_pairs_per_head(self) -> int:
         """Number of visible (query row, key) pairs for one (batch, head)."""
@@ -45,8 +61,15 @@ class Workload:
             return self.Sq * self.Skv
         total = 0
         for s in range(self.Sq):
-            total += min(self.Skv, self.q_offset + s + 1)
+            lo, hi = self.visible_range(s)
+            total += hi - lo
         return total
+
+    def kv_rows_read(self) -> int:
+        """Keys that at least one query row sees: the K/V rows a pass must read."""
+        lo, _ = self.visible_range(0)
+        _, hi = self.visible_range(self.Sq - 1)
+        return hi - lo if self.causal else self.Skv
 
     def flops(self) -> int:
         """Algorithmic FLOPs: 4*D per visible (query, key) pair."""
@@ -56,7 +79,7 @@ class Workload:
         """Algorithmic bytes: Q, K, V read once (bf16); O and LSE written once."""
         ob = 2 if self.out_dtype == "bf16" else 4
         q = self.B * self.Sq * self.Hq * self.D * 2
-        kv = 2 * self.B * self.Skv * self.Hkv * self.D * 2
+        kv = 2 * self.B * self.kv_rows_read() * self.Hkv * self.D * 2
         o = self.B * self.Sq * self.Hq * self.D * ob
         lse = self.B * self.Hq * self.Sq * 4
         return q + kv + o + lse
@@ -83,6 +106,18 @@ WORKLOADS = {
         "spec_verify_decode_d128", "decode", B=4, Hq=32, Hkv=8, Sq=8, Skv=32768, D=128,
         q_offset=32760, causal=True, out_dtype="bf16", num_splits=16,
         note="8 draft rows per sequence, causal among themselves, Skv 32768"),
+    "prefill_4k_d128_softcap_alibi_sinks": Workload(
+        "prefill_4k_d128_softcap_alibi_sinks", "prefill", B=1, Hq=32, Hkv=8, Sq=4096, Skv=4096, D=128,
+        q_offset=0, causal=True, out_dtype="bf16", softcap=30.0, alibi_max_bias=8.0, sinks=True,
+        note="the 4k causal GQA prefill with logit softcap 30, ALiBi (max bias 8) and per-head sinks"),
+    "sliding_window_prefill_16k_w4096_d128": Workload(
+        "sliding_window_prefill_16k_w4096_d128", "prefill", B=1, Hq=32, Hkv=8, Sq=16384, Skv=16384, D=128,
+        q_offset=0, causal=True, out_dtype="bf16", window=4096,
+        note="B1 Hq32 Hkv8 S16384 D128, causal with a 4096-key sliding window"),
+    "split_kv_decode_d512_softcap_alibi_sinks": Workload(
+        "split_kv_decode_d512_softcap_alibi_sinks", "decode", B=16, Hq=16, Hkv=1, Sq=1, Skv=16384, D=512,
+        q_offset=16383, causal=True, out_dtype="bf16", num_splits=32, softcap=30.0, alibi_max_bias=8.0,
+        sinks=True, note="the D512 split-KV decode with softcap 30, ALiBi (max bias 8) and sinks in the merge"),
 }
 
 
@@ -97,6 +132,13 @@ def make_qkv(B, Hq, Hkv, Sq, Skv, D, *, seed=0, device="cpu"):
     v = torch.randn((B, Skv, Hkv, D), generator=gen, dtype=torch.float32, device=device)
     v = v.to(torch.bfloat16)
     return q, k, v
+
+
+def make_sinks(Hq, *, seed=0, std=3.0, device="cpu"):
+    """Seeded fp32 sink logits [Hq] ~ N(0, std^2), one per query head."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    return torch.randn((Hq,), generator=gen, dtype=torch.float32, device=device) * std
 
 
 def make_workload_inputs(w: Workload, *, seed=0, device="cpu"):

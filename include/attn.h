@@ -161,6 +161,56 @@ int attn_decode_noalloc(const void* q, const void* k, const void* v, void* out, 
                         int B, int Hq, int Hkv, int Sq, int Skv, int D, int q_offset, int causal,
                         float scale, int num_splits, int out_dtype, void* stream);
 
+/*
+ * Optional terms of the attention logit, from the parameters of the
+ * FLASH_ATTN_EXT operator ("ggml-org/llama.cpp PR #28507", Crash 1: the test
+ * case list carries sinks, max_bias and logit_softcap).  With z the scaled
+ * logit scale * q.k_t of query row s (position pos = q_offset + s) and key t:
+ *
+ *   softcap > 0          z = softcap * tanh(z / softcap)
+ *   alibi_max_bias > 0   z = z + slope_h * (t - pos), slope_h geometric per
+ *                        head: n2 = largest power of two <= Hq,
+ *                        m0 = 2^(-max_bias / n2), m1 = 2^(-max_bias / (2 n2)),
+ *                        slope_h = m0^(h+1) for h < n2, else m1^(2(h-n2)+1)
+ *   sinks != NULL        device array [Hq] of fp32 sink logits: exp(sinks[h])
+ *                        joins the softmax denominator (and the LSE), with no
+ *                        value row
+ *   window > 0           key t is visible only if pos - window < t; needs
+ *                        causal = 1 and q_offset + Sq <= Skv (every query
+ *                        position has its key), else ATTN_ERR_UNSUPPORTED
+ *
+ * Zero / NULL fields are off.  softcap and alibi_max_bias must be finite and
+ * >= 0, window >= 0 (else ATTN_ERR_INVALID_ARG); sinks must be 4-byte aligned
+ * (else ATTN_ERR_ALIGNMENT).  The caller owns *opt and the sink array; the
+ * call reads *opt on the host before it returns and the sink array on the
+ * device, in stream order.
+ */
+typedef struct attn_options {
+  float softcap;
+  float alibi_max_bias;
+  const float* sinks;
+  int window;
+} attn_options;
+
+/* attn_prefill with the optional terms of *opt (opt may be NULL). */
+int attn_prefill_ex(const void* q, const void* k, const void* v, void* out, float* lse,
+                    int B, int Hq, int Hkv, int Sq, int Skv, int D, int q_offset, int causal,
+                    float scale, int out_dtype, const attn_options* opt, void* stream);
+
+/* attn_decode_split with softcap, ALiBi and window from *opt (opt may be
+ * NULL).  Sinks belong to the merge, which adds them once per row:
+ * opt->sinks must be NULL here (else ATTN_ERR_INVALID_ARG). */
+int attn_decode_split_ex(const void* q, const void* k, const void* v, float* partial_out,
+                         float* partial_lse, int B, int Hq, int Hkv, int Sq, int Skv, int D,
+                         int q_offset, int causal, float scale, int num_splits,
+                         const attn_options* opt, void* stream);
+
+/* attn_merge with optional sink logits (device [Hq] fp32, may be NULL):
+ * M = max(max_s lse_s, sink_h), denominator sum_s w_s + exp(sink_h - M). */
+int attn_merge_ex(const float* partial_out, const float* partial_lse, void* out, float* lse,
+                  int B, int Hq, int Sq, int D, int num_splits, int out_dtype, const float* sinks,
+                  void* stream);
+
 /* Library version, e.g. 0x000100 for 0.1.0. */
 int attn_version(void);
 

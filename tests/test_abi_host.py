@@ -115,3 +115,64 @@ def test_decode_rejects(lib, kw, status):
 ])
 def test_merge_rejects(lib, args, status):
     assert lib.attn_merge(*args, None) == status
+
+
+def _opt(softcap=0.0, alibi=0.0, sinks=None, window=0):
+    return ctypes.byref(ga.AttnOptions(softcap, alibi, sinks, window))
+
+
+@pytest.mark.parametrize("opt,kw,status", [
+    (dict(softcap=-1.0), {}, ga.ATTN_ERR_INVALID_ARG),
+    (dict(softcap=float("nan")), {}, ga.ATTN_ERR_INVALID_ARG),
+    (dict(softcap=float("inf")), {}, ga.ATTN_ERR_INVALID_ARG),
+    (dict(softcap=1e-45), {}, ga.ATTN_ERR_INVALID_ARG),          # scale / softcap overflows
+    (dict(alibi=-0.5), {}, ga.ATTN_ERR_INVALID_ARG),
+    (dict(alibi=float("inf")), {}, ga.ATTN_ERR_INVALID_ARG),
+    (dict(window=-3), {}, ga.ATTN_ERR_INVALID_ARG),
+    (dict(sinks=0x20002), {}, ga.ATTN_ERR_ALIGNMENT),            # misaligned sink array
+    (dict(window=64), dict(causal=0), ga.ATTN_ERR_UNSUPPORTED),
+    (dict(window=64), dict(q_offset=1), ga.ATTN_ERR_UNSUPPORTED),  # q_offset + Sq > Skv
+    (dict(softcap=30.0), dict(q=None), ga.ATTN_ERR_INVALID_ARG),  # shape checks still apply
+    (dict(softcap=30.0), dict(D=72), ga.ATTN_ERR_UNSUPPORTED),
+])
+def test_prefill_ex_rejects(lib, opt, kw, status):
+    a = dict(q=P, k=P, v=P, out=P2, lse=P2, B=1, Hq=8, Hkv=2, Sq=128, Skv=128, D=128, q_offset=0, causal=1,
+             scale=0.125, out_dtype=0)
+    a.update(kw)
+    assert lib.attn_prefill_ex(a["q"], a["k"], a["v"], a["out"], a["lse"], a["B"], a["Hq"], a["Hkv"], a["Sq"],
+                               a["Skv"], a["D"], a["q_offset"], a["causal"], a["scale"], a["out_dtype"],
+                               _opt(**opt), None) == status
+
+
+@pytest.mark.parametrize("opt,kw,status", [
+    (dict(sinks=0x30000), {}, ga.ATTN_ERR_INVALID_ARG),  # sinks belong to the merge
+    (dict(softcap=-2.0), {}, ga.ATTN_ERR_INVALID_ARG),
+    (dict(window=-1), {}, ga.ATTN_ERR_INVALID_ARG),
+    (dict(window=128), dict(causal=0), ga.ATTN_ERR_UNSUPPORTED),
+    (dict(window=128), dict(q_offset=16384), ga.ATTN_ERR_UNSUPPORTED),
+    (dict(alibi=8.0), dict(D=96), ga.ATTN_ERR_UNSUPPORTED),
+])
+def test_decode_split_ex_rejects(lib, opt, kw, status):
+    a = dict(q=P, k=P, v=P, po=P2, pl=P2, B=16, Hq=16, Hkv=1, Sq=1, Skv=16384, D=512, q_offset=16383, causal=1,
+             scale=0.0441941738, S=32)
+    a.update(kw)
+    assert lib.attn_decode_split_ex(a["q"], a["k"], a["v"], a["po"], a["pl"], a["B"], a["Hq"], a["Hkv"],
+                                    a["Sq"], a["Skv"], a["D"], a["q_offset"], a["causal"], a["scale"], a["S"],
+                                    _opt(**opt), None) == status
+
+
+def test_merge_ex_rejects_misaligned_sinks(lib):
+    assert lib.attn_merge_ex(P, P, P2, P2, 1, 2, 3, 128, 4, 0, ctypes.c_void_p(0x30002), None) == \
+        ga.ATTN_ERR_ALIGNMENT
+    # the other checks come first, as in attn_merge
+    assert lib.attn_merge_ex(None, P, P2, P2, 1, 2, 3, 128, 4, 0, P, None) == ga.ATTN_ERR_INVALID_ARG
+
+
+def test_options_struct_matches_header():
+    """AttnOptions mirrors attn_options: float, float, pointer, int."""
+    import re
+    text = open(ga._HEADER).read()
+    body = re.search(r"typedef struct attn_options \{(.*?)\} attn_options;", text, re.S).group(1)
+    fields = [ln.strip().rstrip(";").split()[-1].lstrip("*") for ln in body.strip().splitlines()]
+    assert fields == [f[0] for f in ga.AttnOptions._fields_]
+    assert ctypes.sizeof(ga.AttnOptions) == 24
