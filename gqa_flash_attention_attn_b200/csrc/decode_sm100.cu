@@ -302,7 +302,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                         (!EXT || p.ext.window == 0 || tile0 >= p.q_offset + p.Sq - p.ext.window);
       // optional terms: logit in log2 units, softcap and ALiBi applied
       auto logit2 = [&](float sdot, int r) -> float {
-        const float z = p.ext.cap_a > 0.f ? p.ext.cap_b * tanh_via_exp2(sdot * p.ext.cap_a) : sdot * c2;
+        const float z = p.ext.cap_a > 0.f ? p.ext.cap_b * tanh_approx(sdot * p.ext.cap_a) : sdot * c2;
         return fmaf(slope_sm[r], (float)(key - pos_sm[r]), z);
       };
       auto visible = [&](int r) -> bool {

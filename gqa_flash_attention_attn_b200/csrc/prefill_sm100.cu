@@ -144,16 +144,56 @@ __device__ __forceinline__ int unit_index(int k, int total) {
   return u < total ? (int)u : -1;
 }
 
-// Logits of N consecutive keys in log2 units with the optional terms:
-// softcap (cap_b tanh(s cap_a)) or plain scaling (s c2), then the ALiBi bias
-// slope2 * (key - pos), dist0 being the first key's distance.
-template <int N>
-__device__ __forceinline__ void ext_logits(float (&v)[N], const LogitExt& x, float c2, float slope2, float dist0) {
+// Kernel variants by the optional logit terms they handle (plain runs none):
+//   MODE_MASKS  sliding window and sink logits (no per-element arithmetic)
+//   MODE_ALIBI  ALiBi bias, with or without window and sinks
+//   MODE_CAP    softcap, with or without ALiBi, window and sinks
+constexpr int MODE_PLAIN = 0, MODE_MASKS = 1, MODE_ALIBI = 2, MODE_CAP = 3;
+
+// Logits in log2 units of the N keys of a half tile whose first key sits at
+// distance dist0 = key - pos from the query:
+//   MODE_ALIBI  s c2 + slope2 (dist0 + e)
+//   MODE_CAP    cap_b tanh(s cap_a) + slope2 (dist0 + e)   (slope2 = 0: no ALiBi)
+// in packed pairs.  The ALiBi bias runs as four interleaved sums that start
+// exact at each half tile, so no per-element index arithmetic is needed.
+template <int MODE, bool BIAS, int N>
+__device__ __forceinline__ void ext_logits_run(float (&v)[N], const LogitExt& x, float c2, float slope2,
+                                               int dist0) {
+  static_assert(N % 8 == 0, "whole groups of four pairs");
+  const float b0 = slope2 * (float)dist0;
+  float2 bias[4];
 #pragma unroll
-  for (int e = 0; e < N; ++e) {
-    const float z = x.cap_a > 0.f ? x.cap_b * tanh_via_exp2(v[e] * x.cap_a) : v[e] * c2;
-    v[e] = fmaf(slope2, dist0 + (float)e, z);
+  for (int i = 0; i < 4; ++i)
+    bias[i] = make_float2(fmaf(slope2, (float)(2 * i), b0), fmaf(slope2, (float)(2 * i + 1), b0));
+  const float2 step = make_float2(8.f * slope2, 8.f * slope2);
+#pragma unroll
+  for (int e = 0; e < N; e += 2) {
+    const int i = (e >> 1) & 3;
+    const float2 sp = make_float2(v[e], v[e + 1]);
+    float2 y;
+    if constexpr (MODE == MODE_ALIBI) {
+      y = ffma2(sp, make_float2(c2, c2), bias[i]);
+    } else {
+      const float2 u = fmul2(sp, make_float2(x.cap_a, x.cap_a));
+      const float2 t = make_float2(tanh_approx(u.x), tanh_approx(u.y));
+      y = BIAS ? ffma2(t, make_float2(x.cap_b, x.cap_b), bias[i]) : fmul2(t, make_float2(x.cap_b, x.cap_b));
+    }
+    v[e] = y.x;
+    v[e + 1] = y.y;
+    if (BIAS && i == 3) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) bias[k] = fadd2(bias[k], step);
+    }
   }
+}
+
+// One branch outside the unrolled loop: neither path pays for the other.
+template <int MODE, int N>
+__device__ __forceinline__ void ext_logits(float (&v)[N], const LogitExt& x, float c2, float slope2, int dist0) {
+  if (MODE == MODE_ALIBI || x.alibi)
+    ext_logits_run<MODE, true>(v, x, c2, slope2, dist0);
+  else
+    ext_logits_run<MODE, false>(v, x, c2, slope2, dist0);
 }
 
 // Columns outside [cb, cl) become -inf.
@@ -178,7 +218,7 @@ __device__ __forceinline__ float row_max(const float (&v)[N]) {
   return fmax3(fmax3(mxc[0], mxc[1], mxc[2]), fmax3(mxc[3], mxc[4], mxc[5]), fmaxf(mxc[6], mxc[7]));
 }
 
-template <int D, bool EXT>
+template <int D, int MODE>
 __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
@@ -430,8 +470,9 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
       const int s_row = x.s0 + r;
       const int pos = p.q_offset + s_row;
       const int vis_end = p.causal ? min(p.Skv, pos + 1) : p.Skv;
-      const int vis_begin = (EXT && p.ext.window > 0) ? pos - p.ext.window + 1 : 0;
-      const float slope2 = (EXT && p.ext.alibi) ? alibi_slope_log2e(h, p.ext.l2m0, p.ext.l2m1, p.ext.n2) : 0.f;
+      const int vis_begin = (MODE != MODE_PLAIN && p.ext.window > 0) ? pos - p.ext.window + 1 : 0;
+      const float slope2 =
+          (MODE >= MODE_ALIBI && p.ext.alibi) ? alibi_slope_log2e(h, p.ext.l2m0, p.ext.l2m1, p.ext.n2) : 0.f;
       float m_use = -INFINITY, l = 0.f;
       for (int j = 0; j < n_tiles; ++j) {
         const int G = T + j;
@@ -449,18 +490,25 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
         const bool tile_masked = __any_sync(0xffffffffu, cl < BN || cb > 0);
         float sv[BN];
         float mx;
-        if constexpr (EXT) {
-          // logits in log2 units with the optional softcap and ALiBi terms;
-          // keys 64-127 first, for their maximum only, so that one half of
-          // the row is live at a time
+        if constexpr (MODE >= MODE_ALIBI) {
+          // logits in log2 units with the ALiBi / softcap terms; keys 64-127
+          // first, for their maximum only, so that one half of the row is
+          // live at a time.  Their logits go back to their own TMEM columns
+          // (P only ever covers columns 0-63), where half 1 below reads them.
           float sh[BN / 2];
           tmem_ld64(tS + BN / 2, sh);
-          ext_logits(sh, p.ext, c2, slope2, (float)(key0 + BN / 2 - pos));
+          ext_logits<MODE>(sh, p.ext, c2, slope2, key0 + BN / 2 - pos);
+          {
+            uint32_t u[BN / 2];
+#pragma unroll
+            for (int e = 0; e < BN / 2; ++e) u[e] = __float_as_uint(sh[e]);
+            tmem_st64(tS + BN / 2, u);
+          }
           if (tile_masked) mask_cols(sh, cb - BN / 2, cl - BN / 2);
           const float mx_hi = row_max(sh);
           float (&slo)[BN / 2] = *reinterpret_cast<float(*)[BN / 2]>(sv);
           tmem_ld64(tS, slo);
-          ext_logits(slo, p.ext, c2, slope2, (float)(key0 - pos));
+          ext_logits<MODE>(slo, p.ext, c2, slope2, key0 - pos);
           if (tile_masked) mask_cols(slo, cb, cl);
           mx = fmaxf(mx_hi, row_max(slo));
         } else {
@@ -469,7 +517,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
           if (tile_masked) mask_cols(sv, cb, cl);
           mx = row_max(sv);
         }
-        const float m_tile = EXT ? mx : mx * c2;
+        const float m_tile = (MODE >= MODE_ALIBI) ? mx : mx * c2;
         float m_new = m_use, alpha = 1.f;
         if (m_tile > m_use + 8.f) {
           m_new = m_tile;
@@ -499,7 +547,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
         // partial sums, bf16 pairs for the P.V operand (masked s = -inf -> p = 0).
         // P is handed over in two halves (keys 0-63, then 64-127) so the P.V
         // MMAs on the first half overlap the exponentials of the second.
-        const float2 c2v = EXT ? make_float2(1.f, 1.f) : make_float2(c2, c2);
+        const float2 c2v = (MODE >= MODE_ALIBI) ? make_float2(1.f, 1.f) : make_float2(c2, c2);
         const float2 nmv = make_float2(-m_sub, -m_sub);
         float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
         // half 0: keys 0-63 from the registers; P lands on TMEM columns 0-31,
@@ -522,8 +570,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
         // covers columns 0-63), so their registers need not stay live above
         {
           float sh[BN / 2];
-          tmem_ld64(tS + BN / 2, sh);
-          if constexpr (EXT) ext_logits(sh, p.ext, c2, slope2, (float)(key0 + BN / 2 - pos));
+          tmem_ld64(tS + BN / 2, sh);   // with ALiBi / softcap: logits stored above
           if (tile_masked) mask_cols(sh, cb - BN / 2, cl - BN / 2);
           uint32_t pk[BN / 4];
 #pragma unroll
@@ -557,7 +604,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
         // large sink logit cannot overflow: O = O_acc 2^(m - M) / l',
         // l' = l 2^(m - M) + 2^(sink - M), LSE = M + log2 l'.
         float m_fin = m_use, inv_l;
-        if (EXT && p.ext.sinks != nullptr) {
+        if (MODE != MODE_PLAIN && p.ext.sinks != nullptr) {
           const float s2 = __ldg(p.ext.sinks + h) * 1.4426950408889634f;
           m_fin = fmaxf(m_use, s2);
           const float a = ex2_approx(m_use - m_fin);
@@ -623,17 +670,17 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
   }
 }
 
-template <int D, bool EXT>
+template <int D, int MODE>
 int launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
              const PrefillParams& p, cudaStream_t stream) {
   using C = PrefillCfg<D>;
-  cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D, EXT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)C::SMEM);
   if (e != cudaSuccess) return (int)e;
   const long long units = (long long)p.n_qt * p.B * p.Hkv * p.units_per_kvh;
   if (units <= 0 || units > 0x7fffffffLL || p.num_ctas <= 0) return (int)cudaErrorInvalidValue;
   const long long grid = units < p.num_ctas ? units : p.num_ctas;  // persistent: one CTA per SM
-  prefill_kernel<D, EXT><<<(unsigned)grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, p);
+  prefill_kernel<D, MODE><<<(unsigned)grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, p);
   return (int)cudaGetLastError();
 }
 
@@ -650,12 +697,28 @@ size_t prefill_smem_bytes(int D) {
 
 int prefill_slots(int D) { return D <= 128 ? 2 : 1; }
 
+template <int D>
+int launch_mode(int mode, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                const PrefillParams& p, cudaStream_t stream) {
+  switch (mode) {
+    case MODE_PLAIN: return launch_t<D, MODE_PLAIN>(tq, tk, tv, p, stream);
+    case MODE_MASKS: return launch_t<D, MODE_MASKS>(tq, tk, tv, p, stream);
+    case MODE_ALIBI: return launch_t<D, MODE_ALIBI>(tq, tk, tv, p, stream);
+    default: return launch_t<D, MODE_CAP>(tq, tk, tv, p, stream);
+  }
+}
+
 int launch_prefill(int D, bool ext, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                    const PrefillParams& p, cudaStream_t stream) {
+  // the cheapest variant that covers the requested terms
+  const int mode = !ext ? MODE_PLAIN
+                   : p.ext.cap_a > 0.f ? MODE_CAP
+                   : p.ext.alibi ? MODE_ALIBI
+                   : MODE_MASKS;
   switch (D) {
-    case 64: return ext ? launch_t<64, true>(tq, tk, tv, p, stream) : launch_t<64, false>(tq, tk, tv, p, stream);
-    case 128: return ext ? launch_t<128, true>(tq, tk, tv, p, stream) : launch_t<128, false>(tq, tk, tv, p, stream);
-    case 256: return ext ? launch_t<256, true>(tq, tk, tv, p, stream) : launch_t<256, false>(tq, tk, tv, p, stream);
+    case 64: return launch_mode<64>(mode, tq, tk, tv, p, stream);
+    case 128: return launch_mode<128>(mode, tq, tk, tv, p, stream);
+    case 256: return launch_mode<256>(mode, tq, tk, tv, p, stream);
     default: return (int)cudaErrorInvalidValue;
   }
 }

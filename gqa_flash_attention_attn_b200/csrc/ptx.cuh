@@ -306,14 +306,24 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
   return d;
 }
 
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
 // ---------------------------------------------------- optional logit terms --
-// tanh through the identity tanh(x) = 1 - 2 / (e^(2x) + 1), with e^(2x) from
-// ex2.approx (relative error ~2^-22): accurate to ~1e-7 absolute, unlike the
-// ~5e-4 relative error of the hardware tanh approximation.
-__device__ __forceinline__ float tanh_via_exp2(float x) {
-  float e;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(x * 2.8853900817779268f));  // 2 / ln 2
-  return 1.f - __fdividef(2.f, e + 1.f);
+// The hardware tanh approximation (PTX tanh.approx.f32, one MUFU operation;
+// relative error about 2^-11).  In a softcapped logit c tanh(z / c) its error
+// is at most 2^-11 |z|, of random sign across keys.
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // ALiBi slope of head h (geometric per head; see LogitExt), times log2(e).
