@@ -24,7 +24,7 @@ __all__ = [
     "merge", "decode", "decode_workspace_bytes", "last_status", "status_string",
     "watchdog_selftest", "version", "ATTN_OK", "ATTN_ERR_INVALID_ARG", "ATTN_ERR_UNSUPPORTED",
     "ATTN_ERR_ALIGNMENT", "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT", "ATTN_ERR_TOO_LARGE", "decode_noalloc",
-    "AttnOptions",
+    "AttnOptions", "AttnKVView", "decode_split_kv", "decode_kv",
 ]
 
 ATTN_OK = 0
@@ -57,6 +57,7 @@ _SIGNATURES = {
     "attn_prefill_ex": (_i, [_vp, _vp, _vp, _vp, _vp] + [_i] * 8 + [_f, _i, _vp, _vp]),
     "attn_decode_split_ex": (_i, [_vp, _vp, _vp, _vp, _vp] + [_i] * 8 + [_f, _i, _vp, _vp]),
     "attn_merge_ex": (_i, [_vp, _vp, _vp, _vp] + [_i] * 6 + [_vp, _vp]),
+    "attn_decode_split_kv": (_i, [_vp, _vp, _vp, _vp] + [_i] * 8 + [_f, _i, _vp, _vp]),
 }
 
 
@@ -138,6 +139,42 @@ class AttnOptions(ctypes.Structure):
     """The C ``attn_options`` struct: optional logit terms (zero / NULL = off)."""
     _fields_ = [("softcap", ctypes.c_float), ("alibi_max_bias", ctypes.c_float),
                 ("sinks", ctypes.c_void_p), ("window", ctypes.c_int)]
+
+
+class AttnKVView(ctypes.Structure):
+    """The C ``attn_kv_view`` struct: a strided, optionally paged K/V cache."""
+    _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("stride_seq", ctypes.c_longlong),
+                ("stride_token", ctypes.c_longlong), ("stride_head", ctypes.c_longlong),
+                ("block_table", ctypes.c_void_p), ("max_pages", ctypes.c_int), ("page_size", ctypes.c_int),
+                ("num_pages", ctypes.c_int), ("seq_lens", ctypes.c_void_p)]
+
+
+def _kv_view(k, v, block_table, seq_lens):
+    """AttnKVView of k/v (4-D bf16 views with a contiguous last dim) and Skv.
+
+    Unpaged: k, v are [B, Skv, Hkv, D] views.  Paged: k, v are
+    [num_pages, page_size, Hkv, D] views and block_table is int32 [B, max_pages]."""
+    for t, n in ((k, "k"), (v, "v")):
+        if not isinstance(t, torch.Tensor) or t.device.type != "cuda" or t.dtype != torch.bfloat16 or t.dim() != 4:
+            raise ValueError(f"{n} must be a 4-D bf16 CUDA tensor")
+        if t.stride(3) != 1:
+            raise ValueError(f"{n} must be contiguous in its last dimension")
+    if k.shape != v.shape or k.stride() != v.stride():
+        raise ValueError("k and v must have the same shape and strides")
+    view = AttnKVView(k.data_ptr(), v.data_ptr(), k.stride(0), k.stride(1), k.stride(2), None, 0, 0, 0, None)
+    if block_table is not None:
+        _need(block_table, "block_table", torch.int32, 2)
+        view.block_table = block_table.data_ptr()
+        view.max_pages = block_table.shape[1]
+        view.page_size = k.shape[1]
+        view.num_pages = k.shape[0]
+        skv = block_table.shape[1] * k.shape[1]
+    else:
+        skv = k.shape[1]
+    if seq_lens is not None:
+        _need(seq_lens, "seq_lens", torch.int32, 1)
+        view.seq_lens = seq_lens.data_ptr()
+    return view, skv
 
 
 def _options(softcap, alibi_max_bias, sinks, window, Hq):
@@ -254,6 +291,54 @@ def decode(q, k, v, num_splits, *, causal=True, q_offset=0, scale=None, out_dtyp
     po, pl = decode_split(q, k, v, num_splits, causal=causal, q_offset=q_offset, scale=scale,
                           partial_out=po, partial_lse=pl, stream=stream, softcap=softcap,
                           alibi_max_bias=alibi_max_bias, window=window)
+    return merge(po, pl, out_dtype=out_dtype, out=out, lse=lse, stream=stream, sinks=sinks)
+
+
+def decode_split_kv(q, k, v, num_splits, *, block_table=None, seq_lens=None, causal=True, q_offset=0,
+                    scale=None, partial_out=None, partial_lse=None, stream=None, softcap=0.0,
+                    alibi_max_bias=0.0, window=0):
+    """decode_split over a strided or paged K/V cache (see attn_kv_view).
+
+    Unpaged: k, v are [B, Skv, Hkv, D] views (any strides, last dim
+    contiguous).  Paged: k, v are [num_pages, page_size, Hkv, D] and
+    block_table int32 [B, max_pages] maps logical to physical pages.
+    seq_lens (int32 [B], optional): keys per sequence; the query rows then sit
+    at the last Sq positions of each sequence and q_offset is ignored."""
+    _need(q, "q", torch.bfloat16, 4)
+    B, Sq, Hq, D = q.shape
+    view, Skv = _kv_view(k, v, block_table, seq_lens)
+    Hkv = k.shape[2]
+    if k.shape[3] != D:
+        raise ValueError("k/v head size does not match q")
+    if block_table is None and k.shape[0] != B:
+        raise ValueError("unpaged k/v must have B sequences")
+    if block_table is not None and block_table.shape[0] != B:
+        raise ValueError("block_table must have B rows")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if partial_out is None:
+        partial_out = torch.empty((num_splits, B, Sq, Hq, D), dtype=torch.float32, device=q.device)
+    if partial_lse is None:
+        partial_lse = torch.empty((num_splits, B, Hq, Sq), dtype=torch.float32, device=q.device)
+    opt = _options(softcap, alibi_max_bias, None, window, Hq)
+    st = library().attn_decode_split_kv(_ptr(q), ctypes.byref(view), _ptr(partial_out), _ptr(partial_lse), B, Hq,
+                                        Hkv, Sq, Skv, D, int(q_offset), int(bool(causal)), float(scale),
+                                        int(num_splits), None if opt is None else ctypes.byref(opt),
+                                        _stream_ptr(stream))
+    _check("attn_decode_split_kv", st)
+    return partial_out, partial_lse
+
+
+def decode_kv(q, k, v, num_splits, *, block_table=None, seq_lens=None, causal=True, q_offset=0, scale=None,
+              out_dtype=torch.bfloat16, workspace=None, out=None, lse=None, stream=None, softcap=0.0,
+              alibi_max_bias=0.0, sinks=None, window=0):
+    """decode_split_kv followed by the LSE merge (two launches on one stream)."""
+    po = pl = None
+    if workspace is not None:
+        po, pl = workspace
+    po, pl = decode_split_kv(q, k, v, num_splits, block_table=block_table, seq_lens=seq_lens, causal=causal,
+                             q_offset=q_offset, scale=scale, partial_out=po, partial_lse=pl, stream=stream,
+                             softcap=softcap, alibi_max_bias=alibi_max_bias, window=window)
     return merge(po, pl, out_dtype=out_dtype, out=out, lse=lse, stream=stream, sinks=sinks)
 
 

@@ -68,19 +68,26 @@ int* status_ptr() {
   return g_status_ptr[dev];
 }
 
-// bf16 tensor [d3][d2][d1][d0] (d0 innermost), tiled with 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t d3, uint32_t b0,
-              uint32_t b1, uint32_t b2, uint32_t b3) {
+// bf16 tensor with dimensions d0 (innermost, contiguous) .. d3 and element
+// strides s1..s3 of the outer three, tiled with 128-byte swizzle.
+bool make_map_strided(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t d3,
+                      uint64_t s1, uint64_t s2, uint64_t s3, uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
   EncodeTiledFn enc = encoder();
   if (enc == nullptr) return false;
   const cuuint64_t dims[4] = {d0, d1, d2, d3};
-  const cuuint64_t strides[3] = {d0 * 2, d0 * d1 * 2, d0 * d1 * d2 * 2};
+  const cuuint64_t strides[3] = {s1 * 2, s2 * 2, s3 * 2};
   const cuuint32_t box[4] = {b0, b1, b2, b3};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   std::memset(m, 0, sizeof(*m));
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Contiguous bf16 tensor [d3][d2][d1][d0].
+bool make_map(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t d3, uint32_t b0,
+              uint32_t b1, uint32_t b2, uint32_t b3) {
+  return make_map_strided(m, ptr, d0, d1, d2, d3, d0, d0 * d1, d0 * d1 * d2, b0, b1, b2, b3);
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -216,6 +223,26 @@ int attn_decode_split(const void* q, const void* k, const void* v, float* partia
 int attn_decode_split_ex(const void* q, const void* k, const void* v, float* partial_out, float* partial_lse,
                          int B, int Hq, int Hkv, int Sq, int Skv, int D, int q_offset, int causal, float scale,
                          int num_splits, const attn_options* opt, void* stream) {
+  // the contiguous [B, Skv, Hkv, D] view
+  attn_kv_view kv{};
+  kv.k = k;
+  kv.v = v;
+  kv.stride_head = D;
+  kv.stride_token = (long long)Hkv * D;
+  kv.stride_seq = (long long)Skv * Hkv * D;
+  return attn_decode_split_kv(q, &kv, partial_out, partial_lse, B, Hq, Hkv, Sq, Skv, D, q_offset, causal, scale,
+                              num_splits, opt, stream);
+}
+
+int attn_decode_split_kv(const void* q, const attn_kv_view* kv, float* partial_out, float* partial_lse, int B,
+                         int Hq, int Hkv, int Sq, int Skv, int D, int q_offset, int causal, float scale,
+                         int num_splits, const attn_options* opt, void* stream) {
+  if (kv == nullptr) return ATTN_ERR_INVALID_ARG;
+  const void* k = kv->k;
+  const void* v = kv->v;
+  const bool paged = kv->block_table != nullptr;
+  // with per-sequence lengths q_offset is ignored (rows sit at len_b - Sq + s)
+  if (kv->seq_lens != nullptr) q_offset = 0;
   int st = check_common(q, k, v, B, Hq, Hkv, Sq, Skv, D, q_offset, causal, scale);
   if (st != ATTN_OK) return st;
   gqa::LogitExt ext;
@@ -231,8 +258,22 @@ int attn_decode_split_ex(const void* q, const void* k, const void* v, float* par
   if (RP * (2 + D / 128) > 256) return ATTN_ERR_UNSUPPORTED;  // TMEM: two S^T buffers + O^T
   if (g > 256 || Sq > 256) return ATTN_ERR_UNSUPPORTED;  // TMA box extents
   if ((long long)B * Hkv > 65535) return ATTN_ERR_INVALID_ARG;
+  // the view: strides positive, below 2^37 elements, 16-byte multiples
+  const long long strides[3] = {kv->stride_head, kv->stride_token, kv->stride_seq};
+  for (long long x : strides)
+    if (x < 1 || x >= (1LL << 37)) return ATTN_ERR_INVALID_ARG;
+  if (paged) {
+    const int ps = kv->page_size;
+    if (!(ps == 16 || ps == 32 || ps == 64 || (ps >= 128 && ps % 128 == 0))) return ATTN_ERR_INVALID_ARG;
+    if (kv->max_pages < 1 || kv->num_pages < 1) return ATTN_ERR_INVALID_ARG;
+    if ((long long)kv->max_pages * ps != Skv) return ATTN_ERR_INVALID_ARG;
+    if (!aligned(kv->block_table, 4)) return ATTN_ERR_ALIGNMENT;
+  }
+  if (kv->seq_lens != nullptr && !aligned(kv->seq_lens, 4)) return ATTN_ERR_ALIGNMENT;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(partial_out, 16))
     return ATTN_ERR_ALIGNMENT;
+  for (long long x : strides)
+    if (x % 8 != 0) return ATTN_ERR_ALIGNMENT;
   if (!aligned(partial_lse, 4)) return ATTN_ERR_ALIGNMENT;
 
   gqa::DecodeParams p{};
@@ -249,13 +290,22 @@ int attn_decode_split_ex(const void* q, const void* k, const void* v, float* par
   p.c2 = scale * kLog2e;
   p.timeout_ns = kWaitLimitNs;
   p.ext = ext;
+  p.seq_lens = kv->seq_lens;
+  p.block_table = kv->block_table;
+  p.max_pages = paged ? kv->max_pages : 0;
+  p.page_size = paged ? kv->page_size : 0;
 
   p.status = status_ptr();
   if (p.status == nullptr) return cuda_fail();
   CUtensorMap tq, tk, tv;
   if (!make_map(&tq, q, D, Hq, Sq, B, 64, (uint32_t)g, (uint32_t)Sq, 1)) return cuda_fail();
-  if (!make_map(&tk, k, D, Hkv, Skv, B, 64, 1, 128, 1)) return cuda_fail();
-  if (!make_map(&tv, v, D, Hkv, Skv, B, 64, 1, 128, 1)) return cuda_fail();
+  // K/V: (d, kvh, key, sequence) unpaged, (d, kvh, row in page, page) paged
+  const uint64_t d2 = paged ? (uint64_t)kv->page_size : (uint64_t)Skv;
+  const uint64_t d3 = paged ? (uint64_t)kv->num_pages : (uint64_t)B;
+  const uint32_t rows = paged && kv->page_size < 128 ? (uint32_t)kv->page_size : 128u;
+  const uint64_t s1 = (uint64_t)kv->stride_head, s2 = (uint64_t)kv->stride_token, s3 = (uint64_t)kv->stride_seq;
+  if (!make_map_strided(&tk, k, D, Hkv, d2, d3, s1, s2, s3, 64, 1, rows, 1)) return cuda_fail();
+  if (!make_map_strided(&tv, v, D, Hkv, d2, d3, s1, s2, s3, 64, 1, rows, 1)) return cuda_fail();
   return gqa::launch_decode_split(D, ext_on, tq, tk, tv, p, static_cast<cudaStream_t>(stream)) == 0 ? ATTN_OK
                                                                                                : ATTN_ERR_CUDA;
 }

@@ -119,12 +119,23 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = blockIdx.x;
   const int b = blockIdx.y / p.Hkv, kvh = blockIdx.y % p.Hkv;
-  const long long lo_ll = (long long)split * p.chunk;
-  const int lo = (int)min(lo_ll, (long long)p.Skv);
-  const int hi = (int)min(lo_ll + p.chunk, (long long)p.Skv);
-  const int eff_hi = p.causal ? min(hi, p.q_offset + p.Sq) : hi;
+  // this sequence's keys and the position of its first query row
+  int Skv = p.Skv, q_offset = p.q_offset;
+  long long chunk = p.chunk;
+  if (p.seq_lens != nullptr) {
+    const int len = __ldg(p.seq_lens + b);
+    Skv = min(max(len, 0), p.Skv);
+    if (Skv != len && split == 0 && kvh == 0 && threadIdx.x == 0) atomicCAS(p.status, kStatusOk, kStatusInvalidArg);
+    q_offset = Skv - p.Sq;
+    chunk = (Skv + p.num_splits - 1) / p.num_splits;
+  }
+  if (p.block_table != nullptr) chunk = (chunk + BN - 1) / BN * BN;  // no tile crosses a page
+  const long long lo_ll = (long long)split * chunk;
+  const int lo = (int)min(lo_ll, (long long)Skv);
+  const int hi = (int)min(lo_ll + chunk, (long long)Skv);
+  const int eff_hi = p.causal ? (int)min((long long)hi, (long long)q_offset + p.Sq) : hi;
   // a sliding window hides every key at or before q_offset - window from all rows
-  const int eff_lo = (EXT && p.ext.window > 0) ? max(lo, p.q_offset - p.ext.window + 1) : lo;
+  const int eff_lo = (EXT && p.ext.window > 0) ? max(lo, q_offset - p.ext.window + 1) : lo;
   const int kbase = lo + ((eff_lo - lo) / BN) * BN;   // first tile, on the split's tile grid
   const int n_tiles = eff_hi > eff_lo ? (eff_hi - kbase + BN - 1) / BN : 0;
   const size_t split_out = (size_t)split * p.B * p.Sq * p.Hq * D;
@@ -155,8 +166,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     m_sm[r] = -INFINITY;
     l_sm[r] = 0.f;
     // last visible key of row r (padding rows see none)
-    lim_sm[r] = r < R ? (p.causal ? p.q_offset + r / g : 0x7fffffff) : -1;
-    pos_sm[r] = p.q_offset + (r < R ? r / g : 0);
+    lim_sm[r] = r < R ? (p.causal ? q_offset + r / g : 0x7fffffff) : -1;
+    pos_sm[r] = q_offset + (r < R ? r / g : 0);
     limlo_sm[r] = (EXT && p.ext.window > 0) ? pos_sm[r] - p.ext.window : -1;
     slope_sm[r] = (EXT && p.ext.alibi && r < R)
                       ? alibi_slope_log2e(kvh * g + (r - (r / g) * g), p.ext.l2m0, p.ext.l2m1, p.ext.n2)
@@ -216,8 +227,25 @@ __global__ void __launch_bounds__(THREADS, 1)
           mbar_arrive_expect_tx(bar(bar_full(slot)), SLOT_BYTES);
           const uint32_t dst = base + L.off_ring + (uint32_t)slot * SLOT_BYTES;
           const int key0 = kbase + j * BN;
-          tma_load_4d(dst, tm, bar(bar_full(slot)), (2 * c) * 64, kvh, key0, b);
-          tma_load_4d(dst + BOX_BYTES, tm, bar(bar_full(slot)), (2 * c + 1) * 64, kvh, key0, b);
+          if (p.block_table == nullptr) {
+            tma_load_4d(dst, tm, bar(bar_full(slot)), (2 * c) * 64, kvh, key0, b);
+            tma_load_4d(dst + BOX_BYTES, tm, bar(bar_full(slot)), (2 * c + 1) * 64, kvh, key0, b);
+          } else {
+            // paged: each page-sized run of keys from its physical page (the
+            // tensor map's outer dimensions are row-in-page and page); a
+            // logical page past the table reads as zeros (page -1)
+            const int* bt = p.block_table + (size_t)b * p.max_pages;
+            const int ps = p.page_size, rows = ps < BN ? ps : BN;
+            for (int sub = 0; sub < BN / rows; ++sub) {
+              const int key = key0 + sub * rows;
+              const int lp = key / ps;
+              const int page = lp < p.max_pages ? __ldg(bt + lp) : -1;
+              const uint32_t off = (uint32_t)(sub * rows) * 128u;
+              tma_load_4d(dst + off, tm, bar(bar_full(slot)), (2 * c) * 64, kvh, key - lp * ps, page);
+              tma_load_4d(dst + BOX_BYTES + off, tm, bar(bar_full(slot)), (2 * c + 1) * 64, kvh, key - lp * ps,
+                          page);
+            }
+          }
           issued = n + 1;
         }
       };
@@ -298,8 +326,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int tile0 = kbase + j * BN;
       const int key = tile0 + t;
       // whole tile visible to every real row: no per-element mask
-      const bool full = (tile0 + BN - 1 < hi) && (!p.causal || tile0 + BN - 1 <= p.q_offset) &&
-                        (!EXT || p.ext.window == 0 || tile0 >= p.q_offset + p.Sq - p.ext.window);
+      const bool full = (tile0 + BN - 1 < hi) && (!p.causal || tile0 + BN - 1 <= q_offset) &&
+                        (!EXT || p.ext.window == 0 || tile0 >= q_offset + p.Sq - p.ext.window);
       // optional terms: logit in log2 units, softcap and ALiBi applied
       auto logit2 = [&](float sdot, int r) -> float {
         const float z = p.ext.cap_a > 0.f ? p.ext.cap_b * tanh_approx(sdot * p.ext.cap_a) : sdot * c2;

@@ -45,6 +45,10 @@ struct DecodeParams {
   float c2;
   unsigned long long timeout_ns;
   LogitExt ext;       // sinks unused: the merge adds them
+  // K/V view: per-sequence lengths and paging (both optional)
+  const int* seq_lens;     // [B] or nullptr: every sequence has Skv keys
+  const int* block_table;  // [B, max_pages] or nullptr: unpaged
+  int max_pages, page_size;
 };
 
 struct MergeParams {

@@ -13,6 +13,7 @@ namespace gqa {
 // ---------------------------------------------------------------- status ----
 enum : int {
   kStatusOk = 0,
+  kStatusInvalidArg = -1,   // a device-side argument (a sequence length) was out of range
   kStatusTimeout = -5,
 };
 

@@ -141,6 +141,35 @@ def make_sinks(Hq, *, seed=0, std=3.0, device="cpu"):
     return torch.randn((Hq,), generator=gen, dtype=torch.float32, device=device) * std
 
 
+def make_paged(k, v, page_size, *, seed=0, extra_pages=3):
+    """Scatter contiguous k, v [B, Skv, Hkv, D] into a paged cache.
+
+    Returns (k_cache, v_cache, block_table): caches [num_pages, page_size, Hkv, D]
+    with num_pages = B * ceil(Skv / page_size) + extra_pages, logical page j of
+    sequence b stored at physical page block_table[b, j] (a seeded random
+    permutation; the extra pages hold unrelated random rows), and the unused
+    tail of each sequence's last page filled with random rows too."""
+    B, Skv, Hkv, D = k.shape
+    mp = (Skv + page_size - 1) // page_size
+    n = B * mp + extra_pages
+    gen = torch.Generator().manual_seed(seed)
+    perm = torch.randperm(n, generator=gen)[: B * mp].reshape(B, mp).to(torch.int32)
+    kc = torch.randn((n, page_size, Hkv, D), generator=gen).to(k.dtype)
+    vc = torch.randn((n, page_size, Hkv, D), generator=gen).to(v.dtype)
+    for b in range(B):
+        for j in range(mp):
+            t0, t1 = j * page_size, min(Skv, (j + 1) * page_size)
+            kc[perm[b, j], : t1 - t0] = k[b, t0:t1]
+            vc[perm[b, j], : t1 - t0] = v[b, t0:t1]
+    return kc, vc, perm
+
+
+def make_seq_lens(B, Skv, *, seed=0, low=1):
+    """Seeded per-sequence key counts, uniform in [low, Skv], int32 [B]."""
+    gen = torch.Generator().manual_seed(seed)
+    return torch.randint(low, Skv + 1, (B,), generator=gen, dtype=torch.int64).to(torch.int32)
+
+
 def make_workload_inputs(w: Workload, *, seed=0, device="cpu"):
     return make_qkv(w.B, w.Hq, w.Hkv, w.Sq, w.Skv, w.D, seed=seed, device=device)
 

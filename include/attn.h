@@ -211,6 +211,60 @@ int attn_merge_ex(const float* partial_out, const float* partial_lse, void* out,
                   int B, int Hq, int Sq, int D, int num_splits, int out_dtype, const float* sinks,
                   void* stream);
 
+/*
+ * A K/V cache view for decode: strided, optionally paged, optionally with a
+ * length per sequence (paged K/V as in the paged indexer of the
+ * "amd-sriram/vllm PR #32" Validation section; strided K/V views as in the
+ * kv_view and permute parameters of the FLASH_ATTN_EXT test cases in
+ * "ggml-org/llama.cpp PR #28507", Crash 1).  All strides are in elements,
+ * D is innermost and contiguous.
+ *
+ * Unpaged (block_table == NULL): key t of sequence b, K/V head kvh is at
+ *   k + b*stride_seq + t*stride_token + kvh*stride_head   (same for v)
+ * for t < Skv.
+ * Paged: logical page j of sequence b is physical page block_table[b*max_pages + j];
+ * key t of sequence b is row t % page_size of page block_table[b*max_pages + t / page_size]:
+ *   k + page*stride_seq + (t % page_size)*stride_token + kvh*stride_head
+ * with 0 <= page < num_pages.  page_size is 16, 32, 64 or a multiple of 128;
+ * Skv must equal max_pages * page_size.  A physical page index outside
+ * [0, num_pages) reads as zeros (never out of bounds).
+ *
+ * seq_lens (device [B] int32, or NULL): sequence b has min(seq_lens[b], Skv)
+ * keys and its Sq query rows sit at positions len_b - Sq + s (q_offset is
+ * ignored); rows at a negative position see no key.  A negative or too large
+ * length is clamped to [0, Skv] and sets ATTN_ERR_INVALID_ARG in the device
+ * status word (see attn_last_status).  Without seq_lens every sequence has Skv
+ * keys and q_offset applies.
+ *
+ * Alignment: k, v 16-byte aligned; stride_seq, stride_token and stride_head
+ * multiples of 8 elements (16 bytes) and each below 2^37 elements, else
+ * ATTN_ERR_ALIGNMENT / ATTN_ERR_INVALID_ARG.  The caller owns every buffer.
+ */
+typedef struct attn_kv_view {
+  const void* k;            /* bf16 */
+  const void* v;            /* bf16 */
+  long long stride_seq;     /* between sequences (unpaged) or pages (paged) */
+  long long stride_token;   /* between consecutive keys */
+  long long stride_head;    /* between K/V heads */
+  const int* block_table;   /* device [B, max_pages], or NULL: unpaged */
+  int max_pages;            /* columns of block_table */
+  int page_size;            /* keys per page */
+  int num_pages;            /* physical pages in the cache */
+  const int* seq_lens;      /* device [B], or NULL */
+} attn_kv_view;
+
+/*
+ * attn_decode_split over a K/V view (optional logit terms in *opt, which may
+ * be NULL; sinks belong to attn_merge_ex).  Splits: chunk = ceil(len_b /
+ * num_splits) keys of sequence b per split, rounded up to a multiple of 128
+ * when paged so that no 128-key tile crosses a page; splits past the end
+ * publish lse = -inf and O = 0.  Other arguments, limits and errors as in
+ * attn_decode_split.
+ */
+int attn_decode_split_kv(const void* q, const attn_kv_view* kv, float* partial_out, float* partial_lse,
+                         int B, int Hq, int Hkv, int Sq, int Skv, int D, int q_offset, int causal,
+                         float scale, int num_splits, const attn_options* opt, void* stream);
+
 /* Library version, e.g. 0x000100 for 0.1.0. */
 int attn_version(void);
 

@@ -176,3 +176,51 @@ def test_options_struct_matches_header():
     fields = [ln.strip().rstrip(";").split()[-1].lstrip("*") for ln in body.strip().splitlines()]
     assert fields == [f[0] for f in ga.AttnOptions._fields_]
     assert ctypes.sizeof(ga.AttnOptions) == 24
+
+
+def _kv_decode(lib, view=None, **kw):
+    a = dict(q=P, po=P2, pl=P2, B=2, Hq=16, Hkv=1, Sq=1, Skv=1024, D=512, q_offset=1023, causal=1,
+             scale=0.0441941738, S=4)
+    a.update(kw)
+    if view is None:
+        view = {}
+    vw = dict(k=0x40000, v=0x50000, stride_seq=1024 * 512, stride_token=512, stride_head=512, block_table=None,
+              max_pages=0, page_size=0, num_pages=0, seq_lens=None)
+    vw.update(view)
+    v = ga.AttnKVView(**vw)
+    return lib.attn_decode_split_kv(a["q"], ctypes.byref(v), a["po"], a["pl"], a["B"], a["Hq"], a["Hkv"], a["Sq"],
+                                    a["Skv"], a["D"], a["q_offset"], a["causal"], a["scale"], a["S"], None, None)
+
+
+@pytest.mark.parametrize("view,kw,status", [
+    (dict(k=None), {}, ga.ATTN_ERR_INVALID_ARG),
+    (dict(stride_token=0), {}, ga.ATTN_ERR_INVALID_ARG),
+    (dict(stride_seq=-512), {}, ga.ATTN_ERR_INVALID_ARG),
+    (dict(stride_head=1 << 37), {}, ga.ATTN_ERR_INVALID_ARG),
+    (dict(stride_token=516), {}, ga.ATTN_ERR_ALIGNMENT),             # 1032 bytes: not a 16-byte multiple
+    (dict(v=0x50008), {}, ga.ATTN_ERR_ALIGNMENT),
+    (dict(seq_lens=0x60002), {}, ga.ATTN_ERR_ALIGNMENT),
+    (dict(block_table=0x70000, max_pages=8, page_size=100, num_pages=64), {}, ga.ATTN_ERR_INVALID_ARG),
+    (dict(block_table=0x70000, max_pages=8, page_size=8, num_pages=64), dict(Skv=64), ga.ATTN_ERR_INVALID_ARG),
+    (dict(block_table=0x70000, max_pages=4, page_size=128, num_pages=64), {}, ga.ATTN_ERR_INVALID_ARG),  # 4*128 != Skv
+    (dict(block_table=0x70000, max_pages=0, page_size=128, num_pages=64), {}, ga.ATTN_ERR_INVALID_ARG),
+    (dict(block_table=0x70000, max_pages=8, page_size=128, num_pages=0), dict(Skv=1024), ga.ATTN_ERR_INVALID_ARG),
+    (dict(block_table=0x70002, max_pages=8, page_size=128, num_pages=64), dict(Skv=1024), ga.ATTN_ERR_ALIGNMENT),
+    ({}, dict(D=64), ga.ATTN_ERR_UNSUPPORTED),
+])
+def test_decode_split_kv_rejects(lib, view, kw, status):
+    assert _kv_decode(lib, view, **kw) == status
+
+
+def test_decode_split_kv_rejects_null_view(lib):
+    assert lib.attn_decode_split_kv(P, None, P2, P2, 1, 8, 1, 1, 128, 128, 127, 1, 0.08, 1, None, None) == \
+        ga.ATTN_ERR_INVALID_ARG
+
+
+def test_kv_view_struct_matches_header():
+    import re
+    text = open(ga._HEADER).read()
+    body = re.search(r"typedef struct attn_kv_view \{(.*?)\} attn_kv_view;", text, re.S).group(1)
+    fields = [ln.split(";")[0].split()[-1].lstrip("*") for ln in body.strip().splitlines() if ";" in ln]
+    assert fields == [f[0] for f in ga.AttnKVView._fields_]
+    assert ctypes.sizeof(ga.AttnKVView) == 72
