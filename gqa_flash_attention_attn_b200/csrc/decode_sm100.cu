@@ -81,7 +81,7 @@ __device__ __forceinline__ float warp_reduce16(float (&v)[16], int lane) {
   return kMax ? fmaxf(v[0], other) : v[0] + other;
 }
 
-template <int D, bool EXT>
+template <int D, bool EXT, bool PAGED>
 __global__ void __launch_bounds__(THREADS, 1)
     decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
@@ -129,7 +129,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     q_offset = Skv - p.Sq;
     chunk = (Skv + p.num_splits - 1) / p.num_splits;
   }
-  if (p.block_table != nullptr) chunk = (chunk + BN - 1) / BN * BN;  // no tile crosses a page
+  if (PAGED) chunk = (chunk + BN - 1) / BN * BN;  // no tile crosses a page
   const long long lo_ll = (long long)split * chunk;
   const int lo = (int)min(lo_ll, (long long)Skv);
   const int hi = (int)min(lo_ll + chunk, (long long)Skv);
@@ -227,7 +227,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           mbar_arrive_expect_tx(bar(bar_full(slot)), SLOT_BYTES);
           const uint32_t dst = base + L.off_ring + (uint32_t)slot * SLOT_BYTES;
           const int key0 = kbase + j * BN;
-          if (p.block_table == nullptr) {
+          if constexpr (!PAGED) {
             tma_load_4d(dst, tm, bar(bar_full(slot)), (2 * c) * 64, kvh, key0, b);
             tma_load_4d(dst + BOX_BYTES, tm, bar(bar_full(slot)), (2 * c + 1) * 64, kvh, key0, b);
           } else {
@@ -474,16 +474,24 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-template <int D, bool EXT>
+template <int D, bool EXT, bool PAGED>
 int launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
              const DecodeParams& p, cudaStream_t stream) {
   const Layout L(D, p.RP, p.nbuf);
-  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, EXT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)L.total);
+  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, EXT, PAGED>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
   if (e != cudaSuccess) return (int)e;
   dim3 grid((unsigned)p.num_splits, (unsigned)(p.B * p.Hkv));
-  decode_split_kernel<D, EXT><<<grid, THREADS, L.total, stream>>>(tq, tk, tv, p);
+  decode_split_kernel<D, EXT, PAGED><<<grid, THREADS, L.total, stream>>>(tq, tk, tv, p);
   return (int)cudaGetLastError();
+}
+
+template <int D>
+int launch_d(bool ext, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+             const DecodeParams& p, cudaStream_t stream) {
+  const bool paged = p.block_table != nullptr;
+  if (ext) return paged ? launch_t<D, true, true>(tq, tk, tv, p, stream) : launch_t<D, true, false>(tq, tk, tv, p, stream);
+  return paged ? launch_t<D, false, true>(tq, tk, tv, p, stream) : launch_t<D, false, false>(tq, tk, tv, p, stream);
 }
 
 }  // namespace
@@ -495,9 +503,9 @@ int decode_max_nbuf() { return MAX_NBUF; }
 int launch_decode_split(int D, bool ext, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                         const DecodeParams& p, cudaStream_t stream) {
   switch (D) {
-    case 128: return ext ? launch_t<128, true>(tq, tk, tv, p, stream) : launch_t<128, false>(tq, tk, tv, p, stream);
-    case 256: return ext ? launch_t<256, true>(tq, tk, tv, p, stream) : launch_t<256, false>(tq, tk, tv, p, stream);
-    case 512: return ext ? launch_t<512, true>(tq, tk, tv, p, stream) : launch_t<512, false>(tq, tk, tv, p, stream);
+    case 128: return launch_d<128>(ext, tq, tk, tv, p, stream);
+    case 256: return launch_d<256>(ext, tq, tk, tv, p, stream);
+    case 512: return launch_d<512>(ext, tq, tk, tv, p, stream);
     default: return (int)cudaErrorInvalidValue;
   }
 }

@@ -38,6 +38,9 @@ class Workload:
     alibi_max_bias: float = 0.0
     sinks: bool = False
     window: int = 0
+    # K/V cache layout: 0 = contiguous [B, Skv, Hkv, D]; else paged with this
+    # many keys per page (pages scattered by make_paged(k, v, page_size, seed=0))
+    page_size: int = 0
 
     @property
     def has_options(self) -> bool:
@@ -118,6 +121,10 @@ WORKLOADS = {
         "split_kv_decode_d512_softcap_alibi_sinks", "decode", B=16, Hq=16, Hkv=1, Sq=1, Skv=16384, D=512,
         q_offset=16383, causal=True, out_dtype="bf16", num_splits=32, softcap=30.0, alibi_max_bias=8.0,
         sinks=True, note="the D512 split-KV decode with softcap 30, ALiBi (max bias 8) and sinks in the merge"),
+    "paged_decode_d512_p64": Workload(
+        "paged_decode_d512_p64", "decode", B=16, Hq=16, Hkv=1, Sq=1, Skv=16384, D=512,
+        q_offset=16383, causal=True, out_dtype="bf16", num_splits=32, page_size=64,
+        note="the D512 split-KV decode over a paged cache: 64-key pages in scattered order"),
 }
 
 

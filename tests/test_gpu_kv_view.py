@@ -144,3 +144,21 @@ def test_pages_outside_the_cache_read_as_zeros():
     want_o, want_l = oracle.attention(q, kz, vz, scale=_scale(D), causal=True, q_offset=Skv - Sq)
     assert_o_close(out, want_o, "zero pages")
     assert_lse_close(lse, want_l, "zero pages")
+
+
+def test_paged_workload_full_size_sampled():
+    """The timed paged-decode workload, in its timed launch configuration."""
+    from gqa_flash_attention_attn_b200.inputs import WORKLOADS, make_workload_inputs, sample_rows
+    from parity import gather_rows, oracle_rows_by_batch
+    w = WORKLOADS["paged_decode_d512_p64"]
+    q, k, v = make_workload_inputs(w, seed=0)
+    kc, vc, bt = make_paged(k, v, w.page_size, seed=0)
+    out, lse = ga.decode_kv(q.cuda(), kc.cuda(), vc.cuda(), w.num_splits, block_table=bt.cuda(),
+                            causal=w.causal, q_offset=w.q_offset, scale=w.scale)
+    torch.cuda.synchronize()
+    assert ga.last_status() == ga.ATTN_OK
+    rows = sample_rows(w, 40, seed=23)
+    got_o, got_l = gather_rows(out, lse, rows)
+    want_o, want_l = oracle_rows_by_batch(q, k, v, rows, scale=w.scale, causal=w.causal, q_offset=w.q_offset)
+    assert_o_close(got_o, want_o, w.name)
+    assert_lse_close(got_l, want_l, w.name)
