@@ -23,7 +23,7 @@ Functions and the passage each follows (all pinned by tests/test_oracle_pins.py)
                   combine kernel for parallel_blocks > 1)
   *_ex            the same with the optional logit terms of the FLASH_ATTN_EXT
                   operator ("ggml-org/llama.cpp PR #28507", Crash 1: sinks,
-                  max_bias, logit_softcap) and a sliding window (see oracle.c)
+                  max_bias, logit_softcap, mask) and a sliding window (see oracle.c)
 """
 from __future__ import annotations
 
@@ -83,14 +83,15 @@ def _bind(lib):
     lib.oracle_merge.restype = None
     lib.oracle_num_threads.argtypes = []
     lib.oracle_num_threads.restype = ctypes.c_int
-    ext = [ctypes.c_double, ctypes.c_double, _dp, _i64]
+    msk = [_dp, _i64, _i64]
+    ext = [ctypes.c_double, ctypes.c_double, _dp, _i64] + msk
     lib.oracle_attention_ex.argtypes = [_dp, _dp, _dp, _dp, _dp] + [_i64] * 7 + [ctypes.c_int, ctypes.c_double] + ext
     lib.oracle_attention_ex.restype = None
     lib.oracle_attention_rows_ex.argtypes = ([_dp, _dp, _dp, _lp, _i64, _dp, _dp] + [_i64] * 7 +
                                              [ctypes.c_int, ctypes.c_double] + ext)
     lib.oracle_attention_rows_ex.restype = None
     lib.oracle_split_ex.argtypes = ([_dp, _dp, _dp, _dp, _dp] + [_i64] * 7 + [ctypes.c_int, ctypes.c_double, _i64] +
-                                    [ctypes.c_double, ctypes.c_double, _i64])
+                                    [ctypes.c_double, ctypes.c_double, _i64] + msk)
     lib.oracle_split_ex.restype = None
     lib.oracle_merge_ex.argtypes = [_dp, _dp, _dp, _dp] + [_i64] * 5 + [_dp]
     lib.oracle_merge_ex.restype = None
@@ -194,52 +195,71 @@ def _sinks_arg(sinks):
     return arr, _ptr(arr)
 
 
+def _mask_arg(mask, B, Sq, Skv):
+    """An additive mask [Sq, Skv], [1, Sq, Skv] or [B, Sq, Skv] as a float64
+    array with its batch and row strides (batch stride 0: shared)."""
+    if mask is None:
+        return None, None, 0, 0
+    arr = _f64(mask)
+    if arr.ndim == 2:
+        arr = arr[None]
+    if arr.shape[1:] != (Sq, Skv) or arr.shape[0] not in (1, B):
+        raise ValueError(f"mask must be [B or 1, {Sq}, {Skv}]")
+    arr = np.ascontiguousarray(arr)
+    return arr, _ptr(arr), (Sq * Skv if arr.shape[0] == B and B > 1 else 0), Skv
+
+
 def alibi_slope(h, Hq, max_bias, lib=None):
     return (lib or load()).oracle_alibi_slope(int(h), int(Hq), float(max_bias))
 
 
 def attention_ex(q, k, v, *, scale, causal=True, q_offset=0, softcap=0.0, alibi_max_bias=0.0, sinks=None,
-                 window=0, lib=None):
-    """attention() with softcap, ALiBi, sink logits [Hq] and a sliding window."""
+                 window=0, mask=None, lib=None):
+    """attention() with softcap, ALiBi, sink logits [Hq], a sliding window and
+    an additive mask [B or 1, Sq, Skv]."""
     lib = lib or load()
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, Hq, Hkv, Sq, Skv, D = _dims(q, k)
     sk, skp = _sinks_arg(sinks)
+    mk, mkp, msb, mss = _mask_arg(mask, B, Sq, Skv)
     out = np.zeros((B, Sq, Hq, D), dtype=np.float64)
     lse = np.zeros((B, Hq, Sq), dtype=np.float64)
     lib.oracle_attention_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Skv, D,
                             int(q_offset), int(bool(causal)), float(scale), float(softcap),
-                            float(alibi_max_bias), skp, int(window))
+                            float(alibi_max_bias), skp, int(window), mkp, msb, mss)
     return out, lse
 
 
 def attention_rows_ex(q, k, v, rows, *, scale, causal=True, q_offset=0, softcap=0.0, alibi_max_bias=0.0,
-                      sinks=None, window=0, lib=None):
+                      sinks=None, window=0, mask=None, lib=None):
     lib = lib or load()
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, Hq, Hkv, Sq, Skv, D = _dims(q, k)
     rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
     n = rows.shape[0]
     sk, skp = _sinks_arg(sinks)
+    mk, mkp, msb, mss = _mask_arg(mask, B, Sq, Skv)
     out = np.zeros((n, D), dtype=np.float64)
     lse = np.zeros((n,), dtype=np.float64)
     lib.oracle_attention_rows_ex(_ptr(q), _ptr(k), _ptr(v), rows.ctypes.data_as(_lp), n, _ptr(out), _ptr(lse),
                                  B, Hq, Hkv, Sq, Skv, D, int(q_offset), int(bool(causal)), float(scale),
-                                 float(softcap), float(alibi_max_bias), skp, int(window))
+                                 float(softcap), float(alibi_max_bias), skp, int(window), mkp, msb, mss)
     return out, lse
 
 
 def split_ex(q, k, v, num_splits, *, scale, causal=True, q_offset=0, softcap=0.0, alibi_max_bias=0.0,
-             window=0, lib=None):
-    """split() with softcap, ALiBi and a window (sinks belong to the merge)."""
+             window=0, mask=None, lib=None):
+    """split() with softcap, ALiBi, a window and an additive mask (sinks belong
+    to the merge)."""
     lib = lib or load()
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, Hq, Hkv, Sq, Skv, D = _dims(q, k)
+    mk, mkp, msb, mss = _mask_arg(mask, B, Sq, Skv)
     pout = np.zeros((num_splits, B, Sq, Hq, D), dtype=np.float64)
     plse = np.zeros((num_splits, B, Hq, Sq), dtype=np.float64)
     lib.oracle_split_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(pout), _ptr(plse), B, Hq, Hkv, Sq, Skv, D,
                         int(q_offset), int(bool(causal)), float(scale), int(num_splits), float(softcap),
-                        float(alibi_max_bias), int(window))
+                        float(alibi_max_bias), int(window), mkp, msb, mss)
     return pout, plse
 
 

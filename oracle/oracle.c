@@ -52,6 +52,10 @@
  *                       (and in the LSE), with no value row
  *   window w > 0:       key t is visible only if pos - w < t (with causal,
  *                       each row sees its w most recent keys)
+ *   additive mask M:    z_t += M[b, s, t] (the `mask` parameter of the same
+ *                       test case; -inf removes the key), after softcap and
+ *                       ALiBi; a row whose every logit is -inf, with no
+ *                       sink, has O = 0 and LSE = -inf
  */
 #include <math.h>
 #include <stdint.h>
@@ -75,6 +79,9 @@ typedef struct {
     double alibi_max_bias;  /* 0: off */
     const double* sinks;    /* NULL: off; else [Hq] sink logits */
     int64_t window;         /* 0: off */
+    const double* mask;     /* NULL: off; else additive mask, element (b, s, t) at */
+    int64_t mask_sb;        /*   mask[b * mask_sb + s * mask_ss + t] (mask_sb = 0: */
+    int64_t mask_ss;        /*   one mask for every sequence) */
 } oracle_opts;
 
 /* ALiBi slope of head h out of Hq (see the header comment). */
@@ -119,8 +126,11 @@ static double attend_row(const double* q, const double* k, const double* v,
         const double zt = scale * acc;
         const double zc = softcap > 0.0 ? softcap * tanh(zt / softcap) : zt;
         z[t - t_lo] = zc + slope * (double)(t - pos);
+        if (opt && opt->mask) z[t - t_lo] += opt->mask[b * opt->mask_sb + s * opt->mask_ss + t];
         if (z[t - t_lo] > m) m = z[t - t_lo];
     }
+    /* every visible logit masked to -inf and no sink: no key takes part */
+    if (m == -INFINITY) return -INFINITY;
     /* pass 2: exponentials, their sum, and the weighted sum of V rows */
     double l = has_sink ? exp(opt->sinks[h] - m) : 0.0;
     for (int64_t t = first; t < last; ++t) {
@@ -300,20 +310,25 @@ void oracle_merge(const double* pout, const double* plse, double* out, double* l
     merge_impl(pout, plse, out, lse, B, Hq, Sq, D, num_splits, NULL);
 }
 
-static oracle_opts make_opts(double softcap, double alibi_max_bias, const double* sinks, int64_t window) {
+static oracle_opts make_opts(double softcap, double alibi_max_bias, const double* sinks, int64_t window,
+                             const double* mask, int64_t mask_sb, int64_t mask_ss) {
     oracle_opts o;
     o.softcap = softcap;
     o.alibi_max_bias = alibi_max_bias;
     o.sinks = sinks;
     o.window = window;
+    o.mask = mask;
+    o.mask_sb = mask_sb;
+    o.mask_ss = mask_ss;
     return o;
 }
 
 void oracle_attention_ex(const double* q, const double* k, const double* v, double* out, double* lse,
                          int64_t B, int64_t Hq, int64_t Hkv, int64_t Sq, int64_t Skv, int64_t D,
                          int64_t q_offset, int causal, double scale,
-                         double softcap, double alibi_max_bias, const double* sinks, int64_t window) {
-    const oracle_opts o = make_opts(softcap, alibi_max_bias, sinks, window);
+                         double softcap, double alibi_max_bias, const double* sinks, int64_t window,
+                         const double* mask, int64_t mask_sb, int64_t mask_ss) {
+    const oracle_opts o = make_opts(softcap, alibi_max_bias, sinks, window, mask, mask_sb, mask_ss);
     attention_impl(q, k, v, out, lse, B, Hq, Hkv, Sq, Skv, D, q_offset, causal, scale, &o);
 }
 
@@ -321,8 +336,9 @@ void oracle_attention_rows_ex(const double* q, const double* k, const double* v,
                               const int64_t* rows, int64_t n, double* out_rows, double* lse_rows,
                               int64_t B, int64_t Hq, int64_t Hkv, int64_t Sq, int64_t Skv, int64_t D,
                               int64_t q_offset, int causal, double scale,
-                              double softcap, double alibi_max_bias, const double* sinks, int64_t window) {
-    const oracle_opts o = make_opts(softcap, alibi_max_bias, sinks, window);
+                              double softcap, double alibi_max_bias, const double* sinks, int64_t window,
+                              const double* mask, int64_t mask_sb, int64_t mask_ss) {
+    const oracle_opts o = make_opts(softcap, alibi_max_bias, sinks, window, mask, mask_sb, mask_ss);
     attention_rows_impl(q, k, v, rows, n, out_rows, lse_rows, B, Hq, Hkv, Sq, Skv, D, q_offset, causal,
                         scale, &o);
 }
@@ -330,8 +346,9 @@ void oracle_attention_rows_ex(const double* q, const double* k, const double* v,
 void oracle_split_ex(const double* q, const double* k, const double* v, double* pout, double* plse,
                      int64_t B, int64_t Hq, int64_t Hkv, int64_t Sq, int64_t Skv, int64_t D,
                      int64_t q_offset, int causal, double scale, int64_t num_splits,
-                     double softcap, double alibi_max_bias, int64_t window) {
-    const oracle_opts o = make_opts(softcap, alibi_max_bias, NULL, window);
+                     double softcap, double alibi_max_bias, int64_t window,
+                     const double* mask, int64_t mask_sb, int64_t mask_ss) {
+    const oracle_opts o = make_opts(softcap, alibi_max_bias, NULL, window, mask, mask_sb, mask_ss);
     split_impl(q, k, v, pout, plse, B, Hq, Hkv, Sq, Skv, D, q_offset, causal, scale, num_splits, &o);
 }
 

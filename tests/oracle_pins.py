@@ -470,6 +470,88 @@ def pin_torch_sdpa_bias(lib):
     np.testing.assert_allclose(lse, torch.logsumexp(logits, dim=-1).numpy(), rtol=0, atol=1e-12)
 
 
+def _mask(rng, B, Sq, Skv, p_inf=0.2):
+    """A random additive mask [B, Sq, Skv] with some -inf entries (never a full row)."""
+    m = _normal(rng, (B, Sq, Skv)) * 2.0
+    cut = rng.random((B, Sq, Skv)) < p_inf
+    cut[:, :, 0] = False
+    m[cut] = -np.inf
+    return m
+
+
+def pin_mask_torch_sdpa(lib):
+    """torch's float64 SDPA with the same additive mask (-inf entries included),
+    per-batch and shared across the batch."""
+    rng = _rng(31)
+    B, Hq, Hkv, Sq, Skv, D = 2, 4, 2, 5, 9, 8
+    q, k, v = _normal(rng, (B, Sq, Hq, D)), _normal(rng, (B, Skv, Hkv, D)), _normal(rng, (B, Skv, Hkv, D))
+    g = Hq // Hkv
+    tq = torch.from_numpy(q).permute(0, 2, 1, 3)
+    tk = torch.from_numpy(k).permute(0, 2, 1, 3).repeat_interleave(g, dim=1)
+    tv = torch.from_numpy(v).permute(0, 2, 1, 3).repeat_interleave(g, dim=1)
+    for mask in (_mask(rng, B, Sq, Skv), _mask(rng, 1, Sq, Skv)):
+        out, lse = oracle.attention_ex(q, k, v, scale=0.3, causal=False, mask=mask, lib=lib)
+        tm = torch.from_numpy(mask)[:, None]          # broadcast over heads
+        ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=tm, scale=0.3)
+        np.testing.assert_allclose(out, ref.permute(0, 2, 1, 3).numpy(), rtol=0, atol=1e-12)
+        logits = (tq @ tk.transpose(-1, -2)) * 0.3 + tm
+        np.testing.assert_allclose(lse, torch.logsumexp(logits, dim=-1).numpy(), rtol=0, atol=1e-12)
+
+
+def pin_mask_removes_keys_and_shifts(lib):
+    """A -inf mask entry removes that key (same as dropping the key row); a mask
+    constant along a row leaves O unchanged and adds the constant to the LSE,
+    also under softcap and ALiBi."""
+    rng = _rng(32)
+    B, Hq, Hkv, Sq, Skv, D = 1, 2, 1, 3, 7, 4
+    q, k, v = _normal(rng, (B, Sq, Hq, D)), _normal(rng, (B, Skv, Hkv, D)), _normal(rng, (B, Skv, Hkv, D))
+    keep = np.array([0, 2, 3, 6])
+    mask = np.full((1, Sq, Skv), -np.inf)
+    mask[:, :, keep] = 0.0
+    out, lse = oracle.attention_ex(q, k, v, scale=0.5, causal=False, mask=mask, lib=lib)
+    ref_o, ref_l = oracle.attention(q, k[:, keep], v[:, keep], scale=0.5, causal=False, lib=lib)
+    np.testing.assert_allclose(out, ref_o, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(lse, ref_l, rtol=0, atol=1e-14)
+    c = np.array([0.75, -2.5, 4.0]).reshape(1, Sq, 1) * np.ones((1, Sq, Skv))
+    kw = dict(scale=0.5, causal=True, q_offset=Skv - Sq, softcap=1.5, alibi_max_bias=2.0, lib=lib)
+    o0, l0 = oracle.attention_ex(q, k, v, **kw)
+    o1, l1 = oracle.attention_ex(q, k, v, mask=c, **kw)
+    np.testing.assert_allclose(o1, o0, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(l1, l0 + np.array([0.75, -2.5, 4.0]).reshape(1, 1, Sq), rtol=0, atol=1e-13)
+
+
+def pin_mask_fully_masked_row(lib):
+    """A row whose every visible key is masked: O = 0 and LSE = -inf, or
+    LSE = the sink logit when a sink is present."""
+    rng = _rng(33)
+    B, Hq, Hkv, Sq, Skv, D = 1, 2, 2, 2, 5, 4
+    q, k, v = _normal(rng, (B, Sq, Hq, D)), _normal(rng, (B, Skv, Hkv, D)), _normal(rng, (B, Skv, Hkv, D))
+    mask = np.zeros((1, Sq, Skv))
+    mask[0, 1] = -np.inf
+    out, lse = oracle.attention_ex(q, k, v, scale=0.5, causal=False, mask=mask, lib=lib)
+    assert np.all(out[0, 1] == 0.0) and np.all(np.isneginf(lse[0, :, 1]))
+    assert np.all(np.isfinite(lse[0, :, 0]))
+    sinks = np.array([0.5, -1.0])
+    out, lse = oracle.attention_ex(q, k, v, scale=0.5, causal=False, mask=mask, sinks=sinks, lib=lib)
+    assert np.all(out[0, 1] == 0.0)
+    np.testing.assert_allclose(lse[0, :, 1], sinks, rtol=0, atol=1e-15)
+
+
+def pin_split_merge_mask(lib):
+    """Split-then-merge with a mask equals the unsplit result."""
+    rng = _rng(34)
+    B, Hq, Hkv, Sq, Skv, D = 2, 4, 1, 3, 23, 8
+    q, k, v = _normal(rng, (B, Sq, Hq, D)), _normal(rng, (B, Skv, Hkv, D)), _normal(rng, (B, Skv, Hkv, D))
+    mask = _mask(rng, B, Sq, Skv, p_inf=0.4)
+    kw = dict(scale=0.3, causal=True, q_offset=Skv - Sq, mask=mask, lib=lib)
+    out, lse = oracle.attention_ex(q, k, v, **kw)
+    for S in (1, 4, 23):
+        po, pl = oracle.split_ex(q, k, v, S, **kw)
+        mo, ml = oracle.merge(po, pl, lib=lib)
+        np.testing.assert_allclose(mo, out, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(ml, lse, rtol=0, atol=1e-12)
+
+
 ALL_PINS = [
     pin_bruteforce_decimal,
     pin_golden_three_keys,
@@ -492,4 +574,8 @@ ALL_PINS = [
     pin_window_limits,
     pin_split_merge_ex,
     pin_torch_sdpa_bias,
+    pin_mask_torch_sdpa,
+    pin_mask_removes_keys_and_shifts,
+    pin_mask_fully_masked_row,
+    pin_split_merge_mask,
 ]

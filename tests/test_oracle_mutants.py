@@ -36,6 +36,13 @@ MUTANTS = [
     ("alibi_slope_exponent", "pow(m0, (double)(h + 1))", "pow(m0, (double)h)"),
     ("softcap_ignored", "softcap * tanh(zt / softcap) : zt;", "zt : zt;"),
     ("sink_not_in_denominator", "double l = has_sink ? exp(opt->sinks[h] - m) : 0.0;", "double l = 0.0;"),
+    ("mask_sign", "z[t - t_lo] += opt->mask[b * opt->mask_sb + s * opt->mask_ss + t];",
+     "z[t - t_lo] -= opt->mask[b * opt->mask_sb + s * opt->mask_ss + t];"),
+    ("mask_row_ignored", "z[t - t_lo] += opt->mask[b * opt->mask_sb + s * opt->mask_ss + t];",
+     "z[t - t_lo] += opt->mask[b * opt->mask_sb + t];"),
+    ("mask_batch_ignored", "z[t - t_lo] += opt->mask[b * opt->mask_sb + s * opt->mask_ss + t];",
+     "z[t - t_lo] += opt->mask[s * opt->mask_ss + t];"),
+    ("masked_row_not_empty", "if (m == -INFINITY) return -INFINITY;", ""),
     ("window_off_by_one", "if (opt && opt->window > 0 && pos - opt->window + 1 > first) first = pos - opt->window + 1;",
      "if (opt && opt->window > 0 && pos - opt->window > first) first = pos - opt->window;"),
     ("merge_sink_dropped", "double wsum = sinks ? exp(sinks[h] - M) : 0.0;", "double wsum = 0.0;"),
