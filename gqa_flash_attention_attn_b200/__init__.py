@@ -138,7 +138,8 @@ _OUT_CODES = {torch.bfloat16: 0, torch.float32: 1}
 class AttnOptions(ctypes.Structure):
     """The C ``attn_options`` struct: optional logit terms (zero / NULL = off)."""
     _fields_ = [("softcap", ctypes.c_float), ("alibi_max_bias", ctypes.c_float),
-                ("sinks", ctypes.c_void_p), ("window", ctypes.c_int)]
+                ("sinks", ctypes.c_void_p), ("window", ctypes.c_int), ("mask", ctypes.c_void_p),
+                ("mask_stride_seq", ctypes.c_longlong), ("mask_stride_row", ctypes.c_longlong)]
 
 
 class AttnKVView(ctypes.Structure):
@@ -177,27 +178,42 @@ def _kv_view(k, v, block_table, seq_lens):
     return view, skv
 
 
-def _options(softcap, alibi_max_bias, sinks, window, Hq):
-    """An AttnOptions for the given terms, or None when every term is off."""
-    if not softcap and not alibi_max_bias and sinks is None and not window:
+def _options(softcap, alibi_max_bias, sinks, window, Hq, mask=None, B=None, Sq=None, Skv=None):
+    """An AttnOptions for the given terms, or None when every term is off.
+
+    mask: bf16 [B or 1, Sq, Skv] (or [Sq, Skv]), last dim contiguous; added to
+    the logits (-inf removes a key)."""
+    if not softcap and not alibi_max_bias and sinks is None and not window and mask is None:
         return None
     if sinks is not None:
         _need(sinks, "sinks", torch.float32, 1)
         if sinks.shape[0] != Hq:
             raise ValueError(f"sinks must have Hq = {Hq} entries")
-    return AttnOptions(float(softcap), float(alibi_max_bias),
-                       None if sinks is None else sinks.data_ptr(), int(window))
+    opt = AttnOptions(float(softcap), float(alibi_max_bias), None if sinks is None else sinks.data_ptr(),
+                      int(window), None, 0, 0)
+    if mask is not None:
+        if not isinstance(mask, torch.Tensor) or mask.device.type != "cuda" or mask.dtype != torch.bfloat16:
+            raise ValueError("mask must be a bf16 CUDA tensor")
+        if mask.dim() == 2:
+            mask = mask.unsqueeze(0)
+        if mask.dim() != 3 or mask.shape[1:] != (Sq, Skv) or mask.shape[0] not in (1, B) or mask.stride(2) != 1:
+            raise ValueError(f"mask must be [B or 1, {Sq}, {Skv}] with a contiguous last dim")
+        opt.mask = mask.data_ptr()
+        opt.mask_stride_seq = 0 if mask.shape[0] == 1 else mask.stride(0)
+        opt.mask_stride_row = mask.stride(1)
+    return opt
 
 
 def prefill(q, k, v, *, causal=True, q_offset=0, scale=None, out_dtype=torch.bfloat16,
             out=None, lse=None, return_lse=True, stream=None, softcap=0.0, alibi_max_bias=0.0,
-            sinks=None, window=0):
+            sinks=None, window=0, mask=None):
     """O = softmax(scale * Q K^T + causal mask) V and its LSE, in one launch.
 
     Optional logit terms (off by default): softcap (z = c tanh(z / c)),
     alibi_max_bias (per-head geometric slope times (t - pos)), sinks (fp32 [Hq]
     logits that join only the softmax denominator) and window (key t visible
-    only when pos - window < t; needs causal and q_offset + Sq <= Skv)."""
+    only when pos - window < t; needs causal and q_offset + Sq <= Skv) and
+    mask (bf16 [B or 1, Sq, Skv] added to the logits; -inf removes a key)."""
     _need(q, "q", torch.bfloat16, 4)
     _need(k, "k", torch.bfloat16, 4)
     _need(v, "v", torch.bfloat16, 4)
@@ -215,7 +231,7 @@ def prefill(q, k, v, *, causal=True, q_offset=0, scale=None, out_dtype=torch.bfl
         raise ValueError("out must be bf16 or fp32")
     if lse is None and return_lse:
         lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
-    opt = _options(softcap, alibi_max_bias, sinks, window, Hq)
+    opt = _options(softcap, alibi_max_bias, sinks, window, Hq, mask, B, Sq, Skv)
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Skv, D, int(q_offset),
             int(bool(causal)), float(scale), _OUT_CODES[out.dtype])
     if opt is None:
@@ -231,10 +247,10 @@ def decode_workspace_bytes(B, Hq, Sq, D, num_splits) -> int:
 
 def decode_split(q, k, v, num_splits, *, causal=True, q_offset=0, scale=None,
                  partial_out=None, partial_lse=None, stream=None, softcap=0.0, alibi_max_bias=0.0,
-                 window=0):
+                 window=0, mask=None):
     """Per-split normalised partial outputs [S,B,Sq,Hq,D] and LSEs [S,B,Hq,Sq].
 
-    softcap, alibi_max_bias and window as in prefill(); sinks belong to merge()."""
+    softcap, alibi_max_bias, window and mask as in prefill(); sinks belong to merge()."""
     _need(q, "q", torch.bfloat16, 4)
     _need(k, "k", torch.bfloat16, 4)
     _need(v, "v", torch.bfloat16, 4)
@@ -246,7 +262,7 @@ def decode_split(q, k, v, num_splits, *, causal=True, q_offset=0, scale=None,
         partial_out = torch.empty((num_splits, B, Sq, Hq, D), dtype=torch.float32, device=q.device)
     if partial_lse is None:
         partial_lse = torch.empty((num_splits, B, Hq, Sq), dtype=torch.float32, device=q.device)
-    opt = _options(softcap, alibi_max_bias, None, window, Hq)
+    opt = _options(softcap, alibi_max_bias, None, window, Hq, mask, B, Sq, Skv)
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(partial_out), _ptr(partial_lse), B, Hq, Hkv, Sq, Skv, D,
             int(q_offset), int(bool(causal)), float(scale), int(num_splits))
     if opt is None:
@@ -282,7 +298,7 @@ def merge(partial_out, partial_lse, *, out_dtype=torch.bfloat16, out=None, lse=N
 
 def decode(q, k, v, num_splits, *, causal=True, q_offset=0, scale=None, out_dtype=torch.bfloat16,
            workspace=None, out=None, lse=None, stream=None, softcap=0.0, alibi_max_bias=0.0, sinks=None,
-           window=0):
+           window=0, mask=None):
     """Split-KV decode followed by the LSE merge (two launches on one stream)."""
     B, Sq, Hq, D = q.shape
     po = pl = None
@@ -290,13 +306,13 @@ def decode(q, k, v, num_splits, *, causal=True, q_offset=0, scale=None, out_dtyp
         po, pl = workspace
     po, pl = decode_split(q, k, v, num_splits, causal=causal, q_offset=q_offset, scale=scale,
                           partial_out=po, partial_lse=pl, stream=stream, softcap=softcap,
-                          alibi_max_bias=alibi_max_bias, window=window)
+                          alibi_max_bias=alibi_max_bias, window=window, mask=mask)
     return merge(po, pl, out_dtype=out_dtype, out=out, lse=lse, stream=stream, sinks=sinks)
 
 
 def decode_split_kv(q, k, v, num_splits, *, block_table=None, seq_lens=None, causal=True, q_offset=0,
                     scale=None, partial_out=None, partial_lse=None, stream=None, softcap=0.0,
-                    alibi_max_bias=0.0, window=0):
+                    alibi_max_bias=0.0, window=0, mask=None):
     """decode_split over a strided or paged K/V cache (see attn_kv_view).
 
     Unpaged: k, v are [B, Skv, Hkv, D] views (any strides, last dim
@@ -320,7 +336,7 @@ def decode_split_kv(q, k, v, num_splits, *, block_table=None, seq_lens=None, cau
         partial_out = torch.empty((num_splits, B, Sq, Hq, D), dtype=torch.float32, device=q.device)
     if partial_lse is None:
         partial_lse = torch.empty((num_splits, B, Hq, Sq), dtype=torch.float32, device=q.device)
-    opt = _options(softcap, alibi_max_bias, None, window, Hq)
+    opt = _options(softcap, alibi_max_bias, None, window, Hq, mask, B, Sq, Skv)
     st = library().attn_decode_split_kv(_ptr(q), ctypes.byref(view), _ptr(partial_out), _ptr(partial_lse), B, Hq,
                                         Hkv, Sq, Skv, D, int(q_offset), int(bool(causal)), float(scale),
                                         int(num_splits), None if opt is None else ctypes.byref(opt),
@@ -331,14 +347,14 @@ def decode_split_kv(q, k, v, num_splits, *, block_table=None, seq_lens=None, cau
 
 def decode_kv(q, k, v, num_splits, *, block_table=None, seq_lens=None, causal=True, q_offset=0, scale=None,
               out_dtype=torch.bfloat16, workspace=None, out=None, lse=None, stream=None, softcap=0.0,
-              alibi_max_bias=0.0, sinks=None, window=0):
+              alibi_max_bias=0.0, sinks=None, window=0, mask=None):
     """decode_split_kv followed by the LSE merge (two launches on one stream)."""
     po = pl = None
     if workspace is not None:
         po, pl = workspace
     po, pl = decode_split_kv(q, k, v, num_splits, block_table=block_table, seq_lens=seq_lens, causal=causal,
                              q_offset=q_offset, scale=scale, partial_out=po, partial_lse=pl, stream=stream,
-                             softcap=softcap, alibi_max_bias=alibi_max_bias, window=window)
+                             softcap=softcap, alibi_max_bias=alibi_max_bias, window=window, mask=mask)
     return merge(po, pl, out_dtype=out_dtype, out=out, lse=lse, stream=stream, sinks=sinks)
 
 

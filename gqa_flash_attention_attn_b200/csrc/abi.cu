@@ -133,9 +133,16 @@ int make_ext(const attn_options* opt, int Hq, int Sq, int Skv, int q_offset, int
     ext->l2m0 = -opt->alibi_max_bias / (float)n2;
     ext->l2m1 = -opt->alibi_max_bias / (float)(2 * n2);
   }
+  if (opt->mask != nullptr) {
+    if (opt->mask_stride_seq < 0 || opt->mask_stride_row < 0) return ATTN_ERR_INVALID_ARG;
+    if (!aligned(opt->mask, 2)) return ATTN_ERR_ALIGNMENT;
+    ext->mask = static_cast<const uint16_t*>(opt->mask);
+    ext->mask_sb = opt->mask_stride_seq;
+    ext->mask_sr = opt->mask_stride_row;
+  }
   ext->sinks = opt->sinks;
   ext->window = opt->window;
-  *on = ext->cap_a > 0.f || ext->alibi != 0 || ext->sinks != nullptr || ext->window > 0;
+  *on = ext->cap_a > 0.f || ext->alibi != 0 || ext->sinks != nullptr || ext->window > 0 || ext->mask != nullptr;
   return ATTN_OK;
 }
 
@@ -143,7 +150,7 @@ int make_ext(const attn_options* opt, int Hq, int Sq, int Skv, int q_offset, int
 
 extern "C" {
 
-int attn_version(void) { return 0x000100; }
+int attn_version(void) { return 0x000200; }
 
 const char* attn_status_string(int status) {
   switch (status) {

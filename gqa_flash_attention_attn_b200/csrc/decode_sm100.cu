@@ -47,7 +47,7 @@ struct Layout {
     off_ring = (off_p + 2u * 2u * RP * 128u + 1023u) & ~1023u;  // two P buffers
     off_red = off_ring + (uint32_t)nbuf * SLOT_BYTES;
     off_row = off_red + 2u * 4u * RP * 4u;     // red_max[4][RP], red_sum[4][RP]
-    off_bar = off_row + 9u * RP * 4u;          // m, l, alpha, msub, inv, lim, limlo, pos, slope
+    off_bar = off_row + 11u * RP * 4u;         // m, l, alpha, msub, inv, lim, limlo, pos, slope, mask row
     off_bar = (off_bar + 7u) & ~7u;
     off_misc = off_bar + (uint32_t)(1 + 2 * nbuf + 7) * 8u;
     total = off_misc + 16u + 1024u;
@@ -104,6 +104,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   int* limlo_sm = lim_sm + RP;                             // keys <= this are outside the window
   int* pos_sm = limlo_sm + RP;                             // query position of row r
   float* slope_sm = reinterpret_cast<float*>(pos_sm + RP); // ALiBi slope * log2(e) of row r
+  const uint16_t** mrow_sm = reinterpret_cast<const uint16_t**>(slope_sm + RP);  // mask row of row r
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L.off_misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L.off_misc + 4);
   volatile int* resc_flag = reinterpret_cast<volatile int*>(gbase + L.off_misc + 8);
@@ -172,6 +173,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     slope_sm[r] = (EXT && p.ext.alibi && r < R)
                       ? alibi_slope_log2e(kvh * g + (r - (r / g) * g), p.ext.l2m0, p.ext.l2m1, p.ext.n2)
                       : 0.f;
+    mrow_sm[r] = (EXT && p.ext.mask != nullptr && r < R)
+                     ? p.ext.mask + (size_t)b * p.ext.mask_sb + (size_t)(r / g) * p.ext.mask_sr
+                     : nullptr;
   }
   if (threadIdx.x == 0) {
     mbar_init(bar(BAR_Q), 1);
@@ -331,7 +335,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       // optional terms: logit in log2 units, softcap and ALiBi applied
       auto logit2 = [&](float sdot, int r) -> float {
         const float z = p.ext.cap_a > 0.f ? p.ext.cap_b * tanh_approx(sdot * p.ext.cap_a) : sdot * c2;
-        return fmaf(slope_sm[r], (float)(key - pos_sm[r]), z);
+        float y = fmaf(slope_sm[r], (float)(key - pos_sm[r]), z);
+        // additive mask, read only inside the split (key < hi <= Skv)
+        const uint16_t* mr = mrow_sm[r];
+        if (mr != nullptr && key < hi)
+          y = fmaf(__uint_as_float((uint32_t)__ldg(mr + key) << 16), 1.4426950408889634f, y);
+        return y;
       };
       auto visible = [&](int r) -> bool {
         return key < hi && key <= lim_sm[r] && (!EXT || key > limlo_sm[r]);

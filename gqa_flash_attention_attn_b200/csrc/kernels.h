@@ -9,7 +9,8 @@ namespace gqa {
 // Optional logit terms, prepared on the host.  The logit in log2 units is
 //   L = (cap_a > 0 ? cap_b * tanh(s * cap_a) : s * c2) + slope_h * log2(e) * (t - pos)
 // with s the raw Q.K dot product; slope_h = 2^(l2m0 * (h + 1)) for h < n2,
-// else 2^(l2m1 * (2 (h - n2) + 1)), and 0 when alibi is off.
+// else 2^(l2m1 * (2 (h - n2) + 1)), and 0 when alibi is off; plus
+// log2(e) * mask[b, s, t] when a mask is given.
 struct LogitExt {
   float cap_a;        // scale / softcap, or 0 when off
   float cap_b;        // softcap * log2(e)
@@ -18,6 +19,8 @@ struct LogitExt {
   int n2;             // largest power of two <= Hq
   const float* sinks; // [Hq] natural-log sink logits, or nullptr
   int window;         // 0: off
+  const uint16_t* mask;        // bf16 bits of the additive mask, or nullptr
+  long long mask_sb, mask_sr;  // element strides: sequence, query row
 };
 
 struct PrefillParams {

@@ -146,8 +146,9 @@ __device__ __forceinline__ int unit_index(int k, int total) {
 
 // Kernel variants by the optional logit terms they handle (plain runs none):
 //   MODE_MASKS  sliding window and sink logits (no per-element arithmetic)
-//   MODE_ALIBI  ALiBi bias, with or without window and sinks
-//   MODE_CAP    softcap, with or without ALiBi, window and sinks
+//   MODE_ALIBI  ALiBi bias and / or an additive mask, with or without window
+//               and sinks
+//   MODE_CAP    softcap, with or without ALiBi, mask, window and sinks
 constexpr int MODE_PLAIN = 0, MODE_MASKS = 1, MODE_ALIBI = 2, MODE_CAP = 3;
 
 // Logits in log2 units of the N keys of a half tile whose first key sits at
@@ -156,9 +157,12 @@ constexpr int MODE_PLAIN = 0, MODE_MASKS = 1, MODE_ALIBI = 2, MODE_CAP = 3;
 //   MODE_CAP    cap_b tanh(s cap_a) + slope2 (dist0 + e)   (slope2 = 0: no ALiBi)
 // in packed pairs.  The ALiBi bias runs as four interleaved sums that start
 // exact at each half tile, so no per-element index arithmetic is needed.
-template <int MODE, bool BIAS, int N>
+// MASK: 0 no mask; 1 mask read as 16-byte vectors (all N keys inside the
+// mask, row 16-byte aligned); 2 mask read one key at a time, keys at or past
+// nvalid read as 0.
+template <int MODE, bool BIAS, int MASK, int N>
 __device__ __forceinline__ void ext_logits_run(float (&v)[N], const LogitExt& x, float c2, float slope2,
-                                               int dist0) {
+                                               int dist0, const uint16_t* mk, int nvalid) {
   static_assert(N % 8 == 0, "whole groups of four pairs");
   const float b0 = slope2 * (float)dist0;
   float2 bias[4];
@@ -166,17 +170,31 @@ __device__ __forceinline__ void ext_logits_run(float (&v)[N], const LogitExt& x,
   for (int i = 0; i < 4; ++i)
     bias[i] = make_float2(fmaf(slope2, (float)(2 * i), b0), fmaf(slope2, (float)(2 * i + 1), b0));
   const float2 step = make_float2(8.f * slope2, 8.f * slope2);
+  const float2 l2e = make_float2(1.4426950408889634f, 1.4426950408889634f);
+  uint4 mw = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
   for (int e = 0; e < N; e += 2) {
     const int i = (e >> 1) & 3;
     const float2 sp = make_float2(v[e], v[e + 1]);
     float2 y;
     if constexpr (MODE == MODE_ALIBI) {
-      y = ffma2(sp, make_float2(c2, c2), bias[i]);
+      y = BIAS ? ffma2(sp, make_float2(c2, c2), bias[i]) : fmul2(sp, make_float2(c2, c2));
     } else {
       const float2 u = fmul2(sp, make_float2(x.cap_a, x.cap_a));
       const float2 t = make_float2(tanh_approx(u.x), tanh_approx(u.y));
       y = BIAS ? ffma2(t, make_float2(x.cap_b, x.cap_b), bias[i]) : fmul2(t, make_float2(x.cap_b, x.cap_b));
+    }
+    if constexpr (MASK != 0) {
+      uint32_t w;
+      if constexpr (MASK == 1) {
+        if ((e & 7) == 0) mw = __ldg(reinterpret_cast<const uint4*>(mk + e));
+        w = i == 0 ? mw.x : i == 1 ? mw.y : i == 2 ? mw.z : mw.w;
+      } else {
+        const uint32_t lo = e < nvalid ? (uint32_t)__ldg(mk + e) : 0u;
+        const uint32_t hi = e + 1 < nvalid ? (uint32_t)__ldg(mk + e + 1) : 0u;
+        w = lo | (hi << 16);
+      }
+      y = ffma2(make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)), l2e, y);
     }
     v[e] = y.x;
     v[e + 1] = y.y;
@@ -187,13 +205,27 @@ __device__ __forceinline__ void ext_logits_run(float (&v)[N], const LogitExt& x,
   }
 }
 
-// One branch outside the unrolled loop: neither path pays for the other.
-template <int MODE, int N>
-__device__ __forceinline__ void ext_logits(float (&v)[N], const LogitExt& x, float c2, float slope2, int dist0) {
-  if (MODE == MODE_ALIBI || x.alibi)
-    ext_logits_run<MODE, true>(v, x, c2, slope2, dist0);
+template <int MODE, bool BIAS, int N>
+__device__ __forceinline__ void ext_logits_m(float (&v)[N], const LogitExt& x, float c2, float slope2, int dist0,
+                                             const uint16_t* mk, int nvalid) {
+  if (mk == nullptr)
+    ext_logits_run<MODE, BIAS, 0>(v, x, c2, slope2, dist0, mk, nvalid);
+  else if (nvalid >= N && (reinterpret_cast<uintptr_t>(mk) & 15u) == 0)
+    ext_logits_run<MODE, BIAS, 1>(v, x, c2, slope2, dist0, mk, nvalid);
   else
-    ext_logits_run<MODE, false>(v, x, c2, slope2, dist0);
+    ext_logits_run<MODE, BIAS, 2>(v, x, c2, slope2, dist0, mk, nvalid);
+}
+
+// Logits of a half tile.  mk: this row's mask at the half's first key (or
+// nullptr), nvalid: keys of the half inside the mask.  The branches sit
+// outside the unrolled loops: no path pays for another.
+template <int MODE, int N>
+__device__ __forceinline__ void ext_logits(float (&v)[N], const LogitExt& x, float c2, float slope2, int dist0,
+                                           const uint16_t* mk, int nvalid) {
+  if (x.alibi)
+    ext_logits_m<MODE, true>(v, x, c2, slope2, dist0, mk, nvalid);
+  else
+    ext_logits_m<MODE, false>(v, x, c2, slope2, dist0, mk, nvalid);
 }
 
 // Columns outside [cb, cl) become -inf.
@@ -473,6 +505,10 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
       const int vis_begin = (MODE != MODE_PLAIN && p.ext.window > 0) ? pos - p.ext.window + 1 : 0;
       const float slope2 =
           (MODE >= MODE_ALIBI && p.ext.alibi) ? alibi_slope_log2e(h, p.ext.l2m0, p.ext.l2m1, p.ext.n2) : 0.f;
+      // this row's mask (padding rows past Sq read the last row's: never stored)
+      const uint16_t* mrow = (MODE >= MODE_ALIBI && p.ext.mask != nullptr)
+                                 ? p.ext.mask + (size_t)x.b * p.ext.mask_sb + (size_t)min(s_row, p.Sq - 1) * p.ext.mask_sr
+                                 : nullptr;
       float m_use = -INFINITY, l = 0.f;
       for (int j = 0; j < n_tiles; ++j) {
         const int G = T + j;
@@ -497,7 +533,8 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
           // (P only ever covers columns 0-63), where half 1 below reads them.
           float sh[BN / 2];
           tmem_ld64(tS + BN / 2, sh);
-          ext_logits<MODE>(sh, p.ext, c2, slope2, key0 + BN / 2 - pos);
+          ext_logits<MODE>(sh, p.ext, c2, slope2, key0 + BN / 2 - pos, mrow ? mrow + key0 + BN / 2 : nullptr,
+                           p.Skv - (key0 + BN / 2));
           {
             uint32_t u[BN / 2];
 #pragma unroll
@@ -508,7 +545,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
           const float mx_hi = row_max(sh);
           float (&slo)[BN / 2] = *reinterpret_cast<float(*)[BN / 2]>(sv);
           tmem_ld64(tS, slo);
-          ext_logits<MODE>(slo, p.ext, c2, slope2, key0 - pos);
+          ext_logits<MODE>(slo, p.ext, c2, slope2, key0 - pos, mrow ? mrow + key0 : nullptr, p.Skv - key0);
           if (tile_masked) mask_cols(slo, cb, cl);
           mx = fmaxf(mx_hi, row_max(slo));
         } else {
@@ -713,7 +750,7 @@ int launch_prefill(int D, bool ext, const CUtensorMap& tq, const CUtensorMap& tk
   // the cheapest variant that covers the requested terms
   const int mode = !ext ? MODE_PLAIN
                    : p.ext.cap_a > 0.f ? MODE_CAP
-                   : p.ext.alibi ? MODE_ALIBI
+                   : (p.ext.alibi || p.ext.mask != nullptr) ? MODE_ALIBI
                    : MODE_MASKS;
   switch (D) {
     case 64: return launch_mode<64>(mode, tq, tk, tv, p, stream);

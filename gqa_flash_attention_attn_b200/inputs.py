@@ -177,6 +177,17 @@ def make_seq_lens(B, Skv, *, seed=0, low=1):
     return torch.randint(low, Skv + 1, (B,), generator=gen, dtype=torch.int64).to(torch.int32)
 
 
+def make_mask(B, Sq, Skv, *, seed=0, std=2.0, p_inf=0.2, device="cpu"):
+    """Seeded additive bf16 mask [B, Sq, Skv]: N(0, std^2) values with a
+    fraction p_inf of the entries at -inf (key 0 of every row is kept)."""
+    gen = torch.Generator().manual_seed(seed)
+    m = torch.randn((B, Sq, Skv), generator=gen) * std
+    cut = torch.rand((B, Sq, Skv), generator=gen) < p_inf
+    cut[:, :, 0] = False
+    m[cut] = float("-inf")
+    return m.to(torch.bfloat16).to(device)
+
+
 def make_workload_inputs(w: Workload, *, seed=0, device="cpu"):
     return make_qkv(w.B, w.Hq, w.Hkv, w.Sq, w.Skv, w.D, seed=seed, device=device)
 

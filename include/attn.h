@@ -178,18 +178,31 @@ int attn_decode_noalloc(const void* q, const void* k, const void* v, void* out, 
  *   window > 0           key t is visible only if pos - window < t; needs
  *                        causal = 1 and q_offset + Sq <= Skv (every query
  *                        position has its key), else ATTN_ERR_UNSUPPORTED
+ *   mask != NULL         additive bf16 mask (the `mask` parameter of the same
+ *                        test case): z += mask[b*mask_stride_seq +
+ *                        s*mask_stride_row + t] for t < Skv, after softcap and
+ *                        ALiBi; -inf removes the key.  mask_stride_seq = 0
+ *                        shares one [Sq, Skv] mask across the batch.  A row
+ *                        whose every visible key is masked gets O = 0 and
+ *                        LSE = -inf (or the sink logit with a sink).
  *
  * Zero / NULL fields are off.  softcap and alibi_max_bias must be finite and
  * >= 0, window >= 0 (else ATTN_ERR_INVALID_ARG); sinks must be 4-byte aligned
- * (else ATTN_ERR_ALIGNMENT).  The caller owns *opt and the sink array; the
- * call reads *opt on the host before it returns and the sink array on the
- * device, in stream order.
+ * (else ATTN_ERR_ALIGNMENT); the mask must be 2-byte aligned (else
+ * ATTN_ERR_ALIGNMENT) with non-negative strides (else ATTN_ERR_INVALID_ARG);
+ * rows that start 16-byte aligned (mask 16-byte aligned, strides multiples of
+ * 8) are read with vector loads, others one element at a time.
+ * The caller owns *opt, the sink array and the mask; the call reads *opt on
+ * the host before it returns and the arrays on the device, in stream order.
  */
 typedef struct attn_options {
   float softcap;
   float alibi_max_bias;
   const float* sinks;
   int window;
+  const void* mask;             /* bf16, or NULL */
+  long long mask_stride_seq;    /* elements between sequences (0: shared) */
+  long long mask_stride_row;    /* elements between query rows */
 } attn_options;
 
 /* attn_prefill with the optional terms of *opt (opt may be NULL). */
@@ -265,7 +278,7 @@ int attn_decode_split_kv(const void* q, const attn_kv_view* kv, float* partial_o
                          int B, int Hq, int Hkv, int Sq, int Skv, int D, int q_offset, int causal,
                          float scale, int num_splits, const attn_options* opt, void* stream);
 
-/* Library version, e.g. 0x000100 for 0.1.0. */
+/* Library version, e.g. 0x000200 for 0.2.0. */
 int attn_version(void);
 
 #ifdef __cplusplus

@@ -22,7 +22,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert ga.version() == 0x000100
+    assert ga.version() == 0x000200
     assert ga.status_string(ga.ATTN_OK) == "ok"
     assert ga.status_string(ga.ATTN_ERR_TIMEOUT) == "pipeline wait timed out"
     assert ga.status_string(12345) == "unknown status"
@@ -117,8 +117,8 @@ def test_merge_rejects(lib, args, status):
     assert lib.attn_merge(*args, None) == status
 
 
-def _opt(softcap=0.0, alibi=0.0, sinks=None, window=0):
-    return ctypes.byref(ga.AttnOptions(softcap, alibi, sinks, window))
+def _opt(softcap=0.0, alibi=0.0, sinks=None, window=0, mask=None, msb=0, msr=0):
+    return ctypes.byref(ga.AttnOptions(softcap, alibi, sinks, window, mask, msb, msr))
 
 
 @pytest.mark.parametrize("opt,kw,status", [
@@ -134,6 +134,9 @@ def _opt(softcap=0.0, alibi=0.0, sinks=None, window=0):
     (dict(window=64), dict(q_offset=1), ga.ATTN_ERR_UNSUPPORTED),  # q_offset + Sq > Skv
     (dict(softcap=30.0), dict(q=None), ga.ATTN_ERR_INVALID_ARG),  # shape checks still apply
     (dict(softcap=30.0), dict(D=72), ga.ATTN_ERR_UNSUPPORTED),
+    (dict(mask=0x80001), {}, ga.ATTN_ERR_ALIGNMENT),             # bf16 mask at an odd address
+    (dict(mask=0x80000, msr=-128), {}, ga.ATTN_ERR_INVALID_ARG),
+    (dict(mask=0x80000, msb=-1, msr=128), {}, ga.ATTN_ERR_INVALID_ARG),
 ])
 def test_prefill_ex_rejects(lib, opt, kw, status):
     a = dict(q=P, k=P, v=P, out=P2, lse=P2, B=1, Hq=8, Hkv=2, Sq=128, Skv=128, D=128, q_offset=0, causal=1,
@@ -173,9 +176,9 @@ def test_options_struct_matches_header():
     import re
     text = open(ga._HEADER).read()
     body = re.search(r"typedef struct attn_options \{(.*?)\} attn_options;", text, re.S).group(1)
-    fields = [ln.strip().rstrip(";").split()[-1].lstrip("*") for ln in body.strip().splitlines()]
+    fields = [ln.split(";")[0].split()[-1].lstrip("*") for ln in body.strip().splitlines() if ";" in ln]
     assert fields == [f[0] for f in ga.AttnOptions._fields_]
-    assert ctypes.sizeof(ga.AttnOptions) == 24
+    assert ctypes.sizeof(ga.AttnOptions) == 48
 
 
 def _kv_decode(lib, view=None, **kw):

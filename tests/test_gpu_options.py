@@ -222,3 +222,68 @@ def test_headline_prefill_with_every_term_sampled():
     want_o, want_l = _rows_oracle_ex(w, q, k, v, rows, sinks)
     assert_o_close(got_o, want_o, "4k prefill, every term")
     assert_lse_close(got_l, want_l, "4k prefill, every term")
+
+
+# (B, Hq, Hkv, Sq, Skv, D, q_offset, causal, softcap, alibi, sinks, window, mask batch)
+MASKED_PREFILL = [
+    (2, 8, 2, 200, 384, 128, 184, True, 0.0, 0.0, False, 0, 2),     # per-sequence masks, vector path
+    (1, 8, 2, 300, 300, 128, 0, True, 0.0, 0.0, False, 0, 1),       # ragged Skv: scalar tail
+    (2, 4, 2, 130, 517, 64, 0, False, 0.0, 0.0, True, 0, 1),        # shared mask, non-causal, sinks
+    (1, 8, 2, 256, 640, 128, 384, True, 20.0, 4.0, True, 256, 1),  # every term
+    (1, 4, 2, 200, 600, 256, 400, True, 0.0, 8.0, False, 0, 1),     # D = 256 with ALiBi
+    (1, 4, 2, 150, 333, 256, 183, True, 10.0, 0.0, True, 0, 1),     # D = 256 softcap, ragged
+]
+
+
+@pytest.mark.parametrize("case", MASKED_PREFILL, ids=[f"c{i}" for i in range(len(MASKED_PREFILL))])
+def test_prefill_mask_matches_oracle(case):
+    from gqa_flash_attention_attn_b200.inputs import make_mask
+    B, Hq, Hkv, Sq, Skv, D, q_offset, causal, cap, ab, use_sinks, window, mb = case
+    q, k, v = make_qkv(B, Hq, Hkv, Sq, Skv, D, seed=51)
+    mask = make_mask(mb, Sq, Skv, seed=52)
+    mask[0, 3] = float("-inf")                # a fully masked row
+    sinks = _sinks(Hq, seed=53) if use_sinks else None
+    scale = _scale(D)
+    out, lse = ga.prefill(q.cuda(), k.cuda(), v.cuda(), causal=causal, q_offset=q_offset, scale=scale,
+                          out_dtype=torch.float32, softcap=cap, alibi_max_bias=ab, window=window,
+                          sinks=None if sinks is None else sinks.cuda(), mask=mask.cuda())
+    torch.cuda.synchronize()
+    assert ga.last_status() == ga.ATTN_OK
+    want_o, want_l = oracle.attention_ex(q, k, v, scale=scale, causal=causal, q_offset=q_offset, softcap=cap,
+                                         alibi_max_bias=ab, window=window, mask=mask,
+                                         sinks=None if sinks is None else sinks.numpy())
+    assert_o_close(out, want_o, str(case))
+    assert_lse_close(lse, want_l, str(case))
+
+
+def test_prefill_mask_of_zeros_equals_no_mask():
+    q, k, v = make_qkv(1, 8, 2, 256, 256, 128, seed=54)
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    zero = torch.zeros((1, 256, 256), dtype=torch.bfloat16, device="cuda")
+    o1, l1 = ga.prefill(qc, kc, vc, alibi_max_bias=2.0)
+    o2, l2 = ga.prefill(qc, kc, vc, alibi_max_bias=2.0, mask=zero)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("paged", [False, True])
+def test_decode_mask_matches_oracle(paged):
+    from gqa_flash_attention_attn_b200.inputs import make_mask, make_paged
+    B, Hq, Hkv, Sq, Skv, D, S = 2, 32, 8, 8, 1024, 128, 5
+    q, k, v = make_qkv(B, Hq, Hkv, Sq, Skv, D, seed=55)
+    mask = make_mask(B, Sq, Skv, seed=56, p_inf=0.5)     # e.g. a tree of draft tokens
+    mask[1, 2] = float("-inf")
+    sinks = _sinks(Hq, seed=57)
+    kw = dict(causal=True, q_offset=Skv - Sq, softcap=15.0, alibi_max_bias=2.0, mask=mask.cuda())
+    if paged:
+        kc, vc, bt = make_paged(k, v, 64, seed=58)
+        out, lse = ga.decode_kv(q.cuda(), kc.cuda(), vc.cuda(), S, block_table=bt.cuda(), out_dtype=torch.float32,
+                                sinks=sinks.cuda(), **kw)
+    else:
+        out, lse = ga.decode(q.cuda(), k.cuda(), v.cuda(), S, out_dtype=torch.float32, sinks=sinks.cuda(), **kw)
+    torch.cuda.synchronize()
+    assert ga.last_status() == ga.ATTN_OK
+    want_o, want_l = oracle.attention_ex(q, k, v, scale=_scale(D), causal=True, q_offset=Skv - Sq, softcap=15.0,
+                                         alibi_max_bias=2.0, mask=mask, sinks=sinks.numpy())
+    assert_o_close(out, want_o, f"decode mask paged={paged}")
+    assert_lse_close(lse, want_l, f"decode mask paged={paged}")
