@@ -164,7 +164,7 @@ def make_runner(ga, w, device):
     """Device-resident inputs/outputs and a closure that launches one step.
     Returns (step_fn, n_kernels_per_step, events_split) where the closure
     records optional inner events between the split and the merge."""
-    from gqa_flash_attention_attn_b200.inputs import make_paged, make_qkv, make_sinks
+    from gqa_flash_attention_attn_b200.inputs import make_mask, make_paged, make_qkv, make_sinks
     q, k, v = make_qkv(w.B, w.Hq, w.Hkv, w.Sq, w.Skv, w.D, seed=0, device=device)
     bt = None
     if w.page_size:
@@ -174,7 +174,8 @@ def make_runner(ga, w, device):
     out = torch.empty((w.B, w.Sq, w.Hq, w.D), dtype=odt, device=device)
     lse = torch.empty((w.B, w.Hq, w.Sq), dtype=torch.float32, device=device)
     sinks = make_sinks(w.Hq, seed=0).to(device) if w.sinks else None
-    terms = dict(softcap=w.softcap, alibi_max_bias=w.alibi_max_bias, window=w.window)
+    mask = make_mask(w.mask_batch, w.Sq, w.Skv, seed=0).to(device) if w.mask_batch else None
+    terms = dict(softcap=w.softcap, alibi_max_bias=w.alibi_max_bias, window=w.window, mask=mask)
     if w.kind == "prefill":
         def step(mid=None):
             ga.prefill(q, k, v, causal=w.causal, q_offset=w.q_offset, scale=w.scale, out=out, lse=lse,

@@ -291,8 +291,16 @@ int attn_decode_split_kv(const void* q, const attn_kv_view* kv, float* partial_o
   p.g = g; p.R = (int)R; p.RP = (int)RP;
   p.num_splits = num_splits;
   p.chunk = (Skv + num_splits - 1) / num_splits;
+  // stage the additive mask per tile in shared memory (cp.async, 16-byte
+  // chunks) for up to 32 query rows when its rows are 16-byte aligned
+  p.mask_rows = (ext.mask != nullptr && Sq <= 32 && aligned(ext.mask, 16) && ext.mask_sb % 8 == 0 &&
+                 ext.mask_sr % 8 == 0)
+                    ? Sq
+                    : 0;
   int nbuf = 2;
-  while (nbuf < gqa::decode_max_nbuf() && gqa::decode_smem_bytes(D, p.RP, nbuf + 1) <= kTwoCtaSmemLimit) ++nbuf;
+  while (nbuf < gqa::decode_max_nbuf() &&
+         gqa::decode_smem_bytes(D, p.RP, nbuf + 1, p.mask_rows) <= kTwoCtaSmemLimit)
+    ++nbuf;
   p.nbuf = nbuf;
   p.c2 = scale * kLog2e;
   p.timeout_ns = kWaitLimitNs;

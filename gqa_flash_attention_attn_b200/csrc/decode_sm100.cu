@@ -37,17 +37,23 @@ constexpr int THREADS = 192;                   // warps 0-3 softmax, 4 producer,
 constexpr int WARP_PRODUCER = 4;
 constexpr int WARP_MMA = 5;
 constexpr int MAX_NBUF = 6;
+// A staged mask row: the tile's 128 keys in an 8-key-aligned window of 136
+// (17 chunks of 16 bytes), so every cp.async source is 16-byte aligned.
+constexpr int MROW_KEYS = 136;
+constexpr uint32_t MROW_BYTES = MROW_KEYS * 2u;
 
 struct Layout {
-  uint32_t off_q, off_p, off_ring, off_red, off_row, off_bar, off_misc, total;
-  __host__ __device__ Layout(int D, int RP, int nbuf) {
+  uint32_t off_q, off_p, off_ring, off_red, off_row, off_mask, off_bar, off_misc, total;
+  // mrows: query rows s whose additive-mask values are staged per tile
+  __host__ __device__ Layout(int D, int RP, int nbuf, int mrows) {
     off_q = 0;
     const uint32_t qbytes = (uint32_t)(D / 64) * RP * 128u;
     off_p = (off_q + qbytes + 1023u) & ~1023u;
     off_ring = (off_p + 2u * 2u * RP * 128u + 1023u) & ~1023u;  // two P buffers
     off_red = off_ring + (uint32_t)nbuf * SLOT_BYTES;
     off_row = off_red + 2u * 4u * RP * 4u;     // red_max[4][RP], red_sum[4][RP]
-    off_bar = off_row + 11u * RP * 4u;         // m, l, alpha, msub, inv, lim, limlo, pos, slope, mask row
+    off_mask = off_row + 11u * RP * 4u;        // m, l, alpha, msub, inv, lim, limlo, pos, slope, mask row
+    off_bar = off_mask + (uint32_t)mrows * 2u * MROW_BYTES;  // staged mask [2][mrows][136 keys] bf16
     off_bar = (off_bar + 7u) & ~7u;
     off_misc = off_bar + (uint32_t)(1 + 2 * nbuf + 7) * 8u;
     total = off_misc + 16u + 1024u;
@@ -81,13 +87,64 @@ __device__ __forceinline__ float warp_reduce16(float (&v)[16], int lane) {
   return kMax ? fmaxf(v[0], other) : v[0] + other;
 }
 
+// Logits in log2 units of this thread's key for the 16 rows 16q..16q+15 with
+// the optional terms: softcap or plain scaling, ALiBi slope * (key - pos), and
+// the additive mask (staged per tile in shared memory, or read directly).
+// Per-row constants come in as 16-byte shared-memory vectors and every term's
+// test sits outside the unrolled loops.
+__device__ __forceinline__ void ext_rows16(float (&v)[16], const LogitExt& x, float c2, int key, int t, int q,
+                                           const float* slope_sm, const int* pos_sm, const uint16_t* mst,
+                                           int mask_rows, int q_offset, const uint16_t* const* mrow_sm, int hi) {
+  if (x.cap_a > 0.f) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) v[e] = x.cap_b * tanh_approx(v[e] * x.cap_a);
+  } else {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) v[e] *= c2;
+  }
+  if (x.alibi || mask_rows > 0) {
+    int ps[16];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int4 w = reinterpret_cast<const int4*>(pos_sm + 16 * q)[i];
+      ps[4 * i] = w.x; ps[4 * i + 1] = w.y; ps[4 * i + 2] = w.z; ps[4 * i + 3] = w.w;
+    }
+    if (x.alibi) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float4 w = reinterpret_cast<const float4*>(slope_sm + 16 * q)[i];
+        v[4 * i] = fmaf(w.x, (float)(key - ps[4 * i]), v[4 * i]);
+        v[4 * i + 1] = fmaf(w.y, (float)(key - ps[4 * i + 1]), v[4 * i + 1]);
+        v[4 * i + 2] = fmaf(w.z, (float)(key - ps[4 * i + 2]), v[4 * i + 2]);
+        v[4 * i + 3] = fmaf(w.w, (float)(key - ps[4 * i + 3]), v[4 * i + 3]);
+      }
+    }
+    if (mask_rows > 0) {
+      // mst: this tile's staged mask, already offset to this thread's key
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+        v[e] = fmaf(__uint_as_float((uint32_t)mst[(ps[e] - q_offset) * MROW_KEYS] << 16), 1.4426950408889634f,
+                    v[e]);
+    }
+  }
+  if (x.mask != nullptr && mask_rows == 0) {
+    // too many rows to stage: read inside the split only (key < hi <= Skv)
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const uint16_t* mr = mrow_sm[16 * q + e];
+      if (mr != nullptr && key < hi)
+        v[e] = fmaf(__uint_as_float((uint32_t)__ldg(mr + key) << 16), 1.4426950408889634f, v[e]);
+    }
+  }
+}
+
 template <int D, bool EXT, bool PAGED>
 __global__ void __launch_bounds__(THREADS, 1)
     decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
   constexpr int KC = D / 128;  // 128-column slots per K (or V) tile
   const int RP = p.RP, R = p.R, g = p.g, nbuf = p.nbuf;
-  const Layout L(D, RP, nbuf);
+  const Layout L(D, RP, nbuf, p.mask_rows);
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -105,6 +162,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   int* pos_sm = limlo_sm + RP;                             // query position of row r
   float* slope_sm = reinterpret_cast<float*>(pos_sm + RP); // ALiBi slope * log2(e) of row r
   const uint16_t** mrow_sm = reinterpret_cast<const uint16_t**>(slope_sm + RP);  // mask row of row r
+  // staged mask: [2 tiles][mask_rows][136 keys] bf16, filled by cp.async one
+  // tile ahead by all softmax threads
+  const uint32_t mstage_u32 = base + L.off_mask;
+  const uint16_t* mstage = reinterpret_cast<const uint16_t*>(gbase + L.off_mask);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L.off_misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L.off_misc + 4);
   volatile int* resc_flag = reinterpret_cast<volatile int*>(gbase + L.off_misc + 8);
@@ -324,24 +385,41 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int sb = j & 1;
       // every give-up is decided jointly (barrier + OR) so no thread is left
       // waiting at a named barrier or inside a warp-collective TMEM access
+      if (EXT && p.mask_rows > 0) {
+        // stage tile j+1's mask rows (and tile 0's first) with cp.async; the
+        // copies stay in flight across this tile's barriers, and tile j's are
+        // complete (and, after the barrier below, visible) before use
+        auto stage = [&](int jj) {
+          const int tile_al = (kbase + jj * BN) & ~7;
+          const uint32_t dst0 = mstage_u32 + (uint32_t)(jj & 1) * p.mask_rows * MROW_BYTES;
+          for (int c = t; c < p.mask_rows * 17; c += 128) {
+            const int row = c / 17, k8 = (c - row * 17) * 8;
+            const int key8 = tile_al + k8;
+            const int n = min(max(hi - key8, 0), 8);   // keys inside the split (hi <= Skv)
+            const uint16_t* src = n > 0 ? p.ext.mask + (size_t)b * p.ext.mask_sb + (size_t)row * p.ext.mask_sr + key8
+                                        : p.ext.mask;
+            cp_async16(dst0 + (uint32_t)row * MROW_BYTES + (uint32_t)k8 * 2u, src, (uint32_t)n * 2u);
+          }
+          cp_async_commit();
+        };
+        if (j == 0) stage(0);
+        if (j + 1 < n_tiles) {
+          stage(j + 1);
+          cp_async_wait<1>();
+        } else {
+          cp_async_wait<0>();
+        }
+      }
       const bool got_s = mbar_wait(bar(BAR_S0 + sb), (uint32_t)(j >> 1) & 1u, wd);
       if (named_bar_or(1, 128, !got_s)) { ok = false; break; }
       tc_fence_after();
       const int tile0 = kbase + j * BN;
       const int key = tile0 + t;
+      // this tile's staged mask at this thread's key
+      const uint16_t* mtile = mstage + (size_t)(j & 1) * p.mask_rows * MROW_KEYS + (tile0 & 7) + t;
       // whole tile visible to every real row: no per-element mask
       const bool full = (tile0 + BN - 1 < hi) && (!p.causal || tile0 + BN - 1 <= q_offset) &&
                         (!EXT || p.ext.window == 0 || tile0 >= q_offset + p.Sq - p.ext.window);
-      // optional terms: logit in log2 units, softcap and ALiBi applied
-      auto logit2 = [&](float sdot, int r) -> float {
-        const float z = p.ext.cap_a > 0.f ? p.ext.cap_b * tanh_approx(sdot * p.ext.cap_a) : sdot * c2;
-        float y = fmaf(slope_sm[r], (float)(key - pos_sm[r]), z);
-        // additive mask, read only inside the split (key < hi <= Skv)
-        const uint16_t* mr = mrow_sm[r];
-        if (mr != nullptr && key < hi)
-          y = fmaf(__uint_as_float((uint32_t)__ldg(mr + key) << 16), 1.4426950408889634f, y);
-        return y;
-      };
       auto visible = [&](int r) -> bool {
         return key < hi && key <= lim_sm[r] && (!EXT || key > limlo_sm[r]);
       };
@@ -349,10 +427,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int q = 0; q < RP / 16; ++q) {
         float v[16];
         tmem_ld16(tmem + lane_off + TS(sb) + 16 * q, v);
-        if (EXT) {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) v[e] = logit2(v[e], 16 * q + e);
-        }
+        if (EXT)
+          ext_rows16(v, p.ext, c2, key, t, q, slope_sm, pos_sm, mtile, p.mask_rows, q_offset, mrow_sm, hi);
         if (!full) {
 #pragma unroll
           for (int e = 0; e < 16; ++e)
@@ -389,10 +465,18 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int q = 0; q < RP / 16; ++q) {
           float v[16];
           tmem_ld16(tmem + lane_off + TS(sb) + 16 * q, v);
+          if (EXT) {
+            ext_rows16(v, p.ext, c2, key, t, q, slope_sm, pos_sm, mtile, p.mask_rows, q_offset, mrow_sm, hi);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float4 w = reinterpret_cast<const float4*>(msub_sm + 16 * q)[i];
+              v[4 * i] -= w.x; v[4 * i + 1] -= w.y; v[4 * i + 2] -= w.z; v[4 * i + 3] -= w.w;
+            }
+          }
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int r = 16 * q + e;
-            float pv = EXT ? ex2_approx(logit2(v[e], r) - msub_sm[r]) : ex2_approx(fmaf(v[e], c2, -msub_sm[r]));
+            float pv = EXT ? ex2_approx(v[e]) : ex2_approx(fmaf(v[e], c2, -msub_sm[r]));
             if (!full && !visible(r)) pv = 0.f;
             *reinterpret_cast<__nv_bfloat16*>(pcol + (size_t)r * 128 + ((chunk16 ^ (r & 7)) << 4)) =
                 __float2bfloat16_rn(pv);
@@ -429,6 +513,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_before();
       mbar_arrive(bar(BAR_P0 + sb));
     }
+    // no mask copy may outlive the loop (it also ends early on a give-up)
+    if (EXT && p.mask_rows > 0) cp_async_wait<0>();
     // ---- epilogue: normalised partial O and the split's LSE ----
     const int last = n_tiles - 1;
     const bool got_o = ok && mbar_wait(bar(BAR_PV0 + (last & 1)), (uint32_t)(last >> 1) & 1u, wd);
@@ -486,7 +572,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 template <int D, bool EXT, bool PAGED>
 int launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
              const DecodeParams& p, cudaStream_t stream) {
-  const Layout L(D, p.RP, p.nbuf);
+  const Layout L(D, p.RP, p.nbuf, p.mask_rows);
   cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, EXT, PAGED>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
   if (e != cudaSuccess) return (int)e;
@@ -505,7 +591,7 @@ int launch_d(bool ext, const CUtensorMap& tq, const CUtensorMap& tk, const CUten
 
 }  // namespace
 
-size_t decode_smem_bytes(int D, int RP, int nbuf) { return Layout(D, RP, nbuf).total; }
+size_t decode_smem_bytes(int D, int RP, int nbuf, int mask_rows) { return Layout(D, RP, nbuf, mask_rows).total; }
 
 int decode_max_nbuf() { return MAX_NBUF; }
 

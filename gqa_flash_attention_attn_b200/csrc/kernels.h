@@ -52,6 +52,7 @@ struct DecodeParams {
   const int* seq_lens;     // [B] or nullptr: every sequence has Skv keys
   const int* block_table;  // [B, max_pages] or nullptr: unpaged
   int max_pages, page_size;
+  int mask_rows;           // query rows whose mask values are staged in shared memory (0: none)
 };
 
 struct MergeParams {
@@ -69,7 +70,7 @@ int launch_prefill(int D, bool ext, const CUtensorMap& tq, const CUtensorMap& tk
 size_t prefill_smem_bytes(int D);
 int launch_decode_split(int D, bool ext, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                         const DecodeParams& p, cudaStream_t stream);
-size_t decode_smem_bytes(int D, int RP, int nbuf);
+size_t decode_smem_bytes(int D, int RP, int nbuf, int mask_rows);
 int launch_merge(const MergeParams& p, cudaStream_t stream);
 int launch_watchdog_selftest(int* status, unsigned long long limit_ns, cudaStream_t stream);
 

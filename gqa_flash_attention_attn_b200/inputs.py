@@ -41,10 +41,13 @@ class Workload:
     # K/V cache layout: 0 = contiguous [B, Skv, Hkv, D]; else paged with this
     # many keys per page (pages scattered by make_paged(k, v, page_size, seed=0))
     page_size: int = 0
+    # additive mask drawn by make_mask(mask_batch, Sq, Skv, seed=0); 0 = none,
+    # 1 = one mask shared by the batch, B = one per sequence
+    mask_batch: int = 0
 
     @property
     def has_options(self) -> bool:
-        return bool(self.softcap or self.alibi_max_bias or self.sinks or self.window)
+        return bool(self.softcap or self.alibi_max_bias or self.sinks or self.window or self.mask_batch)
 
     @property
     def scale(self) -> float:
@@ -121,6 +124,14 @@ WORKLOADS = {
         "split_kv_decode_d512_softcap_alibi_sinks", "decode", B=16, Hq=16, Hkv=1, Sq=1, Skv=16384, D=512,
         q_offset=16383, causal=True, out_dtype="bf16", num_splits=32, softcap=30.0, alibi_max_bias=8.0,
         sinks=True, note="the D512 split-KV decode with softcap 30, ALiBi (max bias 8) and sinks in the merge"),
+    "prefill_4k_d128_mask": Workload(
+        "prefill_4k_d128_mask", "prefill", B=1, Hq=32, Hkv=8, Sq=4096, Skv=4096, D=128,
+        q_offset=0, causal=True, out_dtype="bf16", mask_batch=1,
+        note="the 4k causal GQA prefill plus a shared additive bf16 mask (20 % of entries -inf)"),
+    "spec_verify_decode_d128_mask": Workload(
+        "spec_verify_decode_d128_mask", "decode", B=4, Hq=32, Hkv=8, Sq=8, Skv=32768, D=128,
+        q_offset=32760, causal=True, out_dtype="bf16", num_splits=16, mask_batch=4,
+        note="the 8-row verify decode with a per-sequence additive mask over all keys"),
     "paged_decode_d512_p64": Workload(
         "paged_decode_d512_p64", "decode", B=16, Hq=16, Hkv=1, Sq=1, Skv=16384, D=512,
         q_offset=16383, causal=True, out_dtype="bf16", num_splits=32, page_size=64,

@@ -161,7 +161,7 @@ def test_merge_sinks_on_oracle_partials():
     assert_lse_close(lse, want_lse, "merge sinks")
 
 
-def _rows_oracle_ex(w, q, k, v, rows, sinks):
+def _rows_oracle_ex(w, q, k, v, rows, sinks, mask=None):
     rows_np = np.asarray(rows, dtype=np.int64)
     want_o = np.zeros((len(rows), w.D))
     want_l = np.zeros((len(rows),))
@@ -169,9 +169,10 @@ def _rows_oracle_ex(w, q, k, v, rows, sinks):
         sel = np.nonzero(rows_np[:, 0] == b)[0]
         sub = rows_np[sel].copy()
         sub[:, 0] = 0
+        mb = None if mask is None else mask[b:b + 1] if mask.shape[0] > 1 else mask
         o, l = oracle.attention_rows_ex(q[b:b + 1], k[b:b + 1], v[b:b + 1], sub, scale=w.scale, causal=w.causal,
                                         q_offset=w.q_offset, softcap=w.softcap, alibi_max_bias=w.alibi_max_bias,
-                                        sinks=None if sinks is None else sinks.numpy(), window=w.window)
+                                        sinks=None if sinks is None else sinks.numpy(), window=w.window, mask=mb)
         want_o[sel] = o
         want_l[sel] = l
     return want_o, want_l
@@ -186,9 +187,12 @@ def test_option_workload_full_size_sampled(name):
     launch configuration, on sampled rows."""
     w = WORKLOADS[name]
     q, k, v = make_workload_inputs(w, seed=0)
+    from gqa_flash_attention_attn_b200.inputs import make_mask
     sinks = make_sinks(w.Hq, seed=0) if w.sinks else None
     sk = None if sinks is None else sinks.cuda()
-    terms = dict(softcap=w.softcap, alibi_max_bias=w.alibi_max_bias, window=w.window)
+    mask = make_mask(w.mask_batch, w.Sq, w.Skv, seed=0) if w.mask_batch else None
+    terms = dict(softcap=w.softcap, alibi_max_bias=w.alibi_max_bias, window=w.window,
+                 mask=None if mask is None else mask.cuda())
     if w.kind == "prefill":
         out, lse = ga.prefill(q.cuda(), k.cuda(), v.cuda(), causal=w.causal, q_offset=w.q_offset, scale=w.scale,
                               sinks=sk, **terms)
@@ -199,7 +203,7 @@ def test_option_workload_full_size_sampled(name):
     assert ga.last_status() == ga.ATTN_OK
     rows = sample_rows(w, 40, seed=21)
     got_o, got_l = gather_rows(out, lse, rows)
-    want_o, want_l = _rows_oracle_ex(w, q, k, v, rows, sinks)
+    want_o, want_l = _rows_oracle_ex(w, q, k, v, rows, sinks, mask)
     assert_o_close(got_o, want_o, name)
     assert_lse_close(got_l, want_l, name)
 
@@ -287,3 +291,22 @@ def test_decode_mask_matches_oracle(paged):
                                          alibi_max_bias=2.0, mask=mask, sinks=sinks.numpy())
     assert_o_close(out, want_o, f"decode mask paged={paged}")
     assert_lse_close(lse, want_l, f"decode mask paged={paged}")
+
+
+@pytest.mark.parametrize("shape", [(1, 8, 1, 4, 1001, 256, 3), (1, 4, 2, 40, 700, 128, 2)],
+                         ids=["unaligned_rows", "sq40_unstaged"])
+def test_decode_mask_unstaged_paths(shape):
+    """Masks the decode kernel reads directly instead of staging them: rows
+    that are not 16-byte aligned (Skv = 1001), and more than 32 query rows."""
+    from gqa_flash_attention_attn_b200.inputs import make_mask
+    B, Hq, Hkv, Sq, Skv, D, S = shape
+    q, k, v = make_qkv(B, Hq, Hkv, Sq, Skv, D, seed=59)
+    mask = make_mask(B, Sq, Skv, seed=60)
+    out, lse = ga.decode(q.cuda(), k.cuda(), v.cuda(), S, q_offset=Skv - Sq, out_dtype=torch.float32,
+                         mask=mask.cuda(), alibi_max_bias=1.0)
+    torch.cuda.synchronize()
+    assert ga.last_status() == ga.ATTN_OK
+    want_o, want_l = oracle.attention_ex(q, k, v, scale=_scale(D), causal=True, q_offset=Skv - Sq,
+                                         alibi_max_bias=1.0, mask=mask)
+    assert_o_close(out, want_o, str(shape))
+    assert_lse_close(lse, want_l, str(shape))
