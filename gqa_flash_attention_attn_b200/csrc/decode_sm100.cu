@@ -200,6 +200,11 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int eff_lo = (EXT && p.ext.window > 0) ? max(lo, q_offset - p.ext.window + 1) : lo;
   const int kbase = lo + ((eff_lo - lo) / BN) * BN;   // first tile, on the split's tile grid
   const int n_tiles = eff_hi > eff_lo ? (eff_hi - kbase + BN - 1) / BN : 0;
+  // With ALiBi the bias grows toward each query's own position: visiting the
+  // split's tiles newest first sets the running maximum on the first tile and
+  // spares the O rescales (the tile order does not change the result).
+  const bool rev = EXT && p.ext.alibi != 0;
+  auto tile_key0 = [&](int jj) { return kbase + (rev ? n_tiles - 1 - jj : jj) * BN; };
   const size_t split_out = (size_t)split * p.B * p.Sq * p.Hq * D;
   const size_t split_lse = (size_t)split * p.B * p.Hq * p.Sq;
 
@@ -291,7 +296,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
           mbar_arrive_expect_tx(bar(bar_full(slot)), SLOT_BYTES);
           const uint32_t dst = base + L.off_ring + (uint32_t)slot * SLOT_BYTES;
-          const int key0 = kbase + j * BN;
+          const int key0 = tile_key0(j);
           if constexpr (!PAGED) {
             tma_load_4d(dst, tm, bar(bar_full(slot)), (2 * c) * 64, kvh, key0, b);
             tma_load_4d(dst + BOX_BYTES, tm, bar(bar_full(slot)), (2 * c + 1) * 64, kvh, key0, b);
@@ -390,7 +395,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         // copies stay in flight across this tile's barriers, and tile j's are
         // complete (and, after the barrier below, visible) before use
         auto stage = [&](int jj) {
-          const int tile_al = (kbase + jj * BN) & ~7;
+          const int tile_al = tile_key0(jj) & ~7;
           const uint32_t dst0 = mstage_u32 + (uint32_t)(jj & 1) * p.mask_rows * MROW_BYTES;
           for (int c = t; c < p.mask_rows * 17; c += 128) {
             const int row = c / 17, k8 = (c - row * 17) * 8;
@@ -413,7 +418,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const bool got_s = mbar_wait(bar(BAR_S0 + sb), (uint32_t)(j >> 1) & 1u, wd);
       if (named_bar_or(1, 128, !got_s)) { ok = false; break; }
       tc_fence_after();
-      const int tile0 = kbase + j * BN;
+      const int tile0 = tile_key0(j);
       const int key = tile0 + t;
       // this tile's staged mask at this thread's key
       const uint16_t* mtile = mstage + (size_t)(j & 1) * p.mask_rows * MROW_KEYS + (tile0 & 7) + t;

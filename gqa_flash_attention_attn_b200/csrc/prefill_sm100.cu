@@ -148,8 +148,9 @@ __device__ __forceinline__ int unit_index(int k, int total) {
 //   MODE_MASKS  sliding window and sink logits (no per-element arithmetic)
 //   MODE_ALIBI  ALiBi bias and / or an additive mask, with or without window
 //               and sinks
-//   MODE_CAP    softcap, with or without ALiBi, mask, window and sinks
-constexpr int MODE_PLAIN = 0, MODE_MASKS = 1, MODE_ALIBI = 2, MODE_CAP = 3;
+//   MODE_CAP    softcap, with or without ALiBi, window and sinks
+//   MODE_CAP_MASK  softcap with an additive mask (and any other term)
+constexpr int MODE_PLAIN = 0, MODE_MASKS = 1, MODE_ALIBI = 2, MODE_CAP = 3, MODE_CAP_MASK = 4;
 
 // Logits in log2 units of the N keys of a half tile whose first key sits at
 // distance dist0 = key - pos from the query:
@@ -208,7 +209,7 @@ __device__ __forceinline__ void ext_logits_run(float (&v)[N], const LogitExt& x,
 template <int MODE, bool BIAS, int N>
 __device__ __forceinline__ void ext_logits_m(float (&v)[N], const LogitExt& x, float c2, float slope2, int dist0,
                                              const uint16_t* mk, int nvalid) {
-  if (mk == nullptr)
+  if (MODE == MODE_CAP || mk == nullptr)
     ext_logits_run<MODE, BIAS, 0>(v, x, c2, slope2, dist0, mk, nvalid);
   else if (nvalid >= N && (reinterpret_cast<uintptr_t>(mk) & 15u) == 0)
     ext_logits_run<MODE, BIAS, 1>(v, x, c2, slope2, dist0, mk, nvalid);
@@ -266,6 +267,10 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int total_units = p.n_qt * p.B * p.Hkv * p.units_per_kvh;
+  // With ALiBi the bias grows toward each query's own position: visiting a
+  // unit's K/V tiles newest first sets the running maximum on the first tile
+  // and spares the O rescales (the tile order does not change the result).
+  const bool rev = MODE >= MODE_ALIBI && p.ext.alibi != 0;
 
   if (threadIdx.x == 0) {
     mbar_init(bar(C::BAR_Q), 1);
@@ -332,7 +337,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
           mbar_arrive_expect_tx(bar(C::bar_full(buf)), C::TILE);
           for (int kb = 0; kb < C::KB; ++kb)
             tma_load_4d(base + C::OFF_KV + buf * C::TILE + kb * BOX_BYTES, tm, bar(C::bar_full(buf)),
-                        kb * 64, x.kvh, (x.t0 + tile) * BN, x.b);
+                        kb * 64, x.kvh, (x.t0 + (rev ? x.n_tiles - 1 - tile : tile)) * BN, x.b);
           issued = n + 1;
         }
       }
@@ -506,7 +511,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
       const float slope2 =
           (MODE >= MODE_ALIBI && p.ext.alibi) ? alibi_slope_log2e(h, p.ext.l2m0, p.ext.l2m1, p.ext.n2) : 0.f;
       // this row's mask (padding rows past Sq read the last row's: never stored)
-      const uint16_t* mrow = (MODE >= MODE_ALIBI && p.ext.mask != nullptr)
+      const uint16_t* mrow = ((MODE == MODE_ALIBI || MODE == MODE_CAP_MASK) && p.ext.mask != nullptr)
                                  ? p.ext.mask + (size_t)x.b * p.ext.mask_sb + (size_t)min(s_row, p.Sq - 1) * p.ext.mask_sr
                                  : nullptr;
       float m_use = -INFINITY, l = 0.f;
@@ -520,7 +525,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
         const bool got = mbar_wait(bar(C::bar_s(sb)), ph, wd);
         if (__any_sync(0xffffffffu, !got)) { ok = false; break; }
         tc_fence_after();
-        const int key0 = (x.t0 + j) * BN;
+        const int key0 = (x.t0 + (rev ? n_tiles - 1 - j : j)) * BN;
         const int cl = vis_end - key0;    // visible columns of this tile: [cb, cl)
         const int cb = vis_begin - key0;
         const bool tile_masked = __any_sync(0xffffffffu, cl < BN || cb > 0);
@@ -741,7 +746,8 @@ int launch_mode(int mode, const CUtensorMap& tq, const CUtensorMap& tk, const CU
     case MODE_PLAIN: return launch_t<D, MODE_PLAIN>(tq, tk, tv, p, stream);
     case MODE_MASKS: return launch_t<D, MODE_MASKS>(tq, tk, tv, p, stream);
     case MODE_ALIBI: return launch_t<D, MODE_ALIBI>(tq, tk, tv, p, stream);
-    default: return launch_t<D, MODE_CAP>(tq, tk, tv, p, stream);
+    case MODE_CAP: return launch_t<D, MODE_CAP>(tq, tk, tv, p, stream);
+    default: return launch_t<D, MODE_CAP_MASK>(tq, tk, tv, p, stream);
   }
 }
 
@@ -749,7 +755,7 @@ int launch_prefill(int D, bool ext, const CUtensorMap& tq, const CUtensorMap& tk
                    const PrefillParams& p, cudaStream_t stream) {
   // the cheapest variant that covers the requested terms
   const int mode = !ext ? MODE_PLAIN
-                   : p.ext.cap_a > 0.f ? MODE_CAP
+                   : p.ext.cap_a > 0.f ? (p.ext.mask != nullptr ? MODE_CAP_MASK : MODE_CAP)
                    : (p.ext.alibi || p.ext.mask != nullptr) ? MODE_ALIBI
                    : MODE_MASKS;
   switch (D) {
