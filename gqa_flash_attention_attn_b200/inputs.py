@@ -199,6 +199,21 @@ def make_mask(B, Sq, Skv, *, seed=0, std=2.0, p_inf=0.2, device="cpu"):
     return m.to(torch.bfloat16).to(device)
 
 
+def make_fp8_kv(k, v):
+    """An fp8 e4m3 K/V cache from bf16 k, v [B, Skv, Hkv, D]: per K/V head
+    scale = max |x| / 448 (the largest e4m3 value), codes = x / scale cast to
+    float8_e4m3fn (round to nearest even).  Returns (k_codes, v_codes,
+    k_scale, v_scale): uint8 [B, Skv, Hkv, D] and fp32 [Hkv]."""
+    out = []
+    for x in (k, v):
+        xf = x.float()
+        amax = xf.abs().amax(dim=(0, 1, 3)).clamp_min(1e-12)
+        sc = (amax / 448.0).to(torch.float32)
+        codes = (xf / sc.view(1, 1, -1, 1)).to(torch.float8_e4m3fn).view(torch.uint8)
+        out.append((codes, sc))
+    return out[0][0], out[1][0], out[0][1], out[1][1]
+
+
 def make_workload_inputs(w: Workload, *, seed=0, device="cpu"):
     return make_qkv(w.B, w.Hq, w.Hkv, w.Sq, w.Skv, w.D, seed=seed, device=device)
 

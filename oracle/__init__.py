@@ -21,6 +21,8 @@ Functions and the passage each follows (all pinned by tests/test_oracle_pins.py)
                   publishes its (max, rowsum))
   merge           the LSE combine of split partials (same page, review of the
                   combine kernel for parallel_blocks > 1)
+  attention_fp8   attention over an fp8 e4m3 K/V cache with per-head scales
+                  (decodes each code from the format's definition)
   *_ex            the same with the optional logit terms of the FLASH_ATTN_EXT
                   operator ("ggml-org/llama.cpp PR #28507", Crash 1: sinks,
                   max_bias, logit_softcap, mask) and a sliding window (see oracle.c)
@@ -95,6 +97,12 @@ def _bind(lib):
     lib.oracle_split_ex.restype = None
     lib.oracle_merge_ex.argtypes = [_dp, _dp, _dp, _dp] + [_i64] * 5 + [_dp]
     lib.oracle_merge_ex.restype = None
+    lib.oracle_e4m3_value.argtypes = [ctypes.c_int]
+    lib.oracle_e4m3_value.restype = ctypes.c_double
+    _bp = ctypes.POINTER(ctypes.c_ubyte)
+    lib.oracle_attention_fp8.argtypes = ([_dp, _bp, _bp, _dp, _dp, _dp, _dp] + [_i64] * 7 +
+                                         [ctypes.c_int, ctypes.c_double] + ext)
+    lib.oracle_attention_fp8.restype = None
     lib.oracle_alibi_slope.argtypes = [_i64, _i64, ctypes.c_double]
     lib.oracle_alibi_slope.restype = ctypes.c_double
     return lib
@@ -207,6 +215,48 @@ def _mask_arg(mask, B, Sq, Skv):
         raise ValueError(f"mask must be [B or 1, {Sq}, {Skv}]")
     arr = np.ascontiguousarray(arr)
     return arr, _ptr(arr), (Sq * Skv if arr.shape[0] == B and B > 1 else 0), Skv
+
+
+def e4m3_value(code, lib=None):
+    """The value of one fp8 e4m3 code (0..255)."""
+    return (lib or load()).oracle_e4m3_value(int(code))
+
+
+def attention_fp8(q, k_codes, v_codes, k_scale, v_scale, *, scale, causal=True, q_offset=0, softcap=0.0,
+                  alibi_max_bias=0.0, sinks=None, window=0, mask=None, lib=None):
+    """attention_ex() over an fp8 e4m3 K/V cache: codes uint8 [B, Skv, Hkv, D]
+    (or torch float8_e4m3fn), one fp32 scale per K/V head for K and for V."""
+    lib = lib or load()
+    q = _f64(q)
+    kc, vc = _codes(k_codes), _codes(v_codes)
+    B, Sq, Hq, D = q.shape
+    _, Skv, Hkv, _ = kc.shape
+    ks, vs = _f64(k_scale).reshape(-1), _f64(v_scale).reshape(-1)
+    if ks.shape[0] != Hkv or vs.shape[0] != Hkv:
+        raise ValueError("one K and one V scale per K/V head")
+    sk, skp = _sinks_arg(sinks)
+    mk, mkp, msb, mss = _mask_arg(mask, B, Sq, Skv)
+    out = np.zeros((B, Sq, Hq, D), dtype=np.float64)
+    lse = np.zeros((B, Hq, Sq), dtype=np.float64)
+    _bp = ctypes.POINTER(ctypes.c_ubyte)
+    lib.oracle_attention_fp8(_ptr(q), kc.ctypes.data_as(_bp), vc.ctypes.data_as(_bp), _ptr(ks), _ptr(vs),
+                             _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Skv, D, int(q_offset), int(bool(causal)),
+                             float(scale), float(softcap), float(alibi_max_bias), skp, int(window), mkp, msb, mss)
+    return out, lse
+
+
+def _codes(x):
+    """uint8 codes of an fp8 array (numpy uint8, or a torch uint8 / float8 tensor)."""
+    if hasattr(x, "detach"):  # torch tensor: reinterpret float8 storage as bytes
+        import torch
+        x = x.detach().to("cpu")
+        if x.dtype != torch.uint8:
+            x = x.view(torch.uint8)
+        x = x.numpy()
+    x = np.ascontiguousarray(x)
+    if x.dtype != np.uint8:
+        raise ValueError("fp8 codes must be uint8")
+    return x
 
 
 def alibi_slope(h, Hq, max_bias, lib=None):

@@ -357,6 +357,43 @@ void oracle_merge_ex(const double* pout, const double* plse, double* out, double
     merge_impl(pout, plse, out, lse, B, Hq, Sq, D, num_splits, sinks);
 }
 
+/* Value of an fp8 e4m3 code: 1 sign bit, 4 exponent bits with bias 7 and 3
+ * mantissa bits.  Exponent 0 is subnormal (m/8 * 2^-6); codes 0x7f and 0xff
+ * are NaN; the format has no infinity ("ggml-org/llama.cpp PR #28507",
+ * Setup: the q8_0 K cache; "Anbeeld/beellama.cpp PR #149", Overview: a
+ * quantised K/V cache read by the attention kernel). */
+double oracle_e4m3_value(int code) {
+    const int sign = (code >> 7) & 1, e = (code >> 3) & 15, m = code & 7;
+    double mag;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) mag = ldexp((double)m / 8.0, -6);
+    else mag = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sign ? -mag : mag;
+}
+
+/* Attention over an fp8 e4m3 K/V cache with one scale per K/V head:
+ * K = e4m3(k_codes) * k_scale[kvh], V = e4m3(v_codes) * v_scale[kvh], then
+ * the extended attention above (codes [B, Skv, Hkv, D], one byte each). */
+void oracle_attention_fp8(const double* q, const unsigned char* k_codes, const unsigned char* v_codes,
+                          const double* k_scale, const double* v_scale, double* out, double* lse,
+                          int64_t B, int64_t Hq, int64_t Hkv, int64_t Sq, int64_t Skv, int64_t D,
+                          int64_t q_offset, int causal, double scale,
+                          double softcap, double alibi_max_bias, const double* sinks, int64_t window,
+                          const double* mask, int64_t mask_sb, int64_t mask_ss) {
+    const int64_t n = B * Skv * Hkv * D;
+    double* k = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+    double* v = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+    for (int64_t i = 0; i < n; ++i) {
+        const int64_t kvh = (i / D) % Hkv;
+        k[i] = oracle_e4m3_value(k_codes[i]) * k_scale[kvh];
+        v[i] = oracle_e4m3_value(v_codes[i]) * v_scale[kvh];
+    }
+    const oracle_opts o = make_opts(softcap, alibi_max_bias, sinks, window, mask, mask_sb, mask_ss);
+    attention_impl(q, k, v, out, lse, B, Hq, Hkv, Sq, Skv, D, q_offset, causal, scale, &o);
+    free(k);
+    free(v);
+}
+
 int oracle_num_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();

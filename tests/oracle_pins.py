@@ -552,6 +552,37 @@ def pin_split_merge_mask(lib):
         np.testing.assert_allclose(ml, lse, rtol=0, atol=1e-12)
 
 
+def pin_e4m3_codes_match_torch(lib):
+    """The oracle's e4m3 decoder against torch's float8_e4m3fn for all 256 codes."""
+    codes = torch.arange(256, dtype=torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).double().numpy()
+    got = np.array([oracle.e4m3_value(c, lib=lib) for c in range(256)])
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(got[ok], ref[ok])
+    assert got[0x7e] == 448.0 and got[0x01] == 2.0 ** -9 and got[0x08] == 2.0 ** -6 and got[0xb8] == -1.0
+
+
+def pin_fp8_attention_equals_dequantized(lib):
+    """Attention over fp8 codes with per-head scales equals attention over the
+    values torch decodes, times the scales (non-unit, per head)."""
+    rng = _rng(41)
+    B, Hq, Hkv, Sq, Skv, D = 2, 4, 2, 3, 9, 8
+    q = _normal(rng, (B, Sq, Hq, D))
+    kc = torch.from_numpy(rng.integers(0, 256, (B, Skv, Hkv, D), dtype=np.uint8))
+    vc = torch.from_numpy(rng.integers(0, 256, (B, Skv, Hkv, D), dtype=np.uint8))
+    kc[(kc & 0x7f) == 0x7f] = 0x3c                   # no NaN codes
+    vc[(vc & 0x7f) == 0x7f] = 0x41
+    ks, vs = np.array([0.01, 0.003]), np.array([0.5, 0.02])
+    kd = kc.view(torch.float8_e4m3fn).double().numpy() * ks.reshape(1, 1, -1, 1)
+    vd = vc.view(torch.float8_e4m3fn).double().numpy() * vs.reshape(1, 1, -1, 1)
+    kw = dict(scale=0.3, causal=True, q_offset=Skv - Sq, lib=lib)
+    out, lse = oracle.attention_fp8(q, kc, vc, ks, vs, **kw)
+    ref_o, ref_l = oracle.attention(q, kd, vd, **kw)
+    np.testing.assert_array_equal(out, ref_o)
+    np.testing.assert_array_equal(lse, ref_l)
+
+
 ALL_PINS = [
     pin_bruteforce_decimal,
     pin_golden_three_keys,
@@ -578,4 +609,6 @@ ALL_PINS = [
     pin_mask_removes_keys_and_shifts,
     pin_mask_fully_masked_row,
     pin_split_merge_mask,
+    pin_e4m3_codes_match_torch,
+    pin_fp8_attention_equals_dequantized,
 ]

@@ -43,6 +43,12 @@ MUTANTS = [
     ("mask_batch_ignored", "z[t - t_lo] += opt->mask[b * opt->mask_sb + s * opt->mask_ss + t];",
      "z[t - t_lo] += opt->mask[s * opt->mask_ss + t];"),
     ("masked_row_not_empty", "if (m == -INFINITY) return -INFINITY;", ""),
+    ("e4m3_bias_8", "else mag = ldexp(1.0 + (double)m / 8.0, e - 7);", "else mag = ldexp(1.0 + (double)m / 8.0, e - 8);"),
+    ("e4m3_subnormal_as_normal", "if (e == 0) mag = ldexp((double)m / 8.0, -6);",
+     "if (e == 0) mag = ldexp(1.0 + (double)m / 8.0, -7);"),
+    ("e4m3_sign_dropped", "return sign ? -mag : mag;", "return mag;"),
+    ("fp8_v_scale_from_k", "v[i] = oracle_e4m3_value(v_codes[i]) * v_scale[kvh];",
+     "v[i] = oracle_e4m3_value(v_codes[i]) * k_scale[kvh];"),
     ("window_off_by_one", "if (opt && opt->window > 0 && pos - opt->window + 1 > first) first = pos - opt->window + 1;",
      "if (opt && opt->window > 0 && pos - opt->window > first) first = pos - opt->window;"),
     ("merge_sink_dropped", "double wsum = sinks ? exp(sinks[h] - M) : 0.0;", "double wsum = 0.0;"),
