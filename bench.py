@@ -164,9 +164,13 @@ def make_runner(ga, w, device):
     """Device-resident inputs/outputs and a closure that launches one step.
     Returns (step_fn, n_kernels_per_step, events_split) where the closure
     records optional inner events between the split and the merge."""
-    from gqa_flash_attention_attn_b200.inputs import make_mask, make_paged, make_qkv, make_sinks
+    from gqa_flash_attention_attn_b200.inputs import make_fp8_kv, make_mask, make_paged, make_qkv, make_sinks
     q, k, v = make_qkv(w.B, w.Hq, w.Hkv, w.Sq, w.Skv, w.D, seed=0, device=device)
     bt = None
+    scales = {}
+    if w.kv_dtype == "fp8":
+        k, v, ks, vs = make_fp8_kv(k, v)
+        scales = dict(k_scale=ks, v_scale=vs)
     if w.page_size:
         kc, vc, bt = make_paged(k.cpu(), v.cpu(), w.page_size, seed=0)
         k, v, bt = kc.to(device), vc.to(device), bt.to(device)
@@ -185,12 +189,12 @@ def make_runner(ga, w, device):
     pl = torch.empty((w.num_splits, w.B, w.Hq, w.Sq), dtype=torch.float32, device=device)
 
     def step(mid=None):
-        if bt is None:
+        if bt is None and not scales:
             ga.decode_split(q, k, v, w.num_splits, causal=w.causal, q_offset=w.q_offset, scale=w.scale,
                             partial_out=po, partial_lse=pl, **terms)
         else:
             ga.decode_split_kv(q, k, v, w.num_splits, block_table=bt, causal=w.causal, q_offset=w.q_offset,
-                               scale=w.scale, partial_out=po, partial_lse=pl, **terms)
+                               scale=w.scale, partial_out=po, partial_lse=pl, **scales, **terms)
         if mid is not None:
             mid.record()
         ga.merge(po, pl, out=out, lse=lse, sinks=sinks)

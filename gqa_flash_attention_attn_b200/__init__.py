@@ -24,7 +24,7 @@ __all__ = [
     "merge", "decode", "decode_workspace_bytes", "last_status", "status_string",
     "watchdog_selftest", "version", "ATTN_OK", "ATTN_ERR_INVALID_ARG", "ATTN_ERR_UNSUPPORTED",
     "ATTN_ERR_ALIGNMENT", "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT", "ATTN_ERR_TOO_LARGE", "decode_noalloc",
-    "AttnOptions", "AttnKVView", "decode_split_kv", "decode_kv",
+    "AttnOptions", "AttnKVView", "decode_split_kv", "decode_kv", "ATTN_FP8_E4M3",
 ]
 
 ATTN_OK = 0
@@ -147,22 +147,40 @@ class AttnKVView(ctypes.Structure):
     _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("stride_seq", ctypes.c_longlong),
                 ("stride_token", ctypes.c_longlong), ("stride_head", ctypes.c_longlong),
                 ("block_table", ctypes.c_void_p), ("max_pages", ctypes.c_int), ("page_size", ctypes.c_int),
-                ("num_pages", ctypes.c_int), ("seq_lens", ctypes.c_void_p)]
+                ("num_pages", ctypes.c_int), ("seq_lens", ctypes.c_void_p), ("kv_dtype", ctypes.c_int),
+                ("k_scale", ctypes.c_void_p), ("v_scale", ctypes.c_void_p)]
 
 
-def _kv_view(k, v, block_table, seq_lens):
-    """AttnKVView of k/v (4-D bf16 views with a contiguous last dim) and Skv.
+ATTN_FP8_E4M3 = 2
+_FP8_DTYPES = (torch.uint8, torch.float8_e4m3fn)
+
+
+def _kv_view(k, v, block_table, seq_lens, k_scale=None, v_scale=None):
+    """AttnKVView of k/v (4-D views with a contiguous last dim) and Skv.
 
     Unpaged: k, v are [B, Skv, Hkv, D] views.  Paged: k, v are
-    [num_pages, page_size, Hkv, D] views and block_table is int32 [B, max_pages]."""
+    [num_pages, page_size, Hkv, D] views and block_table is int32 [B, max_pages].
+    bf16 K/V, or fp8 e4m3 codes (uint8 or float8_e4m3fn) with fp32 per-head
+    k_scale and v_scale [Hkv]."""
+    fp8 = isinstance(k, torch.Tensor) and k.dtype in _FP8_DTYPES
     for t, n in ((k, "k"), (v, "v")):
-        if not isinstance(t, torch.Tensor) or t.device.type != "cuda" or t.dtype != torch.bfloat16 or t.dim() != 4:
-            raise ValueError(f"{n} must be a 4-D bf16 CUDA tensor")
+        ok_dtype = t.dtype in _FP8_DTYPES if fp8 else t.dtype == torch.bfloat16
+        if not isinstance(t, torch.Tensor) or t.device.type != "cuda" or not ok_dtype or t.dim() != 4:
+            raise ValueError(f"{n} must be a 4-D CUDA tensor, bf16 or fp8 e4m3 like the other")
         if t.stride(3) != 1:
             raise ValueError(f"{n} must be contiguous in its last dimension")
     if k.shape != v.shape or k.stride() != v.stride():
         raise ValueError("k and v must have the same shape and strides")
-    view = AttnKVView(k.data_ptr(), v.data_ptr(), k.stride(0), k.stride(1), k.stride(2), None, 0, 0, 0, None)
+    view = AttnKVView(k.data_ptr(), v.data_ptr(), k.stride(0), k.stride(1), k.stride(2), None, 0, 0, 0, None,
+                      0, None, None)
+    if fp8:
+        for sc, n in ((k_scale, "k_scale"), (v_scale, "v_scale")):
+            _need(sc, n, torch.float32, 1)
+            if sc.shape[0] != k.shape[2]:
+                raise ValueError(f"{n} must have one entry per K/V head")
+        view.kv_dtype = ATTN_FP8_E4M3
+        view.k_scale = k_scale.data_ptr()
+        view.v_scale = v_scale.data_ptr()
     if block_table is not None:
         _need(block_table, "block_table", torch.int32, 2)
         view.block_table = block_table.data_ptr()
@@ -312,17 +330,19 @@ def decode(q, k, v, num_splits, *, causal=True, q_offset=0, scale=None, out_dtyp
 
 def decode_split_kv(q, k, v, num_splits, *, block_table=None, seq_lens=None, causal=True, q_offset=0,
                     scale=None, partial_out=None, partial_lse=None, stream=None, softcap=0.0,
-                    alibi_max_bias=0.0, window=0, mask=None):
+                    alibi_max_bias=0.0, window=0, mask=None, k_scale=None, v_scale=None):
     """decode_split over a strided or paged K/V cache (see attn_kv_view).
 
     Unpaged: k, v are [B, Skv, Hkv, D] views (any strides, last dim
     contiguous).  Paged: k, v are [num_pages, page_size, Hkv, D] and
     block_table int32 [B, max_pages] maps logical to physical pages.
+    fp8 e4m3 K/V: k, v as uint8 codes (or float8_e4m3fn) with fp32 k_scale,
+    v_scale [Hkv]: K = code * k_scale[kvh], V = code * v_scale[kvh].
     seq_lens (int32 [B], optional): keys per sequence; the query rows then sit
     at the last Sq positions of each sequence and q_offset is ignored."""
     _need(q, "q", torch.bfloat16, 4)
     B, Sq, Hq, D = q.shape
-    view, Skv = _kv_view(k, v, block_table, seq_lens)
+    view, Skv = _kv_view(k, v, block_table, seq_lens, k_scale, v_scale)
     Hkv = k.shape[2]
     if k.shape[3] != D:
         raise ValueError("k/v head size does not match q")
@@ -347,14 +367,15 @@ def decode_split_kv(q, k, v, num_splits, *, block_table=None, seq_lens=None, cau
 
 def decode_kv(q, k, v, num_splits, *, block_table=None, seq_lens=None, causal=True, q_offset=0, scale=None,
               out_dtype=torch.bfloat16, workspace=None, out=None, lse=None, stream=None, softcap=0.0,
-              alibi_max_bias=0.0, sinks=None, window=0, mask=None):
+              alibi_max_bias=0.0, sinks=None, window=0, mask=None, k_scale=None, v_scale=None):
     """decode_split_kv followed by the LSE merge (two launches on one stream)."""
     po = pl = None
     if workspace is not None:
         po, pl = workspace
     po, pl = decode_split_kv(q, k, v, num_splits, block_table=block_table, seq_lens=seq_lens, causal=causal,
                              q_offset=q_offset, scale=scale, partial_out=po, partial_lse=pl, stream=stream,
-                             softcap=softcap, alibi_max_bias=alibi_max_bias, window=window, mask=mask)
+                             softcap=softcap, alibi_max_bias=alibi_max_bias, window=window, mask=mask,
+                             k_scale=k_scale, v_scale=v_scale)
     return merge(po, pl, out_dtype=out_dtype, out=out, lse=lse, stream=stream, sinks=sinks)
 
 

@@ -68,18 +68,21 @@ int* status_ptr() {
   return g_status_ptr[dev];
 }
 
-// bf16 tensor with dimensions d0 (innermost, contiguous) .. d3 and element
-// strides s1..s3 of the outer three, tiled with 128-byte swizzle.
+// Tensor with dimensions d0 (innermost, contiguous) .. d3 and element strides
+// s1..s3 of the outer three, tiled with 128-byte swizzle; bf16, or one-byte
+// codes when fp8.
 bool make_map_strided(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t d3,
-                      uint64_t s1, uint64_t s2, uint64_t s3, uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
+                      uint64_t s1, uint64_t s2, uint64_t s3, uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3,
+                      bool fp8 = false) {
   EncodeTiledFn enc = encoder();
   if (enc == nullptr) return false;
+  const uint64_t eb = fp8 ? 1 : 2;
   const cuuint64_t dims[4] = {d0, d1, d2, d3};
-  const cuuint64_t strides[3] = {s1 * 2, s2 * 2, s3 * 2};
+  const cuuint64_t strides[3] = {s1 * eb, s2 * eb, s3 * eb};
   const cuuint32_t box[4] = {b0, b1, b2, b3};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   std::memset(m, 0, sizeof(*m));
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+  return enc(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -150,7 +153,7 @@ int make_ext(const attn_options* opt, int Hq, int Sq, int Skv, int q_offset, int
 
 extern "C" {
 
-int attn_version(void) { return 0x000200; }
+int attn_version(void) { return 0x000300; }
 
 const char* attn_status_string(int status) {
   switch (status) {
@@ -277,10 +280,15 @@ int attn_decode_split_kv(const void* q, const attn_kv_view* kv, float* partial_o
     if (!aligned(kv->block_table, 4)) return ATTN_ERR_ALIGNMENT;
   }
   if (kv->seq_lens != nullptr && !aligned(kv->seq_lens, 4)) return ATTN_ERR_ALIGNMENT;
+  if (kv->kv_dtype != ATTN_BF16 && kv->kv_dtype != ATTN_FP8_E4M3) return ATTN_ERR_INVALID_ARG;
+  const bool fp8 = kv->kv_dtype == ATTN_FP8_E4M3;
+  if (fp8 && (kv->k_scale == nullptr || kv->v_scale == nullptr || !aligned(kv->k_scale, 4) ||
+              !aligned(kv->v_scale, 4)))
+    return ATTN_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(partial_out, 16))
     return ATTN_ERR_ALIGNMENT;
   for (long long x : strides)
-    if (x % 8 != 0) return ATTN_ERR_ALIGNMENT;
+    if (x % (fp8 ? 16 : 8) != 0) return ATTN_ERR_ALIGNMENT;
   if (!aligned(partial_lse, 4)) return ATTN_ERR_ALIGNMENT;
 
   gqa::DecodeParams p{};
@@ -299,7 +307,7 @@ int attn_decode_split_kv(const void* q, const attn_kv_view* kv, float* partial_o
                     : 0;
   int nbuf = 2;
   while (nbuf < gqa::decode_max_nbuf() &&
-         gqa::decode_smem_bytes(D, p.RP, nbuf + 1, p.mask_rows) <= kTwoCtaSmemLimit)
+         gqa::decode_smem_bytes(D, p.RP, nbuf + 1, p.mask_rows, fp8) <= kTwoCtaSmemLimit)
     ++nbuf;
   p.nbuf = nbuf;
   p.c2 = scale * kLog2e;
@@ -309,6 +317,8 @@ int attn_decode_split_kv(const void* q, const attn_kv_view* kv, float* partial_o
   p.block_table = kv->block_table;
   p.max_pages = paged ? kv->max_pages : 0;
   p.page_size = paged ? kv->page_size : 0;
+  p.k_scale = fp8 ? kv->k_scale : nullptr;
+  p.v_scale = fp8 ? kv->v_scale : nullptr;
 
   p.status = status_ptr();
   if (p.status == nullptr) return cuda_fail();
@@ -319,9 +329,10 @@ int attn_decode_split_kv(const void* q, const attn_kv_view* kv, float* partial_o
   const uint64_t d3 = paged ? (uint64_t)kv->num_pages : (uint64_t)B;
   const uint32_t rows = paged && kv->page_size < 128 ? (uint32_t)kv->page_size : 128u;
   const uint64_t s1 = (uint64_t)kv->stride_head, s2 = (uint64_t)kv->stride_token, s3 = (uint64_t)kv->stride_seq;
-  if (!make_map_strided(&tk, k, D, Hkv, d2, d3, s1, s2, s3, 64, 1, rows, 1)) return cuda_fail();
-  if (!make_map_strided(&tv, v, D, Hkv, d2, d3, s1, s2, s3, 64, 1, rows, 1)) return cuda_fail();
-  return gqa::launch_decode_split(D, ext_on, tq, tk, tv, p, static_cast<cudaStream_t>(stream)) == 0 ? ATTN_OK
+  const uint32_t b0 = fp8 ? 128u : 64u;   // 128-byte box rows either way
+  if (!make_map_strided(&tk, k, D, Hkv, d2, d3, s1, s2, s3, b0, 1, rows, 1, fp8)) return cuda_fail();
+  if (!make_map_strided(&tv, v, D, Hkv, d2, d3, s1, s2, s3, b0, 1, rows, 1, fp8)) return cuda_fail();
+  return gqa::launch_decode_split(D, ext_on, fp8, tq, tk, tv, p, static_cast<cudaStream_t>(stream)) == 0 ? ATTN_OK
                                                                                                : ATTN_ERR_CUDA;
 }
 

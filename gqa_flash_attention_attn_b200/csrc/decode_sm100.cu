@@ -43,19 +43,22 @@ constexpr int MROW_KEYS = 136;
 constexpr uint32_t MROW_BYTES = MROW_KEYS * 2u;
 
 struct Layout {
-  uint32_t off_q, off_p, off_ring, off_red, off_row, off_mask, off_bar, off_misc, total;
-  // mrows: query rows s whose additive-mask values are staged per tile
-  __host__ __device__ Layout(int D, int RP, int nbuf, int mrows) {
+  uint32_t off_q, off_q8, off_p, off_ring, off_red, off_row, off_mask, off_bar, off_misc, total;
+  // mrows: query rows s whose additive-mask values are staged per tile;
+  // fp8: K/V slots of 128 e4m3 columns (16 KB) and Q as two e4m3 planes
+  __host__ __device__ Layout(int D, int RP, int nbuf, int mrows, bool fp8) {
     off_q = 0;
     const uint32_t qbytes = (uint32_t)(D / 64) * RP * 128u;
-    off_p = (off_q + qbytes + 1023u) & ~1023u;
+    off_q8 = (off_q + qbytes + 1023u) & ~1023u;
+    const uint32_t q8bytes = fp8 ? 2u * (uint32_t)(D / 128) * RP * 128u : 0u;   // hi, lo planes
+    off_p = (off_q8 + q8bytes + 1023u) & ~1023u;
     off_ring = (off_p + 2u * 2u * RP * 128u + 1023u) & ~1023u;  // two P buffers
-    off_red = off_ring + (uint32_t)nbuf * SLOT_BYTES;
+    off_red = off_ring + (uint32_t)nbuf * (fp8 ? BOX_BYTES : SLOT_BYTES);
     off_row = off_red + 2u * 4u * RP * 4u;     // red_max[4][RP], red_sum[4][RP]
     off_mask = off_row + 11u * RP * 4u;        // m, l, alpha, msub, inv, lim, limlo, pos, slope, mask row
     off_bar = off_mask + (uint32_t)mrows * 2u * MROW_BYTES;  // staged mask [2][mrows][136 keys] bf16
     off_bar = (off_bar + 7u) & ~7u;
-    off_misc = off_bar + (uint32_t)(1 + 2 * nbuf + 7) * 8u;
+    off_misc = off_bar + (uint32_t)(1 + 2 * nbuf + 8) * 8u;
     total = off_misc + 16u + 1024u;
   }
 };
@@ -138,13 +141,14 @@ __device__ __forceinline__ void ext_rows16(float (&v)[16], const LogitExt& x, fl
   }
 }
 
-template <int D, bool EXT, bool PAGED>
+template <int D, bool EXT, bool PAGED, bool FP8>
 __global__ void __launch_bounds__(THREADS, 1)
     decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
   constexpr int KC = D / 128;  // 128-column slots per K (or V) tile
   const int RP = p.RP, R = p.R, g = p.g, nbuf = p.nbuf;
-  const Layout L(D, RP, nbuf, p.mask_rows);
+  const Layout L(D, RP, nbuf, p.mask_rows, FP8);
+  constexpr uint32_t SLOTB = FP8 ? BOX_BYTES : SLOT_BYTES;   // bytes of one 128-column K/V slot
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -177,6 +181,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int BAR_P0 = BAR_S0 + 2;         // p_full[2]
   const int BAR_PV0 = BAR_S0 + 4;        // pv_done per P buffer [2]
   const int BAR_DRAIN = BAR_S0 + 6;
+  const int BAR_Q8 = BAR_S0 + 7;         // fp8: Q planes written
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = blockIdx.x;
@@ -255,6 +260,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(bar(BAR_PV0 + i), 1);
     }
     mbar_init(bar(BAR_DRAIN), 1);
+    mbar_init(bar(BAR_Q8), 1);
     *abort_flag = 0;
     *resc_flag = 0;
     fence_mbar_init();
@@ -294,12 +300,16 @@ __global__ void __launch_bounds__(THREADS, 1)
             ok = false;
             return;
           }
-          mbar_arrive_expect_tx(bar(bar_full(slot)), SLOT_BYTES);
-          const uint32_t dst = base + L.off_ring + (uint32_t)slot * SLOT_BYTES;
+          mbar_arrive_expect_tx(bar(bar_full(slot)), SLOTB);
+          const uint32_t dst = base + L.off_ring + (uint32_t)slot * SLOTB;
           const int key0 = tile_key0(j);
           if constexpr (!PAGED) {
-            tma_load_4d(dst, tm, bar(bar_full(slot)), (2 * c) * 64, kvh, key0, b);
-            tma_load_4d(dst + BOX_BYTES, tm, bar(bar_full(slot)), (2 * c + 1) * 64, kvh, key0, b);
+            if (FP8) {
+              tma_load_4d(dst, tm, bar(bar_full(slot)), c * 128, kvh, key0, b);   // 128 e4m3 columns
+            } else {
+              tma_load_4d(dst, tm, bar(bar_full(slot)), (2 * c) * 64, kvh, key0, b);
+              tma_load_4d(dst + BOX_BYTES, tm, bar(bar_full(slot)), (2 * c + 1) * 64, kvh, key0, b);
+            }
           } else {
             // paged: each page-sized run of keys from its physical page (the
             // tensor map's outer dimensions are row-in-page and page); a
@@ -311,9 +321,13 @@ __global__ void __launch_bounds__(THREADS, 1)
               const int lp = key / ps;
               const int page = lp < p.max_pages ? __ldg(bt + lp) : -1;
               const uint32_t off = (uint32_t)(sub * rows) * 128u;
-              tma_load_4d(dst + off, tm, bar(bar_full(slot)), (2 * c) * 64, kvh, key - lp * ps, page);
-              tma_load_4d(dst + BOX_BYTES + off, tm, bar(bar_full(slot)), (2 * c + 1) * 64, kvh, key - lp * ps,
-                          page);
+              if (FP8) {
+                tma_load_4d(dst + off, tm, bar(bar_full(slot)), c * 128, kvh, key - lp * ps, page);
+              } else {
+                tma_load_4d(dst + off, tm, bar(bar_full(slot)), (2 * c) * 64, kvh, key - lp * ps, page);
+                tma_load_4d(dst + BOX_BYTES + off, tm, bar(bar_full(slot)), (2 * c + 1) * 64, kvh, key - lp * ps,
+                            page);
+              }
             }
           }
           issued = n + 1;
@@ -327,9 +341,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else if (warp == WARP_MMA) {
     if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16_f32(128, RP, false, false);
-      const uint32_t idesc_o = idesc_bf16_f32(128, RP, true, false);
-      bool ok = mbar_wait(bar(BAR_Q), 0, wd);
+      const uint32_t idesc_s = FP8 ? idesc_e4m3_f32(128, RP, false, false) : idesc_bf16_f32(128, RP, false, false);
+      const uint32_t idesc_o = FP8 ? idesc_e4m3_f32(128, RP, true, false) : idesc_bf16_f32(128, RP, true, false);
+      // fp8: the softmax warps turn Q into two e4m3 planes first
+      bool ok = mbar_wait(bar(FP8 ? BAR_Q8 : BAR_Q), 0, wd);
       tc_fence_after();
       int n = 0;
       // S^T_j = K_j Q^T into S buffer j%2, one 128-column slot at a time
@@ -338,14 +353,29 @@ __global__ void __launch_bounds__(THREADS, 1)
           const int slot = n % nbuf;
           if (!mbar_wait(bar(bar_full(slot)), (uint32_t)(n / nbuf) & 1u, wd)) { ok = false; return; }
           tc_fence_after();
-          const uint32_t kb = base + L.off_ring + (uint32_t)slot * SLOT_BYTES;
+          const uint32_t kb = base + L.off_ring + (uint32_t)slot * SLOTB;
+          if constexpr (FP8) {
+            // K rows of 128 e4m3 (one 128-byte swizzled row); Q as hi + lo
+            // planes: S^T = K Q_hi^T + K Q_lo^T, 32 columns per MMA
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t in_box = (uint32_t)(kk & 3) * 32u;
-            const uint32_t a = kb + (uint32_t)(kk >> 2) * BOX_BYTES + in_box;
-            const uint32_t qb = base + L.off_q + (uint32_t)(2 * c + (kk >> 2)) * RP * 128u + in_box;
-            mma_ss(tmem + TS(j & 1), sdesc_sw128(a, 16, 1024), sdesc_sw128(qb, 16, 1024), idesc_s,
-                   (c > 0 || kk > 0) ? 1u : 0u);
+            for (int pl = 0; pl < 2; ++pl) {
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint32_t a = kb + (uint32_t)kk * 32u;
+                const uint32_t qb = base + L.off_q8 + (uint32_t)(pl * KC + c) * RP * 128u + (uint32_t)kk * 32u;
+                mma_ss_f8(tmem + TS(j & 1), sdesc_sw128(a, 16, 1024), sdesc_sw128(qb, 16, 1024), idesc_s,
+                          (c > 0 || pl > 0 || kk > 0) ? 1u : 0u);
+              }
+            }
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t in_box = (uint32_t)(kk & 3) * 32u;
+              const uint32_t a = kb + (uint32_t)(kk >> 2) * BOX_BYTES + in_box;
+              const uint32_t qb = base + L.off_q + (uint32_t)(2 * c + (kk >> 2)) * RP * 128u + in_box;
+              mma_ss(tmem + TS(j & 1), sdesc_sw128(a, 16, 1024), sdesc_sw128(qb, 16, 1024), idesc_s,
+                     (c > 0 || kk > 0) ? 1u : 0u);
+            }
           }
           mma_commit(bar(bar_empty(slot)));
         }
@@ -366,13 +396,28 @@ __global__ void __launch_bounds__(THREADS, 1)
           const int slot = n % nbuf;
           if (!mbar_wait(bar(bar_full(slot)), (uint32_t)(n / nbuf) & 1u, wd)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t vb = base + L.off_ring + (uint32_t)slot * SLOT_BYTES;
+          const uint32_t vb = base + L.off_ring + (uint32_t)slot * SLOTB;
+          if constexpr (FP8) {
+            // V^T (MN-major: a 128-byte row holds 128 d-columns of one key),
+            // 32 keys per MMA; P^T as hi + lo planes of 128 keys per row
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t a = vb + (uint32_t)kk * 2048u;
-            const uint32_t pb = base + PB(j & 1) + (uint32_t)(kk >> 2) * RP * 128u + (uint32_t)(kk & 3) * 32u;
-            mma_ss(tmem + TO(c), sdesc_sw128(a, BOX_BYTES, 1024), sdesc_sw128(pb, 16, 1024), idesc_o,
-                   (j > 0 || kk > 0) ? 1u : 0u);
+            for (int pl = 0; pl < 2; ++pl) {
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint32_t a = vb + (uint32_t)kk * 4096u;
+                const uint32_t pb = base + PB(j & 1) + (uint32_t)pl * RP * 128u + (uint32_t)kk * 32u;
+                mma_ss_f8(tmem + TO(c), sdesc_sw128(a, BOX_BYTES, 1024), sdesc_sw128(pb, 16, 1024), idesc_o,
+                          (j > 0 || pl > 0 || kk > 0) ? 1u : 0u);
+              }
+            }
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t a = vb + (uint32_t)kk * 2048u;
+              const uint32_t pb = base + PB(j & 1) + (uint32_t)(kk >> 2) * RP * 128u + (uint32_t)(kk & 3) * 32u;
+              mma_ss(tmem + TO(c), sdesc_sw128(a, BOX_BYTES, 1024), sdesc_sw128(pb, 16, 1024), idesc_o,
+                     (j > 0 || kk > 0) ? 1u : 0u);
+            }
           }
           mma_commit(bar(bar_empty(slot)));
         }
@@ -384,9 +429,71 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ---- softmax: thread t <-> key t of the tile (TMEM lane t) ----
     const int t = threadIdx.x;          // 0..127
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    const float c2 = p.c2;
+    float c2 = p.c2;          // logit scale * log2(e) (times the K scale with fp8 K/V)
+    LogitExt xe = p.ext;      // the optional terms (softcap rescaled with fp8 K/V)
+    float vs = 1.f;           // V scale applied in the epilogue
     bool ok = true;
-    for (int j = 0; j < n_tiles; ++j) {
+    if constexpr (FP8) {
+      // Q -> two e4m3 planes, hi and lo, of q * qs with qs a power of two that
+      // puts max |q| in [128, 256): hi + lo holds every bf16 value exactly
+      // (4 + 4 significant bits) unless it underflows below 2^-17 of max |q|.
+      // The MMAs then give K_code . (q * qs); the logit scale takes
+      // k_scale / qs.
+      const bool got_q = mbar_wait(bar(BAR_Q), 0, wd);
+      if (named_bar_or(1, 128, !got_q)) {
+        ok = false;
+      } else {
+        tc_fence_after();
+        const int cpr = D / 8;   // 16-byte chunks of 8 bf16 per row
+        auto qoff = [&](int r, int col) -> uint32_t {
+          return (uint32_t)(col >> 6) * RP * 128u + (uint32_t)r * 128u + ((uint32_t)(((col & 63) >> 3) ^ (r & 7)) << 4);
+        };
+        float amax = 0.f;
+        for (int i = t; i < RP * cpr; i += 128) {
+          const int r = i / cpr, col = (i - r * cpr) * 8;
+          const uint4 w = *reinterpret_cast<const uint4*>(gbase + L.off_q + qoff(r, col));
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            amax = fmax3(amax, fabsf(__uint_as_float(ww[k] << 16)), fabsf(__uint_as_float(ww[k] & 0xffff0000u)));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        if (lane == 0) red_sum[warp] = amax;
+        named_bar_sync(1, 128);
+        const float qmax = fmaxf(fmaxf(red_sum[0], red_sum[1]), fmaxf(red_sum[2], red_sum[3]));
+        const int ex = max((__float_as_int(qmax) >> 23) - 127, -120);
+        const float qs = qmax > 0.f ? __int_as_float((127 + 7 - ex) << 23) : 1.f;
+        for (int i = t; i < RP * cpr; i += 128) {
+          const int r = i / cpr, col = (i - r * cpr) * 8;
+          const uint4 w = *reinterpret_cast<const uint4*>(gbase + L.off_q + qoff(r, col));
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+          uint32_t hi[2], lo[2];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float x0 = __uint_as_float(ww[k] << 16) * qs, x1 = __uint_as_float(ww[k] & 0xffff0000u) * qs;
+            const uint32_t h = e4m3x2_from(x0, x1);
+            const float2 bk = e4m3x2_value(h);
+            const uint32_t l = e4m3x2_from(x0 - bk.x, x1 - bk.y);
+            hi[k >> 1] = (k & 1) ? (hi[k >> 1] | (h << 16)) : h;
+            lo[k >> 1] = (k & 1) ? (lo[k >> 1] | (l << 16)) : l;
+          }
+          const int c8 = col & 127;
+          const uint32_t o8 = (uint32_t)(col >> 7) * RP * 128u + (uint32_t)r * 128u +
+                              ((uint32_t)((c8 >> 4) ^ (r & 7)) << 4) + (uint32_t)(c8 & 15);
+          *reinterpret_cast<uint2*>(gbase + L.off_q8 + o8) = make_uint2(hi[0], hi[1]);
+          *reinterpret_cast<uint2*>(gbase + L.off_q8 + (uint32_t)KC * RP * 128u + o8) = make_uint2(lo[0], lo[1]);
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (t == 0) mbar_arrive(bar(BAR_Q8));
+        const float kq = __ldg(p.k_scale + kvh) / qs;
+        c2 *= kq;
+        if (xe.cap_a > 0.f) xe.cap_a *= kq;
+        vs = __ldg(p.v_scale + kvh);
+      }
+    }
+    for (int j = 0; ok && j < n_tiles; ++j) {
       const int sb = j & 1;
       // every give-up is decided jointly (barrier + OR) so no thread is left
       // waiting at a named barrier or inside a warp-collective TMEM access
@@ -433,7 +540,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         float v[16];
         tmem_ld16(tmem + lane_off + TS(sb) + 16 * q, v);
         if (EXT)
-          ext_rows16(v, p.ext, c2, key, t, q, slope_sm, pos_sm, mtile, p.mask_rows, q_offset, mrow_sm, hi);
+          ext_rows16(v, xe, c2, key, t, q, slope_sm, pos_sm, mtile, p.mask_rows, q_offset, mrow_sm, hi);
         if (!full) {
 #pragma unroll
           for (int e = 0; e < 16; ++e)
@@ -448,14 +555,16 @@ __global__ void __launch_bounds__(THREADS, 1)
         const float m_tile = EXT ? mt : mt * c2;
         const float m_old = m_sm[t];
         float m_new = m_old, alpha = 1.f;
-        if (m_tile > m_old + 8.f) {
+        // stale-maximum threshold: 8 (log2 units) keeps p <= 2^8 for bf16 P;
+        // fp8 P is stored as 64 p (p <= 4 keeps it <= 256, inside e4m3)
+        if (m_tile > m_old + (FP8 ? 2.f : 8.f)) {
           m_new = m_tile;
           alpha = ex2_approx(m_old - m_new);
           *resc_flag = 1;
         }
         m_sm[t] = m_new;
         alpha_sm[t] = alpha;
-        msub_sm[t] = (m_new == -INFINITY) ? 0.f : m_new;
+        msub_sm[t] = (m_new == -INFINITY) ? 0.f : m_new - (FP8 ? 6.f : 0.f);
       }
       // P buffer sb was read by the P.V of tile j-2: wait for it before rewriting
       const bool got_pb = (j < 2) || mbar_wait(bar(BAR_PV0 + sb), (uint32_t)((j - 2) >> 1) & 1u, wd);
@@ -471,7 +580,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           float v[16];
           tmem_ld16(tmem + lane_off + TS(sb) + 16 * q, v);
           if (EXT) {
-            ext_rows16(v, p.ext, c2, key, t, q, slope_sm, pos_sm, mtile, p.mask_rows, q_offset, mrow_sm, hi);
+            ext_rows16(v, xe, c2, key, t, q, slope_sm, pos_sm, mtile, p.mask_rows, q_offset, mrow_sm, hi);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const float4 w = reinterpret_cast<const float4*>(msub_sm + 16 * q)[i];
@@ -483,9 +592,29 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int r = 16 * q + e;
             float pv = EXT ? ex2_approx(v[e]) : ex2_approx(fmaf(v[e], c2, -msub_sm[r]));
             if (!full && !visible(r)) pv = 0.f;
-            *reinterpret_cast<__nv_bfloat16*>(pcol + (size_t)r * 128 + ((chunk16 ^ (r & 7)) << 4)) =
-                __float2bfloat16_rn(pv);
+            if constexpr (!FP8)
+              *reinterpret_cast<__nv_bfloat16*>(pcol + (size_t)r * 128 + ((chunk16 ^ (r & 7)) << 4)) =
+                  __float2bfloat16_rn(pv);
             v[e] = pv;
+          }
+          if constexpr (FP8) {
+            // P as hi + lo e4m3 planes (row r: 128 keys, one 128-byte
+            // swizzled row per plane), two rows per conversion
+            uint8_t* p8 = gbase + PB(sb) + (t & 15);
+            const int ck = t >> 4;
+#pragma unroll
+            for (int e = 0; e < 16; e += 2) {
+              const int r = 16 * q + e;
+              const uint32_t h = e4m3x2_from(v[e], v[e + 1]);
+              const float2 bk = e4m3x2_value(h);
+              const uint32_t l = e4m3x2_from(v[e] - bk.x, v[e + 1] - bk.y);
+              const uint32_t o0 = (uint32_t)r * 128u + ((uint32_t)(ck ^ (r & 7)) << 4);
+              const uint32_t o1 = (uint32_t)(r + 1) * 128u + ((uint32_t)(ck ^ ((r + 1) & 7)) << 4);
+              p8[o0] = (uint8_t)h;
+              p8[o1] = (uint8_t)(h >> 8);
+              p8[(uint32_t)RP * 128u + o0] = (uint8_t)l;
+              p8[(uint32_t)RP * 128u + o1] = (uint8_t)(l >> 8);
+            }
           }
           const float s = warp_reduce16<false>(v, lane);
           if (lane < 16) red_sum[warp * RP + 16 * q + lane] = s;
@@ -527,11 +656,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_after();
       if (t < RP) {
         const float l = l_sm[t];
-        inv_sm[t] = l > 0.f ? 1.f / l : 0.f;
+        inv_sm[t] = l > 0.f ? vs / l : 0.f;
         if (t < R) {
           const int s = t / g, h = kvh * g + (t - s * g);
           p.part_lse[split_lse + ((size_t)b * p.Hq + h) * p.Sq + s] =
-              l > 0.f ? (m_sm[t] + log2f(l)) * LN2 : -INFINITY;
+              l > 0.f ? (m_sm[t] + log2f(l) - (FP8 ? 6.f : 0.f)) * LN2 : -INFINITY;
         }
       }
       named_bar_sync(1, 128);
@@ -574,38 +703,43 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-template <int D, bool EXT, bool PAGED>
+template <int D, bool EXT, bool PAGED, bool FP8>
 int launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
              const DecodeParams& p, cudaStream_t stream) {
-  const Layout L(D, p.RP, p.nbuf, p.mask_rows);
-  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, EXT, PAGED>,
+  const Layout L(D, p.RP, p.nbuf, p.mask_rows, FP8);
+  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, EXT, PAGED, FP8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
   if (e != cudaSuccess) return (int)e;
   dim3 grid((unsigned)p.num_splits, (unsigned)(p.B * p.Hkv));
-  decode_split_kernel<D, EXT, PAGED><<<grid, THREADS, L.total, stream>>>(tq, tk, tv, p);
+  decode_split_kernel<D, EXT, PAGED, FP8><<<grid, THREADS, L.total, stream>>>(tq, tk, tv, p);
   return (int)cudaGetLastError();
 }
 
-template <int D>
+template <int D, bool FP8>
 int launch_d(bool ext, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
              const DecodeParams& p, cudaStream_t stream) {
   const bool paged = p.block_table != nullptr;
-  if (ext) return paged ? launch_t<D, true, true>(tq, tk, tv, p, stream) : launch_t<D, true, false>(tq, tk, tv, p, stream);
-  return paged ? launch_t<D, false, true>(tq, tk, tv, p, stream) : launch_t<D, false, false>(tq, tk, tv, p, stream);
+  if (ext)
+    return paged ? launch_t<D, true, true, FP8>(tq, tk, tv, p, stream)
+                 : launch_t<D, true, false, FP8>(tq, tk, tv, p, stream);
+  return paged ? launch_t<D, false, true, FP8>(tq, tk, tv, p, stream)
+               : launch_t<D, false, false, FP8>(tq, tk, tv, p, stream);
 }
 
 }  // namespace
 
-size_t decode_smem_bytes(int D, int RP, int nbuf, int mask_rows) { return Layout(D, RP, nbuf, mask_rows).total; }
+size_t decode_smem_bytes(int D, int RP, int nbuf, int mask_rows, bool fp8) {
+  return Layout(D, RP, nbuf, mask_rows, fp8).total;
+}
 
 int decode_max_nbuf() { return MAX_NBUF; }
 
-int launch_decode_split(int D, bool ext, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                        const DecodeParams& p, cudaStream_t stream) {
+int launch_decode_split(int D, bool ext, bool fp8, const CUtensorMap& tq, const CUtensorMap& tk,
+                        const CUtensorMap& tv, const DecodeParams& p, cudaStream_t stream) {
   switch (D) {
-    case 128: return launch_d<128>(ext, tq, tk, tv, p, stream);
-    case 256: return launch_d<256>(ext, tq, tk, tv, p, stream);
-    case 512: return launch_d<512>(ext, tq, tk, tv, p, stream);
+    case 128: return fp8 ? launch_d<128, true>(ext, tq, tk, tv, p, stream) : launch_d<128, false>(ext, tq, tk, tv, p, stream);
+    case 256: return fp8 ? launch_d<256, true>(ext, tq, tk, tv, p, stream) : launch_d<256, false>(ext, tq, tk, tv, p, stream);
+    case 512: return fp8 ? launch_d<512, true>(ext, tq, tk, tv, p, stream) : launch_d<512, false>(ext, tq, tk, tv, p, stream);
     default: return (int)cudaErrorInvalidValue;
   }
 }

@@ -53,6 +53,9 @@ struct DecodeParams {
   const int* block_table;  // [B, max_pages] or nullptr: unpaged
   int max_pages, page_size;
   int mask_rows;           // query rows whose mask values are staged in shared memory (0: none)
+  // fp8 e4m3 K/V: one scale per K/V head (K = code * k_scale[kvh], same for V)
+  const float* k_scale;
+  const float* v_scale;
 };
 
 struct MergeParams {
@@ -68,9 +71,9 @@ struct MergeParams {
 int launch_prefill(int D, bool ext, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                    const PrefillParams& p, cudaStream_t stream);
 size_t prefill_smem_bytes(int D);
-int launch_decode_split(int D, bool ext, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                        const DecodeParams& p, cudaStream_t stream);
-size_t decode_smem_bytes(int D, int RP, int nbuf, int mask_rows);
+int launch_decode_split(int D, bool ext, bool fp8, const CUtensorMap& tq, const CUtensorMap& tk,
+                        const CUtensorMap& tv, const DecodeParams& p, cudaStream_t stream);
+size_t decode_smem_bytes(int D, int RP, int nbuf, int mask_rows, bool fp8);
 int launch_merge(const MergeParams& p, cudaStream_t stream);
 int launch_watchdog_selftest(int* status, unsigned long long limit_ns, cudaStream_t stream);
 

@@ -44,6 +44,9 @@ class Workload:
     # additive mask drawn by make_mask(mask_batch, Sq, Skv, seed=0); 0 = none,
     # 1 = one mask shared by the batch, B = one per sequence
     mask_batch: int = 0
+    # K/V element type: "bf16", or "fp8" (e4m3 codes with per-head scales from
+    # make_fp8_kv of the bf16 draw)
+    kv_dtype: str = "bf16"
 
     @property
     def has_options(self) -> bool:
@@ -85,7 +88,7 @@ class Workload:
         """Algorithmic bytes: Q, K, V read once (bf16); O and LSE written once."""
         ob = 2 if self.out_dtype == "bf16" else 4
         q = self.B * self.Sq * self.Hq * self.D * 2
-        kv = 2 * self.B * self.kv_rows_read() * self.Hkv * self.D * 2
+        kv = 2 * self.B * self.kv_rows_read() * self.Hkv * self.D * (1 if self.kv_dtype == "fp8" else 2)
         o = self.B * self.Sq * self.Hq * self.D * ob
         lse = self.B * self.Hq * self.Sq * 4
         return q + kv + o + lse
@@ -132,6 +135,14 @@ WORKLOADS = {
         "spec_verify_decode_d128_mask", "decode", B=4, Hq=32, Hkv=8, Sq=8, Skv=32768, D=128,
         q_offset=32760, causal=True, out_dtype="bf16", num_splits=16, mask_batch=4,
         note="the 8-row verify decode with a per-sequence additive mask over all keys"),
+    "fp8_kv_decode_d512": Workload(
+        "fp8_kv_decode_d512", "decode", B=16, Hq=16, Hkv=1, Sq=1, Skv=16384, D=512,
+        q_offset=16383, causal=True, out_dtype="bf16", num_splits=32, kv_dtype="fp8",
+        note="the D512 split-KV decode over an fp8 e4m3 K/V cache with per-head scales"),
+    "fp8_kv_spec_verify_decode_d128": Workload(
+        "fp8_kv_spec_verify_decode_d128", "decode", B=4, Hq=32, Hkv=8, Sq=8, Skv=32768, D=128,
+        q_offset=32760, causal=True, out_dtype="bf16", num_splits=16, kv_dtype="fp8",
+        note="the 8-row verify decode over an fp8 e4m3 K/V cache"),
     "paged_decode_d512_p64": Workload(
         "paged_decode_d512_p64", "decode", B=16, Hq=16, Hkv=1, Sq=1, Skv=16384, D=512,
         q_offset=16383, causal=True, out_dtype="bf16", num_splits=32, page_size=64,

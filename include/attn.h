@@ -55,7 +55,7 @@ typedef enum {
   ATTN_ERR_TOO_LARGE = -6     /* attn_decode_noalloc: partials exceed the fixed scratch array */
 } attn_status;
 
-typedef enum { ATTN_BF16 = 0, ATTN_F32 = 1 } attn_dtype;
+typedef enum { ATTN_BF16 = 0, ATTN_F32 = 1, ATTN_FP8_E4M3 = 2 } attn_dtype;
 
 /*
  * Prefill: all Sq query rows against all Skv keys in one pass.  The flash
@@ -249,9 +249,20 @@ int attn_merge_ex(const float* partial_out, const float* partial_lse, void* out,
  * status word (see attn_last_status).  Without seq_lens every sequence has Skv
  * keys and q_offset applies.
  *
+ * Quantised K/V (kv_dtype = ATTN_FP8_E4M3): k and v hold one e4m3 code per
+ * element and K = e4m3(code) * k_scale[kvh], V = e4m3(code) * v_scale[kvh]
+ * (the quantised K/V cache of "ggml-org/llama.cpp PR #28507", Setup, and
+ * "Anbeeld/beellama.cpp PR #149", Overview).  The tensor cores read the codes
+ * directly (kind::f8f6f4); Q and P enter as two e4m3 planes each (hi + lo),
+ * which carry a bf16 value's 8 significant bits.  Q is scaled by a power of
+ * two per CTA first, so it needs no range condition.  k_scale and v_scale
+ * must be finite and > 0 (not checked on the device).
+ *
  * Alignment: k, v 16-byte aligned; stride_seq, stride_token and stride_head
- * multiples of 8 elements (16 bytes) and each below 2^37 elements, else
- * ATTN_ERR_ALIGNMENT / ATTN_ERR_INVALID_ARG.  The caller owns every buffer.
+ * multiples of 16 bytes (8 bf16 or 16 fp8 elements) and each below 2^37
+ * elements, else ATTN_ERR_ALIGNMENT / ATTN_ERR_INVALID_ARG; k_scale and
+ * v_scale non-NULL and 4-byte aligned for fp8 (else ATTN_ERR_INVALID_ARG).
+ * The caller owns every buffer.
  */
 typedef struct attn_kv_view {
   const void* k;            /* bf16 */
@@ -264,6 +275,9 @@ typedef struct attn_kv_view {
   int page_size;            /* keys per page */
   int num_pages;            /* physical pages in the cache */
   const int* seq_lens;      /* device [B], or NULL */
+  int kv_dtype;             /* ATTN_BF16 or ATTN_FP8_E4M3 */
+  const float* k_scale;     /* fp8: device [Hkv], K = code * k_scale[kvh] */
+  const float* v_scale;     /* fp8: device [Hkv], V = code * v_scale[kvh] */
 } attn_kv_view;
 
 /*
@@ -278,7 +292,7 @@ int attn_decode_split_kv(const void* q, const attn_kv_view* kv, float* partial_o
                          int B, int Hq, int Hkv, int Sq, int Skv, int D, int q_offset, int causal,
                          float scale, int num_splits, const attn_options* opt, void* stream);
 
-/* Library version, e.g. 0x000200 for 0.2.0. */
+/* Library version, e.g. 0x000300 for 0.3.0. */
 int attn_version(void);
 
 #ifdef __cplusplus

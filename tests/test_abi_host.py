@@ -22,7 +22,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert ga.version() == 0x000200
+    assert ga.version() == 0x000300
     assert ga.status_string(ga.ATTN_OK) == "ok"
     assert ga.status_string(ga.ATTN_ERR_TIMEOUT) == "pipeline wait timed out"
     assert ga.status_string(12345) == "unknown status"
@@ -188,7 +188,7 @@ def _kv_decode(lib, view=None, **kw):
     if view is None:
         view = {}
     vw = dict(k=0x40000, v=0x50000, stride_seq=1024 * 512, stride_token=512, stride_head=512, block_table=None,
-              max_pages=0, page_size=0, num_pages=0, seq_lens=None)
+              max_pages=0, page_size=0, num_pages=0, seq_lens=None, kv_dtype=0, k_scale=None, v_scale=None)
     vw.update(view)
     v = ga.AttnKVView(**vw)
     return lib.attn_decode_split_kv(a["q"], ctypes.byref(v), a["po"], a["pl"], a["B"], a["Hq"], a["Hkv"], a["Sq"],
@@ -210,6 +210,11 @@ def _kv_decode(lib, view=None, **kw):
     (dict(block_table=0x70000, max_pages=8, page_size=128, num_pages=0), dict(Skv=1024), ga.ATTN_ERR_INVALID_ARG),
     (dict(block_table=0x70002, max_pages=8, page_size=128, num_pages=64), dict(Skv=1024), ga.ATTN_ERR_ALIGNMENT),
     ({}, dict(D=64), ga.ATTN_ERR_UNSUPPORTED),
+    (dict(kv_dtype=5), {}, ga.ATTN_ERR_INVALID_ARG),
+    (dict(kv_dtype=2), {}, ga.ATTN_ERR_INVALID_ARG),                           # fp8 without scales
+    (dict(kv_dtype=2, k_scale=0x90000, v_scale=0x90002), {}, ga.ATTN_ERR_INVALID_ARG),
+    (dict(kv_dtype=2, k_scale=0x90000, v_scale=0x90010, stride_head=520,
+          stride_token=520, stride_seq=520 * 1024), {}, ga.ATTN_ERR_ALIGNMENT),  # 520 bytes: not 16-byte multiples
 ])
 def test_decode_split_kv_rejects(lib, view, kw, status):
     assert _kv_decode(lib, view, **kw) == status
@@ -226,4 +231,4 @@ def test_kv_view_struct_matches_header():
     body = re.search(r"typedef struct attn_kv_view \{(.*?)\} attn_kv_view;", text, re.S).group(1)
     fields = [ln.split(";")[0].split()[-1].lstrip("*") for ln in body.strip().splitlines() if ";" in ln]
     assert fields == [f[0] for f in ga.AttnKVView._fields_]
-    assert ctypes.sizeof(ga.AttnKVView) == 72
+    assert ctypes.sizeof(ga.AttnKVView) == 96
