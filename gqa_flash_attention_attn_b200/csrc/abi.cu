@@ -1,6 +1,7 @@
 // C ABI of the library: argument checks, TMA descriptors, launches, status.
 // Every check that can fail runs on the host before any CUDA call, so bad
 // arguments never reach a kernel.
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -310,6 +311,23 @@ int attn_decode_split_kv(const void* q, const attn_kv_view* kv, float* partial_o
          gqa::decode_smem_bytes(D, p.RP, nbuf + 1, p.mask_rows, fp8) <= kTwoCtaSmemLimit)
     ++nbuf;
   p.nbuf = nbuf;
+  // Consecutive splits per CTA: enough that the CTAs fit the resident slots
+  // (two per SM when the shared memory allows) in one wave, at most 8, for
+  // splits of at most 8 tiles.
+  {
+    const int nsm = sm_count();
+    if (nsm <= 0) return cuda_fail();
+    const long long slots =
+        (long long)nsm * (gqa::decode_smem_bytes(D, p.RP, nbuf, p.mask_rows, fp8) <= kTwoCtaSmemLimit ? 2 : 1);
+    const long long units = (long long)num_splits * B * Hkv;
+    long long grp = (units + slots - 1) / slots;
+    // long splits already amortise a CTA's start and end: group short ones only
+    if ((p.chunk + 127) / 128 > 8) grp = 1;
+    grp = std::min<long long>(std::min<long long>(grp, gqa::decode_max_group()), num_splits);
+    p.group = (int)std::max<long long>(grp, 1);
+    // two O^T buffers when split boundaries exist and two CTAs' TMEM still fits
+    p.obuf = (p.group > 1 && RP * (2 + 2 * (D / 128)) <= 256) ? 2 : 1;
+  }
   p.c2 = scale * kLog2e;
   p.timeout_ns = kWaitLimitNs;
   p.ext = ext;

@@ -37,13 +37,47 @@ constexpr int THREADS = 192;                   // warps 0-3 softmax, 4 producer,
 constexpr int WARP_PRODUCER = 4;
 constexpr int WARP_MMA = 5;
 constexpr int MAX_NBUF = 6;
+constexpr int MAX_GROUP = 8;                   // consecutive splits per CTA
+
+// One split of a CTA's group: its tiles are first .. first+nt-1 of the CTA's
+// tile stream; keys from kbase on a 128-key grid, the split ending at hi.
+struct SegInfo {
+  int first, nt, kbase, hi;
+  int ob, pad0, pad1, pad2;   // ob: the O^T buffer the split accumulates in
+};
+
+// Walks a CTA's tile stream in order: the split of tile j in registers,
+// reading the shared table only when a split boundary is crossed.
+struct SegCursor {
+  const SegInfo* tab;
+  int n, i, next_first;
+  int first, nt, kbase, hi, ob;   // the current split's entry
+  __device__ __forceinline__ void load(int k) {
+    first = tab[k].first;
+    nt = tab[k].nt;
+    kbase = tab[k].kbase;
+    hi = tab[k].hi;
+    ob = tab[k].ob;
+    next_first = k + 1 < n ? tab[k + 1].first : 0x7fffffff;
+  }
+  __device__ __forceinline__ SegCursor(const SegInfo* t, int nseg) : tab(t), n(nseg), i(0) { load(0); }
+  // position on tile j (non-decreasing over calls)
+  __device__ __forceinline__ void to(int j) {
+    while (j >= next_first) load(++i);
+  }
+  // first key of tile j (its split's tiles reversed under ALiBi)
+  __device__ __forceinline__ int key0(int j, bool rev) const {
+    const int jj = j - first;
+    return kbase + (rev ? nt - 1 - jj : jj) * 128;
+  }
+};
 // A staged mask row: the tile's 128 keys in an 8-key-aligned window of 136
 // (17 chunks of 16 bytes), so every cp.async source is 16-byte aligned.
 constexpr int MROW_KEYS = 136;
 constexpr uint32_t MROW_BYTES = MROW_KEYS * 2u;
 
 struct Layout {
-  uint32_t off_q, off_q8, off_p, off_ring, off_red, off_row, off_mask, off_bar, off_misc, total;
+  uint32_t off_q, off_q8, off_p, off_ring, off_red, off_row, off_mask, off_bar, off_misc, off_seg, total;
   // mrows: query rows s whose additive-mask values are staged per tile;
   // fp8: K/V slots of 128 e4m3 columns (16 KB) and Q as two e4m3 planes
   __host__ __device__ Layout(int D, int RP, int nbuf, int mrows, bool fp8) {
@@ -59,7 +93,8 @@ struct Layout {
     off_bar = off_mask + (uint32_t)mrows * 2u * MROW_BYTES;  // staged mask [2][mrows][136 keys] bf16
     off_bar = (off_bar + 7u) & ~7u;
     off_misc = off_bar + (uint32_t)(1 + 2 * nbuf + 8) * 8u;
-    total = off_misc + 16u + 1024u;
+    off_seg = off_misc + 16u;                  // SegInfo[MAX_GROUP]
+    total = off_seg + (uint32_t)MAX_GROUP * 32u + 1024u;
   }
 };
 
@@ -142,7 +177,7 @@ __device__ __forceinline__ void ext_rows16(float (&v)[16], const LogitExt& x, fl
 }
 
 template <int D, bool EXT, bool PAGED, bool FP8>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(THREADS, 2)
     decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
   constexpr int KC = D / 128;  // 128-column slots per K (or V) tile
@@ -184,7 +219,6 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int BAR_Q8 = BAR_S0 + 7;         // fp8: Q planes written
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int split = blockIdx.x;
   const int b = blockIdx.y / p.Hkv, kvh = blockIdx.y % p.Hkv;
   // this sequence's keys and the position of its first query row
   int Skv = p.Skv, q_offset = p.q_offset;
@@ -192,40 +226,58 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (p.seq_lens != nullptr) {
     const int len = __ldg(p.seq_lens + b);
     Skv = min(max(len, 0), p.Skv);
-    if (Skv != len && split == 0 && kvh == 0 && threadIdx.x == 0) atomicCAS(p.status, kStatusOk, kStatusInvalidArg);
+    if (Skv != len && blockIdx.x == 0 && kvh == 0 && threadIdx.x == 0)
+      atomicCAS(p.status, kStatusOk, kStatusInvalidArg);
     q_offset = Skv - p.Sq;
     chunk = (Skv + p.num_splits - 1) / p.num_splits;
   }
   if (PAGED) chunk = (chunk + BN - 1) / BN * BN;  // no tile crosses a page
-  const long long lo_ll = (long long)split * chunk;
-  const int lo = (int)min(lo_ll, (long long)Skv);
-  const int hi = (int)min(lo_ll + chunk, (long long)Skv);
-  const int eff_hi = p.causal ? (int)min((long long)hi, (long long)q_offset + p.Sq) : hi;
-  // a sliding window hides every key at or before q_offset - window from all rows
-  const int eff_lo = (EXT && p.ext.window > 0) ? max(lo, q_offset - p.ext.window + 1) : lo;
-  const int kbase = lo + ((eff_lo - lo) / BN) * BN;   // first tile, on the split's tile grid
-  const int n_tiles = eff_hi > eff_lo ? (eff_hi - kbase + BN - 1) / BN : 0;
-  // With ALiBi the bias grows toward each query's own position: visiting the
+  // With ALiBi the bias grows toward each query's own position: visiting a
   // split's tiles newest first sets the running maximum on the first tile and
   // spares the O rescales (the tile order does not change the result).
   const bool rev = EXT && p.ext.alibi != 0;
-  auto tile_key0 = [&](int jj) { return kbase + (rev ? n_tiles - 1 - jj : jj) * BN; };
-  const size_t split_out = (size_t)split * p.B * p.Sq * p.Hq * D;
-  const size_t split_lse = (size_t)split * p.B * p.Hq * p.Sq;
-
-  if (n_tiles == 0) {
-    // No visible key in this split: publish (-inf, 0) for every row.
-    for (int i = threadIdx.x; i < R * D; i += THREADS) {
-      const int r = i / D, d = i - r * D;
-      const int s = r / g, h = kvh * g + (r - s * g);
-      p.part_out[split_out + (((size_t)b * p.Sq + s) * p.Hq + h) * D + d] = 0.f;
+  // This CTA's splits sg0 .. sg0+nseg-1 of (b, kvh) run as one tile stream
+  // (same Q, one pipeline); each split's partial is published at its end.
+  const int sg0 = blockIdx.x * p.group;
+  const int nseg = min(p.group, p.num_splits - sg0);
+  SegInfo* seg_sm = reinterpret_cast<SegInfo*>(gbase + L.off_seg);
+  int T = 0;  // tiles of the whole stream
+  int filled = 0;  // non-empty splits so far: consecutive ones alternate O^T buffers
+  for (int i = 0; i < nseg; ++i) {
+    const long long lo_ll = (long long)(sg0 + i) * chunk;
+    const int lo = (int)min(lo_ll, (long long)Skv);
+    const int hi = (int)min(lo_ll + chunk, (long long)Skv);
+    const int eff_hi = p.causal ? (int)min((long long)hi, (long long)q_offset + p.Sq) : hi;
+    // a sliding window hides every key at or before q_offset - window from all rows
+    const int eff_lo = (EXT && p.ext.window > 0) ? max(lo, q_offset - p.ext.window + 1) : lo;
+    const int kb = lo + ((eff_lo - lo) / BN) * BN;   // first tile, on the split's tile grid
+    const int nt = eff_hi > eff_lo ? (eff_hi - kb + BN - 1) / BN : 0;
+    if (threadIdx.x == 0) seg_sm[i] = SegInfo{T, nt, kb, hi, p.obuf == 2 ? (filled & 1) : 0, 0, 0, 0};
+    filled += nt > 0 ? 1 : 0;
+    if (nt == 0) {
+      // No visible key in this split: publish (-inf, 0) for every row.
+      const size_t so = (size_t)(sg0 + i) * p.B * p.Sq * p.Hq * D;
+      const size_t sl = (size_t)(sg0 + i) * p.B * p.Hq * p.Sq;
+      for (int x = threadIdx.x; x < R * D; x += THREADS) {
+        const int r = x / D, d = x - r * D;
+        const int s = r / g, h = kvh * g + (r - s * g);
+        p.part_out[so + (((size_t)b * p.Sq + s) * p.Hq + h) * D + d] = 0.f;
+      }
+      for (int r = threadIdx.x; r < R; r += THREADS) {
+        const int s = r / g, h = kvh * g + (r - s * g);
+        p.part_lse[sl + ((size_t)b * p.Hq + h) * p.Sq + s] = -INFINITY;
+      }
     }
-    for (int r = threadIdx.x; r < R; r += THREADS) {
-      const int s = r / g, h = kvh * g + (r - s * g);
-      p.part_lse[split_lse + ((size_t)b * p.Hq + h) * p.Sq + s] = -INFINITY;
-    }
-    return;
+    T += nt;
   }
+  if (T == 0) return;
+  // split of stream tile j (empty splits share their successor's first tile);
+  // for the rare boundary work, the per-tile paths use SegCursor
+  auto seg_of = [&](int j) -> int {
+    int i = 0;
+    while (i + 1 < nseg && j >= seg_sm[i + 1].first) ++i;
+    return i;
+  };
 
   // Zero the padding rows of Q (rows R..RP-1 of every 64-column box).
   for (int i = threadIdx.x; i < (D / 64) * (RP - R) * 32; i += THREADS) {
@@ -266,7 +318,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     fence_mbar_init();
   }
   uint32_t tmem_cols = 32;
-  while (tmem_cols < (uint32_t)(RP * (2 + KC))) tmem_cols <<= 1;
+  while (tmem_cols < (uint32_t)(RP * (2 + p.obuf * KC))) tmem_cols <<= 1;
   if (warp == WARP_MMA) {
     tmem_alloc(smem_u32(tmem_slot), tmem_cols);
     tmem_relinquish();
@@ -277,7 +329,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   auto TS = [&](int buf) { return (uint32_t)(RP * buf); };            // S^T buffers
-  auto TO = [&](int c) { return (uint32_t)(RP * (2 + c)); };          // O^T chunk c
+  auto TO = [&](int c, int ob) { return (uint32_t)(RP * (2 + ob * KC + c)); };  // O^T chunk c, buffer ob
   auto PB = [&](int buf) { return L.off_p + (uint32_t)buf * 2u * RP * 128u; };  // P buffers
   const Watchdog wd{abort_flag, p.status, p.timeout_ns};
   int issued = 0;
@@ -293,7 +345,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       // ring order: K_0, then (K_{j+1}, V_j) for j = 0..n-1; KC slots each
       bool ok = true;
       int n = 0;
-      auto issue = [&](const CUtensorMap* tm, int j) {
+      SegCursor ck(seg_sm, nseg), cv(seg_sm, nseg);   // the K and the V stream
+      auto issue = [&](const CUtensorMap* tm, int j, SegCursor& cu) {
+        cu.to(j);
+        const int key0 = cu.key0(j, rev);
         for (int c = 0; c < KC; ++c, ++n) {
           const int slot = n % nbuf, use = n / nbuf;
           if (use > 0 && !mbar_wait(bar(bar_empty(slot)), (uint32_t)(use - 1) & 1u, wd)) {
@@ -302,7 +357,6 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
           mbar_arrive_expect_tx(bar(bar_full(slot)), SLOTB);
           const uint32_t dst = base + L.off_ring + (uint32_t)slot * SLOTB;
-          const int key0 = tile_key0(j);
           if constexpr (!PAGED) {
             if (FP8) {
               tma_load_4d(dst, tm, bar(bar_full(slot)), c * 128, kvh, key0, b);   // 128 e4m3 columns
@@ -333,10 +387,10 @@ __global__ void __launch_bounds__(THREADS, 1)
           issued = n + 1;
         }
       };
-      issue(&tm_k, 0);
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        if (j + 1 < n_tiles) issue(&tm_k, j + 1);
-        if (ok) issue(&tm_v, j);
+      issue(&tm_k, 0, ck);
+      for (int j = 0; ok && j < T; ++j) {
+        if (j + 1 < T) issue(&tm_k, j + 1, ck);
+        if (ok) issue(&tm_v, j, cv);
       }
     }
   } else if (warp == WARP_MMA) {
@@ -382,16 +436,20 @@ __global__ void __launch_bounds__(THREADS, 1)
         mma_commit(bar(BAR_S0 + (j & 1)));
       };
       if (ok) mma_s(0);
-      for (int j = 0; ok && j < n_tiles; ++j) {
+      SegCursor cpv(seg_sm, nseg);
+      for (int j = 0; ok && j < T; ++j) {
         // S buffer (j+1)%2 was last read by softmax j-1, whose P the PV of
         // tile j-1 (issued before this point) already waited for.
-        if (j + 1 < n_tiles) {
+        if (j + 1 < T) {
           mma_s(j + 1);
           if (!ok) break;
         }
         if (!mbar_wait(bar(BAR_P0 + (j & 1)), (uint32_t)(j >> 1) & 1u, wd)) { ok = false; break; }
         tc_fence_after();
-        // O^T(c) += V_j^T(c) P_j^T
+        // O^T(c) += V_j^T(c) P_j^T; a split's first tile starts O afresh (the
+        // softmax read the previous split's O before it handed over P_j)
+        cpv.to(j);
+        const uint32_t acc0 = (j == cpv.first) ? 0u : 1u;
         for (int c = 0; ok && c < KC; ++c, ++n) {
           const int slot = n % nbuf;
           if (!mbar_wait(bar(bar_full(slot)), (uint32_t)(n / nbuf) & 1u, wd)) { ok = false; break; }
@@ -406,8 +464,8 @@ __global__ void __launch_bounds__(THREADS, 1)
               for (int kk = 0; kk < 4; ++kk) {
                 const uint32_t a = vb + (uint32_t)kk * 4096u;
                 const uint32_t pb = base + PB(j & 1) + (uint32_t)pl * RP * 128u + (uint32_t)kk * 32u;
-                mma_ss_f8(tmem + TO(c), sdesc_sw128(a, BOX_BYTES, 1024), sdesc_sw128(pb, 16, 1024), idesc_o,
-                          (j > 0 || pl > 0 || kk > 0) ? 1u : 0u);
+                mma_ss_f8(tmem + TO(c, cpv.ob), sdesc_sw128(a, BOX_BYTES, 1024), sdesc_sw128(pb, 16, 1024), idesc_o,
+                          (acc0 || pl > 0 || kk > 0) ? 1u : 0u);
               }
             }
           } else {
@@ -415,8 +473,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int kk = 0; kk < 8; ++kk) {
               const uint32_t a = vb + (uint32_t)kk * 2048u;
               const uint32_t pb = base + PB(j & 1) + (uint32_t)(kk >> 2) * RP * 128u + (uint32_t)(kk & 3) * 32u;
-              mma_ss(tmem + TO(c), sdesc_sw128(a, BOX_BYTES, 1024), sdesc_sw128(pb, 16, 1024), idesc_o,
-                     (j > 0 || kk > 0) ? 1u : 0u);
+              mma_ss(tmem + TO(c, cpv.ob), sdesc_sw128(a, BOX_BYTES, 1024), sdesc_sw128(pb, 16, 1024), idesc_o,
+                     (acc0 || kk > 0) ? 1u : 0u);
             }
           }
           mma_commit(bar(bar_empty(slot)));
@@ -493,8 +551,82 @@ __global__ void __launch_bounds__(THREADS, 1)
         vs = __ldg(p.v_scale + kvh);
       }
     }
-    for (int j = 0; ok && j < n_tiles; ++j) {
+    // Publishing split si of the group: stats() turns its (max, sum) into the
+    // LSE and 1/l (rows t < RP, from shared memory: needs no wait), write_o()
+    // stores O^T / l from its TMEM buffer (after its last P.V completed).
+    auto stats = [&](int si) {
+      if (t < RP) {
+        const float l = l_sm[t];
+        inv_sm[t] = l > 0.f ? vs / l : 0.f;
+        if (t < R) {
+          const int s = t / g, h = kvh * g + (t - s * g);
+          const size_t sl = (size_t)(sg0 + si) * p.B * p.Hq * p.Sq;
+          p.part_lse[sl + ((size_t)b * p.Hq + h) * p.Sq + s] =
+              l > 0.f ? (m_sm[t] + log2f(l) - (FP8 ? 6.f : 0.f)) * LN2 : -INFINITY;
+        }
+      }
+    };
+    auto write_o = [&](int si) {
+      named_bar_sync(1, 128);   // inv_sm of every row
+      const size_t so = (size_t)(sg0 + si) * p.B * p.Sq * p.Hq * D;
+      const int ob = seg_sm[si].ob;
+      for (int c = 0; c < KC; ++c) {
+        for (int q = 0; q < RP / 16; ++q) {
+          float v[16];
+          tmem_ld16(tmem + lane_off + TO(c, ob) + 16 * q, v);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int r = 16 * q + e;
+            if (r < R) {
+              const int s = r / g, h = kvh * g + (r - s * g);
+              p.part_out[so + (((size_t)b * p.Sq + s) * p.Hq + h) * D + c * 128 + t] = v[e] * inv_sm[r];
+            }
+          }
+        }
+      }
+      named_bar_sync(1, 128);   // every row's inv_sm read before stats() rewrites it
+    };
+    // wait (jointly) for the P.V of stream tile j
+    auto pv_done = [&](int j) -> bool {
+      const bool got = mbar_wait(bar(BAR_PV0 + (j & 1)), (uint32_t)(j >> 1) & 1u, wd);
+      if (named_bar_or(1, 128, !got)) return false;
+      tc_fence_after();
+      return true;
+    };
+    // With two O^T buffers a finished split's O is written out one tile
+    // later (after the next hand-off of P, off the critical path), when the
+    // P-buffer wait has shown its last P.V complete: pend / pend_last.
+    int pend = -1, pend_last = -1;
+    SegCursor cs(seg_sm, nseg), cm(seg_sm, nseg);   // this tile; the mask stage's tile
+    for (int j = 0; ok && j < T; ++j) {
       const int sb = j & 1;
+      cs.to(j);
+      const int si = cs.i;
+      const int jl = j - cs.first;   // tile within its split
+      const int hi = cs.hi;           // the split's end key
+      if (jl == 0 && j > 0) {
+        // a new split: publish the previous one, then restart the running
+        // (max, sum).  With one O^T buffer its O is read now, before this
+        // split's first P.V (which waits for P_j) overwrites it.
+        if (pend >= 0) {   // the split before had a single tile: flush it first
+          if (!pv_done(pend_last)) { ok = false; break; }
+          write_o(pend);
+          pend = -1;
+        }
+        const int prev = seg_of(j - 1);
+        stats(prev);
+        if (p.obuf == 2) {
+          pend = prev;
+          pend_last = j - 1;
+        } else {
+          if (!pv_done(j - 1)) { ok = false; break; }
+          write_o(prev);
+        }
+        if (t < RP) {
+          m_sm[t] = -INFINITY;
+          l_sm[t] = 0.f;
+        }
+      }
       // every give-up is decided jointly (barrier + OR) so no thread is left
       // waiting at a named barrier or inside a warp-collective TMEM access
       if (EXT && p.mask_rows > 0) {
@@ -502,12 +634,14 @@ __global__ void __launch_bounds__(THREADS, 1)
         // copies stay in flight across this tile's barriers, and tile j's are
         // complete (and, after the barrier below, visible) before use
         auto stage = [&](int jj) {
-          const int tile_al = tile_key0(jj) & ~7;
+          cm.to(jj);
+          const int tile_al = cm.key0(jj, rev) & ~7;
+          const int shi = cm.hi;
           const uint32_t dst0 = mstage_u32 + (uint32_t)(jj & 1) * p.mask_rows * MROW_BYTES;
           for (int c = t; c < p.mask_rows * 17; c += 128) {
             const int row = c / 17, k8 = (c - row * 17) * 8;
             const int key8 = tile_al + k8;
-            const int n = min(max(hi - key8, 0), 8);   // keys inside the split (hi <= Skv)
+            const int n = min(max(shi - key8, 0), 8);   // keys inside the split (end <= Skv)
             const uint16_t* src = n > 0 ? p.ext.mask + (size_t)b * p.ext.mask_sb + (size_t)row * p.ext.mask_sr + key8
                                         : p.ext.mask;
             cp_async16(dst0 + (uint32_t)row * MROW_BYTES + (uint32_t)k8 * 2u, src, (uint32_t)n * 2u);
@@ -515,7 +649,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           cp_async_commit();
         };
         if (j == 0) stage(0);
-        if (j + 1 < n_tiles) {
+        if (j + 1 < T) {
           stage(j + 1);
           cp_async_wait<1>();
         } else {
@@ -525,7 +659,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const bool got_s = mbar_wait(bar(BAR_S0 + sb), (uint32_t)(j >> 1) & 1u, wd);
       if (named_bar_or(1, 128, !got_s)) { ok = false; break; }
       tc_fence_after();
-      const int tile0 = tile_key0(j);
+      const int tile0 = cs.key0(j, rev);
       const int key = tile0 + t;
       // this tile's staged mask at this thread's key
       const uint16_t* mtile = mstage + (size_t)(j & 1) * p.mask_rows * MROW_KEYS + (tile0 & 7) + t;
@@ -570,7 +704,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const bool got_pb = (j < 2) || mbar_wait(bar(BAR_PV0 + sb), (uint32_t)((j - 2) >> 1) & 1u, wd);
       if (named_bar_or(1, 128, !got_pb)) { ok = false; break; }
       tc_fence_after();
-      const bool rescale = (j > 0) && (*resc_flag != 0);
+      const bool rescale = (jl > 0) && (*resc_flag != 0);
       // pass 2: exponentials, P (bf16) into the swizzled B-operand buffer
       {
         const int half = t >> 6, tt = t & 63;
@@ -628,7 +762,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int c = 0; c < KC; ++c) {
           for (int q = 0; q < RP / 16; ++q) {
             float v[16];
-            const uint32_t addr = tmem + lane_off + TO(c) + 16 * q;
+            const uint32_t addr = tmem + lane_off + TO(c, cs.ob) + 16 * q;
             tmem_ld16(addr, v);
             uint32_t u[16];
 #pragma unroll
@@ -646,38 +780,25 @@ __global__ void __launch_bounds__(THREADS, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(BAR_P0 + sb));
+      // the pending split's last P.V is P.V(j-1) or earlier, and the wait for
+      // P buffer sb above (tile j >= 2) covered P.V(j-2); flush it once that
+      // covers it
+      if (pend >= 0 && j >= 2 && pend_last <= j - 2) {
+        write_o(pend);
+        pend = -1;
+      }
     }
     // no mask copy may outlive the loop (it also ends early on a give-up)
     if (EXT && p.mask_rows > 0) cp_async_wait<0>();
-    // ---- epilogue: normalised partial O and the split's LSE ----
-    const int last = n_tiles - 1;
-    const bool got_o = ok && mbar_wait(bar(BAR_PV0 + (last & 1)), (uint32_t)(last >> 1) & 1u, wd);
-    if (ok && !named_bar_or(1, 128, !got_o)) {
-      tc_fence_after();
-      if (t < RP) {
-        const float l = l_sm[t];
-        inv_sm[t] = l > 0.f ? vs / l : 0.f;
-        if (t < R) {
-          const int s = t / g, h = kvh * g + (t - s * g);
-          p.part_lse[split_lse + ((size_t)b * p.Hq + h) * p.Sq + s] =
-              l > 0.f ? (m_sm[t] + log2f(l) - (FP8 ? 6.f : 0.f)) * LN2 : -INFINITY;
-        }
-      }
-      named_bar_sync(1, 128);
-      for (int c = 0; c < KC; ++c) {
-        for (int q = 0; q < RP / 16; ++q) {
-          float v[16];
-          tmem_ld16(tmem + lane_off + TO(c) + 16 * q, v);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int r = 16 * q + e;
-            if (r < R) {
-              const int s = r / g, h = kvh * g + (r - s * g);
-              p.part_out[split_out + (((size_t)b * p.Sq + s) * p.Hq + h) * D + c * 128 + t] = v[e] * inv_sm[r];
-            }
-          }
-        }
-      }
+    // ---- the pending split and the last one ----
+    if (ok && pend >= 0) {
+      if (pv_done(pend_last)) write_o(pend);
+      else ok = false;
+    }
+    if (ok) {
+      stats(seg_of(T - 1));
+      if (pv_done(T - 1)) write_o(seg_of(T - 1));
+      else ok = false;
     }
     tc_fence_before();
   }
@@ -710,7 +831,7 @@ int launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv
   cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, EXT, PAGED, FP8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
   if (e != cudaSuccess) return (int)e;
-  dim3 grid((unsigned)p.num_splits, (unsigned)(p.B * p.Hkv));
+  dim3 grid((unsigned)((p.num_splits + p.group - 1) / p.group), (unsigned)(p.B * p.Hkv));
   decode_split_kernel<D, EXT, PAGED, FP8><<<grid, THREADS, L.total, stream>>>(tq, tk, tv, p);
   return (int)cudaGetLastError();
 }
@@ -733,6 +854,8 @@ size_t decode_smem_bytes(int D, int RP, int nbuf, int mask_rows, bool fp8) {
 }
 
 int decode_max_nbuf() { return MAX_NBUF; }
+
+int decode_max_group() { return MAX_GROUP; }
 
 int launch_decode_split(int D, bool ext, bool fp8, const CUtensorMap& tq, const CUtensorMap& tk,
                         const CUtensorMap& tv, const DecodeParams& p, cudaStream_t stream) {

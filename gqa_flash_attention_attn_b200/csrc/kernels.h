@@ -44,6 +44,8 @@ struct DecodeParams {
   int B, Hq, Hkv, Sq, Skv, q_offset, causal;
   int g, R, RP;       // rows per K/V head = g*Sq, padded to a multiple of 16
   int num_splits, chunk;  // keys per split
+  int group;              // consecutive splits per CTA (1..8), one tile stream
+  int obuf;               // O^T buffers in TMEM (2: a split's O is written out one tile late)
   int nbuf;           // K/V ring slots (32 KB each)
   float c2;
   unsigned long long timeout_ns;
@@ -74,6 +76,7 @@ size_t prefill_smem_bytes(int D);
 int launch_decode_split(int D, bool ext, bool fp8, const CUtensorMap& tq, const CUtensorMap& tk,
                         const CUtensorMap& tv, const DecodeParams& p, cudaStream_t stream);
 size_t decode_smem_bytes(int D, int RP, int nbuf, int mask_rows, bool fp8);
+int decode_max_group();
 int launch_merge(const MergeParams& p, cudaStream_t stream);
 int launch_watchdog_selftest(int* status, unsigned long long limit_ns, cudaStream_t stream);
 

@@ -97,3 +97,30 @@ def test_full_size_workload_sampled_rows(name):
     assert_o_close(got_o, want_o, name)
     assert_lse_close(got_lse, want_lse, name)
     assert torch.isfinite(out).all() and torch.isfinite(lse).all()
+
+
+# (B, Hq, Hkv, Sq, Skv, D, q_offset, causal, num_splits): enough CTAs that each
+# takes a group of consecutive splits (3, 4 and 8 per CTA on a 148-SM part)
+GROUPED = [
+    (100, 8, 1, 1, 300, 128, 299, True, 7),      # groups of 3, the last of 1
+    (64, 16, 2, 2, 513, 256, 100, True, 9),      # causal: splits past key 101 empty inside groups
+    (128, 8, 4, 1, 2048, 128, 2047, True, 8),    # groups of 8
+    (40, 16, 1, 1, 1000, 512, 0, False, 30),     # non-causal D512, groups of 3
+]
+
+
+@pytest.mark.parametrize("case", GROUPED, ids=[f"B{c[0]}H{c[1]}/{c[2]}x{c[4]}D{c[5]}S{c[8]}" for c in GROUPED])
+def test_grouped_splits_publish_every_partial(case):
+    B, Hq, Hkv, Sq, Skv, D, q_offset, causal, S = case
+    q, k, v = make_qkv(B, Hq, Hkv, Sq, Skv, D, seed=81)
+    scale = _scale(D)
+    po, pl = ga.decode_split(q.cuda(), k.cuda(), v.cuda(), S, causal=causal, q_offset=q_offset, scale=scale)
+    out, lse = ga.merge(po, pl, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert ga.last_status() == ga.ATTN_OK
+    want_po, want_pl = oracle.split(q, k, v, S, scale=scale, causal=causal, q_offset=q_offset)
+    assert_lse_close(pl, want_pl, f"partial lse {case}")
+    assert_o_close(po, want_po, f"partial out {case}")
+    want_o, want_lse = oracle.merge(want_po, want_pl)
+    assert_o_close(out, want_o, f"merged {case}")
+    assert_lse_close(lse, want_lse, f"merged {case}")

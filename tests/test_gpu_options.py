@@ -310,3 +310,25 @@ def test_decode_mask_unstaged_paths(shape):
                                          alibi_max_bias=1.0, mask=mask)
     assert_o_close(out, want_o, str(shape))
     assert_lse_close(lse, want_l, str(shape))
+
+
+def test_decode_terms_with_grouped_splits():
+    """Short splits and many CTAs (several consecutive splits per CTA), with a
+    staged mask, ALiBi (tiles newest first) and a window crossing the splits."""
+    from gqa_flash_attention_attn_b200.inputs import make_mask
+    B, Hq, Hkv, Sq, Skv, D, S = 64, 16, 2, 4, 512, 128, 8
+    q, k, v = make_qkv(B, Hq, Hkv, Sq, Skv, D, seed=91)
+    mask = make_mask(B, Sq, Skv, seed=92)
+    terms = dict(alibi_max_bias=4.0, window=300, softcap=25.0)
+    po, pl = ga.decode_split(q.cuda(), k.cuda(), v.cuda(), S, q_offset=Skv - Sq, mask=mask.cuda(), **terms)
+    out, lse = ga.merge(po, pl, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert ga.last_status() == ga.ATTN_OK
+    want_po, want_pl = oracle.split_ex(q, k, v, S, scale=_scale(D), causal=True, q_offset=Skv - Sq, mask=mask,
+                                       **terms)
+    assert_lse_close(pl, want_pl, "grouped partial lse")
+    assert_o_close(po, want_po, "grouped partial out")
+    want_o, want_l = oracle.attention_ex(q, k, v, scale=_scale(D), causal=True, q_offset=Skv - Sq, mask=mask,
+                                         **terms)
+    assert_o_close(out, want_o, "grouped merged")
+    assert_lse_close(lse, want_l, "grouped merged")
