@@ -213,7 +213,19 @@ int attn_prefill_ex(const void* q, const void* k, const void* v, void* out, floa
   if (!make_map(&tq, q, D, Hq, Sq, B, 64, 1, 128, 1)) return cuda_fail();
   if (!make_map(&tk, k, D, Hkv, Skv, B, 64, 1, 128, 1)) return cuda_fail();
   if (!make_map(&tv, v, D, Hkv, Skv, B, 64, 1, 128, 1)) return cuda_fail();
-  return gqa::launch_prefill(D, ext_on, tq, tk, tv, p, static_cast<cudaStream_t>(stream)) == 0 ? ATTN_OK
+  // the additive mask staged by TMA: 16-byte aligned rows, and every head
+  // slot of a CTA visits every tile (one slot, or an even group size)
+  CUtensorMap tm;
+  std::memset(&tm, 0, sizeof(tm));
+  if (ext.mask != nullptr && aligned(ext.mask, 16) && ext.mask_sr % 8 == 0 && ext.mask_sb % 8 == 0 &&
+      ext.mask_sr > 0 && (gqa::prefill_slots(D) == 1 || g % 2 == 0)) {
+    const uint64_t bm = ext.mask_sb != 0 ? (uint64_t)B : 1u;
+    const uint64_t s2 = ext.mask_sb != 0 ? (uint64_t)ext.mask_sb : (uint64_t)Sq * ext.mask_sr;
+    if (!make_map_strided(&tm, ext.mask, Skv, Sq, bm, 1, (uint64_t)ext.mask_sr, s2, s2 * bm, 64, 128, 1, 1))
+      return cuda_fail();
+    p.mask_tma = 1;
+  }
+  return gqa::launch_prefill(D, ext_on, tq, tk, tv, tm, p, static_cast<cudaStream_t>(stream)) == 0 ? ATTN_OK
                                                                                           : ATTN_ERR_CUDA;
 }
 

@@ -601,7 +601,6 @@ __global__ void __launch_bounds__(THREADS, 2)
     for (int j = 0; ok && j < T; ++j) {
       const int sb = j & 1;
       cs.to(j);
-      const int si = cs.i;
       const int jl = j - cs.first;   // tile within its split
       const int hi = cs.hi;           // the split's end key
       if (jl == 0 && j > 0) {

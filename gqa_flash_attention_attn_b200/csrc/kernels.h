@@ -35,6 +35,7 @@ struct PrefillParams {
   float c2;           // scale * log2(e)
   unsigned long long timeout_ns;
   LogitExt ext;
+  int mask_tma;       // the mask is staged by TMA (its map is the kernel's tm_m)
 };
 
 struct DecodeParams {
@@ -71,7 +72,7 @@ struct MergeParams {
 
 // Each returns a cudaError_t value (as int) from the launch.
 int launch_prefill(int D, bool ext, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                   const PrefillParams& p, cudaStream_t stream);
+                   const CUtensorMap& tm, const PrefillParams& p, cudaStream_t stream);
 size_t prefill_smem_bytes(int D);
 int launch_decode_split(int D, bool ext, bool fp8, const CUtensorMap& tq, const CUtensorMap& tk,
                         const CUtensorMap& tv, const DecodeParams& p, cudaStream_t stream);

@@ -42,7 +42,8 @@ constexpr int BN = 128;   // keys per tile
 constexpr uint32_t BOX_BYTES = 128u * 128u;  // 128 rows x 64 bf16 columns
 constexpr float LN2 = 0.6931471805599453f;
 
-template <int D>
+// MB: the variant reads an additive mask, staged by TMA in two 64-key halves.
+template <int D, bool MB = false>
 struct PrefillCfg {
   static constexpr int NSLOT = (D <= 128) ? 2 : 1;
   static constexpr int KB = D / 64;
@@ -53,10 +54,12 @@ struct PrefillCfg {
   static constexpr int WARP_MMA = 4 * NSLOT + 1;
   static constexpr uint32_t OFF_Q = 0;
   static constexpr uint32_t OFF_KV = NSLOT * TILE;
-  static constexpr uint32_t OFF_BAR = OFF_KV + NBUF * TILE;
+  static constexpr uint32_t MASK_HALF = BM * 128u;          // 128 rows x 64 bf16 keys
+  static constexpr uint32_t OFF_MASK = OFF_KV + NBUF * TILE;
+  static constexpr uint32_t OFF_BAR = OFF_MASK + (MB ? 2u * MASK_HALF : 0u);
   // q_full, q_empty, kv_full[NBUF], kv_empty[NBUF], s_full[2], p_lo[2], p_hi[2],
-  // pv_done[2], o_free[2], drain
-  static constexpr int NBARS = 2 + 2 * NBUF + 10 + 1;
+  // pv_done[2], o_free[2], drain; with MB mask_full[2], mask_empty[2]
+  static constexpr int NBARS = 2 + 2 * NBUF + 10 + 1 + (MB ? 4 : 0);
   static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
   static constexpr uint32_t SMEM = OFF_MISC + 16 + 1024;  // + alignment slack
   // Two S buffers (one per slot, or a double buffer for one slot), P aliased
@@ -74,6 +77,8 @@ struct PrefillCfg {
   __host__ __device__ static constexpr int bar_pv(int i) { return 8 + 2 * NBUF + i; }
   __host__ __device__ static constexpr int bar_ofree(int i) { return 10 + 2 * NBUF + i; }
   static constexpr int BAR_DRAIN = 12 + 2 * NBUF;
+  __host__ __device__ static constexpr int bar_mfull(int h) { return 13 + 2 * NBUF + h; }
+  __host__ __device__ static constexpr int bar_mempty(int h) { return 15 + 2 * NBUF + h; }
   static_assert(256 + NSLOT * D <= 512, "TMEM budget");
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(D % 64 == 0, "head dim must be a multiple of 64");
@@ -146,11 +151,11 @@ __device__ __forceinline__ int unit_index(int k, int total) {
 
 // Kernel variants by the optional logit terms they handle (plain runs none):
 //   MODE_MASKS  sliding window and sink logits (no per-element arithmetic)
-//   MODE_ALIBI  ALiBi bias and / or an additive mask, with or without window
-//               and sinks
+//   MODE_ALIBI  ALiBi bias, with or without window and sinks
+//   MODE_ALIBI_MASK  an additive mask, with or without ALiBi, window and sinks
 //   MODE_CAP    softcap, with or without ALiBi, window and sinks
 //   MODE_CAP_MASK  softcap with an additive mask (and any other term)
-constexpr int MODE_PLAIN = 0, MODE_MASKS = 1, MODE_ALIBI = 2, MODE_CAP = 3, MODE_CAP_MASK = 4;
+constexpr int MODE_PLAIN = 0, MODE_MASKS = 1, MODE_ALIBI = 2, MODE_CAP = 3, MODE_CAP_MASK = 4, MODE_ALIBI_MASK = 5;
 
 // Logits in log2 units of the N keys of a half tile whose first key sits at
 // distance dist0 = key - pos from the query:
@@ -160,10 +165,11 @@ constexpr int MODE_PLAIN = 0, MODE_MASKS = 1, MODE_ALIBI = 2, MODE_CAP = 3, MODE
 // exact at each half tile, so no per-element index arithmetic is needed.
 // MASK: 0 no mask; 1 mask read as 16-byte vectors (all N keys inside the
 // mask, row 16-byte aligned); 2 mask read one key at a time, keys at or past
-// nvalid read as 0.
+// nvalid read as 0; 3 mask row staged in shared memory (msm, swizzle swz).
 template <int MODE, bool BIAS, int MASK, int N>
 __device__ __forceinline__ void ext_logits_run(float (&v)[N], const LogitExt& x, float c2, float slope2,
-                                               int dist0, const uint16_t* mk, int nvalid) {
+                                               int dist0, const uint16_t* mk, int nvalid,
+                                               const uint8_t* msm = nullptr, int swz = 0) {
   static_assert(N % 8 == 0, "whole groups of four pairs");
   const float b0 = slope2 * (float)dist0;
   float2 bias[4];
@@ -178,7 +184,7 @@ __device__ __forceinline__ void ext_logits_run(float (&v)[N], const LogitExt& x,
     const int i = (e >> 1) & 3;
     const float2 sp = make_float2(v[e], v[e + 1]);
     float2 y;
-    if constexpr (MODE == MODE_ALIBI) {
+    if constexpr (MODE == MODE_ALIBI || MODE == MODE_ALIBI_MASK) {
       y = BIAS ? ffma2(sp, make_float2(c2, c2), bias[i]) : fmul2(sp, make_float2(c2, c2));
     } else {
       const float2 u = fmul2(sp, make_float2(x.cap_a, x.cap_a));
@@ -189,6 +195,10 @@ __device__ __forceinline__ void ext_logits_run(float (&v)[N], const LogitExt& x,
       uint32_t w;
       if constexpr (MASK == 1) {
         if ((e & 7) == 0) mw = __ldg(reinterpret_cast<const uint4*>(mk + e));
+        w = i == 0 ? mw.x : i == 1 ? mw.y : i == 2 ? mw.z : mw.w;
+      } else if constexpr (MASK == 3) {
+        // staged in shared memory: 16-byte chunk e/8 of a 128-byte swizzled row
+        if ((e & 7) == 0) mw = *reinterpret_cast<const uint4*>(msm + ((uint32_t)((e >> 3) ^ swz) << 4));
         w = i == 0 ? mw.x : i == 1 ? mw.y : i == 2 ? mw.z : mw.w;
       } else {
         const uint32_t lo = e < nvalid ? (uint32_t)__ldg(mk + e) : 0u;
@@ -208,8 +218,12 @@ __device__ __forceinline__ void ext_logits_run(float (&v)[N], const LogitExt& x,
 
 template <int MODE, bool BIAS, int N>
 __device__ __forceinline__ void ext_logits_m(float (&v)[N], const LogitExt& x, float c2, float slope2, int dist0,
-                                             const uint16_t* mk, int nvalid) {
-  if (MODE == MODE_CAP || mk == nullptr)
+                                             const uint16_t* mk, int nvalid, const uint8_t* msm, int swz) {
+  if (MODE == MODE_ALIBI || MODE == MODE_CAP)   // no mask in these variants
+    ext_logits_run<MODE, BIAS, 0>(v, x, c2, slope2, dist0, mk, nvalid);
+  else if (msm != nullptr)
+    ext_logits_run<MODE, BIAS, 3>(v, x, c2, slope2, dist0, mk, nvalid, msm, swz);
+  else if (mk == nullptr)
     ext_logits_run<MODE, BIAS, 0>(v, x, c2, slope2, dist0, mk, nvalid);
   else if (nvalid >= N && (reinterpret_cast<uintptr_t>(mk) & 15u) == 0)
     ext_logits_run<MODE, BIAS, 1>(v, x, c2, slope2, dist0, mk, nvalid);
@@ -222,11 +236,12 @@ __device__ __forceinline__ void ext_logits_m(float (&v)[N], const LogitExt& x, f
 // outside the unrolled loops: no path pays for another.
 template <int MODE, int N>
 __device__ __forceinline__ void ext_logits(float (&v)[N], const LogitExt& x, float c2, float slope2, int dist0,
-                                           const uint16_t* mk, int nvalid) {
+                                           const uint16_t* mk, int nvalid, const uint8_t* msm = nullptr,
+                                           int swz = 0) {
   if (x.alibi)
-    ext_logits_m<MODE, true>(v, x, c2, slope2, dist0, mk, nvalid);
+    ext_logits_m<MODE, true>(v, x, c2, slope2, dist0, mk, nvalid, msm, swz);
   else
-    ext_logits_m<MODE, false>(v, x, c2, slope2, dist0, mk, nvalid);
+    ext_logits_m<MODE, false>(v, x, c2, slope2, dist0, mk, nvalid, msm, swz);
 }
 
 // Columns outside [cb, cl) become -inf.
@@ -252,10 +267,12 @@ __device__ __forceinline__ float row_max(const float (&v)[N]) {
 }
 
 template <int D, int MODE>
-__global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
+__global__ void __launch_bounds__(PrefillCfg<D, MODE == MODE_ALIBI_MASK || MODE == MODE_CAP_MASK>::THREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
-  using C = PrefillCfg<D>;
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_m,
+                   const PrefillParams p) {
+  constexpr bool MB = MODE == MODE_ALIBI_MASK || MODE == MODE_CAP_MASK;
+  using C = PrefillCfg<D, MB>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -287,6 +304,12 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
       mbar_init(bar(C::bar_ofree(i)), 128);
     }
     mbar_init(bar(C::BAR_DRAIN), 1);
+    if constexpr (MB) {
+      for (int h = 0; h < 2; ++h) {
+        mbar_init(bar(C::bar_mfull(h)), 1);
+        mbar_init(bar(C::bar_mempty(h)), 4 * C::NSLOT);   // one arrival per softmax warp
+      }
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -302,6 +325,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
 
   int issued = 0;    // producer: K/V ring items issued
   int q_issued = 0;  // producer: Q tiles issued (one per unit)
+  int m_issued = 0;  // producer lane 1: mask tiles issued
 
   if (warp == C::WARP_PRODUCER) {
     if (lane == 0) {
@@ -339,6 +363,32 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
             tma_load_4d(base + C::OFF_KV + buf * C::TILE + kb * BOX_BYTES, tm, bar(C::bar_full(buf)),
                         kb * 64, x.kvh, (x.t0 + (rev ? x.n_tiles - 1 - tile : tile)) * BN, x.b);
           issued = n + 1;
+        }
+      }
+    } else if (MB && lane == 1 && p.mask_tma) {
+      // The additive mask of every tile, in the K/V stream's tile order, as
+      // two 64-key halves (16 KB each, 128-byte swizzled rows); a half is
+      // refilled once every softmax warp has released it.  Each slot visits
+      // every tile (one slot, or an even group size), so the counts agree.
+      tma_prefetch_desc(&tm_m);
+      bool ok = true;
+      int tg = 0;   // this CTA's tiles so far
+      for (int k = 0; ok; ++k) {
+        const int u = unit_index(k, total_units);
+        if (u < 0) break;
+        const Unit x = unit_at<C::NSLOT>(u, p);
+        for (int j = 0; ok && j < x.n_tiles; ++j, ++tg) {
+          const int key0 = (x.t0 + (rev ? x.n_tiles - 1 - j : j)) * BN;
+          for (int h = 0; h < 2; ++h) {
+            if (tg > 0 && !mbar_wait(bar(C::bar_mempty(h)), (uint32_t)(tg - 1) & 1u, wd)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(bar(C::bar_mfull(h)), C::MASK_HALF);
+            tma_load_4d(base + C::OFF_MASK + h * C::MASK_HALF, &tm_m, bar(C::bar_mfull(h)), key0 + 64 * h, x.s0,
+                        p.ext.mask_sb != 0 ? x.b : 0, 0);
+          }
+          m_issued = tg + 1;
         }
       }
     }
@@ -511,7 +561,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
       const float slope2 =
           (MODE >= MODE_ALIBI && p.ext.alibi) ? alibi_slope_log2e(h, p.ext.l2m0, p.ext.l2m1, p.ext.n2) : 0.f;
       // this row's mask (padding rows past Sq read the last row's: never stored)
-      const uint16_t* mrow = ((MODE == MODE_ALIBI || MODE == MODE_CAP_MASK) && p.ext.mask != nullptr)
+      const uint16_t* mrow = ((MODE == MODE_ALIBI_MASK || MODE == MODE_CAP_MASK) && p.ext.mask != nullptr)
                                  ? p.ext.mask + (size_t)x.b * p.ext.mask_sb + (size_t)min(s_row, p.Sq - 1) * p.ext.mask_sr
                                  : nullptr;
       float m_use = -INFINITY, l = 0.f;
@@ -536,10 +586,21 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
           // first, for their maximum only, so that one half of the row is
           // live at a time.  Their logits go back to their own TMEM columns
           // (P only ever covers columns 0-63), where half 1 below reads them.
+          // staged mask: wait for this tile's halves (global tile T + j)
+          const bool mstaged = MB && p.mask_tma;
+          const uint8_t* msm_hi = nullptr;
+          const uint8_t* msm_lo = nullptr;
+          if (mstaged) {
+            const uint32_t mph = (uint32_t)(T + j) & 1u;
+            const bool got_m = mbar_wait(bar(C::bar_mfull(1)), mph, wd) && mbar_wait(bar(C::bar_mfull(0)), mph, wd);
+            if (__any_sync(0xffffffffu, !got_m)) { ok = false; break; }
+            msm_lo = gbase + C::OFF_MASK + (uint32_t)r * 128u;
+            msm_hi = msm_lo + C::MASK_HALF;
+          }
           float sh[BN / 2];
           tmem_ld64(tS + BN / 2, sh);
           ext_logits<MODE>(sh, p.ext, c2, slope2, key0 + BN / 2 - pos, mrow ? mrow + key0 + BN / 2 : nullptr,
-                           p.Skv - (key0 + BN / 2));
+                           p.Skv - (key0 + BN / 2), msm_hi, r & 7);
           {
             uint32_t u[BN / 2];
 #pragma unroll
@@ -550,7 +611,16 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
           const float mx_hi = row_max(sh);
           float (&slo)[BN / 2] = *reinterpret_cast<float(*)[BN / 2]>(sv);
           tmem_ld64(tS, slo);
-          ext_logits<MODE>(slo, p.ext, c2, slope2, key0 - pos, mrow ? mrow + key0 : nullptr, p.Skv - key0);
+          ext_logits<MODE>(slo, p.ext, c2, slope2, key0 - pos, mrow ? mrow + key0 : nullptr, p.Skv - key0, msm_lo,
+                           r & 7);
+          if (mstaged) {
+            // both halves read into registers: release them to the producer
+            __syncwarp();
+            if (lane == 0) {
+              mbar_arrive(bar(C::bar_mempty(0)));
+              mbar_arrive(bar(C::bar_mempty(1)));
+            }
+          }
           if (tile_masked) mask_cols(slo, cb, cl);
           mx = fmaxf(mx_hi, row_max(slo));
         } else {
@@ -696,6 +766,13 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
     // Nothing may still write this CTA's shared memory or TMEM when it exits.
     if (warp == C::WARP_PRODUCER && lane == 0) {
       if (q_issued > 0) drain_wait(bar(C::BAR_Q), (uint32_t)(q_issued - 1) & 1u, p.timeout_ns);
+    }
+    if (MB && warp == C::WARP_PRODUCER && lane == 1 && m_issued > 0) {
+      // only the last mask tile can still be in flight: an earlier one was
+      // consumed (after it arrived) before its buffer was reloaded
+      for (int h = 0; h < 2; ++h) drain_wait(bar(C::bar_mfull(h)), (uint32_t)(m_issued - 1) & 1u, p.timeout_ns);
+    }
+    if (warp == C::WARP_PRODUCER && lane == 0) {
       for (int n = max(0, issued - C::NBUF); n < issued; ++n)
         drain_wait(bar(C::bar_full(n % C::NBUF)), (uint32_t)(n / C::NBUF) & 1u, p.timeout_ns);
     }
@@ -713,16 +790,16 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
 }
 
 template <int D, int MODE>
-int launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+int launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tm,
              const PrefillParams& p, cudaStream_t stream) {
-  using C = PrefillCfg<D>;
+  using C = PrefillCfg<D, MODE == MODE_ALIBI_MASK || MODE == MODE_CAP_MASK>;
   cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)C::SMEM);
   if (e != cudaSuccess) return (int)e;
   const long long units = (long long)p.n_qt * p.B * p.Hkv * p.units_per_kvh;
   if (units <= 0 || units > 0x7fffffffLL || p.num_ctas <= 0) return (int)cudaErrorInvalidValue;
   const long long grid = units < p.num_ctas ? units : p.num_ctas;  // persistent: one CTA per SM
-  prefill_kernel<D, MODE><<<(unsigned)grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, p);
+  prefill_kernel<D, MODE><<<(unsigned)grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, tm, p);
   return (int)cudaGetLastError();
 }
 
@@ -740,28 +817,30 @@ size_t prefill_smem_bytes(int D) {
 int prefill_slots(int D) { return D <= 128 ? 2 : 1; }
 
 template <int D>
-int launch_mode(int mode, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+int launch_mode(int mode, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tm,
                 const PrefillParams& p, cudaStream_t stream) {
   switch (mode) {
-    case MODE_PLAIN: return launch_t<D, MODE_PLAIN>(tq, tk, tv, p, stream);
-    case MODE_MASKS: return launch_t<D, MODE_MASKS>(tq, tk, tv, p, stream);
-    case MODE_ALIBI: return launch_t<D, MODE_ALIBI>(tq, tk, tv, p, stream);
-    case MODE_CAP: return launch_t<D, MODE_CAP>(tq, tk, tv, p, stream);
-    default: return launch_t<D, MODE_CAP_MASK>(tq, tk, tv, p, stream);
+    case MODE_PLAIN: return launch_t<D, MODE_PLAIN>(tq, tk, tv, tm, p, stream);
+    case MODE_MASKS: return launch_t<D, MODE_MASKS>(tq, tk, tv, tm, p, stream);
+    case MODE_ALIBI: return launch_t<D, MODE_ALIBI>(tq, tk, tv, tm, p, stream);
+    case MODE_CAP: return launch_t<D, MODE_CAP>(tq, tk, tv, tm, p, stream);
+    case MODE_ALIBI_MASK: return launch_t<D, MODE_ALIBI_MASK>(tq, tk, tv, tm, p, stream);
+    default: return launch_t<D, MODE_CAP_MASK>(tq, tk, tv, tm, p, stream);
   }
 }
 
 int launch_prefill(int D, bool ext, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                   const PrefillParams& p, cudaStream_t stream) {
+                   const CUtensorMap& tm, const PrefillParams& p, cudaStream_t stream) {
   // the cheapest variant that covers the requested terms
   const int mode = !ext ? MODE_PLAIN
                    : p.ext.cap_a > 0.f ? (p.ext.mask != nullptr ? MODE_CAP_MASK : MODE_CAP)
-                   : (p.ext.alibi || p.ext.mask != nullptr) ? MODE_ALIBI
+                   : p.ext.mask != nullptr ? MODE_ALIBI_MASK
+                   : p.ext.alibi ? MODE_ALIBI
                    : MODE_MASKS;
   switch (D) {
-    case 64: return launch_mode<64>(mode, tq, tk, tv, p, stream);
-    case 128: return launch_mode<128>(mode, tq, tk, tv, p, stream);
-    case 256: return launch_mode<256>(mode, tq, tk, tv, p, stream);
+    case 64: return launch_mode<64>(mode, tq, tk, tv, tm, p, stream);
+    case 128: return launch_mode<128>(mode, tq, tk, tv, tm, p, stream);
+    case 256: return launch_mode<256>(mode, tq, tk, tv, tm, p, stream);
     default: return (int)cudaErrorInvalidValue;
   }
 }
