@@ -324,8 +324,7 @@ int attn_decode_split_kv(const void* q, const attn_kv_view* kv, float* partial_o
     ++nbuf;
   p.nbuf = nbuf;
   // Consecutive splits per CTA: enough that the CTAs fit the resident slots
-  // (two per SM when the shared memory allows) in one wave, at most 8, for
-  // splits of at most 8 tiles.
+  // (two per SM when the shared memory allows) in one wave, at most 8.
   {
     const int nsm = sm_count();
     if (nsm <= 0) return cuda_fail();
@@ -333,8 +332,6 @@ int attn_decode_split_kv(const void* q, const attn_kv_view* kv, float* partial_o
         (long long)nsm * (gqa::decode_smem_bytes(D, p.RP, nbuf, p.mask_rows, fp8) <= kTwoCtaSmemLimit ? 2 : 1);
     const long long units = (long long)num_splits * B * Hkv;
     long long grp = (units + slots - 1) / slots;
-    // long splits already amortise a CTA's start and end: group short ones only
-    if ((p.chunk + 127) / 128 > 8) grp = 1;
     grp = std::min<long long>(std::min<long long>(grp, gqa::decode_max_group()), num_splits);
     p.group = (int)std::max<long long>(grp, 1);
     // two O^T buffers when split boundaries exist and two CTAs' TMEM still fits

@@ -176,6 +176,29 @@ __device__ __forceinline__ void ext_rows16(float (&v)[16], const LogitExt& x, fl
   }
 }
 
+// O^T / l of one split from TMEM to the fp32 partial (rows r < R of this
+// CTA's group), called once per split: kept out of line so the tile loop
+// stays small.  Thread t owns column t of each 128-column chunk.
+template <int KC>
+__device__ __noinline__ void write_partial_o(uint32_t taddr, int RP, int R, int g, int kvh, int b, int Sq, int Hq,
+                                             float* part_out, const float* inv_sm, int t) {
+  constexpr int D = KC * 128;
+  for (int c = 0; c < KC; ++c) {
+    for (int q = 0; q < RP / 16; ++q) {
+      float v[16];
+      tmem_ld16(taddr + (uint32_t)(c * RP + 16 * q), v);
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int r = 16 * q + e;
+        if (r < R) {
+          const int s = r / g, h = kvh * g + (r - s * g);
+          part_out[(((size_t)b * Sq + s) * Hq + h) * D + c * 128 + t] = v[e] * inv_sm[r];
+        }
+      }
+    }
+  }
+}
+
 template <int D, bool EXT, bool PAGED, bool FP8>
 __global__ void __launch_bounds__(THREADS, 2)
     decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -569,21 +592,8 @@ __global__ void __launch_bounds__(THREADS, 2)
     auto write_o = [&](int si) {
       named_bar_sync(1, 128);   // inv_sm of every row
       const size_t so = (size_t)(sg0 + si) * p.B * p.Sq * p.Hq * D;
-      const int ob = seg_sm[si].ob;
-      for (int c = 0; c < KC; ++c) {
-        for (int q = 0; q < RP / 16; ++q) {
-          float v[16];
-          tmem_ld16(tmem + lane_off + TO(c, ob) + 16 * q, v);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int r = 16 * q + e;
-            if (r < R) {
-              const int s = r / g, h = kvh * g + (r - s * g);
-              p.part_out[so + (((size_t)b * p.Sq + s) * p.Hq + h) * D + c * 128 + t] = v[e] * inv_sm[r];
-            }
-          }
-        }
-      }
+      write_partial_o<KC>(tmem + lane_off + TO(0, seg_sm[si].ob), RP, R, g, kvh, b, p.Sq, p.Hq, p.part_out + so,
+                          inv_sm, t);
       named_bar_sync(1, 128);   // every row's inv_sm read before stats() rewrites it
     };
     // wait (jointly) for the P.V of stream tile j
