@@ -117,8 +117,10 @@ int attn_merge(const float* partial_out, const float* partial_lse, void* out, fl
 size_t attn_decode_workspace_bytes(int B, int Hq, int Sq, int D, int num_splits);
 
 /* Synchronises `stream`, then returns and clears the device status word of
- * the current device: ATTN_OK, or ATTN_ERR_TIMEOUT if a kernel gave up on a
- * stalled pipeline since the last call.  ATTN_ERR_CUDA if the sync fails. */
+ * the current device: ATTN_OK; ATTN_ERR_TIMEOUT if a kernel gave up on a
+ * stalled pipeline since the last call; ATTN_ERR_INVALID_ARG if a device-side
+ * sequence length (attn_kv_view.seq_lens) was outside [0, Skv] and was
+ * clamped.  ATTN_ERR_CUDA if the sync fails. */
 int attn_last_status(void* stream);
 
 /* Human-readable name of a status code (static storage). */
