@@ -150,6 +150,53 @@ int make_ext(const attn_options* opt, int Hq, int Sq, int Skv, int q_offset, int
   return ATTN_OK;
 }
 
+// Prefill at D = 512: the split-KV kernel with one split, query rows cut into
+// chunks of 32 / g positions per CTA (its TMEM holds 2 S^T buffers and
+// O^T for <= 32 rows at D = 512), writing the final O and LSE directly.
+int prefill_wide(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv, int Sq,
+                 int Skv, int D, int q_offset, int causal, float scale, int out_dtype, const gqa::LogitExt& ext,
+                 bool ext_on, void* stream) {
+  const int g = Hq / Hkv;
+  if (g > 32) return ATTN_ERR_UNSUPPORTED;
+  const int qchunk = std::min(32 / g, Sq);
+  const int nqc = (Sq + qchunk - 1) / qchunk;
+  if ((long long)B * Hkv * nqc > 65535) return ATTN_ERR_UNSUPPORTED;   // grid rows
+  gqa::DecodeParams p{};
+  p.part_out = nullptr;
+  p.part_lse = lse;
+  p.fout = out;
+  p.fout_bf16 = out_dtype == ATTN_BF16;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Sq = Sq; p.Skv = Skv;
+  p.q_offset = q_offset; p.causal = causal;
+  p.g = g; p.R = g * qchunk; p.RP = (p.R + 15) / 16 * 16;
+  p.qchunk = qchunk;
+  p.nqc = nqc;
+  p.num_splits = 1;
+  p.chunk = Skv;
+  p.group = 1;
+  p.obuf = 1;
+  p.mask_rows = (ext.mask != nullptr && aligned(ext.mask, 16) && ext.mask_sb % 8 == 0 && ext.mask_sr % 8 == 0)
+                    ? qchunk
+                    : 0;
+  int nbuf = 2;
+  while (nbuf < gqa::decode_max_nbuf() &&
+         gqa::decode_smem_bytes(D, p.RP, nbuf + 1, p.mask_rows, false) <= kTwoCtaSmemLimit)
+    ++nbuf;
+  p.nbuf = nbuf;
+  p.c2 = scale * kLog2e;
+  p.timeout_ns = kWaitLimitNs;
+  p.ext = ext;
+  p.status = status_ptr();
+  if (p.status == nullptr) return cuda_fail();
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q, D, Hq, Sq, B, 64, (uint32_t)g, (uint32_t)qchunk, 1)) return cuda_fail();
+  if (!make_map(&tk, k, D, Hkv, Skv, B, 64, 1, 128, 1)) return cuda_fail();
+  if (!make_map(&tv, v, D, Hkv, Skv, B, 64, 1, 128, 1)) return cuda_fail();
+  return gqa::launch_decode_split(D, ext_on, false, tq, tk, tv, p, static_cast<cudaStream_t>(stream)) == 0
+             ? ATTN_OK
+             : ATTN_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
@@ -186,9 +233,12 @@ int attn_prefill_ex(const void* q, const void* k, const void* v, void* out, floa
   if (st != ATTN_OK) return st;
   if (out == nullptr) return ATTN_ERR_INVALID_ARG;
   if (out_dtype != ATTN_BF16 && out_dtype != ATTN_F32) return ATTN_ERR_INVALID_ARG;
-  if (D != 64 && D != 128 && D != 256) return ATTN_ERR_UNSUPPORTED;
+  if (D != 64 && D != 128 && D != 256 && D != 512) return ATTN_ERR_UNSUPPORTED;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16)) return ATTN_ERR_ALIGNMENT;
   if (lse != nullptr && !aligned(lse, 4)) return ATTN_ERR_ALIGNMENT;
+  if (D == 512)
+    return prefill_wide(q, k, v, out, lse, B, Hq, Hkv, Sq, Skv, D, q_offset, causal, scale, out_dtype, ext, ext_on,
+                        stream);
 
   const int nslot = gqa::prefill_slots(D);
   const int g = Hq / Hkv;
@@ -346,6 +396,9 @@ int attn_decode_split_kv(const void* q, const attn_kv_view* kv, float* partial_o
   p.page_size = paged ? kv->page_size : 0;
   p.k_scale = fp8 ? kv->k_scale : nullptr;
   p.v_scale = fp8 ? kv->v_scale : nullptr;
+  p.qchunk = Sq;
+  p.nqc = 1;
+  p.fout = nullptr;
 
   p.status = status_ptr();
   if (p.status == nullptr) return cuda_fail();

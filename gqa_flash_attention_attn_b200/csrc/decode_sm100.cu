@@ -180,8 +180,8 @@ __device__ __forceinline__ void ext_rows16(float (&v)[16], const LogitExt& x, fl
 // CTA's group), called once per split: kept out of line so the tile loop
 // stays small.  Thread t owns column t of each 128-column chunk.
 template <int KC>
-__device__ __noinline__ void write_partial_o(uint32_t taddr, int RP, int R, int g, int kvh, int b, int Sq, int Hq,
-                                             float* part_out, const float* inv_sm, int t) {
+__device__ __noinline__ void write_partial_o(uint32_t taddr, int RP, int R, int g, int kvh, int b, int s0, int Sq,
+                                             int Hq, void* out, bool out_bf16, const float* inv_sm, int t) {
   constexpr int D = KC * 128;
   for (int c = 0; c < KC; ++c) {
     for (int q = 0; q < RP / 16; ++q) {
@@ -191,8 +191,12 @@ __device__ __noinline__ void write_partial_o(uint32_t taddr, int RP, int R, int 
       for (int e = 0; e < 16; ++e) {
         const int r = 16 * q + e;
         if (r < R) {
-          const int s = r / g, h = kvh * g + (r - s * g);
-          part_out[(((size_t)b * Sq + s) * Hq + h) * D + c * 128 + t] = v[e] * inv_sm[r];
+          const int s = s0 + r / g, h = kvh * g + (r % g);
+          const size_t o = (((size_t)b * Sq + s) * Hq + h) * D + c * 128 + t;
+          if (out_bf16)
+            reinterpret_cast<__nv_bfloat16*>(out)[o] = __float2bfloat16_rn(v[e] * inv_sm[r]);
+          else
+            reinterpret_cast<float*>(out)[o] = v[e] * inv_sm[r];
         }
       }
     }
@@ -204,7 +208,7 @@ __global__ void __launch_bounds__(THREADS, 2)
     decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
   constexpr int KC = D / 128;  // 128-column slots per K (or V) tile
-  const int RP = p.RP, R = p.R, g = p.g, nbuf = p.nbuf;
+  const int RP = p.RP, g = p.g, nbuf = p.nbuf;
   const Layout L(D, RP, nbuf, p.mask_rows, FP8);
   constexpr uint32_t SLOTB = FP8 ? BOX_BYTES : SLOT_BYTES;   // bytes of one 128-column K/V slot
 
@@ -242,7 +246,13 @@ __global__ void __launch_bounds__(THREADS, 2)
   const int BAR_Q8 = BAR_S0 + 7;         // fp8: Q planes written
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int b = blockIdx.y / p.Hkv, kvh = blockIdx.y % p.Hkv;
+  const int bkv = blockIdx.y / p.nqc, qc = blockIdx.y - bkv * p.nqc;
+  const int b = bkv / p.Hkv, kvh = bkv % p.Hkv;
+  const int s0 = qc * p.qchunk;               // this CTA's first query row
+  const int Sqc = min(p.qchunk, p.Sq - s0);   // and its query rows
+  const int Rbox = g * p.qchunk;               // rows the Q box brings (past Sq: zeros)
+  const int R = g * Sqc;                       // real rows
+  const int mrows = min(p.mask_rows, Sqc);     // staged mask rows
   // this sequence's keys and the position of its first query row
   int Skv = p.Skv, q_offset = p.q_offset;
   long long chunk = p.chunk;
@@ -255,6 +265,7 @@ __global__ void __launch_bounds__(THREADS, 2)
     chunk = (Skv + p.num_splits - 1) / p.num_splits;
   }
   if (PAGED) chunk = (chunk + BN - 1) / BN * BN;  // no tile crosses a page
+  q_offset += s0;   // this CTA's rows sit at q_offset .. q_offset + Sqc - 1
   // With ALiBi the bias grows toward each query's own position: visiting a
   // split's tiles newest first sets the running maximum on the first tile and
   // spares the O rescales (the tile order does not change the result).
@@ -270,7 +281,7 @@ __global__ void __launch_bounds__(THREADS, 2)
     const long long lo_ll = (long long)(sg0 + i) * chunk;
     const int lo = (int)min(lo_ll, (long long)Skv);
     const int hi = (int)min(lo_ll + chunk, (long long)Skv);
-    const int eff_hi = p.causal ? (int)min((long long)hi, (long long)q_offset + p.Sq) : hi;
+    const int eff_hi = p.causal ? (int)min((long long)hi, (long long)q_offset + Sqc) : hi;
     // a sliding window hides every key at or before q_offset - window from all rows
     const int eff_lo = (EXT && p.ext.window > 0) ? max(lo, q_offset - p.ext.window + 1) : lo;
     const int kb = lo + ((eff_lo - lo) / BN) * BN;   // first tile, on the split's tile grid
@@ -283,11 +294,14 @@ __global__ void __launch_bounds__(THREADS, 2)
       const size_t sl = (size_t)(sg0 + i) * p.B * p.Hq * p.Sq;
       for (int x = threadIdx.x; x < R * D; x += THREADS) {
         const int r = x / D, d = x - r * D;
-        const int s = r / g, h = kvh * g + (r - s * g);
-        p.part_out[so + (((size_t)b * p.Sq + s) * p.Hq + h) * D + d] = 0.f;
+        const int s = s0 + r / g, h = kvh * g + (r % g);
+        const size_t o = so + (((size_t)b * p.Sq + s) * p.Hq + h) * D + d;
+        if (p.fout == nullptr) p.part_out[o] = 0.f;
+        else if (p.fout_bf16) reinterpret_cast<__nv_bfloat16*>(p.fout)[o] = __float2bfloat16_rn(0.f);
+        else reinterpret_cast<float*>(p.fout)[o] = 0.f;
       }
-      for (int r = threadIdx.x; r < R; r += THREADS) {
-        const int s = r / g, h = kvh * g + (r - s * g);
+      for (int r = threadIdx.x; r < R && p.part_lse != nullptr; r += THREADS) {
+        const int s = s0 + r / g, h = kvh * g + (r % g);
         p.part_lse[sl + ((size_t)b * p.Hq + h) * p.Sq + s] = -INFINITY;
       }
     }
@@ -302,11 +316,11 @@ __global__ void __launch_bounds__(THREADS, 2)
     return i;
   };
 
-  // Zero the padding rows of Q (rows R..RP-1 of every 64-column box).
-  for (int i = threadIdx.x; i < (D / 64) * (RP - R) * 32; i += THREADS) {
-    const int box = i / ((RP - R) * 32);
-    const int w = i - box * (RP - R) * 32;
-    reinterpret_cast<uint32_t*>(gbase + L.off_q + (uint32_t)box * RP * 128u + (uint32_t)R * 128u)[w] = 0u;
+  // Zero the padding rows of Q (rows Rbox..RP-1 of every 64-column box).
+  for (int i = threadIdx.x; i < (D / 64) * (RP - Rbox) * 32; i += THREADS) {
+    const int box = i / ((RP - Rbox) * 32);
+    const int w = i - box * (RP - Rbox) * 32;
+    reinterpret_cast<uint32_t*>(gbase + L.off_q + (uint32_t)box * RP * 128u + (uint32_t)Rbox * 128u)[w] = 0u;
   }
   if (threadIdx.x < RP) {
     const int r = threadIdx.x;
@@ -320,7 +334,7 @@ __global__ void __launch_bounds__(THREADS, 2)
                       ? alibi_slope_log2e(kvh * g + (r - (r / g) * g), p.ext.l2m0, p.ext.l2m1, p.ext.n2)
                       : 0.f;
     mrow_sm[r] = (EXT && p.ext.mask != nullptr && r < R)
-                     ? p.ext.mask + (size_t)b * p.ext.mask_sb + (size_t)(r / g) * p.ext.mask_sr
+                     ? p.ext.mask + (size_t)b * p.ext.mask_sb + (size_t)(s0 + r / g) * p.ext.mask_sr
                      : nullptr;
   }
   if (threadIdx.x == 0) {
@@ -362,9 +376,9 @@ __global__ void __launch_bounds__(THREADS, 2)
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      mbar_arrive_expect_tx(bar(BAR_Q), (uint32_t)(D / 64) * R * 128u);
+      mbar_arrive_expect_tx(bar(BAR_Q), (uint32_t)(D / 64) * Rbox * 128u);
       for (int kb = 0; kb < D / 64; ++kb)
-        tma_load_4d(base + L.off_q + (uint32_t)kb * RP * 128u, &tm_q, bar(BAR_Q), kb * 64, kvh * g, 0, b);
+        tma_load_4d(base + L.off_q + (uint32_t)kb * RP * 128u, &tm_q, bar(BAR_Q), kb * 64, kvh * g, s0, b);
       // ring order: K_0, then (K_{j+1}, V_j) for j = 0..n-1; KC slots each
       bool ok = true;
       int n = 0;
@@ -579,21 +593,35 @@ __global__ void __launch_bounds__(THREADS, 2)
     // stores O^T / l from its TMEM buffer (after its last P.V completed).
     auto stats = [&](int si) {
       if (t < RP) {
-        const float l = l_sm[t];
-        inv_sm[t] = l > 0.f ? vs / l : 0.f;
-        if (t < R) {
-          const int s = t / g, h = kvh * g + (t - s * g);
+        float l = l_sm[t];
+        float m = m_sm[t];
+        if (EXT && p.fout != nullptr && p.ext.sinks != nullptr && t < R) {
+          // final output (one split, no merge): fold the sink in against a
+          // common maximum, as the merge would
+          const float s2 = __ldg(p.ext.sinks + kvh * g + (t % g)) * 1.4426950408889634f + (FP8 ? 6.f : 0.f);
+          const float mf = fmaxf(m, s2);
+          const float a = ex2_approx(m - mf);
+          l = l * a + ex2_approx(s2 - mf);
+          inv_sm[t] = vs * a / l;
+          m = mf;
+        } else {
+          inv_sm[t] = l > 0.f ? vs / l : 0.f;
+        }
+        if (t < R && p.part_lse != nullptr) {
+          const int s = s0 + t / g, h = kvh * g + (t % g);
           const size_t sl = (size_t)(sg0 + si) * p.B * p.Hq * p.Sq;
           p.part_lse[sl + ((size_t)b * p.Hq + h) * p.Sq + s] =
-              l > 0.f ? (m_sm[t] + log2f(l) - (FP8 ? 6.f : 0.f)) * LN2 : -INFINITY;
+              l > 0.f ? (m + log2f(l) - (FP8 ? 6.f : 0.f)) * LN2 : -INFINITY;
         }
       }
     };
     auto write_o = [&](int si) {
       named_bar_sync(1, 128);   // inv_sm of every row
       const size_t so = (size_t)(sg0 + si) * p.B * p.Sq * p.Hq * D;
-      write_partial_o<KC>(tmem + lane_off + TO(0, seg_sm[si].ob), RP, R, g, kvh, b, p.Sq, p.Hq, p.part_out + so,
-                          inv_sm, t);
+      // partials (fp32), or with one split the final output itself
+      void* dst = p.fout != nullptr ? p.fout : static_cast<void*>(p.part_out + so);
+      write_partial_o<KC>(tmem + lane_off + TO(0, seg_sm[si].ob), RP, R, g, kvh, b, s0, p.Sq, p.Hq, dst,
+                          p.fout != nullptr && p.fout_bf16, inv_sm, t);
       named_bar_sync(1, 128);   // every row's inv_sm read before stats() rewrites it
     };
     // wait (jointly) for the P.V of stream tile j
@@ -647,11 +675,11 @@ __global__ void __launch_bounds__(THREADS, 2)
           const int tile_al = cm.key0(jj, rev) & ~7;
           const int shi = cm.hi;
           const uint32_t dst0 = mstage_u32 + (uint32_t)(jj & 1) * p.mask_rows * MROW_BYTES;
-          for (int c = t; c < p.mask_rows * 17; c += 128) {
+          for (int c = t; c < mrows * 17; c += 128) {
             const int row = c / 17, k8 = (c - row * 17) * 8;
             const int key8 = tile_al + k8;
             const int n = min(max(shi - key8, 0), 8);   // keys inside the split (end <= Skv)
-            const uint16_t* src = n > 0 ? p.ext.mask + (size_t)b * p.ext.mask_sb + (size_t)row * p.ext.mask_sr + key8
+            const uint16_t* src = n > 0 ? p.ext.mask + (size_t)b * p.ext.mask_sb + (size_t)(s0 + row) * p.ext.mask_sr + key8
                                         : p.ext.mask;
             cp_async16(dst0 + (uint32_t)row * MROW_BYTES + (uint32_t)k8 * 2u, src, (uint32_t)n * 2u);
           }
@@ -674,7 +702,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       const uint16_t* mtile = mstage + (size_t)(j & 1) * p.mask_rows * MROW_KEYS + (tile0 & 7) + t;
       // whole tile visible to every real row: no per-element mask
       const bool full = (tile0 + BN - 1 < hi) && (!p.causal || tile0 + BN - 1 <= q_offset) &&
-                        (!EXT || p.ext.window == 0 || tile0 >= q_offset + p.Sq - p.ext.window);
+                        (!EXT || p.ext.window == 0 || tile0 >= q_offset + Sqc - p.ext.window);
       auto visible = [&](int r) -> bool {
         return key < hi && key <= lim_sm[r] && (!EXT || key > limlo_sm[r]);
       };
@@ -683,7 +711,7 @@ __global__ void __launch_bounds__(THREADS, 2)
         float v[16];
         tmem_ld16(tmem + lane_off + TS(sb) + 16 * q, v);
         if (EXT)
-          ext_rows16(v, xe, c2, key, t, q, slope_sm, pos_sm, mtile, p.mask_rows, q_offset, mrow_sm, hi);
+          ext_rows16(v, xe, c2, key, t, q, slope_sm, pos_sm, mtile, mrows, q_offset, mrow_sm, hi);
         if (!full) {
 #pragma unroll
           for (int e = 0; e < 16; ++e)
@@ -723,7 +751,7 @@ __global__ void __launch_bounds__(THREADS, 2)
           float v[16];
           tmem_ld16(tmem + lane_off + TS(sb) + 16 * q, v);
           if (EXT) {
-            ext_rows16(v, xe, c2, key, t, q, slope_sm, pos_sm, mtile, p.mask_rows, q_offset, mrow_sm, hi);
+            ext_rows16(v, xe, c2, key, t, q, slope_sm, pos_sm, mtile, mrows, q_offset, mrow_sm, hi);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const float4 w = reinterpret_cast<const float4*>(msub_sm + 16 * q)[i];
@@ -840,7 +868,7 @@ int launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv
   cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, EXT, PAGED, FP8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
   if (e != cudaSuccess) return (int)e;
-  dim3 grid((unsigned)((p.num_splits + p.group - 1) / p.group), (unsigned)(p.B * p.Hkv));
+  dim3 grid((unsigned)((p.num_splits + p.group - 1) / p.group), (unsigned)(p.B * p.Hkv * p.nqc));
   decode_split_kernel<D, EXT, PAGED, FP8><<<grid, THREADS, L.total, stream>>>(tq, tk, tv, p);
   return (int)cudaGetLastError();
 }

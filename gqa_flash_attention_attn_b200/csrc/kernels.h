@@ -59,6 +59,13 @@ struct DecodeParams {
   // fp8 e4m3 K/V: one scale per K/V head (K = code * k_scale[kvh], same for V)
   const float* k_scale;
   const float* v_scale;
+  // query rows per CTA (Sq for decode; fewer when a long Sq is cut into
+  // chunks, one CTA row of the grid each: nqc chunks)
+  int qchunk, nqc;
+  // final output instead of partials (one split): O [B, Sq, Hq, D] as bf16
+  // (fout_bf16) or fp32 at fout, LSE at part_lse (may be nullptr)
+  void* fout;
+  int fout_bf16;
 };
 
 struct MergeParams {

@@ -143,6 +143,10 @@ WORKLOADS = {
         "fp8_kv_spec_verify_decode_d128", "decode", B=4, Hq=32, Hkv=8, Sq=8, Skv=32768, D=128,
         q_offset=32760, causal=True, out_dtype="bf16", num_splits=16, kv_dtype="fp8",
         note="the 8-row verify decode over an fp8 e4m3 K/V cache"),
+    "prefill_d512_g16_4k": Workload(
+        "prefill_d512_g16_4k", "prefill", B=1, Hq=16, Hkv=1, Sq=4096, Skv=4096, D=512,
+        q_offset=0, causal=True, out_dtype="bf16",
+        note="B1 Hq16 Hkv1 Sq=Skv=4096 D512, causal: head size 512 with one K/V head (MLA-like width)"),
     "paged_decode_d512_p64": Workload(
         "paged_decode_d512_p64", "decode", B=16, Hq=16, Hkv=1, Sq=1, Skv=16384, D=512,
         q_offset=16383, causal=True, out_dtype="bf16", num_splits=32, page_size=64,

@@ -65,7 +65,8 @@ def _prefill(lib, **kw):
     (dict(out_dtype=7), ga.ATTN_ERR_INVALID_ARG),
     (dict(D=72), ga.ATTN_ERR_UNSUPPORTED),     # the head size that crashed a staging path
     (dict(D=32), ga.ATTN_ERR_UNSUPPORTED),
-    (dict(D=512), ga.ATTN_ERR_UNSUPPORTED),
+    (dict(D=512, Hq=64, Hkv=1), ga.ATTN_ERR_UNSUPPORTED),   # D = 512 needs a group of at most 32
+    (dict(D=320), ga.ATTN_ERR_UNSUPPORTED),
     (dict(q=MIS), ga.ATTN_ERR_ALIGNMENT),
     (dict(v=MIS), ga.ATTN_ERR_ALIGNMENT),
     (dict(out=MIS), ga.ATTN_ERR_ALIGNMENT),

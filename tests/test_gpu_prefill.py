@@ -103,3 +103,51 @@ def test_full_size_workload_sampled_rows(name):
     # every row, not only the sampled ones, is finite
     assert torch.isfinite(out).all()
     assert torch.isfinite(lse).all()
+
+
+# D = 512 (the split-KV kernel in query-chunk mode):
+# (B, Hq, Hkv, Sq, Skv, q_offset, causal, out_dtype, options)
+WIDE = [
+    (1, 4, 1, 300, 300, 0, True, torch.float32, {}),                 # group 4: 8 rows per CTA
+    (2, 16, 1, 130, 130, 0, True, torch.bfloat16, {}),               # group 16: 2 rows per CTA
+    (1, 8, 8, 77, 500, 423, True, torch.bfloat16, {}),               # MHA at depth, 32 rows per CTA
+    (1, 8, 2, 64, 333, 0, False, torch.float32, {}),                 # non-causal, ragged keys
+    (1, 8, 1, 100, 400, 300, True, torch.float32,
+     dict(softcap=20.0, alibi_max_bias=4.0, window=150, sinks=True, mask=True)),
+]
+
+
+@pytest.mark.parametrize("case", WIDE, ids=[f"w{i}" for i in range(len(WIDE))])
+def test_prefill_d512_matches_oracle(case):
+    from gqa_flash_attention_attn_b200.inputs import make_mask, make_sinks
+    B, Hq, Hkv, Sq, Skv, q_offset, causal, out_dtype, opts = case
+    D = 512
+    q, k, v = make_qkv(B, Hq, Hkv, Sq, Skv, D, seed=61)
+    scale = float(torch.tensor(1.0 / math.sqrt(D), dtype=torch.float32))
+    kw = {kk: vv for kk, vv in opts.items() if kk not in ("sinks", "mask")}
+    sinks = make_sinks(Hq, seed=62) if opts.get("sinks") else None
+    mask = make_mask(B, Sq, Skv, seed=63) if opts.get("mask") else None
+    out, lse = ga.prefill(q.cuda(), k.cuda(), v.cuda(), causal=causal, q_offset=q_offset, scale=scale,
+                          out_dtype=out_dtype, sinks=None if sinks is None else sinks.cuda(),
+                          mask=None if mask is None else mask.cuda(), **kw)
+    torch.cuda.synchronize()
+    assert ga.last_status() == ga.ATTN_OK
+    want_o, want_l = oracle.attention_ex(q, k, v, scale=scale, causal=causal, q_offset=q_offset,
+                                         sinks=None if sinks is None else sinks.numpy(), mask=mask, **kw)
+    assert out.dtype == out_dtype
+    assert_o_close(out, want_o, str(case))
+    assert_lse_close(lse, want_l, str(case))
+
+
+def test_prefill_d512_workload_full_size_sampled():
+    """The timed D = 512 prefill workload, in its timed launch configuration."""
+    w = WORKLOADS["prefill_d512_g16_4k"]
+    q, k, v = make_workload_inputs(w, seed=0)
+    out, lse = ga.prefill(q.cuda(), k.cuda(), v.cuda(), causal=w.causal, q_offset=w.q_offset, scale=w.scale)
+    torch.cuda.synchronize()
+    assert ga.last_status() == ga.ATTN_OK
+    rows = sample_rows(w, 40, seed=31)
+    got_o, got_l = gather_rows(out, lse, rows)
+    want_o, want_l = oracle_rows_by_batch(q, k, v, rows, scale=w.scale, causal=w.causal, q_offset=w.q_offset)
+    assert_o_close(got_o, want_o, w.name)
+    assert_lse_close(got_l, want_l, w.name)
