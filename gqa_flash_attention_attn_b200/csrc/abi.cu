@@ -22,6 +22,7 @@ __device__ int g_attn_status = 0;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per pipeline wait
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr size_t kTwoCtaSmemLimit = 115712;  // two CTAs per SM
+constexpr size_t kOneCtaSmemLimit = 232448;  // the most one CTA may have
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -151,14 +152,16 @@ int make_ext(const attn_options* opt, int Hq, int Sq, int Skv, int q_offset, int
 }
 
 // Prefill at D = 512: the split-KV kernel with one split, query rows cut into
-// chunks of 32 / g positions per CTA (its TMEM holds 2 S^T buffers and
-// O^T for <= 32 rows at D = 512), writing the final O and LSE directly.
+// chunks of 80 / g positions per CTA, writing the final O and LSE directly.
+// 80 rows fill TMEM (2 S^T buffers + O^T: 6 x 80 of 512 columns), so a CTA
+// takes a whole SM (its shared memory is sized past half of it); every K/V
+// tile a CTA streams from L2 then serves up to 80 query rows.
 int prefill_wide(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv, int Sq,
                  int Skv, int D, int q_offset, int causal, float scale, int out_dtype, const gqa::LogitExt& ext,
                  bool ext_on, void* stream) {
   const int g = Hq / Hkv;
   if (g > 32) return ATTN_ERR_UNSUPPORTED;
-  const int qchunk = std::min(32 / g, Sq);
+  const int qchunk = std::min(80 / g, Sq);
   const int nqc = (Sq + qchunk - 1) / qchunk;
   if ((long long)B * Hkv * nqc > 65535) return ATTN_ERR_UNSUPPORTED;   // grid rows
   gqa::DecodeParams p{};
@@ -175,13 +178,16 @@ int prefill_wide(const void* q, const void* k, const void* v, void* out, float* 
   p.chunk = Skv;
   p.group = 1;
   p.obuf = 1;
-  p.mask_rows = (ext.mask != nullptr && aligned(ext.mask, 16) && ext.mask_sb % 8 == 0 && ext.mask_sr % 8 == 0)
+  p.mask_rows = (ext.mask != nullptr && qchunk <= 32 && aligned(ext.mask, 16) && ext.mask_sb % 8 == 0 &&
+                 ext.mask_sr % 8 == 0)
                     ? qchunk
                     : 0;
+  // one CTA per SM: at least half of the shared memory, at most what fits
   int nbuf = 2;
   while (nbuf < gqa::decode_max_nbuf() &&
-         gqa::decode_smem_bytes(D, p.RP, nbuf + 1, p.mask_rows, false) <= kTwoCtaSmemLimit)
+         gqa::decode_smem_bytes(D, p.RP, nbuf + 1, p.mask_rows, false) <= kOneCtaSmemLimit)
     ++nbuf;
+  if (gqa::decode_smem_bytes(D, p.RP, nbuf, p.mask_rows, false) > kOneCtaSmemLimit) return ATTN_ERR_UNSUPPORTED;
   p.nbuf = nbuf;
   p.c2 = scale * kLog2e;
   p.timeout_ns = kWaitLimitNs;

@@ -70,7 +70,7 @@ typedef enum { ATTN_BF16 = 0, ATTN_F32 = 1, ATTN_FP8_E4M3 = 2 } attn_dtype;
  *
  *   D          64, 128, 256 or 512 (else ATTN_ERR_UNSUPPORTED).  D = 512 runs the
  *              split-KV kernel with one split and the query rows cut into
- *              chunks of 32 / (Hq/Hkv) positions per CTA, writing O and LSE
+ *              chunks of 80 / (Hq/Hkv) positions per CTA, writing O and LSE
  *              directly; it needs Hq/Hkv <= 32 (else ATTN_ERR_UNSUPPORTED)
  *   scale      > 0 and finite (else ATTN_ERR_INVALID_ARG)
  *   causal     0 or 1; q_offset >= 0
