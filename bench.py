@@ -164,8 +164,9 @@ def make_runner(ga, w, device):
     """Device-resident inputs/outputs and a closure that launches one step.
     Returns (step_fn, n_kernels_per_step, events_split) where the closure
     records optional inner events between the split and the merge."""
-    from gqa_flash_attention_attn_b200.inputs import make_fp8_kv, make_mask, make_paged, make_qkv, make_sinks
-    q, k, v = make_qkv(w.B, w.Hq, w.Hkv, w.Sq, w.Skv, w.D, seed=0, device=device)
+    from gqa_flash_attention_attn_b200.inputs import (make_fp8_kv, make_mask, make_paged, make_sinks,
+                                                      make_workload_inputs)
+    q, k, v = make_workload_inputs(w, seed=0, device=device)
     bt = None
     scales = {}
     if w.kv_dtype == "fp8":
@@ -175,21 +176,25 @@ def make_runner(ga, w, device):
         kc, vc, bt = make_paged(k.cpu(), v.cpu(), w.page_size, seed=0)
         k, v, bt = kc.to(device), vc.to(device), bt.to(device)
     odt = torch.float32 if w.out_dtype == "f32" else torch.bfloat16
-    out = torch.empty((w.B, w.Sq, w.Hq, w.D), dtype=odt, device=device)
+    out = torch.empty((w.B, w.Sq, w.Hq, w.dv), dtype=odt, device=device)
     lse = torch.empty((w.B, w.Hq, w.Sq), dtype=torch.float32, device=device)
     sinks = make_sinks(w.Hq, seed=0).to(device) if w.sinks else None
     mask = make_mask(w.mask_batch, w.Sq, w.Skv, seed=0).to(device) if w.mask_batch else None
     terms = dict(softcap=w.softcap, alibi_max_bias=w.alibi_max_bias, window=w.window, mask=mask)
     if w.kind == "prefill":
         def step(mid=None):
-            ga.prefill(q, k, v, causal=w.causal, q_offset=w.q_offset, scale=w.scale, out=out, lse=lse,
-                       sinks=sinks, **terms)
+            if w.dv == w.D:
+                ga.prefill(q, k, v, causal=w.causal, q_offset=w.q_offset, scale=w.scale, out=out, lse=lse,
+                           sinks=sinks, **terms)
+            else:
+                ga.prefill_kv(q, k, v, causal=w.causal, q_offset=w.q_offset, scale=w.scale, out=out, lse=lse,
+                              sinks=sinks, **terms)
         return step, 1, (q, k, v, out, lse)
-    po = torch.empty((w.num_splits, w.B, w.Sq, w.Hq, w.D), dtype=torch.float32, device=device)
+    po = torch.empty((w.num_splits, w.B, w.Sq, w.Hq, w.dv), dtype=torch.float32, device=device)
     pl = torch.empty((w.num_splits, w.B, w.Hq, w.Sq), dtype=torch.float32, device=device)
 
     def step(mid=None):
-        if bt is None and not scales:
+        if bt is None and not scales and w.dv == w.D:
             ga.decode_split(q, k, v, w.num_splits, causal=w.causal, q_offset=w.q_offset, scale=w.scale,
                             partial_out=po, partial_lse=pl, **terms)
         else:
@@ -253,14 +258,15 @@ def time_e2e(ga, w, steps, warmup, dist_on, device):
     buffered on the device, uploads on one stream, kernels on another,
     downloads on a third, so step i's download overlaps step i+1's upload
     (PCIe is full duplex) and the kernels overlap both."""
-    from gqa_flash_attention_attn_b200.inputs import make_qkv
-    q, k, v = make_qkv(w.B, w.Hq, w.Hkv, w.Sq, w.Skv, w.D, seed=0)
-    hq, hk, hv = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    from gqa_flash_attention_attn_b200.inputs import make_workload_inputs
+    q, k, v = make_workload_inputs(w, seed=0)
+    # a V that is a view of K travels inside K
+    host_in = [t.pin_memory() for t in ((q, k) if w.v_of_k else (q, k, v))]
     odt = torch.float32 if w.out_dtype == "f32" else torch.bfloat16
-    ho = [torch.empty((w.B, w.Sq, w.Hq, w.D), dtype=odt).pin_memory() for _ in range(2)]
+    ho = [torch.empty((w.B, w.Sq, w.Hq, w.dv), dtype=odt).pin_memory() for _ in range(2)]
     hl = [torch.empty((w.B, w.Hq, w.Sq), dtype=torch.float32).pin_memory() for _ in range(2)]
-    dev_in = [[torch.empty_like(t, device=device) for t in (q, k, v)] for _ in range(2)]
-    dev_out = [torch.empty((w.B, w.Sq, w.Hq, w.D), dtype=odt, device=device) for _ in range(2)]
+    dev_in = [[torch.empty_like(t, device=device) for t in host_in] for _ in range(2)]
+    dev_out = [torch.empty((w.B, w.Sq, w.Hq, w.dv), dtype=odt, device=device) for _ in range(2)]
     dev_lse = [torch.empty((w.B, w.Hq, w.Sq), dtype=torch.float32, device=device) for _ in range(2)]
     s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
     s_comp = torch.cuda.current_stream(device)
@@ -273,20 +279,20 @@ def time_e2e(ga, w, steps, warmup, dist_on, device):
         with torch.cuda.stream(s_in):
             if state["in_free"][b] is not None:
                 s_in.wait_event(state["in_free"][b])
-            for dst, src in zip(dev_in[b], (hq, hk, hv)):
+            for dst, src in zip(dev_in[b], host_in):
                 dst.copy_(src, non_blocking=True)
             uploaded = ev()
             uploaded.record(s_in)
         s_comp.wait_event(uploaded)
         if state["out_free"][b] is not None:
             s_comp.wait_event(state["out_free"][b])      # step i-2's download of out[b] is done
-        dq, dk, dv = dev_in[b]
+        dq, dk = dev_in[b][0], dev_in[b][1]
+        dv = dk[..., :w.dv] if w.v_of_k else dev_in[b][2]
+        kw = dict(causal=w.causal, q_offset=w.q_offset, scale=w.scale, out=dev_out[b], lse=dev_lse[b])
         if w.kind == "prefill":
-            ga.prefill(dq, dk, dv, causal=w.causal, q_offset=w.q_offset, scale=w.scale, out=dev_out[b],
-                       lse=dev_lse[b])
+            (ga.prefill if w.dv == w.D else ga.prefill_kv)(dq, dk, dv, **kw)
         else:
-            ga.decode(dq, dk, dv, w.num_splits, causal=w.causal, q_offset=w.q_offset, scale=w.scale,
-                      out=dev_out[b], lse=dev_lse[b])
+            (ga.decode if w.dv == w.D else ga.decode_kv)(dq, dk, dv, w.num_splits, **kw)
         computed = ev()
         computed.record(s_comp)
         state["in_free"][b] = computed
@@ -314,7 +320,7 @@ def time_e2e(ga, w, steps, warmup, dist_on, device):
     torch.cuda.synchronize()
     barrier(dist_on)
     ms = max_over_ranks(start.elapsed_time(end) / steps, dist_on, device)
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
     d2h = ho[0].numel() * ho[0].element_size() + hl[0].numel() * hl[0].element_size()
     return ms, h2d, d2h
 
@@ -342,8 +348,8 @@ def cpu_baseline(w, seconds):
         t0 = time.perf_counter()
         oracle.attention_rows(qd, kd, vd, rows, scale=w.scale, causal=w.causal, q_offset=w.q_offset)
         dt = time.perf_counter() - t0
-        flops = sum(4 * w.D * visible(s) for _, _, s in rows)
-        kv_bytes = sum(2 * 2 * w.D * visible(s) for _, _, s in rows)  # K and V rows each row reads
+        flops = sum(2 * (w.D + w.dv) * visible(s) for _, _, s in rows)
+        kv_bytes = sum(2 * (w.D + w.dv) * visible(s) for _, _, s in rows)  # K and V rows each row reads
         return dt, flops, kv_bytes, len(rows)
 
     dt, _, _, _ = run(256, 11)
@@ -457,7 +463,7 @@ def run_reference(args):
 
     def one(n, seed):
         rows = sample_rows(w, n, seed=seed, include_edges=False)
-        fl = sum(4 * w.D * min(w.Skv, w.q_offset + s + 1) for _, _, s in rows)
+        fl = sum(2 * (w.D + w.dv) * min(w.Skv, w.q_offset + s + 1) for _, _, s in rows)
         t0 = time.perf_counter()
         oracle.attention_rows(qd, kd, vd, rows, scale=w.scale, causal=w.causal, q_offset=w.q_offset)
         return time.perf_counter() - t0, fl

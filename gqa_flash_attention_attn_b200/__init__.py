@@ -24,7 +24,7 @@ __all__ = [
     "merge", "decode", "decode_workspace_bytes", "last_status", "status_string",
     "watchdog_selftest", "version", "ATTN_OK", "ATTN_ERR_INVALID_ARG", "ATTN_ERR_UNSUPPORTED",
     "ATTN_ERR_ALIGNMENT", "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT", "ATTN_ERR_TOO_LARGE", "decode_noalloc",
-    "AttnOptions", "AttnKVView", "decode_split_kv", "decode_kv", "ATTN_FP8_E4M3",
+    "AttnOptions", "AttnKVView", "decode_split_kv", "decode_kv", "ATTN_FP8_E4M3", "prefill_kv",
 ]
 
 ATTN_OK = 0
@@ -58,6 +58,7 @@ _SIGNATURES = {
     "attn_decode_split_ex": (_i, [_vp, _vp, _vp, _vp, _vp] + [_i] * 8 + [_f, _i, _vp, _vp]),
     "attn_merge_ex": (_i, [_vp, _vp, _vp, _vp] + [_i] * 6 + [_vp, _vp]),
     "attn_decode_split_kv": (_i, [_vp, _vp, _vp, _vp] + [_i] * 8 + [_f, _i, _vp, _vp]),
+    "attn_prefill_kv": (_i, [_vp, _vp, _vp, _vp] + [_i] * 8 + [_f, _i, _vp, _vp]),
 }
 
 
@@ -148,7 +149,9 @@ class AttnKVView(ctypes.Structure):
                 ("stride_token", ctypes.c_longlong), ("stride_head", ctypes.c_longlong),
                 ("block_table", ctypes.c_void_p), ("max_pages", ctypes.c_int), ("page_size", ctypes.c_int),
                 ("num_pages", ctypes.c_int), ("seq_lens", ctypes.c_void_p), ("kv_dtype", ctypes.c_int),
-                ("k_scale", ctypes.c_void_p), ("v_scale", ctypes.c_void_p)]
+                ("k_scale", ctypes.c_void_p), ("v_scale", ctypes.c_void_p), ("head_dim_v", ctypes.c_int),
+                ("v_stride_seq", ctypes.c_longlong), ("v_stride_token", ctypes.c_longlong),
+                ("v_stride_head", ctypes.c_longlong)]
 
 
 ATTN_FP8_E4M3 = 2
@@ -161,7 +164,9 @@ def _kv_view(k, v, block_table, seq_lens, k_scale=None, v_scale=None):
     Unpaged: k, v are [B, Skv, Hkv, D] views.  Paged: k, v are
     [num_pages, page_size, Hkv, D] views and block_table is int32 [B, max_pages].
     bf16 K/V, or fp8 e4m3 codes (uint8 or float8_e4m3fn) with fp32 per-head
-    k_scale and v_scale [Hkv]."""
+    k_scale and v_scale [Hkv].  v may have fewer columns than k (Dv < D: the
+    head sizes (576, 512), (320, 256), (192, 128)), e.g. v = k[..., :Dv] for
+    a cache whose V is the front of K; v's strides may differ from k's."""
     fp8 = isinstance(k, torch.Tensor) and k.dtype in _FP8_DTYPES
     for t, n in ((k, "k"), (v, "v")):
         ok_dtype = t.dtype in _FP8_DTYPES if fp8 else t.dtype == torch.bfloat16
@@ -169,10 +174,12 @@ def _kv_view(k, v, block_table, seq_lens, k_scale=None, v_scale=None):
             raise ValueError(f"{n} must be a 4-D CUDA tensor, bf16 or fp8 e4m3 like the other")
         if t.stride(3) != 1:
             raise ValueError(f"{n} must be contiguous in its last dimension")
-    if k.shape != v.shape or k.stride() != v.stride():
-        raise ValueError("k and v must have the same shape and strides")
+    if k.shape[:3] != v.shape[:3]:
+        raise ValueError("k and v must have the same leading shape")
     view = AttnKVView(k.data_ptr(), v.data_ptr(), k.stride(0), k.stride(1), k.stride(2), None, 0, 0, 0, None,
-                      0, None, None)
+                      0, None, None, 0 if v.shape[3] == k.shape[3] else v.shape[3])
+    if v.stride()[:3] != k.stride()[:3]:
+        view.v_stride_seq, view.v_stride_token, view.v_stride_head = v.stride(0), v.stride(1), v.stride(2)
     if fp8:
         for sc, n in ((k_scale, "k_scale"), (v_scale, "v_scale")):
             _need(sc, n, torch.float32, 1)
@@ -338,6 +345,7 @@ def decode_split_kv(q, k, v, num_splits, *, block_table=None, seq_lens=None, cau
     block_table int32 [B, max_pages] maps logical to physical pages.
     fp8 e4m3 K/V: k, v as uint8 codes (or float8_e4m3fn) with fp32 k_scale,
     v_scale [Hkv]: K = code * k_scale[kvh], V = code * v_scale[kvh].
+    v may be Dv < D columns wide (see _kv_view); the partials are then Dv wide.
     seq_lens (int32 [B], optional): keys per sequence; the query rows then sit
     at the last Sq positions of each sequence and q_offset is ignored."""
     _need(q, "q", torch.bfloat16, 4)
@@ -352,8 +360,9 @@ def decode_split_kv(q, k, v, num_splits, *, block_table=None, seq_lens=None, cau
         raise ValueError("block_table must have B rows")
     if scale is None:
         scale = 1.0 / math.sqrt(D)
+    Dv = v.shape[3]
     if partial_out is None:
-        partial_out = torch.empty((num_splits, B, Sq, Hq, D), dtype=torch.float32, device=q.device)
+        partial_out = torch.empty((num_splits, B, Sq, Hq, Dv), dtype=torch.float32, device=q.device)
     if partial_lse is None:
         partial_lse = torch.empty((num_splits, B, Hq, Sq), dtype=torch.float32, device=q.device)
     opt = _options(softcap, alibi_max_bias, None, window, Hq, mask, B, Sq, Skv)
@@ -377,6 +386,41 @@ def decode_kv(q, k, v, num_splits, *, block_table=None, seq_lens=None, causal=Tr
                              softcap=softcap, alibi_max_bias=alibi_max_bias, window=window, mask=mask,
                              k_scale=k_scale, v_scale=v_scale)
     return merge(po, pl, out_dtype=out_dtype, out=out, lse=lse, stream=stream, sinks=sinks)
+
+
+def prefill_kv(q, k, v, *, block_table=None, seq_lens=None, causal=True, q_offset=0, scale=None,
+               out_dtype=torch.bfloat16, out=None, lse=None, return_lse=True, stream=None, softcap=0.0,
+               alibi_max_bias=0.0, sinks=None, window=0, mask=None, k_scale=None, v_scale=None):
+    """prefill() over a strided or paged K/V cache, fp8 codes, lengths per
+    sequence or Dv < D (k, v, block_table, seq_lens, k_scale, v_scale as in
+    decode_split_kv).  One launch; out is [B, Sq, Hq, Dv]."""
+    _need(q, "q", torch.bfloat16, 4)
+    B, Sq, Hq, D = q.shape
+    view, Skv = _kv_view(k, v, block_table, seq_lens, k_scale, v_scale)
+    Hkv = k.shape[2]
+    if k.shape[3] != D:
+        raise ValueError("k head size does not match q")
+    if block_table is None and k.shape[0] != B:
+        raise ValueError("unpaged k/v must have B sequences")
+    if block_table is not None and block_table.shape[0] != B:
+        raise ValueError("block_table must have B rows")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    Dv = v.shape[3]
+    if out is None:
+        out = torch.empty((B, Sq, Hq, Dv), dtype=out_dtype, device=q.device)
+    else:
+        _need(out, "out", out.dtype, 4)
+    if out.dtype not in _OUT_CODES:
+        raise ValueError("out must be bf16 or fp32")
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    opt = _options(softcap, alibi_max_bias, sinks, window, Hq, mask, B, Sq, Skv)
+    st = library().attn_prefill_kv(_ptr(q), ctypes.byref(view), _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Skv, D,
+                                   int(q_offset), int(bool(causal)), float(scale), _OUT_CODES[out.dtype],
+                                   None if opt is None else ctypes.byref(opt), _stream_ptr(stream))
+    _check("attn_prefill_kv", st)
+    return out, lse
 
 
 def last_status(stream=None) -> int:

@@ -151,17 +151,101 @@ int make_ext(const attn_options* opt, int Hq, int Sq, int Skv, int q_offset, int
   return ATTN_OK;
 }
 
-// Prefill at D = 512: the split-KV kernel with one split, query rows cut into
+// Checks of a K/V view before any CUDA call: strides, paging, element type.
+// *fp8 tells the element type.
+int check_view(const attn_kv_view* kv, int Skv, bool* fp8) {
+  const bool own_v = kv->v_stride_seq != 0 || kv->v_stride_token != 0 || kv->v_stride_head != 0;
+  const long long strides[6] = {kv->stride_head,  kv->stride_token, kv->stride_seq,
+                                own_v ? kv->v_stride_head : kv->stride_head,
+                                own_v ? kv->v_stride_token : kv->stride_token,
+                                own_v ? kv->v_stride_seq : kv->stride_seq};
+  for (long long x : strides)
+    if (x < 1 || x >= (1LL << 37)) return ATTN_ERR_INVALID_ARG;
+  if (kv->block_table != nullptr) {
+    const int ps = kv->page_size;
+    if (!(ps == 16 || ps == 32 || ps == 64 || (ps >= 128 && ps % 128 == 0))) return ATTN_ERR_INVALID_ARG;
+    if (kv->max_pages < 1 || kv->num_pages < 1) return ATTN_ERR_INVALID_ARG;
+    if ((long long)kv->max_pages * ps != Skv) return ATTN_ERR_INVALID_ARG;
+    if (!aligned(kv->block_table, 4)) return ATTN_ERR_ALIGNMENT;
+  }
+  if (kv->seq_lens != nullptr && !aligned(kv->seq_lens, 4)) return ATTN_ERR_ALIGNMENT;
+  if (kv->kv_dtype != ATTN_BF16 && kv->kv_dtype != ATTN_FP8_E4M3) return ATTN_ERR_INVALID_ARG;
+  *fp8 = kv->kv_dtype == ATTN_FP8_E4M3;
+  if (*fp8 && (kv->k_scale == nullptr || kv->v_scale == nullptr || !aligned(kv->k_scale, 4) ||
+               !aligned(kv->v_scale, 4)))
+    return ATTN_ERR_INVALID_ARG;
+  if (kv->head_dim_v < 0) return ATTN_ERR_INVALID_ARG;
+  if (kv->k == nullptr || kv->v == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(kv->k, 16) || !aligned(kv->v, 16)) return ATTN_ERR_ALIGNMENT;
+  for (long long x : strides)
+    if (x % (*fp8 ? 16 : 8) != 0) return ATTN_ERR_ALIGNMENT;
+  return ATTN_OK;
+}
+
+struct ViewStrides {
+  uint64_t head, token, seq;
+};
+ViewStrides k_strides(const attn_kv_view* kv) {
+  return {(uint64_t)kv->stride_head, (uint64_t)kv->stride_token, (uint64_t)kv->stride_seq};
+}
+// V's strides: its own when any is set, else K's
+ViewStrides v_strides(const attn_kv_view* kv) {
+  if (kv->v_stride_seq != 0 || kv->v_stride_token != 0 || kv->v_stride_head != 0)
+    return {(uint64_t)kv->v_stride_head, (uint64_t)kv->v_stride_token, (uint64_t)kv->v_stride_seq};
+  return k_strides(kv);
+}
+
+// Tensor maps of a K/V view for the split-KV kernel: K (D columns) and V (Dv
+// columns) over (d, kvh, key, sequence), or (d, kvh, row in page, page).
+bool view_maps(const attn_kv_view* kv, int D, int Dv, int Hkv, int Skv, int B, bool fp8, CUtensorMap* tk,
+               CUtensorMap* tv) {
+  const bool paged = kv->block_table != nullptr;
+  const uint64_t d2 = paged ? (uint64_t)kv->page_size : (uint64_t)Skv;
+  const uint64_t d3 = paged ? (uint64_t)kv->num_pages : (uint64_t)B;
+  const uint32_t rows = paged && kv->page_size < 128 ? (uint32_t)kv->page_size : 128u;
+  const uint32_t b0 = fp8 ? 128u : 64u;   // 128-byte box rows either way
+  const ViewStrides k = k_strides(kv), v = v_strides(kv);
+  return make_map_strided(tk, kv->k, D, Hkv, d2, d3, k.head, k.token, k.seq, b0, 1, rows, 1, fp8) &&
+         make_map_strided(tv, kv->v, Dv, Hkv, d2, d3, v.head, v.token, v.seq, b0, 1, rows, 1, fp8);
+}
+
+// The view's fields in the split-KV kernel's parameters.
+void view_params(const attn_kv_view* kv, bool fp8, gqa::DecodeParams& p) {
+  const bool paged = kv->block_table != nullptr;
+  p.seq_lens = kv->seq_lens;
+  p.block_table = kv->block_table;
+  p.max_pages = paged ? kv->max_pages : 0;
+  p.page_size = paged ? kv->page_size : 0;
+  p.k_scale = fp8 ? kv->k_scale : nullptr;
+  p.v_scale = fp8 ? kv->v_scale : nullptr;
+}
+
+// Prefill through the split-KV kernel (D = 512, asymmetric head sizes,
+// paged or fp8 K/V, lengths per sequence): one split, query rows cut into
 // chunks of 80 / g positions per CTA, writing the final O and LSE directly.
-// 80 rows fill TMEM (2 S^T buffers + O^T: 6 x 80 of 512 columns), so a CTA
-// takes a whole SM (its shared memory is sized past half of it); every K/V
-// tile a CTA streams from L2 then serves up to 80 query rows.
-int prefill_wide(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv, int Sq,
-                 int Skv, int D, int q_offset, int causal, float scale, int out_dtype, const gqa::LogitExt& ext,
-                 bool ext_on, void* stream) {
+// 80 rows fill TMEM (2 S^T buffers + O^T: 6 x 80 of 512 columns at Dv = 512),
+// so a CTA takes a whole SM (its shared memory is sized past half of it);
+// every K/V tile a CTA streams from L2 then serves up to 80 query rows.
+int prefill_wide(const void* q, const attn_kv_view* kv, bool fp8, void* out, float* lse, int B, int Hq, int Hkv,
+                 int Sq, int Skv, int D, int Dv, int q_offset, int causal, float scale, int out_dtype,
+                 const gqa::LogitExt& ext, bool ext_on, void* stream) {
   const int g = Hq / Hkv;
   if (g > 32) return ATTN_ERR_UNSUPPORTED;
-  const int qchunk = std::min(80 / g, Sq);
+  if (!gqa::decode_dims_supported(D, Dv, fp8)) return ATTN_ERR_UNSUPPORTED;
+  // rows per CTA: TMEM holds 2 S^T buffers and O^T, (2 + Dv/128) x RP of 512 columns
+  const int max_rows = std::min(128, (512 / (2 + Dv / 128)) / 16 * 16);
+  int qchunk = std::max(1, std::min(max_rows / g, Sq));
+  // fewer rows when two K/V slots and the Q, P buffers of that many rows do
+  // not fit one CTA's shared memory (fp8 at D = 512: two more Q planes)
+  auto mrows_of = [&](int qc) {
+    return (ext.mask != nullptr && qc <= 32 && aligned(ext.mask, 16) && ext.mask_sb % 8 == 0 &&
+            ext.mask_sr % 8 == 0)
+               ? qc
+               : 0;
+  };
+  auto rp_of = [&](int qc) { return (g * qc + 15) / 16 * 16; };
+  while (qchunk > 1 && gqa::decode_smem_bytes(D, rp_of(qchunk), 2, mrows_of(qchunk), fp8) > kOneCtaSmemLimit)
+    --qchunk;
   const int nqc = (Sq + qchunk - 1) / qchunk;
   if ((long long)B * Hkv * nqc > 65535) return ATTN_ERR_UNSUPPORTED;   // grid rows
   gqa::DecodeParams p{};
@@ -178,36 +262,85 @@ int prefill_wide(const void* q, const void* k, const void* v, void* out, float* 
   p.chunk = Skv;
   p.group = 1;
   p.obuf = 1;
-  p.mask_rows = (ext.mask != nullptr && qchunk <= 32 && aligned(ext.mask, 16) && ext.mask_sb % 8 == 0 &&
-                 ext.mask_sr % 8 == 0)
-                    ? qchunk
-                    : 0;
+  p.mask_rows = mrows_of(qchunk);
   // one CTA per SM: at least half of the shared memory, at most what fits
   int nbuf = 2;
   while (nbuf < gqa::decode_max_nbuf() &&
-         gqa::decode_smem_bytes(D, p.RP, nbuf + 1, p.mask_rows, false) <= kOneCtaSmemLimit)
+         gqa::decode_smem_bytes(D, p.RP, nbuf + 1, p.mask_rows, fp8) <= kOneCtaSmemLimit)
     ++nbuf;
-  if (gqa::decode_smem_bytes(D, p.RP, nbuf, p.mask_rows, false) > kOneCtaSmemLimit) return ATTN_ERR_UNSUPPORTED;
+  if (gqa::decode_smem_bytes(D, p.RP, nbuf, p.mask_rows, fp8) > kOneCtaSmemLimit) return ATTN_ERR_UNSUPPORTED;
   p.nbuf = nbuf;
   p.c2 = scale * kLog2e;
   p.timeout_ns = kWaitLimitNs;
   p.ext = ext;
+  view_params(kv, fp8, p);
   p.status = status_ptr();
   if (p.status == nullptr) return cuda_fail();
   CUtensorMap tq, tk, tv;
   if (!make_map(&tq, q, D, Hq, Sq, B, 64, (uint32_t)g, (uint32_t)qchunk, 1)) return cuda_fail();
-  if (!make_map(&tk, k, D, Hkv, Skv, B, 64, 1, 128, 1)) return cuda_fail();
-  if (!make_map(&tv, v, D, Hkv, Skv, B, 64, 1, 128, 1)) return cuda_fail();
-  return gqa::launch_decode_split(D, ext_on, false, tq, tk, tv, p, static_cast<cudaStream_t>(stream)) == 0
+  if (!view_maps(kv, D, Dv, Hkv, Skv, B, fp8, &tk, &tv)) return cuda_fail();
+  return gqa::launch_decode_split(D, Dv, ext_on, fp8, tq, tk, tv, p, static_cast<cudaStream_t>(stream)) == 0
              ? ATTN_OK
              : ATTN_ERR_CUDA;
+}
+
+// The prefill kernel over given K/V tensor maps (D 64, 128 or 256).
+int prefill_fast(const void* q, const CUtensorMap& tk, const CUtensorMap& tv, void* out, float* lse, int B, int Hq,
+                 int Hkv, int Sq, int Skv, int D, int q_offset, int causal, float scale, int out_dtype,
+                 const gqa::LogitExt& ext, bool ext_on, void* stream) {
+  const int nslot = gqa::prefill_slots(D);
+  const int g = Hq / Hkv;
+  gqa::PrefillParams p{};
+  p.out = out;
+  p.lse = lse;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Sq = Sq; p.Skv = Skv;
+  p.q_offset = q_offset; p.causal = causal; p.out_f32 = (out_dtype == ATTN_F32);
+  p.g = g;
+  p.units_per_kvh = (g + nslot - 1) / nslot;
+  p.n_qt = (Sq + 127) / 128;
+  p.c2 = scale * kLog2e;
+  p.timeout_ns = kWaitLimitNs;
+  p.ext = ext;
+  if ((long long)p.n_qt * B * Hkv * p.units_per_kvh > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+
+  p.status = status_ptr();
+  if (p.status == nullptr) return cuda_fail();
+  p.num_ctas = sm_count();
+  if (p.num_ctas <= 0) return cuda_fail();
+  CUtensorMap tq;
+  if (!make_map(&tq, q, D, Hq, Sq, B, 64, 1, 128, 1)) return cuda_fail();
+  // the additive mask staged by TMA: 16-byte aligned rows, and every head
+  // slot of a CTA visits every tile (one slot, or an even group size)
+  CUtensorMap tm;
+  std::memset(&tm, 0, sizeof(tm));
+  if (ext.mask != nullptr && aligned(ext.mask, 16) && ext.mask_sr % 8 == 0 && ext.mask_sb % 8 == 0 &&
+      ext.mask_sr > 0 && (gqa::prefill_slots(D) == 1 || g % 2 == 0)) {
+    const uint64_t bm = ext.mask_sb != 0 ? (uint64_t)B : 1u;
+    const uint64_t s2 = ext.mask_sb != 0 ? (uint64_t)ext.mask_sb : (uint64_t)Sq * ext.mask_sr;
+    if (!make_map_strided(&tm, ext.mask, Skv, Sq, bm, 1, (uint64_t)ext.mask_sr, s2, s2 * bm, 64, 128, 1, 1))
+      return cuda_fail();
+    p.mask_tma = 1;
+  }
+  return gqa::launch_prefill(D, ext_on, tq, tk, tv, tm, p, static_cast<cudaStream_t>(stream)) == 0 ? ATTN_OK
+                                                                                          : ATTN_ERR_CUDA;
+}
+
+// The contiguous [B, Skv, Hkv, D] view of k and v.
+attn_kv_view contiguous_view(const void* k, const void* v, int Skv, int Hkv, int D) {
+  attn_kv_view kv{};
+  kv.k = k;
+  kv.v = v;
+  kv.stride_head = D;
+  kv.stride_token = (long long)Hkv * D;
+  kv.stride_seq = (long long)Skv * Hkv * D;
+  return kv;
 }
 
 }  // namespace
 
 extern "C" {
 
-int attn_version(void) { return 0x000300; }
+int attn_version(void) { return 0x000400; }
 
 const char* attn_status_string(int status) {
   switch (status) {
@@ -242,47 +375,49 @@ int attn_prefill_ex(const void* q, const void* k, const void* v, void* out, floa
   if (D != 64 && D != 128 && D != 256 && D != 512) return ATTN_ERR_UNSUPPORTED;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16)) return ATTN_ERR_ALIGNMENT;
   if (lse != nullptr && !aligned(lse, 4)) return ATTN_ERR_ALIGNMENT;
-  if (D == 512)
-    return prefill_wide(q, k, v, out, lse, B, Hq, Hkv, Sq, Skv, D, q_offset, causal, scale, out_dtype, ext, ext_on,
-                        stream);
-
-  const int nslot = gqa::prefill_slots(D);
-  const int g = Hq / Hkv;
-  gqa::PrefillParams p{};
-  p.out = out;
-  p.lse = lse;
-  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Sq = Sq; p.Skv = Skv;
-  p.q_offset = q_offset; p.causal = causal; p.out_f32 = (out_dtype == ATTN_F32);
-  p.g = g;
-  p.units_per_kvh = (g + nslot - 1) / nslot;
-  p.n_qt = (Sq + 127) / 128;
-  p.c2 = scale * kLog2e;
-  p.timeout_ns = kWaitLimitNs;
-  p.ext = ext;
-  if ((long long)p.n_qt * B * Hkv * p.units_per_kvh > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
-
-  p.status = status_ptr();
-  if (p.status == nullptr) return cuda_fail();
-  p.num_ctas = sm_count();
-  if (p.num_ctas <= 0) return cuda_fail();
-  CUtensorMap tq, tk, tv;
-  if (!make_map(&tq, q, D, Hq, Sq, B, 64, 1, 128, 1)) return cuda_fail();
+  if (D == 512) {
+    const attn_kv_view kv = contiguous_view(k, v, Skv, Hkv, D);
+    return prefill_wide(q, &kv, false, out, lse, B, Hq, Hkv, Sq, Skv, D, D, q_offset, causal, scale, out_dtype, ext,
+                        ext_on, stream);
+  }
+  CUtensorMap tk, tv;
   if (!make_map(&tk, k, D, Hkv, Skv, B, 64, 1, 128, 1)) return cuda_fail();
   if (!make_map(&tv, v, D, Hkv, Skv, B, 64, 1, 128, 1)) return cuda_fail();
-  // the additive mask staged by TMA: 16-byte aligned rows, and every head
-  // slot of a CTA visits every tile (one slot, or an even group size)
-  CUtensorMap tm;
-  std::memset(&tm, 0, sizeof(tm));
-  if (ext.mask != nullptr && aligned(ext.mask, 16) && ext.mask_sr % 8 == 0 && ext.mask_sb % 8 == 0 &&
-      ext.mask_sr > 0 && (gqa::prefill_slots(D) == 1 || g % 2 == 0)) {
-    const uint64_t bm = ext.mask_sb != 0 ? (uint64_t)B : 1u;
-    const uint64_t s2 = ext.mask_sb != 0 ? (uint64_t)ext.mask_sb : (uint64_t)Sq * ext.mask_sr;
-    if (!make_map_strided(&tm, ext.mask, Skv, Sq, bm, 1, (uint64_t)ext.mask_sr, s2, s2 * bm, 64, 128, 1, 1))
-      return cuda_fail();
-    p.mask_tma = 1;
-  }
-  return gqa::launch_prefill(D, ext_on, tq, tk, tv, tm, p, static_cast<cudaStream_t>(stream)) == 0 ? ATTN_OK
-                                                                                          : ATTN_ERR_CUDA;
+  return prefill_fast(q, tk, tv, out, lse, B, Hq, Hkv, Sq, Skv, D, q_offset, causal, scale, out_dtype, ext, ext_on,
+                      stream);
+}
+
+int attn_prefill_kv(const void* q, const attn_kv_view* kv, void* out, float* lse, int B, int Hq, int Hkv, int Sq,
+                    int Skv, int D, int q_offset, int causal, float scale, int out_dtype, const attn_options* opt,
+                    void* stream) {
+  if (kv == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (kv->seq_lens != nullptr) q_offset = 0;   // rows sit at len_b - Sq + s
+  int st = check_common(q, kv->k, kv->v, B, Hq, Hkv, Sq, Skv, D, q_offset, causal, scale);
+  if (st != ATTN_OK) return st;
+  gqa::LogitExt ext;
+  bool ext_on;
+  st = make_ext(opt, Hq, Sq, Skv, q_offset, causal, scale, true, &ext, &ext_on);
+  if (st != ATTN_OK) return st;
+  if (out == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (out_dtype != ATTN_BF16 && out_dtype != ATTN_F32) return ATTN_ERR_INVALID_ARG;
+  bool fp8 = false;
+  st = check_view(kv, Skv, &fp8);
+  if (st != ATTN_OK) return st;
+  const int Dv = kv->head_dim_v != 0 ? kv->head_dim_v : D;
+  const bool fast = D == Dv && (D == 64 || D == 128 || D == 256) && !fp8 && kv->block_table == nullptr &&
+                    kv->seq_lens == nullptr;
+  if (!fast && !gqa::decode_dims_supported(D, Dv, fp8)) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(out, 16)) return ATTN_ERR_ALIGNMENT;
+  if (lse != nullptr && !aligned(lse, 4)) return ATTN_ERR_ALIGNMENT;
+  if (!fast)
+    return prefill_wide(q, kv, fp8, out, lse, B, Hq, Hkv, Sq, Skv, D, Dv, q_offset, causal, scale, out_dtype, ext,
+                        ext_on, stream);
+  CUtensorMap tk, tv;
+  const ViewStrides ks = k_strides(kv), vs = v_strides(kv);
+  if (!make_map_strided(&tk, kv->k, D, Hkv, Skv, B, ks.head, ks.token, ks.seq, 64, 1, 128, 1)) return cuda_fail();
+  if (!make_map_strided(&tv, kv->v, D, Hkv, Skv, B, vs.head, vs.token, vs.seq, 64, 1, 128, 1)) return cuda_fail();
+  return prefill_fast(q, tk, tv, out, lse, B, Hq, Hkv, Sq, Skv, D, q_offset, causal, scale, out_dtype, ext, ext_on,
+                      stream);
 }
 
 size_t attn_decode_workspace_bytes(int B, int Hq, int Sq, int D, int num_splits) {
@@ -302,13 +437,7 @@ int attn_decode_split(const void* q, const void* k, const void* v, float* partia
 int attn_decode_split_ex(const void* q, const void* k, const void* v, float* partial_out, float* partial_lse,
                          int B, int Hq, int Hkv, int Sq, int Skv, int D, int q_offset, int causal, float scale,
                          int num_splits, const attn_options* opt, void* stream) {
-  // the contiguous [B, Skv, Hkv, D] view
-  attn_kv_view kv{};
-  kv.k = k;
-  kv.v = v;
-  kv.stride_head = D;
-  kv.stride_token = (long long)Hkv * D;
-  kv.stride_seq = (long long)Skv * Hkv * D;
+  const attn_kv_view kv = contiguous_view(k, v, Skv, Hkv, D);
   return attn_decode_split_kv(q, &kv, partial_out, partial_lse, B, Hq, Hkv, Sq, Skv, D, q_offset, causal, scale,
                               num_splits, opt, stream);
 }
@@ -317,12 +446,9 @@ int attn_decode_split_kv(const void* q, const attn_kv_view* kv, float* partial_o
                          int Hq, int Hkv, int Sq, int Skv, int D, int q_offset, int causal, float scale,
                          int num_splits, const attn_options* opt, void* stream) {
   if (kv == nullptr) return ATTN_ERR_INVALID_ARG;
-  const void* k = kv->k;
-  const void* v = kv->v;
-  const bool paged = kv->block_table != nullptr;
   // with per-sequence lengths q_offset is ignored (rows sit at len_b - Sq + s)
   if (kv->seq_lens != nullptr) q_offset = 0;
-  int st = check_common(q, k, v, B, Hq, Hkv, Sq, Skv, D, q_offset, causal, scale);
+  int st = check_common(q, kv->k, kv->v, B, Hq, Hkv, Sq, Skv, D, q_offset, causal, scale);
   if (st != ATTN_OK) return st;
   gqa::LogitExt ext;
   bool ext_on;
@@ -330,34 +456,18 @@ int attn_decode_split_kv(const void* q, const attn_kv_view* kv, float* partial_o
   if (st != ATTN_OK) return st;
   if (partial_out == nullptr || partial_lse == nullptr) return ATTN_ERR_INVALID_ARG;
   if (num_splits < 1 || num_splits > Skv || num_splits > 65535) return ATTN_ERR_INVALID_ARG;
-  if (D != 128 && D != 256 && D != 512) return ATTN_ERR_UNSUPPORTED;
+  bool fp8 = false;
+  st = check_view(kv, Skv, &fp8);
+  if (st != ATTN_OK) return st;
+  const int Dv = kv->head_dim_v != 0 ? kv->head_dim_v : D;
+  if (!gqa::decode_dims_supported(D, Dv, fp8)) return ATTN_ERR_UNSUPPORTED;
   const int g = Hq / Hkv;
   const long long R = (long long)g * Sq;
   const long long RP = (R + 15) / 16 * 16;
-  if (RP * (2 + D / 128) > 256) return ATTN_ERR_UNSUPPORTED;  // TMEM: two S^T buffers + O^T
+  if (RP * (2 + Dv / 128) > 256) return ATTN_ERR_UNSUPPORTED;  // TMEM: two S^T buffers + O^T
   if (g > 256 || Sq > 256) return ATTN_ERR_UNSUPPORTED;  // TMA box extents
   if ((long long)B * Hkv > 65535) return ATTN_ERR_INVALID_ARG;
-  // the view: strides positive, below 2^37 elements, 16-byte multiples
-  const long long strides[3] = {kv->stride_head, kv->stride_token, kv->stride_seq};
-  for (long long x : strides)
-    if (x < 1 || x >= (1LL << 37)) return ATTN_ERR_INVALID_ARG;
-  if (paged) {
-    const int ps = kv->page_size;
-    if (!(ps == 16 || ps == 32 || ps == 64 || (ps >= 128 && ps % 128 == 0))) return ATTN_ERR_INVALID_ARG;
-    if (kv->max_pages < 1 || kv->num_pages < 1) return ATTN_ERR_INVALID_ARG;
-    if ((long long)kv->max_pages * ps != Skv) return ATTN_ERR_INVALID_ARG;
-    if (!aligned(kv->block_table, 4)) return ATTN_ERR_ALIGNMENT;
-  }
-  if (kv->seq_lens != nullptr && !aligned(kv->seq_lens, 4)) return ATTN_ERR_ALIGNMENT;
-  if (kv->kv_dtype != ATTN_BF16 && kv->kv_dtype != ATTN_FP8_E4M3) return ATTN_ERR_INVALID_ARG;
-  const bool fp8 = kv->kv_dtype == ATTN_FP8_E4M3;
-  if (fp8 && (kv->k_scale == nullptr || kv->v_scale == nullptr || !aligned(kv->k_scale, 4) ||
-              !aligned(kv->v_scale, 4)))
-    return ATTN_ERR_INVALID_ARG;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(partial_out, 16))
-    return ATTN_ERR_ALIGNMENT;
-  for (long long x : strides)
-    if (x % (fp8 ? 16 : 8) != 0) return ATTN_ERR_ALIGNMENT;
+  if (!aligned(q, 16) || !aligned(partial_out, 16)) return ATTN_ERR_ALIGNMENT;
   if (!aligned(partial_lse, 4)) return ATTN_ERR_ALIGNMENT;
 
   gqa::DecodeParams p{};
@@ -374,10 +484,14 @@ int attn_decode_split_kv(const void* q, const attn_kv_view* kv, float* partial_o
                  ext.mask_sr % 8 == 0)
                     ? Sq
                     : 0;
+  // ring slots: as many as keep two CTAs per SM, or, when even two slots
+  // leave room for one CTA only, as many as that CTA can hold
+  const size_t smem_limit =
+      gqa::decode_smem_bytes(D, p.RP, 2, p.mask_rows, fp8) <= kTwoCtaSmemLimit ? kTwoCtaSmemLimit : kOneCtaSmemLimit;
   int nbuf = 2;
-  while (nbuf < gqa::decode_max_nbuf() &&
-         gqa::decode_smem_bytes(D, p.RP, nbuf + 1, p.mask_rows, fp8) <= kTwoCtaSmemLimit)
+  while (nbuf < gqa::decode_max_nbuf() && gqa::decode_smem_bytes(D, p.RP, nbuf + 1, p.mask_rows, fp8) <= smem_limit)
     ++nbuf;
+  if (gqa::decode_smem_bytes(D, p.RP, nbuf, p.mask_rows, fp8) > kOneCtaSmemLimit) return ATTN_ERR_UNSUPPORTED;
   p.nbuf = nbuf;
   // Consecutive splits per CTA: enough that the CTAs fit the resident slots
   // (two per SM when the shared memory allows) in one wave, at most 8.
@@ -391,17 +505,12 @@ int attn_decode_split_kv(const void* q, const attn_kv_view* kv, float* partial_o
     grp = std::min<long long>(std::min<long long>(grp, gqa::decode_max_group()), num_splits);
     p.group = (int)std::max<long long>(grp, 1);
     // two O^T buffers when split boundaries exist and two CTAs' TMEM still fits
-    p.obuf = (p.group > 1 && RP * (2 + 2 * (D / 128)) <= 256) ? 2 : 1;
+    p.obuf = (p.group > 1 && RP * (2 + 2 * (Dv / 128)) <= 256) ? 2 : 1;
   }
   p.c2 = scale * kLog2e;
   p.timeout_ns = kWaitLimitNs;
   p.ext = ext;
-  p.seq_lens = kv->seq_lens;
-  p.block_table = kv->block_table;
-  p.max_pages = paged ? kv->max_pages : 0;
-  p.page_size = paged ? kv->page_size : 0;
-  p.k_scale = fp8 ? kv->k_scale : nullptr;
-  p.v_scale = fp8 ? kv->v_scale : nullptr;
+  view_params(kv, fp8, p);
   p.qchunk = Sq;
   p.nqc = 1;
   p.fout = nullptr;
@@ -410,16 +519,10 @@ int attn_decode_split_kv(const void* q, const attn_kv_view* kv, float* partial_o
   if (p.status == nullptr) return cuda_fail();
   CUtensorMap tq, tk, tv;
   if (!make_map(&tq, q, D, Hq, Sq, B, 64, (uint32_t)g, (uint32_t)Sq, 1)) return cuda_fail();
-  // K/V: (d, kvh, key, sequence) unpaged, (d, kvh, row in page, page) paged
-  const uint64_t d2 = paged ? (uint64_t)kv->page_size : (uint64_t)Skv;
-  const uint64_t d3 = paged ? (uint64_t)kv->num_pages : (uint64_t)B;
-  const uint32_t rows = paged && kv->page_size < 128 ? (uint32_t)kv->page_size : 128u;
-  const uint64_t s1 = (uint64_t)kv->stride_head, s2 = (uint64_t)kv->stride_token, s3 = (uint64_t)kv->stride_seq;
-  const uint32_t b0 = fp8 ? 128u : 64u;   // 128-byte box rows either way
-  if (!make_map_strided(&tk, k, D, Hkv, d2, d3, s1, s2, s3, b0, 1, rows, 1, fp8)) return cuda_fail();
-  if (!make_map_strided(&tv, v, D, Hkv, d2, d3, s1, s2, s3, b0, 1, rows, 1, fp8)) return cuda_fail();
-  return gqa::launch_decode_split(D, ext_on, fp8, tq, tk, tv, p, static_cast<cudaStream_t>(stream)) == 0 ? ATTN_OK
-                                                                                               : ATTN_ERR_CUDA;
+  if (!view_maps(kv, D, Dv, Hkv, Skv, B, fp8, &tk, &tv)) return cuda_fail();
+  return gqa::launch_decode_split(D, Dv, ext_on, fp8, tq, tk, tv, p, static_cast<cudaStream_t>(stream)) == 0
+             ? ATTN_OK
+             : ATTN_ERR_CUDA;
 }
 
 int attn_merge(const float* partial_out, const float* partial_lse, void* out, float* lse, int B, int Hq, int Sq,

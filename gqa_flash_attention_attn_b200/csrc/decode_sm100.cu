@@ -203,13 +203,20 @@ __device__ __noinline__ void write_partial_o(uint32_t taddr, int RP, int R, int 
   }
 }
 
-template <int D, bool EXT, bool PAGED, bool FP8>
+template <int DK, int DV, bool EXT, bool PAGED, bool FP8>
 __global__ void __launch_bounds__(THREADS, 2)
     decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
-  constexpr int KC = D / 128;  // 128-column slots per K (or V) tile
+  // K tiles are DK columns wide (Q . K over DK), V tiles and O are DV wide;
+  // a K tile takes KCK 128-column slots, the last one half filled when DK is
+  // an odd multiple of 64 (e.g. 320, 576)
+  constexpr int KCK = (DK + 127) / 128;
+  constexpr bool KHALF = (DK % 128) != 0;
+  constexpr int KC = DV / 128;   // V slots per tile, and O^T chunks
+  constexpr int D = DV;          // output width
+  static_assert(DK % 64 == 0 && DV % 128 == 0 && (!FP8 || DK == DV), "head sizes");
   const int RP = p.RP, g = p.g, nbuf = p.nbuf;
-  const Layout L(D, RP, nbuf, p.mask_rows, FP8);
+  const Layout L(DK, RP, nbuf, p.mask_rows, FP8);
   constexpr uint32_t SLOTB = FP8 ? BOX_BYTES : SLOT_BYTES;   // bytes of one 128-column K/V slot
 
   extern __shared__ uint8_t smem_raw[];
@@ -317,7 +324,7 @@ __global__ void __launch_bounds__(THREADS, 2)
   };
 
   // Zero the padding rows of Q (rows Rbox..RP-1 of every 64-column box).
-  for (int i = threadIdx.x; i < (D / 64) * (RP - Rbox) * 32; i += THREADS) {
+  for (int i = threadIdx.x; i < (DK / 64) * (RP - Rbox) * 32; i += THREADS) {
     const int box = i / ((RP - Rbox) * 32);
     const int w = i - box * (RP - Rbox) * 32;
     reinterpret_cast<uint32_t*>(gbase + L.off_q + (uint32_t)box * RP * 128u + (uint32_t)Rbox * 128u)[w] = 0u;
@@ -376,8 +383,8 @@ __global__ void __launch_bounds__(THREADS, 2)
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      mbar_arrive_expect_tx(bar(BAR_Q), (uint32_t)(D / 64) * Rbox * 128u);
-      for (int kb = 0; kb < D / 64; ++kb)
+      mbar_arrive_expect_tx(bar(BAR_Q), (uint32_t)(DK / 64) * Rbox * 128u);
+      for (int kb = 0; kb < DK / 64; ++kb)
         tma_load_4d(base + L.off_q + (uint32_t)kb * RP * 128u, &tm_q, bar(BAR_Q), kb * 64, kvh * g, s0, b);
       // ring order: K_0, then (K_{j+1}, V_j) for j = 0..n-1; KC slots each
       bool ok = true;
@@ -386,20 +393,24 @@ __global__ void __launch_bounds__(THREADS, 2)
       auto issue = [&](const CUtensorMap* tm, int j, SegCursor& cu) {
         cu.to(j);
         const int key0 = cu.key0(j, rev);
-        for (int c = 0; c < KC; ++c, ++n) {
+        const bool is_k = tm == &tm_k;
+        const int nslot = is_k ? KCK : KC;
+        for (int c = 0; c < nslot; ++c, ++n) {
           const int slot = n % nbuf, use = n / nbuf;
           if (use > 0 && !mbar_wait(bar(bar_empty(slot)), (uint32_t)(use - 1) & 1u, wd)) {
             ok = false;
             return;
           }
-          mbar_arrive_expect_tx(bar(bar_full(slot)), SLOTB);
+          // a half-filled last K slot (DK an odd multiple of 64) takes one box
+          const bool half = KHALF && is_k && c == KCK - 1;
+          mbar_arrive_expect_tx(bar(bar_full(slot)), half ? BOX_BYTES : SLOTB);
           const uint32_t dst = base + L.off_ring + (uint32_t)slot * SLOTB;
           if constexpr (!PAGED) {
             if (FP8) {
               tma_load_4d(dst, tm, bar(bar_full(slot)), c * 128, kvh, key0, b);   // 128 e4m3 columns
             } else {
               tma_load_4d(dst, tm, bar(bar_full(slot)), (2 * c) * 64, kvh, key0, b);
-              tma_load_4d(dst + BOX_BYTES, tm, bar(bar_full(slot)), (2 * c + 1) * 64, kvh, key0, b);
+              if (!half) tma_load_4d(dst + BOX_BYTES, tm, bar(bar_full(slot)), (2 * c + 1) * 64, kvh, key0, b);
             }
           } else {
             // paged: each page-sized run of keys from its physical page (the
@@ -416,8 +427,9 @@ __global__ void __launch_bounds__(THREADS, 2)
                 tma_load_4d(dst + off, tm, bar(bar_full(slot)), c * 128, kvh, key - lp * ps, page);
               } else {
                 tma_load_4d(dst + off, tm, bar(bar_full(slot)), (2 * c) * 64, kvh, key - lp * ps, page);
-                tma_load_4d(dst + BOX_BYTES + off, tm, bar(bar_full(slot)), (2 * c + 1) * 64, kvh, key - lp * ps,
-                            page);
+                if (!half)
+                  tma_load_4d(dst + BOX_BYTES + off, tm, bar(bar_full(slot)), (2 * c + 1) * 64, kvh, key - lp * ps,
+                              page);
               }
             }
           }
@@ -440,7 +452,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       int n = 0;
       // S^T_j = K_j Q^T into S buffer j%2, one 128-column slot at a time
       auto mma_s = [&](int j) {
-        for (int c = 0; c < KC; ++c, ++n) {
+        for (int c = 0; c < KCK; ++c, ++n) {
           const int slot = n % nbuf;
           if (!mbar_wait(bar(bar_full(slot)), (uint32_t)(n / nbuf) & 1u, wd)) { ok = false; return; }
           tc_fence_after();
@@ -459,8 +471,11 @@ __global__ void __launch_bounds__(THREADS, 2)
               }
             }
           } else {
+            // 16 columns per MMA: 8 per full slot, 4 for a half-filled last K slot
+            const int nkk = (KHALF && c == KCK - 1) ? 4 : 8;
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
+              if (kk >= nkk) break;
               const uint32_t in_box = (uint32_t)(kk & 3) * 32u;
               const uint32_t a = kb + (uint32_t)(kk >> 2) * BOX_BYTES + in_box;
               const uint32_t qb = base + L.off_q + (uint32_t)(2 * c + (kk >> 2)) * RP * 128u + in_box;
@@ -539,7 +554,7 @@ __global__ void __launch_bounds__(THREADS, 2)
         ok = false;
       } else {
         tc_fence_after();
-        const int cpr = D / 8;   // 16-byte chunks of 8 bf16 per row
+        const int cpr = DK / 8;   // 16-byte chunks of 8 bf16 per row
         auto qoff = [&](int r, int col) -> uint32_t {
           return (uint32_t)(col >> 6) * RP * 128u + (uint32_t)r * 128u + ((uint32_t)(((col & 63) >> 3) ^ (r & 7)) << 4);
         };
@@ -861,27 +876,27 @@ __global__ void __launch_bounds__(THREADS, 2)
   }
 }
 
-template <int D, bool EXT, bool PAGED, bool FP8>
+template <int DK, int DV, bool EXT, bool PAGED, bool FP8>
 int launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
              const DecodeParams& p, cudaStream_t stream) {
-  const Layout L(D, p.RP, p.nbuf, p.mask_rows, FP8);
-  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, EXT, PAGED, FP8>,
+  const Layout L(DK, p.RP, p.nbuf, p.mask_rows, FP8);
+  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<DK, DV, EXT, PAGED, FP8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
   if (e != cudaSuccess) return (int)e;
   dim3 grid((unsigned)((p.num_splits + p.group - 1) / p.group), (unsigned)(p.B * p.Hkv * p.nqc));
-  decode_split_kernel<D, EXT, PAGED, FP8><<<grid, THREADS, L.total, stream>>>(tq, tk, tv, p);
+  decode_split_kernel<DK, DV, EXT, PAGED, FP8><<<grid, THREADS, L.total, stream>>>(tq, tk, tv, p);
   return (int)cudaGetLastError();
 }
 
-template <int D, bool FP8>
+template <int DK, int DV, bool FP8>
 int launch_d(bool ext, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
              const DecodeParams& p, cudaStream_t stream) {
   const bool paged = p.block_table != nullptr;
   if (ext)
-    return paged ? launch_t<D, true, true, FP8>(tq, tk, tv, p, stream)
-                 : launch_t<D, true, false, FP8>(tq, tk, tv, p, stream);
-  return paged ? launch_t<D, false, true, FP8>(tq, tk, tv, p, stream)
-               : launch_t<D, false, false, FP8>(tq, tk, tv, p, stream);
+    return paged ? launch_t<DK, DV, true, true, FP8>(tq, tk, tv, p, stream)
+                 : launch_t<DK, DV, true, false, FP8>(tq, tk, tv, p, stream);
+  return paged ? launch_t<DK, DV, false, true, FP8>(tq, tk, tv, p, stream)
+               : launch_t<DK, DV, false, false, FP8>(tq, tk, tv, p, stream);
 }
 
 }  // namespace
@@ -894,14 +909,27 @@ int decode_max_nbuf() { return MAX_NBUF; }
 
 int decode_max_group() { return MAX_GROUP; }
 
-int launch_decode_split(int D, bool ext, bool fp8, const CUtensorMap& tq, const CUtensorMap& tk,
+int launch_decode_split(int D, int Dv, bool ext, bool fp8, const CUtensorMap& tq, const CUtensorMap& tk,
                         const CUtensorMap& tv, const DecodeParams& p, cudaStream_t stream) {
-  switch (D) {
-    case 128: return fp8 ? launch_d<128, true>(ext, tq, tk, tv, p, stream) : launch_d<128, false>(ext, tq, tk, tv, p, stream);
-    case 256: return fp8 ? launch_d<256, true>(ext, tq, tk, tv, p, stream) : launch_d<256, false>(ext, tq, tk, tv, p, stream);
-    case 512: return fp8 ? launch_d<512, true>(ext, tq, tk, tv, p, stream) : launch_d<512, false>(ext, tq, tk, tv, p, stream);
-    default: return (int)cudaErrorInvalidValue;
+  if (D == Dv) {
+    switch (D) {
+      case 128: return fp8 ? launch_d<128, 128, true>(ext, tq, tk, tv, p, stream) : launch_d<128, 128, false>(ext, tq, tk, tv, p, stream);
+      case 256: return fp8 ? launch_d<256, 256, true>(ext, tq, tk, tv, p, stream) : launch_d<256, 256, false>(ext, tq, tk, tv, p, stream);
+      case 512: return fp8 ? launch_d<512, 512, true>(ext, tq, tk, tv, p, stream) : launch_d<512, 512, false>(ext, tq, tk, tv, p, stream);
+      default: return (int)cudaErrorInvalidValue;
+    }
   }
+  // asymmetric head sizes (bf16 K/V): Q.K over D columns, V and O over Dv
+  if (fp8) return (int)cudaErrorInvalidValue;
+  if (D == 576 && Dv == 512) return launch_d<576, 512, false>(ext, tq, tk, tv, p, stream);
+  if (D == 320 && Dv == 256) return launch_d<320, 256, false>(ext, tq, tk, tv, p, stream);
+  if (D == 192 && Dv == 128) return launch_d<192, 128, false>(ext, tq, tk, tv, p, stream);
+  return (int)cudaErrorInvalidValue;
+}
+
+bool decode_dims_supported(int D, int Dv, bool fp8) {
+  if (D == Dv) return D == 128 || D == 256 || D == 512;
+  return !fp8 && ((D == 576 && Dv == 512) || (D == 320 && Dv == 256) || (D == 192 && Dv == 128));
 }
 
 }  // namespace gqa

@@ -81,8 +81,11 @@ struct MergeParams {
 int launch_prefill(int D, bool ext, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                    const CUtensorMap& tm, const PrefillParams& p, cudaStream_t stream);
 size_t prefill_smem_bytes(int D);
-int launch_decode_split(int D, bool ext, bool fp8, const CUtensorMap& tq, const CUtensorMap& tk,
+// D: the Q and K head size; Dv: the V and O head size (pairs with D != Dv:
+// 576/512, 320/256, 192/128, bf16 only)
+int launch_decode_split(int D, int Dv, bool ext, bool fp8, const CUtensorMap& tq, const CUtensorMap& tk,
                         const CUtensorMap& tv, const DecodeParams& p, cudaStream_t stream);
+bool decode_dims_supported(int D, int Dv, bool fp8);
 size_t decode_smem_bytes(int D, int RP, int nbuf, int mask_rows, bool fp8);
 int decode_max_group();
 int launch_merge(const MergeParams& p, cudaStream_t stream);

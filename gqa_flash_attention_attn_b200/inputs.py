@@ -47,6 +47,14 @@ class Workload:
     # K/V element type: "bf16", or "fp8" (e4m3 codes with per-head scales from
     # make_fp8_kv of the bf16 draw)
     kv_dtype: str = "bf16"
+    # V head size (0: D); v_of_k: V is the first Dv columns of K (one cache
+    # holds both, as for multi-head latent attention)
+    Dv: int = 0
+    v_of_k: bool = False
+
+    @property
+    def dv(self) -> int:
+        return self.Dv or self.D
 
     @property
     def has_options(self) -> bool:
@@ -81,15 +89,17 @@ class Workload:
         return hi - lo if self.causal else self.Skv
 
     def flops(self) -> int:
-        """Algorithmic FLOPs: 4*D per visible (query, key) pair."""
-        return 4 * self.D * self.visible_pairs_per_head() * self.B * self.Hq
+        """Algorithmic FLOPs: 2*D (Q.K) + 2*Dv (P.V) per visible (query, key) pair."""
+        return 2 * (self.D + self.dv) * self.visible_pairs_per_head() * self.B * self.Hq
 
     def io_bytes(self) -> int:
-        """Algorithmic bytes: Q, K, V read once (bf16); O and LSE written once."""
+        """Algorithmic bytes: Q, K, V read once (bf16; V counted in K when it
+        is a view of K); O and LSE written once."""
         ob = 2 if self.out_dtype == "bf16" else 4
         q = self.B * self.Sq * self.Hq * self.D * 2
-        kv = 2 * self.B * self.kv_rows_read() * self.Hkv * self.D * (1 if self.kv_dtype == "fp8" else 2)
-        o = self.B * self.Sq * self.Hq * self.D * ob
+        cols = self.D + (0 if self.v_of_k else self.dv)
+        kv = self.B * self.kv_rows_read() * self.Hkv * cols * (1 if self.kv_dtype == "fp8" else 2)
+        o = self.B * self.Sq * self.Hq * self.dv * ob
         lse = self.B * self.Hq * self.Sq * 4
         return q + kv + o + lse
 
@@ -151,18 +161,27 @@ WORKLOADS = {
         "paged_decode_d512_p64", "decode", B=16, Hq=16, Hkv=1, Sq=1, Skv=16384, D=512,
         q_offset=16383, causal=True, out_dtype="bf16", num_splits=32, page_size=64,
         note="the D512 split-KV decode over a paged cache: 64-key pages in scattered order"),
+    "mla_decode_d576_v512": Workload(
+        "mla_decode_d576_v512", "decode", B=16, Hq=16, Hkv=1, Sq=1, Skv=16384, D=576, Dv=512, v_of_k=True,
+        q_offset=16383, causal=True, out_dtype="bf16", num_splits=32,
+        note="B16 Hq16 Hkv1 Skv16384, K 576 wide and V its first 512 columns (latent-cache decode)"),
+    "prefill_d192_v128_4k": Workload(
+        "prefill_d192_v128_4k", "prefill", B=1, Hq=32, Hkv=8, Sq=4096, Skv=4096, D=192, Dv=128,
+        q_offset=0, causal=True, out_dtype="bf16",
+        note="the 4k causal GQA prefill with Q/K head size 192 and V/O head size 128"),
 }
 
 
-def make_qkv(B, Hq, Hkv, Sq, Skv, D, *, seed=0, device="cpu"):
-    """Seeded q [B,Sq,Hq,D], k and v [B,Skv,Hkv,D], all bf16, drawn q, k, v in order."""
+def make_qkv(B, Hq, Hkv, Sq, Skv, D, *, seed=0, device="cpu", Dv=None):
+    """Seeded q [B,Sq,Hq,D], k [B,Skv,Hkv,D] and v [B,Skv,Hkv,Dv] (Dv = D by
+    default), all bf16, drawn q, k, v in order."""
     gen = torch.Generator(device=device)
     gen.manual_seed(seed)
     q = torch.randn((B, Sq, Hq, D), generator=gen, dtype=torch.float32, device=device)
     q = q.to(torch.bfloat16)
     k = torch.randn((B, Skv, Hkv, D), generator=gen, dtype=torch.float32, device=device)
     k = k.to(torch.bfloat16)
-    v = torch.randn((B, Skv, Hkv, D), generator=gen, dtype=torch.float32, device=device)
+    v = torch.randn((B, Skv, Hkv, Dv or D), generator=gen, dtype=torch.float32, device=device)
     v = v.to(torch.bfloat16)
     return q, k, v
 
@@ -230,7 +249,11 @@ def make_fp8_kv(k, v):
 
 
 def make_workload_inputs(w: Workload, *, seed=0, device="cpu"):
-    return make_qkv(w.B, w.Hq, w.Hkv, w.Sq, w.Skv, w.D, seed=seed, device=device)
+    """q, k, v of a workload; with v_of_k, v is the view k[..., :Dv]."""
+    q, k, v = make_qkv(w.B, w.Hq, w.Hkv, w.Sq, w.Skv, w.D, seed=seed, device=device, Dv=w.dv)
+    if w.v_of_k:
+        v = k[..., :w.dv]
+    return q, k, v
 
 
 def sample_rows(w: Workload, n: int, *, seed=1234, include_edges=True):

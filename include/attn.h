@@ -268,6 +268,22 @@ int attn_merge_ex(const float* partial_out, const float* partial_lse, void* out,
  * elements, else ATTN_ERR_ALIGNMENT / ATTN_ERR_INVALID_ARG; k_scale and
  * v_scale non-NULL and 4-byte aligned for fp8 (else ATTN_ERR_INVALID_ARG).
  * The caller owns every buffer.
+ *
+ * Head sizes (head_dim_v): K has D columns per head (D = the Q head size
+ * argument), V has Dv = head_dim_v columns (0 means Dv = D), and O and the
+ * partials have Dv columns: out and partial_out are [.., Hq, Dv] instead of
+ * [.., Hq, D].  Pairs with Dv != D are (D, Dv) = (576, 512), (320, 256) and
+ * (192, 128), bf16 only ("ggml-org/llama.cpp PR #28507", the FLASH_ATTN_EXT
+ * cases with hsk=320, hsv=256 and the v_is_view_of_k flag; "Anbeeld/beellama.cpp
+ * PR #149", the D256 tile follow-up and the (576, 512) rows of the review).
+ * V may be a view of K: v = k with the same strides reads the first Dv
+ * columns of each K row (multi-head latent attention caches).  Other pairs
+ * give ATTN_ERR_UNSUPPORTED.
+ *
+ * V strides (v_stride_*): V's elements sit at v + (same index expression)
+ * with v_stride_seq, v_stride_token and v_stride_head in place of K's, for
+ * separate K and V tensors of different widths or layouts.  All three 0
+ * means V shares K's strides; otherwise each obeys the rules for K's.
  */
 typedef struct attn_kv_view {
   const void* k;            /* bf16 */
@@ -283,6 +299,10 @@ typedef struct attn_kv_view {
   int kv_dtype;             /* ATTN_BF16 or ATTN_FP8_E4M3 */
   const float* k_scale;     /* fp8: device [Hkv], K = code * k_scale[kvh] */
   const float* v_scale;     /* fp8: device [Hkv], V = code * v_scale[kvh] */
+  int head_dim_v;           /* V and O head size Dv, or 0: Dv = D */
+  long long v_stride_seq;   /* V's own strides, or all three 0: V uses K's */
+  long long v_stride_token;
+  long long v_stride_head;
 } attn_kv_view;
 
 /*
@@ -290,14 +310,35 @@ typedef struct attn_kv_view {
  * be NULL; sinks belong to attn_merge_ex).  Splits: chunk = ceil(len_b /
  * num_splits) keys of sequence b per split, rounded up to a multiple of 128
  * when paged so that no 128-key tile crosses a page; splits past the end
- * publish lse = -inf and O = 0.  Other arguments, limits and errors as in
+ * publish lse = -inf and O = 0.  With head_dim_v = Dv != D the partials are
+ * [S, B, Sq, Hq, Dv] and the row limit reads (2 + Dv/128) * R16 <= 256; merge
+ * them with attn_merge at D = Dv.  Other arguments, limits and errors as in
  * attn_decode_split.
  */
 int attn_decode_split_kv(const void* q, const attn_kv_view* kv, float* partial_out, float* partial_lse,
                          int B, int Hq, int Hkv, int Sq, int Skv, int D, int q_offset, int causal,
                          float scale, int num_splits, const attn_options* opt, void* stream);
 
-/* Library version, e.g. 0x000300 for 0.3.0. */
+/*
+ * Prefill over a K/V view: attn_prefill_ex with K and V described by *kv
+ * (strides, paging, lengths per sequence, fp8 codes, Dv != D).  out is
+ * [B, Sq, Hq, Dv].  With seq_lens, q_offset is ignored and the Sq rows of
+ * sequence b sit at positions len_b - Sq + s, as in attn_decode_split_kv.
+ *   - D = Dv in {64, 128, 256}, bf16, unpaged, no seq_lens: the prefill
+ *     kernel, reading K and V through the view's strides.
+ *   - otherwise (D = Dv = 512, the pairs with Dv != D, paged, fp8 or
+ *     seq_lens): the split-KV kernel with one split and the query rows cut
+ *     into chunks per CTA, writing O and LSE directly, as attn_prefill does
+ *     at D = 512.  Dims: D = Dv in {128, 256, 512}, or a pair listed under
+ *     attn_kv_view; Hq/Hkv <= 32.  Else ATTN_ERR_UNSUPPORTED.
+ * Arguments, options (*opt may be NULL; sinks apply here), alignment and
+ * errors otherwise as in attn_prefill_ex and attn_decode_split_kv.
+ */
+int attn_prefill_kv(const void* q, const attn_kv_view* kv, void* out, float* lse, int B, int Hq, int Hkv,
+                    int Sq, int Skv, int D, int q_offset, int causal, float scale, int out_dtype,
+                    const attn_options* opt, void* stream);
+
+/* Library version, e.g. 0x000400 for 0.4.0. */
 int attn_version(void);
 
 #ifdef __cplusplus

@@ -26,6 +26,11 @@ Functions and the passage each follows (all pinned by tests/test_oracle_pins.py)
   *_ex            the same with the optional logit terms of the FLASH_ATTN_EXT
                   operator ("ggml-org/llama.cpp PR #28507", Crash 1: sinks,
                   max_bias, logit_softcap, mask) and a sliding window (see oracle.c)
+
+V narrower than K (attention_ex, attention_rows_ex: v with Dv < D columns, the
+hsk != hsv cases of the FLASH_ATTN_EXT list, e.g. hsk=320, hsv=256): column j
+of O = P V reads only column j of V, so V is zero-padded to D columns, the
+fp64 kernel runs unchanged and the first Dv columns of O are returned.
 """
 from __future__ import annotations
 
@@ -259,6 +264,18 @@ def _codes(x):
     return x
 
 
+def _pad_v(k, v):
+    """v widened to k's head size with zero columns, and the original Dv."""
+    D, Dv = k.shape[-1], v.shape[-1]
+    if Dv == D:
+        return v, Dv
+    if Dv > D or v.shape[:-1] != k.shape[:-1]:
+        raise ValueError("v must have k's leading shape and at most D columns")
+    pad = np.zeros(v.shape[:-1] + (D,), dtype=np.float64)
+    pad[..., :Dv] = v
+    return pad, Dv
+
+
 def alibi_slope(h, Hq, max_bias, lib=None):
     return (lib or load()).oracle_alibi_slope(int(h), int(Hq), float(max_bias))
 
@@ -266,9 +283,10 @@ def alibi_slope(h, Hq, max_bias, lib=None):
 def attention_ex(q, k, v, *, scale, causal=True, q_offset=0, softcap=0.0, alibi_max_bias=0.0, sinks=None,
                  window=0, mask=None, lib=None):
     """attention() with softcap, ALiBi, sink logits [Hq], a sliding window and
-    an additive mask [B or 1, Sq, Skv]."""
+    an additive mask [B or 1, Sq, Skv].  v may have Dv < D columns."""
     lib = lib or load()
     q, k, v = _f64(q), _f64(k), _f64(v)
+    v, Dv = _pad_v(k, v)
     B, Hq, Hkv, Sq, Skv, D = _dims(q, k)
     sk, skp = _sinks_arg(sinks)
     mk, mkp, msb, mss = _mask_arg(mask, B, Sq, Skv)
@@ -277,13 +295,15 @@ def attention_ex(q, k, v, *, scale, causal=True, q_offset=0, softcap=0.0, alibi_
     lib.oracle_attention_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Skv, D,
                             int(q_offset), int(bool(causal)), float(scale), float(softcap),
                             float(alibi_max_bias), skp, int(window), mkp, msb, mss)
-    return out, lse
+    return np.ascontiguousarray(out[..., :Dv]), lse
 
 
 def attention_rows_ex(q, k, v, rows, *, scale, causal=True, q_offset=0, softcap=0.0, alibi_max_bias=0.0,
                       sinks=None, window=0, mask=None, lib=None):
+    """attention_ex() on selected (b, h, s) rows; v may have Dv < D columns."""
     lib = lib or load()
     q, k, v = _f64(q), _f64(k), _f64(v)
+    v, Dv = _pad_v(k, v)
     B, Hq, Hkv, Sq, Skv, D = _dims(q, k)
     rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
     n = rows.shape[0]
@@ -294,7 +314,7 @@ def attention_rows_ex(q, k, v, rows, *, scale, causal=True, q_offset=0, softcap=
     lib.oracle_attention_rows_ex(_ptr(q), _ptr(k), _ptr(v), rows.ctypes.data_as(_lp), n, _ptr(out), _ptr(lse),
                                  B, Hq, Hkv, Sq, Skv, D, int(q_offset), int(bool(causal)), float(scale),
                                  float(softcap), float(alibi_max_bias), skp, int(window), mkp, msb, mss)
-    return out, lse
+    return np.ascontiguousarray(out[:, :Dv]), lse
 
 
 def split_ex(q, k, v, num_splits, *, scale, causal=True, q_offset=0, softcap=0.0, alibi_max_bias=0.0,

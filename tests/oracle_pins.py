@@ -26,6 +26,8 @@ What pins what:
                     force, the standard ALiBi slope values, geometric-series and
                     single-key closed forms, limits (huge cap, window 1 / Skv,
                     sink -inf), split/merge identity, torch SDPA with a bias
+  narrow V          V with Dv < D columns: 40-digit decimal brute force and
+                    torch SDPA with a value head size unlike the key's
 """
 from __future__ import annotations
 
@@ -583,6 +585,58 @@ def pin_fp8_attention_equals_dequantized(lib):
     np.testing.assert_array_equal(lse, ref_l)
 
 
+def pin_narrow_v_bruteforce_decimal(lib):
+    """V with fewer columns than K (Dv < D): textbook softmax in 40-digit
+    decimals, through attention_ex and attention_rows_ex."""
+    decimal.getcontext().prec = 40
+    Dd = decimal.Decimal
+    rng = _rng(41)
+    for (B, Hq, Hkv, Sq, Skv, D, Dv, q_offset, causal, window, use_sink) in [
+        (1, 2, 1, 3, 5, 3, 2, 2, True, 0, False),
+        (2, 4, 2, 2, 4, 4, 1, 0, False, 0, True),
+        (1, 4, 1, 3, 6, 5, 2, 3, True, 2, True),
+    ]:
+        q = rng.integers(-2, 3, size=(B, Sq, Hq, D)).astype(np.float64)
+        k = rng.integers(-2, 3, size=(B, Skv, Hkv, D)).astype(np.float64)
+        v = rng.integers(-3, 4, size=(B, Skv, Hkv, Dv)).astype(np.float64)
+        sinks = rng.integers(-2, 3, size=(Hq,)).astype(np.float64) if use_sink else None
+        scale = 0.5
+        kw = dict(scale=scale, causal=causal, q_offset=q_offset, sinks=sinks, window=window, lib=lib)
+        out, lse = oracle.attention_ex(q, k, v, **kw)
+        assert out.shape == (B, Sq, Hq, Dv)
+        rows = [(b, h, s) for b in range(B) for h in range(Hq) for s in range(Sq)]
+        ro, rl = oracle.attention_rows_ex(q, k, v, rows, **kw)
+        assert ro.shape == (len(rows), Dv)
+        g = Hq // Hkv
+        for i, (b, h, s) in enumerate(rows):
+            pos = q_offset + s
+            ts = [t for t in range(Skv) if ((not causal) or t <= pos) and (window == 0 or t > pos - window)]
+            ex = [(Dd(scale) * sum(Dd(int(q[b, s, h, d])) * Dd(int(k[b, t, h // g, d])) for d in range(D))).exp()
+                  for t in ts]
+            den = sum(ex) + (Dd(int(sinks[h])).exp() if use_sink else Dd(0))
+            for d in range(Dv):
+                want = float(sum(e * Dd(int(v[b, t, h // g, d])) for e, t in zip(ex, ts)) / den)
+                assert abs(want - out[b, s, h, d]) < 1e-13 and abs(want - ro[i, d]) < 1e-13, (b, h, s, d)
+            assert abs(float(den.ln()) - lse[b, h, s]) < 1e-13 and abs(float(den.ln()) - rl[i]) < 1e-13
+
+
+def pin_narrow_v_torch_sdpa(lib):
+    """V with Dv < D columns against torch's float64 SDPA, which takes a value
+    head size unlike the key's."""
+    rng = _rng(42)
+    B, Hq, Hkv, Sq, Skv, D, Dv = 2, 6, 2, 5, 11, 12, 8
+    q = _normal(rng, (B, Sq, Hq, D))
+    k = _normal(rng, (B, Skv, Hkv, D))
+    v = _normal(rng, (B, Skv, Hkv, Dv))
+    out, _ = oracle.attention_ex(q, k, v, scale=0.3, causal=False, lib=lib)
+    g = Hq // Hkv
+    tq = torch.from_numpy(q).permute(0, 2, 1, 3)
+    tk = torch.from_numpy(k).permute(0, 2, 1, 3).repeat_interleave(g, dim=1)
+    tv = torch.from_numpy(v).permute(0, 2, 1, 3).repeat_interleave(g, dim=1)
+    ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, scale=0.3).permute(0, 2, 1, 3).numpy()
+    np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-12)
+
+
 ALL_PINS = [
     pin_bruteforce_decimal,
     pin_golden_three_keys,
@@ -611,4 +665,6 @@ ALL_PINS = [
     pin_split_merge_mask,
     pin_e4m3_codes_match_torch,
     pin_fp8_attention_equals_dequantized,
+    pin_narrow_v_bruteforce_decimal,
+    pin_narrow_v_torch_sdpa,
 ]

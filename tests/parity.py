@@ -45,19 +45,20 @@ def assert_lse_close(got, want, what=""):
         assert err <= LSE_ABS, f"{what}: LSE abs error {err:.3e}"
 
 
-def oracle_rows_by_batch(q, k, v, rows, *, scale, causal, q_offset):
-    """Oracle O rows [n, D] and LSE [n] for (b, h, s) triples, slicing per batch so
-    only one batch entry is widened to float64 at a time."""
+def oracle_rows_by_batch(q, k, v, rows, *, scale, causal, q_offset, **terms):
+    """Oracle O rows [n, Dv] and LSE [n] for (b, h, s) triples, slicing per batch so
+    only one batch entry is widened to float64 at a time.  terms (softcap,
+    sinks, ...) or a V narrower than K go through attention_rows_ex."""
     rows = np.asarray(rows, dtype=np.int64).reshape(-1, 3)
-    D = q.shape[3]
-    out = np.zeros((rows.shape[0], D))
+    Dv = v.shape[3]
+    fn = oracle.attention_rows_ex if (terms or Dv != k.shape[3]) else oracle.attention_rows
+    out = np.zeros((rows.shape[0], Dv))
     lse = np.zeros((rows.shape[0],))
     for b in np.unique(rows[:, 0]):
         sel = np.nonzero(rows[:, 0] == b)[0]
         sub = rows[sel].copy()
         sub[:, 0] = 0
-        o, l = oracle.attention_rows(q[b:b + 1], k[b:b + 1], v[b:b + 1], sub, scale=scale, causal=causal,
-                                     q_offset=q_offset)
+        o, l = fn(q[b:b + 1], k[b:b + 1], v[b:b + 1], sub, scale=scale, causal=causal, q_offset=q_offset, **terms)
         out[sel] = o
         lse[sel] = l
     return out, lse

@@ -22,7 +22,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert ga.version() == 0x000300
+    assert ga.version() == 0x000400
     assert ga.status_string(ga.ATTN_OK) == "ok"
     assert ga.status_string(ga.ATTN_ERR_TIMEOUT) == "pipeline wait timed out"
     assert ga.status_string(12345) == "unknown status"
@@ -182,16 +182,21 @@ def test_options_struct_matches_header():
     assert ctypes.sizeof(ga.AttnOptions) == 48
 
 
+def _view(view):
+    vw = dict(k=0x40000, v=0x50000, stride_seq=1024 * 512, stride_token=512, stride_head=512, block_table=None,
+              max_pages=0, page_size=0, num_pages=0, seq_lens=None, kv_dtype=0, k_scale=None, v_scale=None,
+              head_dim_v=0, v_stride_seq=0, v_stride_token=0, v_stride_head=0)
+    vw.update(view or {})
+    return ga.AttnKVView(**vw)
+
+
 def _kv_decode(lib, view=None, **kw):
     a = dict(q=P, po=P2, pl=P2, B=2, Hq=16, Hkv=1, Sq=1, Skv=1024, D=512, q_offset=1023, causal=1,
              scale=0.0441941738, S=4)
     a.update(kw)
     if view is None:
         view = {}
-    vw = dict(k=0x40000, v=0x50000, stride_seq=1024 * 512, stride_token=512, stride_head=512, block_table=None,
-              max_pages=0, page_size=0, num_pages=0, seq_lens=None, kv_dtype=0, k_scale=None, v_scale=None)
-    vw.update(view)
-    v = ga.AttnKVView(**vw)
+    v = _view(view)
     return lib.attn_decode_split_kv(a["q"], ctypes.byref(v), a["po"], a["pl"], a["B"], a["Hq"], a["Hkv"], a["Sq"],
                                     a["Skv"], a["D"], a["q_offset"], a["causal"], a["scale"], a["S"], None, None)
 
@@ -216,6 +221,15 @@ def _kv_decode(lib, view=None, **kw):
     (dict(kv_dtype=2, k_scale=0x90000, v_scale=0x90002), {}, ga.ATTN_ERR_INVALID_ARG),
     (dict(kv_dtype=2, k_scale=0x90000, v_scale=0x90010, stride_head=520,
           stride_token=520, stride_seq=520 * 1024), {}, ga.ATTN_ERR_ALIGNMENT),  # 520 bytes: not 16-byte multiples
+    (dict(head_dim_v=-1), {}, ga.ATTN_ERR_INVALID_ARG),
+    (dict(v_stride_token=512), {}, ga.ATTN_ERR_INVALID_ARG),                  # own V strides: all three
+    (dict(v_stride_token=516, v_stride_head=512, v_stride_seq=1024 * 512), {}, ga.ATTN_ERR_ALIGNMENT),
+    (dict(head_dim_v=256), {}, ga.ATTN_ERR_UNSUPPORTED),                       # (512, 256): no kernel
+    (dict(head_dim_v=512), dict(D=320), ga.ATTN_ERR_UNSUPPORTED),              # Dv > D
+    (dict(head_dim_v=512, stride_token=576, stride_head=576, stride_seq=576 * 1024), dict(D=576, Hq=48),
+     ga.ATTN_ERR_UNSUPPORTED),                                                 # 48 rows x (2 + 4) > 256
+    (dict(head_dim_v=512, kv_dtype=2, k_scale=0x90000, v_scale=0x90010, stride_token=576, stride_head=576,
+          stride_seq=576 * 1024), dict(D=576), ga.ATTN_ERR_UNSUPPORTED),     # fp8 pairs: no kernel
 ])
 def test_decode_split_kv_rejects(lib, view, kw, status):
     assert _kv_decode(lib, view, **kw) == status
@@ -232,4 +246,37 @@ def test_kv_view_struct_matches_header():
     body = re.search(r"typedef struct attn_kv_view \{(.*?)\} attn_kv_view;", text, re.S).group(1)
     fields = [ln.split(";")[0].split()[-1].lstrip("*") for ln in body.strip().splitlines() if ";" in ln]
     assert fields == [f[0] for f in ga.AttnKVView._fields_]
-    assert ctypes.sizeof(ga.AttnKVView) == 96
+    assert ctypes.sizeof(ga.AttnKVView) == 128
+
+
+def _kv_prefill(lib, view=None, opt=None, **kw):
+    a = dict(q=P, out=P2, lse=P2, B=2, Hq=16, Hkv=1, Sq=64, Skv=1024, D=512, q_offset=960, causal=1,
+             scale=0.0441941738, out_dtype=0)
+    a.update(kw)
+    v = _view(view)
+    return lib.attn_prefill_kv(a["q"], ctypes.byref(v), a["out"], a["lse"], a["B"], a["Hq"], a["Hkv"], a["Sq"],
+                               a["Skv"], a["D"], a["q_offset"], a["causal"], a["scale"], a["out_dtype"],
+                               None if opt is None else ctypes.byref(opt), None)
+
+
+@pytest.mark.parametrize("view,kw,status", [
+    (dict(k=None), {}, ga.ATTN_ERR_INVALID_ARG),
+    ({}, dict(out=None), ga.ATTN_ERR_INVALID_ARG),
+    ({}, dict(out_dtype=2), ga.ATTN_ERR_INVALID_ARG),
+    ({}, dict(D=96), ga.ATTN_ERR_UNSUPPORTED),
+    (dict(block_table=0x70000, max_pages=8, page_size=128, num_pages=64), dict(D=64), ga.ATTN_ERR_UNSUPPORTED),
+    ({}, dict(Hq=64), ga.ATTN_ERR_UNSUPPORTED),                                # g = 64 > 32 on the wide path
+    (dict(head_dim_v=256), {}, ga.ATTN_ERR_UNSUPPORTED),
+    (dict(stride_token=516), {}, ga.ATTN_ERR_ALIGNMENT),
+    ({}, dict(q=ctypes.c_void_p(0x10008)), ga.ATTN_ERR_ALIGNMENT),
+    ({}, dict(lse=ctypes.c_void_p(0x20002)), ga.ATTN_ERR_ALIGNMENT),
+    ({}, dict(scale=0.0), ga.ATTN_ERR_INVALID_ARG),
+    ({}, dict(q_offset=-1), ga.ATTN_ERR_INVALID_ARG),
+])
+def test_prefill_kv_rejects(lib, view, kw, status):
+    assert _kv_prefill(lib, view, **kw) == status
+
+
+def test_prefill_kv_rejects_null_view(lib):
+    assert lib.attn_prefill_kv(P, None, P2, P2, 1, 8, 1, 128, 128, 128, 0, 1, 0.08, 0, None, None) == \
+        ga.ATTN_ERR_INVALID_ARG

@@ -62,3 +62,20 @@ def test_workload_byte_and_flop_counts():
     sw = WORKLOADS["sliding_window_prefill_16k_w4096_d128"]
     lo, hi = sw.visible_range(10000)
     assert (lo, hi) == (10000 - 4096 + 1, 10001)
+
+
+def test_narrow_v_workloads():
+    """Workloads with Dv < D: V drawn Dv wide, or a view of K's first Dv columns."""
+    from gqa_flash_attention_attn_b200.inputs import make_workload_inputs
+    w = WORKLOADS["prefill_d192_v128_4k"]
+    assert w.dv == 128
+    assert w.flops() == 2 * (192 + 128) * (4096 * 4097 // 2) * 32
+    q, k, v = make_qkv(1, 4, 2, 3, 5, 192, seed=9, Dv=128)
+    q2, k2, _ = make_qkv(1, 4, 2, 3, 5, 192, seed=9)
+    assert v.shape == (1, 5, 2, 128) and torch.equal(q, q2) and torch.equal(k, k2)
+    m = WORKLOADS["mla_decode_d576_v512"]
+    small = m.__class__(**{**m.__dict__, "B": 2, "Skv": 64, "q_offset": 63})
+    q, k, v = make_workload_inputs(small)
+    assert v.shape[-1] == 512 and v.data_ptr() == k.data_ptr() and torch.equal(v, k[..., :512])
+    # V inside K: only K's bytes are read
+    assert m.io_bytes() == (16 * 16 * 576 * 2 + 16 * 16384 * 576 * 2 + 16 * 16 * 512 * 2 + 16 * 16 * 4)

@@ -70,3 +70,33 @@ def test_mutant_is_caught(tmp_path, name, old, new):
         except (AssertionError, ValueError, FloatingPointError):
             caught.append(pin.__name__)
     assert caught, f"no pin rejects the planted mistake {name}"
+
+
+def _pad_v_at_end(k, v):
+    import numpy as np
+    pad = np.zeros(v.shape[:-1] + (k.shape[-1],))
+    pad[..., k.shape[-1] - v.shape[-1]:] = v
+    return pad, v.shape[-1]
+
+
+def _pad_v_unsliced(k, v):
+    import numpy as np
+    pad = np.zeros(v.shape[:-1] + (k.shape[-1],))
+    pad[..., :v.shape[-1]] = v
+    return pad, k.shape[-1]
+
+
+@pytest.mark.parametrize("mutant", [_pad_v_at_end, _pad_v_unsliced], ids=["v_at_end", "unsliced"])
+def test_narrow_v_mutant_is_caught(monkeypatch, mutant):
+    """A wrong widening of a narrow V (values in the last columns; O returned
+    D wide with the padding columns) fails a narrow-V pin."""
+    from oracle_pins import pin_narrow_v_bruteforce_decimal, pin_narrow_v_torch_sdpa
+    monkeypatch.setattr(oracle, "_pad_v", mutant)
+    lib = oracle.load()
+    caught = 0
+    for pin in (pin_narrow_v_bruteforce_decimal, pin_narrow_v_torch_sdpa):
+        try:
+            pin(lib)
+        except AssertionError:
+            caught += 1
+    assert caught > 0
