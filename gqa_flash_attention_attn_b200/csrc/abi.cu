@@ -11,7 +11,8 @@
 #include "kernels.h"
 
 namespace gqa {
-int prefill_slots(int D);
+int prefill_slots(int Dv);
+bool prefill_dims_supported(int D, int Dv);
 int decode_max_nbuf();
 }  // namespace gqa
 
@@ -212,6 +213,8 @@ bool view_maps(const attn_kv_view* kv, int D, int Dv, int Hkv, int Skv, int B, b
 // The view's fields in the split-KV kernel's parameters.
 void view_params(const attn_kv_view* kv, bool fp8, gqa::DecodeParams& p) {
   const bool paged = kv->block_table != nullptr;
+  const ViewStrides ks = k_strides(kv), vs = v_strides(kv);
+  p.kv_shared = kv->v == kv->k && ks.head == vs.head && ks.token == vs.token && ks.seq == vs.seq;
   p.seq_lens = kv->seq_lens;
   p.block_table = kv->block_table;
   p.max_pages = paged ? kv->max_pages : 0;
@@ -284,11 +287,12 @@ int prefill_wide(const void* q, const attn_kv_view* kv, bool fp8, void* out, flo
              : ATTN_ERR_CUDA;
 }
 
-// The prefill kernel over given K/V tensor maps (D 64, 128 or 256).
+// The prefill kernel over given K/V tensor maps (D = Dv in 64, 128, 256, or
+// D = 192 with Dv = 128).
 int prefill_fast(const void* q, const CUtensorMap& tk, const CUtensorMap& tv, void* out, float* lse, int B, int Hq,
-                 int Hkv, int Sq, int Skv, int D, int q_offset, int causal, float scale, int out_dtype,
+                 int Hkv, int Sq, int Skv, int D, int Dv, int q_offset, int causal, float scale, int out_dtype,
                  const gqa::LogitExt& ext, bool ext_on, void* stream) {
-  const int nslot = gqa::prefill_slots(D);
+  const int nslot = gqa::prefill_slots(Dv);
   const int g = Hq / Hkv;
   gqa::PrefillParams p{};
   p.out = out;
@@ -314,15 +318,16 @@ int prefill_fast(const void* q, const CUtensorMap& tk, const CUtensorMap& tv, vo
   CUtensorMap tm;
   std::memset(&tm, 0, sizeof(tm));
   if (ext.mask != nullptr && aligned(ext.mask, 16) && ext.mask_sr % 8 == 0 && ext.mask_sb % 8 == 0 &&
-      ext.mask_sr > 0 && (gqa::prefill_slots(D) == 1 || g % 2 == 0)) {
+      ext.mask_sr > 0 && (nslot == 1 || g % 2 == 0)) {
     const uint64_t bm = ext.mask_sb != 0 ? (uint64_t)B : 1u;
     const uint64_t s2 = ext.mask_sb != 0 ? (uint64_t)ext.mask_sb : (uint64_t)Sq * ext.mask_sr;
     if (!make_map_strided(&tm, ext.mask, Skv, Sq, bm, 1, (uint64_t)ext.mask_sr, s2, s2 * bm, 64, 128, 1, 1))
       return cuda_fail();
     p.mask_tma = 1;
   }
-  return gqa::launch_prefill(D, ext_on, tq, tk, tv, tm, p, static_cast<cudaStream_t>(stream)) == 0 ? ATTN_OK
-                                                                                          : ATTN_ERR_CUDA;
+  return gqa::launch_prefill(D, Dv, ext_on, tq, tk, tv, tm, p, static_cast<cudaStream_t>(stream)) == 0
+             ? ATTN_OK
+             : ATTN_ERR_CUDA;
 }
 
 // The contiguous [B, Skv, Hkv, D] view of k and v.
@@ -383,7 +388,7 @@ int attn_prefill_ex(const void* q, const void* k, const void* v, void* out, floa
   CUtensorMap tk, tv;
   if (!make_map(&tk, k, D, Hkv, Skv, B, 64, 1, 128, 1)) return cuda_fail();
   if (!make_map(&tv, v, D, Hkv, Skv, B, 64, 1, 128, 1)) return cuda_fail();
-  return prefill_fast(q, tk, tv, out, lse, B, Hq, Hkv, Sq, Skv, D, q_offset, causal, scale, out_dtype, ext, ext_on,
+  return prefill_fast(q, tk, tv, out, lse, B, Hq, Hkv, Sq, Skv, D, D, q_offset, causal, scale, out_dtype, ext, ext_on,
                       stream);
 }
 
@@ -404,7 +409,7 @@ int attn_prefill_kv(const void* q, const attn_kv_view* kv, void* out, float* lse
   st = check_view(kv, Skv, &fp8);
   if (st != ATTN_OK) return st;
   const int Dv = kv->head_dim_v != 0 ? kv->head_dim_v : D;
-  const bool fast = D == Dv && (D == 64 || D == 128 || D == 256) && !fp8 && kv->block_table == nullptr &&
+  const bool fast = gqa::prefill_dims_supported(D, Dv) && !fp8 && kv->block_table == nullptr &&
                     kv->seq_lens == nullptr;
   if (!fast && !gqa::decode_dims_supported(D, Dv, fp8)) return ATTN_ERR_UNSUPPORTED;
   if (!aligned(q, 16) || !aligned(out, 16)) return ATTN_ERR_ALIGNMENT;
@@ -415,8 +420,8 @@ int attn_prefill_kv(const void* q, const attn_kv_view* kv, void* out, float* lse
   CUtensorMap tk, tv;
   const ViewStrides ks = k_strides(kv), vs = v_strides(kv);
   if (!make_map_strided(&tk, kv->k, D, Hkv, Skv, B, ks.head, ks.token, ks.seq, 64, 1, 128, 1)) return cuda_fail();
-  if (!make_map_strided(&tv, kv->v, D, Hkv, Skv, B, vs.head, vs.token, vs.seq, 64, 1, 128, 1)) return cuda_fail();
-  return prefill_fast(q, tk, tv, out, lse, B, Hq, Hkv, Sq, Skv, D, q_offset, causal, scale, out_dtype, ext, ext_on,
+  if (!make_map_strided(&tv, kv->v, Dv, Hkv, Skv, B, vs.head, vs.token, vs.seq, 64, 1, 128, 1)) return cuda_fail();
+  return prefill_fast(q, tk, tv, out, lse, B, Hq, Hkv, Sq, Skv, D, Dv, q_offset, causal, scale, out_dtype, ext, ext_on,
                       stream);
 }
 

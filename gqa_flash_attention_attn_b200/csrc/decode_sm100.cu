@@ -388,6 +388,8 @@ __global__ void __launch_bounds__(THREADS, 2)
         tma_load_4d(base + L.off_q + (uint32_t)kb * RP * 128u, &tm_q, bar(BAR_Q), kb * 64, kvh * g, s0, b);
       // ring order: K_0, then (K_{j+1}, V_j) for j = 0..n-1; KC slots each
       bool ok = true;
+      const uint64_t pol_k = p.kv_shared ? l2_policy_evict_last() : l2_policy_evict_normal();
+      const uint64_t pol_v = p.kv_shared ? l2_policy_evict_first() : l2_policy_evict_normal();
       int n = 0;
       SegCursor ck(seg_sm, nseg), cv(seg_sm, nseg);   // the K and the V stream
       auto issue = [&](const CUtensorMap* tm, int j, SegCursor& cu) {
@@ -396,6 +398,8 @@ __global__ void __launch_bounds__(THREADS, 2)
         const bool is_k = tm == &tm_k;
         const int nslot = is_k ? KCK : KC;
         for (int c = 0; c < nslot; ++c, ++n) {
+          // K columns at or past DV are never read again as V
+          const uint64_t pol = (is_k && c * 128 < DV) ? pol_k : pol_v;
           const int slot = n % nbuf, use = n / nbuf;
           if (use > 0 && !mbar_wait(bar(bar_empty(slot)), (uint32_t)(use - 1) & 1u, wd)) {
             ok = false;
@@ -407,10 +411,10 @@ __global__ void __launch_bounds__(THREADS, 2)
           const uint32_t dst = base + L.off_ring + (uint32_t)slot * SLOTB;
           if constexpr (!PAGED) {
             if (FP8) {
-              tma_load_4d(dst, tm, bar(bar_full(slot)), c * 128, kvh, key0, b);   // 128 e4m3 columns
+              tma_load_4d_hint(dst, tm, bar(bar_full(slot)), c * 128, kvh, key0, b, pol);   // 128 e4m3 columns
             } else {
-              tma_load_4d(dst, tm, bar(bar_full(slot)), (2 * c) * 64, kvh, key0, b);
-              if (!half) tma_load_4d(dst + BOX_BYTES, tm, bar(bar_full(slot)), (2 * c + 1) * 64, kvh, key0, b);
+              tma_load_4d_hint(dst, tm, bar(bar_full(slot)), (2 * c) * 64, kvh, key0, b, pol);
+              if (!half) tma_load_4d_hint(dst + BOX_BYTES, tm, bar(bar_full(slot)), (2 * c + 1) * 64, kvh, key0, b, pol);
             }
           } else {
             // paged: each page-sized run of keys from its physical page (the
@@ -424,12 +428,12 @@ __global__ void __launch_bounds__(THREADS, 2)
               const int page = lp < p.max_pages ? __ldg(bt + lp) : -1;
               const uint32_t off = (uint32_t)(sub * rows) * 128u;
               if (FP8) {
-                tma_load_4d(dst + off, tm, bar(bar_full(slot)), c * 128, kvh, key - lp * ps, page);
+                tma_load_4d_hint(dst + off, tm, bar(bar_full(slot)), c * 128, kvh, key - lp * ps, page, pol);
               } else {
-                tma_load_4d(dst + off, tm, bar(bar_full(slot)), (2 * c) * 64, kvh, key - lp * ps, page);
+                tma_load_4d_hint(dst + off, tm, bar(bar_full(slot)), (2 * c) * 64, kvh, key - lp * ps, page, pol);
                 if (!half)
-                  tma_load_4d(dst + BOX_BYTES + off, tm, bar(bar_full(slot)), (2 * c + 1) * 64, kvh, key - lp * ps,
-                              page);
+                  tma_load_4d_hint(dst + BOX_BYTES + off, tm, bar(bar_full(slot)), (2 * c + 1) * 64, kvh, key - lp * ps,
+                              page, pol);
               }
             }
           }

@@ -24,7 +24,7 @@ struct LogitExt {
 };
 
 struct PrefillParams {
-  void* out;          // [B, Sq, Hq, D] bf16 or f32
+  void* out;          // [B, Sq, Hq, Dv] bf16 or f32
   float* lse;         // [B, Hq, Sq] or nullptr
   int* status;        // device status word
   int B, Hq, Hkv, Sq, Skv, q_offset, causal, out_f32;
@@ -66,6 +66,9 @@ struct DecodeParams {
   // (fout_bf16) or fp32 at fout, LSE at part_lse (may be nullptr)
   void* fout;
   int fout_bf16;
+  // V is a view of K (same base and strides): K tiles stay in L2 (evict_last)
+  // until their V reads, which then drop them (evict_first)
+  int kv_shared;
 };
 
 struct MergeParams {
@@ -78,9 +81,11 @@ struct MergeParams {
 };
 
 // Each returns a cudaError_t value (as int) from the launch.
-int launch_prefill(int D, bool ext, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+// D: the Q and K head size; Dv: the V and O head size (D = Dv in 64, 128,
+// 256, or D = 192 with Dv = 128)
+int launch_prefill(int D, int Dv, bool ext, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                    const CUtensorMap& tm, const PrefillParams& p, cudaStream_t stream);
-size_t prefill_smem_bytes(int D);
+size_t prefill_smem_bytes(int D, int Dv);
 // D: the Q and K head size; Dv: the V and O head size (pairs with D != Dv:
 // 576/512, 320/256, 192/128, bf16 only)
 int launch_decode_split(int D, int Dv, bool ext, bool fp8, const CUtensorMap& tq, const CUtensorMap& tk,

@@ -41,14 +41,22 @@ constexpr int BM = 128;   // query rows per slot (TMEM lanes)
 constexpr int BN = 128;   // keys per tile
 constexpr uint32_t BOX_BYTES = 128u * 128u;  // 128 rows x 64 bf16 columns
 constexpr float LN2 = 0.6931471805599453f;
+// Softmax exponentials: pair e of each 64-key half (e = 0..31) goes to the
+// polynomial exp2_poly2 when bit e is set, else to MUFU ex2.  Moving one
+// exponential in eight to the FMA pipe relieves the MUFU unit, which
+// otherwise paces the tensor cores at D = 128; more than that loads the FMA
+// and issue slots past the point of gain (measured).
+constexpr uint32_t kPolyPairs = 0x80808080u;
 
 // MB: the variant reads an additive mask, staged by TMA in two 64-key halves.
-template <int D, bool MB = false>
+// DK: the Q and K head size; DV: the V and O head size (DV <= DK).
+template <int DK, int DV = DK, bool MB = false>
 struct PrefillCfg {
-  static constexpr int NSLOT = (D <= 128) ? 2 : 1;
-  static constexpr int KB = D / 64;
-  static constexpr uint32_t TILE = KB * BOX_BYTES;
-  static constexpr int NBUF = (D == 64) ? 8 : (D == 128 ? 4 : 2);
+  static constexpr int NSLOT = (DV <= 128) ? 2 : 1;
+  static constexpr int KB = DK / 64;   // 64-column boxes of a Q or K tile
+  static constexpr int VB = DV / 64;   // and of a V tile
+  static constexpr uint32_t TILE = KB * BOX_BYTES;   // a Q slot or a ring slot (K or V)
+  static constexpr int NBUF = (DK == 64) ? 8 : (DK == 128 ? 4 : 2);
   static constexpr int THREADS = 128 * NSLOT + 64;
   static constexpr int WARP_PRODUCER = 4 * NSLOT;
   static constexpr int WARP_MMA = 4 * NSLOT + 1;
@@ -65,7 +73,7 @@ struct PrefillCfg {
   // Two S buffers (one per slot, or a double buffer for one slot), P aliased
   // at the start of its S buffer, then O per slot.
   static constexpr uint32_t TMEM_S = 0;                   // S buffer b at b*128
-  static constexpr uint32_t TMEM_O = 256;                 // O_i at TMEM_O + i*D
+  static constexpr uint32_t TMEM_O = 256;                 // O_i at TMEM_O + i*DV
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int BAR_Q = 0;
   static constexpr int BAR_QE = 1;
@@ -79,9 +87,9 @@ struct PrefillCfg {
   static constexpr int BAR_DRAIN = 12 + 2 * NBUF;
   __host__ __device__ static constexpr int bar_mfull(int h) { return 13 + 2 * NBUF + h; }
   __host__ __device__ static constexpr int bar_mempty(int h) { return 15 + 2 * NBUF + h; }
-  static_assert(256 + NSLOT * D <= 512, "TMEM budget");
+  static_assert(256 + NSLOT * DV <= 512, "TMEM budget");
   static_assert(SMEM <= 232448, "shared memory budget");
-  static_assert(D % 64 == 0, "head dim must be a multiple of 64");
+  static_assert(DK % 64 == 0 && DV % 64 == 0 && DV <= DK, "head dims");
 };
 
 // Wait that ignores the abort flag: used only to drain in-flight work.
@@ -266,13 +274,14 @@ __device__ __forceinline__ float row_max(const float (&v)[N]) {
   return fmax3(fmax3(mxc[0], mxc[1], mxc[2]), fmax3(mxc[3], mxc[4], mxc[5]), fmaxf(mxc[6], mxc[7]));
 }
 
-template <int D, int MODE>
-__global__ void __launch_bounds__(PrefillCfg<D, MODE == MODE_ALIBI_MASK || MODE == MODE_CAP_MASK>::THREADS, 1)
+template <int DK, int DV, int MODE>
+__global__ void __launch_bounds__(PrefillCfg<DK, DV, MODE == MODE_ALIBI_MASK || MODE == MODE_CAP_MASK>::THREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_m,
                    const PrefillParams p) {
   constexpr bool MB = MODE == MODE_ALIBI_MASK || MODE == MODE_CAP_MASK;
-  using C = PrefillCfg<D, MB>;
+  using C = PrefillCfg<DK, DV, MB>;
+  constexpr int D = DV;   // the output head size
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -358,8 +367,9 @@ __global__ void __launch_bounds__(PrefillCfg<D, MODE == MODE_ALIBI_MASK || MODE 
           int tile;
           const bool is_v = ring_item<C::NSLOT>(m, x.n_tiles, tile);
           const CUtensorMap* tm = is_v ? &tm_v : &tm_k;
-          mbar_arrive_expect_tx(bar(C::bar_full(buf)), C::TILE);
-          for (int kb = 0; kb < C::KB; ++kb)
+          const int nb = is_v ? C::VB : C::KB;
+          mbar_arrive_expect_tx(bar(C::bar_full(buf)), (uint32_t)nb * BOX_BYTES);
+          for (int kb = 0; kb < nb; ++kb)
             tma_load_4d(base + C::OFF_KV + buf * C::TILE + kb * BOX_BYTES, tm, bar(C::bar_full(buf)),
                         kb * 64, x.kvh, (x.t0 + (rev ? x.n_tiles - 1 - tile : tile)) * BN, x.b);
           issued = n + 1;
@@ -413,7 +423,7 @@ __global__ void __launch_bounds__(PrefillCfg<D, MODE == MODE_ALIBI_MASK || MODE 
         const uint64_t qd = qdesc0 + (uint64_t)(((uint32_t)qslot * C::TILE) >> 4);
         const uint64_t kd = kdesc0 + (uint64_t)(((uint32_t)(ring_n % C::NBUF) * C::TILE) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < DK / 16; ++kk) {
           const uint64_t off = (uint64_t)((((uint32_t)(kk >> 2) * BOX_BYTES) + (uint32_t)(kk & 3) * 32u) >> 4);
           mma_ss(tmem + C::TMEM_S + sb * 128, qd + off, kd + off, IDESC_QK, kk > 0 ? 1u : 0u);
         }
@@ -669,7 +679,8 @@ __global__ void __launch_bounds__(PrefillCfg<D, MODE == MODE_ALIBI_MASK || MODE 
 #pragma unroll
           for (int e = 0; e < BN / 4; ++e) {
             const float2 x = ffma2(make_float2(sv[2 * e], sv[2 * e + 1]), c2v, nmv);
-            const float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            const float2 pr = ((kPolyPairs >> e) & 1u) ? exp2_poly2(x)
+                                                              : make_float2(ex2_approx(x.x), ex2_approx(x.y));
             if (e & 1) acc1 = fadd2(acc1, pr); else acc0 = fadd2(acc0, pr);
             pk[e] = pack_bf16x2(pr.x, pr.y);
           }
@@ -688,7 +699,8 @@ __global__ void __launch_bounds__(PrefillCfg<D, MODE == MODE_ALIBI_MASK || MODE 
 #pragma unroll
           for (int e = 0; e < BN / 4; ++e) {
             const float2 x = ffma2(make_float2(sh[2 * e], sh[2 * e + 1]), c2v, nmv);
-            const float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            const float2 pr = ((kPolyPairs >> e) & 1u) ? exp2_poly2(x)
+                                                              : make_float2(ex2_approx(x.x), ex2_approx(x.y));
             if (e & 1) acc1 = fadd2(acc1, pr); else acc0 = fadd2(acc0, pr);
             pk[e] = pack_bf16x2(pr.x, pr.y);
           }
@@ -789,47 +801,54 @@ __global__ void __launch_bounds__(PrefillCfg<D, MODE == MODE_ALIBI_MASK || MODE 
   }
 }
 
-template <int D, int MODE>
+template <int DK, int DV, int MODE>
 int launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tm,
              const PrefillParams& p, cudaStream_t stream) {
-  using C = PrefillCfg<D, MODE == MODE_ALIBI_MASK || MODE == MODE_CAP_MASK>;
-  cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  using C = PrefillCfg<DK, DV, MODE == MODE_ALIBI_MASK || MODE == MODE_CAP_MASK>;
+  cudaError_t e = cudaFuncSetAttribute(prefill_kernel<DK, DV, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)C::SMEM);
   if (e != cudaSuccess) return (int)e;
   const long long units = (long long)p.n_qt * p.B * p.Hkv * p.units_per_kvh;
   if (units <= 0 || units > 0x7fffffffLL || p.num_ctas <= 0) return (int)cudaErrorInvalidValue;
   const long long grid = units < p.num_ctas ? units : p.num_ctas;  // persistent: one CTA per SM
-  prefill_kernel<D, MODE><<<(unsigned)grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, tm, p);
+  prefill_kernel<DK, DV, MODE><<<(unsigned)grid, C::THREADS, C::SMEM, stream>>>(tq, tk, tv, tm, p);
   return (int)cudaGetLastError();
 }
 
 }  // namespace
 
-size_t prefill_smem_bytes(int D) {
-  switch (D) {
-    case 64: return PrefillCfg<64>::SMEM;
-    case 128: return PrefillCfg<128>::SMEM;
-    case 256: return PrefillCfg<256>::SMEM;
-    default: return 0;
+size_t prefill_smem_bytes(int D, int Dv) {
+  if (D == Dv) {
+    switch (D) {
+      case 64: return PrefillCfg<64>::SMEM;
+      case 128: return PrefillCfg<128>::SMEM;
+      case 256: return PrefillCfg<256>::SMEM;
+      default: return 0;
+    }
   }
+  return (D == 192 && Dv == 128) ? PrefillCfg<192, 128>::SMEM : 0;
 }
 
-int prefill_slots(int D) { return D <= 128 ? 2 : 1; }
+int prefill_slots(int Dv) { return Dv <= 128 ? 2 : 1; }
 
-template <int D>
+bool prefill_dims_supported(int D, int Dv) {
+  return (D == Dv && (D == 64 || D == 128 || D == 256)) || (D == 192 && Dv == 128);
+}
+
+template <int DK, int DV>
 int launch_mode(int mode, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tm,
                 const PrefillParams& p, cudaStream_t stream) {
   switch (mode) {
-    case MODE_PLAIN: return launch_t<D, MODE_PLAIN>(tq, tk, tv, tm, p, stream);
-    case MODE_MASKS: return launch_t<D, MODE_MASKS>(tq, tk, tv, tm, p, stream);
-    case MODE_ALIBI: return launch_t<D, MODE_ALIBI>(tq, tk, tv, tm, p, stream);
-    case MODE_CAP: return launch_t<D, MODE_CAP>(tq, tk, tv, tm, p, stream);
-    case MODE_ALIBI_MASK: return launch_t<D, MODE_ALIBI_MASK>(tq, tk, tv, tm, p, stream);
-    default: return launch_t<D, MODE_CAP_MASK>(tq, tk, tv, tm, p, stream);
+    case MODE_PLAIN: return launch_t<DK, DV, MODE_PLAIN>(tq, tk, tv, tm, p, stream);
+    case MODE_MASKS: return launch_t<DK, DV, MODE_MASKS>(tq, tk, tv, tm, p, stream);
+    case MODE_ALIBI: return launch_t<DK, DV, MODE_ALIBI>(tq, tk, tv, tm, p, stream);
+    case MODE_CAP: return launch_t<DK, DV, MODE_CAP>(tq, tk, tv, tm, p, stream);
+    case MODE_ALIBI_MASK: return launch_t<DK, DV, MODE_ALIBI_MASK>(tq, tk, tv, tm, p, stream);
+    default: return launch_t<DK, DV, MODE_CAP_MASK>(tq, tk, tv, tm, p, stream);
   }
 }
 
-int launch_prefill(int D, bool ext, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+int launch_prefill(int D, int Dv, bool ext, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                    const CUtensorMap& tm, const PrefillParams& p, cudaStream_t stream) {
   // the cheapest variant that covers the requested terms
   const int mode = !ext ? MODE_PLAIN
@@ -837,10 +856,12 @@ int launch_prefill(int D, bool ext, const CUtensorMap& tq, const CUtensorMap& tk
                    : p.ext.mask != nullptr ? MODE_ALIBI_MASK
                    : p.ext.alibi ? MODE_ALIBI
                    : MODE_MASKS;
+  if (D == 192 && Dv == 128) return launch_mode<192, 128>(mode, tq, tk, tv, tm, p, stream);
+  if (D != Dv) return (int)cudaErrorInvalidValue;
   switch (D) {
-    case 64: return launch_mode<64>(mode, tq, tk, tv, tm, p, stream);
-    case 128: return launch_mode<128>(mode, tq, tk, tv, tm, p, stream);
-    case 256: return launch_mode<256>(mode, tq, tk, tv, tm, p, stream);
+    case 64: return launch_mode<64, 64>(mode, tq, tk, tv, tm, p, stream);
+    case 128: return launch_mode<128, 128>(mode, tq, tk, tv, tm, p, stream);
+    case 256: return launch_mode<256, 256>(mode, tq, tk, tv, tm, p, stream);
     default: return (int)cudaErrorInvalidValue;
   }
 }

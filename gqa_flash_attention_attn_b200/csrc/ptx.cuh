@@ -95,6 +95,34 @@ __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
 }
 
 // 4-D tiled load, completion counted on `bar` in bytes.  No multicast.
+// The same load with an L2 eviction-priority policy (from l2_policy_*).
+__device__ __forceinline__ void tma_load_4d_hint(uint32_t dst, const void* tmap, uint32_t bar, int c0, int c1,
+                                                 int c2, int c3, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2], %7;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "l"(policy)
+      : "memory");
+}
+
+// L2 policies for every line an access touches: kept past normal lines
+// (evict_last), ordinary (evict_normal), or dropped first (evict_first).
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_normal() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
 __device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* tmap, uint32_t bar, int c0,
                                             int c1, int c2, int c3) {
   asm volatile(
@@ -395,6 +423,33 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x for a pair of floats on the FMA and integer pipes, leaving the MUFU
+// unit (the softmax's bottleneck next to the tensor cores) to other pairs.
+// Range reduction: x = n + f, n = round-to-nearest(x) by adding and removing
+// 1.5 * 2^23, f = x - n in [-1/2, 1/2] exactly.  2^f = 1 + c1 f + c2 f^2 +
+// c3 f^3 with the coefficients that minimise the largest relative error on
+// [-1/2, 1/2] (a linear-programming minimax fit at 4001 points, p(0) = 1
+// exactly): relative error <= 1.02e-4, well below the bf16 rounding of P.
+// 2^n is a float built from its exponent field, (n + 127) << 23; x is
+// clamped to >= -127 first, so that -inf and anything below gives exactly 0
+// (the field is 0) and no input can wrap the field.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kRound = 12582912.f;   // 1.5 * 2^23
+  x.x = fmaxf(x.x, -127.f);
+  x.y = fmaxf(x.y, -127.f);
+  const float2 t = fadd2(x, make_float2(kRound, kRound));
+  const float2 n = fadd2(t, make_float2(-kRound, -kRound));
+  const float2 f = ffma2(n, make_float2(-1.f, -1.f), x);
+  float2 q = ffma2(make_float2(0.055009059607982635f, 0.055009059607982635f), f,
+                   make_float2(0.2422109693288803f, 0.2422109693288803f));
+  q = ffma2(q, f, make_float2(0.6932829022407532f, 0.6932829022407532f));
+  q = ffma2(q, f, make_float2(1.f, 1.f));
+  // t's low mantissa bits hold n, so (bits(t) << 23) == n << 23 (mod 2^32)
+  const float2 sc = make_float2(__int_as_float((__float_as_int(t.x) << 23) + 0x3F800000),
+                                __int_as_float((__float_as_int(t.y) << 23) + 0x3F800000));
+  return fmul2(q, sc);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -324,8 +324,9 @@ int attn_decode_split_kv(const void* q, const attn_kv_view* kv, float* partial_o
  * (strides, paging, lengths per sequence, fp8 codes, Dv != D).  out is
  * [B, Sq, Hq, Dv].  With seq_lens, q_offset is ignored and the Sq rows of
  * sequence b sit at positions len_b - Sq + s, as in attn_decode_split_kv.
- *   - D = Dv in {64, 128, 256}, bf16, unpaged, no seq_lens: the prefill
- *     kernel, reading K and V through the view's strides.
+ *   - D = Dv in {64, 128, 256}, or D = 192 with Dv = 128; bf16, unpaged, no
+ *     seq_lens: the prefill kernel, reading K and V through the view's
+ *     strides.
  *   - otherwise (D = Dv = 512, the pairs with Dv != D, paged, fp8 or
  *     seq_lens): the split-KV kernel with one split and the query rows cut
  *     into chunks per CTA, writing O and LSE directly, as attn_prefill does
