@@ -91,12 +91,21 @@ def kernel_source_sha(files):
 
 KERNEL_SOURCES = {
     "prefill": ["prefill_sm100.cu", "ptx.cuh"],
+    # prefill that runs on the split-KV kernel in query-chunk mode
+    "prefill_wide": ["decode_sm100.cu", "ptx.cuh"],
     "decode": ["decode_sm100.cu", "ptx.cuh"],
     "merge": ["merge.cu", "ptx.cuh"],
 }
 
 
-def profiled_traffic(kind, workload):
+def prefill_sources(w):
+    """Which kernel a prefill workload runs: the prefill kernel for D = Dv in
+    {64, 128, 256} or (192, 128), else the split-KV kernel."""
+    fast = (w.D == w.dv and w.D in (64, 128, 256)) or (w.D, w.dv) == (192, 128)
+    return "prefill" if fast and w.kv_dtype == "bf16" and not w.page_size else "prefill_wide"
+
+
+def profiled_traffic(kind, workload, sources=None):
     """DRAM bytes per launch from a committed ncu summary, or None when the
     summary is missing or the kernel source changed since it was taken."""
     path = os.path.join(ROOT, "profiles", f"{kind}_{workload}.md")
@@ -106,7 +115,7 @@ def profiled_traffic(kind, workload):
         return None
     m = re.search(r"traffic-bytes-per-launch:\s*([0-9]+)", text)
     s = re.search(r"kernel-source-sha256:\s*([0-9a-f]+)", text)
-    if not m or not s or s.group(1) != kernel_source_sha(KERNEL_SOURCES[kind]):
+    if not m or not s or s.group(1) != kernel_source_sha(KERNEL_SOURCES[sources or kind]):
         return None
     return int(m.group(1))
 
@@ -189,6 +198,13 @@ def make_runner(ga, w, device):
             else:
                 ga.prefill_kv(q, k, v, causal=w.causal, q_offset=w.q_offset, scale=w.scale, out=out, lse=lse,
                               sinks=sinks, **terms)
+        return step, 1, (q, k, v, out, lse)
+    if w.fused:
+        vv = k[..., :w.dv] if w.v_of_k else v
+
+        def step(mid=None):
+            ga.decode_fused(q, k, vv, w.num_splits, block_table=bt, causal=w.causal, q_offset=w.q_offset,
+                            scale=w.scale, out=out, lse=lse, sinks=sinks, **scales, **terms)
         return step, 1, (q, k, v, out, lse)
     po = torch.empty((w.num_splits, w.B, w.Sq, w.Hq, w.dv), dtype=torch.float32, device=device)
     pl = torch.empty((w.num_splits, w.B, w.Hq, w.Sq), dtype=torch.float32, device=device)
@@ -292,7 +308,10 @@ def time_e2e(ga, w, steps, warmup, dist_on, device):
         if w.kind == "prefill":
             (ga.prefill if w.dv == w.D else ga.prefill_kv)(dq, dk, dv, **kw)
         else:
-            (ga.decode if w.dv == w.D else ga.decode_kv)(dq, dk, dv, w.num_splits, **kw)
+            if w.fused:
+                ga.decode_fused(dq, dk, dv, w.num_splits, **kw)
+            else:
+                (ga.decode if w.dv == w.D else ga.decode_kv)(dq, dk, dv, w.num_splits, **kw)
         computed = ev()
         computed.record(s_comp)
         state["in_free"][b] = computed
@@ -401,7 +420,7 @@ def run_ours(args):
             roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                     "peak_source": f"{peak_src} copy bandwidth"}
         roof["kernel"] = kind
-        roof["traffic"] = profiled_traffic(kind, name)
+        roof["traffic"] = profiled_traffic(kind, name, prefill_sources(w) if kind == "prefill" else None)
         results[name] = {"value": value, "unit": unit, "ms_per_step": ms, "kernel_ms": ms_first,
                          "kernels_per_step": nk, "roofline": roof}
         del step

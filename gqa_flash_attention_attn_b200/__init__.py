@@ -25,6 +25,7 @@ __all__ = [
     "watchdog_selftest", "version", "ATTN_OK", "ATTN_ERR_INVALID_ARG", "ATTN_ERR_UNSUPPORTED",
     "ATTN_ERR_ALIGNMENT", "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT", "ATTN_ERR_TOO_LARGE", "decode_noalloc",
     "AttnOptions", "AttnKVView", "decode_split_kv", "decode_kv", "ATTN_FP8_E4M3", "prefill_kv",
+    "decode_fused",
 ]
 
 ATTN_OK = 0
@@ -59,6 +60,7 @@ _SIGNATURES = {
     "attn_merge_ex": (_i, [_vp, _vp, _vp, _vp] + [_i] * 6 + [_vp, _vp]),
     "attn_decode_split_kv": (_i, [_vp, _vp, _vp, _vp] + [_i] * 8 + [_f, _i, _vp, _vp]),
     "attn_prefill_kv": (_i, [_vp, _vp, _vp, _vp] + [_i] * 8 + [_f, _i, _vp, _vp]),
+    "attn_decode_fused": (_i, [_vp, _vp, _vp, _vp] + [_i] * 8 + [_f, _i, _i, _vp, _vp]),
 }
 
 
@@ -386,6 +388,43 @@ def decode_kv(q, k, v, num_splits, *, block_table=None, seq_lens=None, causal=Tr
                              softcap=softcap, alibi_max_bias=alibi_max_bias, window=window, mask=mask,
                              k_scale=k_scale, v_scale=v_scale)
     return merge(po, pl, out_dtype=out_dtype, out=out, lse=lse, stream=stream, sinks=sinks)
+
+
+def decode_fused(q, k, v, num_splits, *, block_table=None, seq_lens=None, causal=True, q_offset=0, scale=None,
+                 out_dtype=torch.bfloat16, out=None, lse=None, return_lse=True, stream=None, softcap=0.0,
+                 alibi_max_bias=0.0, sinks=None, window=0, mask=None, k_scale=None, v_scale=None):
+    """decode_kv in one launch: the key ranges of each (sequence, K/V head)
+    form a thread-block cluster that merges them in shared memory (n = the
+    largest power of two <= min(num_splits, 8) ranges).  Arguments as in
+    decode_kv; returns out [B, Sq, Hq, Dv] and lse [B, Hq, Sq]."""
+    _need(q, "q", torch.bfloat16, 4)
+    B, Sq, Hq, D = q.shape
+    view, Skv = _kv_view(k, v, block_table, seq_lens, k_scale, v_scale)
+    Hkv = k.shape[2]
+    if k.shape[3] != D:
+        raise ValueError("k head size does not match q")
+    if block_table is None and k.shape[0] != B:
+        raise ValueError("unpaged k/v must have B sequences")
+    if block_table is not None and block_table.shape[0] != B:
+        raise ValueError("block_table must have B rows")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    Dv = v.shape[3]
+    if out is None:
+        out = torch.empty((B, Sq, Hq, Dv), dtype=out_dtype, device=q.device)
+    else:
+        _need(out, "out", out.dtype, 4)
+    if out.dtype not in _OUT_CODES:
+        raise ValueError("out must be bf16 or fp32")
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    opt = _options(softcap, alibi_max_bias, sinks, window, Hq, mask, B, Sq, Skv)
+    st = library().attn_decode_fused(_ptr(q), ctypes.byref(view), _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Skv, D,
+                                     int(q_offset), int(bool(causal)), float(scale), int(num_splits),
+                                     _OUT_CODES[out.dtype], None if opt is None else ctypes.byref(opt),
+                                     _stream_ptr(stream))
+    _check("attn_decode_fused", st)
+    return out, lse
 
 
 def prefill_kv(q, k, v, *, block_table=None, seq_lens=None, causal=True, q_offset=0, scale=None,

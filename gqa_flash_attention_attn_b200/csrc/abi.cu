@@ -24,6 +24,7 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per pipeline 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr size_t kTwoCtaSmemLimit = 115712;  // two CTAs per SM
 constexpr size_t kOneCtaSmemLimit = 232448;  // the most one CTA may have
+constexpr int kMaxFusedCluster = 8;          // CTAs per cluster in attn_decode_fused
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -341,6 +342,118 @@ attn_kv_view contiguous_view(const void* k, const void* v, int Skv, int Hkv, int
   return kv;
 }
 
+// Split-KV decode over a view: partials (fused = false), or one launch whose
+// clusters merge the key ranges and write the final O and LSE (fused).
+int decode_run(const void* q, const attn_kv_view* kv, float* partial_out, float* partial_lse, void* out,
+               float* lse, int out_dtype, bool fused, int B, int Hq, int Hkv, int Sq, int Skv, int D, int q_offset,
+               int causal, float scale, int num_splits, const attn_options* opt, void* stream) {
+  if (kv == nullptr) return ATTN_ERR_INVALID_ARG;
+  // with per-sequence lengths q_offset is ignored (rows sit at len_b - Sq + s)
+  if (kv->seq_lens != nullptr) q_offset = 0;
+  int st = check_common(q, kv->k, kv->v, B, Hq, Hkv, Sq, Skv, D, q_offset, causal, scale);
+  if (st != ATTN_OK) return st;
+  gqa::LogitExt ext;
+  bool ext_on;
+  st = make_ext(opt, Hq, Sq, Skv, q_offset, causal, scale, fused, &ext, &ext_on);
+  if (st != ATTN_OK) return st;
+  if (fused) {
+    if (out == nullptr) return ATTN_ERR_INVALID_ARG;
+    if (out_dtype != ATTN_BF16 && out_dtype != ATTN_F32) return ATTN_ERR_INVALID_ARG;
+  } else if (partial_out == nullptr || partial_lse == nullptr) {
+    return ATTN_ERR_INVALID_ARG;
+  }
+  if (num_splits < 1 || num_splits > Skv || num_splits > 65535) return ATTN_ERR_INVALID_ARG;
+  bool fp8 = false;
+  st = check_view(kv, Skv, &fp8);
+  if (st != ATTN_OK) return st;
+  const int Dv = kv->head_dim_v != 0 ? kv->head_dim_v : D;
+  if (!gqa::decode_dims_supported(D, Dv, fp8)) return ATTN_ERR_UNSUPPORTED;
+  const int g = Hq / Hkv;
+  const long long R = (long long)g * Sq;
+  const long long RP = (R + 15) / 16 * 16;
+  if (RP * (2 + Dv / 128) > 256) return ATTN_ERR_UNSUPPORTED;  // TMEM: two S^T buffers + O^T
+  if (g > 256 || Sq > 256) return ATTN_ERR_UNSUPPORTED;  // TMA box extents
+  if ((long long)B * Hkv > 65535) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(q, 16)) return ATTN_ERR_ALIGNMENT;
+  if (fused) {
+    if (!aligned(out, 16) || (lse != nullptr && !aligned(lse, 4))) return ATTN_ERR_ALIGNMENT;
+  } else if (!aligned(partial_out, 16) || !aligned(partial_lse, 4)) {
+    return ATTN_ERR_ALIGNMENT;
+  }
+  // fused: key ranges per (b, kvh) = the cluster size, the largest power of
+  // two <= min(num_splits, 8).  Clusters of 16 ran slower in every measured
+  // shape (D512 decode 145 vs 117 us, verify 182 vs 111 us): fewer of them
+  // are resident at once than their CTA count suggests.
+  int nsplit = num_splits;
+  if (fused) {
+    nsplit = 1;
+    while (nsplit * 2 <= std::min(num_splits, kMaxFusedCluster)) nsplit *= 2;
+  }
+
+  gqa::DecodeParams p{};
+  p.part_out = fused ? nullptr : partial_out;
+  p.part_lse = fused ? lse : partial_lse;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Sq = Sq; p.Skv = Skv;
+  p.q_offset = q_offset; p.causal = causal;
+  p.g = g; p.R = (int)R; p.RP = (int)RP;
+  p.num_splits = nsplit;
+  p.chunk = (Skv + nsplit - 1) / nsplit;
+  // stage the additive mask per tile in shared memory (cp.async, 16-byte
+  // chunks) for up to 32 query rows when its rows are 16-byte aligned
+  p.mask_rows = (ext.mask != nullptr && Sq <= 32 && aligned(ext.mask, 16) && ext.mask_sb % 8 == 0 &&
+                 ext.mask_sr % 8 == 0)
+                    ? Sq
+                    : 0;
+  // ring slots: as many as keep two CTAs per SM, or, when even two slots
+  // leave room for one CTA only, as many as that CTA can hold
+  const size_t smem_limit =
+      gqa::decode_smem_bytes(D, p.RP, 2, p.mask_rows, fp8) <= kTwoCtaSmemLimit ? kTwoCtaSmemLimit : kOneCtaSmemLimit;
+  int nbuf = 2;
+  while (nbuf < gqa::decode_max_nbuf() && gqa::decode_smem_bytes(D, p.RP, nbuf + 1, p.mask_rows, fp8) <= smem_limit)
+    ++nbuf;
+  if (gqa::decode_smem_bytes(D, p.RP, nbuf, p.mask_rows, fp8) > kOneCtaSmemLimit) return ATTN_ERR_UNSUPPORTED;
+  p.nbuf = nbuf;
+  if (fused) {
+    // the merge's shared memory (X [RP][Dv] fp32, weights [16][RP], 1/L [RP])
+    // reuses the idle K/V ring
+    const long long need = RP * Dv * 4 + (long long)(gqa::decode_max_cluster() + 1) * RP * 4;
+    if (need > (long long)nbuf * (fp8 ? 16384 : 32768)) return ATTN_ERR_UNSUPPORTED;
+    p.group = 1;
+    p.obuf = 1;
+    p.cmerge = 1;
+    p.fout = out;
+    p.fout_bf16 = out_dtype == ATTN_BF16;
+  } else {
+    // Consecutive splits per CTA: enough that the CTAs fit the resident slots
+    // (two per SM when the shared memory allows) in one wave, at most 8.
+    const int nsm = sm_count();
+    if (nsm <= 0) return cuda_fail();
+    const long long slots =
+        (long long)nsm * (gqa::decode_smem_bytes(D, p.RP, nbuf, p.mask_rows, fp8) <= kTwoCtaSmemLimit ? 2 : 1);
+    const long long units = (long long)num_splits * B * Hkv;
+    long long grp = (units + slots - 1) / slots;
+    grp = std::min<long long>(std::min<long long>(grp, gqa::decode_max_group()), num_splits);
+    p.group = (int)std::max<long long>(grp, 1);
+    // two O^T buffers when split boundaries exist and two CTAs' TMEM still fits
+    p.obuf = (p.group > 1 && RP * (2 + 2 * (Dv / 128)) <= 256) ? 2 : 1;
+    p.fout = nullptr;
+  }
+  p.c2 = scale * kLog2e;
+  p.timeout_ns = kWaitLimitNs;
+  p.ext = ext;
+  view_params(kv, fp8, p);
+  p.qchunk = Sq;
+  p.nqc = 1;
+
+  p.status = status_ptr();
+  if (p.status == nullptr) return cuda_fail();
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q, D, Hq, Sq, B, 64, (uint32_t)g, (uint32_t)Sq, 1)) return cuda_fail();
+  if (!view_maps(kv, D, Dv, Hkv, Skv, B, fp8, &tk, &tv)) return cuda_fail();
+  const cudaStream_t st_ = static_cast<cudaStream_t>(stream);
+  return gqa::launch_decode_split(D, Dv, ext_on, fp8, tq, tk, tv, p, st_) == 0 ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
@@ -450,84 +563,15 @@ int attn_decode_split_ex(const void* q, const void* k, const void* v, float* par
 int attn_decode_split_kv(const void* q, const attn_kv_view* kv, float* partial_out, float* partial_lse, int B,
                          int Hq, int Hkv, int Sq, int Skv, int D, int q_offset, int causal, float scale,
                          int num_splits, const attn_options* opt, void* stream) {
-  if (kv == nullptr) return ATTN_ERR_INVALID_ARG;
-  // with per-sequence lengths q_offset is ignored (rows sit at len_b - Sq + s)
-  if (kv->seq_lens != nullptr) q_offset = 0;
-  int st = check_common(q, kv->k, kv->v, B, Hq, Hkv, Sq, Skv, D, q_offset, causal, scale);
-  if (st != ATTN_OK) return st;
-  gqa::LogitExt ext;
-  bool ext_on;
-  st = make_ext(opt, Hq, Sq, Skv, q_offset, causal, scale, false, &ext, &ext_on);
-  if (st != ATTN_OK) return st;
-  if (partial_out == nullptr || partial_lse == nullptr) return ATTN_ERR_INVALID_ARG;
-  if (num_splits < 1 || num_splits > Skv || num_splits > 65535) return ATTN_ERR_INVALID_ARG;
-  bool fp8 = false;
-  st = check_view(kv, Skv, &fp8);
-  if (st != ATTN_OK) return st;
-  const int Dv = kv->head_dim_v != 0 ? kv->head_dim_v : D;
-  if (!gqa::decode_dims_supported(D, Dv, fp8)) return ATTN_ERR_UNSUPPORTED;
-  const int g = Hq / Hkv;
-  const long long R = (long long)g * Sq;
-  const long long RP = (R + 15) / 16 * 16;
-  if (RP * (2 + Dv / 128) > 256) return ATTN_ERR_UNSUPPORTED;  // TMEM: two S^T buffers + O^T
-  if (g > 256 || Sq > 256) return ATTN_ERR_UNSUPPORTED;  // TMA box extents
-  if ((long long)B * Hkv > 65535) return ATTN_ERR_INVALID_ARG;
-  if (!aligned(q, 16) || !aligned(partial_out, 16)) return ATTN_ERR_ALIGNMENT;
-  if (!aligned(partial_lse, 4)) return ATTN_ERR_ALIGNMENT;
+  return decode_run(q, kv, partial_out, partial_lse, nullptr, nullptr, ATTN_BF16, false, B, Hq, Hkv, Sq, Skv, D,
+                    q_offset, causal, scale, num_splits, opt, stream);
+}
 
-  gqa::DecodeParams p{};
-  p.part_out = partial_out;
-  p.part_lse = partial_lse;
-  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Sq = Sq; p.Skv = Skv;
-  p.q_offset = q_offset; p.causal = causal;
-  p.g = g; p.R = (int)R; p.RP = (int)RP;
-  p.num_splits = num_splits;
-  p.chunk = (Skv + num_splits - 1) / num_splits;
-  // stage the additive mask per tile in shared memory (cp.async, 16-byte
-  // chunks) for up to 32 query rows when its rows are 16-byte aligned
-  p.mask_rows = (ext.mask != nullptr && Sq <= 32 && aligned(ext.mask, 16) && ext.mask_sb % 8 == 0 &&
-                 ext.mask_sr % 8 == 0)
-                    ? Sq
-                    : 0;
-  // ring slots: as many as keep two CTAs per SM, or, when even two slots
-  // leave room for one CTA only, as many as that CTA can hold
-  const size_t smem_limit =
-      gqa::decode_smem_bytes(D, p.RP, 2, p.mask_rows, fp8) <= kTwoCtaSmemLimit ? kTwoCtaSmemLimit : kOneCtaSmemLimit;
-  int nbuf = 2;
-  while (nbuf < gqa::decode_max_nbuf() && gqa::decode_smem_bytes(D, p.RP, nbuf + 1, p.mask_rows, fp8) <= smem_limit)
-    ++nbuf;
-  if (gqa::decode_smem_bytes(D, p.RP, nbuf, p.mask_rows, fp8) > kOneCtaSmemLimit) return ATTN_ERR_UNSUPPORTED;
-  p.nbuf = nbuf;
-  // Consecutive splits per CTA: enough that the CTAs fit the resident slots
-  // (two per SM when the shared memory allows) in one wave, at most 8.
-  {
-    const int nsm = sm_count();
-    if (nsm <= 0) return cuda_fail();
-    const long long slots =
-        (long long)nsm * (gqa::decode_smem_bytes(D, p.RP, nbuf, p.mask_rows, fp8) <= kTwoCtaSmemLimit ? 2 : 1);
-    const long long units = (long long)num_splits * B * Hkv;
-    long long grp = (units + slots - 1) / slots;
-    grp = std::min<long long>(std::min<long long>(grp, gqa::decode_max_group()), num_splits);
-    p.group = (int)std::max<long long>(grp, 1);
-    // two O^T buffers when split boundaries exist and two CTAs' TMEM still fits
-    p.obuf = (p.group > 1 && RP * (2 + 2 * (Dv / 128)) <= 256) ? 2 : 1;
-  }
-  p.c2 = scale * kLog2e;
-  p.timeout_ns = kWaitLimitNs;
-  p.ext = ext;
-  view_params(kv, fp8, p);
-  p.qchunk = Sq;
-  p.nqc = 1;
-  p.fout = nullptr;
-
-  p.status = status_ptr();
-  if (p.status == nullptr) return cuda_fail();
-  CUtensorMap tq, tk, tv;
-  if (!make_map(&tq, q, D, Hq, Sq, B, 64, (uint32_t)g, (uint32_t)Sq, 1)) return cuda_fail();
-  if (!view_maps(kv, D, Dv, Hkv, Skv, B, fp8, &tk, &tv)) return cuda_fail();
-  return gqa::launch_decode_split(D, Dv, ext_on, fp8, tq, tk, tv, p, static_cast<cudaStream_t>(stream)) == 0
-             ? ATTN_OK
-             : ATTN_ERR_CUDA;
+int attn_decode_fused(const void* q, const attn_kv_view* kv, void* out, float* lse, int B, int Hq, int Hkv, int Sq,
+                      int Skv, int D, int q_offset, int causal, float scale, int num_splits, int out_dtype,
+                      const attn_options* opt, void* stream) {
+  return decode_run(q, kv, nullptr, nullptr, out, lse, out_dtype, true, B, Hq, Hkv, Sq, Skv, D, q_offset, causal,
+                    scale, num_splits, opt, stream);
 }
 
 int attn_merge(const float* partial_out, const float* partial_lse, void* out, float* lse, int B, int Hq, int Sq,

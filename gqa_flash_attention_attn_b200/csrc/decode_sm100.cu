@@ -16,18 +16,26 @@
 // Every split publishes its normalised partial O and its log-sum-exp, also
 // when it has no visible key (lse = -inf, O = 0) ("Anbeeld/beellama.cpp PR
 // #149", Overview, ub>64 fix: every block publishes its (max, rowsum)); the
-// merge is attn_merge.
+// merge is attn_merge.  Or (cmerge) the splits of one (b, kvh) form a thread-
+// block cluster: each CTA leaves its (max, rowsum) and unnormalised O in its
+// own shared memory and every CTA merges a slice of the columns from all of
+// them over distributed shared memory, writing the final O and LSE, so no
+// partial reaches HBM and no second launch runs.
 //
 // The kernel is HBM-bound, so the pipeline keeps loads flowing while the
 // softmax works: S^T and P are double-buffered, the MMA thread computes
 // S_{j+1} before it waits for P_j, and the producer streams the ring in the
 // same order (K_0, K_1, V_0, K_2, V_1, ...).  Ring slots are 32 KB (128 keys
 // x 128 columns, two TMA boxes); two CTAs run per SM.
+#include <cooperative_groups.h>
+
 #include "kernels.h"
 #include "ptx.cuh"
 
 namespace gqa {
 namespace {
+
+namespace cg = cooperative_groups;
 
 constexpr int BN = 128;                        // keys per tile
 constexpr uint32_t BOX_BYTES = 128u * 128u;    // 128 rows x 64 bf16
@@ -38,6 +46,7 @@ constexpr int WARP_PRODUCER = 4;
 constexpr int WARP_MMA = 5;
 constexpr int MAX_NBUF = 6;
 constexpr int MAX_GROUP = 8;                   // consecutive splits per CTA
+constexpr int MAX_CLUSTER = 16;                // CTAs of one (b, kvh) merged in a cluster
 
 // One split of a CTA's group: its tiles are first .. first+nt-1 of the CTA's
 // tile stream; keys from kbase on a 128-key grid, the split ending at hi.
@@ -203,6 +212,59 @@ __device__ __noinline__ void write_partial_o(uint32_t taddr, int RP, int R, int 
   }
 }
 
+// The merge of a cluster's key ranges (cmerge).  CTA rank k holds, for rows
+// r < RP, m_k[r] and l_k[r] (log2 units; with fp8 P carries the factor 2^6
+// of the tile loop) and X_k[r][d] = v_scale * unnormalised O.  With M =
+// max_k m_k (and the sink logit, which joins only M and the denominator),
+// w_k = 2^(m_k - M), L = sum_k w_k l_k:  O = sum_k w_k X_k / L and LSE =
+// (M + log2 L) ln 2.  Rank c writes columns [c DV/n, (c+1) DV/n) of every
+// row, reading them from all n CTAs over distributed shared memory; rank 0
+// writes the LSE.  Threads t = 0..127 (named barrier 1).
+template <int DV, bool EXT, bool FP8>
+__device__ __noinline__ void cluster_merge(const DecodeParams& p, float* m_sm, float* l_sm, float* xbuf, float* wbuf,
+                                           int R, int RP, int g, int kvh, int b, int s0, int t) {
+  cg::cluster_group cl = cg::this_cluster();
+  const int n = (int)cl.num_blocks();
+  const int c = (int)cl.block_rank();
+  float* inv = wbuf + MAX_CLUSTER * RP;   // 1 / L per row, after the weights W[k][r]
+  const float off = FP8 ? 6.f : 0.f;
+  for (int r = t; r < RP; r += 128) {
+    float sink2 = -INFINITY;
+    if (EXT && p.ext.sinks != nullptr && r < R)
+      sink2 = __ldg(p.ext.sinks + kvh * g + (r % g)) * 1.4426950408889634f + off;
+    float M = sink2;
+    for (int k = 0; k < n; ++k) M = fmaxf(M, cl.map_shared_rank(m_sm, k)[r]);
+    float L = 0.f;
+    for (int k = 0; k < n; ++k) {
+      const float mk = cl.map_shared_rank(m_sm, k)[r];
+      const float w = (mk == -INFINITY) ? 0.f : ex2_approx(mk - M);
+      wbuf[k * RP + r] = w;
+      L = fmaf(w, cl.map_shared_rank(l_sm, k)[r], L);
+    }
+    if (sink2 != -INFINITY) L += ex2_approx(sink2 - M);
+    inv[r] = L > 0.f ? 1.f / L : 0.f;
+    if (c == 0 && r < R && p.part_lse != nullptr) {
+      const int s = s0 + r / g, h = kvh * g + (r % g);
+      p.part_lse[((size_t)b * p.Hq + h) * p.Sq + s] = L > 0.f ? (M + log2f(L) - off) * LN2 : -INFINITY;
+    }
+  }
+  named_bar_sync(1, 128);
+  const int cols = DV / n;
+  const int c0 = c * cols;
+  for (int idx = t; idx < R * cols; idx += 128) {
+    const int r = idx / cols, d = c0 + (idx - r * cols);
+    float acc = 0.f;
+    for (int k = 0; k < n; ++k) {
+      const float w = wbuf[k * RP + r];
+      if (w != 0.f) acc = fmaf(w, cl.map_shared_rank(xbuf, k)[(size_t)r * DV + d], acc);
+    }
+    const int s = s0 + r / g, h = kvh * g + (r % g);
+    const size_t o = (((size_t)b * p.Sq + s) * p.Hq + h) * DV + d;
+    if (p.fout_bf16) reinterpret_cast<__nv_bfloat16*>(p.fout)[o] = __float2bfloat16_rn(acc * inv[r]);
+    else reinterpret_cast<float*>(p.fout)[o] = acc * inv[r];
+  }
+}
+
 template <int DK, int DV, bool EXT, bool PAGED, bool FP8>
 __global__ void __launch_bounds__(THREADS, 2)
     decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -295,7 +357,7 @@ __global__ void __launch_bounds__(THREADS, 2)
     const int nt = eff_hi > eff_lo ? (eff_hi - kb + BN - 1) / BN : 0;
     if (threadIdx.x == 0) seg_sm[i] = SegInfo{T, nt, kb, hi, p.obuf == 2 ? (filled & 1) : 0, 0, 0, 0};
     filled += nt > 0 ? 1 : 0;
-    if (nt == 0) {
+    if (nt == 0 && !p.cmerge) {
       // No visible key in this split: publish (-inf, 0) for every row.
       const size_t so = (size_t)(sg0 + i) * p.B * p.Sq * p.Hq * D;
       const size_t sl = (size_t)(sg0 + i) * p.B * p.Hq * p.Sq;
@@ -314,7 +376,20 @@ __global__ void __launch_bounds__(THREADS, 2)
     }
     T += nt;
   }
-  if (T == 0) return;
+  float* xbuf = reinterpret_cast<float*>(gbase + L.off_ring);   // cmerge: X, then the weights
+  float* wbuf = xbuf + (size_t)RP * D;
+  if (T == 0) {
+    if (!p.cmerge) return;
+    // an empty key range still takes part in the cluster's merge, with weight 0
+    if (threadIdx.x < RP) {
+      m_sm[threadIdx.x] = -INFINITY;
+      l_sm[threadIdx.x] = 0.f;
+    }
+    cg::this_cluster().sync();
+    if (threadIdx.x < 128) cluster_merge<DV, EXT, FP8>(p, m_sm, l_sm, xbuf, wbuf, R, RP, g, kvh, b, s0, threadIdx.x);
+    cg::this_cluster().sync();
+    return;
+  }
   // split of stream tile j (empty splits share their successor's first tile);
   // for the rare boundary work, the per-tile paths use SegCursor
   auto seg_of = [&](int j) -> int {
@@ -851,7 +926,23 @@ __global__ void __launch_bounds__(THREADS, 2)
       if (pv_done(pend_last)) write_o(pend);
       else ok = false;
     }
-    if (ok) {
+    if (ok && p.cmerge) {
+      // the whole range is one split: leave (m, l) and v_scale * O^T (as
+      // X[row][d]) in shared memory for the cluster's merge; the ring is
+      // idle once the last P.V has completed
+      if (pv_done(T - 1)) {
+        for (int c = 0; c < KC; ++c) {
+          for (int q = 0; q < RP / 16; ++q) {
+            float v[16];
+            tmem_ld16(tmem + lane_off + TO(c, seg_sm[0].ob) + 16 * q, v);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) xbuf[(size_t)(16 * q + e) * D + c * 128 + t] = v[e] * vs;
+          }
+        }
+      } else {
+        ok = false;
+      }
+    } else if (ok) {
       stats(seg_of(T - 1));
       if (pv_done(T - 1)) write_o(seg_of(T - 1));
       else ok = false;
@@ -878,6 +969,11 @@ __global__ void __launch_bounds__(THREADS, 2)
     tc_fence_after();
     tmem_dealloc(tmem, tmem_cols);
   }
+  if (p.cmerge) {
+    cg::this_cluster().sync();   // every CTA's (m, l) and X are in place
+    if (threadIdx.x < 128) cluster_merge<DV, EXT, FP8>(p, m_sm, l_sm, xbuf, wbuf, R, RP, g, kvh, b, s0, threadIdx.x);
+    cg::this_cluster().sync();   // no CTA exits while a peer reads its shared memory
+  }
 }
 
 template <int DK, int DV, bool EXT, bool PAGED, bool FP8>
@@ -888,6 +984,31 @@ int launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
   if (e != cudaSuccess) return (int)e;
   dim3 grid((unsigned)((p.num_splits + p.group - 1) / p.group), (unsigned)(p.B * p.Hkv * p.nqc));
+  if (p.cmerge) {
+    // one cluster of num_splits CTAs per (b, kvh)
+    const int n = p.num_splits;
+    if (p.group != 1 || n < 1 || n > MAX_CLUSTER || (n & (n - 1)) != 0 || DV % n != 0) return (int)cudaErrorInvalidValue;
+    if (n > 8) {
+      e = cudaFuncSetAttribute(decode_split_kernel<DK, DV, EXT, PAGED, FP8>,
+                               cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e != cudaSuccess) return (int)e;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = L.total;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)n;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, decode_split_kernel<DK, DV, EXT, PAGED, FP8>, tq, tk, tv, p);
+    if (e != cudaSuccess) return (int)e;
+    return (int)cudaGetLastError();
+  }
   decode_split_kernel<DK, DV, EXT, PAGED, FP8><<<grid, THREADS, L.total, stream>>>(tq, tk, tv, p);
   return (int)cudaGetLastError();
 }
@@ -912,6 +1033,8 @@ size_t decode_smem_bytes(int D, int RP, int nbuf, int mask_rows, bool fp8) {
 int decode_max_nbuf() { return MAX_NBUF; }
 
 int decode_max_group() { return MAX_GROUP; }
+
+int decode_max_cluster() { return MAX_CLUSTER; }
 
 int launch_decode_split(int D, int Dv, bool ext, bool fp8, const CUtensorMap& tq, const CUtensorMap& tk,
                         const CUtensorMap& tv, const DecodeParams& p, cudaStream_t stream) {

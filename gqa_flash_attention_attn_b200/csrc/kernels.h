@@ -69,6 +69,10 @@ struct DecodeParams {
   // V is a view of K (same base and strides): K tiles stay in L2 (evict_last)
   // until their V reads, which then drop them (evict_first)
   int kv_shared;
+  // 1: the num_splits CTAs of one (b, kvh) run as one thread-block cluster
+  // and merge their key ranges through distributed shared memory: final O at
+  // fout and LSE at part_lse ([B, Hq, Sq]), no partials (group must be 1)
+  int cmerge;
 };
 
 struct MergeParams {
@@ -93,6 +97,7 @@ int launch_decode_split(int D, int Dv, bool ext, bool fp8, const CUtensorMap& tq
 bool decode_dims_supported(int D, int Dv, bool fp8);
 size_t decode_smem_bytes(int D, int RP, int nbuf, int mask_rows, bool fp8);
 int decode_max_group();
+int decode_max_cluster();
 int launch_merge(const MergeParams& p, cudaStream_t stream);
 int launch_watchdog_selftest(int* status, unsigned long long limit_ns, cudaStream_t stream);
 

@@ -51,6 +51,9 @@ class Workload:
     # holds both, as for multi-head latent attention)
     Dv: int = 0
     v_of_k: bool = False
+    # decode: one launch whose thread-block clusters merge the key ranges
+    # (num_splits -> the largest power of two <= min(num_splits, 8) ranges)
+    fused: bool = False
 
     @property
     def dv(self) -> int:
@@ -161,6 +164,14 @@ WORKLOADS = {
         "paged_decode_d512_p64", "decode", B=16, Hq=16, Hkv=1, Sq=1, Skv=16384, D=512,
         q_offset=16383, causal=True, out_dtype="bf16", num_splits=32, page_size=64,
         note="the D512 split-KV decode over a paged cache: 64-key pages in scattered order"),
+    "split_kv_decode_d512_fused": Workload(
+        "split_kv_decode_d512_fused", "decode", B=16, Hq=16, Hkv=1, Sq=1, Skv=16384, D=512,
+        q_offset=16383, causal=True, out_dtype="bf16", num_splits=8, fused=True,
+        note="the D512 decode in one launch: 8 key ranges per sequence merged inside an 8-CTA cluster"),
+    "spec_verify_decode_d128_fused": Workload(
+        "spec_verify_decode_d128_fused", "decode", B=4, Hq=32, Hkv=8, Sq=8, Skv=32768, D=128,
+        q_offset=32760, causal=True, out_dtype="bf16", num_splits=8, fused=True,
+        note="the verify decode in one launch: 8 key ranges per (sequence, K/V head) merged in a cluster"),
     "mla_decode_d576_v512": Workload(
         "mla_decode_d576_v512", "decode", B=16, Hq=16, Hkv=1, Sq=1, Skv=16384, D=576, Dv=512, v_of_k=True,
         q_offset=16383, causal=True, out_dtype="bf16", num_splits=32,

@@ -320,6 +320,30 @@ int attn_decode_split_kv(const void* q, const attn_kv_view* kv, float* partial_o
                          float scale, int num_splits, const attn_options* opt, void* stream);
 
 /*
+ * Split-KV decode and merge in ONE launch ("flash decoding" with the combine
+ * fused into the split kernel): the key ranges of one (sequence, K/V head)
+ * run as one thread-block cluster of n CTAs; each CTA leaves its (max,
+ * rowsum) and unnormalised O in its shared memory and every CTA merges a
+ * slice of the output columns from all n over distributed shared memory
+ * (the last-CTA combine of "Anbeeld/beellama.cpp PR #149", review of the
+ * combine kernel for parallel_blocks > 1, done by all CTAs at once).  No
+ * partial goes to HBM, no workspace is needed.
+ *   n            the largest power of two <= min(num_splits, 8): key range
+ *                k of n covers keys [k c, (k+1) c), c = ceil(len / n)
+ *                (rounded up to 128 when paged); the result is the attention
+ *                of attn_decode_split_kv + attn_merge_ex with n splits.  It
+ *                pays off when B * Hkv * n fills the GPU (two CTAs per SM)
+ *   out, lse     as attn_merge_ex's: out [B, Sq, Hq, Dv] (out_dtype), lse
+ *                [B, Hq, Sq] fp32 or NULL; opt->sinks apply here
+ *   limits       those of attn_decode_split_kv, and the merge's shared memory
+ *                (RP x Dv fp32 plus 17 RP floats) must fit the K/V ring the
+ *                launch gets, else ATTN_ERR_UNSUPPORTED
+ */
+int attn_decode_fused(const void* q, const attn_kv_view* kv, void* out, float* lse, int B, int Hq, int Hkv,
+                      int Sq, int Skv, int D, int q_offset, int causal, float scale, int num_splits,
+                      int out_dtype, const attn_options* opt, void* stream);
+
+/*
  * Prefill over a K/V view: attn_prefill_ex with K and V described by *kv
  * (strides, paging, lengths per sequence, fp8 codes, Dv != D).  out is
  * [B, Sq, Hq, Dv].  With seq_lens, q_offset is ignored and the Sq rows of

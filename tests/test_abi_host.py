@@ -280,3 +280,28 @@ def test_prefill_kv_rejects(lib, view, kw, status):
 def test_prefill_kv_rejects_null_view(lib):
     assert lib.attn_prefill_kv(P, None, P2, P2, 1, 8, 1, 128, 128, 128, 0, 1, 0.08, 0, None, None) == \
         ga.ATTN_ERR_INVALID_ARG
+
+
+def _kv_fused(lib, view=None, opt=None, **kw):
+    a = dict(q=P, out=P2, lse=P2, B=2, Hq=16, Hkv=1, Sq=1, Skv=1024, D=512, q_offset=1023, causal=1,
+             scale=0.0441941738, S=16, out_dtype=0)
+    a.update(kw)
+    v = _view(view)
+    return lib.attn_decode_fused(a["q"], ctypes.byref(v), a["out"], a["lse"], a["B"], a["Hq"], a["Hkv"], a["Sq"],
+                                 a["Skv"], a["D"], a["q_offset"], a["causal"], a["scale"], a["S"], a["out_dtype"],
+                                 None if opt is None else ctypes.byref(opt), None)
+
+
+@pytest.mark.parametrize("view,kw,status", [
+    (dict(k=None), {}, ga.ATTN_ERR_INVALID_ARG),
+    ({}, dict(out=None), ga.ATTN_ERR_INVALID_ARG),
+    ({}, dict(out_dtype=7), ga.ATTN_ERR_INVALID_ARG),
+    ({}, dict(S=0), ga.ATTN_ERR_INVALID_ARG),
+    ({}, dict(D=64), ga.ATTN_ERR_UNSUPPORTED),
+    ({}, dict(out=ctypes.c_void_p(0x20008)), ga.ATTN_ERR_ALIGNMENT),
+    ({}, dict(lse=ctypes.c_void_p(0x20002)), ga.ATTN_ERR_ALIGNMENT),
+    (dict(stride_token=128, stride_head=128, stride_seq=128 * 1024), dict(D=128, Hq=64, Hkv=1, Sq=2),
+     ga.ATTN_ERR_UNSUPPORTED),   # 128 rows x (2 + 1) TMEM column groups > 256
+])
+def test_decode_fused_rejects(lib, view, kw, status):
+    assert _kv_fused(lib, view, **kw) == status
