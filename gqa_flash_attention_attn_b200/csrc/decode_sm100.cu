@@ -265,7 +265,8 @@ __device__ __noinline__ void cluster_merge(const DecodeParams& p, float* m_sm, f
   }
 }
 
-template <int DK, int DV, bool EXT, bool PAGED, bool FP8>
+// CM: the cluster merge (cmerge) variant; the plain kernels carry none of its code.
+template <int DK, int DV, bool EXT, bool PAGED, bool FP8, bool CM>
 __global__ void __launch_bounds__(THREADS, 2)
     decode_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
@@ -357,7 +358,7 @@ __global__ void __launch_bounds__(THREADS, 2)
     const int nt = eff_hi > eff_lo ? (eff_hi - kb + BN - 1) / BN : 0;
     if (threadIdx.x == 0) seg_sm[i] = SegInfo{T, nt, kb, hi, p.obuf == 2 ? (filled & 1) : 0, 0, 0, 0};
     filled += nt > 0 ? 1 : 0;
-    if (nt == 0 && !p.cmerge) {
+    if (nt == 0 && !CM) {
       // No visible key in this split: publish (-inf, 0) for every row.
       const size_t so = (size_t)(sg0 + i) * p.B * p.Sq * p.Hq * D;
       const size_t sl = (size_t)(sg0 + i) * p.B * p.Hq * p.Sq;
@@ -379,15 +380,17 @@ __global__ void __launch_bounds__(THREADS, 2)
   float* xbuf = reinterpret_cast<float*>(gbase + L.off_ring);   // cmerge: X, then the weights
   float* wbuf = xbuf + (size_t)RP * D;
   if (T == 0) {
-    if (!p.cmerge) return;
-    // an empty key range still takes part in the cluster's merge, with weight 0
-    if (threadIdx.x < RP) {
-      m_sm[threadIdx.x] = -INFINITY;
-      l_sm[threadIdx.x] = 0.f;
+    if constexpr (CM) {
+      // an empty key range still takes part in the cluster's merge, with weight 0
+      if (threadIdx.x < RP) {
+        m_sm[threadIdx.x] = -INFINITY;
+        l_sm[threadIdx.x] = 0.f;
+      }
+      cg::this_cluster().sync();
+      if (threadIdx.x < 128)
+        cluster_merge<DV, EXT, FP8>(p, m_sm, l_sm, xbuf, wbuf, R, RP, g, kvh, b, s0, threadIdx.x);
+      cg::this_cluster().sync();
     }
-    cg::this_cluster().sync();
-    if (threadIdx.x < 128) cluster_merge<DV, EXT, FP8>(p, m_sm, l_sm, xbuf, wbuf, R, RP, g, kvh, b, s0, threadIdx.x);
-    cg::this_cluster().sync();
     return;
   }
   // split of stream tile j (empty splits share their successor's first tile);
@@ -926,7 +929,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       if (pv_done(pend_last)) write_o(pend);
       else ok = false;
     }
-    if (ok && p.cmerge) {
+    if (CM && ok) {
       // the whole range is one split: leave (m, l) and v_scale * O^T (as
       // X[row][d]) in shared memory for the cluster's merge; the ring is
       // idle once the last P.V has completed
@@ -969,7 +972,7 @@ __global__ void __launch_bounds__(THREADS, 2)
     tc_fence_after();
     tmem_dealloc(tmem, tmem_cols);
   }
-  if (p.cmerge) {
+  if constexpr (CM) {
     cg::this_cluster().sync();   // every CTA's (m, l) and X are in place
     if (threadIdx.x < 128) cluster_merge<DV, EXT, FP8>(p, m_sm, l_sm, xbuf, wbuf, R, RP, g, kvh, b, s0, threadIdx.x);
     cg::this_cluster().sync();   // no CTA exits while a peer reads its shared memory
@@ -980,17 +983,17 @@ template <int DK, int DV, bool EXT, bool PAGED, bool FP8>
 int launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
              const DecodeParams& p, cudaStream_t stream) {
   const Layout L(DK, p.RP, p.nbuf, p.mask_rows, FP8);
-  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<DK, DV, EXT, PAGED, FP8>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
-  if (e != cudaSuccess) return (int)e;
   dim3 grid((unsigned)((p.num_splits + p.group - 1) / p.group), (unsigned)(p.B * p.Hkv * p.nqc));
+  cudaError_t e;
   if (p.cmerge) {
     // one cluster of num_splits CTAs per (b, kvh)
+    auto kern = decode_split_kernel<DK, DV, EXT, PAGED, FP8, true>;
     const int n = p.num_splits;
     if (p.group != 1 || n < 1 || n > MAX_CLUSTER || (n & (n - 1)) != 0 || DV % n != 0) return (int)cudaErrorInvalidValue;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
+    if (e != cudaSuccess) return (int)e;
     if (n > 8) {
-      e = cudaFuncSetAttribute(decode_split_kernel<DK, DV, EXT, PAGED, FP8>,
-                               cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
       if (e != cudaSuccess) return (int)e;
     }
     cudaLaunchConfig_t cfg = {};
@@ -1005,11 +1008,14 @@ int launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, decode_split_kernel<DK, DV, EXT, PAGED, FP8>, tq, tk, tv, p);
+    e = cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, p);
     if (e != cudaSuccess) return (int)e;
     return (int)cudaGetLastError();
   }
-  decode_split_kernel<DK, DV, EXT, PAGED, FP8><<<grid, THREADS, L.total, stream>>>(tq, tk, tv, p);
+  auto kern = decode_split_kernel<DK, DV, EXT, PAGED, FP8, false>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
+  if (e != cudaSuccess) return (int)e;
+  kern<<<grid, THREADS, L.total, stream>>>(tq, tk, tv, p);
   return (int)cudaGetLastError();
 }
 
