@@ -860,10 +860,21 @@ __global__ void __launch_bounds__(THREADS, 2)
             const int r = 16 * q + e;
             float pv = EXT ? ex2_approx(v[e]) : ex2_approx(fmaf(v[e], c2, -msub_sm[r]));
             if (!full && !visible(r)) pv = 0.f;
-            if constexpr (!FP8)
-              *reinterpret_cast<__nv_bfloat16*>(pcol + (size_t)r * 128 + ((chunk16 ^ (r & 7)) << 4)) =
-                  __float2bfloat16_rn(pv);
             v[e] = pv;
+          }
+          if constexpr (!FP8) {
+            // bf16 P, one 32-bit word (keys t & ~1, t | 1) per store: for
+            // each pair of rows the even lane writes the even row and the odd
+            // lane the odd row, each taking its neighbour's value by shuffle
+            const bool odd = (t & 1) != 0;
+            uint8_t* pword = pcol - (size_t)(tt & 1) * 2;
+#pragma unroll
+            for (int e = 0; e < 16; e += 2) {
+              const float other = __shfl_xor_sync(0xffffffffu, odd ? v[e] : v[e + 1], 1);
+              const int r = 16 * q + e + (odd ? 1 : 0);
+              const uint32_t w = odd ? pack_bf16x2(other, v[e + 1]) : pack_bf16x2(v[e], other);
+              *reinterpret_cast<uint32_t*>(pword + (size_t)r * 128 + ((chunk16 ^ (r & 7)) << 4)) = w;
+            }
           }
           if constexpr (FP8) {
             // P as hi + lo e4m3 planes (row r: 128 keys, one 128-byte
