@@ -878,21 +878,51 @@ __global__ void __launch_bounds__(THREADS, 2)
           }
           if constexpr (FP8) {
             // P as hi + lo e4m3 planes (row r: 128 keys, one 128-byte
-            // swizzled row per plane), two rows per conversion
-            uint8_t* p8 = gbase + PB(sb) + (t & 15);
+            // swizzled row per plane).  A lane holds one key of 4 rows; a
+            // 4 x 4 byte transpose in each quad of lanes (two shuffle stages,
+            // both planes in one word) gives lane j the 4 keys of row e + j,
+            // so every store is a 32-bit word.
+            const int j4 = t & 3;
+            uint8_t* p8 = gbase + PB(sb) + ((t & 15) & ~3);
             const int ck = t >> 4;
 #pragma unroll
-            for (int e = 0; e < 16; e += 2) {
-              const int r = 16 * q + e;
-              const uint32_t h = e4m3x2_from(v[e], v[e + 1]);
-              const float2 bk = e4m3x2_value(h);
-              const uint32_t l = e4m3x2_from(v[e] - bk.x, v[e + 1] - bk.y);
-              const uint32_t o0 = (uint32_t)r * 128u + ((uint32_t)(ck ^ (r & 7)) << 4);
-              const uint32_t o1 = (uint32_t)(r + 1) * 128u + ((uint32_t)(ck ^ ((r + 1) & 7)) << 4);
-              p8[o0] = (uint8_t)h;
-              p8[o1] = (uint8_t)(h >> 8);
-              p8[(uint32_t)RP * 128u + o0] = (uint8_t)l;
-              p8[(uint32_t)RP * 128u + o1] = (uint8_t)(l >> 8);
+            for (int e = 0; e < 16; e += 4) {
+              const uint32_t h01 = e4m3x2_from(v[e], v[e + 1]);
+              const uint32_t h23 = e4m3x2_from(v[e + 2], v[e + 3]);
+              const float2 b01 = e4m3x2_value(h01);
+              const float2 b23 = e4m3x2_value(h23);
+              const uint32_t l01 = e4m3x2_from(v[e] - b01.x, v[e + 1] - b01.y);
+              const uint32_t l23 = e4m3x2_from(v[e + 2] - b23.x, v[e + 3] - b23.y);
+              uint32_t H = h01 | (h23 << 16), Lw = l01 | (l23 << 16);   // byte i: row e + i
+              // stage 1 (lanes j, j ^ 1): even lanes end with rows e, e+2 and
+              // odd lanes with rows e+1, e+3, each for keys (j & ~1, j | 1)
+              {
+                const uint32_t snd = (j4 & 1) ? __byte_perm(H, Lw, 0x6420) : __byte_perm(H, Lw, 0x7531);
+                const uint32_t rcv = __shfl_xor_sync(0xffffffffu, snd, 1);
+                if (j4 & 1) {
+                  H = __byte_perm(H, rcv, 0x3514);
+                  Lw = __byte_perm(Lw, rcv, 0x3716);
+                } else {
+                  H = __byte_perm(H, rcv, 0x5240);
+                  Lw = __byte_perm(Lw, rcv, 0x7260);
+                }
+              }
+              // stage 2 (lanes j, j ^ 2): lane j ends with row e + j, keys 0-3
+              {
+                const uint32_t snd = (j4 & 2) ? __byte_perm(H, Lw, 0x5410) : __byte_perm(H, Lw, 0x7632);
+                const uint32_t rcv = __shfl_xor_sync(0xffffffffu, snd, 2);
+                if (j4 & 2) {
+                  H = __byte_perm(H, rcv, 0x3254);
+                  Lw = __byte_perm(Lw, rcv, 0x3276);
+                } else {
+                  H = __byte_perm(H, rcv, 0x5410);
+                  Lw = __byte_perm(Lw, rcv, 0x7610);
+                }
+              }
+              const int r = 16 * q + e + j4;
+              const uint32_t o = (uint32_t)r * 128u + ((uint32_t)(ck ^ (r & 7)) << 4);
+              *reinterpret_cast<uint32_t*>(p8 + o) = H;
+              *reinterpret_cast<uint32_t*>(p8 + (uint32_t)RP * 128u + o) = Lw;
             }
           }
           const float s = warp_reduce16<false>(v, lane);
