@@ -8,6 +8,21 @@ an error.
 
 Layouts: q/out [B, Sq, Hq, D], k/v [B, Skv, Hkv, D] (bf16, contiguous),
 lse [B, Hq, Sq] fp32, partials [S, B, Sq, Hq, D] and [S, B, Hq, Sq] fp32.
+
+Calls (each returns torch tensors it allocated unless out/lse are given):
+  prefill(q, k, v)                      one launch; D 64, 128, 256, 512
+  decode_split / merge / decode         split-KV partials, their LSE merge,
+                                        or both (two launches)
+  decode_fused(q, k, v, num_splits)     split and merge in one launch
+  decode_split_kv / decode_kv / prefill_kv
+                                        over strided or paged K/V (block_table),
+                                        lengths per sequence (seq_lens), fp8
+                                        e4m3 K/V (k_scale, v_scale) and V
+                                        narrower than K (576/512, 320/256,
+                                        192/128)
+  decode_noalloc                        decode + merge with no workspace
+Optional logit terms on every call: softcap, alibi_max_bias, sinks (fp32
+[Hq]), window, mask (bf16 [B or 1, Sq, Skv]).
 """
 from __future__ import annotations
 
