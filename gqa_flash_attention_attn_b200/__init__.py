@@ -21,8 +21,9 @@ Calls (each returns torch tensors it allocated unless out/lse are given):
                                         narrower than K (576/512, 320/256,
                                         192/128)
   decode_noalloc                        decode + merge with no workspace
-Optional logit terms on every call: softcap, alibi_max_bias, sinks (fp32
-[Hq]), window, mask (bf16 [B or 1, Sq, Skv]).
+Optional logit terms: softcap, alibi_max_bias, window, mask (bf16 [B or 1,
+Sq, Skv]) on every attention call; sinks (fp32 [Hq]) on the calls that
+produce the final O (prefill*, merge, decode*, decode_fused).
 """
 from __future__ import annotations
 
