@@ -316,7 +316,11 @@ __global__ void __launch_bounds__(THREADS, 2)
   const int BAR_Q8 = BAR_S0 + 7;         // fp8: Q planes written
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bkv = blockIdx.y / p.nqc, qc = blockIdx.y - bkv * p.nqc;
+  const int bkv = blockIdx.y / p.nqc;
+  // query chunks in reverse: with a causal mask the last chunks see the most
+  // keys, and CTAs launch in grid order, so the longest start first
+  const int qc_in = blockIdx.y - bkv * p.nqc;
+  const int qc = p.causal ? p.nqc - 1 - qc_in : qc_in;
   const int b = bkv / p.Hkv, kvh = bkv % p.Hkv;
   const int s0 = qc * p.qchunk;               // this CTA's first query row
   const int Sqc = min(p.qchunk, p.Sq - s0);   // and its query rows
