@@ -458,7 +458,7 @@ int decode_run(const void* q, const attn_kv_view* kv, float* partial_out, float*
 
 extern "C" {
 
-int attn_version(void) { return 0x000400; }
+int attn_version(void) { return 0x000500; }
 
 const char* attn_status_string(int status) {
   switch (status) {

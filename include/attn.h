@@ -363,7 +363,7 @@ int attn_prefill_kv(const void* q, const attn_kv_view* kv, void* out, float* lse
                     int Sq, int Skv, int D, int q_offset, int causal, float scale, int out_dtype,
                     const attn_options* opt, void* stream);
 
-/* Library version, e.g. 0x000400 for 0.4.0. */
+/* Library version, e.g. 0x000500 for 0.5.0. */
 int attn_version(void);
 
 #ifdef __cplusplus

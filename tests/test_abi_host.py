@@ -22,7 +22,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert ga.version() == 0x000400
+    assert ga.version() == 0x000500
     assert ga.status_string(ga.ATTN_OK) == "ok"
     assert ga.status_string(ga.ATTN_ERR_TIMEOUT) == "pipeline wait timed out"
     assert ga.status_string(12345) == "unknown status"
