@@ -4,12 +4,16 @@
 
 One step is one launch sequence of the attention path over one batch of
 synthetic, seeded bf16 inputs already resident in HBM.  The headline workload
-is the GQA causal prefill (B1 Hq32 Hkv8 Sq=Skv=4096 D128); the other four
-workloads (tiny prefill, prefill at depth with D256, D512 split-KV decode with
-its LSE merge, 8-row speculative-verify decode) are timed the same way and
-reported under "workloads".  L2 is flushed between timed steps (a 256 MiB
-write, then a 256 MiB read so no dirty lines are left behind); the flush is
-outside the timed events.
+is the GQA causal prefill (B1 Hq32 Hkv8 Sq=Skv=4096 D128).  All five base
+workloads (tiny prefill, the headline, prefill at depth with D256, D512
+split-KV decode with its LSE merge, 8-row speculative-verify decode) are timed
+the same way and reported under "configs", the last key of the JSON line; the
+widened workloads (logit terms, masks, windows, fp8, paged, fused, latent
+cache, D512 prefill) come before it under "workloads".  Each carries the
+roofline fraction of its whole step (a decode step is the split kernel plus
+the merge) and, as kernel_frac, that of its first kernel alone.  L2 is
+flushed between timed steps (a 256 MiB write, then a 256 MiB read so no dirty
+lines are left behind); the flush is outside the timed events.
 
 Under torchrun (N > 1) every rank runs the same problems independently (the
 path does not shard: replicas only); times are the max over ranks and the
@@ -37,6 +41,11 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 HEADLINE = "gqa_causal_prefill_4k_d128"
+# The five base workloads (tiny prefill, headline prefill, prefill at depth,
+# D512 split-KV decode, 8-row verify decode): reported last in the JSON line,
+# after the widened workloads, so that a reader of its tail sees all five.
+BASE_CONFIGS = ["tiny_causal_gqa_prefill", "gqa_causal_prefill_4k_d128", "prefill_at_depth_d256",
+                "split_kv_decode_d512", "spec_verify_decode_d128"]
 METRIC = "prefill TFLOP/s and decode KV GB/s on 1 B200, as % of roofline"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
@@ -380,6 +389,29 @@ def cpu_baseline(w, seconds):
             "sample": f"{n} random (b,h,s) rows of {w.name}, {fl / 1e9:.1f} GFLOP fp64 in {dt:.1f} s"}
 
 
+def _sig(x, digits=4):
+    return float(f"{x:.{digits}g}") if isinstance(x, float) else x
+
+
+def compact(r):
+    """One workload's figures for the JSON line: per step value and time,
+    the roofline fraction of the step and of its first kernel, and the ncu
+    DRAM bytes of that kernel (or null)."""
+    roof = r["roofline"]
+    return {"value": _sig(r["value"]), "unit": r["unit"], "ms_per_step": _sig(r["ms_per_step"]),
+            "kernel_ms": _sig(r["kernel_ms"]), "roofline_frac": _sig(roof["frac"], 3),
+            "kernel_frac": _sig(roof["kernel_frac"], 3), "bound": roof["bound"], "traffic": roof["traffic"]}
+
+
+def workload_config(w, world):
+    """The config object of the JSON line for workload w (same keys in both arms)."""
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Sq": w.Sq, "Skv": w.Skv, "D": w.D,
+            "q_offset": w.q_offset, "causal": w.causal, "out": w.out_dtype,
+            "num_splits": w.num_splits if w.kind == "decode" else None,
+            "l2": "flushed between timed steps (256 MiB write, then 256 MiB read)",
+            "parallelism": f"replicas x{world}"}
+
+
 def run_ours(args):
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -411,14 +443,19 @@ def run_ours(args):
         unit, work = workload_metric(w)
         value, ms = replica_throughput(work, ms, dist_on, device)
         ms_first = max_over_ranks(ms_first, dist_on, device)
+        # The fraction is for the whole step (for a decode: the split kernel
+        # and the merge); kernel_frac is the first kernel alone.
         if w.kind == "prefill":
-            kind, achieved = "prefill", w.flops() / (ms_first / 1e3) / 1e12
+            kind, achieved = "prefill", w.flops() / (ms / 1e3) / 1e12
             roof = {"bound": "tensor", "achieved": achieved, "peak": tf_burst, "unit": "TFLOP/s",
                     "frac": achieved / tf_burst, "peak_source": f"{peak_src} bf16 burst"}
+            kernel_frac = w.flops() / (ms_first / 1e3) / 1e12 / tf_burst
         else:
-            kind, achieved = "decode", w.io_bytes() / (ms_first / 1e3) / 1e9
+            kind, achieved = "decode", w.io_bytes() / (ms / 1e3) / 1e9
             roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                     "peak_source": f"{peak_src} copy bandwidth"}
+            kernel_frac = w.io_bytes() / (ms_first / 1e3) / 1e9 / hbm
+        roof["kernel_frac"] = kernel_frac
         roof["kernel"] = kind
         roof["traffic"] = profiled_traffic(kind, name, prefill_sources(w) if kind == "prefill" else None)
         results[name] = {"value": value, "unit": unit, "ms_per_step": ms, "kernel_ms": ms_first,
@@ -444,22 +481,17 @@ def run_ours(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded iid N(0,1) cast to bf16)",
-        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Sq": w.Sq, "Skv": w.Skv, "D": w.D,
-                   "q_offset": w.q_offset, "causal": w.causal, "out": w.out_dtype,
-                   "num_splits": w.num_splits if w.kind == "decode" else None,
-                   "l2": "flushed between timed steps (256 MiB write, then 256 MiB read)", "parallelism": f"replicas x{world}"},
+        "config": workload_config(w, world),
         "roofline": head["roofline"],
         "e2e": {"value": world * work / (e2e_ms / 1e3), "unit": unit, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": head["kernels_per_step"] * args.steps,
         "clocks": clocks,
-        "workloads": {n: {k2: r[k2] for k2 in ("value", "unit", "ms_per_step", "kernel_ms")} |
-                      {"roofline_frac": r["roofline"]["frac"], "bound": r["roofline"]["bound"],
-                       "traffic": r["roofline"]["traffic"]}
-                      for n, r in results.items()},
+        "workloads": {n: compact(r) for n, r in results.items() if n not in BASE_CONFIGS},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+    line["configs"] = {n: compact(results[n]) for n in BASE_CONFIGS if n in results}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist_on:
@@ -503,8 +535,7 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded iid N(0,1) cast to bf16)",
-        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Sq": w.Sq, "Skv": w.Skv, "D": w.D,
-                   "q_offset": w.q_offset, "causal": w.causal},
+        "config": workload_config(w, world),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                          "sample": f"{n} random (b,h,s) rows of {w.name} per step"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

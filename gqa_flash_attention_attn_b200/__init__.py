@@ -497,14 +497,31 @@ def decode_noalloc(q, k, v, num_splits, *, causal=True, q_offset=0, scale=None, 
     _need(v, "v", torch.bfloat16, 4)
     B, Sq, Hq, D = q.shape
     _, Skv, Hkv, _ = k.shape
+    if v.shape != k.shape or k.shape[0] != B or k.shape[3] != D:
+        raise ValueError("k/v shapes do not match q")
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     if out is None:
         out = torch.empty((B, Sq, Hq, D), dtype=out_dtype, device=q.device)
+    else:
+        if out.dtype not in _OUT_CODES:
+            raise ValueError("out must be bf16 or fp32")
+        _need(out, "out", out.dtype, 4)
+        if tuple(out.shape) != (B, Sq, Hq, D):
+            raise ValueError(f"out must be [{B}, {Sq}, {Hq}, {D}]")
     if lse is None and return_lse:
         lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
-    st = library().attn_decode_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Skv, D,
-                                       int(q_offset), int(bool(causal)), float(scale), int(num_splits),
-                                       _OUT_CODES[out.dtype], _stream_ptr(stream))
+    elif lse is not None:
+        _need(lse, "lse", torch.float32, 3)
+        if tuple(lse.shape) != (B, Hq, Sq):
+            raise ValueError(f"lse must be [{B}, {Hq}, {Sq}]")
+    for t, n in ((k, "k"), (v, "v"), (out, "out"), (lse, "lse")):
+        if t is not None and t.device != q.device:
+            raise ValueError(f"{n} must be on {q.device}, like q")
+    # the library looks up its scratch array on the current device: make it q's
+    with torch.cuda.device(q.device):
+        st = library().attn_decode_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Skv,
+                                           D, int(q_offset), int(bool(causal)), float(scale), int(num_splits),
+                                           _OUT_CODES[out.dtype], _stream_ptr(stream))
     _check("attn_decode_noalloc", st)
     return out, lse

@@ -236,8 +236,8 @@ int prefill_wide(const void* q, const attn_kv_view* kv, bool fp8, void* out, flo
   const int g = Hq / Hkv;
   if (g > 32) return ATTN_ERR_UNSUPPORTED;
   if (!gqa::decode_dims_supported(D, Dv, fp8)) return ATTN_ERR_UNSUPPORTED;
-  // rows per CTA: TMEM holds 2 S^T buffers and O^T, (2 + Dv/128) x RP of 512 columns
-  const int max_rows = std::min(128, (512 / (2 + Dv / 128)) / 16 * 16);
+  // rows per CTA: TMEM holds 2 S^T buffers and O^T, (2 + ceil(Dv/128)) x RP of 512 columns
+  const int max_rows = std::min(128, (512 / (2 + (Dv + 127) / 128)) / 16 * 16);
   int qchunk = std::max(1, std::min(max_rows / g, Sq));
   // fewer rows when two K/V slots and the Q, P buffers of that many rows do
   // not fit one CTA's shared memory (fp8 at D = 512: two more Q planes)
@@ -371,7 +371,8 @@ int decode_run(const void* q, const attn_kv_view* kv, float* partial_out, float*
   const int g = Hq / Hkv;
   const long long R = (long long)g * Sq;
   const long long RP = (R + 15) / 16 * 16;
-  if (RP * (2 + Dv / 128) > 256) return ATTN_ERR_UNSUPPORTED;  // TMEM: two S^T buffers + O^T
+  const int vchunks = (Dv + 127) / 128;   // O^T chunks of 128 d-rows (one at Dv = 64)
+  if (RP * (2 + vchunks) > 256) return ATTN_ERR_UNSUPPORTED;  // TMEM: two S^T buffers + O^T
   if (g > 256 || Sq > 256) return ATTN_ERR_UNSUPPORTED;  // TMA box extents
   if ((long long)B * Hkv > 65535) return ATTN_ERR_INVALID_ARG;
   if (!aligned(q, 16)) return ATTN_ERR_ALIGNMENT;
@@ -435,7 +436,7 @@ int decode_run(const void* q, const attn_kv_view* kv, float* partial_out, float*
     grp = std::min<long long>(std::min<long long>(grp, gqa::decode_max_group()), num_splits);
     p.group = (int)std::max<long long>(grp, 1);
     // two O^T buffers when split boundaries exist and two CTAs' TMEM still fits
-    p.obuf = (p.group > 1 && RP * (2 + 2 * (Dv / 128)) <= 256) ? 2 : 1;
+    p.obuf = (p.group > 1 && RP * (2 + 2 * vchunks) <= 256) ? 2 : 1;
     p.fout = nullptr;
   }
   p.c2 = scale * kLog2e;

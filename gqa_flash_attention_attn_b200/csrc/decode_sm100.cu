@@ -187,11 +187,13 @@ __device__ __forceinline__ void ext_rows16(float (&v)[16], const LogitExt& x, fl
 
 // O^T / l of one split from TMEM to the fp32 partial (rows r < R of this
 // CTA's group), called once per split: kept out of line so the tile loop
-// stays small.  Thread t owns column t of each 128-column chunk.
-template <int KC>
+// stays small.  Thread t owns column t of each 128-column chunk (of the one
+// 64-column chunk when D = 64: threads 64-127 then hold no column).
+template <int D>
 __device__ __noinline__ void write_partial_o(uint32_t taddr, int RP, int R, int g, int kvh, int b, int s0, int Sq,
                                              int Hq, void* out, bool out_bf16, const float* inv_sm, int t) {
-  constexpr int D = KC * 128;
+  constexpr int KC = (D + 127) / 128;
+  if (t >= (D < 128 ? D : 128)) return;
   for (int c = 0; c < KC; ++c) {
     for (int q = 0; q < RP / 16; ++q) {
       float v[16];
@@ -275,9 +277,14 @@ __global__ void __launch_bounds__(THREADS, 2)
   // an odd multiple of 64 (e.g. 320, 576)
   constexpr int KCK = (DK + 127) / 128;
   constexpr bool KHALF = (DK % 128) != 0;
-  constexpr int KC = DV / 128;   // V slots per tile, and O^T chunks
+  // V slots per tile, and O^T chunks of 128 d-rows; DV = 64 fills the first
+  // half of one slot (one box), and O^T rows 64-127 of the P.V MMA (which
+  // read the slot's unused second box) are never stored
+  constexpr int KC = (DV + 127) / 128;
+  constexpr bool VHALF = (DV % 128) != 0;
   constexpr int D = DV;          // output width
-  static_assert(DK % 64 == 0 && DV % 128 == 0 && (!FP8 || DK == DV), "head sizes");
+  static_assert(DK % 64 == 0 && DV % 64 == 0 && (!VHALF || DV == 64) && (!FP8 || (DK == DV && !VHALF)),
+                "head sizes");
   const int RP = p.RP, g = p.g, nbuf = p.nbuf;
   const Layout L(DK, RP, nbuf, p.mask_rows, FP8);
   constexpr uint32_t SLOTB = FP8 ? BOX_BYTES : SLOT_BYTES;   // bytes of one 128-column K/V slot
@@ -487,8 +494,9 @@ __global__ void __launch_bounds__(THREADS, 2)
             ok = false;
             return;
           }
-          // a half-filled last K slot (DK an odd multiple of 64) takes one box
-          const bool half = KHALF && is_k && c == KCK - 1;
+          // a half-filled last K slot (DK an odd multiple of 64) takes one
+          // box, and so does the V slot when DV = 64
+          const bool half = (KHALF && is_k && c == KCK - 1) || (VHALF && !is_k);
           mbar_arrive_expect_tx(bar(bar_full(slot)), half ? BOX_BYTES : SLOTB);
           const uint32_t dst = base + L.off_ring + (uint32_t)slot * SLOTB;
           if constexpr (!PAGED) {
@@ -721,7 +729,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       const size_t so = (size_t)(sg0 + si) * p.B * p.Sq * p.Hq * D;
       // partials (fp32), or with one split the final output itself
       void* dst = p.fout != nullptr ? p.fout : static_cast<void*>(p.part_out + so);
-      write_partial_o<KC>(tmem + lane_off + TO(0, seg_sm[si].ob), RP, R, g, kvh, b, s0, p.Sq, p.Hq, dst,
+      write_partial_o<D>(tmem + lane_off + TO(0, seg_sm[si].ob), RP, R, g, kvh, b, s0, p.Sq, p.Hq, dst,
                           p.fout != nullptr && p.fout_bf16, inv_sm, t);
       named_bar_sync(1, 128);   // every row's inv_sm read before stats() rewrites it
     };
@@ -982,9 +990,10 @@ __global__ void __launch_bounds__(THREADS, 2)
         for (int c = 0; c < KC; ++c) {
           for (int q = 0; q < RP / 16; ++q) {
             float v[16];
-            tmem_ld16(tmem + lane_off + TO(c, seg_sm[0].ob) + 16 * q, v);
+            tmem_ld16(tmem + lane_off + TO(c, seg_sm[0].ob) + 16 * q, v);   // warp-collective
+            if (c * 128 + t < D)
 #pragma unroll
-            for (int e = 0; e < 16; ++e) xbuf[(size_t)(16 * q + e) * D + c * 128 + t] = v[e] * vs;
+              for (int e = 0; e < 16; ++e) xbuf[(size_t)(16 * q + e) * D + c * 128 + t] = v[e] * vs;
           }
         }
       } else {
@@ -1091,6 +1100,7 @@ int launch_decode_split(int D, int Dv, bool ext, bool fp8, const CUtensorMap& tq
                         const CUtensorMap& tv, const DecodeParams& p, cudaStream_t stream) {
   if (D == Dv) {
     switch (D) {
+      case 64: return fp8 ? (int)cudaErrorInvalidValue : launch_d<64, 64, false>(ext, tq, tk, tv, p, stream);
       case 128: return fp8 ? launch_d<128, 128, true>(ext, tq, tk, tv, p, stream) : launch_d<128, 128, false>(ext, tq, tk, tv, p, stream);
       case 256: return fp8 ? launch_d<256, 256, true>(ext, tq, tk, tv, p, stream) : launch_d<256, 256, false>(ext, tq, tk, tv, p, stream);
       case 512: return fp8 ? launch_d<512, 512, true>(ext, tq, tk, tv, p, stream) : launch_d<512, 512, false>(ext, tq, tk, tv, p, stream);
@@ -1106,7 +1116,7 @@ int launch_decode_split(int D, int Dv, bool ext, bool fp8, const CUtensorMap& tq
 }
 
 bool decode_dims_supported(int D, int Dv, bool fp8) {
-  if (D == Dv) return D == 128 || D == 256 || D == 512;
+  if (D == Dv) return (D == 64 && !fp8) || D == 128 || D == 256 || D == 512;
   return !fp8 && ((D == 576 && Dv == 512) || (D == 320 && Dv == 256) || (D == 192 && Dv == 128));
 }
 

@@ -91,11 +91,15 @@ int attn_prefill(const void* q, const void* k, const void* v, void* out, float* 
  * Overview, the ub>64 fix: whole-tile blocks must publish their (max, rowsum)
  * or the merge silently drops their rows).
  *
- *   D            128, 256 or 512 (else ATTN_ERR_UNSUPPORTED)
+ *   D            64, 128, 256 or 512 (else ATTN_ERR_UNSUPPORTED); the pages'
+ *                kernels carry D = 64 K/V heads ("Anbeeld/beellama.cpp PR
+ *                #149", Base: v0.4.7, D=64 KV-head support; the HEAD_DIM
+ *                dispatch of "ViperEkura/AstrAI commit 7ba43a7,
+ *                gqa_prefill_attn_mma.cuh")
  *   rows         R = (Hq/Hkv) * Sq query rows share one K/V head; R rounded up
- *                to a multiple of 16 must satisfy (2 + D/128) * R16 <= 256
- *                (else ATTN_ERR_UNSUPPORTED): at most 128 rows for D = 128,
- *                64 for D = 256, 32 for D = 512
+ *                to a multiple of 16 must satisfy (2 + ceil(D/128)) * R16 <= 256
+ *                (else ATTN_ERR_UNSUPPORTED): at most 80 rows for D = 64 and
+ *                D = 128, 64 for D = 256, 32 for D = 512
  *   num_splits   1 <= num_splits <= Skv (else ATTN_ERR_INVALID_ARG)
  *   partial_out  num_splits*B*Sq*Hq*D floats; partial_lse num_splits*B*Hq*Sq
  */
@@ -311,7 +315,7 @@ typedef struct attn_kv_view {
  * num_splits) keys of sequence b per split, rounded up to a multiple of 128
  * when paged so that no 128-key tile crosses a page; splits past the end
  * publish lse = -inf and O = 0.  With head_dim_v = Dv != D the partials are
- * [S, B, Sq, Hq, Dv] and the row limit reads (2 + Dv/128) * R16 <= 256; merge
+ * [S, B, Sq, Hq, Dv] and the row limit reads (2 + ceil(Dv/128)) * R16 <= 256; merge
  * them with attn_merge at D = Dv.  Other arguments, limits and errors as in
  * attn_decode_split.
  */
@@ -331,8 +335,15 @@ int attn_decode_split_kv(const void* q, const attn_kv_view* kv, float* partial_o
  *   n            the largest power of two <= min(num_splits, 8): key range
  *                k of n covers keys [k c, (k+1) c), c = ceil(len / n)
  *                (rounded up to 128 when paged); the result is the attention
- *                of attn_decode_split_kv + attn_merge_ex with n splits.  It
- *                pays off when B * Hkv * n fills the GPU (two CTAs per SM)
+ *                of attn_decode_split_kv + attn_merge_ex with n splits.
+ *                When to call it: it saves the merge launch and the partials'
+ *                round trip through HBM, but it runs only B * Hkv * n CTAs
+ *                (n <= 8), where attn_decode_split_kv runs B * Hkv * num_splits
+ *                (grouped to fill the GPU).  Measured on B200 (148 SMs, two
+ *                CTAs each): with B * Hkv * n >= 2 * 148 it is faster (8-row
+ *                verify, B4 Hkv8 D128: 98 vs 111 us per step); with fewer
+ *                CTAs it is not (B16 Hkv1 D512: 118 vs 111 us), so such
+ *                shapes should call attn_decode_split_kv + attn_merge_ex
  *   out, lse     as attn_merge_ex's: out [B, Sq, Hq, Dv] (out_dtype), lse
  *                [B, Hq, Sq] fp32 or NULL; opt->sinks apply here
  *   limits       those of attn_decode_split_kv, and the merge's shared memory
@@ -354,7 +365,7 @@ int attn_decode_fused(const void* q, const attn_kv_view* kv, void* out, float* l
  *   - otherwise (D = Dv = 512, the pairs with Dv != D, paged, fp8 or
  *     seq_lens): the split-KV kernel with one split and the query rows cut
  *     into chunks per CTA, writing O and LSE directly, as attn_prefill does
- *     at D = 512.  Dims: D = Dv in {128, 256, 512}, or a pair listed under
+ *     at D = 512.  Dims: D = Dv in {64 (bf16 only), 128, 256, 512}, or a pair listed under
  *     attn_kv_view; Hq/Hkv <= 32.  Else ATTN_ERR_UNSUPPORTED.
  * Arguments, options (*opt may be NULL; sinks apply here), alignment and
  * errors otherwise as in attn_prefill_ex and attn_decode_split_kv.

@@ -64,6 +64,21 @@ def oracle_rows_by_batch(q, k, v, rows, *, scale, causal, q_offset, **terms):
     return out, lse
 
 
+def oracle_attention_by_batch(q, k, v, *, scale, causal, q_offset):
+    """oracle.attention over every row, one batch entry at a time, so only
+    one sequence's K/V is widened to float64 at once (a 32K-key decode cache
+    is gigabytes in float64)."""
+    B, Sq, Hq, _ = q.shape
+    Dv = v.shape[3]
+    out = np.zeros((B, Sq, Hq, Dv))
+    lse = np.zeros((B, Hq, Sq))
+    for b in range(B):
+        o, l = oracle.attention(q[b:b + 1], k[b:b + 1], v[b:b + 1], scale=scale, causal=causal, q_offset=q_offset)
+        out[b] = o[0]
+        lse[b] = l[0]
+    return out, lse
+
+
 def gather_rows(out, lse, rows):
     """GPU O [B,Sq,Hq,D] and LSE [B,Hq,Sq] at (b, h, s) triples."""
     rows = torch.as_tensor(np.asarray(rows, dtype=np.int64).reshape(-1, 3))

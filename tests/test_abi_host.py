@@ -91,7 +91,8 @@ def _decode(lib, **kw):
     (dict(po=None), ga.ATTN_ERR_INVALID_ARG),
     (dict(pl=None), ga.ATTN_ERR_INVALID_ARG),
     (dict(Hq=12, Hkv=8), ga.ATTN_ERR_INVALID_ARG),
-    (dict(D=64), ga.ATTN_ERR_UNSUPPORTED),
+    (dict(D=64, Hq=96, Hkv=1), ga.ATTN_ERR_UNSUPPORTED),   # 96 rows x (2 + 1) > 256 TMEM columns
+    (dict(D=32), ga.ATTN_ERR_UNSUPPORTED),
     (dict(D=96), ga.ATTN_ERR_UNSUPPORTED),
     (dict(Hq=64, Sq=1), ga.ATTN_ERR_UNSUPPORTED),   # 64 rows x (2 + 512/128) > 256 TMEM columns
     (dict(D=128, Hq=32, Hkv=1, Sq=8), ga.ATTN_ERR_UNSUPPORTED),  # 256 rows
@@ -215,7 +216,9 @@ def _kv_decode(lib, view=None, **kw):
     (dict(block_table=0x70000, max_pages=0, page_size=128, num_pages=64), {}, ga.ATTN_ERR_INVALID_ARG),
     (dict(block_table=0x70000, max_pages=8, page_size=128, num_pages=0), dict(Skv=1024), ga.ATTN_ERR_INVALID_ARG),
     (dict(block_table=0x70002, max_pages=8, page_size=128, num_pages=64), dict(Skv=1024), ga.ATTN_ERR_ALIGNMENT),
-    ({}, dict(D=64), ga.ATTN_ERR_UNSUPPORTED),
+    ({}, dict(D=32), ga.ATTN_ERR_UNSUPPORTED),
+    (dict(kv_dtype=2, k_scale=0x90000, v_scale=0x90010, stride_token=64, stride_head=64, stride_seq=64 * 1024),
+     dict(D=64), ga.ATTN_ERR_UNSUPPORTED),                                    # fp8 at D = 64: no kernel
     (dict(kv_dtype=5), {}, ga.ATTN_ERR_INVALID_ARG),
     (dict(kv_dtype=2), {}, ga.ATTN_ERR_INVALID_ARG),                           # fp8 without scales
     (dict(kv_dtype=2, k_scale=0x90000, v_scale=0x90002), {}, ga.ATTN_ERR_INVALID_ARG),
@@ -264,7 +267,9 @@ def _kv_prefill(lib, view=None, opt=None, **kw):
     ({}, dict(out=None), ga.ATTN_ERR_INVALID_ARG),
     ({}, dict(out_dtype=2), ga.ATTN_ERR_INVALID_ARG),
     ({}, dict(D=96), ga.ATTN_ERR_UNSUPPORTED),
-    (dict(block_table=0x70000, max_pages=8, page_size=128, num_pages=64), dict(D=64), ga.ATTN_ERR_UNSUPPORTED),
+    (dict(block_table=0x70000, max_pages=8, page_size=128, num_pages=64), dict(D=32), ga.ATTN_ERR_UNSUPPORTED),
+    (dict(kv_dtype=2, k_scale=0x90000, v_scale=0x90010, stride_token=64, stride_head=64, stride_seq=64 * 1024),
+     dict(D=64), ga.ATTN_ERR_UNSUPPORTED),                                    # fp8 at D = 64: no kernel
     ({}, dict(Hq=64), ga.ATTN_ERR_UNSUPPORTED),                                # g = 64 > 32 on the wide path
     (dict(head_dim_v=256), {}, ga.ATTN_ERR_UNSUPPORTED),
     (dict(stride_token=516), {}, ga.ATTN_ERR_ALIGNMENT),
@@ -297,7 +302,9 @@ def _kv_fused(lib, view=None, opt=None, **kw):
     ({}, dict(out=None), ga.ATTN_ERR_INVALID_ARG),
     ({}, dict(out_dtype=7), ga.ATTN_ERR_INVALID_ARG),
     ({}, dict(S=0), ga.ATTN_ERR_INVALID_ARG),
-    ({}, dict(D=64), ga.ATTN_ERR_UNSUPPORTED),
+    ({}, dict(D=32), ga.ATTN_ERR_UNSUPPORTED),
+    (dict(kv_dtype=2, k_scale=0x90000, v_scale=0x90010, stride_token=64, stride_head=64, stride_seq=64 * 1024),
+     dict(D=64), ga.ATTN_ERR_UNSUPPORTED),                                    # fp8 at D = 64: no kernel
     ({}, dict(out=ctypes.c_void_p(0x20008)), ga.ATTN_ERR_ALIGNMENT),
     ({}, dict(lse=ctypes.c_void_p(0x20002)), ga.ATTN_ERR_ALIGNMENT),
     (dict(stride_token=128, stride_head=128, stride_seq=128 * 1024), dict(D=128, Hq=64, Hkv=1, Sq=2),

@@ -22,6 +22,24 @@ def test_reference_arm_prints_one_contract_line():
     assert d["config"]["workload"] == "gqa_causal_prefill_4k_d128"
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+    # the reference arm describes its workload with the GPU arm's config keys and values
+    sys.path.insert(0, ROOT)
+    import bench
+    from gqa_flash_attention_attn_b200.inputs import WORKLOADS
+    assert d["config"] == bench.workload_config(WORKLOADS[bench.HEADLINE], 1)
+
+
+def test_base_configs_are_compact_and_per_step():
+    sys.path.insert(0, ROOT)
+    import bench
+    from gqa_flash_attention_attn_b200.inputs import WORKLOADS
+    assert all(n in WORKLOADS for n in bench.BASE_CONFIGS) and len(bench.BASE_CONFIGS) == 5
+    r = {"value": 4831.123456, "unit": "GB/s", "ms_per_step": 0.11123456, "kernel_ms": 0.0989123,
+         "roofline": {"frac": 0.73912345, "kernel_frac": 0.8312345, "bound": "hbm", "traffic": None}}
+    c = bench.compact(r)
+    assert c == {"value": 4831.0, "unit": "GB/s", "ms_per_step": 0.1112, "kernel_ms": 0.09891,
+                 "roofline_frac": 0.739, "kernel_frac": 0.831, "bound": "hbm", "traffic": None}
+    assert len(json.dumps({n: c for n in bench.BASE_CONFIGS})) < 1200
 
 
 def test_workload_metric_units():

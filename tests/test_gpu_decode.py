@@ -8,7 +8,7 @@ import torch
 import gqa_flash_attention_attn_b200 as ga
 from gqa_flash_attention_attn_b200.inputs import WORKLOADS, make_qkv, make_workload_inputs, sample_rows
 import oracle
-from parity import (assert_lse_close, assert_o_close, gather_rows, oracle_rows_by_batch, to_f64)
+from parity import (oracle_attention_by_batch, assert_lse_close, assert_o_close, gather_rows, oracle_rows_by_batch, to_f64)
 
 pytestmark = pytest.mark.gpu
 
@@ -23,6 +23,13 @@ CASES = [
     (1, 16, 4, 2, 300, 512, 298, True, 2),      # 8 rows padded to 16
     (1, 8, 1, 1, 777, 128, 0, False, 6),        # non-causal
     (1, 16, 2, 8, 515, 128, 507, True, 1),      # 64 rows, one split, ragged tail
+    # D = 64: one 64-column box per K and V tile
+    (2, 8, 1, 1, 1000, 64, 999, True, 4),       # single-query decode
+    (1, 32, 8, 8, 700, 64, 692, True, 3),       # 8 draft rows per sequence (32 rows per K/V head)
+    (1, 8, 1, 1, 100, 64, 99, True, 30),        # splits 25..29 hold no key
+    (1, 4, 1, 8, 1000, 64, 0, True, 9),         # causal at q_offset 0: most splits fully masked
+    (1, 8, 1, 1, 777, 64, 0, False, 6),         # non-causal
+    (1, 80, 8, 8, 333, 64, 325, True, 2),       # 80 rows per K/V head (the D = 64 limit), ragged
 ]
 
 
@@ -84,19 +91,20 @@ def test_split_count_does_not_change_result():
 
 
 @pytest.mark.parametrize("name", ["split_kv_decode_d512", "spec_verify_decode_d128"])
-def test_full_size_workload_sampled_rows(name):
+def test_full_size_workload_every_row(name):
+    """The timed decode workloads at full size, in the launch configuration
+    the benchmark times (decode_split with its split count, then merge):
+    every output row against the float64 oracle."""
     w = WORKLOADS[name]
     q, k, v = make_workload_inputs(w)
-    out, lse = ga.decode(q.cuda(), k.cuda(), v.cuda(), w.num_splits, causal=w.causal, q_offset=w.q_offset,
-                         scale=w.scale, out_dtype=torch.bfloat16)
+    po, pl = ga.decode_split(q.cuda(), k.cuda(), v.cuda(), w.num_splits, causal=w.causal, q_offset=w.q_offset,
+                             scale=w.scale)
+    out, lse = ga.merge(po, pl, out_dtype=torch.bfloat16)
     torch.cuda.synchronize()
     assert ga.last_status() == ga.ATTN_OK
-    rows = sample_rows(w, 48)
-    want_o, want_lse = oracle_rows_by_batch(q, k, v, rows, scale=w.scale, causal=w.causal, q_offset=w.q_offset)
-    got_o, got_lse = gather_rows(out, lse, rows)
-    assert_o_close(got_o, want_o, name)
-    assert_lse_close(got_lse, want_lse, name)
-    assert torch.isfinite(out).all() and torch.isfinite(lse).all()
+    want_o, want_lse = oracle_attention_by_batch(q, k, v, scale=w.scale, causal=w.causal, q_offset=w.q_offset)
+    assert_o_close(out, want_o, name)
+    assert_lse_close(lse, want_lse, name)
 
 
 # (B, Hq, Hkv, Sq, Skv, D, q_offset, causal, num_splits): enough CTAs that each
@@ -106,6 +114,8 @@ GROUPED = [
     (64, 16, 2, 2, 513, 256, 100, True, 9),      # causal: splits past key 101 empty inside groups
     (128, 8, 4, 1, 2048, 128, 2047, True, 8),    # groups of 8
     (40, 16, 1, 1, 1000, 512, 0, False, 30),     # non-causal D512, groups of 3
+    (128, 8, 2, 1, 2048, 64, 2047, True, 8),     # D64, groups of 8
+    (64, 16, 2, 2, 513, 64, 100, True, 9),       # D64, causal: empty splits inside groups
 ]
 
 

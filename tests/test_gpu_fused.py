@@ -33,6 +33,7 @@ CASES = [
     (1, 8, 1, 1, 777, 128, 0, False, 3),          # non-causal, 2 ranges
     (2, 16, 2, 4, 640, 128, 636, True, 1),        # a cluster of one
     (1, 64, 8, 2, 5000, 128, 4998, True, 16),     # 16 rows per K/V head
+    (2, 32, 4, 4, 1300, 64, 1296, True, 8),       # D = 64: 32 rows per K/V head, 8 ranges
 ]
 
 

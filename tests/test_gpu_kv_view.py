@@ -34,7 +34,8 @@ def _oracle_per_sequence(q, k, v, lens, *, scale, causal=True, **terms):
 
 
 # (B, Hq, Hkv, Sq, Skv, D, num_splits)
-SHAPES = [(2, 16, 1, 1, 1024, 512, 4), (1, 32, 8, 8, 1024, 128, 4), (2, 8, 2, 3, 1024, 256, 2)]
+SHAPES = [(2, 16, 1, 1, 1024, 512, 4), (1, 32, 8, 8, 1024, 128, 4), (2, 8, 2, 3, 1024, 256, 2),
+          (2, 32, 4, 2, 1024, 64, 4)]
 
 
 @pytest.mark.parametrize("page_size", [16, 32, 64, 128, 256])

@@ -8,7 +8,7 @@ import torch
 import gqa_flash_attention_attn_b200 as ga
 from gqa_flash_attention_attn_b200.inputs import WORKLOADS, make_qkv, make_workload_inputs, sample_rows
 import oracle
-from parity import (assert_lse_close, assert_o_close, gather_rows, oracle_rows_by_batch)
+from parity import (oracle_attention_by_batch, assert_lse_close, assert_o_close, gather_rows, oracle_rows_by_batch)
 
 pytestmark = pytest.mark.gpu
 
@@ -87,22 +87,41 @@ def test_repeated_calls_are_deterministic():
     assert torch.equal(a, b) and torch.equal(la, lb)
 
 
-@pytest.mark.parametrize("name", ["gqa_causal_prefill_4k_d128", "prefill_at_depth_d256"])
-def test_full_size_workload_sampled_rows(name):
+@pytest.mark.parametrize("name", ["tiny_causal_gqa_prefill", "gqa_causal_prefill_4k_d128", "prefill_at_depth_d256"])
+def test_full_size_workload_every_row(name):
+    """The timed prefill workloads at full size, in the launch configuration
+    the benchmark times: every output row against the float64 oracle."""
     w = WORKLOADS[name]
     q, k, v = make_workload_inputs(w)
+    odt = torch.float32 if w.out_dtype == "f32" else torch.bfloat16
     out, lse = ga.prefill(q.cuda(), k.cuda(), v.cuda(), causal=w.causal, q_offset=w.q_offset, scale=w.scale,
-                          out_dtype=torch.bfloat16)
+                          out_dtype=odt)
     torch.cuda.synchronize()
     assert ga.last_status() == ga.ATTN_OK
-    rows = sample_rows(w, 96)
-    want_o, want_lse = oracle_rows_by_batch(q, k, v, rows, scale=w.scale, causal=w.causal, q_offset=w.q_offset)
-    got_o, got_lse = gather_rows(out, lse, rows)
-    assert_o_close(got_o, want_o, name)
-    assert_lse_close(got_lse, want_lse, name)
-    # every row, not only the sampled ones, is finite
-    assert torch.isfinite(out).all()
-    assert torch.isfinite(lse).all()
+    want_o, want_lse = oracle_attention_by_batch(q, k, v, scale=w.scale, causal=w.causal, q_offset=w.q_offset)
+    assert_o_close(out, want_o, name)
+    assert_lse_close(lse, want_lse, name)
+
+
+# More work units than twice the persistent grid (148 CTAs on a B200), so
+# every CTA runs several units and carries its barrier phases, TMEM buffers
+# and K/V ring position from one unit to the next.
+# (B, Hq, Hkv, Sq, Skv, D, q_offset, causal, out_dtype)
+MULTI_UNIT = [
+    (2, 32, 8, 2048, 2048, 128, 0, True, torch.bfloat16),     # 2 x 16 x 16 = 512 units, two head slots
+    (2, 16, 8, 2048, 2048, 256, 0, True, torch.bfloat16),     # 2 x 16 x 16 = 512 units, one slot, S double buffered
+    (3, 12, 4, 700, 1500, 128, 800, True, torch.float32),     # odd group (3): second slot idle in half the units
+    (4, 8, 8, 640, 640, 64, 0, False, torch.bfloat16),        # non-causal D = 64, 160 equal units
+]
+
+
+@pytest.mark.parametrize("case", MULTI_UNIT, ids=[f"B{c[0]}H{c[1]}/{c[2]}S{c[3]}x{c[4]}D{c[5]}" for c in MULTI_UNIT])
+def test_prefill_many_units_per_cta(case):
+    B, Hq, Hkv, Sq, Skv, D, q_offset, causal, out_dtype = case
+    q, k, v, scale, out, lse = _run(*case, seed=11)
+    want_o, want_lse = oracle.attention(q, k, v, scale=scale, causal=causal, q_offset=q_offset)
+    assert_o_close(out, want_o, str(case))
+    assert_lse_close(lse, want_lse, str(case))
 
 
 # D = 512 (the split-KV kernel in query-chunk mode):
