@@ -8,6 +8,7 @@ import os
 import shutil
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
@@ -39,14 +40,23 @@ def stale() -> bool:
 
 
 def build(verbose: bool = False, force: bool = False) -> str:
+    """Compile each source to an object in _build/ (in parallel), then link
+    the shared library."""
     if not force and not stale():
         return LIB
-    cmd = [nvcc(), "-O3", "-std=c++17", *ARCH, "-lineinfo", "-Xcompiler", "-fPIC", "-shared",
-           "-I", os.path.join(ROOT, "include"), "-o", LIB]
+    obj_dir = os.path.join(ROOT, "_build")
+    os.makedirs(obj_dir, exist_ok=True)
+    flags = [nvcc(), "-O3", "-std=c++17", *ARCH, "-lineinfo", "-Xcompiler", "-fPIC",
+             "-I", os.path.join(ROOT, "include")]
     if verbose:
-        cmd += ["-Xptxas", "-v"]
-    cmd += [os.path.join(CSRC, s) for s in SOURCES]
-    subprocess.run(cmd, check=True)
+        flags += ["-Xptxas", "-v"]
+    objs = [os.path.join(obj_dir, os.path.splitext(s)[0] + ".o") for s in SOURCES]
+    with ThreadPoolExecutor(max_workers=max(1, min(len(SOURCES), os.cpu_count() or 1))) as ex:
+        jobs = [ex.submit(subprocess.run, flags + ["-c", os.path.join(CSRC, s), "-o", o], check=True)
+                for s, o in zip(SOURCES, objs)]
+        for j in jobs:
+            j.result()
+    subprocess.run([nvcc(), *ARCH, "-shared", "-o", LIB, *objs], check=True)
     return LIB
 
 
