@@ -289,19 +289,21 @@ int prefill_wide(const void* q, const attn_kv_view* kv, bool fp8, void* out, flo
 }
 
 // The prefill kernel over given K/V tensor maps (D = Dv in 64, 128, 256, or
-// D = 192 with Dv = 128).
-int prefill_fast(const void* q, const CUtensorMap& tk, const CUtensorMap& tv, void* out, float* lse, int B, int Hq,
-                 int Hkv, int Sq, int Skv, int D, int Dv, int q_offset, int causal, float scale, int out_dtype,
-                 const gqa::LogitExt& ext, bool ext_on, void* stream) {
+// D = 192 with Dv = 128).  tk64 (K in 64-key boxes, or nullptr) enables the
+// CTA-pair form at D = Dv = 256 with an even group size and no mask.
+int prefill_fast(const void* q, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap* tk64, void* out,
+                 float* lse, int B, int Hq, int Hkv, int Sq, int Skv, int D, int Dv, int q_offset, int causal,
+                 float scale, int out_dtype, const gqa::LogitExt& ext, bool ext_on, void* stream) {
   const int nslot = gqa::prefill_slots(Dv);
   const int g = Hq / Hkv;
+  const bool pair = tk64 != nullptr && D == 256 && Dv == 256 && g % 2 == 0 && ext.mask == nullptr;
   gqa::PrefillParams p{};
   p.out = out;
   p.lse = lse;
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Sq = Sq; p.Skv = Skv;
   p.q_offset = q_offset; p.causal = causal; p.out_f32 = (out_dtype == ATTN_F32);
   p.g = g;
-  p.units_per_kvh = (g + nslot - 1) / nslot;
+  p.units_per_kvh = pair ? g / 2 : (g + nslot - 1) / nslot;
   p.n_qt = (Sq + 127) / 128;
   p.c2 = scale * kLog2e;
   p.timeout_ns = kWaitLimitNs;
@@ -314,6 +316,10 @@ int prefill_fast(const void* q, const CUtensorMap& tk, const CUtensorMap& tv, vo
   if (p.num_ctas <= 0) return cuda_fail();
   CUtensorMap tq;
   if (!make_map(&tq, q, D, Hq, Sq, B, 64, 1, 128, 1)) return cuda_fail();
+  if (pair)
+    return gqa::launch_prefill_pair(D, ext_on, tq, *tk64, tv, p, static_cast<cudaStream_t>(stream)) == 0
+               ? ATTN_OK
+               : ATTN_ERR_CUDA;
   // the additive mask staged by TMA: 16-byte aligned rows, and every head
   // slot of a CTA visits every tile (one slot, or an even group size)
   CUtensorMap tm;
@@ -499,11 +505,13 @@ int attn_prefill_ex(const void* q, const void* k, const void* v, void* out, floa
     return prefill_wide(q, &kv, false, out, lse, B, Hq, Hkv, Sq, Skv, D, D, q_offset, causal, scale, out_dtype, ext,
                         ext_on, stream);
   }
-  CUtensorMap tk, tv;
+  CUtensorMap tk, tv, tk64;
   if (!make_map(&tk, k, D, Hkv, Skv, B, 64, 1, 128, 1)) return cuda_fail();
   if (!make_map(&tv, v, D, Hkv, Skv, B, 64, 1, 128, 1)) return cuda_fail();
-  return prefill_fast(q, tk, tv, out, lse, B, Hq, Hkv, Sq, Skv, D, D, q_offset, causal, scale, out_dtype, ext, ext_on,
-                      stream);
+  const bool k64 = D == 256;   // K in 64-key boxes for the CTA-pair form
+  if (k64 && !make_map(&tk64, k, D, Hkv, Skv, B, 64, 1, 64, 1)) return cuda_fail();
+  return prefill_fast(q, tk, tv, k64 ? &tk64 : nullptr, out, lse, B, Hq, Hkv, Sq, Skv, D, D, q_offset, causal, scale,
+                      out_dtype, ext, ext_on, stream);
 }
 
 int attn_prefill_kv(const void* q, const attn_kv_view* kv, void* out, float* lse, int B, int Hq, int Hkv, int Sq,
@@ -531,12 +539,15 @@ int attn_prefill_kv(const void* q, const attn_kv_view* kv, void* out, float* lse
   if (!fast)
     return prefill_wide(q, kv, fp8, out, lse, B, Hq, Hkv, Sq, Skv, D, Dv, q_offset, causal, scale, out_dtype, ext,
                         ext_on, stream);
-  CUtensorMap tk, tv;
+  CUtensorMap tk, tv, tk64;
   const ViewStrides ks = k_strides(kv), vs = v_strides(kv);
   if (!make_map_strided(&tk, kv->k, D, Hkv, Skv, B, ks.head, ks.token, ks.seq, 64, 1, 128, 1)) return cuda_fail();
   if (!make_map_strided(&tv, kv->v, Dv, Hkv, Skv, B, vs.head, vs.token, vs.seq, 64, 1, 128, 1)) return cuda_fail();
-  return prefill_fast(q, tk, tv, out, lse, B, Hq, Hkv, Sq, Skv, D, Dv, q_offset, causal, scale, out_dtype, ext, ext_on,
-                      stream);
+  const bool k64 = D == 256 && Dv == 256;   // K in 64-key boxes for the CTA-pair form
+  if (k64 && !make_map_strided(&tk64, kv->k, D, Hkv, Skv, B, ks.head, ks.token, ks.seq, 64, 1, 64, 1))
+    return cuda_fail();
+  return prefill_fast(q, tk, tv, k64 ? &tk64 : nullptr, out, lse, B, Hq, Hkv, Sq, Skv, D, Dv, q_offset, causal, scale,
+                      out_dtype, ext, ext_on, stream);
 }
 
 size_t attn_decode_workspace_bytes(int B, int Hq, int Sq, int D, int num_splits) {

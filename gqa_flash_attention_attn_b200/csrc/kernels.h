@@ -90,6 +90,12 @@ struct MergeParams {
 int launch_prefill(int D, int Dv, bool ext, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                    const CUtensorMap& tm, const PrefillParams& p, cudaStream_t stream);
 size_t prefill_smem_bytes(int D, int Dv);
+// The CTA-pair prefill (D = Dv = 256, even Hq/Hkv, no additive mask): each
+// cluster of two CTAs runs the two query heads of a K/V group; tk64 tiles K
+// in boxes of 64 keys (64 columns x 64 rows), tv and tq as for launch_prefill.
+// p.units_per_kvh must be (Hq/Hkv)/2.
+int launch_prefill_pair(int D, bool ext, const CUtensorMap& tq, const CUtensorMap& tk64, const CUtensorMap& tv,
+                        const PrefillParams& p, cudaStream_t stream);
 // D: the Q and K head size; Dv: the V and O head size (pairs with D != Dv:
 // 576/512, 320/256, 192/128, bf16 only)
 int launch_decode_split(int D, int Dv, bool ext, bool fp8, const CUtensorMap& tq, const CUtensorMap& tk,

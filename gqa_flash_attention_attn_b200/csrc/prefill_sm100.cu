@@ -27,15 +27,29 @@
 //              Q*scale to bf16), P rounded to bf16 into TMEM, O rescaled in
 //              TMEM only when the running max grew by more than 2^8.
 //
+// CTA pairs (D = 256 with an even group size): the two CTAs of a cluster hold
+// the two query heads of a K/V group (one head slot each, S double buffered),
+// each loads half of every K/V tile (keys 64r..64r+63 of K, D columns
+// 128r..128r+127 of V, r = the CTA's rank) and the leader issues 2-CTA MMAs
+// (tcgen05 cta_group::2, M = 256 rows over the pair) that read both halves, so
+// each K/V tile crosses from L2 into shared memory once per group ("ggml-org/
+// llama.cpp PR #28507", Setup: GQA 8, head size 256).  The peer's loads land
+// on its own barriers and a thread of the peer forwards each completion to the
+// leader; the leader's MMA completions arrive on both CTAs' barriers.
+//
 // Causal masking: key t is visible to row s iff t <= q_offset + s; tiles past
 // the last row's diagonal are never loaded.  Every pipeline wait is bounded:
 // on expiry the CTA records a timeout status, drains its own copies and MMAs,
 // frees TMEM and exits.
+#include <cooperative_groups.h>
+
 #include "kernels.h"
 #include "ptx.cuh"
 
 namespace gqa {
 namespace {
+
+namespace cg = cooperative_groups;
 
 constexpr int BM = 128;   // query rows per slot (TMEM lanes)
 constexpr int BN = 128;   // keys per tile
@@ -50,20 +64,27 @@ constexpr uint32_t kPolyPairs = 0x80808080u;
 
 // MB: the variant reads an additive mask, staged by TMA in two 64-key halves.
 // DK: the Q and K head size; DV: the V and O head size (DV <= DK).
-template <int DK, int DV = DK, bool MB = false>
+// PAIR: the CTA-pair form (one head slot per CTA, half K/V tiles per CTA).
+template <int DK, int DV = DK, bool MB = false, bool PAIR = false>
 struct PrefillCfg {
-  static constexpr int NSLOT = (DV <= 128) ? 2 : 1;
+  static constexpr int NSLOT = (DV <= 128 && !PAIR) ? 2 : 1;
   static constexpr int KB = DK / 64;   // 64-column boxes of a Q or K tile
   static constexpr int VB = DV / 64;   // and of a V tile
-  static constexpr uint32_t TILE = KB * BOX_BYTES;   // a Q slot or a ring slot (K or V)
-  static constexpr int NBUF = (DK == 64) ? 8 : (DK == 128 ? 4 : 2);
-  static constexpr int THREADS = 128 * NSLOT + 64;
+  static constexpr uint32_t TILE = KB * BOX_BYTES;   // a Q slot, or a ring slot (K or V)
+  // PAIR: a ring slot holds half a tile: 64 keys x DK of K (KB boxes of 64
+  // rows) or 128 keys x DV/2 of V (VB/2 boxes of 128 rows)
+  static constexpr uint32_t RSLOT = PAIR ? TILE / 2 : TILE;
+  static constexpr int NBUF = PAIR ? 5 : (DK == 64) ? 8 : (DK == 128 ? 4 : 2);
+  // PAIR: one more warp, whose thread in the peer relays the P-ready and
+  // O-free signals of the peer's softmax warps to the leader
+  static constexpr int THREADS = 128 * NSLOT + 64 + (PAIR ? 32 : 0);
   static constexpr int WARP_PRODUCER = 4 * NSLOT;
   static constexpr int WARP_MMA = 4 * NSLOT + 1;
+  static constexpr int WARP_RELAY = 4 * NSLOT + 2;
   static constexpr uint32_t OFF_Q = 0;
   static constexpr uint32_t OFF_KV = NSLOT * TILE;
   static constexpr uint32_t MASK_HALF = BM * 128u;          // 128 rows x 64 bf16 keys
-  static constexpr uint32_t OFF_MASK = OFF_KV + NBUF * TILE;
+  static constexpr uint32_t OFF_MASK = OFF_KV + NBUF * RSLOT;
   static constexpr uint32_t OFF_BAR = OFF_MASK + (MB ? 2u * MASK_HALF : 0u);
   // q_full, q_empty, kv_full[NBUF], kv_empty[NBUF], s_full[2], p_lo[2], p_hi[2],
   // pv_done[2], o_free[2], drain; with MB mask_full[2], mask_empty[2]
@@ -90,6 +111,7 @@ struct PrefillCfg {
   static_assert(256 + NSLOT * DV <= 512, "TMEM budget");
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(DK % 64 == 0 && DV % 64 == 0 && DV <= DK, "head dims");
+  static_assert(!PAIR || (DK == DV && !MB && VB % 2 == 0), "pair form: equal head sizes, no staged mask");
 };
 
 // Wait that ignores the abort flag: used only to drain in-flight work.
@@ -153,6 +175,13 @@ __device__ __forceinline__ Unit unit_at(int u, const PrefillParams& p) {
 // shared counter.
 __device__ __forceinline__ int unit_index(int k, int total) {
   const long long G = gridDim.x, c = blockIdx.x;
+  const long long u = (long long)k * G + ((k & 1) ? (G - 1 - c) : c);
+  return u < total ? (int)u : -1;
+}
+
+// The same over CTA pairs: both CTAs of a cluster of two take the same units.
+__device__ __forceinline__ int unit_index_pair(int k, int total) {
+  const long long G = gridDim.x >> 1, c = blockIdx.x >> 1;
   const long long u = (long long)k * G + ((k & 1) ? (G - 1 - c) : c);
   return u < total ? (int)u : -1;
 }
@@ -274,13 +303,14 @@ __device__ __forceinline__ float row_max(const float (&v)[N]) {
   return fmax3(fmax3(mxc[0], mxc[1], mxc[2]), fmax3(mxc[3], mxc[4], mxc[5]), fmaxf(mxc[6], mxc[7]));
 }
 
-template <int DK, int DV, int MODE>
-__global__ void __launch_bounds__(PrefillCfg<DK, DV, MODE == MODE_ALIBI_MASK || MODE == MODE_CAP_MASK>::THREADS, 1)
+// PAIR: launched in clusters of two CTAs; tm_k then tiles K in 64-key boxes.
+template <int DK, int DV, int MODE, bool PAIR = false>
+__global__ void __launch_bounds__(PrefillCfg<DK, DV, MODE == MODE_ALIBI_MASK || MODE == MODE_CAP_MASK, PAIR>::THREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_m,
                    const PrefillParams p) {
   constexpr bool MB = MODE == MODE_ALIBI_MASK || MODE == MODE_CAP_MASK;
-  using C = PrefillCfg<DK, DV, MB>;
+  using C = PrefillCfg<DK, DV, MB, PAIR>;
   constexpr int D = DV;   // the output head size
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -293,24 +323,39 @@ __global__ void __launch_bounds__(PrefillCfg<DK, DV, MODE == MODE_ALIBI_MASK || 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int total_units = p.n_qt * p.B * p.Hkv * p.units_per_kvh;
+  // PAIR: this CTA's rank in its cluster of two (0 leads: it issues the MMAs)
+  // and the pair-aware unit order
+  const uint32_t rank = PAIR ? (blockIdx.x & 1u) : 0u;
+  constexpr int UG = PAIR ? 2 : C::NSLOT;   // query heads per unit
+  auto next_unit = [&](int k) -> int { return PAIR ? unit_index_pair(k, total_units) : unit_index(k, total_units); };
+  // Waits on barriers that the peer arrives on (PAIR leader) acquire at cluster scope
+  auto wait_x = [&](uint32_t b, uint32_t parity, const Watchdog& w) -> bool {
+    return PAIR ? mbar_wait_cluster(b, parity, w) : mbar_wait(b, parity, w);
+  };
   // With ALiBi the bias grows toward each query's own position: visiting a
   // unit's K/V tiles newest first sets the running maximum on the first tile
   // and spares the O rescales (the tile order does not change the result).
   const bool rev = MODE >= MODE_ALIBI && p.ext.alibi != 0;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(C::BAR_Q), 1);
+    // PAIR: the leader's Q and ring barriers also count the peer's forwarded
+    // completion; P and O-free barriers count one arrival per softmax warp,
+    // plus (leader) the relayed arrival of the peer's four (the single-CTA
+    // form: one per softmax thread)
+    const uint32_t nfull = (PAIR && rank == 0) ? 2u : 1u;
+    const uint32_t nsoft = PAIR ? (rank == 0 ? 5u : 4u) : 128u;
+    mbar_init(bar(C::BAR_Q), nfull);
     mbar_init(bar(C::BAR_QE), 1);
     for (int i = 0; i < C::NBUF; ++i) {
-      mbar_init(bar(C::bar_full(i)), 1);
+      mbar_init(bar(C::bar_full(i)), nfull);
       mbar_init(bar(C::bar_empty(i)), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(C::bar_s(i)), 1);
-      mbar_init(bar(C::bar_plo(i)), 128);
-      mbar_init(bar(C::bar_phi(i)), 128);
+      mbar_init(bar(C::bar_plo(i)), nsoft);
+      mbar_init(bar(C::bar_phi(i)), nsoft);
       mbar_init(bar(C::bar_pv(i)), 1);
-      mbar_init(bar(C::bar_ofree(i)), 128);
+      mbar_init(bar(C::bar_ofree(i)), nsoft);
     }
     mbar_init(bar(C::BAR_DRAIN), 1);
     if constexpr (MB) {
@@ -323,11 +368,21 @@ __global__ void __launch_bounds__(PrefillCfg<DK, DV, MODE == MODE_ALIBI_MASK || 
     fence_mbar_init();
   }
   if (warp == C::WARP_MMA) {
-    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc2(smem_u32(tmem_slot), C::TMEM_COLS);
+      tmem_relinquish2();
+    } else {
+      tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR) {
+    // both CTAs' barriers are initialised before either arrives on the other's
+    cg::this_cluster().sync();
+  } else {
+    __syncthreads();
+  }
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Watchdog wd{abort_flag, p.status, p.timeout_ns};
@@ -344,20 +399,28 @@ __global__ void __launch_bounds__(PrefillCfg<DK, DV, MODE == MODE_ALIBI_MASK || 
       int n = 0;
       bool ok = true;
       for (int k = 0; ok; ++k) {
-        const int u = unit_index(k, total_units);
+        const int u = next_unit(k);
         if (u < 0) break;
-        const Unit x = unit_at<C::NSLOT>(u, p);
+        const Unit x = unit_at<UG>(u, p);
         // the previous unit's last S MMA must be done reading Q
         if (k > 0 && !mbar_wait(bar(C::BAR_QE), (uint32_t)(k - 1) & 1u, wd)) break;
-        int nact = 0;
-        for (int i = 0; i < C::NSLOT; ++i) nact += (x.hl0 + i < p.g) ? 1 : 0;
-        mbar_arrive_expect_tx(bar(C::BAR_Q), (uint32_t)nact * C::TILE);
-        for (int i = 0; i < C::NSLOT; ++i) {
-          if (x.hl0 + i >= p.g) continue;
-          const int h = x.kvh * p.g + x.hl0 + i;
+        if constexpr (PAIR) {
+          // this CTA's head of the pair
+          mbar_arrive_expect_tx(bar(C::BAR_Q), C::TILE);
           for (int kb = 0; kb < C::KB; ++kb)
-            tma_load_4d(base + C::OFF_Q + i * C::TILE + kb * BOX_BYTES, &tm_q, bar(C::BAR_Q), kb * 64, h,
-                        x.s0, x.b);
+            tma_load_4d(base + C::OFF_Q + kb * BOX_BYTES, &tm_q, bar(C::BAR_Q), kb * 64,
+                        x.kvh * p.g + x.hl0 + (int)rank, x.s0, x.b);
+        } else {
+          int nact = 0;
+          for (int i = 0; i < C::NSLOT; ++i) nact += (x.hl0 + i < p.g) ? 1 : 0;
+          mbar_arrive_expect_tx(bar(C::BAR_Q), (uint32_t)nact * C::TILE);
+          for (int i = 0; i < C::NSLOT; ++i) {
+            if (x.hl0 + i >= p.g) continue;
+            const int h = x.kvh * p.g + x.hl0 + i;
+            for (int kb = 0; kb < C::KB; ++kb)
+              tma_load_4d(base + C::OFF_Q + i * C::TILE + kb * BOX_BYTES, &tm_q, bar(C::BAR_Q), kb * 64, h,
+                          x.s0, x.b);
+          }
         }
         q_issued = k + 1;
         for (int m = 0; m < 2 * x.n_tiles; ++m, ++n) {
@@ -366,12 +429,28 @@ __global__ void __launch_bounds__(PrefillCfg<DK, DV, MODE == MODE_ALIBI_MASK || 
           if (use > 0 && !mbar_wait(bar(C::bar_empty(buf)), (uint32_t)(use - 1) & 1u, wd)) { ok = false; break; }
           int tile;
           const bool is_v = ring_item<C::NSLOT>(m, x.n_tiles, tile);
-          const CUtensorMap* tm = is_v ? &tm_v : &tm_k;
-          const int nb = is_v ? C::VB : C::KB;
-          mbar_arrive_expect_tx(bar(C::bar_full(buf)), (uint32_t)nb * BOX_BYTES);
-          for (int kb = 0; kb < nb; ++kb)
-            tma_load_4d(base + C::OFF_KV + buf * C::TILE + kb * BOX_BYTES, tm, bar(C::bar_full(buf)),
-                        kb * 64, x.kvh, (x.t0 + (rev ? x.n_tiles - 1 - tile : tile)) * BN, x.b);
+          const int key0 = (x.t0 + (rev ? x.n_tiles - 1 - tile : tile)) * BN;
+          const uint32_t dst = base + C::OFF_KV + buf * C::RSLOT;
+          // a K or V tile (VB boxes for V when DV < DK), or half of one (PAIR)
+          mbar_arrive_expect_tx(bar(C::bar_full(buf)), PAIR ? C::RSLOT : (uint32_t)(is_v ? C::VB : C::KB) * BOX_BYTES);
+          if constexpr (PAIR) {
+            if (is_v) {
+              // V: all 128 keys, D columns rank*DV/2 .. (rank+1)*DV/2 - 1
+              for (int vb = 0; vb < C::VB / 2; ++vb)
+                tma_load_4d(dst + vb * BOX_BYTES, &tm_v, bar(C::bar_full(buf)), (int)rank * (DV / 2) + vb * 64, x.kvh,
+                            key0, x.b);
+            } else {
+              // K: keys key0 + 64*rank .. + 63 (tm_k tiles K in 64-key boxes)
+              for (int kb = 0; kb < C::KB; ++kb)
+                tma_load_4d(dst + kb * (BOX_BYTES / 2), &tm_k, bar(C::bar_full(buf)), kb * 64, x.kvh,
+                            key0 + 64 * (int)rank, x.b);
+            }
+          } else {
+            const CUtensorMap* tm = is_v ? &tm_v : &tm_k;
+            const int nb = is_v ? C::VB : C::KB;
+            for (int kb = 0; kb < nb; ++kb)
+              tma_load_4d(dst + kb * BOX_BYTES, tm, bar(C::bar_full(buf)), kb * 64, x.kvh, key0, x.b);
+          }
           issued = n + 1;
         }
       }
@@ -384,9 +463,9 @@ __global__ void __launch_bounds__(PrefillCfg<DK, DV, MODE == MODE_ALIBI_MASK || 
       bool ok = true;
       int tg = 0;   // this CTA's tiles so far
       for (int k = 0; ok; ++k) {
-        const int u = unit_index(k, total_units);
+        const int u = next_unit(k);
         if (u < 0) break;
-        const Unit x = unit_at<C::NSLOT>(u, p);
+        const Unit x = unit_at<UG>(u, p);
         for (int j = 0; ok && j < x.n_tiles; ++j, ++tg) {
           const int key0 = (x.t0 + (rev ? x.n_tiles - 1 - j : j)) * BN;
           for (int h = 0; h < 2; ++h) {
@@ -403,11 +482,35 @@ __global__ void __launch_bounds__(PrefillCfg<DK, DV, MODE == MODE_ALIBI_MASK || 
       }
     }
   } else if (warp == C::WARP_MMA) {
-    if (lane == 0) {
-      constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, false, false);
-      constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, false, true);
+    if (PAIR && rank == 1 && lane == 0) {
+      // The peer's loads complete on its own barriers; forward each completion
+      // (Q of every unit, then its ring items in order) to the leader's
+      // barrier of the same index, where the MMAs wait for both halves.
+      int n = 0;
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int u = next_unit(k);
+        if (u < 0) break;
+        const Unit x = unit_at<UG>(u, p);
+        if (!(ok = mbar_wait(bar(C::BAR_Q), (uint32_t)k & 1u, wd))) break;
+        mbar_relay_cluster(mapa_shared(bar(C::BAR_Q), 0));
+        for (int m = 0; m < 2 * x.n_tiles; ++m, ++n) {
+          if (!(ok = mbar_wait(bar(C::bar_full(n % C::NBUF)), (uint32_t)(n / C::NBUF) & 1u, wd))) break;
+          mbar_relay_cluster(mapa_shared(bar(C::bar_full(n % C::NBUF)), 0));
+        }
+      }
+    } else if (lane == 0 && (!PAIR || rank == 0)) {
+      // PAIR: 2-CTA MMAs over M = 256 rows (both heads of the pair)
+      constexpr uint32_t IDESC_QK = idesc_bf16_f32(PAIR ? 2 * BM : BM, BN, false, false);
+      constexpr uint32_t IDESC_PV = idesc_bf16_f32(PAIR ? 2 * BM : BM, D, false, true);
+      // completions arrive on this CTA's barrier, or on the barrier at the same
+      // offset in both CTAs of the pair
+      auto commit = [&](uint32_t b) {
+        if constexpr (PAIR) mma_commit_pair(b);
+        else mma_commit(b);
+      };
       auto wait_full = [&](int n) -> bool {
-        if (!mbar_wait(bar(C::bar_full(n % C::NBUF)), (uint32_t)(n / C::NBUF) & 1u, wd)) return false;
+        if (!wait_x(bar(C::bar_full(n % C::NBUF)), (uint32_t)(n / C::NBUF) & 1u, wd)) return false;
         tc_fence_after();
         return true;
       };
@@ -418,35 +521,46 @@ __global__ void __launch_bounds__(PrefillCfg<DK, DV, MODE == MODE_ALIBI_MASK || 
       const uint64_t qdesc0 = sdesc_sw128(base + C::OFF_Q, 16, 1024);
       const uint64_t kdesc0 = sdesc_sw128(base + C::OFF_KV, 16, 1024);
       const uint64_t vdesc0 = sdesc_sw128(base + C::OFF_KV, BOX_BYTES, 1024);
+      // K boxes: 128 rows (64 in the pair form) of 128 bytes
+      constexpr uint32_t KBOX = PAIR ? BOX_BYTES / 2 : BOX_BYTES;
       // S buffer sb = Q(qslot) K^T
       auto gemm_s = [&](int sb, int qslot, int ring_n) {
         const uint64_t qd = qdesc0 + (uint64_t)(((uint32_t)qslot * C::TILE) >> 4);
-        const uint64_t kd = kdesc0 + (uint64_t)(((uint32_t)(ring_n % C::NBUF) * C::TILE) >> 4);
+        const uint64_t kd = kdesc0 + (uint64_t)(((uint32_t)(ring_n % C::NBUF) * C::RSLOT) >> 4);
 #pragma unroll
         for (int kk = 0; kk < DK / 16; ++kk) {
-          const uint64_t off = (uint64_t)((((uint32_t)(kk >> 2) * BOX_BYTES) + (uint32_t)(kk & 3) * 32u) >> 4);
-          mma_ss(tmem + C::TMEM_S + sb * 128, qd + off, kd + off, IDESC_QK, kk > 0 ? 1u : 0u);
+          const uint64_t qo = (uint64_t)((((uint32_t)(kk >> 2) * BOX_BYTES) + (uint32_t)(kk & 3) * 32u) >> 4);
+          const uint64_t ko = (uint64_t)((((uint32_t)(kk >> 2) * KBOX) + (uint32_t)(kk & 3) * 32u) >> 4);
+          if constexpr (PAIR)
+            mma_ss_pair(tmem + C::TMEM_S + sb * 128, qd + qo, kd + ko, IDESC_QK, kk > 0 ? 1u : 0u);
+          else
+            mma_ss(tmem + C::TMEM_S + sb * 128, qd + qo, kd + ko, IDESC_QK, kk > 0 ? 1u : 0u);
         }
       };
       // O(oslot) (+)= P(from S buffer pb) V, each half of P as soon as it is
       // in TMEM (phase: completion index of that buffer's P barriers)
       auto gemm_pv = [&](int oslot, int pb, int ring_n, bool first, uint32_t phase) -> bool {
-        const uint64_t vd = vdesc0 + (uint64_t)(((uint32_t)(ring_n % C::NBUF) * C::TILE) >> 4);
+        const uint64_t vd = vdesc0 + (uint64_t)(((uint32_t)(ring_n % C::NBUF) * C::RSLOT) >> 4);
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          if (!mbar_wait(bar(half == 0 ? C::bar_plo(pb) : C::bar_phi(pb)), phase & 1u, wd)) return false;
+          if (!wait_x(bar(half == 0 ? C::bar_plo(pb) : C::bar_phi(pb)), phase & 1u, wd)) return false;
           tc_fence_after();
 #pragma unroll
-          for (int kk = half * (BN / 32); kk < (half + 1) * (BN / 32); ++kk)
-            mma_ts(tmem + C::TMEM_O + oslot * D, tmem + C::TMEM_S + pb * 128 + kk * 8,
-                   vd + (uint64_t)((kk * 2048u) >> 4), IDESC_PV, (!first || kk > 0) ? 1u : 0u);
+          for (int kk = half * (BN / 32); kk < (half + 1) * (BN / 32); ++kk) {
+            if constexpr (PAIR)
+              mma_ts_pair(tmem + C::TMEM_O + oslot * D, tmem + C::TMEM_S + pb * 128 + kk * 8,
+                          vd + (uint64_t)((kk * 2048u) >> 4), IDESC_PV, (!first || kk > 0) ? 1u : 0u);
+            else
+              mma_ts(tmem + C::TMEM_O + oslot * D, tmem + C::TMEM_S + pb * 128 + kk * 8,
+                     vd + (uint64_t)((kk * 2048u) >> 4), IDESC_PV, (!first || kk > 0) ? 1u : 0u);
+          }
         }
         return true;
       };
       auto wait_ofree = [&](int slot, int units_done) -> bool {
         // the previous unit's epilogue on this slot must be done reading O
         if (units_done == 0) return true;
-        if (!mbar_wait(bar(C::bar_ofree(slot)), (uint32_t)(units_done - 1) & 1u, wd)) return false;
+        if (!wait_x(bar(C::bar_ofree(slot)), (uint32_t)(units_done - 1) & 1u, wd)) return false;
         tc_fence_after();
         return true;
       };
@@ -455,48 +569,48 @@ __global__ void __launch_bounds__(PrefillCfg<DK, DV, MODE == MODE_ALIBI_MASK || 
       int T0 = 0, T1 = 0;              // tiles completed per slot (barrier phases)
       int U0 = 0, U1 = 0;              // units completed per slot
       for (int k = 0; ok; ++k) {
-        const int u = unit_index(k, total_units);
+        const int u = next_unit(k);
         if (u < 0) break;
-        const Unit x = unit_at<C::NSLOT>(u, p);
+        const Unit x = unit_at<UG>(u, p);
         const int nt = x.n_tiles;
         const bool act1 = (C::NSLOT == 2) && (x.hl0 + 1 < p.g);
-        if (!(ok = mbar_wait(bar(C::BAR_Q), (uint32_t)k & 1u, wd))) break;
+        if (!(ok = wait_x(bar(C::BAR_Q), (uint32_t)k & 1u, wd))) break;
         tc_fence_after();
         if (C::NSLOT == 2) {
           // tile 0
           if (!(ok = wait_full(n))) break;
           gemm_s(0, 0, n);
-          mma_commit(bar(C::bar_s(0)));
+          commit(bar(C::bar_s(0)));
           if (act1) {
             gemm_s(1, 1, n);
-            mma_commit(bar(C::bar_s(1)));
+            commit(bar(C::bar_s(1)));
           }
-          if (nt == 1) mma_commit(bar(C::BAR_QE));            // last S of the unit
-          mma_commit(bar(C::bar_empty(n % C::NBUF)));
+          if (nt == 1) commit(bar(C::BAR_QE));            // last S of the unit
+          commit(bar(C::bar_empty(n % C::NBUF)));
           if (!(ok = wait_full(n + 1) && wait_ofree(0, U0) &&
                      gemm_pv(0, 0, n + 1, true, (uint32_t)T0)))
             break;
-          mma_commit(bar(C::bar_pv(0)));
+          commit(bar(C::bar_pv(0)));
           for (int i = 1; i < nt; ++i) {
             const int nk = n + 2 * i;
             if (!(ok = wait_full(nk))) break;
             gemm_s(0, 0, nk);                                 // S0_i (behind O0 += P0_{i-1} V_{i-1})
-            mma_commit(bar(C::bar_s(0)));
+            commit(bar(C::bar_s(0)));
             if (act1) {
               if (!(ok = (i > 1 || wait_ofree(1, U1)) &&
                          gemm_pv(1, 1, nk - 1, i == 1, (uint32_t)(T1 + i - 1))))
                 break;                                        // O1 += P1_{i-1} V_{i-1}
-              mma_commit(bar(C::bar_pv(1)));
+              commit(bar(C::bar_pv(1)));
             }
-            mma_commit(bar(C::bar_empty((nk - 1) % C::NBUF)));  // V_{i-1} done
+            commit(bar(C::bar_empty((nk - 1) % C::NBUF)));  // V_{i-1} done
             if (act1) {
               gemm_s(1, 1, nk);                               // S1_i (behind the P1 read)
-              mma_commit(bar(C::bar_s(1)));
+              commit(bar(C::bar_s(1)));
             }
-            if (i == nt - 1) mma_commit(bar(C::BAR_QE));      // last S of the unit
-            mma_commit(bar(C::bar_empty(nk % C::NBUF)));      // K_i done
+            if (i == nt - 1) commit(bar(C::BAR_QE));      // last S of the unit
+            commit(bar(C::bar_empty(nk % C::NBUF)));      // K_i done
             if (!(ok = wait_full(nk + 1) && gemm_pv(0, 0, nk + 1, false, (uint32_t)(T0 + i)))) break;
-            mma_commit(bar(C::bar_pv(0)));                    // O0 += P0_i V_i
+            commit(bar(C::bar_pv(0)));                    // O0 += P0_i V_i
           }
           if (!ok) break;
           const int nv = n + 2 * nt - 1;
@@ -504,9 +618,9 @@ __global__ void __launch_bounds__(PrefillCfg<DK, DV, MODE == MODE_ALIBI_MASK || 
             if (!(ok = (nt > 1 || wait_ofree(1, U1)) &&
                        gemm_pv(1, 1, nv, nt == 1, (uint32_t)(T1 + nt - 1))))
               break;
-            mma_commit(bar(C::bar_pv(1)));
+            commit(bar(C::bar_pv(1)));
           }
-          mma_commit(bar(C::bar_empty(nv % C::NBUF)));
+          commit(bar(C::bar_empty(nv % C::NBUF)));
           T0 += nt;
           ++U0;
           if (act1) {
@@ -517,25 +631,25 @@ __global__ void __launch_bounds__(PrefillCfg<DK, DV, MODE == MODE_ALIBI_MASK || 
           // one slot, S double buffered across tiles and units: buffer (T0 + j) % 2
           if (!(ok = wait_full(n))) break;
           gemm_s(T0 & 1, 0, n);
-          mma_commit(bar(C::bar_s(T0 & 1)));
-          if (nt == 1) mma_commit(bar(C::BAR_QE));
-          mma_commit(bar(C::bar_empty(n % C::NBUF)));
+          commit(bar(C::bar_s(T0 & 1)));
+          if (nt == 1) commit(bar(C::BAR_QE));
+          commit(bar(C::bar_empty(n % C::NBUF)));
           ++n;
           for (int j = 0; j < nt; ++j) {
             const int G = T0 + j;
             if (j + 1 < nt) {
               if (!(ok = wait_full(n))) break;
               gemm_s((G + 1) & 1, 0, n);                      // behind the P.V that read this buffer
-              mma_commit(bar(C::bar_s((G + 1) & 1)));
-              if (j + 2 == nt) mma_commit(bar(C::BAR_QE));    // last S of the unit
-              mma_commit(bar(C::bar_empty(n % C::NBUF)));
+              commit(bar(C::bar_s((G + 1) & 1)));
+              if (j + 2 == nt) commit(bar(C::BAR_QE));    // last S of the unit
+              commit(bar(C::bar_empty(n % C::NBUF)));
               ++n;
             }
             if (!(ok = wait_full(n) && (j > 0 || wait_ofree(0, U0)) &&
                        gemm_pv(0, G & 1, n, j == 0, (uint32_t)(G >> 1))))
               break;
-            mma_commit(bar(C::bar_pv(0)));
-            mma_commit(bar(C::bar_empty(n % C::NBUF)));
+            commit(bar(C::bar_pv(0)));
+            commit(bar(C::bar_empty(n % C::NBUF)));
             ++n;
           }
           if (!ok) break;
@@ -544,6 +658,31 @@ __global__ void __launch_bounds__(PrefillCfg<DK, DV, MODE == MODE_ALIBI_MASK || 
           continue;
         }
         n += 2 * nt;
+      }
+    }
+  } else if (PAIR && warp == C::WARP_RELAY) {
+    if (rank == 1 && lane == 0) {
+      // The peer's softmax warps arrive on its own P and O-free barriers
+      // (a remote arrive stalls the arriving warp); relay each completed
+      // phase, in the order the leader's MMAs wait for them, to the leader's
+      // barrier of the same index.
+      int T = 0;
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int u = next_unit(k);
+        if (u < 0) break;
+        const Unit x = unit_at<UG>(u, p);
+        for (int j = 0; ok && j < x.n_tiles; ++j) {
+          const int G = T + j;
+          for (int half = 0; half < 2; ++half) {
+            const uint32_t b = bar(half == 0 ? C::bar_plo(G & 1) : C::bar_phi(G & 1));
+            if (!(ok = mbar_wait(b, (uint32_t)(G >> 1) & 1u, wd))) break;
+            mbar_relay_cluster(mapa_shared(b, 0));
+          }
+        }
+        if (!ok || !(ok = mbar_wait(bar(C::bar_ofree(0)), (uint32_t)k & 1u, wd))) break;
+        mbar_relay_cluster(mapa_shared(bar(C::bar_ofree(0)), 0));
+        T += x.n_tiles;
       }
     }
   } else {
@@ -557,10 +696,10 @@ __global__ void __launch_bounds__(PrefillCfg<DK, DV, MODE == MODE_ALIBI_MASK || 
     int T = 0;  // tiles this slot completed in earlier units (barrier phases)
     bool ok = true;
     for (int k = 0; ok; ++k) {
-      const int u = unit_index(k, total_units);
+      const int u = next_unit(k);
       if (u < 0) break;
-      const Unit x = unit_at<C::NSLOT>(u, p);
-      const int hl = x.hl0 + slot;
+      const Unit x = unit_at<UG>(u, p);
+      const int hl = x.hl0 + (PAIR ? (int)rank : slot);
       if (hl >= p.g) continue;  // slot unused in this unit (odd group size)
       const int n_tiles = x.n_tiles;
       const int h = x.kvh * p.g + hl;
@@ -687,7 +826,12 @@ __global__ void __launch_bounds__(PrefillCfg<DK, DV, MODE == MODE_ALIBI_MASK || 
           tmem_st32u(tS, pk);
           tmem_wait_st();
           tc_fence_before();
-          mbar_arrive(bar(C::bar_plo(sb)));
+          if constexpr (PAIR) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::bar_plo(sb)));
+          } else {
+            mbar_arrive(bar(C::bar_plo(sb)));
+          }
         }
         // half 1: keys 64-127, re-read from TMEM columns 64-127 (P only ever
         // covers columns 0-63), so their registers need not stay live above
@@ -707,7 +851,12 @@ __global__ void __launch_bounds__(PrefillCfg<DK, DV, MODE == MODE_ALIBI_MASK || 
           tmem_st32u(tS + BN / 4, pk);
           tmem_wait_st();
           tc_fence_before();
-          mbar_arrive(bar(C::bar_phi(sb)));
+          if constexpr (PAIR) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::bar_phi(sb)));
+          } else {
+            mbar_arrive(bar(C::bar_phi(sb)));
+          }
         }
         l = l * alpha + ((acc0.x + acc0.y) + (acc1.x + acc1.y));
         m_use = m_new;
@@ -766,7 +915,12 @@ __global__ void __launch_bounds__(PrefillCfg<DK, DV, MODE == MODE_ALIBI_MASK || 
       }
       // O of this slot may now be overwritten by the next unit's first P.V
       tc_fence_before();
-      mbar_arrive(bar(C::bar_ofree(slot)));
+      if constexpr (PAIR) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(C::bar_ofree(slot)));
+      } else {
+        mbar_arrive(bar(C::bar_ofree(slot)));
+      }
       T += n_tiles;
     }
     tc_fence_before();
@@ -788,16 +942,26 @@ __global__ void __launch_bounds__(PrefillCfg<DK, DV, MODE == MODE_ALIBI_MASK || 
       for (int n = max(0, issued - C::NBUF); n < issued; ++n)
         drain_wait(bar(C::bar_full(n % C::NBUF)), (uint32_t)(n / C::NBUF) & 1u, p.timeout_ns);
     }
-    if (warp == C::WARP_MMA && lane == 0) {
-      mma_commit(bar(C::BAR_DRAIN));
+    if (warp == C::WARP_MMA && lane == 0 && (!PAIR || rank == 0)) {
+      if constexpr (PAIR) mma_commit_pair(bar(C::BAR_DRAIN));
+      else mma_commit(bar(C::BAR_DRAIN));
       drain_wait(bar(C::BAR_DRAIN), 0, p.timeout_ns);
     }
     __syncwarp();
     __syncthreads();
   }
+  if constexpr (PAIR) {
+    // the leader's MMAs read this CTA's shared memory and write its TMEM:
+    // neither CTA frees either before both are done (every wait above is
+    // bounded, so both CTAs reach this barrier)
+    tc_fence_before();
+    cg::this_cluster().sync();
+    tc_fence_after();
+  }
   if (warp == C::WARP_MMA) {
     tc_fence_after();
-    tmem_dealloc(tmem, C::TMEM_COLS);
+    if constexpr (PAIR) tmem_dealloc2(tmem, C::TMEM_COLS);
+    else tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 
@@ -815,7 +979,53 @@ int launch_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv
   return (int)cudaGetLastError();
 }
 
+// The CTA-pair form: clusters of two CTAs, as many as fit at once (at most
+// one per unit); tk64 tiles K in 64-key boxes.
+template <int D, int MODE>
+int launch_pair_t(const CUtensorMap& tq, const CUtensorMap& tk64, const CUtensorMap& tv, const PrefillParams& p,
+                  cudaStream_t stream) {
+  using C = PrefillCfg<D, D, false, true>;
+  auto kern = prefill_kernel<D, D, MODE, true>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+  if (e != cudaSuccess) return (int)e;
+  const long long units = (long long)p.n_qt * p.B * p.Hkv * p.units_per_kvh;
+  if (units <= 0 || units > 0x7fffffffLL || p.num_ctas < 2) return (int)cudaErrorInvalidValue;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  long long clusters = p.num_ctas / 2;
+  cfg.gridDim = dim3((unsigned)(2 * clusters));
+  int fit = 0;
+  if (cudaOccupancyMaxActiveClusters(&fit, kern, &cfg) == cudaSuccess && fit > 0 && fit < clusters) clusters = fit;
+  (void)cudaGetLastError();   // an occupancy query that failed leaves the grid at one cluster per SM pair
+  if (units < clusters) clusters = units;
+  cfg.gridDim = dim3((unsigned)(2 * clusters));
+  e = cudaLaunchKernelEx(&cfg, kern, tq, tk64, tv, tv, p);
+  if (e != cudaSuccess) return (int)e;
+  return (int)cudaGetLastError();
+}
+
 }  // namespace
+
+int launch_prefill_pair(int D, bool ext, const CUtensorMap& tq, const CUtensorMap& tk64, const CUtensorMap& tv,
+                        const PrefillParams& p, cudaStream_t stream) {
+  if (D != 256 || p.ext.mask != nullptr || p.g % 2 != 0) return (int)cudaErrorInvalidValue;
+  const int mode = !ext ? MODE_PLAIN : p.ext.cap_a > 0.f ? MODE_CAP : p.ext.alibi ? MODE_ALIBI : MODE_MASKS;
+  switch (mode) {
+    case MODE_PLAIN: return launch_pair_t<256, MODE_PLAIN>(tq, tk64, tv, p, stream);
+    case MODE_MASKS: return launch_pair_t<256, MODE_MASKS>(tq, tk64, tv, p, stream);
+    case MODE_ALIBI: return launch_pair_t<256, MODE_ALIBI>(tq, tk64, tv, p, stream);
+    default: return launch_pair_t<256, MODE_CAP>(tq, tk64, tv, p, stream);
+  }
+}
 
 size_t prefill_smem_bytes(int D, int Dv) {
   if (D == Dv) {
