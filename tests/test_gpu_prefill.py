@@ -29,6 +29,8 @@ CASES = [
     (2, 8, 8, 128, 128, 64, 0, True, torch.bfloat16),
     (1, 4, 1, 300, 200, 128, 0, True, torch.bfloat16),     # Sq > Skv: late rows see every key
     (1, 4, 2, 256, 1100, 128, 0, False, torch.float32),    # non-causal, many tiles
+    (1, 6, 1, 300, 300, 256, 0, True, torch.bfloat16),     # D = 256, group of 6: three CTA pairs per K/V head
+    (1, 2, 2, 200, 333, 256, 133, True, torch.float32),    # D = 256, MHA: one CTA per head (no pair)
 ]
 
 
