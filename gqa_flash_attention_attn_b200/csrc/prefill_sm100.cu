@@ -335,7 +335,13 @@ __global__ void __launch_bounds__(PrefillCfg<DK, DV, MODE == MODE_ALIBI_MASK || 
   // With ALiBi the bias grows toward each query's own position: visiting a
   // unit's K/V tiles newest first sets the running maximum on the first tile
   // and spares the O rescales (the tile order does not change the result).
-  const bool rev = MODE >= MODE_ALIBI && p.ext.alibi != 0;
+  const bool rev_alibi = MODE >= MODE_ALIBI && p.ext.alibi != 0;
+  // In the CTA-pair form, units a cluster takes second, fourth, ... (odd k)
+  // also run newest first: they start while the first wave's most recent K/V
+  // tiles are still in L2 and reach the oldest tiles last, instead of
+  // re-reading those from DRAM first (prefill at depth: DRAM reads 173 -> 130
+  // MB).  Every role derives a unit's tile order from the same k.
+  auto unit_rev = [&](int k) -> bool { return rev_alibi || (PAIR && (k & 1) != 0); };
 
   if (threadIdx.x == 0) {
     // PAIR: the leader's Q and ring barriers also count the peer's forwarded
@@ -429,7 +435,7 @@ __global__ void __launch_bounds__(PrefillCfg<DK, DV, MODE == MODE_ALIBI_MASK || 
           if (use > 0 && !mbar_wait(bar(C::bar_empty(buf)), (uint32_t)(use - 1) & 1u, wd)) { ok = false; break; }
           int tile;
           const bool is_v = ring_item<C::NSLOT>(m, x.n_tiles, tile);
-          const int key0 = (x.t0 + (rev ? x.n_tiles - 1 - tile : tile)) * BN;
+          const int key0 = (x.t0 + (unit_rev(k) ? x.n_tiles - 1 - tile : tile)) * BN;
           const uint32_t dst = base + C::OFF_KV + buf * C::RSLOT;
           // a K or V tile (VB boxes for V when DV < DK), or half of one (PAIR)
           mbar_arrive_expect_tx(bar(C::bar_full(buf)), PAIR ? C::RSLOT : (uint32_t)(is_v ? C::VB : C::KB) * BOX_BYTES);
@@ -467,7 +473,7 @@ __global__ void __launch_bounds__(PrefillCfg<DK, DV, MODE == MODE_ALIBI_MASK || 
         if (u < 0) break;
         const Unit x = unit_at<UG>(u, p);
         for (int j = 0; ok && j < x.n_tiles; ++j, ++tg) {
-          const int key0 = (x.t0 + (rev ? x.n_tiles - 1 - j : j)) * BN;
+          const int key0 = (x.t0 + (unit_rev(k) ? x.n_tiles - 1 - j : j)) * BN;
           for (int h = 0; h < 2; ++h) {
             if (tg > 0 && !mbar_wait(bar(C::bar_mempty(h)), (uint32_t)(tg - 1) & 1u, wd)) {
               ok = false;
@@ -724,7 +730,7 @@ __global__ void __launch_bounds__(PrefillCfg<DK, DV, MODE == MODE_ALIBI_MASK || 
         const bool got = mbar_wait(bar(C::bar_s(sb)), ph, wd);
         if (__any_sync(0xffffffffu, !got)) { ok = false; break; }
         tc_fence_after();
-        const int key0 = (x.t0 + (rev ? n_tiles - 1 - j : j)) * BN;
+        const int key0 = (x.t0 + (unit_rev(k) ? n_tiles - 1 - j : j)) * BN;
         const int cl = vis_end - key0;    // visible columns of this tile: [cb, cl)
         const int cb = vis_begin - key0;
         const bool tile_masked = __any_sync(0xffffffffu, cl < BN || cb > 0);
