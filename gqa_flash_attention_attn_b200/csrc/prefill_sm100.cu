@@ -62,7 +62,9 @@ constexpr float LN2 = 0.6931471805599453f;
 // and issue slots past the point of gain (measured).
 constexpr uint32_t kPolyPairs = 0x80808080u;
 
-// MB: the variant reads an additive mask, staged by TMA in two 64-key halves.
+// MB: the variant reads an additive mask, staged by TMA in two 64-key halves,
+// in two stages where shared memory allows (D <= 128), so that the next
+// tile's mask loads while both head slots still read this one.
 // DK: the Q and K head size; DV: the V and O head size (DV <= DK).
 // PAIR: the CTA-pair form (one head slot per CTA, half K/V tiles per CTA).
 template <int DK, int DV = DK, bool MB = false, bool PAIR = false>
@@ -74,7 +76,8 @@ struct PrefillCfg {
   // PAIR: a ring slot holds half a tile: 64 keys x DK of K (KB boxes of 64
   // rows) or 128 keys x DV/2 of V (VB/2 boxes of 128 rows)
   static constexpr uint32_t RSLOT = PAIR ? TILE / 2 : TILE;
-  static constexpr int NBUF = PAIR ? 5 : (DK == 64) ? 8 : (DK == 128 ? 4 : 2);
+  static constexpr int NBUF = PAIR ? 5 : (DK == 64) ? 8 : (DK == 128 ? (MB ? 3 : 4) : 2);
+  static constexpr int MSTAGES = DK <= 128 ? 2 : 1;   // mask stages (with MB)
   // PAIR: one more warp, whose thread in the peer relays the P-ready and
   // O-free signals of the peer's softmax warps to the leader
   static constexpr int THREADS = 128 * NSLOT + 64 + (PAIR ? 32 : 0);
@@ -85,10 +88,10 @@ struct PrefillCfg {
   static constexpr uint32_t OFF_KV = NSLOT * TILE;
   static constexpr uint32_t MASK_HALF = BM * 128u;          // 128 rows x 64 bf16 keys
   static constexpr uint32_t OFF_MASK = OFF_KV + NBUF * RSLOT;
-  static constexpr uint32_t OFF_BAR = OFF_MASK + (MB ? 2u * MASK_HALF : 0u);
+  static constexpr uint32_t OFF_BAR = OFF_MASK + (MB ? MSTAGES * 2u * MASK_HALF : 0u);
   // q_full, q_empty, kv_full[NBUF], kv_empty[NBUF], s_full[2], p_lo[2], p_hi[2],
-  // pv_done[2], o_free[2], drain; with MB mask_full[2], mask_empty[2]
-  static constexpr int NBARS = 2 + 2 * NBUF + 10 + 1 + (MB ? 4 : 0);
+  // pv_done[2], o_free[2], drain; with MB mask_full[MSTAGES][2], mask_empty[MSTAGES][2]
+  static constexpr int NBARS = 2 + 2 * NBUF + 10 + 1 + (MB ? 4 * MSTAGES : 0);
   static constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
   static constexpr uint32_t SMEM = OFF_MISC + 16 + 1024;  // + alignment slack
   // Two S buffers (one per slot, or a double buffer for one slot), P aliased
@@ -106,8 +109,14 @@ struct PrefillCfg {
   __host__ __device__ static constexpr int bar_pv(int i) { return 8 + 2 * NBUF + i; }
   __host__ __device__ static constexpr int bar_ofree(int i) { return 10 + 2 * NBUF + i; }
   static constexpr int BAR_DRAIN = 12 + 2 * NBUF;
-  __host__ __device__ static constexpr int bar_mfull(int h) { return 13 + 2 * NBUF + h; }
-  __host__ __device__ static constexpr int bar_mempty(int h) { return 15 + 2 * NBUF + h; }
+  __host__ __device__ static constexpr int bar_mfull(int st, int h) { return 13 + 2 * NBUF + 2 * st + h; }
+  __host__ __device__ static constexpr int bar_mempty(int st, int h) {
+    return 13 + 2 * NBUF + 2 * MSTAGES + 2 * st + h;
+  }
+  // shared-memory offset of half h of mask stage st
+  __host__ __device__ static constexpr uint32_t off_mask(int st, int h) {
+    return OFF_MASK + (uint32_t)(2 * st + h) * MASK_HALF;
+  }
   static_assert(256 + NSLOT * DV <= 512, "TMEM budget");
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(DK % 64 == 0 && DV % 64 == 0 && DV <= DK, "head dims");
@@ -365,10 +374,11 @@ __global__ void __launch_bounds__(PrefillCfg<DK, DV, MODE == MODE_ALIBI_MASK || 
     }
     mbar_init(bar(C::BAR_DRAIN), 1);
     if constexpr (MB) {
-      for (int h = 0; h < 2; ++h) {
-        mbar_init(bar(C::bar_mfull(h)), 1);
-        mbar_init(bar(C::bar_mempty(h)), 4 * C::NSLOT);   // one arrival per softmax warp
-      }
+      for (int st = 0; st < C::MSTAGES; ++st)
+        for (int h = 0; h < 2; ++h) {
+          mbar_init(bar(C::bar_mfull(st, h)), 1);
+          mbar_init(bar(C::bar_mempty(st, h)), 4 * C::NSLOT);   // one arrival per softmax warp
+        }
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -474,13 +484,14 @@ __global__ void __launch_bounds__(PrefillCfg<DK, DV, MODE == MODE_ALIBI_MASK || 
         const Unit x = unit_at<UG>(u, p);
         for (int j = 0; ok && j < x.n_tiles; ++j, ++tg) {
           const int key0 = (x.t0 + (unit_rev(k) ? x.n_tiles - 1 - j : j)) * BN;
+          const int st = tg % C::MSTAGES, use = tg / C::MSTAGES;   // stage, and its use count
           for (int h = 0; h < 2; ++h) {
-            if (tg > 0 && !mbar_wait(bar(C::bar_mempty(h)), (uint32_t)(tg - 1) & 1u, wd)) {
+            if (use > 0 && !mbar_wait(bar(C::bar_mempty(st, h)), (uint32_t)(use - 1) & 1u, wd)) {
               ok = false;
               break;
             }
-            mbar_arrive_expect_tx(bar(C::bar_mfull(h)), C::MASK_HALF);
-            tma_load_4d(base + C::OFF_MASK + h * C::MASK_HALF, &tm_m, bar(C::bar_mfull(h)), key0 + 64 * h, x.s0,
+            mbar_arrive_expect_tx(bar(C::bar_mfull(st, h)), C::MASK_HALF);
+            tma_load_4d(base + C::off_mask(st, h), &tm_m, bar(C::bar_mfull(st, h)), key0 + 64 * h, x.s0,
                         p.ext.mask_sb != 0 ? x.b : 0, 0);
           }
           m_issued = tg + 1;
@@ -741,16 +752,20 @@ __global__ void __launch_bounds__(PrefillCfg<DK, DV, MODE == MODE_ALIBI_MASK || 
           // first, for their maximum only, so that one half of the row is
           // live at a time.  Their logits go back to their own TMEM columns
           // (P only ever covers columns 0-63), where half 1 below reads them.
-          // staged mask: wait for this tile's halves (global tile T + j)
+          // staged mask: wait for this tile's halves (tile G of this slot,
+          // and of the producer's mask stream)
           const bool mstaged = MB && p.mask_tma;
           const uint8_t* msm_hi = nullptr;
           const uint8_t* msm_lo = nullptr;
+          int mst = 0;
           if (mstaged) {
-            const uint32_t mph = (uint32_t)(T + j) & 1u;
-            const bool got_m = mbar_wait(bar(C::bar_mfull(1)), mph, wd) && mbar_wait(bar(C::bar_mfull(0)), mph, wd);
+            mst = G % C::MSTAGES;
+            const uint32_t mph = (uint32_t)(G / C::MSTAGES) & 1u;
+            const bool got_m =
+                mbar_wait(bar(C::bar_mfull(mst, 1)), mph, wd) && mbar_wait(bar(C::bar_mfull(mst, 0)), mph, wd);
             if (__any_sync(0xffffffffu, !got_m)) { ok = false; break; }
-            msm_lo = gbase + C::OFF_MASK + (uint32_t)r * 128u;
-            msm_hi = msm_lo + C::MASK_HALF;
+            msm_lo = gbase + C::off_mask(mst, 0) + (uint32_t)r * 128u;
+            msm_hi = gbase + C::off_mask(mst, 1) + (uint32_t)r * 128u;
           }
           float sh[BN / 2];
           tmem_ld64(tS + BN / 2, sh);
@@ -772,8 +787,8 @@ __global__ void __launch_bounds__(PrefillCfg<DK, DV, MODE == MODE_ALIBI_MASK || 
             // both halves read into registers: release them to the producer
             __syncwarp();
             if (lane == 0) {
-              mbar_arrive(bar(C::bar_mempty(0)));
-              mbar_arrive(bar(C::bar_mempty(1)));
+              mbar_arrive(bar(C::bar_mempty(mst, 0)));
+              mbar_arrive(bar(C::bar_mempty(mst, 1)));
             }
           }
           if (tile_masked) mask_cols(slo, cb, cl);
@@ -940,9 +955,11 @@ __global__ void __launch_bounds__(PrefillCfg<DK, DV, MODE == MODE_ALIBI_MASK || 
       if (q_issued > 0) drain_wait(bar(C::BAR_Q), (uint32_t)(q_issued - 1) & 1u, p.timeout_ns);
     }
     if (MB && warp == C::WARP_PRODUCER && lane == 1 && m_issued > 0) {
-      // only the last mask tile can still be in flight: an earlier one was
-      // consumed (after it arrived) before its buffer was reloaded
-      for (int h = 0; h < 2; ++h) drain_wait(bar(C::bar_mfull(h)), (uint32_t)(m_issued - 1) & 1u, p.timeout_ns);
+      // only the last MSTAGES mask tiles can still be in flight: an earlier
+      // one was consumed (after it arrived) before its stage was reloaded
+      for (int tg = max(0, m_issued - C::MSTAGES); tg < m_issued; ++tg)
+        for (int h = 0; h < 2; ++h)
+          drain_wait(bar(C::bar_mfull(tg % C::MSTAGES, h)), (uint32_t)(tg / C::MSTAGES) & 1u, p.timeout_ns);
     }
     if (warp == C::WARP_PRODUCER && lane == 0) {
       for (int n = max(0, issued - C::NBUF); n < issued; ++n)

@@ -236,6 +236,9 @@ MASKED_PREFILL = [
     (1, 8, 2, 256, 640, 128, 384, True, 20.0, 4.0, True, 256, 1),  # every term
     (1, 4, 2, 200, 600, 256, 400, True, 0.0, 8.0, False, 0, 1),     # D = 256 with ALiBi
     (1, 4, 2, 150, 333, 256, 183, True, 10.0, 0.0, True, 0, 1),     # D = 256 softcap, ragged
+    # more units than 2 x 148 CTAs: the mask stages carry across units
+    (2, 32, 8, 1280, 1280, 128, 0, True, 0.0, 4.0, False, 0, 2),
+    (2, 32, 8, 1200, 1280, 64, 80, True, 0.0, 0.0, False, 0, 1),
 ]
 
 
