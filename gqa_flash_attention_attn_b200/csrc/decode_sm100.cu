@@ -47,6 +47,8 @@ constexpr int WARP_MMA = 5;
 constexpr int MAX_NBUF = 6;
 constexpr int MAX_GROUP = 8;                   // consecutive splits per CTA
 constexpr int MAX_CLUSTER = 16;                // CTAs of one (b, kvh) merged in a cluster
+template <int N>
+struct IntC { static constexpr int value = N; };
 
 // One split of a CTA's group: its tiles are first .. first+nt-1 of the CTA's
 // tile stream; keys from kbase on a 128-key grid, the split ending at hi.
@@ -98,7 +100,7 @@ struct Layout {
     off_ring = (off_p + 2u * 2u * RP * 128u + 1023u) & ~1023u;  // two P buffers
     off_red = off_ring + (uint32_t)nbuf * (fp8 ? BOX_BYTES : SLOT_BYTES);
     off_row = off_red + 2u * 4u * RP * 4u;     // red_max[4][RP], red_sum[4][RP]
-    off_mask = off_row + 11u * RP * 4u;        // m, l, alpha, msub, inv, lim, limlo, pos, slope, mask row
+    off_mask = off_row + 13u * RP * 4u;        // m, l, alpha, msub, inv, lim, limlo, pos, slope, mask row, thrx, delta
     off_bar = off_mask + (uint32_t)mrows * 2u * MROW_BYTES;  // staged mask [2][mrows][136 keys] bf16
     off_bar = (off_bar + 7u) & ~7u;
     off_misc = off_bar + (uint32_t)(1 + 2 * nbuf + 8) * 8u;
@@ -305,6 +307,10 @@ __global__ void __launch_bounds__(THREADS, 2)
   int* pos_sm = limlo_sm + RP;                             // query position of row r
   float* slope_sm = reinterpret_cast<float*>(pos_sm + RP); // ALiBi slope * log2(e) of row r
   const uint16_t** mrow_sm = reinterpret_cast<const uint16_t**>(slope_sm + RP);  // mask row of row r
+  // one-pass tile loop: x > thrx_sm[r] moves row r's maximum (-inf while the
+  // row has none); delta_sm[r]: the shift of x when it does
+  float* thrx_sm = reinterpret_cast<float*>(mrow_sm + RP);
+  float* delta_sm = thrx_sm + RP;
   // staged mask: [2 tiles][mask_rows][136 keys] bf16, filled by cp.async one
   // tile ahead by all softmax threads
   const uint32_t mstage_u32 = base + L.off_mask;
@@ -422,6 +428,8 @@ __global__ void __launch_bounds__(THREADS, 2)
     const int r = threadIdx.x;
     m_sm[r] = -INFINITY;
     l_sm[r] = 0.f;
+    msub_sm[r] = 0.f;
+    thrx_sm[r] = -INFINITY;
     // last visible key of row r (padding rows see none)
     lim_sm[r] = r < R ? (p.causal ? q_offset + r / g : 0x7fffffff) : -1;
     pos_sm[r] = q_offset + (r < R ? r / g : 0);
@@ -745,6 +753,303 @@ __global__ void __launch_bounds__(THREADS, 2)
     // P-buffer wait has shown its last P.V complete: pend / pend_last.
     int pend = -1, pend_last = -1;
     SegCursor cs(seg_sm, nseg), cm(seg_sm, nseg);   // this tile; the mask stage's tile
+    // stage tile j+1's mask rows (and tile 0's first) with cp.async; the
+    // copies stay in flight across tile j's barriers, and tile j's are
+    // complete (and, after the next CTA barrier, visible) before use
+    // P of rows 16q..16q+15 at this thread's key (p values in v) into P
+    // buffer sb: bf16, or e4m3 hi + lo planes
+    auto store_p16 = [&](int sb, int q, float (&v)[16]) {
+      const int half = t >> 6, tt = t & 63;
+      uint8_t* pcol = gbase + PB(sb) + (size_t)half * RP * 128 + (size_t)(tt & 7) * 2;
+      const int chunk16 = tt >> 3;
+      if constexpr (!FP8) {
+        // bf16 P, one 32-bit word (keys t & ~1, t | 1) per store: for
+        // each pair of rows the even lane writes the even row and the odd
+        // lane the odd row, each taking its neighbour's value by shuffle
+        const bool odd = (t & 1) != 0;
+        uint8_t* pword = pcol - (size_t)(tt & 1) * 2;
+#pragma unroll
+        for (int e = 0; e < 16; e += 2) {
+          const float other = __shfl_xor_sync(0xffffffffu, odd ? v[e] : v[e + 1], 1);
+          const int r = 16 * q + e + (odd ? 1 : 0);
+          const uint32_t w = odd ? pack_bf16x2(other, v[e + 1]) : pack_bf16x2(v[e], other);
+          *reinterpret_cast<uint32_t*>(pword + (size_t)r * 128 + ((chunk16 ^ (r & 7)) << 4)) = w;
+        }
+      }
+      if constexpr (FP8) {
+        // P as hi + lo e4m3 planes (row r: 128 keys, one 128-byte
+        // swizzled row per plane).  A lane holds one key of 4 rows; a
+        // 4 x 4 byte transpose in each quad of lanes (two shuffle stages,
+        // both planes in one word) gives lane j the 4 keys of row e + j,
+        // so every store is a 32-bit word.
+        const int j4 = t & 3;
+        uint8_t* p8 = gbase + PB(sb) + ((t & 15) & ~3);
+        const int ck = t >> 4;
+#pragma unroll
+        for (int e = 0; e < 16; e += 4) {
+          const uint32_t h01 = e4m3x2_from(v[e], v[e + 1]);
+          const uint32_t h23 = e4m3x2_from(v[e + 2], v[e + 3]);
+          const float2 b01 = e4m3x2_value(h01);
+          const float2 b23 = e4m3x2_value(h23);
+          const uint32_t l01 = e4m3x2_from(v[e] - b01.x, v[e + 1] - b01.y);
+          const uint32_t l23 = e4m3x2_from(v[e + 2] - b23.x, v[e + 3] - b23.y);
+          uint32_t H = h01 | (h23 << 16), Lw = l01 | (l23 << 16);   // byte i: row e + i
+          // stage 1 (lanes j, j ^ 1): even lanes end with rows e, e+2 and
+          // odd lanes with rows e+1, e+3, each for keys (j & ~1, j | 1)
+          {
+            const uint32_t snd = (j4 & 1) ? __byte_perm(H, Lw, 0x6420) : __byte_perm(H, Lw, 0x7531);
+            const uint32_t rcv = __shfl_xor_sync(0xffffffffu, snd, 1);
+            if (j4 & 1) {
+              H = __byte_perm(H, rcv, 0x3514);
+              Lw = __byte_perm(Lw, rcv, 0x3716);
+            } else {
+              H = __byte_perm(H, rcv, 0x5240);
+              Lw = __byte_perm(Lw, rcv, 0x7260);
+            }
+          }
+          // stage 2 (lanes j, j ^ 2): lane j ends with row e + j, keys 0-3
+          {
+            const uint32_t snd = (j4 & 2) ? __byte_perm(H, Lw, 0x5410) : __byte_perm(H, Lw, 0x7632);
+            const uint32_t rcv = __shfl_xor_sync(0xffffffffu, snd, 2);
+            if (j4 & 2) {
+              H = __byte_perm(H, rcv, 0x3254);
+              Lw = __byte_perm(Lw, rcv, 0x3276);
+            } else {
+              H = __byte_perm(H, rcv, 0x5410);
+              Lw = __byte_perm(Lw, rcv, 0x7610);
+            }
+          }
+          const int r = 16 * q + e + j4;
+          const uint32_t o = (uint32_t)r * 128u + ((uint32_t)(ck ^ (r & 7)) << 4);
+          *reinterpret_cast<uint32_t*>(p8 + o) = H;
+          *reinterpret_cast<uint32_t*>(p8 + (uint32_t)RP * 128u + o) = Lw;
+        }
+      }
+    };
+    auto stage_masks = [&](int j) {
+      if (!(EXT && p.mask_rows > 0)) return;
+      auto stage = [&](int jj) {
+        cm.to(jj);
+        const int tile_al = cm.key0(jj, rev) & ~7;
+        const int shi = cm.hi;
+        const uint32_t dst0 = mstage_u32 + (uint32_t)(jj & 1) * p.mask_rows * MROW_BYTES;
+        for (int c = t; c < mrows * 17; c += 128) {
+          const int row = c / 17, k8 = (c - row * 17) * 8;
+          const int key8 = tile_al + k8;
+          const int n = min(max(shi - key8, 0), 8);   // keys inside the split (end <= Skv)
+          const uint16_t* src = n > 0 ? p.ext.mask + (size_t)b * p.ext.mask_sb + (size_t)(s0 + row) * p.ext.mask_sr + key8
+                                      : p.ext.mask;
+          cp_async16(dst0 + (uint32_t)row * MROW_BYTES + (uint32_t)k8 * 2u, src, (uint32_t)n * 2u);
+        }
+        cp_async_commit();
+      };
+      if (j == 0) stage(0);
+      if (j + 1 < T) {
+        stage(j + 1);
+        cp_async_wait<1>();
+      } else {
+        cp_async_wait<0>();
+      }
+    };
+    bool one_pass_done = false;
+    if constexpr (FP8 || EXT) {
+      if (RP <= 32) {
+      // One pass per tile for up to 32 rows (one or two groups of 16 held in
+      // registers), for the variants whose softmax outweighs a tile's load:
+      // fp8 K/V (half the bytes per tile) and the optional logit terms.  (The
+      // plain bf16 kernels keep the two-pass loop below: there the tile
+      // stream is paced by the K/V ring, and an earlier hand-off of P only
+      // moved the MMA thread's waits, measured 5 % slower on the 8-row verify
+      // decode.)  Each logit is taken relative to its row's subtrahend
+      // msub (x = logit - msub, log2 units; p = 2^x) and checked against the
+      // stale-maximum threshold on the spot: x > 8 is a logit more than 8
+      // (bf16 P) or 2 (fp8 P, stored as 64 p: msub = m - 6) above the row's
+      // running maximum m.  Only a tile where that happens runs the
+      // row-maximum reduction; the rule is the one of the two-pass loop
+      // below, so P is the same.  Row sums stay per thread (key) until the
+      // split ends, where one reduction gives l.
+      auto one_pass = [&](auto nq_tag) {
+        constexpr int NQ = decltype(nq_tag)::value;
+        constexpr float OFF = FP8 ? 6.f : 0.f;
+        float lacc[NQ][16];
+#pragma unroll
+        for (int q = 0; q < NQ; ++q)
+#pragma unroll
+          for (int e = 0; e < 16; ++e) lacc[q][e] = 0.f;
+        // the split's row sums into l_sm (rows t < RP); partial sums restart
+        auto reduce_l = [&]() {
+#pragma unroll
+          for (int q = 0; q < NQ; ++q) {
+            float v[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              v[e] = lacc[q][e];
+              lacc[q][e] = 0.f;
+            }
+            const float x = warp_reduce16<false>(v, lane);
+            if (lane < 16) red_sum[warp * RP + 16 * q + lane] = x;
+          }
+          named_bar_sync(1, 128);
+          if (t < RP) l_sm[t] = (red_sum[t] + red_sum[RP + t]) + (red_sum[2 * RP + t] + red_sum[3 * RP + t]);
+        };
+        for (int j = 0; ok && j < T; ++j) {
+          const int sb = j & 1;
+          cs.to(j);
+          const int jl = j - cs.first;   // tile within its split
+          const int hi = cs.hi;           // the split's end key
+          if (jl == 0 && j > 0) {
+            // a new split: publish the previous one (as in the loop below),
+            // then restart its rows
+            if (pend >= 0) {
+              if (!pv_done(pend_last)) { ok = false; break; }
+              write_o(pend);
+              pend = -1;
+            }
+            const int prev = seg_of(j - 1);
+            reduce_l();
+            stats(prev);
+            if (t < RP) {
+              m_sm[t] = -INFINITY;
+              msub_sm[t] = 0.f;
+              thrx_sm[t] = -INFINITY;
+            }
+            named_bar_sync(1, 128);   // the restarted rows, before any thread reads them
+            if (p.obuf == 2) {
+              pend = prev;
+              pend_last = j - 1;
+            } else {
+              if (!pv_done(j - 1)) { ok = false; break; }
+              write_o(prev);
+            }
+          }
+          stage_masks(j);
+          const bool got_s = mbar_wait(bar(BAR_S0 + sb), (uint32_t)(j >> 1) & 1u, wd);
+          // A staged mask needs a CTA barrier to be visible; otherwise a give-up
+          // here only has to be warp-uniform (TMEM loads are warp-collective),
+          // and the joint vote below takes it.
+          const bool fail_s =
+              (EXT && p.mask_rows > 0) ? named_bar_or(1, 128, !got_s) : __any_sync(0xffffffffu, !got_s);
+          const int tile0 = cs.key0(j, rev);
+          const int key = tile0 + t;
+          const uint16_t* mtile = mstage + (size_t)(j & 1) * p.mask_rows * MROW_KEYS + (tile0 & 7) + t;
+          const bool full = (tile0 + BN - 1 < hi) && (!p.causal || tile0 + BN - 1 <= q_offset) &&
+                            (!EXT || p.ext.window == 0 || tile0 >= q_offset + Sqc - p.ext.window);
+          auto visible = [&](int r) -> bool {
+            return key < hi && key <= lim_sm[r] && (!EXT || key > limlo_sm[r]);
+          };
+          float x[NQ][16];
+          bool exceed = false;
+          if (!fail_s) {
+            tc_fence_after();
+#pragma unroll
+            for (int q = 0; q < NQ; ++q) {
+              tmem_ld16(tmem + lane_off + TS(sb) + 16 * q, x[q]);
+              if (EXT) ext_rows16(x[q], xe, c2, key, t, q, slope_sm, pos_sm, mtile, mrows, q_offset, mrow_sm, hi);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float4 ms = reinterpret_cast<const float4*>(msub_sm + 16 * q)[i];
+                const float4 th = reinterpret_cast<const float4*>(thrx_sm + 16 * q)[i];
+                const float msv[4] = {ms.x, ms.y, ms.z, ms.w};
+                const float thv[4] = {th.x, th.y, th.z, th.w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  const int e = 4 * i + k;
+                  float xv = EXT ? x[q][e] - msv[k] : fmaf(x[q][e], c2, -msv[k]);
+                  if (!full && !visible(16 * q + e)) xv = -INFINITY;
+                  exceed = exceed || xv > thv[k];
+                  x[q][e] = xv;
+                }
+              }
+            }
+          }
+          // P buffer sb was read by the P.V of tile j-2: wait for it before rewriting
+          const bool got_pb = (j < 2) || mbar_wait(bar(BAR_PV0 + sb), (uint32_t)((j - 2) >> 1) & 1u, wd);
+          const bool fail = fail_s || !got_pb;
+          if (named_bar_or(1, 128, fail || exceed)) {
+            if (named_bar_or(1, 128, fail)) { ok = false; break; }
+            // some row's maximum moves: the tile's row maxima of x
+#pragma unroll
+            for (int q = 0; q < NQ; ++q) {
+              float v[16];
+#pragma unroll
+              for (int e = 0; e < 16; ++e) v[e] = x[q][e];
+              const float mx = warp_reduce16<true>(v, lane);
+              if (lane < 16) red_max[warp * RP + 16 * q + lane] = mx;
+            }
+            named_bar_sync(1, 128);
+            if (t < RP) {
+              const float mx =
+                  fmaxf(fmaxf(red_max[t], red_max[RP + t]), fmaxf(red_max[2 * RP + t], red_max[3 * RP + t]));
+              float delta = 0.f, alpha = 1.f;
+              if (mx > thrx_sm[t]) {
+                // the row's new maximum m' = msub + mx: msub' = m' - OFF and
+                // x' = x + delta with delta = OFF - mx; O and l scale by
+                // 2^(m - m') = 2^delta (0 while m was -inf)
+                delta = OFF - mx;
+                alpha = (m_sm[t] == -INFINITY) ? 0.f : ex2_approx(delta);
+                const float ms = msub_sm[t] - delta;
+                msub_sm[t] = ms;
+                m_sm[t] = ms + OFF;
+                thrx_sm[t] = 8.f;
+              }
+              delta_sm[t] = delta;
+              alpha_sm[t] = alpha;
+            }
+            named_bar_sync(1, 128);
+#pragma unroll
+            for (int q = 0; q < NQ; ++q)
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                x[q][e] += delta_sm[16 * q + e];
+                lacc[q][e] *= alpha_sm[16 * q + e];
+              }
+            if (jl > 0) {
+              // O^T is accumulated by the P.V of tile j-1: it must have completed
+              const bool got_o = mbar_wait(bar(BAR_PV0 + (sb ^ 1)), (uint32_t)((j - 1) >> 1) & 1u, wd);
+              if (named_bar_or(1, 128, !got_o)) { ok = false; break; }
+              tc_fence_after();
+              for (int c = 0; c < KC; ++c) {
+#pragma unroll
+                for (int q = 0; q < NQ; ++q) {
+                  float v[16];
+                  const uint32_t addr = tmem + lane_off + TO(c, cs.ob) + 16 * q;
+                  tmem_ld16(addr, v);
+                  uint32_t u[16];
+#pragma unroll
+                  for (int e = 0; e < 16; ++e) u[e] = __float_as_uint(v[e] * alpha_sm[16 * q + e]);
+                  tmem_st16(addr, u);
+                }
+              }
+            }
+          }
+          // exponentials, per-thread row sums, P into the B-operand buffer
+#pragma unroll
+          for (int q = 0; q < NQ; ++q) {
+            float v[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              v[e] = ex2_approx(x[q][e]);
+              lacc[q][e] += v[e];
+            }
+            store_p16(sb, q, v);
+          }
+          fence_proxy_async_smem();
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(bar(BAR_P0 + sb));
+          if (pend >= 0 && j >= 2 && pend_last <= j - 2) {
+            write_o(pend);
+            pend = -1;
+          }
+        }
+        if (ok) reduce_l();
+      };
+      if (RP <= 16) one_pass(IntC<1>{});
+      else one_pass(IntC<2>{});
+      one_pass_done = true;
+      }
+    }
+    if (!one_pass_done)
     for (int j = 0; ok && j < T; ++j) {
       const int sb = j & 1;
       cs.to(j);
@@ -775,33 +1080,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       }
       // every give-up is decided jointly (barrier + OR) so no thread is left
       // waiting at a named barrier or inside a warp-collective TMEM access
-      if (EXT && p.mask_rows > 0) {
-        // stage tile j+1's mask rows (and tile 0's first) with cp.async; the
-        // copies stay in flight across this tile's barriers, and tile j's are
-        // complete (and, after the barrier below, visible) before use
-        auto stage = [&](int jj) {
-          cm.to(jj);
-          const int tile_al = cm.key0(jj, rev) & ~7;
-          const int shi = cm.hi;
-          const uint32_t dst0 = mstage_u32 + (uint32_t)(jj & 1) * p.mask_rows * MROW_BYTES;
-          for (int c = t; c < mrows * 17; c += 128) {
-            const int row = c / 17, k8 = (c - row * 17) * 8;
-            const int key8 = tile_al + k8;
-            const int n = min(max(shi - key8, 0), 8);   // keys inside the split (end <= Skv)
-            const uint16_t* src = n > 0 ? p.ext.mask + (size_t)b * p.ext.mask_sb + (size_t)(s0 + row) * p.ext.mask_sr + key8
-                                        : p.ext.mask;
-            cp_async16(dst0 + (uint32_t)row * MROW_BYTES + (uint32_t)k8 * 2u, src, (uint32_t)n * 2u);
-          }
-          cp_async_commit();
-        };
-        if (j == 0) stage(0);
-        if (j + 1 < T) {
-          stage(j + 1);
-          cp_async_wait<1>();
-        } else {
-          cp_async_wait<0>();
-        }
-      }
+      stage_masks(j);
       const bool got_s = mbar_wait(bar(BAR_S0 + sb), (uint32_t)(j >> 1) & 1u, wd);
       if (named_bar_or(1, 128, !got_s)) { ok = false; break; }
       tc_fence_after();
@@ -853,9 +1132,6 @@ __global__ void __launch_bounds__(THREADS, 2)
       const bool rescale = (jl > 0) && (*resc_flag != 0);
       // pass 2: exponentials, P (bf16) into the swizzled B-operand buffer
       {
-        const int half = t >> 6, tt = t & 63;
-        uint8_t* pcol = gbase + PB(sb) + (size_t)half * RP * 128 + (size_t)(tt & 7) * 2;
-        const int chunk16 = tt >> 3;
         for (int q = 0; q < RP / 16; ++q) {
           float v[16];
           tmem_ld16(tmem + lane_off + TS(sb) + 16 * q, v);
@@ -874,69 +1150,7 @@ __global__ void __launch_bounds__(THREADS, 2)
             if (!full && !visible(r)) pv = 0.f;
             v[e] = pv;
           }
-          if constexpr (!FP8) {
-            // bf16 P, one 32-bit word (keys t & ~1, t | 1) per store: for
-            // each pair of rows the even lane writes the even row and the odd
-            // lane the odd row, each taking its neighbour's value by shuffle
-            const bool odd = (t & 1) != 0;
-            uint8_t* pword = pcol - (size_t)(tt & 1) * 2;
-#pragma unroll
-            for (int e = 0; e < 16; e += 2) {
-              const float other = __shfl_xor_sync(0xffffffffu, odd ? v[e] : v[e + 1], 1);
-              const int r = 16 * q + e + (odd ? 1 : 0);
-              const uint32_t w = odd ? pack_bf16x2(other, v[e + 1]) : pack_bf16x2(v[e], other);
-              *reinterpret_cast<uint32_t*>(pword + (size_t)r * 128 + ((chunk16 ^ (r & 7)) << 4)) = w;
-            }
-          }
-          if constexpr (FP8) {
-            // P as hi + lo e4m3 planes (row r: 128 keys, one 128-byte
-            // swizzled row per plane).  A lane holds one key of 4 rows; a
-            // 4 x 4 byte transpose in each quad of lanes (two shuffle stages,
-            // both planes in one word) gives lane j the 4 keys of row e + j,
-            // so every store is a 32-bit word.
-            const int j4 = t & 3;
-            uint8_t* p8 = gbase + PB(sb) + ((t & 15) & ~3);
-            const int ck = t >> 4;
-#pragma unroll
-            for (int e = 0; e < 16; e += 4) {
-              const uint32_t h01 = e4m3x2_from(v[e], v[e + 1]);
-              const uint32_t h23 = e4m3x2_from(v[e + 2], v[e + 3]);
-              const float2 b01 = e4m3x2_value(h01);
-              const float2 b23 = e4m3x2_value(h23);
-              const uint32_t l01 = e4m3x2_from(v[e] - b01.x, v[e + 1] - b01.y);
-              const uint32_t l23 = e4m3x2_from(v[e + 2] - b23.x, v[e + 3] - b23.y);
-              uint32_t H = h01 | (h23 << 16), Lw = l01 | (l23 << 16);   // byte i: row e + i
-              // stage 1 (lanes j, j ^ 1): even lanes end with rows e, e+2 and
-              // odd lanes with rows e+1, e+3, each for keys (j & ~1, j | 1)
-              {
-                const uint32_t snd = (j4 & 1) ? __byte_perm(H, Lw, 0x6420) : __byte_perm(H, Lw, 0x7531);
-                const uint32_t rcv = __shfl_xor_sync(0xffffffffu, snd, 1);
-                if (j4 & 1) {
-                  H = __byte_perm(H, rcv, 0x3514);
-                  Lw = __byte_perm(Lw, rcv, 0x3716);
-                } else {
-                  H = __byte_perm(H, rcv, 0x5240);
-                  Lw = __byte_perm(Lw, rcv, 0x7260);
-                }
-              }
-              // stage 2 (lanes j, j ^ 2): lane j ends with row e + j, keys 0-3
-              {
-                const uint32_t snd = (j4 & 2) ? __byte_perm(H, Lw, 0x5410) : __byte_perm(H, Lw, 0x7632);
-                const uint32_t rcv = __shfl_xor_sync(0xffffffffu, snd, 2);
-                if (j4 & 2) {
-                  H = __byte_perm(H, rcv, 0x3254);
-                  Lw = __byte_perm(Lw, rcv, 0x3276);
-                } else {
-                  H = __byte_perm(H, rcv, 0x5410);
-                  Lw = __byte_perm(Lw, rcv, 0x7610);
-                }
-              }
-              const int r = 16 * q + e + j4;
-              const uint32_t o = (uint32_t)r * 128u + ((uint32_t)(ck ^ (r & 7)) << 4);
-              *reinterpret_cast<uint32_t*>(p8 + o) = H;
-              *reinterpret_cast<uint32_t*>(p8 + (uint32_t)RP * 128u + o) = Lw;
-            }
-          }
+          store_p16(sb, q, v);
           const float s = warp_reduce16<false>(v, lane);
           if (lane < 16) red_sum[warp * RP + 16 * q + lane] = s;
         }
