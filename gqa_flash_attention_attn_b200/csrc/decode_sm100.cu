@@ -328,6 +328,10 @@ __global__ void __launch_bounds__(THREADS, 2)
   const int BAR_DRAIN = BAR_S0 + 6;
   const int BAR_Q8 = BAR_S0 + 7;         // fp8: Q planes written
 
+  // a merge launched after this kernel (programmatic dependent launch) may
+  // be scheduled as soon as every CTA of this grid has started; it waits for
+  // this grid to complete before it reads anything
+  griddep_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bkv = blockIdx.y / p.nqc;
   // query chunks in reverse: with a causal mask the last chunks see the most

@@ -21,7 +21,10 @@ __global__ void __launch_bounds__(128, 8) merge_kernel(const MergeParams p) {
   // partial loads are in flight at once; the four warps' sums are combined in
   // shared memory.
   __shared__ float4 part_acc[3][32];
-  __shared__ float part_w[3];
+  __shared__ float part_w[3], part_m[3];
+  // launched as a dependent of the split kernel: its partials are complete
+  // and visible past this point
+  griddep_wait();
   const int f4_per_row = p.D / 4;
   const int chunks = (f4_per_row + 31) / 32;
   const long long blk = blockIdx.x;
@@ -37,18 +40,16 @@ __global__ void __launch_bounds__(128, 8) merge_kernel(const MergeParams p) {
   const size_t out_stride4 = (size_t)p.B * p.Sq * p.Hq * p.D / 4;
   const float4* src = reinterpret_cast<const float4*>(p.part_out + (size_t)row * p.D) + (active ? f : 0);
 
-  // max of the split LSEs and the sink logit (every warp computes it; the
-  // loads are tiny); the sink joins only the denominator
+  // Warp w merges splits w, w+4, ... against its own running maximum Mw of
+  // their LSEs (eight loads in flight per batch, issued before any
+  // arithmetic); the four warps' (Mw, sum, acc) then combine against the
+  // common M, which the sink logit joins (the sink adds only to the
+  // denominator).  Every lane of a warp loads the same LSEs, so Mw is
+  // warp-uniform.
+  constexpr float L2E = 1.4426950408889634f;
   const float sink = p.sinks != nullptr ? __ldg(p.sinks + h) : -INFINITY;
-  float M = sink;
-  for (int sg = lane; sg < p.num_splits; sg += 32) M = fmaxf(M, __ldg(p.part_lse + sg * lse_stride + lse_row));
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  float wsum = 0.f;
-  // this warp's splits, eight loads in flight per batch; the loads do not
-  // wait for the maximum above (every published partial is finite)
+  float wsum = 0.f, Mw = -INFINITY;
   for (int s0 = warp; s0 < p.num_splits; s0 += 32) {
     float4 o[8];
     float x[8];
@@ -59,13 +60,26 @@ __global__ void __launch_bounds__(128, 8) merge_kernel(const MergeParams p) {
         o[u] = __ldg(src + (size_t)sg * out_stride4);
         x[u] = __ldg(p.part_lse + sg * lse_stride + lse_row);
       } else {
+        o[u] = make_float4(0.f, 0.f, 0.f, 0.f);
         x[u] = -INFINITY;
       }
+    }
+    float mb = Mw;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) mb = fmaxf(mb, x[u]);
+    if (mb != Mw) {   // the batch raised the maximum: rescale what came before
+      const float a = (Mw == -INFINITY) ? 0.f : ex2_approx((Mw - mb) * L2E);
+      wsum *= a;
+      acc.x *= a;
+      acc.y *= a;
+      acc.z *= a;
+      acc.w *= a;
+      Mw = mb;
     }
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       if (x[u] != -INFINITY) {
-        const float w = ex2_approx((x[u] - M) * 1.4426950408889634f);
+        const float w = ex2_approx((x[u] - Mw) * L2E);
         wsum += w;
         acc.x = fmaf(w, o[u].x, acc.x);
         acc.y = fmaf(w, o[u].y, acc.y);
@@ -74,22 +88,38 @@ __global__ void __launch_bounds__(128, 8) merge_kernel(const MergeParams p) {
       }
     }
   }
-  if (warp == 0 && sink != -INFINITY) wsum += ex2_approx((sink - M) * 1.4426950408889634f);
   if (warp > 0) {
     part_acc[warp - 1][lane] = acc;
-    if (lane == 0) part_w[warp - 1] = wsum;
+    if (lane == 0) {
+      part_w[warp - 1] = wsum;
+      part_m[warp - 1] = Mw;
+    }
   }
   __syncthreads();
   if (warp != 0) return;
+  float M = fmaxf(Mw, sink);
+#pragma unroll
+  for (int i = 0; i < 3; ++i) M = fmaxf(M, part_m[i]);
+  {
+    const float a = (Mw == -INFINITY) ? 0.f : ex2_approx((Mw - M) * L2E);
+    wsum *= a;
+    acc.x *= a;
+    acc.y *= a;
+    acc.z *= a;
+    acc.w *= a;
+  }
 #pragma unroll
   for (int i = 0; i < 3; ++i) {
-    const float4 a = part_acc[i][lane];
-    acc.x += a.x;
-    acc.y += a.y;
-    acc.z += a.z;
-    acc.w += a.w;
-    wsum += part_w[i];
+    const float mi = part_m[i];
+    const float a = (mi == -INFINITY) ? 0.f : ex2_approx((mi - M) * L2E);
+    const float4 q = part_acc[i][lane];
+    acc.x = fmaf(a, q.x, acc.x);
+    acc.y = fmaf(a, q.y, acc.y);
+    acc.z = fmaf(a, q.z, acc.z);
+    acc.w = fmaf(a, q.w, acc.w);
+    wsum = fmaf(a, part_w[i], wsum);
   }
+  if (sink != -INFINITY) wsum += ex2_approx((sink - M) * L2E);
   if (M != -INFINITY) {
     const float inv = 1.f / wsum;
     acc.x *= inv;
@@ -132,7 +162,22 @@ int launch_merge(const MergeParams& p, cudaStream_t stream) {
   const long long chunks = (p.D / 4 + 31) / 32;
   const long long blocks = (long long)p.B * p.Sq * p.Hq * chunks;
   if (blocks <= 0 || blocks > 0x7fffffffLL) return (int)cudaErrorInvalidValue;
-  merge_kernel<<<(unsigned)blocks, 128, 0, stream>>>(p);
+  // Programmatic stream serialization: the merge grid may be scheduled while
+  // the kernel before it on the stream (the split kernel, which allows it
+  // from the start of each CTA) is still running; every block waits at
+  // griddep_wait() until that kernel has completed.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)blocks);
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, merge_kernel, p);
+  if (e != cudaSuccess) return (int)e;
   return (int)cudaGetLastError();
 }
 

@@ -90,6 +90,16 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
 }
 
 // ------------------------------------------------------------------- TMA ----
+// Programmatic dependent launch.  launch_dependents: this CTA lets a grid
+// launched after it with programmatic stream serialization start (once every
+// CTA of this grid has issued it or exited); grid_dependency_wait: wait until
+// the grids this one depends on have completed and their memory is visible
+// (returns at once when the grid was launched without that attribute).
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }
