@@ -114,6 +114,11 @@ int attn_decode_split(const void* q, const void* k, const void* v, float* partia
  *     out = sum_s w_s * O_s / sum_s w_s;   lse = M + log(sum_s w_s).
  * Splits with lse = -inf get weight 0.  lse may be NULL.
  *   D            any multiple of 4 in [4, 1024] (else ATTN_ERR_UNSUPPORTED)
+ * The merge is launched with programmatic stream serialization: it may be
+ * scheduled before the kernel ahead of it on the stream has finished (the
+ * split-KV kernel allows that from its start), and every block waits for
+ * that kernel to complete, with its writes visible, before it reads
+ * anything; stream order is kept.
  */
 int attn_merge(const float* partial_out, const float* partial_lse, void* out, float* lse,
                int B, int Hq, int Sq, int D, int num_splits, int out_dtype, void* stream);
