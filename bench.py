@@ -11,7 +11,9 @@ the same way and reported under "configs", the last key of the JSON line; the
 widened workloads (logit terms, masks, windows, fp8, paged, fused, latent
 cache, D512 prefill) come before it under "workloads".  Each carries the
 roofline fraction of its whole step (a decode step is the split kernel plus
-the merge) and, as kernel_frac, that of its first kernel alone.  L2 is
+the merge, timed with no event between the two launches, as a caller runs
+them) and, as kernel_frac, that of its first kernel alone (from a second
+timed pass with an event after the split kernel).  L2 is
 flushed between timed steps (a 256 MiB write, then a 256 MiB read so no dirty
 lines are left behind); the flush is outside the timed events.
 
